@@ -1,0 +1,208 @@
+"""ctypes front end of the CPU oracle (``moe_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU-baseline leg
+import this module; the product package never does. The oracle is a plain, slow C
+restatement of the MoE layer forward (Comet: Fine-grained Computation-communication
+Overlapping for Mixture-of-Experts, §2.1 "MoE Structure"; the tile reorganisation of
+§2.2.1 and §3.1.2). Every function here only marshals numpy arrays into the C entry
+points; no arithmetic of the method lives in Python.
+
+Arrays of bf16 values are passed as ``numpy.uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "moe_oracle.c"
+_LIB = _HERE / "liboracle.so"
+
+ACT_SWIGLU, ACT_GELU_TANH, ACT_RELU, ACT_IDENTITY = 0, 1, 2, 3
+GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL = 0, 1
+
+# Portable flags: the library may be built on one host and run on another.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fopenmp"]
+
+
+def build(force: bool = False, src: Path | None = None, out: Path | None = None) -> Path:
+    """Compile the oracle into a shared library (gcc) and return its path."""
+    src = Path(src) if src is not None else _SRC
+    out = Path(out) if out is not None else _LIB
+    if force or not out.exists() or out.stat().st_mtime < src.stat().st_mtime:
+        tmp = out.with_suffix(f".tmp{os.getpid()}.so")
+        subprocess.run(["gcc", *CFLAGS, "-o", str(tmp), str(src), "-lm"], check=True)
+        os.replace(tmp, out)
+    return out
+
+
+_lib_cache: dict[str, ctypes.CDLL] = {}
+
+
+def load(path: Path | None = None) -> ctypes.CDLL:
+    """Load (building first if needed) the oracle library; cached per path."""
+    p = str(build() if path is None else path)
+    if p in _lib_cache:
+        return _lib_cache[p]
+    lib = ctypes.CDLL(p)
+    i32, i64, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+    lib.oracle_round_to_bf16.argtypes = [ctypes.c_double]
+    lib.oracle_round_to_bf16.restype = ctypes.c_double
+    lib.oracle_router_logits.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+    lib.oracle_router_logits.restype = None
+    lib.oracle_topk_gates.argtypes = [i32, i32, i32, i32, vp, vp, vp]
+    lib.oracle_topk_gates.restype = i32
+    lib.oracle_dispatch.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, i64]
+    lib.oracle_dispatch.restype = i32
+    lib.oracle_expert_ffn_row.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.oracle_expert_ffn_row.restype = None
+    lib.oracle_combine.argtypes = [i32, i32, i32, vp, vp, vp]
+    lib.oracle_combine.restype = None
+    lib.oracle_moe_forward.argtypes = [i32] * 9 + [vp] * 8
+    lib.oracle_moe_forward.restype = i32
+    lib.oracle_moe_tokens.argtypes = [i32] * 8 + [vp] * 5 + [i32, vp, vp, vp, vp]
+    lib.oracle_moe_tokens.restype = i32
+    _lib_cache[p] = lib
+    return lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def round_to_bf16(v: float, lib=None) -> float:
+    return (lib or load()).oracle_round_to_bf16(float(v))
+
+
+def router_logits(x, Wg, bias=None, lib=None):
+    """fp32 logits [T,E] (sequential h-ascending sum; see moe_oracle.c)."""
+    lib = lib or load()
+    x, Wg = _u16(x), _u16(Wg)
+    T, H = x.shape
+    H2, E = Wg.shape
+    assert H == H2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((T, E), np.float32)
+    lib.oracle_router_logits(T, H, E, _p(x), _p(Wg), _p(b), _p(out))
+    return out
+
+
+def topk_gates(logits, k, gate=GATE_SOFTMAX_TOPK, lib=None):
+    lib = lib or load()
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    rc = lib.oracle_topk_gates(T, E, k, gate, _p(logits), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle_topk_gates rc={rc}")
+    return idx, w
+
+
+def padded_rows_max(T, E, k, m_tile=128):
+    return T * k + E * (m_tile - 1)
+
+
+def dispatch(idx, E, m_tile=128, lib=None):
+    """Counting sort of routed pairs into expert-contiguous, m_tile-padded rows."""
+    lib = lib or load()
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    glen = padded_rows_max(T, E, k, m_tile)
+    tcap = glen // m_tile + E
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    poff = np.empty(E + 1, np.int32)
+    gather_idx = np.empty(glen, np.int32)
+    inv_pos = np.empty((T, k), np.int32)
+    te = np.empty(tcap, np.int32)
+    tr = np.empty(tcap, np.int32)
+    tn = np.empty(tcap, np.int32)
+    nt = lib.oracle_dispatch(T, E, k, m_tile, _p(idx), _p(counts), _p(offsets), _p(poff),
+                             _p(gather_idx), glen, _p(inv_pos), _p(te), _p(tr), _p(tn), tcap)
+    if nt < 0:
+        raise ValueError(f"oracle_dispatch rc={nt}")
+    return dict(counts=counts, offsets=offsets, padded_offsets=poff, gather_idx=gather_idx,
+                inv_pos=inv_pos, tile_expert=te[:nt].copy(), tile_row0=tr[:nt].copy(),
+                tile_nvalid=tn[:nt].copy(), num_tiles=nt)
+
+
+def expert_ffn_row(xrow, W1e, W2e, act=ACT_SWIGLU, round_a_bf16=False, lib=None):
+    lib = lib or load()
+    xrow, W1e, W2e = _u16(xrow), _u16(W1e), _u16(W2e)
+    H = xrow.shape[0]
+    F, H2 = W2e.shape
+    assert H2 == H
+    y = np.empty(H, np.float64)
+    lib.oracle_expert_ffn_row(H, F, act, int(round_a_bf16), _p(xrow), _p(W1e), _p(W2e), _p(y))
+    return y
+
+
+def combine(ys, inv_pos, lib=None):
+    """out[t] = sum_j ys[inv_pos[t, j]] (fp64; ys are bf16 rows already gate-scaled)."""
+    lib = lib or load()
+    ys = _u16(ys)
+    inv_pos = np.ascontiguousarray(inv_pos, dtype=np.int32)
+    T, k = inv_pos.shape
+    H = ys.shape[1]
+    out = np.empty((T, H), np.float64)
+    lib.oracle_combine(T, H, k, _p(ys), _p(inv_pos), _p(out))
+    return out
+
+
+def _ffn_dims(W1, W2, act):
+    E, H, c = W1.shape
+    E2, F, H2 = W2.shape
+    assert E == E2 and H == H2
+    assert c == (2 * F if act == ACT_SWIGLU else F), (c, F, act)
+    return E, H, F
+
+
+def moe_forward(x, Wg, bias, W1, W2, k, act=ACT_SWIGLU, gate=GATE_SOFTMAX_TOPK, m_tile=128,
+                round_a_bf16=False, lib=None):
+    """Whole layer (route -> dispatch -> experts -> combine). Returns (out f64 [T,H], idx, w)."""
+    lib = lib or load()
+    x, Wg, W1, W2 = _u16(x), _u16(Wg), _u16(W1), _u16(W2)
+    T, H = x.shape
+    E, H1, F = _ffn_dims(W1, W2, act)
+    assert H1 == H and Wg.shape == (H, E)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((T, H), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    rc = lib.oracle_moe_forward(T, H, F, E, k, act, gate, m_tile, int(round_a_bf16), _p(x), _p(Wg),
+                                _p(b), _p(W1), _p(W2), _p(out), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle_moe_forward rc={rc}")
+    return out, idx, w
+
+
+def moe_tokens(x, Wg, bias, W1, W2, k, tokens, act=ACT_SWIGLU, gate=GATE_SOFTMAX_TOPK,
+               round_a_bf16=False, lib=None):
+    """Layer output for selected tokens straight from the per-token definition."""
+    lib = lib or load()
+    x, Wg, W1, W2 = _u16(x), _u16(Wg), _u16(W1), _u16(W2)
+    T, H = x.shape
+    E, H1, F = _ffn_dims(W1, W2, act)
+    assert H1 == H and Wg.shape == (H, E)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    n = tokens.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((n, H), np.float64)
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    rc = lib.oracle_moe_tokens(T, H, F, E, k, act, gate, int(round_a_bf16), _p(x), _p(Wg), _p(b),
+                               _p(W1), _p(W2), n, _p(tokens), _p(out), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle_moe_tokens rc={rc}")
+    return out, idx, w

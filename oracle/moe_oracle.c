@@ -1,0 +1,476 @@
+/*
+ * moe_oracle.c -- plain CPU oracle for the forward pass of one mixture-of-experts layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. The product library never links, loads or calls this file.
+ * Only the test suite, the smoke check and the bench's CPU-baseline leg use it. It shares
+ * no code, header, table or helper with the CUDA path.
+ *
+ * What is computed, and where the pages say so
+ * (Comet: Fine-grained Computation-communication Overlapping for Mixture-of-Experts):
+ *   - §2.1 "MoE Structure": each token is routed to a few selected experts, each selected
+ *     expert runs its feed-forward network on the token, and the top-k expert outputs are
+ *     gathered back and reduced.                       -> oracle_router_logits,
+ *                                                        oracle_topk_gates,
+ *                                                        oracle_expert_ffn_row,
+ *                                                        oracle_combine
+ *   - §2.2.1 and §3.1.2: the routed tokens are reorganised so that each computation tile
+ *     sees only the rows it needs; layer0 and layer1 run as grouped GEMMs over the
+ *     experts.                                         -> oracle_dispatch
+ *   - §2.2.2: routing is decided at run time, so the per-expert row counts vary.
+ *
+ * Readings taken where the pages are silent (each one is listed in the design notes):
+ *   - router: logits = x . W_g (+ an optional per-expert bias), W_g stored [H, E];
+ *   - selection: the k largest logits, ties broken toward the lower expert id;
+ *   - gates: softmax over the k selected logits (equal, in exact arithmetic, to a softmax
+ *     over all E followed by renormalisation over the selected k); a second mode keeps
+ *     the full-E softmax values without renormalisation;
+ *   - experts: SwiGLU with W1 [E, H, 2F] (columns [0,F) gate, [F,2F) up) or a plain
+ *     activation with W1 [E, H, F]; W2 is [E, F, H];
+ *   - no capacity limit: every routed (token, expert) pair is computed;
+ *   - rows of one expert are ordered by ascending token id; each expert's row block is
+ *     padded up to a multiple of the tile height; pad rows carry the index -1.
+ *
+ * Precision:
+ *   - inputs are bf16 bit patterns, widened to float exactly;
+ *   - the router logits decide integers (the selected experts), so they are computed in
+ *     the precision and order the GPU router uses: fp32, one accumulator, h ascending.
+ *     A bf16 x bf16 product is exact in fp32, so fused and unfused multiply-add agree;
+ *   - everything else (gates, expert FFN, combine) is computed in fp64.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fopenmp. No fast-math.
+ * OpenMP only splits independent tokens or rows across threads; it never changes the
+ * order of any sum.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_ACT_SWIGLU 0
+#define ORACLE_ACT_GELU_TANH 1
+#define ORACLE_ACT_RELU 2
+#define ORACLE_ACT_IDENTITY 3
+
+#define ORACLE_GATE_SOFTMAX_TOPK 0
+#define ORACLE_GATE_SOFTMAX_ALL 1
+
+/* ---------------------------------------------------------------------------------------
+ * bf16 helpers
+ * ------------------------------------------------------------------------------------- */
+
+/* bf16 is the upper half of an IEEE binary32 word, so widening is a 16-bit shift. */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a double to the nearest bf16 value (8 significant bits), ties to even.
+ * Only normal-range values are expected here; zero passes through. */
+double oracle_round_to_bf16(double v)
+{
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    double m = frexp(v, &e);          /* v = m * 2^e, 0.5 <= |m| < 1 */
+    double scaled = ldexp(m, 8);      /* 8 significant bits to the left of the point */
+    double r = nearbyint(scaled);     /* default rounding mode: nearest, ties to even */
+    return ldexp(r, e - 8);
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Router (§2.1: tokens are routed to selected experts)
+ * ------------------------------------------------------------------------------------- */
+
+/* logits[t][e] = sum_h x[t][h] * Wg[h][e]  (+ bias[e]),
+ * in fp32 with a single accumulator and h ascending. x: [T,H], Wg: [H,E], bias: [E] or NULL. */
+void oracle_router_logits(int T, int H, int E, const uint16_t *x, const uint16_t *Wg,
+                          const float *bias, float *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            float acc = 0.0f;
+            for (int h = 0; h < H; ++h) {
+                float p = bf16_to_float(x[(size_t)t * H + h]) * bf16_to_float(Wg[(size_t)h * E + e]);
+                acc = acc + p;
+            }
+            if (bias) acc = acc + bias[e];
+            logits[(size_t)t * E + e] = acc;
+        }
+    }
+}
+
+/* Top-k selection and gate weights for one token.
+ * Selection: repeatedly take the largest remaining logit; on equal values the lower
+ * expert id wins (scan ascending, replace only on strictly greater). Equal compares as
+ * floats, so +0 and -0 tie.
+ * Gates (fp64):
+ *   SOFTMAX_TOPK: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0), i, j over the selected k;
+ *   SOFTMAX_ALL : w_j = exp(l_j - l_0) / sum_e exp(l_e - l_0), e over all E
+ *                 (l_0 is the largest logit in both cases). */
+static void topk_one(int E, int k, int gate, const float *l, int32_t *idx, double *w,
+                     unsigned char *taken)
+{
+    memset(taken, 0, (size_t)E);
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || l[e] > l[best]) best = e;
+        }
+        taken[best] = 1;
+        idx[j] = best;
+    }
+    double m = (double)l[idx[0]];
+    double denom = 0.0;
+    if (gate == ORACLE_GATE_SOFTMAX_ALL) {
+        for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
+    } else {
+        for (int j = 0; j < k; ++j) denom += exp((double)l[idx[j]] - m);
+    }
+    for (int j = 0; j < k; ++j) w[j] = exp((double)l[idx[j]] - m) / denom;
+}
+
+/* logits: [T,E] fp32 -> idx: [T,k] int32 (in selection order), w: [T,k] fp64. */
+int oracle_topk_gates(int T, int E, int k, int gate, const float *logits, int32_t *idx, double *w)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+#pragma omp for schedule(static)
+        for (int t = 0; t < T; ++t) {
+            if (!taken) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            topk_one(E, k, gate, logits + (size_t)t * E, idx + (size_t)t * k, w + (size_t)t * k, taken);
+        }
+        free(taken);
+    }
+    return bad ? -2 : 0;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Dispatch (§2.2.1, §3.1.2: reorganise routed tokens into expert-contiguous tiles)
+ * ------------------------------------------------------------------------------------- */
+
+/* Counting sort of the T*k routed pairs by expert, stable in token id.
+ *   counts[e]      number of pairs routed to e                              [E]
+ *   offsets[e]     exclusive prefix sum of counts                           [E+1]
+ *   poff[e]        exclusive prefix sum of counts rounded up to m_tile      [E+1]
+ *   gather_idx[r]  token of padded row r, -1 for a pad row                 [gather_len]
+ *   inv_pos[t][j]  padded row that holds pair (t, j)                        [T,k]
+ *   tile_expert/tile_row0/tile_nvalid: one entry per m_tile block of rows  [tile_cap]
+ * Returns the number of tiles, or a negative value on bad arguments. */
+int oracle_dispatch(int T, int E, int k, int m_tile, const int32_t *idx, int32_t *counts,
+                    int32_t *offsets, int32_t *poff, int32_t *gather_idx, int64_t gather_len,
+                    int32_t *inv_pos, int32_t *tile_expert, int32_t *tile_row0,
+                    int32_t *tile_nvalid, int64_t tile_cap)
+{
+    if (T < 0 || E < 1 || k < 1 || m_tile < 1) return -1;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t p = 0; p < (int64_t)T * k; ++p) {
+        int e = idx[p];
+        if (e < 0 || e >= E) return -2;
+        counts[e] += 1;
+    }
+    offsets[0] = 0;
+    poff[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        offsets[e + 1] = offsets[e] + counts[e];
+        int padded = ((counts[e] + m_tile - 1) / m_tile) * m_tile;
+        poff[e + 1] = poff[e] + padded;
+    }
+    if ((int64_t)poff[E] > gather_len) return -3;
+    for (int64_t r = 0; r < gather_len; ++r) gather_idx[r] = -1;
+
+    int32_t *cursor = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    if (!cursor) return -4;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            int r = poff[e] + cursor[e];
+            cursor[e] += 1;
+            gather_idx[r] = t;
+            inv_pos[(size_t)t * k + j] = r;
+        }
+    }
+    free(cursor);
+
+    int64_t nt = 0;
+    for (int e = 0; e < E; ++e) {
+        for (int i = 0; i * m_tile < counts[e]; ++i) {
+            if (nt >= tile_cap) return -5;
+            int left = counts[e] - i * m_tile;
+            tile_expert[nt] = e;
+            tile_row0[nt] = poff[e] + i * m_tile;
+            tile_nvalid[nt] = left < m_tile ? left : m_tile;
+            nt += 1;
+        }
+    }
+    return (int)nt;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Expert FFN (§2.1: the selected experts' feed-forward computation)
+ * ------------------------------------------------------------------------------------- */
+
+static double act_apply(int act, double z)
+{
+    switch (act) {
+    case ORACLE_ACT_GELU_TANH: {
+        const double c = sqrt(2.0 / acos(-1.0));
+        return 0.5 * z * (1.0 + tanh(c * (z + 0.044715 * z * z * z)));
+    }
+    case ORACLE_ACT_RELU:
+        return z > 0.0 ? z : 0.0;
+    case ORACLE_ACT_IDENTITY:
+    default:
+        return z;
+    }
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* One expert applied to one token row, fp64 throughout.
+ *   SwiGLU: g_f = sum_h x_h W1[h][f], u_f = sum_h x_h W1[h][F+f], a_f = silu(g_f) * u_f
+ *           (W1 row stride 2F);
+ *   other : a_f = act(sum_h x_h W1[h][f])  (W1 row stride F);
+ *   y_n = sum_f a_f W2[f][n]  (W2 row stride H).
+ * round_a_bf16 != 0 rounds a_f to bf16 first (a diagnostic of the GPU's bf16 h tensor).
+ * scratch must hold 2F doubles. */
+static void ffn_row(int H, int F, int act, int round_a_bf16, const uint16_t *xrow,
+                    const uint16_t *W1e, const uint16_t *W2e, double *y, double *scratch)
+{
+    const int gated = (act == ORACLE_ACT_SWIGLU);
+    const int w1_cols = gated ? 2 * F : F;
+    double *z = scratch; /* w1_cols pre-activations */
+    for (int c = 0; c < w1_cols; ++c) z[c] = 0.0;
+    for (int h = 0; h < H; ++h) {
+        double xh = (double)bf16_to_float(xrow[h]);
+        const uint16_t *wrow = W1e + (size_t)h * w1_cols;
+        for (int c = 0; c < w1_cols; ++c) z[c] += xh * (double)bf16_to_float(wrow[c]);
+    }
+    /* activation in place: a_f is written to z[f] */
+    for (int f = 0; f < F; ++f) {
+        double a = gated ? silu(z[f]) * z[F + f] : act_apply(act, z[f]);
+        z[f] = round_a_bf16 ? oracle_round_to_bf16(a) : a;
+    }
+    for (int n = 0; n < H; ++n) y[n] = 0.0;
+    for (int f = 0; f < F; ++f) {
+        double a = z[f];
+        const uint16_t *wrow = W2e + (size_t)f * H;
+        for (int n = 0; n < H; ++n) y[n] += a * (double)bf16_to_float(wrow[n]);
+    }
+}
+
+static size_t w1_expert_elems(int H, int F, int act)
+{
+    return (size_t)H * (size_t)(act == ORACLE_ACT_SWIGLU ? 2 * F : F);
+}
+
+/* Public single-row entry (used by tests for dense special cases). */
+void oracle_expert_ffn_row(int H, int F, int act, int round_a_bf16, const uint16_t *xrow,
+                           const uint16_t *W1e, const uint16_t *W2e, double *y)
+{
+    double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+    if (!scratch) return;
+    ffn_row(H, F, act, round_a_bf16, xrow, W1e, W2e, y, scratch);
+    free(scratch);
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Combine (§2.1: gather and reduce the top-k outputs)
+ * ------------------------------------------------------------------------------------- */
+
+/* out[t][n] = sum_{j=0..k-1} ys[inv_pos[t][j]][n], j ascending, fp64.
+ * ys holds bf16 rows that already carry the gate weight. */
+void oracle_combine(int T, int H, int k, const uint16_t *ys, const int32_t *inv_pos, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int n = 0; n < H; ++n) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int r = inv_pos[(size_t)t * k + j];
+                s += (double)bf16_to_float(ys[(size_t)r * H + n]);
+            }
+            out[(size_t)t * H + n] = s;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Whole layer
+ * ------------------------------------------------------------------------------------- */
+
+/* The layer in the pages' order: route -> dispatch into expert-contiguous rows ->
+ * per-expert FFN over its rows -> weighted top-k reduce per token.
+ * out: [T,H] fp64. idx_out [T,k] and w_out [T,k] are optional (NULL to skip).
+ * Returns 0 on success. Memory use is about (T*k + E*m_tile) * H doubles, so this entry
+ * is meant for small layers; large layers use oracle_moe_tokens on a token sample. */
+int oracle_moe_forward(int T, int H, int F, int E, int k, int act, int gate, int m_tile,
+                       int round_a_bf16, const uint16_t *x, const uint16_t *Wg, const float *bias,
+                       const uint16_t *W1, const uint16_t *W2, double *out, int32_t *idx_out,
+                       double *w_out)
+{
+    if (T < 0 || H < 1 || F < 1 || E < 1 || k < 1 || k > E || m_tile < 1) return -1;
+    if (T == 0) return 0;
+    const size_t TK = (size_t)T * k;
+    const int64_t gather_len = (int64_t)TK + (int64_t)E * (m_tile - 1);
+    const int64_t tile_cap = gather_len / m_tile + E;
+    int rc = 0;
+
+    float *logits = (float *)malloc(sizeof(float) * (size_t)T * E);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * TK);
+    double *w = (double *)malloc(sizeof(double) * TK);
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *poff = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *gather_idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)gather_len);
+    int32_t *inv_pos = (int32_t *)malloc(sizeof(int32_t) * TK);
+    int32_t *t_e = (int32_t *)malloc(sizeof(int32_t) * (size_t)tile_cap);
+    int32_t *t_r = (int32_t *)malloc(sizeof(int32_t) * (size_t)tile_cap);
+    int32_t *t_n = (int32_t *)malloc(sizeof(int32_t) * (size_t)tile_cap);
+    double *y = (double *)malloc(sizeof(double) * (size_t)gather_len * H);
+    if (!logits || !idx || !w || !counts || !offsets || !poff || !gather_idx || !inv_pos || !t_e ||
+        !t_r || !t_n || !y) {
+        rc = -4;
+        goto done;
+    }
+
+    /* 1. route */
+    oracle_router_logits(T, H, E, x, Wg, bias, logits);
+    rc = oracle_topk_gates(T, E, k, gate, logits, idx, w);
+    if (rc) goto done;
+
+    /* 2. dispatch */
+    rc = oracle_dispatch(T, E, k, m_tile, idx, counts, offsets, poff, gather_idx, gather_len,
+                         inv_pos, t_e, t_r, t_n, tile_cap);
+    if (rc < 0) goto done;
+    rc = 0;
+
+    /* 3. experts: every real row of every expert, in expert-sorted order */
+    {
+        const size_t w1e = w1_expert_elems(H, F, act);
+        const size_t w2e = (size_t)F * H;
+        int bad = 0;
+#pragma omp parallel
+        {
+            double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < (int64_t)poff[E]; ++r) {
+                int t = gather_idx[r];
+                if (t < 0) continue;
+                if (!scratch) {
+#pragma omp atomic write
+                    bad = 1;
+                    continue;
+                }
+                /* the expert that owns padded row r */
+                int e = 0;
+                while (!(r >= poff[e] && r < poff[e + 1])) ++e;
+                ffn_row(H, F, act, round_a_bf16, x + (size_t)t * H, W1 + (size_t)e * w1e,
+                        W2 + (size_t)e * w2e, y + (size_t)r * H, scratch);
+            }
+            free(scratch);
+        }
+        if (bad) {
+            rc = -4;
+            goto done;
+        }
+    }
+
+    /* 4. combine: out[t] = sum_j w[t][j] * y[inv_pos[t][j]], j ascending */
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int n = 0; n < H; ++n) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int r = inv_pos[(size_t)t * k + j];
+                s += w[(size_t)t * k + j] * y[(size_t)r * H + n];
+            }
+            out[(size_t)t * H + n] = s;
+        }
+    }
+    if (idx_out) memcpy(idx_out, idx, sizeof(int32_t) * TK);
+    if (w_out) memcpy(w_out, w, sizeof(double) * TK);
+
+done:
+    free(logits);
+    free(idx);
+    free(w);
+    free(counts);
+    free(offsets);
+    free(poff);
+    free(gather_idx);
+    free(inv_pos);
+    free(t_e);
+    free(t_r);
+    free(t_n);
+    free(y);
+    return rc;
+}
+
+/* The layer output for a list of tokens, straight from the definition in §2.1:
+ *   out[t] = sum_j w_j * FFN_{e_j}(x_t)
+ * with no permutation at all. Tokens are independent, so a sample of tokens of a large
+ * layer is checked exactly as the whole layer would be.
+ * out: [ntok,H] fp64; idx_out [ntok,k] and w_out [ntok,k] optional. */
+int oracle_moe_tokens(int T, int H, int F, int E, int k, int act, int gate, int round_a_bf16,
+                      const uint16_t *x, const uint16_t *Wg, const float *bias, const uint16_t *W1,
+                      const uint16_t *W2, int ntok, const int32_t *tokens, double *out,
+                      int32_t *idx_out, double *w_out)
+{
+    if (H < 1 || F < 1 || E < 1 || k < 1 || k > E || ntok < 0) return -1;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -2;
+    const size_t w1e = w1_expert_elems(H, F, act);
+    const size_t w2e = (size_t)F * H;
+    int bad = 0;
+#pragma omp parallel
+    {
+        float *l = (float *)malloc(sizeof(float) * (size_t)E);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+        const int ok = l && taken && sel && w && y && scratch;
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < ntok; ++i) {
+            if (!ok) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            {
+                int t = tokens[i];
+                oracle_router_logits(1, H, E, x + (size_t)t * H, Wg, bias, l);
+                topk_one(E, k, gate, l, sel, w, taken);
+                double *o = out + (size_t)i * H;
+                for (int n = 0; n < H; ++n) o[n] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    int e = sel[j];
+                    ffn_row(H, F, act, round_a_bf16, x + (size_t)t * H, W1 + (size_t)e * w1e,
+                            W2 + (size_t)e * w2e, y, scratch);
+                    for (int n = 0; n < H; ++n) o[n] += w[j] * y[n];
+                }
+                if (idx_out) memcpy(idx_out + (size_t)i * k, sel, sizeof(int32_t) * (size_t)k);
+                if (w_out) memcpy(w_out + (size_t)i * k, w, sizeof(double) * (size_t)k);
+            }
+        }
+        free(l);
+        free(taken);
+        free(sel);
+        free(w);
+        free(y);
+        free(scratch);
+    }
+    return bad ? -4 : 0;
+}

@@ -1,0 +1,332 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Every pin is one of: a hand-worked closed form (tests/golden), exact integer arithmetic,
+a floating-point error bound, a mathematical identity, a special case that reduces to a
+dense matmul (numpy), or brute force over all experts. Each is chosen so that a plausible
+slip in the oracle (a dropped term, a transposed operand, a wrong index, a wrong tie-break,
+gate and up columns swapped) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_forward_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+ACTS = {"swiglu": oracle.ACT_SWIGLU, "gelu_tanh": oracle.ACT_GELU_TANH, "relu": oracle.ACT_RELU,
+        "identity": oracle.ACT_IDENTITY}
+GATES = {"softmax_topk": oracle.GATE_SOFTMAX_TOPK, "softmax_all": oracle.GATE_SOFTMAX_ALL}
+
+
+def bf16(a):
+    """Exact small values -> bf16 bit patterns (asserts exact representability)."""
+    t = torch.tensor(np.asarray(a, dtype=np.float64), dtype=torch.float64)
+    b = t.to(torch.bfloat16)
+    assert torch.equal(b.to(torch.float64), t), "value not exact in bf16"
+    return synth.bf16_bits(b)
+
+
+def widen(u16):
+    return synth.from_bf16_bits(u16).to(torch.float64).numpy()
+
+
+def rand_bf16(shape, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return synth.bf16_bits((torch.randn(shape, generator=g) * std).to(torch.bfloat16))
+
+
+def distinct_topk_idx(T, E, k, seed):
+    rng = np.random.default_rng(seed)
+    return np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+
+
+# ------------------------------------------------------------------------------------
+# hand-worked closed forms
+# ------------------------------------------------------------------------------------
+
+def test_golden_hand_worked_cases(oracle_lib):
+    with open(os.path.join(GOLDEN, "hand_worked.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        x, Wg, W1, W2 = (bf16(c[n]) for n in ("x", "Wg", "W1", "W2"))
+        out, idx, w = oracle.moe_forward(x, Wg, None, W1, W2, c["k"], act=ACTS[c["act"]],
+                                         gate=GATES[c["gate"]], lib=oracle_lib)
+        assert idx.tolist() == c["expected_idx"], c["name"]
+        np.testing.assert_allclose(w, c["expected_w"], rtol=1e-14, atol=0, err_msg=c["name"])
+        np.testing.assert_allclose(out, c["expected_out"], rtol=1e-14, atol=1e-15, err_msg=c["name"])
+        # the per-token definition path agrees as well
+        out2, idx2, w2 = oracle.moe_tokens(x, Wg, None, W1, W2, c["k"], np.arange(c["T"]),
+                                           act=ACTS[c["act"]], gate=GATES[c["gate"]], lib=oracle_lib)
+        assert idx2.tolist() == c["expected_idx"]
+        np.testing.assert_allclose(out2, c["expected_out"], rtol=1e-14, atol=1e-15)
+
+
+def test_round_to_bf16_hand_cases(oracle_lib):
+    cases = {
+        1.0: 1.0,
+        1 + 2**-8: 1.0,                      # tie, even neighbour is 1.0
+        1 + 3 * 2**-8: 1 + 2**-6,            # tie, even neighbour is 1 + 2/128
+        1 + 2**-8 + 2**-20: 1 + 2**-7,       # just above the tie
+        -3.0: -3.0,
+        0.1: 0.10009765625,                  # bf16 0x3DCD
+        -(2**-100) * 1.00390625: -(2**-100), # tie at a small exponent
+    }
+    for v, want in cases.items():
+        assert oracle.round_to_bf16(v, lib=oracle_lib) == want, v
+
+
+# ------------------------------------------------------------------------------------
+# router logits: exact integers, summation order, error bound
+# ------------------------------------------------------------------------------------
+
+def test_router_logits_small_integers_exact(oracle_lib):
+    rng = np.random.default_rng(1)
+    T, H, E = 7, 96, 5
+    xi = rng.integers(-4, 5, size=(T, H))
+    wi = rng.integers(-4, 5, size=(H, E))
+    bi = rng.integers(-8, 9, size=E).astype(np.float32)
+    got = oracle.router_logits(bf16(xi), bf16(wi), bi, lib=oracle_lib)
+    want = (xi @ wi).astype(np.float64) + bi      # exact integers, well below 2^24
+    np.testing.assert_array_equal(got.astype(np.float64), want)
+
+
+def test_router_logits_sequential_fp32_order(oracle_lib):
+    # x . w with w = 1 and x = [2^24, 1, 1, -2^24]: a single fp32 accumulator walking h
+    # upward loses both ones (2^24 + 1 rounds back to 2^24) and ends at 0; the exact sum
+    # is 2, and the order [1, 1, 2^24, -2^24] keeps them (result 2).
+    x = bf16([[2**24, 1, 1, -(2**24)], [1, 1, 2**24, -(2**24)]])
+    w = bf16(np.ones((4, 1)))
+    got = oracle.router_logits(x, w, None, lib=oracle_lib)
+    assert got[0, 0] == 0.0 and got[1, 0] == 2.0
+
+
+def test_router_logits_within_fp32_error_bound(oracle_lib):
+    T, H, E = 32, 1024, 16
+    x = rand_bf16((T, H), 11)
+    Wg = rand_bf16((H, E), 12, std=1 / math.sqrt(H))
+    bias = np.linspace(-1, 1, E).astype(np.float32)
+    got = oracle.router_logits(x, Wg, bias, lib=oracle_lib).astype(np.float64)
+    xf, wf = widen(x), widen(Wg)
+    exact = xf @ wf + bias.astype(np.float64)
+    absdot = np.abs(xf) @ np.abs(wf)
+    u = 2.0**-24
+    gamma = (H + 1) * u / (1 - (H + 1) * u)       # H products summed, plus the bias add
+    bound = gamma * (absdot + np.abs(bias)) + 1e-30
+    assert np.all(np.abs(got - exact) <= bound)
+    # and it really is fp32 (not a wider accumulator): some entries differ from exact
+    assert np.any(got != exact)
+
+
+# ------------------------------------------------------------------------------------
+# top-k selection and gates
+# ------------------------------------------------------------------------------------
+
+def test_topk_order_and_ties(oracle_lib):
+    l = np.array([[1.0, 3.0, 3.0, 2.0, -0.0, 0.0]], np.float32)
+    idx, _ = oracle.topk_gates(l, 6, lib=oracle_lib)
+    assert idx.tolist() == [[1, 2, 3, 0, 4, 5]]       # equal values: lower id first; -0 == +0
+    idx, _ = oracle.topk_gates(l, 2, lib=oracle_lib)
+    assert idx.tolist() == [[1, 2]]
+
+
+def test_router_ties_from_duplicated_gate_columns(oracle_lib):
+    T, H = 64, 128
+    x = rand_bf16((T, H), 3)
+    base = rand_bf16((H, 4), 4, std=1 / math.sqrt(H))
+    Wg = np.ascontiguousarray(base[:, [0, 1, 2, 3, 3, 2, 1, 0]])   # experts 4..7 copy 3..0
+    logits = oracle.router_logits(x, Wg, None, lib=oracle_lib)
+    assert np.array_equal(logits[:, :4], logits[:, [7, 6, 5, 4]])
+    idx, w = oracle.topk_gates(logits, 2, lib=oracle_lib)
+    # the best logit always appears twice, so both selected experts share one value and
+    # the pair is (lower copy, higher copy)
+    mirror = {0: 7, 1: 6, 2: 5, 3: 4}
+    for t in range(T):
+        a, b = idx[t]
+        assert a < 4 and b == mirror[a]
+        assert w[t, 0] == w[t, 1] == 0.5
+
+
+def test_gates_match_full_softmax_then_renormalise(oracle_lib):
+    T, E, k = 50, 12, 3
+    rng = np.random.default_rng(5)
+    logits = (rng.standard_normal((T, E)) * 3).astype(np.float32)
+    idx, w = oracle.topk_gates(logits, k, lib=oracle_lib)
+    l64 = logits.astype(np.float64)
+    full = np.exp(l64 - l64.max(axis=1, keepdims=True))
+    full /= full.sum(axis=1, keepdims=True)
+    sel = np.take_along_axis(full, idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w, sel / sel.sum(axis=1, keepdims=True), rtol=1e-13)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=k * 2**-52)
+    assert np.all(np.diff(w, axis=1) <= 0)
+    # indices are the k largest, in descending order
+    ref = np.argsort(-l64, axis=1, kind="stable")[:, :k]
+    assert np.array_equal(idx, ref)
+    # SOFTMAX_ALL keeps the full-softmax values
+    idx2, w2 = oracle.topk_gates(logits, k, gate=oracle.GATE_SOFTMAX_ALL, lib=oracle_lib)
+    assert np.array_equal(idx2, idx)
+    np.testing.assert_allclose(w2, sel, rtol=1e-13)
+    # k = 1 gives a weight of exactly one
+    _, w1 = oracle.topk_gates(logits, 1, lib=oracle_lib)
+    assert np.all(w1 == 1.0)
+
+
+# ------------------------------------------------------------------------------------
+# dispatch: counting sort against a library stable sort, plus invariants
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,m_tile", [(300, 8, 2, 128), (97, 64, 8, 128), (5, 16, 3, 4),
+                                          (1000, 3, 3, 128), (0, 4, 1, 128)])
+def test_dispatch_matches_stable_sort(oracle_lib, T, E, k, m_tile):
+    idx = distinct_topk_idx(T, E, k, seed=T + E) if T else np.zeros((0, k), np.int32)
+    d = oracle.dispatch(idx, E, m_tile=m_tile, lib=oracle_lib)
+    flat = idx.reshape(-1)
+    counts = np.bincount(flat, minlength=E)
+    assert np.array_equal(d["counts"], counts)
+    assert d["counts"].sum() == T * k
+    assert np.array_equal(d["offsets"], np.concatenate([[0], np.cumsum(counts)]))
+    padded = -(-counts // m_tile) * m_tile
+    poff = np.concatenate([[0], np.cumsum(padded)])
+    assert np.array_equal(d["padded_offsets"], poff)
+    order = np.argsort(flat, kind="stable")            # pair ids sorted by expert, token-stable
+    gi = d["gather_idx"]
+    for e in range(E):
+        pairs = order[d["offsets"][e]:d["offsets"][e + 1]]
+        rows = gi[poff[e]:poff[e] + counts[e]]
+        assert np.array_equal(rows, pairs // k)
+        assert np.all(np.diff(rows) > 0)                  # ascending token id
+        assert np.all(gi[poff[e] + counts[e]:poff[e + 1]] == -1)
+    assert np.all(gi[poff[E]:] == -1)
+    inv = d["inv_pos"]
+    for t in range(T):
+        for j in range(k):
+            r = inv[t, j]
+            assert gi[r] == t and poff[flat[t * k + j]] <= r < poff[flat[t * k + j] + 1]
+    # tiles: one per m_tile block of each expert's rows
+    nt = int(np.sum(-(-counts // m_tile)))
+    assert d["num_tiles"] == nt
+    want = [(e, poff[e] + i * m_tile, min(m_tile, counts[e] - i * m_tile))
+            for e in range(E) for i in range(-(-counts[e] // m_tile))]
+    got = list(zip(d["tile_expert"], d["tile_row0"], d["tile_nvalid"]))
+    assert [tuple(map(int, g)) for g in got] == [tuple(map(int, w_)) for w_ in want]
+
+
+def test_permute_then_unpermute_is_identity(oracle_lib):
+    T, H, E, k = 200, 24, 10, 4
+    x = rand_bf16((T, H), 9)
+    idx = distinct_topk_idx(T, E, k, seed=9)
+    d = oracle.dispatch(idx, E, lib=oracle_lib)
+    gi = d["gather_idx"]
+    xp = np.zeros((gi.shape[0], H), np.uint16)
+    xp[gi >= 0] = x[gi[gi >= 0]]
+    for j in range(k):
+        assert np.array_equal(xp[d["inv_pos"][:, j]], x)
+
+
+# ------------------------------------------------------------------------------------
+# experts and whole layer
+# ------------------------------------------------------------------------------------
+
+def _np_act(act, z):
+    if act == oracle.ACT_GELU_TANH:
+        return 0.5 * z * (1 + np.tanh(math.sqrt(2 / math.pi) * (z + 0.044715 * z**3)))
+    if act == oracle.ACT_RELU:
+        return np.maximum(z, 0)
+    return z
+
+
+def _np_ffn(x64, W1e, W2e, act, F):
+    z = x64 @ W1e
+    a = z[:, :F] / (1 + np.exp(-z[:, :F])) * z[:, F:] if act == oracle.ACT_SWIGLU else _np_act(act, z)
+    return a @ W2e
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_SWIGLU, oracle.ACT_GELU_TANH, oracle.ACT_RELU,
+                                 oracle.ACT_IDENTITY])
+def test_single_expert_top1_is_dense_ffn(oracle_lib, act):
+    T, H, F = 9, 64, 40
+    c = 2 * F if act == oracle.ACT_SWIGLU else F
+    x = rand_bf16((T, H), 21)
+    Wg = rand_bf16((H, 1), 22)
+    W1 = rand_bf16((1, H, c), 23, std=1 / math.sqrt(H))
+    W2 = rand_bf16((1, F, H), 24, std=1 / math.sqrt(F))
+    out, idx, w = oracle.moe_forward(x, Wg, None, W1, W2, 1, act=act, lib=oracle_lib)
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    want = _np_ffn(widen(x), widen(W1[0]), widen(W2[0]), act, F)
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_experts_reproduce_x(oracle_lib):
+    T, H, E, k = 40, 16, 5, 3
+    x = rand_bf16((T, H), 31)
+    Wg = rand_bf16((H, E), 32, std=1 / math.sqrt(H))
+    eye = np.broadcast_to(np.eye(H), (E, H, H))
+    W = bf16(eye)
+    out, _, w = oracle.moe_forward(x, Wg, None, W, W, k, act=oracle.ACT_IDENTITY, lib=oracle_lib)
+    np.testing.assert_allclose(out, widen(x), rtol=4e-16 * k, atol=0)
+
+
+@pytest.mark.parametrize("act,gate,use_bias", [(oracle.ACT_SWIGLU, oracle.GATE_SOFTMAX_TOPK, False),
+                                               (oracle.ACT_SWIGLU, oracle.GATE_SOFTMAX_ALL, True),
+                                               (oracle.ACT_GELU_TANH, oracle.GATE_SOFTMAX_TOPK, True),
+                                               (oracle.ACT_RELU, oracle.GATE_SOFTMAX_TOPK, False)])
+def test_layer_equals_dense_masked_sum_over_all_experts(oracle_lib, act, gate, use_bias):
+    """Brute force: run every expert on every token (numpy matmuls), then mask with the
+    gate matrix; routing from fp64 logits with a full stable sort."""
+    T, H, F, E, k = 48, 64, 32, 6, 2
+    c = 2 * F if act == oracle.ACT_SWIGLU else F
+    x = rand_bf16((T, H), 41)
+    Wg = rand_bf16((H, E), 42)            # unscaled: well separated logits
+    W1 = rand_bf16((E, H, c), 43, std=1 / math.sqrt(H))
+    W2 = rand_bf16((E, F, H), 44, std=1 / math.sqrt(F))
+    bias = np.linspace(0.5, -0.5, E).astype(np.float32) if use_bias else None
+    out, idx, w = oracle.moe_forward(x, Wg, bias, W1, W2, k, act=act, gate=gate, lib=oracle_lib)
+
+    xf = widen(x)
+    # the fp32 logits are pinned by the router tests above; from here on everything is
+    # recomputed independently: full stable sort, full softmax, every expert on every token
+    l = oracle.router_logits(x, Wg, bias, lib=oracle_lib).astype(np.float64)
+    l_exact = xf @ widen(Wg) + (0 if bias is None else bias.astype(np.float64))
+    np.testing.assert_allclose(l, l_exact, rtol=0, atol=1e-3)
+    sel = np.argsort(-l, axis=1, kind="stable")[:, :k]
+    G = np.zeros((T, E))
+    p = np.exp(l - l.max(axis=1, keepdims=True))
+    for t in range(T):
+        if gate == oracle.GATE_SOFTMAX_ALL:
+            G[t, sel[t]] = p[t, sel[t]] / p[t].sum()
+        else:
+            G[t, sel[t]] = p[t, sel[t]] / p[t, sel[t]].sum()
+    dense = np.stack([_np_ffn(xf, widen(W1[e]), widen(W2[e]), act, F) for e in range(E)], axis=1)
+    want = np.einsum("te,teh->th", G, dense)
+    assert np.array_equal(idx, sel)
+    np.testing.assert_allclose(out, want, rtol=1e-10, atol=1e-12)
+    toks = np.array([0, 5, 17, 47], np.int32)
+    out_t, idx_t, _ = oracle.moe_tokens(x, Wg, bias, W1, W2, k, toks, act=act, gate=gate, lib=oracle_lib)
+    assert np.array_equal(idx_t, sel[toks])
+    np.testing.assert_allclose(out_t, want[toks], rtol=1e-10, atol=1e-12)
+
+
+def test_combine_is_row_gather_sum(oracle_lib):
+    T, H, E, k = 77, 40, 9, 3
+    idx = distinct_topk_idx(T, E, k, seed=51)
+    d = oracle.dispatch(idx, E, lib=oracle_lib)
+    ys = rand_bf16((d["gather_idx"].shape[0], H), 52)
+    got = oracle.combine(ys, d["inv_pos"], lib=oracle_lib)
+    want = widen(ys)[d["inv_pos"]].sum(axis=1)
+    np.testing.assert_allclose(got, want, rtol=1e-15, atol=0)
+
+
+def test_round_a_bf16_flag_changes_only_by_rounding(oracle_lib):
+    T, H, F, E, k = 16, 64, 64, 4, 2
+    x = rand_bf16((T, H), 61)
+    Wg = rand_bf16((H, E), 62)
+    W1 = rand_bf16((E, H, 2 * F), 63, std=1 / math.sqrt(H))
+    W2 = rand_bf16((E, F, H), 64, std=1 / math.sqrt(F))
+    a, _, _ = oracle.moe_forward(x, Wg, None, W1, W2, k, lib=oracle_lib)
+    b, _, _ = oracle.moe_forward(x, Wg, None, W1, W2, k, round_a_bf16=True, lib=oracle_lib)
+    assert not np.array_equal(a, b)
+    np.testing.assert_allclose(a, b, rtol=0, atol=2**-8 * np.abs(a).max() * 2)
