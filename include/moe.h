@@ -1,0 +1,196 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of one mixture-of-experts layer.
+ *
+ * The layer is the one described in "Comet: Fine-grained Computation-communication
+ * Overlapping for Mixture-of-Experts", §2.1 "MoE Structure": every token is routed to
+ * its top-k experts, each selected expert applies its feed-forward network to the token,
+ * and the k expert outputs are gathered back and reduced with the gate weights. The
+ * dispatch step reorganises the routed tokens into expert-contiguous, tile-aligned rows
+ * (§2.2.1 and §3.1.2, "How to reschedule the decomposed shared tensor?"); layer0 is
+ * decomposed along M (token rows) and layer1 along N (output columns) (§3.1.1).
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, unless the entry point
+ *     says HOST. The library never allocates device memory: scratch space comes from the
+ *     caller's workspace (moe_workspace_size()).
+ *   - bf16 tensors are passed as moe_bf16 (the raw 16-bit pattern), row-major, 16-byte
+ *     aligned. int32/fp32 tensors are 4-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). All work is enqueued
+ *     asynchronously on it; no entry point synchronises except moe_get_device_status and
+ *     moe_forward_host (which waits for its own device-to-host copy).
+ *   - Host-detectable errors (NULL pointers, unsupported sizes, a short workspace) are
+ *     returned at once and nothing is launched. Errors found on the device (an expert id
+ *     out of range, a bounded wait that ran out) are written to a status word in the
+ *     workspace and returned by moe_get_device_status().
+ *   - No C++ exception crosses this boundary.
+ *   - The caller's buffers may not overlap each other or the workspace.
+ *   - Concurrent calls that share one workspace race; give each stream its own.
+ *
+ * Supported problem sizes: T >= 0, H % 64 == 0, F % 64 == 0, 1 <= top_k <= E <= 1024,
+ * m_tile == 128; anything else returns MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bfloat16 bit pattern (sign, 8 exponent bits, 7 mantissa bits). */
+typedef uint16_t moe_bf16;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,    /* NULL pointer, negative size, top_k > E, ... */
+    MOE_ERR_UNSUPPORTED = -2,    /* legal but not supported by these kernels (see above) */
+    MOE_ERR_WORKSPACE = -3,      /* ws_bytes smaller than moe_workspace_size() */
+    MOE_ERR_CUDA = -4,           /* a CUDA runtime call failed (launch, copy, attribute) */
+    MOE_ERR_DEVICE_TIMEOUT = -5, /* a bounded device wait ran out (status word) */
+    MOE_ERR_DEVICE_BAD_INDEX = -6 /* an expert id or row index out of range (status word) */
+} moe_status;
+
+/* Expert activation. SWIGLU uses W1 [E, H, 2F]: columns [0, F) are the gate projection
+ * (through silu), columns [F, 2F) the up projection; h = silu(x W_gate) * (x W_up).
+ * The other three use W1 [E, H, F] and h = act(x W1). */
+typedef enum {
+    MOE_ACT_SWIGLU = 0,
+    MOE_ACT_GELU_TANH = 1,
+    MOE_ACT_RELU = 2,
+    MOE_ACT_IDENTITY = 3
+} moe_act;
+
+/* Gate weights of the k selected experts (selection is always the k largest logits,
+ * ties broken toward the lower expert id).
+ * SOFTMAX_TOPK: softmax over the k selected logits. In exact arithmetic this equals a
+ *   softmax over all E logits renormalised over the selected k (Mixtral's "softmax over
+ *   the top-k logits" and Qwen2's "renormalised top-k gates" are the same function).
+ * SOFTMAX_ALL: the full-E softmax values of the selected experts, not renormalised. */
+typedef enum {
+    MOE_GATE_SOFTMAX_TOPK = 0,
+    MOE_GATE_SOFTMAX_ALL = 1
+} moe_gate;
+
+typedef struct {
+    int32_t T;      /* tokens */
+    int32_t H;      /* hidden size (model dimension) */
+    int32_t F;      /* expert FFN size */
+    int32_t E;      /* number of experts */
+    int32_t top_k;  /* experts per token */
+    int32_t act;    /* moe_act */
+    int32_t gate;   /* moe_gate */
+    int32_t m_tile; /* row-tile height of the grouped GEMMs; must be 128 */
+} moe_problem;
+
+/* Number of stage boundaries recorded by moe_forward_staged: before routing, after
+ * routing, after dispatch, after layer0, after layer1, after combine. */
+#define MOE_NUM_STAGE_EVENTS 6
+
+/* Bytes of workspace that is enough for every entry point on problem *p (moe_forward_host
+ * uses all of it; moe_route, moe_dispatch and moe_forward use a prefix of it and accept a
+ * buffer of this size). The caller allocates it, 256-byte aligned, and may reuse it across
+ * calls on one stream. 0 if *p is invalid. */
+MOE_API size_t moe_workspace_size(const moe_problem *p);
+
+/* Upper bound on the padded row count P_pad = sum_e ceil(c_e / m_tile) * m_tile, namely
+ * T*top_k + min(E, T*top_k) * (m_tile - 1). gather_idx and ys buffers are sized with it,
+ * so no host read of the expert counts is ever needed. -1 if *p is invalid. */
+MOE_API int64_t moe_padded_rows_max(const moe_problem *p);
+
+/* Router (§2.1: tokens are routed to selected experts at run time; §2.2.2: the
+ * resulting expert loads vary).
+ *   logits[t][e] = sum_h x[t][h] * Wg[h][e] (+ bias[e]), fp32, one accumulator per
+ *   (t, e) walking h upward (this order is part of the contract: the selection below
+ *   is bit-exact against a CPU reference that sums the same way);
+ *   topk_idx[t][0..k-1] = the k largest logits, descending, ties to the lower id;
+ *   topk_w[t][j] = gate weight per moe_gate.
+ * x [T, H] bf16; Wg [H, E] bf16 (E contiguous); bias [E] fp32 or NULL;
+ * topk_idx [T, k] int32 (out); topk_w [T, k] fp32 (out); ws/ws_bytes: workspace. */
+MOE_API moe_status moe_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                     const float *bias, int32_t *topk_idx, float *topk_w, void *ws,
+                     size_t ws_bytes, void *stream);
+
+/* Dispatch (§2.2.1 and §3.1.2: expose to each computation tile only the rows it needs;
+ * regroup the routed rows into whole GEMM tiles). A counting sort of the T*k routed
+ * pairs by expert, stable in token id, with each expert's rows padded to a multiple of
+ * m_tile:
+ *   counts[e]         pairs routed to expert e                                  [E]
+ *   offsets[e]        exclusive prefix sum of counts                            [E+1]
+ *   padded_offsets[e] exclusive prefix sum of ceil(counts/m_tile)*m_tile        [E+1]
+ *   gather_idx[r]     token held by padded row r, -1 for a pad row   [moe_padded_rows_max]
+ *   inv_pos[t][j]     padded row that holds pair (t, j)                         [T, k]
+ *   x_perm (optional, may be NULL): x_perm[r] = x[gather_idx[r]], zeros on pad rows,
+ *                     [moe_padded_rows_max, H] bf16; needs x.
+ * topk_idx [T, k] int32 must hold distinct experts per token; an id outside [0, E) is
+ * skipped and reported as MOE_ERR_DEVICE_BAD_INDEX by moe_get_device_status. */
+MOE_API moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *counts,
+                        int32_t *offsets, int32_t *padded_offsets, int32_t *gather_idx,
+                        int32_t *inv_pos, moe_bf16 *x_perm, const moe_bf16 *x, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/* The whole layer: route -> dispatch -> layer0 grouped GEMM with the activation fused
+ * in its epilogue (decomposed along M, §3.1.1) -> layer1 grouped GEMM with the gate
+ * weight fused in its epilogue (decomposed along N, §3.1.1, column-wise §3.1.2) ->
+ * deterministic top-k reduce (j ascending, fp32, rounded once to bf16).
+ *   x [T, H] bf16; Wg [H, E] bf16; bias [E] fp32 or NULL;
+ *   W1 [E, H, 2F] bf16 for SWIGLU, [E, H, F] otherwise; W2 [E, F, H] bf16;
+ *   out [T, H] bf16 (out);
+ *   topk_idx_out [T, k] int32 and topk_w_out [T, k] fp32: optional copies of the routing
+ *   (NULL to keep them in the workspace only). */
+MOE_API moe_status moe_forward(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                       const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
+                       int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* moe_forward, plus cudaEventRecord of events[i] (cudaEvent_t handles owned by the
+ * caller) at the MOE_NUM_STAGE_EVENTS stage boundaries, for per-stage timing.
+ * n_events must be 0 (no events) or MOE_NUM_STAGE_EVENTS. */
+MOE_API moe_status moe_forward_staged(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                              const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                              moe_bf16 *out, int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                              size_t ws_bytes, void *stream, void *const *events, int n_events);
+
+/* moe_forward with HOST activations: x_host [T, H] and out_host [T, H] are host buffers
+ * (pinned for asynchronous copies); the weights stay on the device. The call copies x
+ * into the workspace, runs the layer, copies out back and waits for that copy, so
+ * out_host is valid on return. */
+MOE_API moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const moe_bf16 *Wg,
+                            const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                            moe_bf16 *out_host, void *ws, size_t ws_bytes, void *stream);
+
+/* Combine (§2.1: gather and reduce the top-k outputs).
+ *   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] ), fp32 sum, j ascending.
+ * ys [ys_rows, H] bf16 holds expert-sorted rows that already carry their gate weight;
+ * inv_pos [T, k] int32 as produced by moe_dispatch. A row index outside [0, ys_rows)
+ * contributes nothing; if ws is not NULL it is also reported as MOE_ERR_DEVICE_BAD_INDEX
+ * through moe_get_device_status (ws may be NULL, then ws_bytes is ignored). */
+MOE_API moe_status moe_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_rows,
+                       const int32_t *inv_pos, moe_bf16 *out, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Synchronises `stream`, then reads and clears the device status word in ws.
+ * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BAD_INDEX or MOE_ERR_CUDA.
+ * Every other entry point clears the word when its first kernel starts. */
+MOE_API moe_status moe_get_device_status(void *ws, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char *moe_status_string(moe_status s);
+
+/* Test hook for the bounded device waits: the timeout, in nanoseconds, that every
+ * bounded wait of later launches uses (default 2e9; values <= 0 restore the default).
+ * Returns the previous value. Not thread-safe; meant for tests. */
+MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,1 +1,34 @@
-"""B200-native forward pass of one mixture-of-experts layer (placeholder; binding follows)."""
+"""B200-native (sm_100a) forward pass of one mixture-of-experts layer.
+
+The layer (Comet: Fine-grained Computation-communication Overlapping for Mixture-of-Experts,
+§2.1 "MoE Structure") runs entirely in the CUDA kernels of ``libmoe_b200.so``; this package
+only marshals arguments to its C ABI (include/moe.h). PyTorch supplies device memory and
+streams. There is no CPU fallback: if the library is missing every call raises.
+
+Public names mirror the C ABI: ``moe_workspace_size``, ``moe_padded_rows_max``,
+``moe_route``, ``moe_dispatch``, ``moe_forward``, ``moe_forward_staged``,
+``moe_forward_host``, ``moe_combine``, ``moe_get_device_status``.
+"""
+from ._native import (  # noqa: F401
+    ACT_GELU_TANH,
+    ACT_IDENTITY,
+    ACT_RELU,
+    ACT_SWIGLU,
+    GATE_SOFTMAX_ALL,
+    GATE_SOFTMAX_TOPK,
+    MOE_NUM_STAGE_EVENTS,
+    MoeError,
+    Problem,
+    library,
+    library_path,
+    moe_combine,
+    moe_dispatch,
+    moe_forward,
+    moe_forward_host,
+    moe_forward_staged,
+    moe_get_device_status,
+    moe_padded_rows_max,
+    moe_route,
+    moe_set_wait_timeout_ns,
+    moe_workspace_size,
+)

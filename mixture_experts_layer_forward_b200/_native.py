@@ -1,0 +1,225 @@
+"""ctypes binding of libmoe_b200.so (include/moe.h). Argument marshalling only.
+
+Every function takes torch tensors (or None for optional pointers), checks dtype, device
+and contiguity, passes ``data_ptr()`` and the current CUDA stream to the C entry point of
+the same name, and raises ``MoeError`` on a non-OK status. No computation of the layer
+happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+from pathlib import Path
+
+import torch
+
+from .build import LIB_PATH
+
+ACT_SWIGLU, ACT_GELU_TANH, ACT_RELU, ACT_IDENTITY = 0, 1, 2, 3
+GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL = 0, 1
+MOE_NUM_STAGE_EVENTS = 6
+M_TILE = 128
+
+STATUS_NAMES = {
+    0: "MOE_OK",
+    -1: "MOE_ERR_INVALID_ARG",
+    -2: "MOE_ERR_UNSUPPORTED",
+    -3: "MOE_ERR_WORKSPACE",
+    -4: "MOE_ERR_CUDA",
+    -5: "MOE_ERR_DEVICE_TIMEOUT",
+    -6: "MOE_ERR_DEVICE_BAD_INDEX",
+}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("gate", ctypes.c_int32), ("m_tile", ctypes.c_int32)]
+
+    @classmethod
+    def make(cls, T, H, F, E, top_k, act=ACT_SWIGLU, gate=GATE_SOFTMAX_TOPK, m_tile=M_TILE):
+        return cls(T, H, F, E, top_k, act, gate, m_tile)
+
+    @classmethod
+    def from_config(cls, cfg):
+        return cls.make(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, cfg.act, cfg.gate)
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> Path:
+    return LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """Load libmoe_b200.so. Raises if it has not been built: there is no fallback path."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not LIB_PATH.exists():
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; "
+                f"g.build()'` (nvcc, sm_100a). There is no CPU fallback.")
+        lib = ctypes.CDLL(str(LIB_PATH))
+        vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64
+        P = ctypes.POINTER(Problem)
+        sig = {
+            "moe_workspace_size": ([P], sz),
+            "moe_padded_rows_max": ([P], i64),
+            "moe_route": ([P, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_dispatch": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_forward": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_forward_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                    ctypes.POINTER(vp), i32], i32),
+            "moe_forward_host": ([P, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
+            "moe_get_device_status": ([vp, vp], i32),
+            "moe_status_string": ([i32], ctypes.c_char_p),
+            "moe_set_wait_timeout_ns": ([i64], i64),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = lib
+        return lib
+
+
+# ---------------------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------------------
+
+def _ptr(t, dtype=None, name="tensor", cuda=True):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not cuda and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MoeError(fn, rc)
+
+
+def _ws(ws):
+    return _ptr(ws, torch.uint8, "ws"), ctypes.c_size_t(ws.numel())
+
+
+# ---------------------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------------------
+
+def moe_workspace_size(p: Problem) -> int:
+    return int(library().moe_workspace_size(ctypes.byref(p)))
+
+
+def moe_padded_rows_max(p: Problem) -> int:
+    return int(library().moe_padded_rows_max(ctypes.byref(p)))
+
+
+def moe_route(p, x, Wg, bias, topk_idx, topk_w, ws, stream=None):
+    bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
+    w, n = _ws(ws)
+    rc = library().moe_route(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                             _ptr(bias, f32, "bias"), _ptr(topk_idx, i32, "topk_idx"),
+                             _ptr(topk_w, f32, "topk_w"), w, n, _stream(stream))
+    _check("moe_route", rc)
+
+
+def moe_dispatch(p, topk_idx, counts, offsets, padded_offsets, gather_idx, inv_pos, ws,
+                 x_perm=None, x=None, stream=None):
+    bf, i32 = torch.bfloat16, torch.int32
+    w, n = _ws(ws)
+    rc = library().moe_dispatch(ctypes.byref(p), _ptr(topk_idx, i32, "topk_idx"),
+                                _ptr(counts, i32, "counts"), _ptr(offsets, i32, "offsets"),
+                                _ptr(padded_offsets, i32, "padded_offsets"),
+                                _ptr(gather_idx, i32, "gather_idx"), _ptr(inv_pos, i32, "inv_pos"),
+                                _ptr(x_perm, bf, "x_perm"), _ptr(x, bf, "x"), w, n, _stream(stream))
+    _check("moe_dispatch", rc)
+
+
+def moe_forward(p, x, Wg, bias, W1, W2, out, ws, topk_idx_out=None, topk_w_out=None, stream=None):
+    bf = torch.bfloat16
+    w, n = _ws(ws)
+    rc = library().moe_forward(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                               _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
+                               _ptr(W2, bf, "W2"), _ptr(out, bf, "out"),
+                               _ptr(topk_idx_out, torch.int32, "topk_idx_out"),
+                               _ptr(topk_w_out, torch.float32, "topk_w_out"), w, n, _stream(stream))
+    _check("moe_forward", rc)
+
+
+def moe_forward_staged(p, x, Wg, bias, W1, W2, out, ws, events, topk_idx_out=None,
+                       topk_w_out=None, stream=None):
+    """``events``: MOE_NUM_STAGE_EVENTS torch.cuda.Event(enable_timing=True) objects."""
+    bf = torch.bfloat16
+    w, n = _ws(ws)
+    if len(events) != MOE_NUM_STAGE_EVENTS:
+        raise ValueError(f"need {MOE_NUM_STAGE_EVENTS} events")
+    arr = (ctypes.c_void_p * MOE_NUM_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    rc = library().moe_forward_staged(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                                      _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
+                                      _ptr(W2, bf, "W2"), _ptr(out, bf, "out"),
+                                      _ptr(topk_idx_out, torch.int32, "topk_idx_out"),
+                                      _ptr(topk_w_out, torch.float32, "topk_w_out"), w, n,
+                                      _stream(stream), arr, MOE_NUM_STAGE_EVENTS)
+    _check("moe_forward_staged", rc)
+
+
+def moe_forward_host(p, x_host, Wg, bias, W1, W2, out_host, ws, stream=None):
+    """Activations on the host (pinned for async copies), weights on the device."""
+    bf = torch.bfloat16
+    w, n = _ws(ws)
+    rc = library().moe_forward_host(ctypes.byref(p), _ptr(x_host, bf, "x_host", cuda=False),
+                                    _ptr(Wg, bf, "Wg"), _ptr(bias, torch.float32, "bias"),
+                                    _ptr(W1, bf, "W1"), _ptr(W2, bf, "W2"),
+                                    _ptr(out_host, bf, "out_host", cuda=False), w, n,
+                                    _stream(stream))
+    _check("moe_forward_host", rc)
+
+
+def moe_combine(p, ys, inv_pos, out, ws=None, stream=None):
+    bf = torch.bfloat16
+    if ws is None:
+        w, n = None, ctypes.c_size_t(0)
+    else:
+        w, n = _ws(ws)
+    rc = library().moe_combine(ctypes.byref(p), _ptr(ys, bf, "ys"), ctypes.c_int64(ys.shape[0]),
+                               _ptr(inv_pos, torch.int32, "inv_pos"), _ptr(out, bf, "out"), w, n,
+                               _stream(stream))
+    _check("moe_combine", rc)
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    """Synchronise the stream, read and clear the device status word; returns the code."""
+    return int(library().moe_get_device_status(_ptr(ws, torch.uint8, "ws"), _stream(stream)))
+
+
+def moe_set_wait_timeout_ns(ns: int) -> int:
+    return int(library().moe_set_wait_timeout_ns(int(ns)))

@@ -1,0 +1,54 @@
+// combine.cuh -- top-k gather-reduce (Comet: Fine-grained Computation-communication
+// Overlapping for Mixture-of-Experts, §2.1 "MoE Structure": gather and reduce the top-k
+// expert outputs of each token).
+//
+//   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] )
+// The sum runs in fp32 with j ascending, so the result does not depend on scheduling.
+// Each thread owns 8 consecutive columns (one 16-byte vector) of one token; the grid
+// strides over T * H/8 vectors. HBM-bound: k*T*H*2 bytes read, T*H*2 bytes written.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256)
+    combine_kernel(const __nv_bfloat16 *__restrict__ ys, int64_t ys_rows,
+                   const int32_t *__restrict__ inv_pos, int T, int H, int k,
+                   __nv_bfloat16 *__restrict__ out, int *status, int clear_status)
+{
+    if (clear_status && status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        status[0] = DEV_OK;
+        status[1] = 0;
+    }
+    const int vec_per_row = H / 8;
+    const int64_t total = (int64_t)T * vec_per_row;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int t = (int)(i / vec_per_row);
+        const int v = (int)(i - (int64_t)t * vec_per_row);
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int r = inv_pos[(size_t)t * k + j];
+            if (r < 0 || (int64_t)r >= ys_rows) {
+                record_status(status, DEV_BAD_INDEX, 3);
+                continue;
+            }
+            const uint4 u = *reinterpret_cast<const uint4 *>(ys + (size_t)r * H + (size_t)v * 8);
+            acc[0] += bf16_lo(u.x); acc[1] += bf16_hi(u.x);
+            acc[2] += bf16_lo(u.y); acc[3] += bf16_hi(u.y);
+            acc[4] += bf16_lo(u.z); acc[5] += bf16_hi(u.z);
+            acc[6] += bf16_lo(u.w); acc[7] += bf16_hi(u.w);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4 *>(out + (size_t)t * H + (size_t)v * 8) = o;
+    }
+}
+
+} // namespace moe

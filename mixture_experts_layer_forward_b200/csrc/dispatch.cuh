@@ -1,0 +1,215 @@
+// dispatch.cuh -- token dispatch into expert-contiguous, tile-padded rows
+// (Comet: Fine-grained Computation-communication Overlapping for Mixture-of-Experts,
+// §2.2.1: expose to each computation tile only the rows it needs; §3.1.2: regroup the
+// decomposed rows into whole GEMM tiles).
+//
+// A deterministic counting sort of the T*k routed pairs by expert, stable in token id:
+//   dispatch_count_kernel   per token chunk, per-expert pair counts           [nchunk][E]
+//   dispatch_scan_kernel    per-expert scan over chunks, expert counts, offsets, padded
+//                           offsets, the m-tile list, pad-row markers         (one block)
+//   dispatch_place_kernel   each pair's row = padded_offset[e] + chunk base + rank of the
+//                           token among the chunk's tokens routed to e (a popcount over a
+//                           per-expert token bitmap, so no ordering depends on atomics)
+//   gather_rows_kernel      optional materialised x_perm[r] = x[gather_idx[r]]
+// Counts and bitmaps are built with shared-memory atomics whose result does not depend on
+// their order, so every output is bit-reproducible.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int DISPATCH_CHUNK = 256; // tokens per chunk (one thread per token)
+constexpr int DISPATCH_WORDS = DISPATCH_CHUNK / 32;
+constexpr int M_TILE = 128;
+
+// Workspace-resident bookkeeping written by the scan and read by the GEMMs.
+struct DispatchMeta {
+    int num_tiles;  // sum_e ceil(c_e / M_TILE)
+    int padded_rows; // P_pad = num_tiles * M_TILE
+};
+
+__global__ void __launch_bounds__(DISPATCH_CHUNK)
+    dispatch_count_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
+                          int32_t *__restrict__ chunk_counts, int *status, int clear_status)
+{
+    extern __shared__ int cnt[];
+    if (clear_status && status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        status[0] = DEV_OK;
+        status[1] = 0;
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * DISPATCH_CHUNK + threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(size_t)t * k + j];
+            if (e >= 0 && e < E) {
+                atomicAdd(&cnt[e], 1);
+            } else {
+                record_status(status, DEV_BAD_INDEX, 1);
+            }
+            // a token's experts must be distinct (checked for the usual small k)
+            if (k <= 16) {
+                for (int j2 = 0; j2 < j; ++j2)
+                    if (topk_idx[(size_t)t * k + j2] == e) record_status(status, DEV_BAD_INDEX, 2);
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Inclusive block scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_inclusive_scan_1024(int v, int *warp_sums)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    if (lane == 31) warp_sums[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int s = warp_sums[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, s, off);
+            if (lane >= off) s += o;
+        }
+        warp_sums[lane] = s;
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_sums[warp - 1];
+    __syncthreads();
+    return v;
+}
+
+// One block of 1024 threads; thread e owns expert e (E <= 1024).
+//   chunk_counts [nchunk][E] is rewritten in place into each chunk's base row within e.
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk, int E,
+                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                         int32_t *__restrict__ padded_offsets, int32_t *__restrict__ tile_off,
+                         int32_t *__restrict__ tile_expert, DispatchMeta *meta,
+                         int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
+                         int64_t padded_rows_max)
+{
+    __shared__ int warp_sums[32];
+    __shared__ int s_poff[1025];
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < E) {
+        int run = 0;
+        for (int ch = 0; ch < nchunk; ++ch) {
+            const int v = chunk_counts[(size_t)ch * E + e];
+            chunk_counts[(size_t)ch * E + e] = run;
+            run += v;
+        }
+        c = run;
+        if (counts != nullptr) counts[e] = c;
+    }
+    const int ntile = (c + M_TILE - 1) / M_TILE;
+    const int inc_c = block_inclusive_scan_1024(c, warp_sums);
+    const int inc_t = block_inclusive_scan_1024(ntile, warp_sums);
+    if (e < E) {
+        if (offsets != nullptr) {
+            offsets[e + 1] = inc_c;
+            if (e == 0) offsets[0] = 0;
+        }
+        const int poff_next = inc_t * M_TILE;
+        const int tile_first = inc_t - ntile;
+        padded_offsets[e + 1] = poff_next;
+        tile_off[e + 1] = inc_t;
+        if (e == 0) {
+            padded_offsets[0] = 0;
+            tile_off[0] = 0;
+        }
+        s_poff[e] = tile_first * M_TILE;
+        for (int i = 0; i < ntile; ++i) tile_expert[tile_first + i] = e;
+        if (e == E - 1) {
+            meta->num_tiles = inc_t;
+            meta->padded_rows = poff_next;
+            s_poff[E] = poff_next;
+        }
+    }
+    __syncthreads();
+    // pad rows of each expert, then everything past P_pad: gather_idx = -1, weight 0
+    if (e < E) {
+        const int first_pad = s_poff[e] + c;
+        const int end = s_poff[e] + ntile * M_TILE;
+        for (int r = first_pad; r < end; ++r) {
+            gather_idx[r] = -1;
+            if (row_w != nullptr) row_w[r] = 0.0f;
+        }
+    }
+    for (int64_t r = (int64_t)s_poff[E] + threadIdx.x; r < padded_rows_max; r += blockDim.x) {
+        gather_idx[r] = -1;
+        if (row_w != nullptr) row_w[r] = 0.0f;
+    }
+}
+
+// Dynamic shared memory: E * DISPATCH_WORDS uint32 (token bitmap per expert).
+__global__ void __launch_bounds__(DISPATCH_CHUNK)
+    dispatch_place_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
+                          int T, int E, int k, const int32_t *__restrict__ chunk_base,
+                          const int32_t *__restrict__ padded_offsets,
+                          int32_t *__restrict__ gather_idx, int32_t *__restrict__ inv_pos,
+                          float *__restrict__ row_w)
+{
+    extern __shared__ uint32_t bits[];
+    for (int i = threadIdx.x; i < E * DISPATCH_WORDS; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    const int tl = threadIdx.x;
+    const int t = blockIdx.x * DISPATCH_CHUNK + tl;
+    const int word = tl >> 5;
+    const uint32_t bit = 1u << (tl & 31);
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(size_t)t * k + j];
+            if (e >= 0 && e < E) atomicOr(&bits[e * DISPATCH_WORDS + word], bit);
+        }
+    }
+    __syncthreads();
+    if (t >= T) return;
+    for (int j = 0; j < k; ++j) {
+        const int e = topk_idx[(size_t)t * k + j];
+        if (e < 0 || e >= E) {
+            inv_pos[(size_t)t * k + j] = -1;
+            continue;
+        }
+        const uint32_t *b = bits + e * DISPATCH_WORDS;
+        int rank = __popc(b[word] & (bit - 1u));
+        for (int w = 0; w < word; ++w) rank += __popc(b[w]);
+        const int r = padded_offsets[e] + chunk_base[(size_t)blockIdx.x * E + e] + rank;
+        gather_idx[r] = t;
+        inv_pos[(size_t)t * k + j] = r;
+        if (row_w != nullptr) row_w[r] = topk_w[(size_t)t * k + j];
+    }
+}
+
+// x_perm[r][:] = x[gather_idx[r]][:] (zeros on pad rows), for r < P_pad. One warp per row.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const __nv_bfloat16 *__restrict__ x, const int32_t *__restrict__ gather_idx,
+                       const DispatchMeta *meta, int T, int H, __nv_bfloat16 *__restrict__ x_perm)
+{
+    const int rows = meta->padded_rows;
+    const int lane = threadIdx.x & 31;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int chunks = H / 8;
+    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nw) {
+        const int t = gather_idx[r];
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * H);
+        if (t >= 0 && t < T) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+            for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+        } else {
+            for (int c = lane; c < chunks; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+} // namespace moe

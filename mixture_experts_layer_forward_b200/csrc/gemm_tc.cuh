@@ -1,0 +1,344 @@
+// gemm_tc.cuh -- persistent grouped GEMM over all experts on the 5th-generation tensor cores
+// (tcgen05 + TMEM), fed by TMA, with the expert epilogues fused.
+//
+// Where it comes from (Comet: Fine-grained Computation-communication Overlapping for
+// Mixture-of-Experts):
+//   §3.1.1  layer0 (hidden -> FFN) is decomposed along M: its work items are 128-row tiles
+//           of expert-sorted token rows; layer1 (FFN -> hidden) is decomposed along N:
+//           each work item owns a 256-column stripe of the output, so the top-k reduce of
+//           a stripe never depends on another stripe.
+//   §3.1.2  rows are regrouped into whole GEMM tiles (128-row padded expert blocks) and the
+//           GroupGEMM covers every expert in one launch.
+//   §3.2.1  thread-block specialisation: inside each CTA one warp only moves data (TMA),
+//           one warp only issues MMAs, four warps only run the epilogue.
+//   §4      the GEMMs are expert-grouped GEMMs; row metadata is read once per tile, not
+//           per K step.
+//
+// Design on sm_100a
+//   - One CTA per SM (persistent), 192 threads:
+//       warp 0  TMA producer: A tile 128 x 64 (one 2D box) and B tile 64 x 256 (four
+//               3D boxes of 64 x 64 from the expert's weight matrix) per K step;
+//       warp 1  allocates 512 TMEM columns (two 128 x 256 fp32 accumulators) and issues
+//               tcgen05.mma (M=128, N=256, K=16) from one thread;
+//       warps 2-5 epilogue: tcgen05.ld of their 32 TMEM lanes, activation or gate scale,
+//               bf16 stores. The two accumulators let the epilogue of tile i overlap the
+//               mainloop of tile i+1.
+//   - 4-stage shared-memory ring (48 KB per stage), 128-byte swizzle; A is K-major, B is
+//     the weight matrix as stored (N contiguous), read MN-major by the MMA.
+//   - Work items are ordered expert-major, then N tile, then M tile, so the CTAs that run
+//     together share one expert's weight stripe and its token rows in L2.
+//   - Every wait is bounded: on timeout the CTA records DEV_TIMEOUT, all roles stop, the
+//     producer waits (bounded) for its in-flight copies, the MMA warp waits for its
+//     in-flight MMAs, and TMEM is released before exit.
+//
+// Kinds:
+//   GEMM_SWIGLU  A = x_perm [rows, H], B = W1[e] [H, 2F]; the B tile holds gate columns
+//                n*128.. and up columns F + n*128..; out h[r][n*128 + c] =
+//                silu(gate) * up (bf16).
+//   GEMM_ACT     A = x_perm, B = W1[e] [H, F]; out h = act(acc) (bf16), 256 columns/tile.
+//   GEMM_SCALE   A = h [rows, F], B = W2[e] [F, H]; out ys[r][n*256 + c] =
+//                row_w[r] * acc (bf16).
+#pragma once
+
+#include "dispatch.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace gemm {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK * 2;    // 16 KB
+constexpr int B_BOX = 64 * BK * 2;     // 8 KB: 64 columns x 64 K rows
+constexpr int B_TILE = BN * BK * 2;    // 32 KB
+constexpr int STAGE = A_TILE + B_TILE; // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE + NUM_BARS * 8 + 16;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*b_mn_major=*/true);
+// descriptor strides
+constexpr uint32_t A_SBO = 1024; // 8 rows x 128 B
+constexpr uint32_t A_LBO = 16;   // unused for swizzled K-major
+constexpr uint32_t B_SBO = 1024; // 8 K rows x 128 B
+constexpr uint32_t B_LBO = B_BOX; // next 64-column block
+} // namespace gemm
+
+enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2 };
+
+struct GemmArgs {
+    const int32_t *tile_off;    // [E+1] first m-tile of each expert
+    const int32_t *tile_expert; // [max_tiles] expert of each m-tile
+    const DispatchMeta *meta;   // num_tiles
+    const float *row_w;         // GEMM_SCALE: gate weight of each padded row
+    __nv_bfloat16 *out;         // [rows, ld_out]
+    int ld_out;                 // elements per output row
+    int n_cols;                 // valid output columns
+    int n_tiles;                // N tiles per m-tile
+    int k_blocks;               // K / 64
+    int up_col;                 // GEMM_SWIGLU: first up column of W1 (= F)
+    int act;                    // GEMM_ACT: 1 gelu-tanh, 2 relu, 3 identity
+    int *status;
+    int64_t timeout_ns;
+};
+
+__device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt)
+{
+    const int q = w / a.n_tiles;
+    e = a.tile_expert[q];
+    const int base = a.tile_off[e];
+    const int cnt = a.tile_off[e + 1] - base;
+    const int local = w - base * a.n_tiles;
+    mt = base + local % cnt;
+    nt = local / cnt;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+__device__ __forceinline__ float act_f(int act, float z)
+{
+    if (act == 1) {
+        const float c = 0.7978845608028654f; // sqrt(2/pi)
+        return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
+    }
+    if (act == 2) return z > 0.0f ? z : 0.0f;
+    return z;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
+    moe_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+{
+    using namespace gemm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 4);
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_tiles = args.meta->num_tiles;
+    const int total = num_tiles * args.n_tiles;
+    const int KB = args.k_blocks;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            int s = 0;
+            uint32_t ph = 0;
+            int armed[STAGES];
+#pragma unroll
+            for (int i = 0; i < STAGES; ++i) armed[i] = -1;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+                int e, mt, nt;
+                gemm_map_work(w, args, e, mt, nt);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
+                                           args.status, 100 + KIND)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_u32(smem + s * STAGE);
+                    const uint32_t b_dst = a_dst + A_TILE;
+                    mbar_arrive_expect_tx(full_bar(s), STAGE);
+                    armed[s] = (int)ph;
+                    tma_load_2d(a_dst, &tmA, full_bar(s), kb * BK, mt * BM);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        int col;
+                        if (KIND == GEMM_SWIGLU)
+                            col = (i < 2 ? nt * 128 + i * 64 : args.up_col + nt * 128 + (i - 2) * 64);
+                        else
+                            col = nt * BN + i * 64;
+                        tma_load_3d(b_dst + i * B_BOX, &tmB, full_bar(s), col, kb * BK, e);
+                    }
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // every copy issued must have landed before the CTA exits (immediate when the
+            // MMA warp consumed them all; bounded after an abort)
+            for (int i = 0; i < STAGES; ++i)
+                if (armed[i] >= 0) {
+                    volatile int never = 0;
+                    mbar_wait_bounded(full_bar(i), (uint32_t)armed[i], &never, args.timeout_ns,
+                                      nullptr, 0);
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, args.timeout_ns,
+                                       args.status, 110 + KIND)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, args.timeout_ns, args.status,
+                                           120 + KIND)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * STAGE);
+                    const uint32_t b_addr = a_addr + A_TILE;
+                    const uint64_t a_desc = sw128_desc(a_addr, A_LBO, A_SBO);
+                    const uint64_t b_desc = sw128_desc(b_addr, B_LBO, B_SBO);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // A: +32 B per K=16 step inside the swizzle atom; B: +16 rows x 128 B
+                        umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                  b_desc + (uint64_t)((k * 16 * 128) >> 4), IDESC,
+                                  (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty_bar(s));
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(tfull_bar(acc));
+            }
+            // every MMA issued so far must finish before TMEM is released
+            umma_commit(done_bar);
+            volatile int never = 0;
+            mbar_wait_bounded(done_bar, 0, &never, args.timeout_ns, args.status, 130 + KIND);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5 ----------------
+        const int q = warp & 3; // TMEM lanes 32q .. 32q+31
+        int it = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+            int e, mt, nt;
+            gemm_map_work(w, args, e, mt, nt);
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            bool ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, args.timeout_ns,
+                                        args.status, 140 + KIND);
+            // the TMEM loads below are warp-collective: the whole warp continues or stops
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int row = mt * BM + q * 32 + lane;
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            if (KIND == GEMM_SWIGLU) {
+                __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * 128;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, g);
+                    tmem_ld_32x32b_x32(t_row + 128 + c * 32, u);
+                    tmem_ld_wait();
+                    if (nt * 128 + c * 32 < args.n_cols) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int h2 = 0; h2 < 4; ++h2) {
+                                const int i = v * 8 + h2 * 2;
+                                const float a0 = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+                                const float a1 =
+                                    silu_f(__uint_as_float(g[i + 1])) * __uint_as_float(u[i + 1]);
+                                p[h2] = pack_bf16x2(a0, a1);
+                            }
+                            dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                }
+            } else {
+                __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * BN;
+                const float wt = (KIND == GEMM_SCALE) ? args.row_w[row] : 1.0f;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    tmem_ld_wait();
+                    if (nt * BN + c * 32 < args.n_cols) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int h2 = 0; h2 < 4; ++h2) {
+                                const int i = v * 8 + h2 * 2;
+                                float a0 = __uint_as_float(r[i]);
+                                float a1 = __uint_as_float(r[i + 1]);
+                                if (KIND == GEMM_SCALE) {
+                                    a0 *= wt;
+                                    a1 *= wt;
+                                } else {
+                                    a0 = act_f(args.act, a0);
+                                    a1 = act_f(args.act, a1);
+                                }
+                                p[h2] = pack_bf16x2(a0, a1);
+                            }
+                            dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+} // namespace moe

@@ -1,0 +1,557 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checks, workspace carving,
+// tensor-map encoding and kernel launches. Every step of the layer runs in the kernels
+// included below; this file only validates and launches.
+#include "moe.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "combine.cuh"
+#include "dispatch.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+#include "route.cuh"
+
+namespace {
+
+using namespace moe;
+
+constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
+std::atomic<int64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+// ---------------------------------------------------------------------------------------
+// problem checks and workspace layout
+// ---------------------------------------------------------------------------------------
+
+moe_status check_problem(const moe_problem *p)
+{
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    if (p->T < 0 || p->H <= 0 || p->F <= 0 || p->E <= 0 || p->top_k <= 0) return MOE_ERR_INVALID_ARG;
+    if (p->top_k > p->E) return MOE_ERR_INVALID_ARG;
+    if (p->act < MOE_ACT_SWIGLU || p->act > MOE_ACT_IDENTITY) return MOE_ERR_INVALID_ARG;
+    if (p->gate != MOE_GATE_SOFTMAX_TOPK && p->gate != MOE_GATE_SOFTMAX_ALL) return MOE_ERR_INVALID_ARG;
+    if (p->m_tile != M_TILE) return MOE_ERR_UNSUPPORTED;
+    if (p->H % 64 != 0 || p->F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (p->E > 1024) return MOE_ERR_UNSUPPORTED;
+    // 32-bit row indices and element offsets inside one expert block
+    const int64_t pmax = (int64_t)p->T * p->top_k + (int64_t)p->E * (M_TILE - 1);
+    if (pmax >= (1LL << 31) - M_TILE) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int64_t padded_rows_max(const moe_problem *p)
+{
+    const int64_t tk = (int64_t)p->T * p->top_k;
+    const int64_t nonempty = tk < p->E ? tk : p->E;
+    return tk + nonempty * (M_TILE - 1);
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct Layout {
+    size_t status, meta, logits, topk_idx, topk_w, chunk, counts, offsets, poff, tile_off,
+        tile_expert, gather_idx, inv_pos, row_w, x_perm, h, ys, x_stage, out_stage;
+    size_t end_route, end_dispatch, end_forward, end_host;
+    int64_t pmax;
+    int nchunk, max_tiles;
+};
+
+Layout make_layout(const moe_problem *p)
+{
+    Layout L{};
+    const size_t T = (size_t)p->T, H = (size_t)p->H, F = (size_t)p->F, E = (size_t)p->E,
+                 K = (size_t)p->top_k;
+    L.pmax = padded_rows_max(p);
+    const size_t P = (size_t)L.pmax;
+    L.nchunk = (int)((T + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK);
+    L.max_tiles = (int)(P / M_TILE) + 1;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align256(o + (bytes ? bytes : 1));
+        return at;
+    };
+    L.status = take(256);
+    L.meta = take(sizeof(DispatchMeta));
+    L.logits = take(T * E * 4);
+    L.end_route = o;
+    L.topk_idx = take(T * K * 4);
+    L.topk_w = take(T * K * 4);
+    L.chunk = take((size_t)L.nchunk * E * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.poff = take((E + 1) * 4);
+    L.tile_off = take((E + 1) * 4);
+    L.tile_expert = take((size_t)L.max_tiles * 4);
+    L.gather_idx = take(P * 4);
+    L.inv_pos = take(T * K * 4);
+    L.row_w = take(P * 4);
+    L.end_dispatch = o;
+    L.x_perm = take(P * H * 2);
+    L.h = take(P * F * 2);
+    L.ys = take(P * H * 2);
+    L.end_forward = o;
+    L.x_stage = take(T * H * 2);
+    L.out_stage = take(T * H * 2);
+    L.end_host = o;
+    return L;
+}
+
+template <typename T> T *at(void *ws, size_t off)
+{
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool aligned4(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+// ---------------------------------------------------------------------------------------
+// device properties and tensor maps
+// ---------------------------------------------------------------------------------------
+
+int sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2D bf16 row-major [rows, cols]; box = 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 [depth, rows, cols]; box = 64 columns x 64 rows x 1, 128-byte swizzle.
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {cols, rows, depth};
+    cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND> cudaError_t gemm_smem_attr()
+{
+    // set once per process and device; cheap to repeat
+    return cudaFuncSetAttribute(moe_grouped_gemm_kernel<KIND>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+}
+
+// ---------------------------------------------------------------------------------------
+// stage launchers (no argument checks; callers validated)
+// ---------------------------------------------------------------------------------------
+
+cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                         const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+                         int *status, cudaStream_t st)
+{
+    const int T = p->T, H = p->H, E = p->E;
+    const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
+    const auto *wb = reinterpret_cast<const __nv_bfloat16 *>(Wg);
+    if (E <= 8) {
+        dim3 grid((T + 31) / 32, 1), block(8, 32);
+        route_logits_kernel<32, 8, 1, 1><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
+    } else if (E <= 16) {
+        dim3 grid((T + 15) / 16, 1), block(16, 16);
+        route_logits_kernel<16, 16, 1, 1><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
+    } else {
+        dim3 grid((T + 63) / 64, (E + 63) / 64), block(16, 16);
+        route_logits_kernel<64, 64, 4, 4><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
+    }
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const size_t smem = (size_t)TOPK_WARPS * E * sizeof(float);
+    route_topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(
+        logits, topk_idx, topk_w, T, E, p->top_k, p->gate);
+    return cudaGetLastError();
+}
+
+struct DispatchOut {
+    int32_t *counts, *offsets, *poff, *gather_idx, *inv_pos, *tile_off, *tile_expert, *chunk;
+    float *row_w;
+    DispatchMeta *meta;
+};
+
+cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t *topk_idx,
+                            const float *topk_w, const DispatchOut &o, int *status, int clear_status,
+                            cudaStream_t st)
+{
+    const int T = p->T, E = p->E, k = p->top_k;
+    const int nchunk = L.nchunk;
+    if (nchunk > 0) {
+        dispatch_count_kernel<<<nchunk, DISPATCH_CHUNK, E * sizeof(int), st>>>(
+            topk_idx, T, E, k, o.chunk, status, clear_status);
+    }
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, o.counts, o.offsets, o.poff,
+                                             o.tile_off, o.tile_expert, o.meta, o.gather_idx,
+                                             o.row_w, L.pmax);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    if (nchunk > 0) {
+        dispatch_place_kernel<<<nchunk, DISPATCH_CHUNK, (size_t)E * DISPATCH_WORDS * 4, st>>>(
+            topk_idx, topk_w, T, E, k, o.chunk, o.poff, o.gather_idx, o.inv_pos, o.row_w);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const moe_problem *p, const moe_bf16 *x, const int32_t *gather_idx,
+                          const DispatchMeta *meta, moe_bf16 *x_perm, cudaStream_t st)
+{
+    const int blocks = sm_count() * 8;
+    gather_rows_kernel<<<blocks > 0 ? blocks : 1024, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(x), gather_idx, meta, p->T, p->H,
+        reinterpret_cast<__nv_bfloat16 *>(x_perm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_rows,
+                           const int32_t *inv_pos, moe_bf16 *out, int *status, int clear_status,
+                           cudaStream_t st)
+{
+    const int64_t vecs = (int64_t)p->T * (p->H / 8);
+    int64_t blocks = (vecs + 255) / 256;
+    const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    combine_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows,
+                                               inv_pos, p->T, p->H, p->top_k,
+                                               reinterpret_cast<__nv_bfloat16 *>(out), status,
+                                               clear_status);
+    return cudaGetLastError();
+}
+
+template <int KIND>
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                        int max_work, cudaStream_t st)
+{
+    cudaError_t err = gemm_smem_attr<KIND>();
+    if (err != cudaSuccess) return err;
+    int grid = sm_count();
+    if (grid <= 0) grid = 148;
+    if (grid > max_work) grid = max_work;
+    if (grid < 1) grid = 1;
+    moe_grouped_gemm_kernel<KIND><<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+    return cudaGetLastError();
+}
+
+moe_status to_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaError_t record(void *const *events, int n, int i, cudaStream_t st)
+{
+    if (n == 0) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+}
+
+moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                        const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
+                        int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                        cudaStream_t st, void *const *events, int n_events)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (n_events != 0 && (n_events != MOE_NUM_STAGE_EVENTS || events == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (ws == nullptr || (p->T > 0 && (x == nullptr || out == nullptr)) || Wg == nullptr ||
+        W1 == nullptr || W2 == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_forward) return MOE_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(W1) || !aligned16(W2) || !aligned16(Wg) ||
+        !aligned16(ws) || !aligned4(bias) || !aligned4(topk_idx_out) || !aligned4(topk_w_out))
+        return MOE_ERR_INVALID_ARG;
+
+    int *status = at<int>(ws, L.status);
+    if (p->T == 0) {
+        // nothing to compute; still clear the status word and mark the stage boundaries
+        cudaError_t e = cudaMemsetAsync(status, 0, 8, st);
+        for (int i = 0; i < n_events && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+        return to_status(e);
+    }
+    int32_t *topk_idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+    float *topk_w = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
+    DispatchOut d;
+    d.counts = at<int32_t>(ws, L.counts);
+    d.offsets = at<int32_t>(ws, L.offsets);
+    d.poff = at<int32_t>(ws, L.poff);
+    d.gather_idx = at<int32_t>(ws, L.gather_idx);
+    d.inv_pos = at<int32_t>(ws, L.inv_pos);
+    d.tile_off = at<int32_t>(ws, L.tile_off);
+    d.tile_expert = at<int32_t>(ws, L.tile_expert);
+    d.chunk = at<int32_t>(ws, L.chunk);
+    d.row_w = at<float>(ws, L.row_w);
+    d.meta = at<DispatchMeta>(ws, L.meta);
+    moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
+    moe_bf16 *h = at<moe_bf16>(ws, L.h);
+    moe_bf16 *ys = at<moe_bf16>(ws, L.ys);
+
+    const int F = p->F, H = p->H, E = p->E;
+    const bool gated = (p->act == MOE_ACT_SWIGLU);
+    CUtensorMap m_x, m_w1, m_h, m_w2;
+    if (!make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM) ||
+        !make_map_3d(&m_w1, W1, (uint64_t)E, (uint64_t)H, (uint64_t)(gated ? 2 * F : F)) ||
+        !make_map_2d(&m_h, h, (uint64_t)L.pmax, (uint64_t)F, gemm::BM) ||
+        !make_map_3d(&m_w2, W2, (uint64_t)E, (uint64_t)F, (uint64_t)H))
+        return MOE_ERR_CUDA;
+
+    const int64_t timeout = g_timeout_ns.load();
+    cudaError_t e = record(events, n_events, 0, st);
+    if (e == cudaSuccess)
+        e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st);
+    if (e == cudaSuccess) e = record(events, n_events, 1, st);
+    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
+    if (e == cudaSuccess) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
+    if (e == cudaSuccess) e = record(events, n_events, 2, st);
+
+    GemmArgs a0{};
+    a0.tile_off = d.tile_off;
+    a0.tile_expert = d.tile_expert;
+    a0.meta = d.meta;
+    a0.row_w = nullptr;
+    a0.out = reinterpret_cast<__nv_bfloat16 *>(h);
+    a0.ld_out = F;
+    a0.n_cols = F;
+    a0.k_blocks = H / gemm::BK;
+    a0.up_col = F;
+    a0.act = p->act;
+    a0.status = status;
+    a0.timeout_ns = timeout;
+    if (gated) {
+        a0.n_tiles = (F + 127) / 128;
+        if (e == cudaSuccess)
+            e = launch_gemm<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+    } else {
+        a0.n_tiles = (F + gemm::BN - 1) / gemm::BN;
+        if (e == cudaSuccess) e = launch_gemm<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+    }
+    if (e == cudaSuccess) e = record(events, n_events, 3, st);
+
+    GemmArgs a1 = a0;
+    a1.row_w = d.row_w;
+    a1.out = reinterpret_cast<__nv_bfloat16 *>(ys);
+    a1.ld_out = H;
+    a1.n_cols = H;
+    a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+    a1.k_blocks = F / gemm::BK;
+    if (e == cudaSuccess) e = launch_gemm<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
+    if (e == cudaSuccess) e = record(events, n_events, 4, st);
+    if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st);
+    if (e == cudaSuccess) e = record(events, n_events, 5, st);
+    return to_status(e);
+}
+
+} // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_problem *p)
+{
+    if (check_problem(p) != MOE_OK) return 0;
+    return make_layout(p).end_host;
+}
+
+int64_t moe_padded_rows_max(const moe_problem *p)
+{
+    if (check_problem(p) != MOE_OK) return -1;
+    return padded_rows_max(p);
+}
+
+moe_status moe_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg, const float *bias,
+                     int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (ws == nullptr || Wg == nullptr) return MOE_ERR_INVALID_ARG;
+    if (p->T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_route) return MOE_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(ws) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(topk_w))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int *status = at<int>(ws, L.status);
+    if (p->T == 0) return to_status(cudaMemsetAsync(status, 0, 8, st));
+    return to_status(launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st));
+}
+
+moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *counts,
+                        int32_t *offsets, int32_t *padded_offsets, int32_t *gather_idx,
+                        int32_t *inv_pos, moe_bf16 *x_perm, const moe_bf16 *x, void *ws,
+                        size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (ws == nullptr || counts == nullptr || offsets == nullptr || padded_offsets == nullptr ||
+        gather_idx == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (p->T > 0 && (topk_idx == nullptr || inv_pos == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x_perm != nullptr && x == nullptr) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_dispatch) return MOE_ERR_WORKSPACE;
+    if (!aligned16(ws) || !aligned16(x_perm) || !aligned16(x) || !aligned4(topk_idx) ||
+        !aligned4(counts) || !aligned4(offsets) || !aligned4(padded_offsets) ||
+        !aligned4(gather_idx) || !aligned4(inv_pos))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int *status = at<int>(ws, L.status);
+    cudaError_t e = cudaSuccess;
+    if (p->T == 0) e = cudaMemsetAsync(status, 0, 8, st);
+    DispatchOut d;
+    d.counts = counts;
+    d.offsets = offsets;
+    d.poff = padded_offsets;
+    d.gather_idx = gather_idx;
+    d.inv_pos = inv_pos;
+    d.tile_off = at<int32_t>(ws, L.tile_off);
+    d.tile_expert = at<int32_t>(ws, L.tile_expert);
+    d.chunk = at<int32_t>(ws, L.chunk);
+    d.row_w = nullptr;
+    d.meta = at<DispatchMeta>(ws, L.meta);
+    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, nullptr, d, status, 1, st);
+    if (e == cudaSuccess && x_perm != nullptr)
+        e = launch_gather(p, x, gather_idx, d.meta, x_perm, st);
+    return to_status(e);
+}
+
+moe_status moe_forward(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg, const float *bias,
+                       const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out, int32_t *topk_idx_out,
+                       float *topk_w_out, void *ws, size_t ws_bytes, void *stream)
+{
+    return forward_impl(p, x, Wg, bias, W1, W2, out, topk_idx_out, topk_w_out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), nullptr, 0);
+}
+
+moe_status moe_forward_staged(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                              const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                              moe_bf16 *out, int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                              size_t ws_bytes, void *stream, void *const *events, int n_events)
+{
+    return forward_impl(p, x, Wg, bias, W1, W2, out, topk_idx_out, topk_w_out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), events, n_events);
+}
+
+moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const moe_bf16 *Wg,
+                            const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                            moe_bf16 *out_host, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (ws == nullptr || (p->T > 0 && (x_host == nullptr || out_host == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_host) return MOE_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)p->T * p->H * 2;
+    moe_bf16 *xd = at<moe_bf16>(ws, L.x_stage);
+    moe_bf16 *od = at<moe_bf16>(ws, L.out_stage);
+    if (bytes > 0 && cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    s = forward_impl(p, xd, Wg, bias, W1, W2, od, nullptr, nullptr, ws, ws_bytes, st, nullptr, 0);
+    if (s != MOE_OK) return s;
+    if (bytes > 0 && cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return to_status(cudaStreamSynchronize(st));
+}
+
+moe_status moe_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_rows,
+                       const int32_t *inv_pos, moe_bf16 *out, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (p->T > 0 && (ys == nullptr || inv_pos == nullptr || out == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (ys_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ys) || !aligned16(out) || !aligned4(inv_pos) || !aligned16(ws))
+        return MOE_ERR_INVALID_ARG;
+    int *status = nullptr;
+    if (ws != nullptr) {
+        if (ws_bytes < 256) return MOE_ERR_WORKSPACE;
+        status = at<int>(ws, 0);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p->T == 0) return status ? to_status(cudaMemsetAsync(status, 0, 8, st)) : MOE_OK;
+    return to_status(launch_combine(p, ys, ys_rows, inv_pos, out, status, 1, st));
+}
+
+moe_status moe_get_device_status(void *ws, void *stream)
+{
+    if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    int host[2] = {0, 0};
+    if (cudaMemcpy(host, ws, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero[2] = {0, 0};
+    if (cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    switch (host[0]) {
+    case DEV_OK: return MOE_OK;
+    case DEV_TIMEOUT: return MOE_ERR_DEVICE_TIMEOUT;
+    case DEV_BAD_INDEX: return MOE_ERR_DEVICE_BAD_INDEX;
+    default: return MOE_ERR_CUDA;
+    }
+}
+
+const char *moe_status_string(moe_status s)
+{
+    switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_DEVICE_BAD_INDEX: return "MOE_ERR_DEVICE_BAD_INDEX";
+    }
+    return "MOE_UNKNOWN_STATUS";
+}
+
+int64_t moe_set_wait_timeout_ns(int64_t ns)
+{
+    return g_timeout_ns.exchange(ns > 0 ? ns : kDefaultTimeoutNs);
+}
+
+} // extern "C"

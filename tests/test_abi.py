@@ -1,0 +1,91 @@
+"""CPU checks of the C ABI library: it builds, loads, exports every function that
+include/moe.h declares, and rejects bad arguments on the host (no kernel is launched and
+no CUDA call is made on these paths)."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import mixture_experts_layer_forward_b200 as moe
+from mixture_experts_layer_forward_b200 import build as native_build
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    native_build.build_library()
+    return moe.library()
+
+
+def declared_functions():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = h.read_text()
+        names += re.findall(r"^MOE_API\s+[^;(]*?\b(moe_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for n in ("moe_route", "moe_dispatch", "moe_forward", "moe_combine", "moe_workspace_size",
+              "moe_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", str(moe.library_path())],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    moe_syms = {s for s in exported if s.startswith("moe_")}
+    assert moe_syms == set(declared_functions())
+
+
+def test_host_side_argument_checks(lib):
+    P = moe.Problem
+    good = P.make(256, 256, 512, 8, 2)
+    assert moe.moe_workspace_size(good) > 0
+    assert moe.moe_padded_rows_max(good) == 256 * 2 + 8 * 127
+    assert moe.moe_padded_rows_max(P.make(1, 256, 512, 8, 1)) == 1 + 1 * 127
+    bad = [P.make(256, 256, 512, 8, 9),          # k > E
+           P.make(-1, 256, 512, 8, 2),           # T < 0
+           P.make(256, 0, 512, 8, 2),            # H = 0
+           P.make(256, 256, 512, 8, 2, act=7),   # unknown activation
+           P.make(256, 256, 512, 8, 2, gate=5)]  # unknown gate
+    for p in bad:
+        assert moe.moe_workspace_size(p) == 0
+        assert lib.moe_forward(ctypes.byref(p), *([None] * 9), 0, None) == -1
+    unsupported = [P.make(256, 100, 512, 8, 2),   # H % 64
+                   P.make(256, 256, 96, 8, 2),    # F % 64
+                   P.make(256, 256, 512, 2048, 2),  # E > 1024
+                   P.make(256, 256, 512, 8, 2, m_tile=64)]
+    for p in unsupported:
+        assert moe.moe_workspace_size(p) == 0
+        assert lib.moe_forward(ctypes.byref(p), *([None] * 9), 0, None) == -2
+    # NULL pointers / short workspace are rejected before any CUDA call
+    assert lib.moe_forward(ctypes.byref(good), *([None] * 9), 0, None) == -1
+    fake = ctypes.c_void_p(1 << 20)
+    args = [fake] * 6 + [None, None]
+    assert lib.moe_forward(ctypes.byref(good), *args, fake, 16, None) == -3
+    assert lib.moe_route(ctypes.byref(good), fake, fake, None, fake, fake, fake, 16, None) == -3
+    assert lib.moe_get_device_status(None, None) == -1
+    assert lib.moe_status_string(-5) == b"MOE_ERR_DEVICE_TIMEOUT"
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    from mixture_experts_layer_forward_b200 import _native
+
+    monkeypatch.setattr(_native, "LIB_PATH", tmp_path / "absent.so")
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _native.library()

@@ -1,0 +1,320 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar (fixed for every case here):
+  - routing indices, expert counts, offsets, padded offsets, gather_idx and inv_pos:
+    bit-exact;
+  - gate weights: |w_gpu - w_ref| <= 1e-5 * w_ref + 1e-7 (fp32 expf vs fp64 exp);
+  - layer output (bf16) against the fp64 oracle: |out - ref| <= 2e-2 + 2e-2 * |ref|
+    element-wise;
+  - combine on given bf16 rows: |out - ref| <= 2^-8 * |ref| + 1e-6 (one bf16 rounding of
+    an fp32 sum);
+  - two identical calls give bit-identical outputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_forward_b200 as moe
+import oracle
+from mixture_experts_layer_forward_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-2, 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    moe.library()
+
+
+def bits(t):
+    return synth.bf16_bits(t)
+
+
+def alloc_ws(p):
+    n = moe.moe_workspace_size(p)
+    assert n > 0
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def cfg_small(name, T, H, F, E, k, **kw):
+    return synth.LayerConfig(name, T=T, H=H, F=F, E=E, k=k, **kw)
+
+
+def run_forward(cfg, inp, ws=None):
+    p = moe.Problem.from_config(cfg)
+    ws = alloc_ws(p) if ws is None else ws
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    moe.moe_forward(p, d["x"], d["Wg"], d["bias"], d["W1"], d["W2"], out, ws, idx, w)
+    assert moe.moe_get_device_status(ws) == 0
+    return out, idx, w, ws
+
+
+def assert_out_close(got_bf16, ref, what=""):
+    got = got_bf16.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    bound = ATOL + RTOL * np.abs(ref)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} elements out of tolerance; max |err| "
+                           f"{err.max():.3e}")
+    return float(err.max())
+
+
+# ---------------------------------------------------------------------------------------
+# router
+# ---------------------------------------------------------------------------------------
+
+ROUTE_CASES = [
+    # name, T, H, E, k, unscaled gate, zipf bias, gate mode
+    ("e8", 300, 256, 8, 2, False, 0.0, 0),
+    ("e16_unscaled", 257, 512, 16, 2, True, 0.0, 0),
+    ("e64_k8", 130, 384, 64, 8, False, 0.0, 0),
+    ("e256_zipf", 70, 448, 256, 8, False, 1.2, 0),
+    ("e8_all", 99, 128, 8, 3, False, 0.0, 1),
+    ("e40_k40", 33, 64, 40, 40, False, 0.0, 0),
+    ("e1024_k33", 9, 64, 1024, 33, False, 0.0, 1),
+]
+
+
+@pytest.mark.parametrize("case", ROUTE_CASES, ids=[c[0] for c in ROUTE_CASES])
+def test_route_bit_exact(case):
+    name, T, H, E, k, unscaled, zipf, gate = case
+    cfg = cfg_small(name, T, H, 64, E, k, gate=gate, gate_std_unscaled=unscaled, zipf_s=zipf)
+    inp = synth.make_inputs(cfg, seed=3)
+    p = moe.Problem.from_config(cfg)
+    ws = alloc_ws(p)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    bias = inp["bias"].cuda() if inp["bias"] is not None else None
+    moe.moe_route(p, inp["x"].cuda(), inp["Wg"].cuda(), bias, idx, w, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    logits = oracle.router_logits(bits(inp["x"]), bits(inp["Wg"]),
+                                  None if bias is None else inp["bias"].numpy())
+    ref_idx, ref_w = oracle.topk_gates(logits, k, gate=gate)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+
+
+def test_route_exact_ties_go_to_lower_id():
+    T, H, E, k = 64, 128, 8, 2
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    base = (torch.randn(H, 4, generator=g) / math.sqrt(H)).to(torch.bfloat16)
+    Wg = base[:, [0, 1, 2, 3, 3, 2, 1, 0]].contiguous()
+    p = moe.Problem.make(T, H, 64, E, k)
+    ws = alloc_ws(p)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.moe_route(p, x.cuda(), Wg.cuda(), None, idx, w, ws)
+    got = idx.cpu().numpy()
+    mirror = {0: 7, 1: 6, 2: 5, 3: 4}
+    for t in range(T):
+        assert got[t, 0] < 4 and got[t, 1] == mirror[got[t, 0]]
+    assert torch.all(w == 0.5)
+
+
+# ---------------------------------------------------------------------------------------
+# dispatch
+# ---------------------------------------------------------------------------------------
+
+def distinct_idx(T, E, k, seed, skew=False):
+    rng = np.random.default_rng(seed)
+    if skew:
+        p = np.arange(1, E + 1, dtype=np.float64) ** -1.2
+        p /= p.sum()
+        return np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    return np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+
+
+DISPATCH_CASES = [(300, 8, 2, False), (1000, 64, 8, False), (513, 256, 8, True), (1, 4, 1, False),
+                  (128, 1, 1, False), (40, 8, 8, False), (2048, 1024, 4, True), (77, 3, 3, False)]
+
+
+@pytest.mark.parametrize("T,E,k,skew", DISPATCH_CASES)
+def test_dispatch_bit_exact(T, E, k, skew):
+    H = 64
+    p = moe.Problem.make(T, H, 64, E, k)
+    ws = alloc_ws(p)
+    idx_np = distinct_idx(T, E, k, seed=T * 7 + E, skew=skew)
+    ref = oracle.dispatch(idx_np, E)
+    pmax = moe.moe_padded_rows_max(p)
+    assert pmax == ref["gather_idx"].shape[0] - E * 127 + min(E, T * k) * 127
+    dev = dict(counts=torch.full((E,), -7, dtype=torch.int32, device="cuda"),
+               offsets=torch.full((E + 1,), -7, dtype=torch.int32, device="cuda"),
+               padded_offsets=torch.full((E + 1,), -7, dtype=torch.int32, device="cuda"),
+               gather_idx=torch.full((pmax,), -7, dtype=torch.int32, device="cuda"),
+               inv_pos=torch.full((T, k), -7, dtype=torch.int32, device="cuda"))
+    x = torch.randn(T, H).to(torch.bfloat16)
+    x_perm = torch.full((pmax, H), 3.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_dispatch(p, torch.from_numpy(idx_np).cuda(), dev["counts"], dev["offsets"],
+                     dev["padded_offsets"], dev["gather_idx"], dev["inv_pos"], ws,
+                     x_perm=x_perm, x=x.cuda())
+    assert moe.moe_get_device_status(ws) == 0
+    for key in ("counts", "offsets", "padded_offsets", "inv_pos"):
+        assert np.array_equal(dev[key].cpu().numpy(), ref[key]), key
+    gi = dev["gather_idx"].cpu().numpy()
+    assert np.array_equal(gi, ref["gather_idx"][:pmax])
+    P_pad = int(ref["padded_offsets"][-1])
+    xp = x_perm[:P_pad].cpu()
+    want = torch.zeros(P_pad, H, dtype=torch.bfloat16)
+    valid = torch.from_numpy(gi[:P_pad] >= 0)
+    want[valid] = x[torch.from_numpy(gi[:P_pad][gi[:P_pad] >= 0]).long()]
+    assert torch.equal(xp, want)
+
+
+def test_dispatch_reports_bad_expert_id():
+    T, E, k = 50, 8, 2
+    p = moe.Problem.make(T, 64, 64, E, k)
+    ws = alloc_ws(p)
+    idx = torch.from_numpy(distinct_idx(T, E, k, 1)).cuda()
+    idx[7, 1] = E + 3
+    pmax = moe.moe_padded_rows_max(p)
+    bufs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, E + 1, pmax)]
+    inv = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    moe.moe_dispatch(p, idx, *bufs, inv, ws)
+    assert moe.moe_get_device_status(ws) == -6
+    assert moe.moe_get_device_status(ws) == 0     # read-and-clear
+
+
+# ---------------------------------------------------------------------------------------
+# combine
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,H,E,k", [(300, 256, 8, 2), (65, 448, 64, 8), (1, 64, 4, 4)])
+def test_combine_matches_oracle(T, H, E, k):
+    idx = distinct_idx(T, E, k, seed=T + H)
+    d = oracle.dispatch(idx, E)
+    rows = d["gather_idx"].shape[0]
+    ys = (torch.randn(rows, H, generator=torch.Generator().manual_seed(2)) * 0.3).to(torch.bfloat16)
+    p = moe.Problem.make(T, H, 64, E, k)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(p, ys.cuda(), torch.from_numpy(d["inv_pos"]).cuda(), out)
+    torch.cuda.synchronize()
+    ref = oracle.combine(bits(ys), d["inv_pos"])
+    got = out.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 2.0**-8 * np.abs(ref) + 1e-6)
+
+
+def test_combine_reports_bad_row():
+    T, H, k = 10, 64, 2
+    p = moe.Problem.make(T, H, 64, 4, k)
+    ws = alloc_ws(p)
+    ys = torch.ones(20, H, dtype=torch.bfloat16, device="cuda")
+    inv = torch.zeros(T, k, dtype=torch.int32, device="cuda")
+    inv[3, 1] = 20
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(p, ys, inv, out, ws=ws)
+    assert moe.moe_get_device_status(ws) == -6
+    assert torch.all(out[3] == 1.0) and torch.all(out[0] == 2.0)
+
+
+# ---------------------------------------------------------------------------------------
+# whole layer, small sizes: several tiles, ragged tails, degenerate cases
+# ---------------------------------------------------------------------------------------
+
+FWD_CASES = [
+    cfg_small("tiny", 256, 256, 512, 8, 2),
+    cfg_small("ragged", 300, 192, 320, 8, 2),              # F % 128 == 64, odd T
+    cfg_small("many_experts", 200, 256, 256, 64, 8),        # mostly 1-tile experts
+    cfg_small("zipf", 160, 320, 192, 32, 4, zipf_s=1.2),    # empty and 0-1 token experts
+    cfg_small("one_token", 1, 128, 128, 8, 2),
+    cfg_small("k_eq_e", 40, 128, 128, 4, 4),
+    cfg_small("single_expert", 130, 128, 256, 1, 1),        # dense FFN
+    cfg_small("softmax_all", 100, 128, 128, 8, 2, gate=1),
+    cfg_small("gelu", 150, 128, 256, 8, 2, act=1),
+    cfg_small("relu", 150, 128, 320, 8, 2, act=2),
+    cfg_small("identity", 90, 128, 192, 8, 2, act=3),
+    cfg_small("deep_k", 64, 1024, 128, 8, 2),               # long K loop, ring wraps many times
+]
+
+
+@pytest.mark.parametrize("cfg", FWD_CASES, ids=[c.name for c in FWD_CASES])
+def test_forward_matches_oracle(cfg):
+    inp = synth.make_inputs(cfg, seed=11)
+    out, idx, w, ws = run_forward(cfg, inp)
+    b = None if inp["bias"] is None else inp["bias"].numpy()
+    ref, ref_idx, ref_w = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                             bits(inp["W2"]), cfg.k, act=cfg.act, gate=cfg.gate)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+    assert_out_close(out, ref, cfg.name)
+    out2, _, _, _ = run_forward(cfg, inp, ws)
+    assert torch.equal(out, out2), "two identical calls differ"
+
+
+def test_forward_all_tokens_on_one_expert():
+    cfg = cfg_small("one_hot", 300, 128, 128, 8, 1)
+    inp = synth.make_inputs(cfg, seed=12)
+    inp["bias"] = torch.tensor([0, 0, 0, 100.0, 0, 0, 0, 0], dtype=torch.float32)
+    out, idx, _, _ = run_forward(cfg, inp)
+    assert torch.all(idx == 3)
+    ref, _, _ = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), inp["bias"].numpy(),
+                                   bits(inp["W1"]), bits(inp["W2"]), 1)
+    assert_out_close(out, ref, "one_hot")
+
+
+def test_forward_empty_batch():
+    cfg = cfg_small("empty", 0, 128, 128, 8, 2)
+    p = moe.Problem.from_config(cfg)
+    ws = alloc_ws(p)
+    inp = synth.make_inputs(cfg_small("w", 1, 128, 128, 8, 2), seed=1)
+    out = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
+    x = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(p, x, inp["Wg"].cuda(), None, inp["W1"].cuda(), inp["W2"].cuda(), out, ws)
+    assert moe.moe_get_device_status(ws) == 0
+
+
+def test_forward_host_buffers():
+    cfg = cfg_small("host", 200, 256, 256, 8, 2)
+    inp = synth.make_inputs(cfg, seed=13)
+    p = moe.Problem.from_config(cfg)
+    ws = alloc_ws(p)
+    x_h = inp["x"].pin_memory()
+    out_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    moe.moe_forward_host(p, x_h, inp["Wg"].cuda(), None, inp["W1"].cuda(), inp["W2"].cuda(), out_h, ws)
+    out_d, _, _, _ = run_forward(cfg, inp)
+    assert torch.equal(out_h, out_d.cpu())
+
+
+# ---------------------------------------------------------------------------------------
+# full-size workloads (the bench configurations), launched exactly as the bench does
+# ---------------------------------------------------------------------------------------
+
+FULL = ["mixtral", "phi35", "qwen2", "skew", "skew_decode"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_config(name):
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    out, idx, w, ws = run_forward(cfg, inp)
+    host = {k: (bits(v) if v is not None and v.dtype == torch.bfloat16 else v) for k, v in inp.items()}
+    b = None if inp["bias"] is None else inp["bias"].cpu().numpy()
+    # routing in full, bit-exact
+    logits = oracle.router_logits(host["x"], host["Wg"], b)
+    ref_idx, ref_w = oracle.topk_gates(logits, cfg.k, gate=cfg.gate)
+    gidx = idx.cpu().numpy()
+    assert np.array_equal(gidx, ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+    # output on a token sample: 8 tokens of the least-loaded active experts + seeded random
+    counts = np.bincount(ref_idx.reshape(-1), minlength=cfg.E)
+    active = np.nonzero(counts)[0]
+    rare = active[np.argsort(counts[active], kind="stable")][:4]
+    toks = []
+    for e in rare:
+        toks += list(np.nonzero((ref_idx == e).any(axis=1))[0][:2])
+    rng = np.random.default_rng(0)
+    toks += list(rng.choice(cfg.T, size=min(cfg.T, 8), replace=False))
+    toks = np.unique(np.array(toks, dtype=np.int32))
+    ref, _, _ = oracle.moe_tokens(host["x"], host["Wg"], b, host["W1"], host["W2"], cfg.k, toks,
+                                  act=cfg.act, gate=cfg.gate)
+    assert_out_close(out[torch.from_numpy(toks).long().cuda()], ref, name)
