@@ -1,0 +1,431 @@
+#!/usr/bin/env python3
+"""Benchmark of the MoE layer forward on B200: tokens/s, TFLOP/s and roofline fractions.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+
+A step is one full layer forward (route -> dispatch -> layer0 grouped GEMM + SwiGLU ->
+layer1 grouped GEMM + gate scale -> top-k combine) through the C ABI on one batch of
+synthetic, seeded inputs already resident in HBM. With N > 1 (torchrun, one rank per GPU)
+every rank runs its own batch of the same workload with the same weights (data-parallel
+replicas, weak scaling); there is no collective on the data path, and the reported time is
+the max over ranks. Rank 0 prints one JSON line.
+
+The per-step working set (Mixtral-shaped layer: 2.8 GB of expert weights plus 0.8 GB of
+intermediates) is far larger than the 126 MB L2, so every step streams its inputs from HBM;
+no separate L2 flush is inserted.
+
+--impl reference times the CPU oracle (oracle/, plain C + OpenMP) on a bounded token sample
+of the same workload on the host cores; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 9  # route logits, top-k, count, scan, place, gather, layer0, layer1, combine
+DOMINANT_KERNEL = "moe_grouped_gemm_kernel<0>"  # layer0 grouped GEMM + SwiGLU
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral")
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--E", type=int, default=None)
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--H", type=int, default=None)
+    ap.add_argument("--F", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU seconds of the oracle sample")
+    return ap.parse_args()
+
+
+def workload(args):
+    from mixture_experts_layer_forward_b200 import synth
+    from dataclasses import replace
+
+    cfg = synth.CONFIGS[args.workload]
+    over = {k: getattr(args, k) for k in ("T", "E", "k", "H", "F") if getattr(args, k) is not None}
+    if over:
+        cfg = replace(cfg, name=cfg.name + "_" + "_".join(f"{k}{v}" for k, v in over.items()), **over)
+    return cfg
+
+
+WORKLOAD_NAMES = {
+    "tiny": "tiny MoE layer",
+    "mixtral": "Mixtral-8x7B-shaped MoE layer",
+    "phi35": "Phi-3.5-MoE-shaped MoE layer",
+    "qwen2": "Qwen2-57B-A14B-shaped MoE layer",
+    "skew": "skewed fine-grained MoE layer (Zipf 1.2 expert prior)",
+    "skew_decode": "skewed fine-grained MoE layer, decode batch",
+}
+
+
+def config_dict(cfg, args, n):
+    return {
+        "workload": WORKLOAD_NAMES.get(args.workload, args.workload) + f" ({cfg.name})",
+        "T_per_gpu": cfg.T, "H": cfg.H, "F": cfg.F, "E": cfg.E, "top_k": cfg.k,
+        "act": ["swiglu", "gelu_tanh", "relu", "identity"][cfg.act],
+        "gate": ["softmax_topk", "softmax_all"][cfg.gate],
+        "global_tokens": cfg.T * n, "parallelism": f"dp{n} replicas (no collective)",
+        "l2": "inputs larger than L2 (per-step working set >> 126 MB); no flush",
+        "seed": args.seed,
+    }
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "mixture_experts_layer_forward_b200" / "csrc").glob("*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, cfg_name):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text())
+    ent = d.get(kernel, {}).get(cfg_name)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self, t_begin, t_end):
+        """Summarise the samples whose nvidia-smi timestamp falls in [t_begin, t_end]
+        (host time.time() values) -- the timed region."""
+        if self.proc is None:
+            return None
+        time.sleep(0.3)  # let the sample that covers the end of the region arrive
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        from datetime import datetime
+
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, mxv = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            # a sample reports the state at its timestamp; keep the ones inside the region
+            # (200 ms sampling: allow one period of slack at each end)
+            if ts < t_begin - 0.2 or ts > t_end + 0.2:
+                continue
+            sm.append(clk)
+            mx = mxv
+            try:
+                power.append(float(parts[3]))
+            except ValueError:
+                pass
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def cpu_oracle_sample(cfg, inputs_host, seconds, tokens_hint=None):
+    """Time the oracle's per-token layer on a token sample sized to ~`seconds` of CPU work.
+    Returns (tokens_per_s, n_tokens, elapsed_s, threads)."""
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except AttributeError:
+        threads = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    threads = int(os.environ["OMP_NUM_THREADS"])
+    import numpy as np
+
+    import oracle
+
+    lib = oracle.load()
+    x, Wg, W1, W2, b = inputs_host
+    rng = np.random.default_rng(1234)
+
+    def run(n):
+        toks = rng.choice(cfg.T, size=min(n, cfg.T), replace=False).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_tokens(x, Wg, b, W1, W2, cfg.k, toks, act=cfg.act, gate=cfg.gate, lib=lib)
+        return len(toks), time.perf_counter() - t0
+
+    n0, t0 = run(max(threads, 4))              # calibration
+    per_tok = t0 / n0
+    n = tokens_hint or int(max(threads, min(cfg.T, seconds / max(per_tok, 1e-9))))
+    n = max(threads, (n // threads) * threads) if n >= threads else n
+    n = min(n, cfg.T)
+    n1, t1 = run(n)
+    return n1 / t1, n1, t1, threads
+
+
+def host_inputs(inp):
+    from mixture_experts_layer_forward_b200 import synth
+
+    b = None if inp["bias"] is None else inp["bias"].cpu().numpy()
+    return (synth.bf16_bits(inp["x"]), synth.bf16_bits(inp["Wg"]), synth.bf16_bits(inp["W1"]),
+            synth.bf16_bits(inp["W2"]), b)
+
+
+def emit(obj):
+    print(json.dumps(obj), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------------------
+
+def run_reference(args):
+    from mixture_experts_layer_forward_b200 import dp, synth
+
+    rank, _, world = dp.env_rank()
+    if rank != 0:
+        return 0
+    cfg = workload(args)
+    inp = synth.make_inputs(cfg, seed=args.seed, device="cpu")
+    hin = host_inputs(inp)
+    K, W = max(1, args.steps), max(0, args.warmup)
+    # each step is a bounded token sample; the whole run stays within a few minutes
+    per_step_s = max(1.0, min(args.cpu_seconds, 150.0 / (K + W)))
+    _, n_tok, _, threads = cpu_oracle_sample(cfg, hin, per_step_s)
+    for _ in range(W):
+        cpu_oracle_sample(cfg, hin, per_step_s, tokens_hint=n_tok)
+    tot_t, tot_n = 0.0, 0
+    for _ in range(K):
+        _, n, t, _ = cpu_oracle_sample(cfg, hin, per_step_s, tokens_hint=n_tok)
+        tot_t += t
+        tot_n += n
+    value = tot_n / tot_t
+    flops_per_tok = cfg.useful_flops / cfg.T
+    emit({
+        "impl": "reference", "metric": "MoE-layer forward tokens/s", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": 1000.0 * tot_t / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (router logits f32)", "data": "synthetic",
+        "config": config_dict(cfg, args, 1),
+        "tflops": value * flops_per_tok / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n_tok} random tokens of the {cfg.T}-token batch per step "
+                                   f"(per-token definition path, fp64)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    })
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_layer_forward_b200 as moe
+    from mixture_experts_layer_forward_b200 import dp, synth
+
+    rank, local_rank, world = dp.env_rank()
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    n = world
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = workload(args)
+    K, W = args.steps, max(3, args.warmup)
+
+    inp = synth.make_inputs(cfg, seed=args.seed, device=dev,
+                            x_seed=dp.replica_x_seed(args.seed, rank) if world > 1 else None)
+    p = moe.Problem.from_config(cfg)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    args_fwd = (p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out, ws)
+
+    for _ in range(W):
+        moe.moe_forward(*args_fwd)
+    torch.cuda.synchronize(dev)
+    assert moe.moe_get_device_status(ws) == 0, "device status after warm-up"
+
+    # stage events of every timed step (recorded on the launch stream by the library)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGE_EVENTS)]
+           for _ in range(K)]
+    for row in evs:          # create the CUDA events now, outside the timed region
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = None
+    sampler = None
+    if not args.no_clocks:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        sampler.start()
+        time.sleep(0.5)
+    dp.barrier(dev)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    start.record(stream)
+    for i in range(K):
+        moe.moe_forward_staged(*args_fwd, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_end = time.time()
+    dp.barrier(dev)
+    if sampler is not None:
+        clocks = sampler.stop(t_begin, t_end)
+    ms_local = start.elapsed_time(end)
+    status = moe.moe_get_device_status(ws)
+    assert status == 0, f"device status {status}"
+    ms = dp.max_over_ranks(ms_local, device=dev)
+    ms_per_step = ms / K
+
+    stage_names = ["route", "dispatch", "layer0_gemm_swiglu", "layer1_gemm_scale", "combine"]
+    stage_ms = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+                for j, nm in enumerate(stage_names)}
+
+    # end to end through the public API with host buffers (x in, out back, every step)
+    e2e = None
+    if not args.no_e2e:
+        x_h = inp["x"].cpu().pin_memory()
+        out_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            moe.moe_forward_host(p, x_h, inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out_h, ws)
+        dp.barrier(dev)
+        torch.cuda.synchronize(dev)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(K):
+            moe.moe_forward_host(p, x_h, inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out_h, ws)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        dp.barrier(dev)
+        e2e_ms = dp.max_over_ranks(s2.elapsed_time(e2), device=dev) / K
+        e2e = {"value": n * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+               "ms_per_step": e2e_ms}
+
+    peaks, peak_src = load_peaks()
+    # Denominator in the clock regime the kernels ran in: the power-capped (sustained) GEMM
+    # peak when the sampled SM clock sat well below its maximum, the burst peak otherwise.
+    sustained = bool(clocks and clocks.get("sm_max_mhz") and
+                     clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"])
+    regime = "sustained" if sustained else "burst"
+    tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
+    layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
+    gemm0_flops = (4 if cfg.act == 0 else 2) * cfg.T * cfg.k * cfg.H * cfg.F
+    g0_ms = stage_ms["layer0_gemm_swiglu"]
+    g0_tflops = gemm0_flops / (g0_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": DOMINANT_KERNEL, "achieved": g0_tflops,
+                "peak": tf_peak, "unit": "TFLOP/s", "frac": g0_tflops / tf_peak,
+                "traffic": traffic_for(DOMINANT_KERNEL, cfg.name),
+                "peak_source": f"{peak_src} bf16 {regime} (sampled SM clock decides the regime)",
+                "algorithmic_flops_per_launch": gemm0_flops, "ms_per_launch": g0_ms}
+
+    line = {
+        "metric": "MoE-layer forward tokens/s", "value": n * cfg.T / (ms_per_step / 1e3),
+        "unit": "tokens/s", "n_gpus": n, "steps": K, "warmup": W, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random inputs and random-init weights of the layer's shape)",
+        "config": config_dict(cfg, args, n),
+        "tflops": layer_tflops * n,
+        "layer_roofline": {"bound": "tensor", "achieved": layer_tflops, "peak": tf_peak,
+                           "unit": "TFLOP/s per GPU", "frac": layer_tflops / tf_peak,
+                           "peak_source": f"{peak_src} bf16 {regime}"},
+        "roofline": roofline,
+        "stage_ms": stage_ms,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+
+    if rank == 0 and not args.no_cpu_baseline:
+        hin = host_inputs(inp)
+        v, n_tok, t, threads = cpu_oracle_sample(cfg, hin, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{n_tok} random tokens of the {cfg.T}-token batch, "
+                                          f"{t:.1f} s (per-token definition path, fp64)"}
+    if rank == 0:
+        emit(line)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

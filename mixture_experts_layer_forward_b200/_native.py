@@ -182,6 +182,9 @@ def moe_forward_staged(p, x, Wg, bias, W1, W2, out, ws, events, topk_idx_out=Non
     w, n = _ws(ws)
     if len(events) != MOE_NUM_STAGE_EVENTS:
         raise ValueError(f"need {MOE_NUM_STAGE_EVENTS} events")
+    for ev in events:
+        if ev.cuda_event == 0:   # torch creates the CUDA event lazily, on its first record
+            ev.record()
     arr = (ctypes.c_void_p * MOE_NUM_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
     rc = library().moe_forward_staged(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
                                       _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
