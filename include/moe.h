@@ -184,6 +184,30 @@ MOE_API moe_status moe_get_device_status(void *ws, void *stream);
 /* Human-readable name of a status code (static storage). */
 MOE_API const char *moe_status_string(moe_status s);
 
+/* Largest T * E that moe_route_noalloc accepts: its logits scratch is a fixed array of
+ * this many floats (4 MiB) inside the library. */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS (1 << 20)
+
+/* moe_route without a workspace, for callers that cannot allocate device memory: code that
+ * is handed only its input and output buffers by a host framework that owns the device
+ * heap (a plugin inside an inference engine, for example), and serving loops that must not
+ * call cudaMalloc/cudaFree after start-up because those calls can synchronise the device
+ * and stall every other stream. The pages have no counterpart of this entry point.
+ *   Same arguments and results as moe_route, minus ws/ws_bytes. The router's fp32 logits
+ *   [T, E] go to a fixed scratch array that the library holds in device memory on every GPU
+ *   that loads it, until the process exits; T * E above MOE_ROUTE_NOALLOC_MAX_LOGITS
+ *   returns MOE_ERR_UNSUPPORTED and launches nothing.
+ *   The first call on a device looks up that array's device address (once per device,
+ *   with the device current); make that first call before any stream capture. Later calls
+ *   do no set-up. The call allocates nothing and frees nothing.
+ *   All calls share the one array and every call overwrites the logits it reads, so nothing
+ *   has to be cleared between calls; but two calls whose kernels overlap on the GPU (on
+ *   different streams, or from different host threads) race on the array and may return
+ *   each other's routing. The current device must be the device of `stream`. */
+MOE_API moe_status moe_route_noalloc(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                                     const float *bias, int32_t *topk_idx, float *topk_w,
+                                     void *stream);
+
 /* Test hook for the bounded device waits: the timeout, in nanoseconds, that every
  * bounded wait of later launches uses (default 2e9; values <= 0 restore the default).
  * Returns the previous value. Not thread-safe; meant for tests. */

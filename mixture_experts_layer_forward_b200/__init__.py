@@ -29,6 +29,7 @@ from ._native import (  # noqa: F401
     moe_get_device_status,
     moe_padded_rows_max,
     moe_route,
+    moe_route_noalloc,
     moe_set_wait_timeout_ns,
     moe_workspace_size,
 )

@@ -76,6 +76,7 @@ def library() -> ctypes.CDLL:
             "moe_workspace_size": ([P], sz),
             "moe_padded_rows_max": ([P], i64),
             "moe_route": ([P, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_route_noalloc": ([P, vp, vp, vp, vp, vp, vp], i32),
             "moe_dispatch": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_forward": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_forward_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
@@ -150,6 +151,17 @@ def moe_route(p, x, Wg, bias, topk_idx, topk_w, ws, stream=None):
                              _ptr(bias, f32, "bias"), _ptr(topk_idx, i32, "topk_idx"),
                              _ptr(topk_w, f32, "topk_w"), w, n, _stream(stream))
     _check("moe_route", rc)
+
+
+def moe_route_noalloc(p, x, Wg, bias, topk_idx, topk_w, stream=None):
+    """moe_route without a workspace (the library's fixed scratch array holds the logits).
+    For callers that cannot allocate device memory; see include/moe.h for the size limit
+    and the rule that overlapping calls race."""
+    bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
+    rc = library().moe_route_noalloc(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                                     _ptr(bias, f32, "bias"), _ptr(topk_idx, i32, "topk_idx"),
+                                     _ptr(topk_w, f32, "topk_w"), _stream(stream))
+    _check("moe_route_noalloc", rc)
 
 
 def moe_dispatch(p, topk_idx, counts, offsets, padded_offsets, gather_idx, inv_pos, ws,

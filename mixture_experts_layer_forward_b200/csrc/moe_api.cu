@@ -282,6 +282,28 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
 
 moe_status to_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Fixed logits scratch of moe_route_noalloc: one copy per GPU that loads the library, held
+// until the process exits. Only device code may name it directly; host code must use the
+// address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) float g_route_noalloc_logits[MOE_ROUTE_NOALLOC_MAX_LOGITS];
+
+// Device address of g_route_noalloc_logits on the current device, looked up on the first
+// call for each device and cached; nullptr if the lookup fails.
+float *route_noalloc_scratch()
+{
+    static std::mutex mu;
+    static float *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_route_noalloc_logits) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<float *>(ptr);
+    }
+    return cache[dev];
+}
+
 cudaError_t record(void *const *events, int n, int i, cudaStream_t st)
 {
     if (n == 0) return cudaSuccess;
@@ -417,6 +439,26 @@ moe_status moe_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg
     int *status = at<int>(ws, L.status);
     if (p->T == 0) return to_status(cudaMemsetAsync(status, 0, 8, st));
     return to_status(launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st));
+}
+
+moe_status moe_route_noalloc(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                             const float *bias, int32_t *topk_idx, float *topk_w, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (Wg == nullptr) return MOE_ERR_INVALID_ARG;
+    if (p->T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)p->T * p->E > (int64_t)MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(topk_w))
+        return MOE_ERR_INVALID_ARG;
+    if (p->T == 0) return MOE_OK;
+    float *logits = route_noalloc_scratch();
+    if (logits == nullptr) return MOE_ERR_CUDA;
+    // the router kernels overwrite every logit before reading it: nothing to clear; there is
+    // no status word to report through (the router raises no device errors)
+    return to_status(launch_route(p, x, Wg, bias, topk_idx, topk_w, logits, nullptr,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *counts,
