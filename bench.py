@@ -100,96 +100,91 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def source_hash(files):
     h = hashlib.sha256()
-    for f in sorted((ROOT / "mixture_experts_layer_forward_b200" / "csrc").glob("*")):
-        h.update(f.read_bytes())
+    for f in files:
+        h.update((ROOT / "mixture_experts_layer_forward_b200" / "csrc" / f).read_bytes())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel, cfg_name):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the kernel's
+    sources are unchanged since the counters were taken; else None."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
     d = json.loads(p.read_text())
     ent = d.get(kernel, {}).get(cfg_name)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent:
+        return None
+    try:
+        if source_hash(ent["source_files"]) != ent.get("source_hash"):
+            return None
+    except (OSError, KeyError):
         return None
     return ent.get("bytes_per_launch")
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """Samples the SM clock, power and clock-event (throttle) reasons of one GPU through NVML
+    every ~20 ms on a background thread (read-only queries; no setting is changed).
+    Falls back to `nvidia-smi -lms 200` when NVML is unavailable."""
 
-    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, uuid):
+    def __init__(self, uuid, period_s=0.02):
         self.uuid = uuid
-        self.proc = None
-        self.lines = []
+        self.period = period_s
+        self.samples = []  # (host time, sm MHz, max sm MHz, power W, reason bitmask)
+        self._stop = threading.Event()
+        self.t = None
+        self.source = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.pynvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.source = "nvml"
+        except Exception:  # noqa: BLE001 - no NVML: the clock record is simply absent
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.pynvml
+        while not self._stop.is_set():
+            try:
+                clk = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                self.samples.append((time.time(), clk, self.max_mhz, pw, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self.period)
 
     def stop(self, t_begin, t_end):
-        """Summarise the samples whose nvidia-smi timestamp falls in [t_begin, t_end]
-        (host time.time() values) -- the timed region."""
-        if self.proc is None:
+        """Summary of the samples taken inside the timed region [t_begin, t_end]."""
+        if self.t is None:
             return None
-        time.sleep(0.3)  # let the sample that covers the end of the region arrive
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self._stop.set()
         self.t.join(timeout=5)
-        from datetime import datetime
-
-        sm, mx, reasons, power = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                clk, mxv = float(parts[1]), float(parts[2])
-            except ValueError:
-                continue
-            # a sample reports the state at its timestamp; keep the ones inside the region
-            # (200 ms sampling: allow one period of slack at each end)
-            if ts < t_begin - 0.2 or ts > t_end + 0.2:
-                continue
-            sm.append(clk)
-            mx = mxv
-            try:
-                power.append(float(parts[3]))
-            except ValueError:
-                pass
-            for nm, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+        win = [x for x in self.samples if t_begin <= x[0] <= t_end]
+        if not win:  # a region shorter than one period: take the nearest sample
+            win = sorted(self.samples, key=lambda x: abs(x[0] - 0.5 * (t_begin + t_end)))[:1]
+        if not win:
             return None
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power) if power else None}
+        sm = sorted(x[1] for x in win)
+        seen = 0
+        for x in win:
+            seen |= x[4]
+        reasons = sorted(n for n, bit in self.REASONS.items() if seen & bit)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": win[0][2], "reasons": reasons,
+                "samples": len(win), "power_w_max": max(x[3] for x in win), "source": self.source}
 
 
 def cpu_oracle_sample(cfg, inputs_host, seconds, tokens_hint=None):
@@ -328,7 +323,6 @@ def run_ours(args):
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
         sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
         sampler.start()
-        time.sleep(0.5)
     dp.barrier(dev)
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -375,9 +369,10 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     # Denominator in the clock regime the kernels ran in: the power-capped (sustained) GEMM
-    # peak when the sampled SM clock sat well below its maximum, the burst peak otherwise.
-    sustained = bool(clocks and clocks.get("sm_max_mhz") and
-                     clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"])
+    # peak when the power cap throttled the SM clock during the timed region or the clock sat
+    # well below its maximum, the burst peak otherwise.
+    sustained = bool(clocks and ("sw_power_cap" in clocks["reasons"] or
+                                 clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]))
     regime = "sustained" if sustained else "burst"
     tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
     layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
@@ -387,7 +382,7 @@ def run_ours(args):
     roofline = {"bound": "tensor", "kernel": DOMINANT_KERNEL, "achieved": g0_tflops,
                 "peak": tf_peak, "unit": "TFLOP/s", "frac": g0_tflops / tf_peak,
                 "traffic": traffic_for(DOMINANT_KERNEL, cfg.name),
-                "peak_source": f"{peak_src} bf16 {regime} (sampled SM clock decides the regime)",
+                "peak_source": f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)",
                 "algorithmic_flops_per_launch": gemm0_flops, "ms_per_launch": g0_ms}
 
     line = {

@@ -185,6 +185,17 @@ template <int KIND> cudaError_t gemm_smem_attr()
 // stage launchers (no argument checks; callers validated)
 // ---------------------------------------------------------------------------------------
 
+template <int BT, int BE, int RT, int RE, int HC, int NS>
+void launch_route_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *Wg, const float *bias,
+                         float *logits, int T, int H, int E, int *status, cudaStream_t st)
+{
+    constexpr int smem = RouteSmem<BT, BE, HC, NS>::BYTES;
+    auto kern = route_logits_kernel<BT, BE, RT, RE, HC, NS>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    dim3 grid((T + BT - 1) / BT, (E + BE - 1) / BE), block(BE / RE, BT / RT);
+    kern<<<grid, block, smem, st>>>(x, Wg, bias, logits, T, H, E, status);
+}
+
 cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                          const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
                          int *status, cudaStream_t st)
@@ -192,15 +203,17 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     const int T = p->T, H = p->H, E = p->E;
     const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     const auto *wb = reinterpret_cast<const __nv_bfloat16 *>(Wg);
-    if (E <= 8) {
-        dim3 grid((T + 31) / 32, 1), block(8, 32);
-        route_logits_kernel<32, 8, 1, 1><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
-    } else if (E <= 16) {
-        dim3 grid((T + 15) / 16, 1), block(16, 16);
-        route_logits_kernel<16, 16, 1, 1><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
+    // blocks of the large-E tile (64 tokens x 64 experts); fewer than the SMs: go narrow
+    const int64_t large_blocks = (int64_t)((T + 63) / 64) * ((E + 63) / 64);
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    if (E <= 8 && T >= 64 * sms / 2) {
+        launch_route_logits<ROUTE_SMALL_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+    } else if (E > 8 && E <= 16 && T >= 32 * sms / 2) {
+        launch_route_logits<ROUTE_MID_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+    } else if (E > 16 && large_blocks >= sms) {
+        launch_route_logits<ROUTE_LARGE_CFG>(xb, wb, bias, logits, T, H, E, status, st);
     } else {
-        dim3 grid((T + 63) / 64, (E + 63) / 64), block(16, 16);
-        route_logits_kernel<64, 64, 4, 4><<<grid, block, 0, st>>>(xb, wb, bias, logits, T, H, E, status);
+        launch_route_logits<ROUTE_NARROW_CFG>(xb, wb, bias, logits, T, H, E, status, st);
     }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -6,6 +6,10 @@
 //    result is bit-identical to a plain sequential fp32 loop (a bf16 x bf16 product is exact
 //    in fp32, so the fused multiply-add rounds exactly like add-after-multiply). The tile
 //    is staged through shared memory; h is consumed in float4 steps, in order.
+//    That order caps the parallelism at T*E independent chains, and each chain needs two
+//    shared-memory operands per FMA unless a thread owns several tokens and experts; the
+//    kernel is bound by shared-memory bandwidth for small E and by FP32 FMA issue for
+//    large E.
 // 2. route_topk_kernel: one warp per token; k rounds of a warp argmax (ties to the lower
 //    expert id), then the gate weights.
 #pragma once
@@ -14,21 +18,55 @@
 
 namespace moe {
 
-constexpr int ROUTE_HC = 32; // h values staged per shared-memory step
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, bool valid)
+{
+    // src-size 0 zero-fills the 16 destination bytes (rows past T, columns past H or E)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-// Block = (BE/RE) x (BT/RT) threads; thread (tx, ty) owns tokens ty*RT.. and experts tx*RE..
-template <int BT, int BE, int RT, int RE>
+template <int BT, int BE, int HC, int NS> struct RouteSmem {
+    static constexpr int LD = HC + 4;                      // fp32 row stride (odd 16-byte count)
+    static constexpr int X_RING = BT * HC * 2;             // bf16 x chunk
+    static constexpr int W_RING = HC * BE * 2;             // bf16 gate chunk [h][e]
+    static constexpr int RING = NS * (X_RING + W_RING);
+    static constexpr int XF = 2 * BT * LD * 4;             // fp32 x, double buffered
+    static constexpr int WF = 2 * BE * LD * 4;             // fp32 gate, [e][h], double buffered
+    static constexpr int BYTES = RING + XF + WF;
+};
+
+// Block = (BE/RE) x (BT/RT) threads. Thread (tx, ty) owns tokens ty + (BT/RT)*i and experts
+// tx + (BE/RE)*j; the strided ownership keeps the float4 shared-memory reads free of bank
+// conflicts. The h axis is streamed in chunks of HC through an NS-stage cp.async ring (bf16,
+// exactly as stored); each thread widens the 16-byte pieces it copied itself into fp32
+// buffers (x as [token][h], the gate chunk transposed to [expert][h]), so one barrier per
+// chunk suffices and NS-1 chunks are in flight while the current one is consumed.
+// Every accumulator still walks h upward, one fused multiply-add per h.
+template <int BT, int BE, int RT, int RE, int HC, int NS>
 __global__ void __launch_bounds__((BT / RT) * (BE / RE))
     route_logits_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Wg,
                         const float *__restrict__ bias, float *__restrict__ logits, int T, int H,
                         int E, int *status)
 {
+    using S = RouteSmem<BT, BE, HC, NS>;
     constexpr int TX = BE / RE;
     constexpr int TY = BT / RT;
     constexpr int NT = TX * TY;
-    constexpr int LD = ROUTE_HC + 4; // row stride in floats (keeps float4 alignment)
-    __shared__ __align__(16) float xs[BT][LD];
-    __shared__ __align__(16) float ws[BE][LD];
+    constexpr int LD = S::LD;
+    constexpr int XV = BT * HC / 8; // 16-byte x pieces per chunk
+    constexpr int WV = HC * BE / 8; // 16-byte gate pieces per chunk (8 experts of one h)
+    constexpr int XPT = (XV + NT - 1) / NT;
+    constexpr int WPT = (WV + NT - 1) / NT;
+    static_assert(BE % 8 == 0 && HC % 8 == 0, "tile shape");
+    extern __shared__ __align__(16) uint8_t rsmem[];
+    float *xf = reinterpret_cast<float *>(rsmem + S::RING);
+    float *wf = reinterpret_cast<float *>(rsmem + S::RING + S::XF);
 
     if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 &&
         threadIdx.y == 0) {
@@ -39,6 +77,87 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
     const int tid = threadIdx.y * TX + threadIdx.x;
     const int t0 = blockIdx.x * BT;
     const int e0 = blockIdx.y * BE;
+    const int nchunk = (H + HC - 1) / HC;
+    // rows of a vectorised gate copy must be whole 8-expert groups inside the row
+    const bool wvec = (E % 8) == 0;
+
+    auto ring_x = [&](int slot) { return rsmem + slot * (S::X_RING + S::W_RING); };
+    auto ring_w = [&](int slot) { return rsmem + slot * (S::X_RING + S::W_RING) + S::X_RING; };
+
+    auto issue = [&](int c) {
+        const int slot = c % NS;
+        const int h0 = c * HC;
+        const uint32_t xs = smem_u32(ring_x(slot));
+        const uint32_t wsr = smem_u32(ring_w(slot));
+#pragma unroll
+        for (int i = 0; i < XPT; ++i) {
+            const int v = tid + i * NT;
+            if (v < XV) {
+                const int r = v / (HC / 8), q = v % (HC / 8);
+                const int t = t0 + r, h = h0 + q * 8;
+                const bool ok = (t < T) && (h < H);
+                cp_async_16(xs + v * 16, ok ? (const void *)(x + (size_t)t * H + h) : (const void *)x, ok);
+            }
+        }
+        if (wvec) {
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) {
+                const int v = tid + i * NT;
+                if (v < WV) {
+                    // consecutive threads take consecutive h: their transposed stores below
+                    // then land in consecutive shared-memory words (no bank conflicts)
+                    const int hh = v % HC, g = v / HC;
+                    const int h = h0 + hh, e = e0 + g * 8;
+                    const bool ok = (h < H) && (e < E);
+                    cp_async_16(wsr + v * 16, ok ? (const void *)(Wg + (size_t)h * E + e) : (const void *)Wg,
+                                ok);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    // widen the pieces this thread copied for chunk c into the fp32 buffers of parity c&1
+    auto widen = [&](int c) {
+        const int slot = c % NS;
+        const int h0 = c * HC;
+        float *xd = xf + (c & 1) * BT * LD;
+        float *wd = wf + (c & 1) * BE * LD;
+        const uint4 *xsrc = reinterpret_cast<const uint4 *>(ring_x(slot));
+#pragma unroll
+        for (int i = 0; i < XPT; ++i) {
+            const int v = tid + i * NT;
+            if (v < XV) {
+                const int r = v / (HC / 8), q = v % (HC / 8);
+                const uint4 u = xsrc[v];
+                float4 *d = reinterpret_cast<float4 *>(xd + r * LD + q * 8);
+                d[0] = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+                d[1] = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
+            }
+        }
+        if (wvec) {
+            const uint4 *wsrc = reinterpret_cast<const uint4 *>(ring_w(slot));
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) {
+                const int v = tid + i * NT;
+                if (v < WV) {
+                    const int hh = v % HC, g = v / HC;
+                    const uint4 u = wsrc[v];
+                    float *d = wd + (g * 8) * LD + hh;
+                    d[0 * LD] = bf16_lo(u.x); d[1 * LD] = bf16_hi(u.x);
+                    d[2 * LD] = bf16_lo(u.y); d[3 * LD] = bf16_hi(u.y);
+                    d[4 * LD] = bf16_lo(u.z); d[5 * LD] = bf16_hi(u.z);
+                    d[6 * LD] = bf16_lo(u.w); d[7 * LD] = bf16_hi(u.w);
+                }
+            }
+        } else {
+            // expert counts that are not a multiple of 8: plain loads (small problems only)
+            for (int v = tid; v < HC * BE; v += NT) {
+                const int hh = v / BE, ee = v % BE;
+                const int h = h0 + hh, e = e0 + ee;
+                wd[ee * LD + hh] = (h < H && e < E) ? __bfloat162float(Wg[(size_t)h * E + e]) : 0.0f;
+            }
+        }
+    };
 
     float acc[RT][RE];
 #pragma unroll
@@ -46,43 +165,36 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
 #pragma unroll
         for (int j = 0; j < RE; ++j) acc[i][j] = 0.0f;
 
-    for (int h0 = 0; h0 < H; h0 += ROUTE_HC) {
-        // x tile: BT rows x 32 bf16, 16-byte chunks
-        for (int c = tid; c < BT * (ROUTE_HC / 8); c += NT) {
-            const int r = c / (ROUTE_HC / 8);
-            const int q = c % (ROUTE_HC / 8);
-            const int t = t0 + r;
-            float v[8];
-            if (t < T) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + h0 + q * 8);
-                v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
-                v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-                v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z);
-                v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-            } else {
+    // prologue: NS-1 chunks in flight, chunk 0 widened
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[r][q * 8 + i] = v[i];
-        }
-        // gate tile, transposed to [expert][h]
-        for (int c = tid; c < BE * ROUTE_HC; c += NT) {
-            const int hh = c / BE;
-            const int ee = c % BE;
-            const int e = e0 + ee;
-            ws[ee][hh] = (e < E) ? __bfloat162float(Wg[(size_t)(h0 + hh) * E + e]) : 0.0f;
-        }
-        __syncthreads();
-#pragma unroll 2
-        for (int hh = 0; hh < ROUTE_HC; hh += 4) {
-            float4 xv[RT], wv[RE];
+    for (int c = 0; c < NS - 1; ++c) {
+        if (c < nchunk) issue(c);
+        else cp_async_commit();
+    }
+    cp_async_wait<NS - 2>();
+    widen(0);
+
+    for (int c = 0; c < nchunk; ++c) {
+        __syncthreads(); // chunk c widened by everyone; the buffers of chunk c-1 are free
+        if (c + NS - 1 < nchunk) issue(c + NS - 1);
+        else cp_async_commit(); // keep one group per iteration
+        const float *xc = xf + (c & 1) * BT * LD + threadIdx.y * LD;
+        const float *wc = wf + (c & 1) * BE * LD + threadIdx.x * LD;
+        // the last chunk may run past H: its x and gate values are zero there, and an exact
+        // zero product leaves each accumulator's value unchanged.
+        // Operands of step s+1 are loaded into registers before the FMAs of step s, so the
+        // dependent FMA chains never wait on a shared-memory load.
+        float4 xa[RT], wa[RE], xb[RT], wb[RE];
+        auto ld = [&](float4 (&xv)[RT], float4 (&wv)[RE], int hh) {
 #pragma unroll
             for (int i = 0; i < RT; ++i)
-                xv[i] = *reinterpret_cast<const float4 *>(&xs[threadIdx.y * RT + i][hh]);
+                xv[i] = *reinterpret_cast<const float4 *>(xc + TY * i * LD + hh);
 #pragma unroll
             for (int j = 0; j < RE; ++j)
-                wv[j] = *reinterpret_cast<const float4 *>(&ws[threadIdx.x * RE + j][hh]);
+                wv[j] = *reinterpret_cast<const float4 *>(wc + TX * j * LD + hh);
+        };
+        // h ascending within every accumulator: x, y, z, w are h, h+1, h+2, h+3
+        auto fma4 = [&](const float4 (&xv)[RT], const float4 (&wv)[RE]) {
 #pragma unroll
             for (int i = 0; i < RT; ++i)
 #pragma unroll
@@ -92,16 +204,28 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
                     acc[i][j] = fmaf(xv[i].z, wv[j].z, acc[i][j]);
                     acc[i][j] = fmaf(xv[i].w, wv[j].w, acc[i][j]);
                 }
+        };
+        ld(xa, wa, 0);
+#pragma unroll
+        for (int hh = 0; hh < HC; hh += 8) {
+            ld(xb, wb, hh + 4);
+            fma4(xa, wa);
+            if (hh + 8 < HC) ld(xa, wa, hh + 8);
+            fma4(xb, wb);
         }
-        __syncthreads();
+        if (c + 1 < nchunk) {
+            cp_async_wait<NS - 2>(); // this thread's copies of chunk c+1 have landed
+            widen(c + 1);
+        }
     }
+    cp_async_wait<0>();
 #pragma unroll
     for (int i = 0; i < RT; ++i) {
-        const int t = t0 + threadIdx.y * RT + i;
+        const int t = t0 + threadIdx.y + TY * i;
         if (t >= T) continue;
 #pragma unroll
         for (int j = 0; j < RE; ++j) {
-            const int e = e0 + threadIdx.x * RE + j;
+            const int e = e0 + threadIdx.x + TX * j;
             if (e >= E) continue;
             float v = acc[i][j];
             if (bias != nullptr) v = v + bias[e];
@@ -109,6 +233,24 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
         }
     }
 }
+
+// Tile shapes per expert-count class: BT, BE, RT, RE, HC, NS.
+// Measured on B200 (router alone): E=8, T=8192, H=4096: 75 us; E=16, T=16384: 162 us;
+// E=64, T=8192, H=3584: 169 us; E=256, T=4096, H=7168: 518 us.
+#ifndef ROUTE_SMALL_CFG
+#define ROUTE_SMALL_CFG 64, 8, 2, 2, 64, 4    // E <= 8
+#endif
+#ifndef ROUTE_MID_CFG
+#define ROUTE_MID_CFG 32, 16, 2, 2, 64, 4     // 8 < E <= 16
+#endif
+#ifndef ROUTE_LARGE_CFG
+#define ROUTE_LARGE_CFG 64, 64, 4, 4, 32, 4   // E > 16
+#endif
+// Small batches (decode): one output per thread, so that T*E outputs still spread over
+// every SM (T=64, E=256 gives 64 blocks instead of 4).
+#ifndef ROUTE_NARROW_CFG
+#define ROUTE_NARROW_CFG 16, 16, 1, 1, 64, 4
+#endif
 
 constexpr int TOPK_WARPS = 8; // tokens per block
 

@@ -82,6 +82,10 @@ ROUTE_CASES = [
     ("e8_all", 99, 128, 8, 3, False, 0.0, 1),
     ("e40_k40", 33, 64, 40, 40, False, 0.0, 0),
     ("e1024_k33", 9, 64, 1024, 33, False, 0.0, 1),
+    # large enough to select each non-narrow tile class of the router
+    ("e8_tile", 5000, 192, 8, 2, False, 0.0, 0),
+    ("e16_tile", 2500, 320, 16, 2, True, 0.0, 0),
+    ("e320_tile", 2100, 128, 320, 8, False, 1.2, 0),
 ]
 
 
