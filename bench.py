@@ -34,7 +34,7 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 9  # route logits, top-k, count, scan, place, gather, layer0, layer1, combine
+LAUNCHES_PER_STEP = 8  # route logits, top-k, count, scan, place, layer0 (gathers x), layer1, combine
 DOMINANT_KERNEL = "moe_grouped_gemm_kernel<0>"  # layer0 grouped GEMM + SwiGLU
 
 
@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--H", type=int, default=None)
     ap.add_argument("--F", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--gemm-mode", choices=["auto", "single", "pair"], default="auto",
+                    help="grouped-GEMM variant (moe_set_gemm_mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -89,6 +91,7 @@ def config_dict(cfg, args, n):
         "global_tokens": cfg.T * n, "parallelism": f"dp{n} replicas (no collective)",
         "l2": "inputs larger than L2 (per-step working set >> 126 MB); no flush",
         "seed": args.seed,
+        "gemm_mode": getattr(args, "gemm_mode", "auto"),
     }
 
 
@@ -296,6 +299,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     cfg = workload(args)
     K, W = args.steps, max(3, args.warmup)
+    moe.moe_set_gemm_mode({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE_CTA,
+                           "pair": moe.GEMM_CTA_PAIR}[args.gemm_mode])
 
     inp = synth.make_inputs(cfg, seed=args.seed, device=dev,
                             x_seed=dp.replica_x_seed(args.seed, rank) if world > 1 else None)

@@ -213,6 +213,17 @@ MOE_API moe_status moe_route_noalloc(const moe_problem *p, const moe_bf16 *x, co
  * Returns the previous value. Not thread-safe; meant for tests. */
 MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
 
+/* Grouped-GEMM variant used by later launches (a tuning and test hook; not thread-safe):
+ * MOE_GEMM_SINGLE_CTA runs one 128 x 256 tile per SM; MOE_GEMM_CTA_PAIR runs one
+ * 256 x 256 tile per pair of SMs (tcgen05 cta_group::2: each SM loads half of the weight
+ * tile); MOE_GEMM_AUTO (the default) picks the single-CTA variant, the faster one under the
+ * sustained power cap. Both compute the same layer. Returns the previous mode, or -1 for an
+ * unknown mode. */
+#define MOE_GEMM_AUTO 0
+#define MOE_GEMM_SINGLE_CTA 1
+#define MOE_GEMM_CTA_PAIR 2
+MOE_API int moe_set_gemm_mode(int mode);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,6 +30,10 @@ from ._native import (  # noqa: F401
     moe_padded_rows_max,
     moe_route,
     moe_route_noalloc,
+    moe_set_gemm_mode,
     moe_set_wait_timeout_ns,
+    GEMM_AUTO,
+    GEMM_CTA_PAIR,
+    GEMM_SINGLE_CTA,
     moe_workspace_size,
 )

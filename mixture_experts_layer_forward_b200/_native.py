@@ -86,6 +86,7 @@ def library() -> ctypes.CDLL:
             "moe_get_device_status": ([vp, vp], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
             "moe_set_wait_timeout_ns": ([i64], i64),
+            "moe_set_gemm_mode": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -238,3 +239,14 @@ def moe_get_device_status(ws, stream=None) -> int:
 
 def moe_set_wait_timeout_ns(ns: int) -> int:
     return int(library().moe_set_wait_timeout_ns(int(ns)))
+
+
+GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR = 0, 1, 2
+
+
+def moe_set_gemm_mode(mode: int) -> int:
+    """Select the grouped-GEMM variant of later launches; returns the previous mode."""
+    rc = int(library().moe_set_gemm_mode(int(mode)))
+    if rc < 0:
+        raise ValueError(f"unknown GEMM mode {mode}")
+    return rc

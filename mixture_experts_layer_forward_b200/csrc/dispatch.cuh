@@ -25,8 +25,10 @@ constexpr int M_TILE = 128;
 
 // Workspace-resident bookkeeping written by the scan and read by the GEMMs.
 struct DispatchMeta {
-    int num_tiles;  // sum_e ceil(c_e / M_TILE)
+    int num_tiles;   // sum_e ceil(c_e / M_TILE)
     int padded_rows; // P_pad = num_tiles * M_TILE
+    int num_ptiles;  // sum_e ceil(ceil(c_e / M_TILE) / 2): pairs of m-tiles of one expert
+    int pad_;
 };
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
@@ -94,7 +96,8 @@ __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk, int E,
                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                          int32_t *__restrict__ padded_offsets, int32_t *__restrict__ tile_off,
-                         int32_t *__restrict__ tile_expert, DispatchMeta *meta,
+                         int32_t *__restrict__ tile_expert, int32_t *__restrict__ ptile_off,
+                         int32_t *__restrict__ ptile_expert, DispatchMeta *meta,
                          int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
                          int64_t padded_rows_max)
 {
@@ -115,6 +118,8 @@ __global__ void __launch_bounds__(1024)
     const int ntile = (c + M_TILE - 1) / M_TILE;
     const int inc_c = block_inclusive_scan_1024(c, warp_sums);
     const int inc_t = block_inclusive_scan_1024(ntile, warp_sums);
+    const int nptile = (ntile + 1) / 2;
+    const int inc_p = block_inclusive_scan_1024(nptile, warp_sums);
     if (e < E) {
         if (offsets != nullptr) {
             offsets[e + 1] = inc_c;
@@ -130,9 +135,15 @@ __global__ void __launch_bounds__(1024)
         }
         s_poff[e] = tile_first * M_TILE;
         for (int i = 0; i < ntile; ++i) tile_expert[tile_first + i] = e;
+        if (ptile_off != nullptr) {
+            ptile_off[e + 1] = inc_p;
+            if (e == 0) ptile_off[0] = 0;
+            for (int i = 0; i < nptile; ++i) ptile_expert[inc_p - nptile + i] = e;
+        }
         if (e == E - 1) {
             meta->num_tiles = inc_t;
             meta->padded_rows = poff_next;
+            meta->num_ptiles = inc_p;
             s_poff[E] = poff_next;
         }
     }

@@ -54,7 +54,9 @@ constexpr int A_TILE = BM * BK * 2;    // 16 KB
 constexpr int B_BOX = 64 * BK * 2;     // 8 KB: 64 columns x 64 K rows
 constexpr int B_TILE = BN * BK * 2;    // 32 KB
 constexpr int STAGE = A_TILE + B_TILE; // 48 KB
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 192;      // TMA warp, MMA warp, 4 epilogue warps
+constexpr int GATHER_THREADS = 128;   // 4 more warps that gather layer0 A rows (cp.async)
+constexpr int NUM_THREADS_GATHER = NUM_THREADS + GATHER_THREADS;
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
@@ -71,8 +73,16 @@ enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2 };
 struct GemmArgs {
     const int32_t *tile_off;    // [E+1] first m-tile of each expert
     const int32_t *tile_expert; // [max_tiles] expert of each m-tile
+    const int32_t *ptile_off;   // [E+1] first m-tile pair of each expert (pair kernel)
+    const int32_t *ptile_expert; // expert of each m-tile pair (pair kernel)
     const DispatchMeta *meta;   // num_tiles
     const float *row_w;         // GEMM_SCALE: gate weight of each padded row
+    const int32_t *gather_idx;  // layer0: token of each padded row (-1: pad), A rows are
+                                // gathered from x with it; nullptr: A rows are contiguous
+    int64_t gather_len;         // entries of gather_idx
+    const __nv_bfloat16 *gather_src; // x [gather_rows, gather_ld]
+    int gather_rows;
+    int gather_ld;
     __nv_bfloat16 *out;         // [rows, ld_out]
     int ld_out;                 // elements per output row
     int n_cols;                 // valid output columns
@@ -107,8 +117,74 @@ __device__ __forceinline__ float act_f(int act, float z)
     return z;
 }
 
+// Epilogue of one accumulator tile for the 32 rows of this warp: thread `lane` owns row `row`
+// and reads its TMEM lane `t_row` (already offset to the accumulator buffer). Warp-collective
+// (tcgen05.ld), so the whole warp calls it.
 template <int KIND>
-__global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
+__device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt)
+{
+    using namespace gemm;
+    if (KIND == GEMM_SWIGLU) {
+        __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, g);
+            tmem_ld_32x32b_x32(t_row + 128 + c * 32, u);
+            tmem_ld_wait();
+            if (nt * 128 + c * 32 < args.n_cols) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint32_t p[4];
+#pragma unroll
+                    for (int h2 = 0; h2 < 4; ++h2) {
+                        const int i = v * 8 + h2 * 2;
+                        const float a0 = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+                        const float a1 =
+                            silu_f(__uint_as_float(g[i + 1])) * __uint_as_float(u[i + 1]);
+                        p[h2] = pack_bf16x2(a0, a1);
+                    }
+                    dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
+                }
+            }
+        }
+    } else {
+        __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * BN;
+        const float wt = (KIND == GEMM_SCALE) ? args.row_w[row] : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, r);
+            tmem_ld_wait();
+            if (nt * BN + c * 32 < args.n_cols) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint32_t p[4];
+#pragma unroll
+                    for (int h2 = 0; h2 < 4; ++h2) {
+                        const int i = v * 8 + h2 * 2;
+                        float a0 = __uint_as_float(r[i]);
+                        float a1 = __uint_as_float(r[i + 1]);
+                        if (KIND == GEMM_SCALE) {
+                            a0 *= wt;
+                            a1 *= wt;
+                        } else {
+                            a0 = act_f(args.act, a0);
+                            a1 = act_f(args.act, a1);
+                        }
+                        p[h2] = pack_bf16x2(a0, a1);
+                    }
+                    dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
+                }
+            }
+        }
+    }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     moe_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
 {
@@ -129,9 +205,12 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // layer0 A rows come from the gather warps (cp.async, one arrival per gather thread);
+    // otherwise A is one TMA box like B
+    const bool gather = (args.gather_idx != nullptr);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+            mbar_init(full_bar(s), gather ? 1 + GATHER_THREADS : 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -177,9 +256,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
                     }
                     const uint32_t a_dst = smem_u32(smem + s * STAGE);
                     const uint32_t b_dst = a_dst + A_TILE;
-                    mbar_arrive_expect_tx(full_bar(s), STAGE);
+                    mbar_arrive_expect_tx(full_bar(s), gather ? B_TILE : STAGE);
                     armed[s] = (int)ph;
-                    tma_load_2d(a_dst, &tmA, full_bar(s), kb * BK, mt * BM);
+                    if (!gather) tma_load_2d(a_dst, &tmA, full_bar(s), kb * BK, mt * BM);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         int col;
@@ -195,8 +274,8 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
                     }
                 }
             }
-            // every copy issued must have landed before the CTA exits (immediate when the
-            // MMA warp consumed them all; bounded after an abort)
+            // every TMA copy issued must have landed before the CTA exits (immediate when
+            // the MMA warp consumed them all; bounded after an abort)
             for (int i = 0; i < STAGES; ++i)
                 if (armed[i] >= 0) {
                     volatile int never = 0;
@@ -227,6 +306,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
+                    // the gathered A rows were written through the generic proxy (cp.async);
+                    // order them before the tensor cores read the stage
+                    if (gather) fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * STAGE);
                     const uint32_t b_addr = a_addr + A_TILE;
@@ -253,6 +335,54 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
             volatile int never = 0;
             mbar_wait_bounded(done_bar, 0, &never, args.timeout_ns, args.status, 130 + KIND);
         }
+    } else if (warp >= 6) {
+        // ---------------- A-row gather: warps 6..9 (layer0 only) ----------------
+        // Thread g copies 16-byte chunk (g & 7) of rows (g >> 3) + 16 i, i = 0..7, of every K
+        // step. The 8 token ids of its rows are read once per tile and kept in registers
+        // (Comet §4: row indices cached in registers instead of re-read every K step).
+        // Destinations follow the 128-byte swizzle the MMA descriptor expects.
+        if (gather) {
+            const int g = threadIdx.x - NUM_THREADS;
+            const int chunk = g & 7;
+            const int r0 = g >> 3;
+            int s = 0;
+            uint32_t ph = 0;
+            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+                int e, mt, nt;
+                gemm_map_work(w, args, e, mt, nt);
+                const __nv_bfloat16 *src[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int64_t r = (int64_t)mt * BM + r0 + 16 * i;
+                    int t = (r < args.gather_len) ? args.gather_idx[r] : -1;
+                    if (t < 0 || t >= args.gather_rows) t = 0; // pad rows read token 0; never used
+                    src[i] = args.gather_src + (size_t)t * args.gather_ld + chunk * 8;
+                }
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    ok = mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
+                                           args.status, 150 + KIND);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_u32(smem + s * STAGE);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + 16 * i;
+                        const uint32_t dst = a_dst + r * 128 + ((chunk ^ (r & 7)) << 4);
+                        cp_async_16_cg(dst, src[i] + kb * BK);
+                    }
+                    cp_async_arrive_noinc(full_bar(s));
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+            cp_async_wait_all(); // this thread's copies land before the CTA exits
+        }
     } else {
         // ---------------- epilogue: warps 2..5 ----------------
         const int q = warp & 3; // TMEM lanes 32q .. 32q+31
@@ -269,63 +399,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
             tc_fence_after();
             const int row = mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            if (KIND == GEMM_SWIGLU) {
-                __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * 128;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(t_row + c * 32, g);
-                    tmem_ld_32x32b_x32(t_row + 128 + c * 32, u);
-                    tmem_ld_wait();
-                    if (nt * 128 + c * 32 < args.n_cols) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint32_t p[4];
-#pragma unroll
-                            for (int h2 = 0; h2 < 4; ++h2) {
-                                const int i = v * 8 + h2 * 2;
-                                const float a0 = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-                                const float a1 =
-                                    silu_f(__uint_as_float(g[i + 1])) * __uint_as_float(u[i + 1]);
-                                p[h2] = pack_bf16x2(a0, a1);
-                            }
-                            dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
-                        }
-                    }
-                }
-            } else {
-                __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * BN;
-                const float wt = (KIND == GEMM_SCALE) ? args.row_w[row] : 1.0f;
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + c * 32, r);
-                    tmem_ld_wait();
-                    if (nt * BN + c * 32 < args.n_cols) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint32_t p[4];
-#pragma unroll
-                            for (int h2 = 0; h2 < 4; ++h2) {
-                                const int i = v * 8 + h2 * 2;
-                                float a0 = __uint_as_float(r[i]);
-                                float a1 = __uint_as_float(r[i + 1]);
-                                if (KIND == GEMM_SCALE) {
-                                    a0 *= wt;
-                                    a1 *= wt;
-                                } else {
-                                    a0 = act_f(args.act, a0);
-                                    a1 = act_f(args.act, a1);
-                                }
-                                p[h2] = pack_bf16x2(a0, a1);
-                            }
-                            dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
-                        }
-                    }
-                }
-            }
+            epilogue_rows<KIND>(args, t_row, row, nt);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
@@ -338,6 +412,246 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+
+// ---------------------------------------------------------------------------------------
+// CTA-pair variant: tcgen05.mma.cta_group::2, M = 256 (128 rows per CTA), N = 256.
+// ---------------------------------------------------------------------------------------
+//
+// Two CTAs of a cluster work on one 256-row x 256-column tile: each CTA loads its own 128
+// token rows of A and its own half (128 columns) of the B tile, so per SM the B traffic and
+// the shared-memory bytes per K step drop by a third compared with the single-CTA tile.
+// The leader CTA (cluster rank 0) issues the MMAs for the pair; its "full" barrier counts
+// the bytes of both CTAs' copies. Its commits arrive on both CTAs' "empty" and "tmem full"
+// barriers; both CTAs' epilogue warps release the leader's "tmem empty" barrier. A pair of
+// m-tiles always belongs to one expert; when an expert has an odd number of m-tiles, the
+// second CTA's half of its last pair is computed on rows of no use and not stored.
+// For layer0 (SwiGLU) CTA 0 loads the 128 gate columns and CTA 1 the matching 128 up
+// columns, so each CTA's accumulator holds [gate | up] for its own rows.
+
+namespace gemm2 {
+constexpr int STAGES = 6;
+constexpr int A_TILE = 128 * gemm::BK * 2;   // 16 KB per CTA
+constexpr int B_TILE = 128 * gemm::BK * 2;   // 16 KB per CTA (two 64-column boxes)
+constexpr int STAGE = A_TILE + B_TILE;       // 32 KB per CTA
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16;
+constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, /*b_mn_major=*/true);
+constexpr uint16_t PAIR_MASK = 0x3;
+} // namespace gemm2
+
+__device__ __forceinline__ void gemm_map_pair(int w, const GemmArgs &a, int &e, int &mt0, int &nt)
+{
+    const int q = w / a.n_tiles;
+    e = a.ptile_expert[q];
+    const int base = a.ptile_off[e];
+    const int cnt = a.ptile_off[e + 1] - base;
+    const int local = w - base * a.n_tiles;
+    mt0 = a.tile_off[e] + 2 * (local % cnt);
+    nt = local / cnt;
+}
+
+template <int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm::NUM_THREADS, 1)
+    moe_grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                                 const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+{
+    using gemm::BK;
+    using gemm::B_BOX;
+    using gemm2::STAGES;
+    using gemm2::STAGE;
+    using gemm2::A_TILE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + gemm2::NUM_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank(); // 0: leader, 1: peer
+    const int pair_id = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);  // leader: its own arrive + both CTAs' bytes
+            mbar_init(empty_bar(s), 1); // the leader's multicast commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 8); // leader: 4 epilogue warps of each CTA
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), gemm::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all(); // barriers of both CTAs initialised before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total = args.meta->num_ptiles * args.n_tiles;
+    const int KB = args.k_blocks;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (whole warp, both CTAs) ----------------
+        const bool gather = (args.gather_idx != nullptr);
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true, issued = false;
+        for (int w = pair_id; ok && w < total; w += npairs) {
+            int e, mt0, nt;
+            gemm_map_pair(w, args, e, mt0, nt);
+            const int my_mt = mt0 + (int)rank;
+            int rows[4] = {0, 0, 0, 0};
+            if (gather) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t r = (int64_t)my_mt * 128 + 4 * lane + i;
+                    const int g = (r < args.gather_len) ? args.gather_idx[r] : -1;
+                    rows[i] = g < 0 ? 0 : g;
+                }
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                ok = mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
+                                       args.status, 200 + KIND);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                if (rank == 0 && lane == 0) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE);
+                __syncwarp();
+                const uint32_t leader_full = mapa_shared(full_bar(s), 0);
+                const uint32_t a_dst = smem_u32(smem + s * STAGE);
+                const uint32_t b_dst = a_dst + A_TILE;
+                if (gather) {
+                    tma_gather4_pair(a_dst + lane * 512, &tmA, leader_full, kb * BK, rows[0],
+                                     rows[1], rows[2], rows[3]);
+                } else if (lane == 0) {
+                    tma_load_2d_pair(a_dst, &tmA, leader_full, kb * BK, my_mt * 128);
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        int col;
+                        if (KIND == GEMM_SWIGLU)
+                            col = (rank == 0 ? 0 : args.up_col) + nt * 128 + i * 64;
+                        else
+                            col = nt * gemm::BN + (int)rank * 128 + i * 64;
+                        tma_load_3d_pair(b_dst + i * B_BOX, &tmB, leader_full, col, kb * BK, e);
+                    }
+                }
+                issued = true;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        if (!ok && issued) {
+            // gave up: copies already issued complete on their own; let them land before
+            // the cluster exits (about 100 us)
+            for (int i = 0; i < 100; ++i) __nanosleep(1000);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            if (rank == 0) {
+                // ---------------- MMA issuer (leader only) ----------------
+                int s = 0;
+                uint32_t ph = 0;
+                int it = 0;
+                bool ok = true;
+                for (int w = pair_id; ok && w < total; w += npairs, ++it) {
+                    const int acc = it & 1;
+                    const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                    if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, args.timeout_ns,
+                                           args.status, 210 + KIND)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(acc * gemm::BN);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, args.timeout_ns,
+                                               args.status, 220 + KIND)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(smem + s * STAGE);
+                        const uint32_t b_addr = a_addr + A_TILE;
+                        const uint64_t a_desc = sw128_desc(a_addr, gemm::A_LBO, gemm::A_SBO);
+                        const uint64_t b_desc = sw128_desc(b_addr, gemm::B_LBO, gemm::B_SBO);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            umma_bf16_pair(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                           b_desc + (uint64_t)((k * 16 * 128) >> 4), gemm2::IDESC,
+                                           (kb | k) != 0 ? 1u : 0u);
+                        }
+                        umma_commit_pair(empty_bar(s), gemm2::PAIR_MASK);
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit_pair(tfull_bar(acc), gemm2::PAIR_MASK);
+                }
+                // every MMA issued so far must finish before either CTA releases TMEM
+                umma_commit_pair(done_bar, gemm2::PAIR_MASK);
+            }
+            volatile int never = 0;
+            mbar_wait_bounded(done_bar, 0, &never, args.timeout_ns, args.status, 230 + KIND);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5 of both CTAs ----------------
+        const int q = warp & 3;
+        int it = 0;
+        for (int w = pair_id; w < total; w += npairs, ++it) {
+            int e, mt0, nt;
+            gemm_map_pair(w, args, e, mt0, nt);
+            const int my_mt = mt0 + (int)rank;
+            const bool valid = my_mt < args.tile_off[e + 1];
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            bool ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, args.timeout_ns,
+                                        args.status, 240 + KIND);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            if (valid) {
+                const int row = my_mt * 128 + q * 32 + lane;
+                const uint32_t t_row =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * gemm::BN);
+                epilogue_rows<KIND>(args, t_row, row, nt);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all(); // no CTA leaves while its peer may still signal its barriers
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, gemm::TMEM_COLS);
     }
 }
 

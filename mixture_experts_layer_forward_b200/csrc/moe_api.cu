@@ -21,6 +21,8 @@ using namespace moe;
 
 constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
 std::atomic<int64_t> g_timeout_ns{kDefaultTimeoutNs};
+// grouped GEMM variant: MOE_GEMM_AUTO / MOE_GEMM_SINGLE_CTA / MOE_GEMM_CTA_PAIR
+std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -53,7 +55,8 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
     size_t status, meta, logits, topk_idx, topk_w, chunk, counts, offsets, poff, tile_off,
-        tile_expert, gather_idx, inv_pos, row_w, x_perm, h, ys, x_stage, out_stage;
+        tile_expert, ptile_off, ptile_expert, gather_idx, inv_pos, row_w, x_perm, h, ys, x_stage,
+        out_stage;
     size_t end_route, end_dispatch, end_forward, end_host;
     int64_t pmax;
     int nchunk, max_tiles;
@@ -86,11 +89,13 @@ Layout make_layout(const moe_problem *p)
     L.poff = take((E + 1) * 4);
     L.tile_off = take((E + 1) * 4);
     L.tile_expert = take((size_t)L.max_tiles * 4);
+    L.ptile_off = take((E + 1) * 4);
+    L.ptile_expert = take((size_t)L.max_tiles * 4);
     L.gather_idx = take(P * 4);
     L.inv_pos = take(T * K * 4);
     L.row_w = take(P * 4);
     L.end_dispatch = o;
-    L.x_perm = take(P * H * 2);
+    L.x_perm = take(P * H * 2); // materialised gather, used by the CTA-pair GEMM variant
     L.h = take(P * F * 2);
     L.ys = take(P * H * 2);
     L.end_forward = o;
@@ -225,6 +230,7 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
 
 struct DispatchOut {
     int32_t *counts, *offsets, *poff, *gather_idx, *inv_pos, *tile_off, *tile_expert, *chunk;
+    int32_t *ptile_off, *ptile_expert;
     float *row_w;
     DispatchMeta *meta;
 };
@@ -242,8 +248,9 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, o.counts, o.offsets, o.poff,
-                                             o.tile_off, o.tile_expert, o.meta, o.gather_idx,
-                                             o.row_w, L.pmax);
+                                             o.tile_off, o.tile_expert, o.ptile_off,
+                                             o.ptile_expert, o.meta, o.gather_idx, o.row_w,
+                                             L.pmax);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
@@ -289,8 +296,49 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
     if (grid <= 0) grid = 148;
     if (grid > max_work) grid = max_work;
     if (grid < 1) grid = 1;
-    moe_grouped_gemm_kernel<KIND><<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+    const int threads = args.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    moe_grouped_gemm_kernel<KIND><<<grid, threads, gemm::SMEM_BYTES, st>>>(ta, tb, args);
     return cudaGetLastError();
+}
+
+template <int KIND>
+cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                             int max_work, cudaStream_t st)
+{
+    auto kern = moe_grouped_gemm_pair_kernel<KIND>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    // persistent grid: as many CTA pairs as can be resident at once (one CTA per SM)
+    static int cache[64][3] = {{0}};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int &pairs = cache[dev][KIND];
+    if (pairs == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
+        cfg.blockDim = dim3(gemm::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm2::SMEM_BYTES;
+        int n = 0;
+        err = cudaOccupancyMaxActiveClusters(&n, (const void *)kern, &cfg);
+        if (err != cudaSuccess) return err;
+        pairs = n > 0 ? n : 1;
+    }
+    int npairs = pairs;
+    if (npairs > max_work) npairs = max_work;
+    if (npairs < 1) npairs = 1;
+    kern<<<2 * npairs, gemm::NUM_THREADS, gemm2::SMEM_BYTES, st>>>(ta, tb, args);
+    return cudaGetLastError();
+}
+
+template <int KIND>
+cudaError_t launch_gemm_any(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                            int max_work, cudaStream_t st)
+{
+    // AUTO = single CTA: under the sustained 1 kW power cap the pair variant keeps the tensor
+    // pipe busier per clock but draws more power per clock, and measured ~4% slower overall
+    if (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR) return launch_gemm_pair<KIND>(ta, tb, args, max_work, st);
+    return launch_gemm<KIND>(ta, tb, args, max_work, st);
 }
 
 moe_status to_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -359,6 +407,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     d.tile_off = at<int32_t>(ws, L.tile_off);
     d.tile_expert = at<int32_t>(ws, L.tile_expert);
     d.chunk = at<int32_t>(ws, L.chunk);
+    d.ptile_off = at<int32_t>(ws, L.ptile_off);
+    d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
     d.row_w = at<float>(ws, L.row_w);
     d.meta = at<DispatchMeta>(ws, L.meta);
     moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
@@ -368,7 +418,12 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     const int F = p->F, H = p->H, E = p->E;
     const bool gated = (p->act == MOE_ACT_SWIGLU);
     CUtensorMap m_x, m_w1, m_h, m_w2;
-    if (!make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM) ||
+    // Single-CTA layer0 gathers its A rows straight from x (cp.async gather warps); the
+    // CTA-pair variant reads a materialised x_perm with TMA.
+    const bool pair = (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR);
+    const bool a_ok = pair ? make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM)
+                           : make_map_2d(&m_x, x, (uint64_t)p->T, (uint64_t)H, 1);
+    if (!a_ok ||
         !make_map_3d(&m_w1, W1, (uint64_t)E, (uint64_t)H, (uint64_t)(gated ? 2 * F : F)) ||
         !make_map_2d(&m_h, h, (uint64_t)L.pmax, (uint64_t)F, gemm::BM) ||
         !make_map_3d(&m_w2, W2, (uint64_t)E, (uint64_t)F, (uint64_t)H))
@@ -380,14 +435,21 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st);
     if (e == cudaSuccess) e = record(events, n_events, 1, st);
     if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
-    if (e == cudaSuccess) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
+    if (e == cudaSuccess && pair) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
     if (e == cudaSuccess) e = record(events, n_events, 2, st);
 
     GemmArgs a0{};
     a0.tile_off = d.tile_off;
     a0.tile_expert = d.tile_expert;
+    a0.ptile_off = d.ptile_off;
+    a0.ptile_expert = d.ptile_expert;
     a0.meta = d.meta;
     a0.row_w = nullptr;
+    a0.gather_idx = pair ? nullptr : d.gather_idx;
+    a0.gather_len = L.pmax;
+    a0.gather_src = reinterpret_cast<const __nv_bfloat16 *>(x);
+    a0.gather_rows = p->T;
+    a0.gather_ld = H;
     a0.out = reinterpret_cast<__nv_bfloat16 *>(h);
     a0.ld_out = F;
     a0.n_cols = F;
@@ -399,21 +461,22 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     if (gated) {
         a0.n_tiles = (F + 127) / 128;
         if (e == cudaSuccess)
-            e = launch_gemm<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+            e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
     } else {
         a0.n_tiles = (F + gemm::BN - 1) / gemm::BN;
-        if (e == cudaSuccess) e = launch_gemm<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+        if (e == cudaSuccess) e = launch_gemm_any<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
     }
     if (e == cudaSuccess) e = record(events, n_events, 3, st);
 
     GemmArgs a1 = a0;
+    a1.gather_idx = nullptr; // layer1 reads h rows in place
     a1.row_w = d.row_w;
     a1.out = reinterpret_cast<__nv_bfloat16 *>(ys);
     a1.ld_out = H;
     a1.n_cols = H;
     a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
     a1.k_blocks = F / gemm::BK;
-    if (e == cudaSuccess) e = launch_gemm<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
+    if (e == cudaSuccess) e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
     if (e == cudaSuccess) e = record(events, n_events, 4, st);
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);
@@ -505,6 +568,8 @@ moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *
     d.tile_off = at<int32_t>(ws, L.tile_off);
     d.tile_expert = at<int32_t>(ws, L.tile_expert);
     d.chunk = at<int32_t>(ws, L.chunk);
+    d.ptile_off = at<int32_t>(ws, L.ptile_off);
+    d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
     d.row_w = nullptr;
     d.meta = at<DispatchMeta>(ws, L.meta);
     if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, nullptr, d, status, 1, st);
@@ -607,6 +672,12 @@ const char *moe_status_string(moe_status s)
 int64_t moe_set_wait_timeout_ns(int64_t ns)
 {
     return g_timeout_ns.exchange(ns > 0 ? ns : kDefaultTimeoutNs);
+}
+
+int moe_set_gemm_mode(int mode)
+{
+    if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_SINGLE_CTA && mode != MOE_GEMM_CTA_PAIR) return -1;
+    return g_gemm_mode.exchange(mode);
 }
 
 } // extern "C"

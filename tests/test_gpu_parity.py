@@ -241,8 +241,15 @@ FWD_CASES = [
 ]
 
 
+@pytest.fixture(params=[moe.GEMM_CTA_PAIR, moe.GEMM_SINGLE_CTA], ids=["cta_pair", "single_cta"])
+def gemm_mode(request):
+    prev = moe.moe_set_gemm_mode(request.param)
+    yield request.param
+    moe.moe_set_gemm_mode(prev)
+
+
 @pytest.mark.parametrize("cfg", FWD_CASES, ids=[c.name for c in FWD_CASES])
-def test_forward_matches_oracle(cfg):
+def test_forward_matches_oracle(cfg, gemm_mode):
     inp = synth.make_inputs(cfg, seed=11)
     out, idx, w, ws = run_forward(cfg, inp)
     b = None if inp["bias"] is None else inp["bias"].numpy()
@@ -253,6 +260,21 @@ def test_forward_matches_oracle(cfg):
     assert_out_close(out, ref, cfg.name)
     out2, _, _, _ = run_forward(cfg, inp, ws)
     assert torch.equal(out, out2), "two identical calls differ"
+
+
+def test_gemm_variants_agree():
+    """The single-CTA and CTA-pair grouped GEMMs compute the same layer."""
+    cfg = cfg_small("variants", 700, 512, 640, 8, 2)
+    inp = synth.make_inputs(cfg, seed=14)
+    prev = moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)
+    try:
+        a, _, _, _ = run_forward(cfg, inp)
+        moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)
+        b, _, _, _ = run_forward(cfg, inp)
+    finally:
+        moe.moe_set_gemm_mode(prev)
+    d = (a.float() - b.float()).abs()
+    assert float(d.max()) <= 2e-2 + 2e-2 * float(a.float().abs().max())
 
 
 def test_forward_all_tokens_on_one_expert():
