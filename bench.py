@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--H", type=int, default=None)
     ap.add_argument("--F", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--gemm-mode", choices=["auto", "single", "pair"], default="auto",
+    ap.add_argument("--gemm-mode", choices=["auto", "single", "pair", "fused"], default="auto",
                     help="grouped-GEMM variant (moe_set_gemm_mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -300,7 +300,7 @@ def run_ours(args):
     cfg = workload(args)
     K, W = args.steps, max(3, args.warmup)
     moe.moe_set_gemm_mode({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE_CTA,
-                           "pair": moe.GEMM_CTA_PAIR}[args.gemm_mode])
+                           "pair": moe.GEMM_CTA_PAIR, "fused": moe.GEMM_FUSED}[args.gemm_mode])
 
     inp = synth.make_inputs(cfg, seed=args.seed, device=dev,
                             x_seed=dp.replica_x_seed(args.seed, rank) if world > 1 else None)

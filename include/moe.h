@@ -222,7 +222,20 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
 #define MOE_GEMM_AUTO 0
 #define MOE_GEMM_SINGLE_CTA 1
 #define MOE_GEMM_CTA_PAIR 2
+/* MOE_GEMM_FUSED: layer0, layer1 and the combine in one persistent launch, scheduled by
+ * tile-level ready flags (a layer1 tile starts when layer0 has finished its 128 h rows; a
+ * combine stripe starts when layer1 has finished that 256-column stripe of every tile).
+ * Stage events 3..5 of moe_forward_staged then all mark the end of that one launch. */
+#define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
+
+/* Test hook for the bounded ready-flag waits of MOE_GEMM_FUSED: the layer0 work item with
+ * this index (in the kernel's static work queue) withholds its ready signal, so the layer1
+ * tiles that need it wait until the timeout (moe_set_wait_timeout_ns) and the call reports
+ * MOE_ERR_DEVICE_TIMEOUT through moe_get_device_status. Nothing faults or hangs: every CTA
+ * leaves within a few timeouts and the context stays usable. -1 switches it off (default).
+ * Returns the previous value. Not thread-safe; meant for tests. */
+MOE_API int moe_set_fault_injection(int layer0_item);
 
 #ifdef __cplusplus
 }

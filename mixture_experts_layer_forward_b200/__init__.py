@@ -33,6 +33,8 @@ from ._native import (  # noqa: F401
     moe_set_gemm_mode,
     moe_set_wait_timeout_ns,
     GEMM_AUTO,
+    GEMM_FUSED,
+    moe_set_fault_injection,
     GEMM_CTA_PAIR,
     GEMM_SINGLE_CTA,
     moe_workspace_size,

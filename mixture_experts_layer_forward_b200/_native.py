@@ -87,6 +87,7 @@ def library() -> ctypes.CDLL:
             "moe_status_string": ([i32], ctypes.c_char_p),
             "moe_set_wait_timeout_ns": ([i64], i64),
             "moe_set_gemm_mode": ([i32], i32),
+            "moe_set_fault_injection": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -241,7 +242,12 @@ def moe_set_wait_timeout_ns(ns: int) -> int:
     return int(library().moe_set_wait_timeout_ns(int(ns)))
 
 
-GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR = 0, 1, 2
+GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED = 0, 1, 2, 3
+
+
+def moe_set_fault_injection(layer0_item: int) -> int:
+    """Test hook: withhold the ready signal of one layer0 work item of the fused kernel."""
+    return int(library().moe_set_fault_injection(int(layer0_item)))
 
 
 def moe_set_gemm_mode(mode: int) -> int:

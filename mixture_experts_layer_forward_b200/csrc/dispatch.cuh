@@ -99,8 +99,10 @@ __global__ void __launch_bounds__(1024)
                          int32_t *__restrict__ tile_expert, int32_t *__restrict__ ptile_off,
                          int32_t *__restrict__ ptile_expert, DispatchMeta *meta,
                          int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
-                         int64_t padded_rows_max)
+                         int64_t padded_rows_max, int *__restrict__ ready, int n_ready)
 {
+    // the fused layer kernel's tile-level ready counters start from zero on every call
+    for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
     __shared__ int warp_sums[32];
     __shared__ int s_poff[1025];
     const int e = threadIdx.x;

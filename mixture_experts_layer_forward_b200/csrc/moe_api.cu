@@ -11,6 +11,7 @@
 
 #include "combine.cuh"
 #include "dispatch.cuh"
+#include "fused.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
@@ -23,6 +24,8 @@ constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
 std::atomic<int64_t> g_timeout_ns{kDefaultTimeoutNs};
 // grouped GEMM variant: MOE_GEMM_AUTO / MOE_GEMM_SINGLE_CTA / MOE_GEMM_CTA_PAIR
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
+// test hook: layer0 work item of the fused kernel whose ready signal is withheld (-1: none)
+std::atomic<int> g_fault_skip{-1};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -55,11 +58,11 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
     size_t status, meta, logits, topk_idx, topk_w, chunk, counts, offsets, poff, tile_off,
-        tile_expert, ptile_off, ptile_expert, gather_idx, inv_pos, row_w, x_perm, h, ys, x_stage,
-        out_stage;
+        tile_expert, ptile_off, ptile_expert, ready, gather_idx, inv_pos, row_w, x_perm, h, ys,
+        x_stage, out_stage;
     size_t end_route, end_dispatch, end_forward, end_host;
     int64_t pmax;
-    int nchunk, max_tiles;
+    int nchunk, max_tiles, n_ready;
 };
 
 Layout make_layout(const moe_problem *p)
@@ -91,6 +94,8 @@ Layout make_layout(const moe_problem *p)
     L.tile_expert = take((size_t)L.max_tiles * 4);
     L.ptile_off = take((E + 1) * 4);
     L.ptile_expert = take((size_t)L.max_tiles * 4);
+    L.n_ready = L.max_tiles + (int)((H + 255) / 256); // fused kernel: per M tile, per stripe
+    L.ready = take((size_t)L.n_ready * 4);
     L.gather_idx = take(P * 4);
     L.inv_pos = take(T * K * 4);
     L.row_w = take(P * 4);
@@ -231,6 +236,8 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
 struct DispatchOut {
     int32_t *counts, *offsets, *poff, *gather_idx, *inv_pos, *tile_off, *tile_expert, *chunk;
     int32_t *ptile_off, *ptile_expert;
+    int *ready;
+    int n_ready;
     float *row_w;
     DispatchMeta *meta;
 };
@@ -250,7 +257,7 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, o.counts, o.offsets, o.poff,
                                              o.tile_off, o.tile_expert, o.ptile_off,
                                              o.ptile_expert, o.meta, o.gather_idx, o.row_w,
-                                             L.pmax);
+                                             L.pmax, o.ready, o.ready ? o.n_ready : 0);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
@@ -341,6 +348,23 @@ cudaError_t launch_gemm_any(const CUtensorMap &ta, const CUtensorMap &tb, const 
     return launch_gemm<KIND>(ta, tb, args, max_work, st);
 }
 
+template <int KIND0>
+cudaError_t launch_fused(const CUtensorMap &w1, const CUtensorMap &hm, const CUtensorMap &w2,
+                         const FusedArgs &fa, int max_work, cudaStream_t st)
+{
+    auto kern = moe_fused_layer_kernel<KIND0>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    // every CTA must be resident at once (the ready-flag waits rely on it): one per SM
+    int grid = sm_count();
+    if (grid <= 0) grid = 148;
+    if (grid > max_work) grid = max_work;
+    if (grid < 1) grid = 1;
+    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(w1, hm, w2, fa);
+    return cudaGetLastError();
+}
+
 moe_status to_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Fixed logits scratch of moe_route_noalloc: one copy per GPU that loads the library, held
@@ -409,6 +433,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     d.chunk = at<int32_t>(ws, L.chunk);
     d.ptile_off = at<int32_t>(ws, L.ptile_off);
     d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
+    d.ready = at<int>(ws, L.ready);
+    d.n_ready = L.n_ready;
     d.row_w = at<float>(ws, L.row_w);
     d.meta = at<DispatchMeta>(ws, L.meta);
     moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
@@ -458,16 +484,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a0.act = p->act;
     a0.status = status;
     a0.timeout_ns = timeout;
-    if (gated) {
-        a0.n_tiles = (F + 127) / 128;
-        if (e == cudaSuccess)
-            e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
-    } else {
-        a0.n_tiles = (F + gemm::BN - 1) / gemm::BN;
-        if (e == cudaSuccess) e = launch_gemm_any<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
-    }
-    if (e == cudaSuccess) e = record(events, n_events, 3, st);
-
+    a0.n_tiles = gated ? (F + 127) / 128 : (F + gemm::BN - 1) / gemm::BN;
     GemmArgs a1 = a0;
     a1.gather_idx = nullptr; // layer1 reads h rows in place
     a1.row_w = d.row_w;
@@ -476,6 +493,39 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a1.n_cols = H;
     a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
     a1.k_blocks = F / gemm::BK;
+
+    if (g_gemm_mode.load() == MOE_GEMM_FUSED) {
+        // one persistent launch: layer0 -> layer1 -> combine, tile-level ready flags
+        FusedArgs fa{};
+        fa.l0 = a0;
+        fa.l1 = a1;
+        fa.ready0 = d.ready;
+        fa.ready1 = d.ready + L.max_tiles;
+        fa.inv_pos = d.inv_pos;
+        fa.out = reinterpret_cast<__nv_bfloat16 *>(out);
+        fa.T = p->T;
+        fa.H = H;
+        fa.k = p->top_k;
+        fa.ys_rows = L.pmax;
+        fa.fault_skip = g_fault_skip.load();
+        const int max_work = L.max_tiles * (a0.n_tiles + a1.n_tiles) +
+                             a1.n_tiles * ((p->T + COMBINE_TOKENS - 1) / COMBINE_TOKENS);
+        if (e == cudaSuccess) {
+            e = gated ? launch_fused<GEMM_SWIGLU>(m_w1, m_h, m_w2, fa, max_work, st)
+                      : launch_fused<GEMM_ACT>(m_w1, m_h, m_w2, fa, max_work, st);
+        }
+        // the three stages share one launch: their boundaries coincide at its end
+        for (int i = 3; i < 6 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+        return to_status(e);
+    }
+
+    if (gated) {
+        if (e == cudaSuccess)
+            e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+    } else {
+        if (e == cudaSuccess) e = launch_gemm_any<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+    }
+    if (e == cudaSuccess) e = record(events, n_events, 3, st);
     if (e == cudaSuccess) e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
     if (e == cudaSuccess) e = record(events, n_events, 4, st);
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st);
@@ -570,6 +620,8 @@ moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *
     d.chunk = at<int32_t>(ws, L.chunk);
     d.ptile_off = at<int32_t>(ws, L.ptile_off);
     d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
+    d.ready = nullptr;
+    d.n_ready = 0;
     d.row_w = nullptr;
     d.meta = at<DispatchMeta>(ws, L.meta);
     if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, nullptr, d, status, 1, st);
@@ -676,8 +728,15 @@ int64_t moe_set_wait_timeout_ns(int64_t ns)
 
 int moe_set_gemm_mode(int mode)
 {
-    if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_SINGLE_CTA && mode != MOE_GEMM_CTA_PAIR) return -1;
+    if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_SINGLE_CTA && mode != MOE_GEMM_CTA_PAIR &&
+        mode != MOE_GEMM_FUSED)
+        return -1;
     return g_gemm_mode.exchange(mode);
+}
+
+int moe_set_fault_injection(int layer0_item)
+{
+    return g_fault_skip.exchange(layer0_item < 0 ? -1 : layer0_item);
 }
 
 } // extern "C"

@@ -241,7 +241,8 @@ FWD_CASES = [
 ]
 
 
-@pytest.fixture(params=[moe.GEMM_CTA_PAIR, moe.GEMM_SINGLE_CTA], ids=["cta_pair", "single_cta"])
+@pytest.fixture(params=[moe.GEMM_CTA_PAIR, moe.GEMM_SINGLE_CTA, moe.GEMM_FUSED],
+                ids=["cta_pair", "single_cta", "fused"])
 def gemm_mode(request):
     prev = moe.moe_set_gemm_mode(request.param)
     yield request.param
@@ -269,12 +270,13 @@ def test_gemm_variants_agree():
     prev = moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)
     try:
         a, _, _, _ = run_forward(cfg, inp)
-        moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)
-        b, _, _, _ = run_forward(cfg, inp)
+        for mode in (moe.GEMM_CTA_PAIR, moe.GEMM_FUSED):
+            moe.moe_set_gemm_mode(mode)
+            b, _, _, _ = run_forward(cfg, inp)
+            d = (a.float() - b.float()).abs()
+            assert float(d.max()) <= 2e-2 + 2e-2 * float(a.float().abs().max()), mode
     finally:
         moe.moe_set_gemm_mode(prev)
-    d = (a.float() - b.float()).abs()
-    assert float(d.max()) <= 2e-2 + 2e-2 * float(a.float().abs().max())
 
 
 def test_forward_all_tokens_on_one_expert():
@@ -319,7 +321,7 @@ FULL = ["mixtral", "phi35", "qwen2", "skew", "skew_decode"]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_config(name):
+def test_full_size_config(name, gemm_mode):
     cfg = synth.CONFIGS[name]
     inp = synth.make_inputs(cfg, seed=0, device="cuda")
     out, idx, w, ws = run_forward(cfg, inp)
