@@ -220,7 +220,7 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
         launch_route_logits<ROUTE_SMALL_CFG>(xb, wb, bias, logits, T, H, E, status, st);
     } else if (E > 8 && E <= 16 && T >= 32 * sms / 2) {
         launch_route_logits<ROUTE_MID_CFG>(xb, wb, bias, logits, T, H, E, status, st);
-    } else if (E > 16 && large_blocks >= sms) {
+    } else if (E > 16 && large_blocks >= sms / 2) {
         launch_route_logits<ROUTE_LARGE_CFG>(xb, wb, bias, logits, T, H, E, status, st);
     } else {
         launch_route_logits<ROUTE_NARROW_CFG>(xb, wb, bias, logits, T, H, E, status, st);
