@@ -34,7 +34,6 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 8  # route logits, top-k, count, scan, place, layer0 (gathers x), layer1, combine
 DOMINANT_KERNEL = "moe_grouped_gemm_kernel<0>"  # layer0 grouped GEMM + SwiGLU
 
 
@@ -402,7 +401,7 @@ def run_ours(args):
                            "peak_source": f"{peak_src} bf16 {regime}"},
         "roofline": roofline,
         "stage_ms": stage_ms,
-        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "gpu_launches": moe.moe_forward_launches(p) * K,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -100,6 +100,13 @@ typedef struct {
  * calls on one stream. 0 if *p is invalid. */
 MOE_API size_t moe_workspace_size(const moe_problem *p);
 
+/* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
+ * current GEMM and router modes, assuming 16-byte aligned operands: the router (2, or 3
+ * with the tensor-core filter), the dispatch (3) and the layers (3: layer0, layer1 and the
+ * combine; 4 with the CTA-pair GEMM, which first gathers x; 1 with MOE_GEMM_FUSED).
+ * 0 for T == 0; -1 if *p is invalid. */
+MOE_API int moe_forward_launches(const moe_problem *p);
+
 /* Upper bound on the padded row count P_pad = sum_e ceil(c_e / m_tile) * m_tile, namely
  * T*top_k + min(E, T*top_k) * (m_tile - 1). gather_idx and ys buffers are sized with it,
  * so no host read of the expert counts is ever needed. -1 if *p is invalid. */
@@ -228,6 +235,22 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
  * Stage events 3..5 of moe_forward_staged then all mark the end of that one launch. */
 #define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
+
+/* Router variant (a tuning and test hook; not thread-safe). All give the same routing and
+ * gates (the selection is always made on the sequential fp32 logits, see moe_route):
+ * MOE_ROUTER_FILTER: for 16 < E <= 512 with E % 8 == 0, MOE_GATE_SOFTMAX_TOPK and 16-byte
+ *   aligned x and Wg, the logits are first computed on the tensor cores; every expert whose
+ *   logit interval (a rigorous bound on the difference between the two fp32 sums) cannot
+ *   reach the top k is dropped, and only the rest get the sequential fp32 logit (other
+ *   problems use the sequential router);
+ * MOE_ROUTER_SEQUENTIAL: every (token, expert) logit is computed sequentially;
+ * MOE_ROUTER_AUTO (default): the filter where it applies and T * E >= 2^16, else sequential.
+ * moe_route_noalloc always uses the sequential router.
+ * Returns the previous mode, or -1 for an unknown mode. */
+#define MOE_ROUTER_AUTO 0
+#define MOE_ROUTER_SEQUENTIAL 1
+#define MOE_ROUTER_FILTER 2
+MOE_API int moe_set_router_mode(int mode);
 
 /* Test hook for the bounded ready-flag waits of MOE_GEMM_FUSED: the layer0 work item with
  * this index (in the kernel's static work queue) withholds its ready signal, so the layer1

@@ -25,12 +25,17 @@ from ._native import (  # noqa: F401
     moe_dispatch,
     moe_forward,
     moe_forward_host,
+    moe_forward_launches,
     moe_forward_staged,
     moe_get_device_status,
     moe_padded_rows_max,
     moe_route,
     moe_route_noalloc,
     moe_set_gemm_mode,
+    moe_set_router_mode,
+    ROUTER_AUTO,
+    ROUTER_SEQUENTIAL,
+    ROUTER_FILTER,
     moe_set_wait_timeout_ns,
     GEMM_AUTO,
     GEMM_FUSED,

@@ -74,6 +74,7 @@ def library() -> ctypes.CDLL:
         P = ctypes.POINTER(Problem)
         sig = {
             "moe_workspace_size": ([P], sz),
+            "moe_forward_launches": ([P], i32),
             "moe_padded_rows_max": ([P], i64),
             "moe_route": ([P, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_route_noalloc": ([P, vp, vp, vp, vp, vp, vp], i32),
@@ -88,6 +89,7 @@ def library() -> ctypes.CDLL:
             "moe_set_wait_timeout_ns": ([i64], i64),
             "moe_set_gemm_mode": ([i32], i32),
             "moe_set_fault_injection": ([i32], i32),
+            "moe_set_router_mode": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -140,6 +142,11 @@ def _ws(ws):
 
 def moe_workspace_size(p: Problem) -> int:
     return int(library().moe_workspace_size(ctypes.byref(p)))
+
+
+def moe_forward_launches(p: Problem) -> int:
+    """Kernels one moe_forward call on p launches under the current GEMM and router modes."""
+    return int(library().moe_forward_launches(ctypes.byref(p)))
 
 
 def moe_padded_rows_max(p: Problem) -> int:
@@ -243,11 +250,21 @@ def moe_set_wait_timeout_ns(ns: int) -> int:
 
 
 GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED = 0, 1, 2, 3
+ROUTER_AUTO, ROUTER_SEQUENTIAL, ROUTER_FILTER = 0, 1, 2
 
 
 def moe_set_fault_injection(layer0_item: int) -> int:
     """Test hook: withhold the ready signal of one layer0 work item of the fused kernel."""
     return int(library().moe_set_fault_injection(int(layer0_item)))
+
+
+def moe_set_router_mode(mode: int) -> int:
+    """Select the router variant for many experts (ROUTER_AUTO, ROUTER_SEQUENTIAL or
+    ROUTER_FILTER); returns the previous mode. All give the same routing and gates."""
+    rc = int(library().moe_set_router_mode(int(mode)))
+    if rc < 0:
+        raise ValueError(f"unknown router mode {mode}")
+    return rc
 
 
 def moe_set_gemm_mode(mode: int) -> int:

@@ -68,7 +68,7 @@ constexpr uint32_t B_SBO = 1024; // 8 K rows x 128 B
 constexpr uint32_t B_LBO = B_BOX; // next 64-column block
 } // namespace gemm
 
-enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2 };
+enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2, GEMM_LOGITS = 3 };
 
 struct GemmArgs {
     const int32_t *tile_off;    // [E+1] first m-tile of each expert
@@ -92,10 +92,31 @@ struct GemmArgs {
     int act;                    // GEMM_ACT: 1 gelu-tanh, 2 relu, 3 identity
     int *status;
     int64_t timeout_ns;
+    // GEMM_LOGITS (router filter): one dense operand A [dense_rows, K] in dense_m_tiles
+    // 128-row tiles, N = 64 * n_boxes columns per tile (n_boxes <= 4); K is split into
+    // k_split contiguous ranges of k-blocks and split s writes its fp32 partial product
+    // column-major: out_f32[(s * n_cols + col) * dense_rows + row]
+    int dense_m_tiles;
+    int dense_rows;
+    int k_split;
+    int n_boxes;
+    float *out_f32;
+    float *xsq_f32; // optional: sum of squares of every A row over each split's K range,
+                    // [k_split, dense_rows] (the epilogue warps read the staged A tiles)
 };
 
-__device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt)
+__device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
+                                              int &ks)
 {
+    ks = 0;
+    if (a.dense_m_tiles > 0) { // one operand, no expert groups; m fastest, then n, then split
+        e = 0;
+        mt = w % a.dense_m_tiles;
+        const int r = w / a.dense_m_tiles;
+        nt = r % a.n_tiles;
+        ks = r / a.n_tiles;
+        return;
+    }
     const int q = w / a.n_tiles;
     e = a.tile_expert[q];
     const int base = a.tile_off[e];
@@ -103,6 +124,12 @@ __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, 
     const int local = w - base * a.n_tiles;
     mt = base + local % cnt;
     nt = local / cnt;
+}
+
+__device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt)
+{
+    int ks;
+    gemm_map_work(w, a, e, mt, nt, ks);
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
@@ -121,7 +148,8 @@ __device__ __forceinline__ float act_f(int act, float z)
 // and reads its TMEM lane `t_row` (already offset to the accumulator buffer). Warp-collective
 // (tcgen05.ld), so the whole warp calls it.
 template <int KIND>
-__device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt)
+__device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt,
+                                              int ks = 0)
 {
     using namespace gemm;
     if (KIND == GEMM_SWIGLU) {
@@ -146,6 +174,23 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
                         p[h2] = pack_bf16x2(a0, a1);
                     }
                     dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
+                }
+            }
+        }
+    } else if (KIND == GEMM_LOGITS) {
+        // column-major partials: the 32 lanes (consecutive rows) store 128 contiguous bytes
+        const int nc = args.n_boxes * 2;
+        float *out = args.out_f32 + (size_t)ks * args.n_cols * args.dense_rows + row;
+#pragma unroll 1
+        for (int c = 0; c < nc; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, r);
+            tmem_ld_wait();
+            if (row < args.dense_rows) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int col = nt * BN + c * 32 + i;
+                    if (col < args.n_cols) out[(size_t)col * args.dense_rows] = __uint_as_float(r[i]);
                 }
             }
         }
@@ -208,10 +253,12 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     // layer0 A rows come from the gather warps (cp.async, one arrival per gather thread);
     // otherwise A is one TMA box like B
     const bool gather = (args.gather_idx != nullptr);
+    // router filter: the four epilogue warps also read every staged A tile (row norms)
+    const bool row_sq = (KIND == GEMM_LOGITS) && args.xsq_f32 != nullptr;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), gather ? 1 + GATHER_THREADS : 1);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(empty_bar(s), row_sq ? 5 : 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
@@ -232,9 +279,15 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_tiles = args.meta->num_tiles;
-    const int total = num_tiles * args.n_tiles;
+    const int num_tiles = args.dense_m_tiles > 0 ? args.dense_m_tiles : args.meta->num_tiles;
+    const int n_split = (args.dense_m_tiles > 0 && args.k_split > 1) ? args.k_split : 1;
+    const int total = num_tiles * args.n_tiles * n_split;
     const int KB = args.k_blocks;
+    // k-blocks [kb_lo(ks), kb_lo(ks + 1)) belong to split ks (n_split <= KB: none is empty)
+    auto kb_lo = [&](int ks) { return (int)(((int64_t)ks * KB) / n_split); };
+    // B boxes of 64 columns per k-block; the router filter narrows N to what E needs
+    const int nbox = (KIND == GEMM_LOGITS && args.n_boxes >= 1 && args.n_boxes < 4) ? args.n_boxes : 4;
+    const uint32_t idesc = (nbox == 4) ? IDESC : idesc_bf16_f32(BM, nbox * 64, /*b_mn_major=*/true);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -246,9 +299,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             for (int i = 0; i < STAGES; ++i) armed[i] = -1;
             bool ok = true;
             for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-                int e, mt, nt;
-                gemm_map_work(w, args, e, mt, nt);
-                for (int kb = 0; kb < KB; ++kb) {
+                int e, mt, nt, ks;
+                gemm_map_work(w, args, e, mt, nt, ks);
+                for (int kb = kb_lo(ks); kb < kb_lo(ks + 1); ++kb) {
                     if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
                                            args.status, 100 + KIND)) {
                         ok = false;
@@ -256,11 +309,10 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                     }
                     const uint32_t a_dst = smem_u32(smem + s * STAGE);
                     const uint32_t b_dst = a_dst + A_TILE;
-                    mbar_arrive_expect_tx(full_bar(s), gather ? B_TILE : STAGE);
+                    mbar_arrive_expect_tx(full_bar(s), (gather ? 0 : A_TILE) + nbox * B_BOX);
                     armed[s] = (int)ph;
                     if (!gather) tma_load_2d(a_dst, &tmA, full_bar(s), kb * BK, mt * BM);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < nbox; ++i) {
                         int col;
                         if (KIND == GEMM_SWIGLU)
                             col = (i < 2 ? nt * 128 + i * 64 : args.up_col + nt * 128 + (i - 2) * 64);
@@ -300,7 +352,13 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < KB; ++kb) {
+                int ks = 0;
+                if (n_split > 1) {
+                    int e_, mt_, nt_;
+                    gemm_map_work(w, args, e_, mt_, nt_, ks);
+                }
+                const int kb_first = kb_lo(ks);
+                for (int kb = kb_first; kb < kb_lo(ks + 1); ++kb) {
                     if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, args.timeout_ns, args.status,
                                            120 + KIND)) {
                         ok = false;
@@ -318,8 +376,8 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                     for (int k = 0; k < BK / 16; ++k) {
                         // A: +32 B per K=16 step inside the swizzle atom; B: +16 rows x 128 B
                         umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
-                                  b_desc + (uint64_t)((k * 16 * 128) >> 4), IDESC,
-                                  (kb | k) != 0 ? 1u : 0u);
+                                  b_desc + (uint64_t)((k * 16 * 128) >> 4), idesc,
+                                  (kb != kb_first || k != 0) ? 1u : 0u);
                     }
                     umma_commit(empty_bar(s));
                     if (++s == STAGES) {
@@ -359,7 +417,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                     src[i] = args.gather_src + (size_t)t * args.gather_ld + chunk * 8;
                 }
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = 0; kb < KB; ++kb) { // layer0 only: never split
                     ok = mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
                                            args.status, 150 + KIND);
                     if (!__all_sync(0xffffffffu, ok)) {
@@ -387,9 +445,46 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         // ---------------- epilogue: warps 2..5 ----------------
         const int q = warp & 3; // TMEM lanes 32q .. 32q+31
         int it = 0;
+        int rs = 0;             // stage ring position (row_sq only)
+        uint32_t rph = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-            int e, mt, nt;
-            gemm_map_work(w, args, e, mt, nt);
+            int e, mt, nt, ks;
+            gemm_map_work(w, args, e, mt, nt, ks);
+            if (row_sq) {
+                // sum of squares of this thread's A row over the item's k-blocks (the order of
+                // the 16-byte pieces does not matter; lane-rotated reads avoid bank conflicts)
+                float ss = 0.0f;
+                bool ok = true;
+                for (int kb = kb_lo(ks); kb < kb_lo(ks + 1); ++kb) {
+                    ok = mbar_wait_bounded(full_bar(rs), rph, abort_flag, args.timeout_ns,
+                                           args.status, 160 + KIND);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *arow = smem + rs * STAGE + (q * 32 + lane) * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(arow + (((j + lane) & 7) << 4));
+                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            ss = fmaf(bf16_lo(w4[i]), bf16_lo(w4[i]), ss);
+                            ss = fmaf(bf16_hi(w4[i]), bf16_hi(w4[i]), ss);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(rs));
+                    if (++rs == STAGES) {
+                        rs = 0;
+                        rph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                const int row = mt * BM + q * 32 + lane;
+                if (nt == 0 && row < args.dense_rows)
+                    args.xsq_f32[(size_t)ks * args.dense_rows + row] = ss;
+            }
             const int acc = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             bool ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, args.timeout_ns,
@@ -399,7 +494,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             tc_fence_after();
             const int row = mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            epilogue_rows<KIND>(args, t_row, row, nt);
+            epilogue_rows<KIND>(args, t_row, row, nt, ks);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));

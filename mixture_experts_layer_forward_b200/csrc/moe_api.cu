@@ -15,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
+#include "route_filter.cuh"
 
 namespace {
 
@@ -26,6 +27,8 @@ std::atomic<int64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 // test hook: layer0 work item of the fused kernel whose ready signal is withheld (-1: none)
 std::atomic<int> g_fault_skip{-1};
+// router variant for many experts: MOE_ROUTER_AUTO (tensor-core filter) or sequential only
+std::atomic<int> g_router_mode{MOE_ROUTER_AUTO};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -57,13 +60,66 @@ int64_t padded_rows_max(const moe_problem *p)
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, meta, logits, topk_idx, topk_w, chunk, counts, offsets, poff, tile_off,
+    size_t status, meta, logits, wgt, wnorm, xsq, topk_idx, topk_w, chunk,
+        counts, offsets, poff, tile_off,
         tile_expert, ptile_off, ptile_expert, ready, gather_idx, inv_pos, row_w, x_perm, h, ys,
         x_stage, out_stage;
     size_t end_route, end_dispatch, end_forward, end_host;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
 };
+
+// Tensor-core filter router (route_filter.cuh): applicable shapes and launch plan. The plan
+// depends on the problem only, so the workspace size does not depend on the device.
+struct FilterPlan {
+    bool ok;
+    int split;      // K ranges of the filter GEMM (fp32 partials [split, E, T])
+    int bt;         // tokens per block of the exact kernel
+    int ring_bytes; // its chunk ring
+    size_t smem;    // its dynamic shared memory
+    float cA;       // interval coefficient
+};
+
+FilterPlan filter_plan(const moe_problem *p)
+{
+    FilterPlan f{false, 1, 0, 0, 0, 0.0f};
+    const int T = p->T, H = p->H, E = p->E;
+    if (T <= 0 || E <= 16 || E > RF_MAX_E || (E % 8) != 0 || (H % gemm::BK) != 0 ||
+        p->gate != MOE_GATE_SOFTMAX_TOPK || (int64_t)T * E >= (1LL << 31) / RF_SPLIT_MAX)
+        return f;
+    const int kb = H / gemm::BK;
+    const int tiles = ((T + gemm::BM - 1) / gemm::BM) * ((E + gemm::BN - 1) / gemm::BN);
+    int split = 148 / tiles; // about one wave of filter-GEMM CTAs on a 148-SM part
+    const int smax = kb < RF_SPLIT_MAX ? kb : RF_SPLIT_MAX;
+    if (split > smax) split = smax;
+    if (split < 1) split = 1;
+    // tokens per block: whole waves of RF_BLOCKS_PER_SM blocks per SM on a 148-SM part (the
+    // latency-bound selection phases of one block overlap another's stream), at most
+    // RF_MAX_BT tokens each
+    const int slots = 148 * RF_BLOCKS_PER_SM;
+    const int waves = (T + slots * RF_MAX_BT - 1) / (slots * RF_MAX_BT);
+    int bt = (T + slots * waves - 1) / (slots * waves);
+    if (bt < 1) bt = 1;
+    // ring: as deep as the blocks that share an SM leave room for (1 KB per block is reserved)
+    const int blocks = (T + bt - 1) / bt;
+    int per_sm = (blocks + 147) / 148;
+    if (per_sm > 4) per_sm = 4;
+    int ring = 0;
+    for (; per_sm >= 1; --per_sm) {
+        const int budget = RF_SMEM_MAX / per_sm - 1024;
+        ring = budget - (int)rf_smem_bytes(bt, E, 0);
+        if (ring >= rf_ring_min(bt, E)) break;
+    }
+    if (per_sm < 1 || rf_smem_bytes(bt, E, ring) > (size_t)RF_SMEM_MAX) return f;
+    const int hs = ((kb + split - 1) / split) * gemm::BK; // longest K range
+    f.ok = true;
+    f.split = split;
+    f.bt = bt;
+    f.ring_bytes = ring;
+    f.smem = rf_smem_bytes(bt, E, ring);
+    f.cA = (float)(1.25 * ((double)H + 4.0 * hs + split + 4.0) * 5.9604644775390625e-8);
+    return f;
+}
 
 Layout make_layout(const moe_problem *p)
 {
@@ -82,7 +138,12 @@ Layout make_layout(const moe_problem *p)
     };
     L.status = take(256);
     L.meta = take(sizeof(DispatchMeta));
-    L.logits = take(T * E * 4);
+    // router logits; the filter router keeps its GEMM partials [split, T, E] here
+    const FilterPlan fp = filter_plan(p);
+    L.logits = take(T * E * 4 * (size_t)(fp.ok ? fp.split : 1));
+    L.wgt = take(fp.ok ? E * H * 2 : 0); // filter router: W_g^T
+    L.wnorm = take(fp.ok ? (H + RF_SLAB - 1) / RF_SLAB * E * 4 : 0); // W_g column sums of squares
+    L.xsq = take(fp.ok ? (size_t)fp.split * T * 4 : 0);              // x row sums of squares
     L.end_route = o;
     L.topk_idx = take(T * K * 4);
     L.topk_w = take(T * K * 4);
@@ -114,6 +175,9 @@ template <typename T> T *at(void *ws, size_t off)
 {
     return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
 }
+
+struct FilterBufs;
+FilterBufs filter_bufs(void *ws, const Layout &L);
 
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 bool aligned4(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
@@ -206,13 +270,109 @@ void launch_route_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *Wg, const 
     kern<<<grid, block, smem, st>>>(x, Wg, bias, logits, T, H, E, status);
 }
 
+// Buffers of the tensor-core filter router (inside the caller's workspace).
+struct FilterBufs {
+    uint16_t *wgt;
+    float *wnorm;
+    float *xsq;
+};
+
+template <int KIND>
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                        int max_work, cudaStream_t st);
+bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols);
+
+FilterBufs filter_bufs(void *ws, const Layout &L)
+{
+    FilterBufs f;
+    f.wgt = at<uint16_t>(ws, L.wgt);
+    f.wnorm = at<float>(ws, L.wnorm);
+    f.xsq = at<float>(ws, L.xsq);
+    return f;
+}
+
+// Exact top-k for many experts: tensor-core filter logits, rigorous intervals, exact
+// sequential recomputation of the candidates only (route_filter.cuh). Three launches.
+cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
+                                const __nv_bfloat16 *xb, const __nv_bfloat16 *wb,
+                                const float *bias, int32_t *topk_idx, float *topk_w,
+                                float *parts, const FilterBufs &fb, int *status, cudaStream_t st)
+{
+    const int T = p->T, H = p->H, E = p->E;
+    route_filter_prep_kernel<<<dim3(E / 8, (H + RF_SLAB - 1) / RF_SLAB), 256, 0, st>>>(
+        wb, H, E, fb.wgt, fb.wnorm, status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    CUtensorMap mx, mw;
+    if (!make_map_2d(&mx, xb, (uint64_t)T, (uint64_t)H, gemm::BM) ||
+        !make_map_3d(&mw, wb, 1, (uint64_t)H, (uint64_t)E))
+        return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.dense_m_tiles = (T + gemm::BM - 1) / gemm::BM;
+    a.dense_rows = T;
+    a.k_split = fp.split;
+    a.n_tiles = (E + gemm::BN - 1) / gemm::BN;
+    a.n_boxes = E <= gemm::BN ? (E + 63) / 64 : 4;
+    a.k_blocks = H / gemm::BK;
+    a.out_f32 = parts;
+    a.xsq_f32 = fb.xsq;
+    a.ld_out = E;
+    a.n_cols = E;
+    a.status = status;
+    a.timeout_ns = g_timeout_ns.load();
+    err = launch_gemm<GEMM_LOGITS>(mx, mw, a, a.dense_m_tiles * a.n_tiles * fp.split, st);
+    if (err != cudaSuccess) return err;
+    RfArgs r{};
+    r.x = xb;
+    r.WgT = reinterpret_cast<const __nv_bfloat16 *>(fb.wgt);
+    r.wpart = fb.wnorm;
+    r.xsq = fb.xsq;
+    r.bias = bias;
+    r.parts = parts;
+    r.topk_idx = topk_idx;
+    r.topk_w = topk_w;
+    r.T = T;
+    r.H = H;
+    r.E = E;
+    r.k = p->top_k;
+    r.S = fp.split;
+    r.bt = fp.bt;
+    r.ring_bytes = fp.ring_bytes;
+    r.cA = fp.cA;
+    r.status = status;
+    r.timeout_ns = g_timeout_ns.load();
+    const size_t smem = fp.smem;
+    err = cudaFuncSetAttribute(route_filter_exact_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    route_filter_exact_kernel<<<(T + fp.bt - 1) / fp.bt, RF_THREADS, smem, st>>>(r);
+    return cudaGetLastError();
+}
+
+// Router choice for AUTO / FILTER / SEQUENTIAL (operands assumed 16-byte aligned).
+bool route_uses_filter(const moe_problem *p)
+{
+    const int mode = g_router_mode.load();
+    // AUTO takes the filter from 2^16 logits on (below, its fixed costs -- the W_g transpose,
+    // the GEMM and one chain of H dependent FMAs per candidate -- outweigh the savings)
+    const bool want = mode == MOE_ROUTER_FILTER ||
+                      (mode == MOE_ROUTER_AUTO && (int64_t)p->T * p->E >= (1 << 16));
+    return want && filter_plan(p).ok;
+}
+
 cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                          const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
-                         int *status, cudaStream_t st)
+                         int *status, cudaStream_t st, const FilterBufs *filter = nullptr)
 {
     const int T = p->T, H = p->H, E = p->E;
     const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     const auto *wb = reinterpret_cast<const __nv_bfloat16 *>(Wg);
+    // many experts: tensor-core filter plus exact recomputation of the candidates (needs the
+    // workspace buffers, W_g rows that TMA can address, and the top-k renormalised gates)
+    if (filter != nullptr && aligned16(x) && aligned16(Wg) && route_uses_filter(p))
+        return launch_route_filter(p, filter_plan(p), xb, wb, bias, topk_idx, topk_w, logits,
+                                   *filter, status, st);
     // blocks of the large-E tile (64 tokens x 64 experts); fewer than the SMs: go narrow
     const int64_t large_blocks = (int64_t)((T + 63) / 64) * ((E + 63) / 64);
     const int sms = sm_count() > 0 ? sm_count() : 148;
@@ -456,9 +616,11 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         return MOE_ERR_CUDA;
 
     const int64_t timeout = g_timeout_ns.load();
+    const FilterBufs fb = filter_bufs(ws, L);
     cudaError_t e = record(events, n_events, 0, st);
     if (e == cudaSuccess)
-        e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st);
+        e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st,
+                         &fb);
     if (e == cudaSuccess) e = record(events, n_events, 1, st);
     if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
     if (e == cudaSuccess && pair) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
@@ -537,6 +699,17 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
 
 extern "C" {
 
+int moe_forward_launches(const moe_problem *p)
+{
+    if (check_problem(p) != MOE_OK) return -1;
+    if (p->T == 0) return 0;
+    const int route = route_uses_filter(p) ? 3 : 2; // filter: prep, GEMM, exact; else logits, top-k
+    const int dispatch = 3;                          // count, scan, place
+    const int mode = g_gemm_mode.load();
+    const int layers = mode == MOE_GEMM_FUSED ? 1 : (mode == MOE_GEMM_CTA_PAIR ? 4 : 3);
+    return route + dispatch + layers;
+}
+
 size_t moe_workspace_size(const moe_problem *p)
 {
     if (check_problem(p) != MOE_OK) return 0;
@@ -564,7 +737,9 @@ moe_status moe_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = at<int>(ws, L.status);
     if (p->T == 0) return to_status(cudaMemsetAsync(status, 0, 8, st));
-    return to_status(launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st));
+    const FilterBufs fb = filter_bufs(ws, L);
+    return to_status(
+        launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st, &fb));
 }
 
 moe_status moe_route_noalloc(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
@@ -732,6 +907,13 @@ int moe_set_gemm_mode(int mode)
         mode != MOE_GEMM_FUSED)
         return -1;
     return g_gemm_mode.exchange(mode);
+}
+
+int moe_set_router_mode(int mode)
+{
+    if (mode != MOE_ROUTER_AUTO && mode != MOE_ROUTER_SEQUENTIAL && mode != MOE_ROUTER_FILTER)
+        return -1;
+    return g_router_mode.exchange(mode);
 }
 
 int moe_set_fault_injection(int layer0_item)

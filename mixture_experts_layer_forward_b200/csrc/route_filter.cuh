@@ -1,0 +1,490 @@
+// route_filter.cuh -- exact top-k routing for many experts with a tensor-core filter.
+//
+// The routing decision is defined on the sequential fp32 logits l[t][e] (one accumulator,
+// h ascending, then + bias; see route.cuh). For large E computing all T*E of them that way
+// costs T*E*H dependent FMAs. Instead:
+//   1. route_filter_prep_kernel: W_g^T (expert rows, for streaming) and partial sums of
+//      squares of every W_g column;
+//   2. m = x . W_g on the tensor cores (GEMM_LOGITS in gemm_tc.cuh), K split into S ranges
+//      of at most hs values; the S fp32 partial products are summed here in fixed order;
+//   3. route_filter_exact_kernel, per block of bt tokens:
+//      a. an interval [m - eta, m + eta] (m including the bias) that holds l, with
+//           eta = cA ||x_t|| ||w_e|| + 4 u (|m| + 1),  u = 2^-24,
+//           cA  = 1.25 (H + 4 hs + S + 4) u.
+//         ||x_t|| ||w_e|| bounds A = sum_h |x_h w_he| (Cauchy-Schwarz; both norms rounded
+//         up). The sequential fp32 chain is within 1.01 H u A of the exact dot product (every
+//         product of two bf16 values is exact in fp32, one rounding per step); the tensor-core
+//         partial of a K range of n values is assumed within 4 n u A_range of it (an adder
+//         that aligns to the largest addend with a 24-bit window and truncates stays near
+//         2.3 n u), and the S partials are summed with S u A; the last term covers the bias
+//         additions and the rounding of the interval ends; 1.25 is margin;
+//      b. an expert whose upper end is below the k-th largest lower end L cannot be in the
+//         top k: the k experts holding the k largest lower ends have exact logits >= L, all
+//         strictly above the excluded one's. The rest are the candidates;
+//      c. every candidate (token, expert) pair gets its exact sequential logit. Two producer
+//         warps stream the x rows of the block's tokens and the W_g^T rows of the union of
+//         their candidates through a ring of 64-value chunks (cp.async, completion counted on
+//         mbarriers); in eight consumer warps a thread owns two candidates of one token, so one
+//         x load serves two chains;
+//      d. top k among the candidates' exact logits, ties to the lower expert id, and the gates
+//         from those exact logits, in the same arithmetic as route_topk_kernel.
+// Hence the selection, its order and the gates equal those of the full sequential router.
+#pragma once
+
+#include "ptx.cuh"
+#include "route.cuh"
+
+namespace moe {
+
+constexpr int RF_CWARPS = 8;                 // consumer warps (pair chains)
+constexpr int RF_CTHREADS = RF_CWARPS * 32;
+constexpr int RF_PWARPS = 2;                 // producer warps (cp.async)
+constexpr int RF_PTHREADS = RF_PWARPS * 32;
+constexpr int RF_WARPS = RF_CWARPS + RF_PWARPS;
+constexpr int RF_THREADS = RF_WARPS * 32;
+constexpr int RF_HC = 64;                    // h values per streamed chunk
+constexpr int RF_ROW = 144;                  // staged row: 128 bytes + 16, so 16-byte column v
+                                             // of row r sits in bank group (r + v) mod 8
+constexpr int RF_NS_MAX = 16;                // deepest chunk ring
+constexpr int RF_MAX_BT = 32;                // tokens per block
+constexpr int RF_BLOCKS_PER_SM = 2;          // blocks the token split aims to co-schedule
+constexpr int RF_MAX_E = 512;
+constexpr int RF_SPLIT_MAX = 16;
+constexpr int RF_SLAB = 256;                 // h values per partial sum of squares of W_g
+constexpr int RF_SMEM_MAX = 232448;
+
+__device__ __forceinline__ float rf_norm_up(float ss, int n)
+{
+    // sqrt of an fp32 sum of n squares, scaled up past its rounding error
+    return sqrtf(ss) * (1.0f + (float)(n + 2) * 5.9604645e-8f);
+}
+
+// order-preserving int key of a float (for warp max/min reductions), and back
+__device__ __forceinline__ int rf_key(float f)
+{
+    const int i = __float_as_int(f);
+    return i >= 0 ? i : (i ^ 0x7fffffff);
+}
+__device__ __forceinline__ float rf_unkey(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff)); }
+
+// Two chains that share the x word: acc0 += x.lo * a.lo, then x.hi * a.hi; acc1 likewise with
+// b. bf16 halves of 32-bit words; each product is exact and each addition is rounded once to
+// fp32 (the arithmetic of fmaf on the widened values).
+__device__ __forceinline__ void fma2x2_bf16(uint32_t x, uint32_t a, uint32_t b, float &acc0,
+                                            float &acc1)
+{
+    asm("{\n\t.reg .b16 xl, xh, al, ah, bl, bh;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "mov.b32 {al, ah}, %3;\n\t"
+        "mov.b32 {bl, bh}, %4;\n\t"
+        "fma.rn.f32.bf16 %0, xl, al, %0;\n\t"
+        "fma.rn.f32.bf16 %1, xl, bl, %1;\n\t"
+        "fma.rn.f32.bf16 %0, xh, ah, %0;\n\t"
+        "fma.rn.f32.bf16 %1, xh, bh, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(x), "r"(a), "r"(b));
+}
+
+// Grid (E/8, ceil(H/RF_SLAB)): W_g^T[e][h] = W_g[h][e] and, per slab of RF_SLAB rows,
+// wpart[slab][e] = sum of W_g[h][e]^2 over the slab. Also clears the status word of the call.
+__global__ void __launch_bounds__(256)
+    route_filter_prep_kernel(const __nv_bfloat16 *__restrict__ Wg, int H, int E,
+                             uint16_t *__restrict__ WgT, float *__restrict__ wpart, int *status)
+{
+    __shared__ float red[8][8];
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && status != nullptr) {
+        status[0] = DEV_OK; // a new call starts with a clean status word
+        status[1] = 0;
+    }
+    const int e0 = blockIdx.x * 8;
+    const int h = blockIdx.y * RF_SLAB + threadIdx.x;
+    float ss[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss[j] = 0.0f;
+    if (h < H) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(Wg + (size_t)h * E + e0);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t b = (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xffffu);
+            const float v = __uint_as_float(b << 16);
+            ss[j] = v * v;
+            WgT[(size_t)(e0 + j) * H + h] = (uint16_t)b;
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float v = ss[j];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) red[warp][j] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < 8) {
+        float v = 0.0f;
+        for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+        wpart[(size_t)blockIdx.y * E + e0 + threadIdx.x] = v;
+    }
+}
+
+struct RfArgs {
+    const __nv_bfloat16 *x;   // [T, H]
+    const __nv_bfloat16 *WgT; // [E, H]
+    const float *wpart;       // [ceil(H / RF_SLAB), E] partial sums of squares of W_g
+    const float *xsq;         // [S, T] partial sums of squares of the x rows
+    const float *bias;        // [E] or nullptr
+    const float *parts;       // [S, E, T] tensor-core partials (column-major)
+    int32_t *topk_idx;        // [T, k]
+    float *topk_w;            // [T, k]
+    int T, H, E, k, S, bt;
+    int ring_bytes;           // bytes of the chunk ring (region 0)
+    float cA;                 // interval coefficient of ||x|| ||w||
+    int *status;
+    int64_t timeout_ns;
+};
+
+// Shared memory of route_filter_exact_kernel. Region 0 holds the filter logits [bt][E + 1],
+// then the chunk ring; the exact logits of the candidates have their own [bt][E].
+__host__ __device__ inline size_t rf_region0_bytes(int bt, int E, int ring_bytes)
+{
+    const size_t mrow = (size_t)bt * (E + 1) * 4;
+    const size_t r = (size_t)ring_bytes > mrow ? (size_t)ring_bytes : mrow;
+    return (r + 127) & ~(size_t)127;
+}
+__host__ __device__ inline size_t rf_smem_bytes(int bt, int E, int ring_bytes)
+{
+    const int ew = (E + 31) / 32;
+    return rf_region0_bytes(bt, E, ring_bytes) + (size_t)bt * E * 4 /*exact*/ +
+           2 * RF_NS_MAX * 8 /*mbarriers*/ +
+           (size_t)(bt + E) * 8 /*row sources*/ + (size_t)E * 4 /*wn*/ +
+           (size_t)bt * ew * 4 /*cand*/ + (size_t)E * 4 * 2 /*union*/ + 16 * 4 * 2 /*words*/ +
+           (size_t)(RF_MAX_BT + 1) * 4 * 2 /*tok_off, unit_off*/ + 16 /*U, abort*/;
+}
+// Smallest ring that holds two chunks of every row a block can stage.
+__host__ __device__ inline int rf_ring_min(int bt, int E) { return 2 * (bt + E) * RF_ROW; }
+
+// r-th set bit (r >= 0) of the candidate words of one token; E when there is none
+__device__ __forceinline__ int rf_nth_bit(const uint32_t *words, int ew, int r, int E)
+{
+    for (int w0 = 0; w0 < ew; ++w0) {
+        uint32_t bits = words[w0];
+        const int pc = __popc(bits);
+        if (r < pc) {
+            for (int i = 0; i < r; ++i) bits &= bits - 1u;
+            return w0 * 32 + __ffs(bits) - 1;
+        }
+        r -= pc;
+    }
+    return E;
+}
+
+__global__ void __launch_bounds__(RF_THREADS)
+    route_filter_exact_kernel(const RfArgs a)
+{
+    extern __shared__ __align__(128) uint8_t rf_smem[];
+    const int E = a.E, H = a.H, T = a.T, k = a.k, bt = a.bt;
+    const int ew = (E + 31) / 32;
+    const int ME = E + 1; // padded filter-logit row
+    const size_t r0 = rf_region0_bytes(bt, E, a.ring_bytes);
+    float *mrow = reinterpret_cast<float *>(rf_smem);                // a/b: [bt][E + 1]
+    float *exact = reinterpret_cast<float *>(rf_smem + r0);          // [bt][E] exact logits
+    uint64_t *bars = reinterpret_cast<uint64_t *>(exact + (size_t)bt * E); // full, empty
+    const __nv_bfloat16 **row_src =
+        reinterpret_cast<const __nv_bfloat16 **>(bars + 2 * RF_NS_MAX); // [bt + U] row starts
+    float *wn = reinterpret_cast<float *>(row_src + bt + E);        // [E] >= ||w_e||
+    uint32_t *cand = reinterpret_cast<uint32_t *>(wn + E);          // [bt][ew]
+    int *uni_row = reinterpret_cast<int *>(cand + (size_t)bt * ew); // [E] expert -> W row
+    int *uni_list = uni_row + E;                                     // [U] W row -> expert
+    uint32_t *uword = reinterpret_cast<uint32_t *>(uni_list + E);   // [16] union words
+    int *ubase = reinterpret_cast<int *>(uword + 16);                // [16] their ranks
+    int *tok_off = ubase + 16;                                       // [bt + 1] candidates
+    int *unit_off = tok_off + RF_MAX_BT + 1;                         // [bt + 1] pair units
+    int *n_union = unit_off + RF_MAX_BT + 1;
+    volatile int *abort_flag = n_union + 1;
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (RF_NS_MAX + s); };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int t0 = blockIdx.x * bt;
+    const int nt = (T - t0) < bt ? (T - t0) : bt; // tokens of this block
+    const size_t ET = (size_t)E * T;
+
+    if (tid == 0) {
+        for (int i = 0; i < RF_NS_MAX; ++i) {
+            mbar_init(full_bar(i), RF_PTHREADS);
+            mbar_init(empty_bar(i), RF_CWARPS);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+
+    // ---- column norms and filter logits (summed over the splits, + bias) ----
+    const int nslab = (H + RF_SLAB - 1) / RF_SLAB;
+    for (int e = tid; e < E; e += RF_THREADS) {
+        float s = 0.0f;
+        for (int j0 = 0; j0 < nslab; j0 += 16) { // sixteen independent loads in flight
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (j0 + j < nslab) s += a.wpart[(size_t)(j0 + j) * E + e];
+        }
+        wn[e] = rf_norm_up(s, H);
+    }
+#pragma unroll 2
+    for (int q = tid; q < E * bt; q += RF_THREADS) {
+        const int e = q / bt, tl = q - e * bt; // consecutive threads: consecutive tokens
+        if (tl < nt) {
+            const float *pp = a.parts + (size_t)e * T + t0 + tl;
+            float s = pp[0];
+#pragma unroll
+            for (int j = 1; j < RF_SPLIT_MAX; ++j) // splits in order; the loads are independent
+                if (j < a.S) s += pp[(size_t)j * ET];
+            if (a.bias != nullptr) s = s + a.bias[e];
+            mrow[tl * ME + e] = s;
+        }
+    }
+    __syncthreads();
+
+    // ---- a/b. intervals and candidates, one warp per token ----
+    for (int tl = warp; tl < bt; tl += RF_WARPS) {
+        if (tl >= nt) {
+            for (int w0 = lane; w0 < ew; w0 += 32) cand[tl * ew + w0] = 0u;
+            continue;
+        }
+        const float *mr = mrow + tl * ME;
+        float ss = 0.0f; // ||x_t||^2 from the filter GEMM's per-split partial sums
+        for (int j = 0; j < a.S; ++j) ss += a.xsq[(size_t)j * T + t0 + tl];
+        const float cx = a.cA * rf_norm_up(ss, H);
+        // L = k-th largest lower end, counted with multiplicity: per round the warp maximum of
+        // the remaining lower ends and how many experts hold it (lane owns e = lane + 32 i)
+        uint32_t removed = 0u;
+        int taken = 0, Lk = (int)0x80000000;
+        while (taken < k) {
+            int best = (int)0x80000000;
+            for (int e = lane, i = 0; e < E; e += 32, ++i) {
+                if ((removed >> i) & 1u) continue;
+                const float m = mr[e];
+                const int key = rf_key(m - (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)));
+                best = key > best ? key : best;
+            }
+            const int mx = __reduce_max_sync(0xffffffffu, best);
+            int mine = 0;
+            for (int e = lane, i = 0; e < E; e += 32, ++i) {
+                if ((removed >> i) & 1u) continue;
+                const float m = mr[e];
+                const int key = rf_key(m - (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)));
+                if (key == mx) {
+                    removed |= 1u << i;
+                    ++mine;
+                }
+            }
+            taken += (int)__reduce_add_sync(0xffffffffu, (unsigned)mine);
+            Lk = mx;
+            if (mx == (int)0x80000000) break; // nothing left (non-finite input)
+        }
+        const float L = rf_unkey(Lk);
+        for (int w0 = 0; w0 < ew; ++w0) {
+            const int e = w0 * 32 + lane;
+            bool c = false;
+            if (e < E) {
+                const float m = mr[e];
+                c = (m + (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)) >= L);
+            }
+            const uint32_t bits = __ballot_sync(0xffffffffu, c);
+            if (lane == 0) cand[tl * ew + w0] = bits;
+        }
+    }
+    __syncthreads();
+
+    // ---- candidate and unit offsets per token, union of the candidate experts ----
+    if (warp == 0) {
+        int cnt = 0;
+        if (lane < bt)
+            for (int w0 = 0; w0 < ew; ++w0) cnt += __popc(cand[lane * ew + w0]);
+        const int units = (cnt + 1) >> 1; // two candidates of one token per thread
+        int inc = cnt, uinc = units;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, inc, off);
+            const int uo = __shfl_up_sync(0xffffffffu, uinc, off);
+            if (lane >= off) {
+                inc += o;
+                uinc += uo;
+            }
+        }
+        if (lane < bt) {
+            tok_off[lane] = inc - cnt;
+            unit_off[lane] = uinc - units;
+        }
+        if (lane == 31) { // lanes >= bt add 0
+            tok_off[bt] = inc;
+            unit_off[bt] = uinc;
+        }
+    } else if (warp == 1) {
+        uint32_t uw = 0u; // union word `lane` (ew <= 16)
+        if (lane < ew)
+            for (int tl = 0; tl < bt; ++tl) uw |= cand[tl * ew + lane];
+        const int pc = __popc(uw);
+        int up = pc;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, up, off);
+            if (lane >= off) up += o;
+        }
+        if (lane < ew) {
+            uword[lane] = uw;
+            ubase[lane] = up - pc;
+        }
+        if (lane == 31) *n_union = up;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += RF_THREADS) {
+        const uint32_t uw = uword[e >> 5];
+        const int b = e & 31;
+        if ((uw >> b) & 1u) {
+            const int r = ubase[e >> 5] + __popc(uw & ((1u << b) - 1u));
+            uni_row[e] = r;
+            uni_list[r] = e;
+            row_src[bt + r] = a.WgT + (size_t)e * H;
+        } else {
+            uni_row[e] = -1;
+        }
+    }
+    for (int r = tid; r < bt; r += RF_THREADS) row_src[r] = a.x + (size_t)(t0 + (r < nt ? r : 0)) * H;
+    __syncthreads();
+
+    // ---- c. exact sequential logits of the candidate pairs ----
+    // Producer warps stream chunk g of every pass into ring slot g % ns; each producer thread
+    // arrives on full[slot] once its copies have landed; the consumer warps release the slot
+    // on empty[slot].
+    const int U = *n_union;
+    const int NU = unit_off[bt];
+    const int rows = bt + U;
+    const uint32_t stage_bytes = (uint32_t)rows * RF_ROW;
+    int ns = a.ring_bytes / (int)stage_bytes;
+    if (ns > RF_NS_MAX) ns = RF_NS_MAX;
+    if (ns < 2) ns = 2; // the host sizes the ring for two chunks of bt + E rows
+    const int nchunk = H / RF_HC;
+    const int npass = (NU + RF_CTHREADS - 1) / RF_CTHREADS;
+    const int total = npass * nchunk;
+
+    if (warp >= RF_CWARPS) {
+        // ---------------- producers ----------------
+        const int pt = tid - RF_CTHREADS;
+        const uint32_t ring0 = smem_u32(rf_smem);
+        for (int g = 0; g < total; ++g) {
+            const int slot = g % ns;
+            if (g >= ns && !mbar_wait_bounded(empty_bar(slot), (uint32_t)((g / ns - 1) & 1),
+                                              abort_flag, a.timeout_ns, a.status, 180))
+                break;
+            const int h0 = (g % nchunk) * RF_HC;
+            const uint32_t base = ring0 + (uint32_t)slot * stage_bytes;
+            for (int p = pt; p < rows * 8; p += RF_PTHREADS) {
+                const int r = p >> 3, v = p & 7;
+                cp_async_16(base + (uint32_t)(r * RF_ROW + v * 16), row_src[r] + h0 + v * 8,
+                            r >= bt || r < nt);
+            }
+            cp_async_arrive_noinc(full_bar(slot));
+        }
+        cp_async_wait_all(); // this thread's copies have landed before the block moves on
+    } else {
+        // ---------------- consumers ----------------
+        bool ok = true;
+        for (int pass = 0; ok && pass < npass; ++pass) {
+            const int u = pass * RF_CTHREADS + tid;
+            const bool active = u < NU;
+            int tl = 0, e0 = 0, e1 = E;
+            if (active) {
+                while (tl + 1 < bt && unit_off[tl + 1] <= u) ++tl;
+                const int r = 2 * (u - unit_off[tl]);
+                e0 = rf_nth_bit(cand + tl * ew, ew, r, E);
+                e1 = rf_nth_bit(cand + tl * ew, ew, r + 1, E); // E: this unit has one chain
+            }
+            const uint32_t xo = (uint32_t)(tl * RF_ROW);
+            const uint32_t wo0 = (uint32_t)((bt + (active ? uni_row[e0] : 0)) * RF_ROW);
+            const uint32_t wo1 = (e1 < E) ? (uint32_t)((bt + uni_row[e1]) * RF_ROW) : wo0;
+            float acc0 = 0.0f, acc1 = 0.0f;
+            for (int c = 0; c < nchunk; ++c) {
+                const int g = pass * nchunk + c;
+                const int slot = g % ns;
+                const bool got = mbar_wait_bounded(full_bar(slot), (uint32_t)((g / ns) & 1),
+                                                   abort_flag, a.timeout_ns, a.status, 181);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                if (active) {
+                    const uint8_t *st = rf_smem + (size_t)slot * stage_bytes;
+                    const uint4 *xa = reinterpret_cast<const uint4 *>(st + xo);
+                    const uint4 *w0 = reinterpret_cast<const uint4 *>(st + wo0);
+                    const uint4 *w1 = reinterpret_cast<const uint4 *>(st + wo1);
+#pragma unroll
+                    for (int vv = 0; vv < RF_HC / 8; ++vv) { // h ascending: storage order
+                        const uint4 p = xa[vv], q0 = w0[vv], q1 = w1[vv];
+                        fma2x2_bf16(p.x, q0.x, q1.x, acc0, acc1);
+                        fma2x2_bf16(p.y, q0.y, q1.y, acc0, acc1);
+                        fma2x2_bf16(p.z, q0.z, q1.z, acc0, acc1);
+                        fma2x2_bf16(p.w, q0.w, q1.w, acc0, acc1);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(slot));
+            }
+            if (ok && active) {
+                float v0 = acc0;
+                if (a.bias != nullptr) v0 = v0 + a.bias[e0];
+                exact[tl * E + e0] = v0;
+                if (e1 < E) {
+                    float v1 = acc1;
+                    if (a.bias != nullptr) v1 = v1 + a.bias[e1];
+                    exact[tl * E + e1] = v1;
+                }
+            }
+        }
+    }
+    __syncthreads(); // exact logits complete
+
+    // ---- d. top k of the candidates' exact logits (ties to the lower id) and the gates ----
+    for (int tl = warp; tl < nt; tl += RF_WARPS) {
+        const int t = t0 + tl;
+        const float *row = exact + tl * E;
+        const uint32_t *cw = cand + tl * ew;
+        uint32_t removed = 0u; // lane owns e = lane + 32 i; non-candidates count as removed
+        for (int e = lane, i = 0; e < E; e += 32, ++i)
+            if (!((cw[e >> 5] >> (e & 31)) & 1u)) removed |= 1u << i;
+        float sel_val = 0.0f, top = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            int best = (int)0x80000000, bi = 0x7fffffff;
+            for (int e = lane, i = 0; e < E; e += 32, ++i) {
+                if ((removed >> i) & 1u) continue;
+                const int key = rf_key(row[e]);
+                if (key > best) { best = key; bi = e; } // e ascending: keeps the lower id
+            }
+            const int mx = __reduce_max_sync(0xffffffffu, best);
+            int w = (int)__reduce_min_sync(0xffffffffu, (unsigned)(best == mx ? bi : 0x7fffffff));
+            if (w < 0 || w >= E) w = 0; // unsupported non-finite rows still index the row
+            const float bv = rf_unkey(mx);
+            if ((w & 31) == lane) removed |= 1u << (w >> 5);
+            if (j == 0) top = bv;
+            if (lane == 0) a.topk_idx[(size_t)t * k + j] = w;
+            if (j < 32 && j == lane) sel_val = bv;
+            if (j >= 32 && lane == 0) a.topk_w[(size_t)t * k + j] = bv;
+        }
+        __syncwarp();
+        float denom = 0.0f;
+        for (int j = lane; j < k; j += 32) {
+            const float v = (j < 32) ? sel_val : a.topk_w[(size_t)t * k + j];
+            denom += expf(v - top);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
+        __syncwarp();
+        for (int j = lane; j < k; j += 32) {
+            const float v = (j < 32) ? sel_val : a.topk_w[(size_t)t * k + j];
+            a.topk_w[(size_t)t * k + j] = expf(v - top) / denom;
+        }
+    }
+}
+
+} // namespace moe

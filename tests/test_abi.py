@@ -89,3 +89,34 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         _native.library()
+
+
+def test_forward_launch_count_follows_the_modes(lib):
+    """moe_forward_launches: host logic only (router and GEMM choice), no GPU needed."""
+    from mixture_experts_layer_forward_b200 import synth
+
+    mixtral = moe.Problem.from_config(synth.CONFIGS["mixtral"])
+    qwen2 = moe.Problem.from_config(synth.CONFIGS["qwen2"])
+    decode = moe.Problem.from_config(synth.CONFIGS["skew_decode"])
+    prev_r = moe.moe_set_router_mode(moe.ROUTER_AUTO)
+    prev_g = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
+    try:
+        assert moe.moe_forward_launches(mixtral) == 8   # E = 8: sequential router
+        assert moe.moe_forward_launches(qwen2) == 9     # T*E >= 2^16: filter router
+        assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential router
+        moe.moe_set_router_mode(moe.ROUTER_FILTER)
+        assert moe.moe_forward_launches(decode) == 9
+        assert moe.moe_forward_launches(mixtral) == 8   # the filter needs E > 16
+        moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
+        assert moe.moe_forward_launches(qwen2) == 8
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED)
+        assert moe.moe_forward_launches(qwen2) == 6
+        moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)
+        assert moe.moe_forward_launches(qwen2) == 9
+        assert moe.moe_forward_launches(moe.Problem.make(0, 128, 128, 8, 2)) == 0
+        assert moe.moe_forward_launches(moe.Problem.make(4, 100, 128, 8, 2)) == -1  # H % 64
+    finally:
+        moe.moe_set_router_mode(prev_r)
+        moe.moe_set_gemm_mode(prev_g)
+    with pytest.raises(ValueError):
+        moe.moe_set_router_mode(7)

@@ -89,8 +89,15 @@ ROUTE_CASES = [
 ]
 
 
+@pytest.fixture(params=[moe.ROUTER_FILTER, moe.ROUTER_SEQUENTIAL], ids=["filter", "sequential"])
+def router_mode(request):
+    prev = moe.moe_set_router_mode(request.param)
+    yield request.param
+    moe.moe_set_router_mode(prev)
+
+
 @pytest.mark.parametrize("case", ROUTE_CASES, ids=[c[0] for c in ROUTE_CASES])
-def test_route_bit_exact(case):
+def test_route_bit_exact(case, router_mode):
     name, T, H, E, k, unscaled, zipf, gate = case
     cfg = cfg_small(name, T, H, 64, E, k, gate=gate, gate_std_unscaled=unscaled, zipf_s=zipf)
     inp = synth.make_inputs(cfg, seed=3)
@@ -106,6 +113,91 @@ def test_route_bit_exact(case):
     ref_idx, ref_w = oracle.topk_gates(logits, k, gate=gate)
     assert np.array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+
+
+def _route(p, x, Wg, bias, T, k):
+    ws = alloc_ws(p)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.moe_route(p, x.cuda(), Wg.cuda(), None if bias is None else bias.cuda(), idx, w, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    return idx.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("unscaled", [False, True], ids=["scaled", "unscaled"])
+def test_route_rounding_level_ties(router_mode, unscaled):
+    """Every expert has the same exact real logit; they differ only in the fp32 rounding of
+    the sequential sum (gate columns are one column with pairs of entries swapped where the
+    token has equal values), so the choice is made at the last bit of the fp32 logits."""
+    T, H, E, k = 300, 256, 64, 8
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn(T, H, generator=g)
+    for j in range(6):
+        x[:, 2 * j + 1] = x[:, 2 * j]
+    x = x.to(torch.bfloat16)
+    col = torch.randn(H, generator=g) / (1.0 if unscaled else math.sqrt(H))
+    cols = []
+    for e in range(E):
+        c = col.clone()
+        for j in range(6):
+            if (e >> j) & 1:
+                c[2 * j], c[2 * j + 1] = col[2 * j + 1], col[2 * j]
+        cols.append(c)
+    Wg = torch.stack(cols, dim=1).to(torch.bfloat16).contiguous()
+    p = moe.Problem.make(T, H, 64, E, k)
+    got_idx, got_w = _route(p, x, Wg, None, T, k)
+    logits = oracle.router_logits(bits(x), bits(Wg), None)
+    ref_idx, ref_w = oracle.topk_gates(logits, k)
+    assert np.array_equal(got_idx, ref_idx)
+    np.testing.assert_allclose(got_w, ref_w, rtol=1e-5, atol=1e-7)
+
+
+def test_route_filter_matches_sequential_bitwise():
+    """Both router variants give bit-identical indices and gates (the gates are computed from
+    the same sequential fp32 logits)."""
+    cfg = cfg_small("filter_vs_seq", 1000, 512, 64, 128, 8, zipf_s=1.2)
+    inp = synth.make_inputs(cfg, seed=22)
+    p = moe.Problem.from_config(cfg)
+    res = []
+    for mode in (moe.ROUTER_FILTER, moe.ROUTER_SEQUENTIAL):
+        prev = moe.moe_set_router_mode(mode)
+        try:
+            res.append(_route(p, inp["x"], inp["Wg"], inp["bias"], cfg.T, cfg.k))
+        finally:
+            moe.moe_set_router_mode(prev)
+    assert np.array_equal(res[0][0], res[1][0])
+    assert np.array_equal(res[0][1].view(np.uint32), res[1][1].view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["qwen2", "skew", "skew_decode"])
+def test_route_filter_matches_sequential_full_size(name):
+    """The bench workloads with many experts: filter and sequential routers agree bitwise."""
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    p = moe.Problem.from_config(cfg)
+    res = []
+    for mode in (moe.ROUTER_FILTER, moe.ROUTER_SEQUENTIAL):
+        prev = moe.moe_set_router_mode(mode)
+        try:
+            res.append(_route(p, inp["x"], inp["Wg"], inp["bias"], cfg.T, cfg.k))
+        finally:
+            moe.moe_set_router_mode(prev)
+    assert np.array_equal(res[0][0], res[1][0])
+    assert np.array_equal(res[0][1].view(np.uint32), res[1][1].view(np.uint32))
+
+
+def test_route_all_experts_equal(router_mode):
+    """Identical gate columns: every logit ties, so the top k are experts 0..k-1 with equal
+    gates (every expert is a candidate of the filter)."""
+    T, H, E, k = 70, 128, 96, 8
+    g = torch.Generator().manual_seed(23)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    col = (torch.randn(H, 1, generator=g) / math.sqrt(H)).to(torch.bfloat16)
+    Wg = col.repeat(1, E).contiguous()
+    p = moe.Problem.make(T, H, 64, E, k)
+    got_idx, got_w = _route(p, x, Wg, None, T, k)
+    assert np.array_equal(got_idx, np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    assert np.all(got_w == np.float32(1.0 / k))
 
 
 def test_route_exact_ties_go_to_lower_id():
@@ -261,6 +353,23 @@ def test_forward_matches_oracle(cfg, gemm_mode):
     assert_out_close(out, ref, cfg.name)
     out2, _, _, _ = run_forward(cfg, inp, ws)
     assert torch.equal(out, out2), "two identical calls differ"
+
+
+def test_forward_with_filter_router():
+    """The whole layer with the tensor-core filter router forced on a small problem."""
+    cfg = cfg_small("filter_fwd", 333, 256, 192, 64, 6, zipf_s=1.2)
+    inp = synth.make_inputs(cfg, seed=15)
+    prev = moe.moe_set_router_mode(moe.ROUTER_FILTER)
+    try:
+        out, idx, w, _ = run_forward(cfg, inp)
+    finally:
+        moe.moe_set_router_mode(prev)
+    b = inp["bias"].numpy()
+    ref, ref_idx, ref_w = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                             bits(inp["W2"]), cfg.k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+    assert_out_close(out, ref, cfg.name)
 
 
 def test_gemm_variants_agree():
