@@ -236,6 +236,17 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
 #define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
 
+/* Work order of the standalone grouped-GEMM launches (a tuning and test hook; not
+ * thread-safe; results are bit-identical either way, every output tile is computed by one
+ * CTA in one K order):
+ * 0 (default): expert-major order (expert, then N tile, then M tile);
+ * 1: the work items of experts with a single m-tile, whose weights are streamed for one
+ *   tile only (HBM bound), are spread evenly among the items of the other experts (tensor
+ *   bound), so both run at the same time. On the skewed layer this measured no gain: under
+ *   the 1 kW cap the GEMMs are power-bound and the order does not change the energy.
+ * Returns the previous setting, or -1 for another value. */
+MOE_API int moe_set_work_order(int interleave);
+
 /* Router variant (a tuning and test hook; not thread-safe). All give the same routing and
  * gates (the selection is always made on the sequential fp32 logits, see moe_route):
  * MOE_ROUTER_FILTER: for 16 < E <= 512 with E % 8 == 0, MOE_GATE_SOFTMAX_TOPK and 16-byte

@@ -33,6 +33,7 @@ from ._native import (  # noqa: F401
     moe_route_noalloc,
     moe_set_gemm_mode,
     moe_set_router_mode,
+    moe_set_work_order,
     ROUTER_AUTO,
     ROUTER_SEQUENTIAL,
     ROUTER_FILTER,

@@ -90,6 +90,7 @@ def library() -> ctypes.CDLL:
             "moe_set_gemm_mode": ([i32], i32),
             "moe_set_fault_injection": ([i32], i32),
             "moe_set_router_mode": ([i32], i32),
+            "moe_set_work_order": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -256,6 +257,15 @@ ROUTER_AUTO, ROUTER_SEQUENTIAL, ROUTER_FILTER = 0, 1, 2
 def moe_set_fault_injection(layer0_item: int) -> int:
     """Test hook: withhold the ready signal of one layer0 work item of the fused kernel."""
     return int(library().moe_set_fault_injection(int(layer0_item)))
+
+
+def moe_set_work_order(interleave: int) -> int:
+    """0: expert-major GEMM work order (default); 1: spread single-tile experts' work among
+    the others. Returns the previous setting."""
+    rc = int(library().moe_set_work_order(int(interleave)))
+    if rc < 0:
+        raise ValueError(f"unknown work order {interleave}")
+    return rc
 
 
 def moe_set_router_mode(mode: int) -> int:

@@ -28,7 +28,7 @@ struct DispatchMeta {
     int num_tiles;   // sum_e ceil(c_e / M_TILE)
     int padded_rows; // P_pad = num_tiles * M_TILE
     int num_ptiles;  // sum_e ceil(ceil(c_e / M_TILE) / 2): pairs of m-tiles of one expert
-    int pad_;
+    int num_cold;    // experts with exactly one m-tile (their weights are read for one tile)
 };
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
@@ -99,7 +99,9 @@ __global__ void __launch_bounds__(1024)
                          int32_t *__restrict__ tile_expert, int32_t *__restrict__ ptile_off,
                          int32_t *__restrict__ ptile_expert, DispatchMeta *meta,
                          int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
-                         int64_t padded_rows_max, int *__restrict__ ready, int n_ready)
+                         int64_t padded_rows_max, int *__restrict__ ready, int n_ready,
+                         int32_t *__restrict__ hot_off, int32_t *__restrict__ hot_tile_expert,
+                         int32_t *__restrict__ cold_tile)
 {
     // the fused layer kernel's tile-level ready counters start from zero on every call
     for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
@@ -122,6 +124,11 @@ __global__ void __launch_bounds__(1024)
     const int inc_t = block_inclusive_scan_1024(ntile, warp_sums);
     const int nptile = (ntile + 1) / 2;
     const int inc_p = block_inclusive_scan_1024(nptile, warp_sums);
+    // work classes of the grouped GEMMs: "cold" experts (one m-tile) stream their weights for
+    // a single tile; the rest ("hot") reuse each weight tile across their m-tiles
+    const int hot_t = ntile >= 2 ? ntile : 0;
+    const int inc_h = block_inclusive_scan_1024(hot_t, warp_sums);
+    const int inc_1 = block_inclusive_scan_1024(ntile == 1 ? 1 : 0, warp_sums);
     if (e < E) {
         if (offsets != nullptr) {
             offsets[e + 1] = inc_c;
@@ -142,10 +149,17 @@ __global__ void __launch_bounds__(1024)
             if (e == 0) ptile_off[0] = 0;
             for (int i = 0; i < nptile; ++i) ptile_expert[inc_p - nptile + i] = e;
         }
+        if (hot_off != nullptr) {
+            hot_off[e + 1] = inc_h;
+            if (e == 0) hot_off[0] = 0;
+            for (int i = 0; i < hot_t; ++i) hot_tile_expert[inc_h - hot_t + i] = e;
+            if (ntile == 1) cold_tile[inc_1 - 1] = tile_first;
+        }
         if (e == E - 1) {
             meta->num_tiles = inc_t;
             meta->padded_rows = poff_next;
             meta->num_ptiles = inc_p;
+            meta->num_cold = inc_1;
             s_poff[E] = poff_next;
         }
     }

@@ -75,7 +75,16 @@ struct GemmArgs {
     const int32_t *tile_expert; // [max_tiles] expert of each m-tile
     const int32_t *ptile_off;   // [E+1] first m-tile pair of each expert (pair kernel)
     const int32_t *ptile_expert; // expert of each m-tile pair (pair kernel)
-    const DispatchMeta *meta;   // num_tiles
+    const DispatchMeta *meta;   // num_tiles, num_cold
+    // interleave != 0: the work items of "cold" experts (one m-tile: weight-bandwidth bound)
+    // are spread evenly among those of the other ("hot", compute bound) experts, so HBM and
+    // the tensor cores are busy at the same time. hot_off [E+1] prefixes the hot experts'
+    // m-tiles, hot_tile_expert lists the expert of each hot m-tile, cold_tile the m-tile of
+    // each cold expert (written by the dispatch scan).
+    int interleave;
+    const int32_t *hot_off;
+    const int32_t *hot_tile_expert;
+    const int32_t *cold_tile;
     const float *row_w;         // GEMM_SCALE: gate weight of each padded row
     const int32_t *gather_idx;  // layer0: token of each padded row (-1: pad), A rows are
                                 // gathered from x with it; nullptr: A rows are contiguous
@@ -115,6 +124,28 @@ __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, 
         const int r = w / a.dense_m_tiles;
         nt = r % a.n_tiles;
         ks = r / a.n_tiles;
+        return;
+    }
+    if (a.interleave) {
+        const int64_t total = (int64_t)a.meta->num_tiles * a.n_tiles;
+        const int64_t cold = (int64_t)a.meta->num_cold * a.n_tiles;
+        const int64_t cb = (int64_t)w * cold / total;        // cold items before slot w
+        const int64_t cb1 = ((int64_t)w + 1) * cold / total;
+        if (cb1 > cb) { // slot w holds cold item cb: the expert's single m-tile, n-tile cb % n
+            const int j = (int)(cb / a.n_tiles);
+            nt = (int)(cb - (int64_t)j * a.n_tiles);
+            mt = a.cold_tile[j];
+            e = a.tile_expert[mt];
+            return;
+        }
+        const int h = (int)(w - cb); // hot item h, in the hot experts' expert-major order
+        e = a.hot_tile_expert[h / a.n_tiles];
+        const int hb = a.hot_off[e];
+        const int base = a.tile_off[e];
+        const int cnt = a.tile_off[e + 1] - base;
+        const int local = h - hb * a.n_tiles;
+        mt = base + local % cnt;
+        nt = local / cnt;
         return;
     }
     const int q = w / a.n_tiles;

@@ -29,6 +29,9 @@ std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fault_skip{-1};
 // router variant for many experts: MOE_ROUTER_AUTO (tensor-core filter) or sequential only
 std::atomic<int> g_router_mode{MOE_ROUTER_AUTO};
+// grouped-GEMM work order (test and tuning hook): expert-major by default; interleaving
+// the single-tile experts' items measured no gain on the skewed layer (power-bound GEMMs)
+std::atomic<int> g_interleave{0};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -62,7 +65,8 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 struct Layout {
     size_t status, meta, logits, wgt, wnorm, xsq, topk_idx, topk_w, chunk,
         counts, offsets, poff, tile_off,
-        tile_expert, ptile_off, ptile_expert, ready, gather_idx, inv_pos, row_w, x_perm, h, ys,
+        tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
+        gather_idx, inv_pos, row_w, x_perm, h, ys,
         x_stage, out_stage;
     size_t end_route, end_dispatch, end_forward, end_host;
     int64_t pmax;
@@ -155,6 +159,9 @@ Layout make_layout(const moe_problem *p)
     L.tile_expert = take((size_t)L.max_tiles * 4);
     L.ptile_off = take((E + 1) * 4);
     L.ptile_expert = take((size_t)L.max_tiles * 4);
+    L.hot_off = take((E + 1) * 4);
+    L.hot_tile_expert = take((size_t)L.max_tiles * 4);
+    L.cold_tile = take(E * 4);
     L.n_ready = L.max_tiles + (int)((H + 255) / 256); // fused kernel: per M tile, per stripe
     L.ready = take((size_t)L.n_ready * 4);
     L.gather_idx = take(P * 4);
@@ -396,6 +403,7 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
 struct DispatchOut {
     int32_t *counts, *offsets, *poff, *gather_idx, *inv_pos, *tile_off, *tile_expert, *chunk;
     int32_t *ptile_off, *ptile_expert;
+    int32_t *hot_off, *hot_tile_expert, *cold_tile;
     int *ready;
     int n_ready;
     float *row_w;
@@ -417,7 +425,8 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, o.counts, o.offsets, o.poff,
                                              o.tile_off, o.tile_expert, o.ptile_off,
                                              o.ptile_expert, o.meta, o.gather_idx, o.row_w,
-                                             L.pmax, o.ready, o.ready ? o.n_ready : 0);
+                                             L.pmax, o.ready, o.ready ? o.n_ready : 0,
+                                             o.hot_off, o.hot_tile_expert, o.cold_tile);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
@@ -593,6 +602,9 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     d.chunk = at<int32_t>(ws, L.chunk);
     d.ptile_off = at<int32_t>(ws, L.ptile_off);
     d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
+    d.hot_off = at<int32_t>(ws, L.hot_off);
+    d.hot_tile_expert = at<int32_t>(ws, L.hot_tile_expert);
+    d.cold_tile = at<int32_t>(ws, L.cold_tile);
     d.ready = at<int>(ws, L.ready);
     d.n_ready = L.n_ready;
     d.row_w = at<float>(ws, L.row_w);
@@ -631,6 +643,9 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a0.tile_expert = d.tile_expert;
     a0.ptile_off = d.ptile_off;
     a0.ptile_expert = d.ptile_expert;
+    a0.hot_off = d.hot_off;
+    a0.hot_tile_expert = d.hot_tile_expert;
+    a0.cold_tile = d.cold_tile;
     a0.meta = d.meta;
     a0.row_w = nullptr;
     a0.gather_idx = pair ? nullptr : d.gather_idx;
@@ -681,6 +696,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         return to_status(e);
     }
 
+    // standalone GEMM launches: spread the cold experts' items among the hot ones
+    a0.interleave = a1.interleave = g_interleave.load();
     if (gated) {
         if (e == cudaSuccess)
             e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
@@ -795,6 +812,9 @@ moe_status moe_dispatch(const moe_problem *p, const int32_t *topk_idx, int32_t *
     d.chunk = at<int32_t>(ws, L.chunk);
     d.ptile_off = at<int32_t>(ws, L.ptile_off);
     d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
+    d.hot_off = at<int32_t>(ws, L.hot_off);
+    d.hot_tile_expert = at<int32_t>(ws, L.hot_tile_expert);
+    d.cold_tile = at<int32_t>(ws, L.cold_tile);
     d.ready = nullptr;
     d.n_ready = 0;
     d.row_w = nullptr;
@@ -907,6 +927,12 @@ int moe_set_gemm_mode(int mode)
         mode != MOE_GEMM_FUSED)
         return -1;
     return g_gemm_mode.exchange(mode);
+}
+
+int moe_set_work_order(int interleave)
+{
+    if (interleave != 0 && interleave != 1) return -1;
+    return g_interleave.exchange(interleave);
 }
 
 int moe_set_router_mode(int mode)

@@ -120,3 +120,5 @@ def test_forward_launch_count_follows_the_modes(lib):
         moe.moe_set_gemm_mode(prev_g)
     with pytest.raises(ValueError):
         moe.moe_set_router_mode(7)
+    with pytest.raises(ValueError):
+        moe.moe_set_work_order(2)

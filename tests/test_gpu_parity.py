@@ -372,6 +372,23 @@ def test_forward_with_filter_router():
     assert_out_close(out, ref, cfg.name)
 
 
+@pytest.mark.parametrize("name", ["skew_small", "skew"])
+def test_work_order_does_not_change_the_output(name):
+    """Interleaving single-tile experts' GEMM items among the others only reorders work: the
+    layer output is bitwise the same as in expert-major order."""
+    cfg = (cfg_small("skew_small", 900, 256, 192, 64, 4, zipf_s=1.2) if name == "skew_small"
+           else synth.CONFIGS["skew"])
+    inp = synth.make_inputs(cfg, seed=16, device="cuda")
+    outs = []
+    for order in (1, 0):
+        prev = moe.moe_set_work_order(order)
+        try:
+            outs.append(run_forward(cfg, inp)[0])
+        finally:
+            moe.moe_set_work_order(prev)
+    assert torch.equal(outs[0], outs[1])
+
+
 def test_gemm_variants_agree():
     """The single-CTA and CTA-pair grouped GEMMs compute the same layer."""
     cfg = cfg_small("variants", 700, 512, 640, 8, 2)
