@@ -101,9 +101,10 @@ typedef struct {
 MOE_API size_t moe_workspace_size(const moe_problem *p);
 
 /* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
- * current GEMM and router modes, assuming 16-byte aligned operands: the router (2, or 3
- * with the tensor-core filter), the dispatch (3) and the layers (3: layer0, layer1 and the
- * combine; 4 with the CTA-pair GEMM, which first gathers x; 1 with MOE_GEMM_FUSED).
+ * current GEMM and router modes, assuming 16-byte aligned operands: the
+ * router (2, or 3 with the tensor-core filter), the dispatch (3) and the layers (layer0,
+ * layer1 and the combine: 3; 4 with the CTA-pair GEMM, which first gathers x; 1 with
+ * MOE_GEMM_FUSED).
  * 0 for T == 0; -1 if *p is invalid. */
 MOE_API int moe_forward_launches(const moe_problem *p);
 
@@ -236,16 +237,22 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
 #define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
 
-/* Work order of the standalone grouped-GEMM launches (a tuning and test hook; not
- * thread-safe; results are bit-identical either way, every output tile is computed by one
- * CTA in one K order):
- * 0 (default): expert-major order (expert, then N tile, then M tile);
- * 1: the work items of experts with a single m-tile, whose weights are streamed for one
- *   tile only (HBM bound), are spread evenly among the items of the other experts (tensor
- *   bound), so both run at the same time. On the skewed layer this measured no gain: under
- *   the 1 kW cap the GEMMs are power-bound and the order does not change the energy.
- * Returns the previous setting, or -1 for another value. */
-MOE_API int moe_set_work_order(int interleave);
+/* Work order of the single-CTA grouped-GEMM launches (a tuning and test hook; not
+ * thread-safe). An expert with a single m-tile ("cold": at most m_tile routed rows) has its
+ * weights streamed for that one tile.
+ * MOE_ORDER_EXPERT: one launch per layer, expert-major (expert, then N tile, then M tile);
+ * MOE_ORDER_MIXED: the same launch with the cold experts' work items spread evenly among
+ *   the others' (measured no gain: the GEMMs are power-bound under the 1 kW cap);
+ * MOE_ORDER_NARROW (default): as MOE_ORDER_EXPERT, except that when every routed expert is
+ *   cold (decode-sized batches) the device runs the layer with the operands swapped (the
+ *   weight tile is the MMA's M = 128, the expert's rows rounded up to 16 its N): the same
+ *   weight bytes with far less tensor-core work (measured 5-7% faster per GEMM there).
+ * The layer outputs agree within the parity tolerance in every order; MOE_ORDER_EXPERT and
+ * MOE_ORDER_MIXED are bitwise identical. Returns the previous order, or -1. */
+#define MOE_ORDER_EXPERT 0
+#define MOE_ORDER_MIXED 1
+#define MOE_ORDER_NARROW 2
+MOE_API int moe_set_work_order(int order);
 
 /* Router variant (a tuning and test hook; not thread-safe). All give the same routing and
  * gates (the selection is always made on the sequential fp32 logits, see moe_route):

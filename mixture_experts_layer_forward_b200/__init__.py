@@ -34,6 +34,9 @@ from ._native import (  # noqa: F401
     moe_set_gemm_mode,
     moe_set_router_mode,
     moe_set_work_order,
+    ORDER_EXPERT,
+    ORDER_MIXED,
+    ORDER_NARROW,
     ROUTER_AUTO,
     ROUTER_SEQUENTIAL,
     ROUTER_FILTER,

@@ -252,6 +252,7 @@ def moe_set_wait_timeout_ns(ns: int) -> int:
 
 GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED = 0, 1, 2, 3
 ROUTER_AUTO, ROUTER_SEQUENTIAL, ROUTER_FILTER = 0, 1, 2
+ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW = 0, 1, 2
 
 
 def moe_set_fault_injection(layer0_item: int) -> int:
@@ -259,12 +260,12 @@ def moe_set_fault_injection(layer0_item: int) -> int:
     return int(library().moe_set_fault_injection(int(layer0_item)))
 
 
-def moe_set_work_order(interleave: int) -> int:
-    """0: expert-major GEMM work order (default); 1: spread single-tile experts' work among
-    the others. Returns the previous setting."""
-    rc = int(library().moe_set_work_order(int(interleave)))
+def moe_set_work_order(order: int) -> int:
+    """ORDER_EXPERT, ORDER_MIXED or ORDER_NARROW (default): how the single-CTA grouped GEMMs
+    treat experts with a single m-tile. Returns the previous order."""
+    rc = int(library().moe_set_work_order(int(order)))
     if rc < 0:
-        raise ValueError(f"unknown work order {interleave}")
+        raise ValueError(f"unknown work order {order}")
     return rc
 
 

@@ -69,6 +69,7 @@ constexpr uint32_t B_LBO = B_BOX; // next 64-column block
 } // namespace gemm
 
 enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2, GEMM_LOGITS = 3 };
+enum GemmOrder { ORDER_EXPERT = 0, ORDER_MIXED = 1 };
 
 struct GemmArgs {
     const int32_t *tile_off;    // [E+1] first m-tile of each expert
@@ -76,12 +77,14 @@ struct GemmArgs {
     const int32_t *ptile_off;   // [E+1] first m-tile pair of each expert (pair kernel)
     const int32_t *ptile_expert; // expert of each m-tile pair (pair kernel)
     const DispatchMeta *meta;   // num_tiles, num_cold
-    // interleave != 0: the work items of "cold" experts (one m-tile: weight-bandwidth bound)
-    // are spread evenly among those of the other ("hot", compute bound) experts, so HBM and
-    // the tensor cores are busy at the same time. hot_off [E+1] prefixes the hot experts'
-    // m-tiles, hot_tile_expert lists the expert of each hot m-tile, cold_tile the m-tile of
-    // each cold expert (written by the dispatch scan).
-    int interleave;
+    // Work order over the experts' m-tiles ("cold" experts have one m-tile, so their weight
+    // tiles are streamed for a single tile; the others are "hot"):
+    //   ORDER_EXPERT  expert-major over all m-tiles;
+    //   ORDER_MIXED   the cold experts' items spread evenly among the hot ones.
+    // hot_off [E+1] prefixes the hot experts' m-tiles, hot_tile_expert lists the expert of
+    // each hot m-tile, cold_tile the m-tile of each cold expert (written by the dispatch scan).
+    int order;
+    const int32_t *expert_rows; // [E] routed rows of each expert (narrow kernel)
     const int32_t *hot_off;
     const int32_t *hot_tile_expert;
     const int32_t *cold_tile;
@@ -126,7 +129,7 @@ __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, 
         ks = r / a.n_tiles;
         return;
     }
-    if (a.interleave) {
+    if (a.order == ORDER_MIXED) {
         const int64_t total = (int64_t)a.meta->num_tiles * a.n_tiles;
         const int64_t cold = (int64_t)a.meta->num_cold * a.n_tiles;
         const int64_t cb = (int64_t)w * cold / total;        // cold items before slot w
@@ -259,15 +262,13 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
     }
 }
 
+// The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
 template <int KIND>
-__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
-    moe_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                            const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+__device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                                 const GemmArgs &args, uint8_t *smem, int w_first,
+                                                 int w_step)
 {
     using namespace gemm;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE);
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
 #pragma unroll
             for (int i = 0; i < STAGES; ++i) armed[i] = -1;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            for (int w = w_first; ok && w < total; w += w_step) {
                 int e, mt, nt, ks;
                 gemm_map_work(w, args, e, mt, nt, ks);
                 for (int kb = kb_lo(ks); kb < kb_lo(ks + 1); ++kb) {
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             uint32_t ph = 0;
             int it = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
+            for (int w = w_first; ok && w < total; w += w_step, ++it) {
                 const int acc = it & 1;
                 const uint32_t aph = (uint32_t)(it >> 1) & 1u;
                 if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, args.timeout_ns,
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             const int r0 = g >> 3;
             int s = 0;
             uint32_t ph = 0;
-            for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            for (int w = w_first; w < total; w += w_step) {
                 int e, mt, nt;
                 gemm_map_work(w, args, e, mt, nt);
                 const __nv_bfloat16 *src[8];
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         int it = 0;
         int rs = 0;             // stage ring position (row_sq only)
         uint32_t rph = 0;
-        for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+        for (int w = w_first; w < total; w += w_step, ++it) {
             int e, mt, nt, ks;
             gemm_map_work(w, args, e, mt, nt, ks);
             if (row_sq) {
@@ -539,6 +540,17 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    grouped_gemm_cta<KIND>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
 }
 
 

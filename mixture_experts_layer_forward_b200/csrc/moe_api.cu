@@ -16,6 +16,7 @@
 #include "ptx.cuh"
 #include "route.cuh"
 #include "route_filter.cuh"
+#include "gemm_narrow.cuh"
 
 namespace {
 
@@ -29,9 +30,8 @@ std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fault_skip{-1};
 // router variant for many experts: MOE_ROUTER_AUTO (tensor-core filter) or sequential only
 std::atomic<int> g_router_mode{MOE_ROUTER_AUTO};
-// grouped-GEMM work order (test and tuning hook): expert-major by default; interleaving
-// the single-tile experts' items measured no gain on the skewed layer (power-bound GEMMs)
-std::atomic<int> g_interleave{0};
+// grouped-GEMM work order (MOE_ORDER_*; test and tuning hook)
+std::atomic<int> g_order{MOE_ORDER_NARROW};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -507,6 +507,24 @@ cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const
     return cudaGetLastError();
 }
 
+// One launch per layer; the device picks the narrow body when every expert owns a single
+// m-tile (moe_grouped_gemm_select_kernel).
+constexpr int SELECT_SMEM = gemm::SMEM_BYTES > gemmn::SMEM_BYTES ? gemm::SMEM_BYTES : gemmn::SMEM_BYTES;
+template <int KIND>
+cudaError_t launch_gemm_select(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &wide,
+                               const GemmArgs &narrow, cudaStream_t st)
+{
+    auto kern = moe_grouped_gemm_select_kernel<KIND>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SELECT_SMEM);
+    if (err != cudaSuccess) return err;
+    int grid = sm_count();
+    if (grid <= 0) grid = 148;
+    const int threads = wide.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    kern<<<grid, threads, SELECT_SMEM, st>>>(ta, tb, wide, narrow);
+    return cudaGetLastError();
+}
+
 template <int KIND>
 cudaError_t launch_gemm_any(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
                             int max_work, cudaStream_t st)
@@ -643,6 +661,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a0.tile_expert = d.tile_expert;
     a0.ptile_off = d.ptile_off;
     a0.ptile_expert = d.ptile_expert;
+    a0.expert_rows = d.counts;
     a0.hot_off = d.hot_off;
     a0.hot_tile_expert = d.hot_tile_expert;
     a0.cold_tile = d.cold_tile;
@@ -696,17 +715,34 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         return to_status(e);
     }
 
-    // standalone GEMM launches: spread the cold experts' items among the hot ones
-    a0.interleave = a1.interleave = g_interleave.load();
-    if (gated) {
+    // work order of the single-CTA launches; MOE_ORDER_NARROW lets the device run the
+    // operand-swapped body (N = the experts' row counts) when every expert is single-tile
+    const int order = g_order.load();
+    const bool narrow = (order == MOE_ORDER_NARROW) && !pair;
+    a0.order = a1.order = (order == MOE_ORDER_MIXED) ? ORDER_MIXED : ORDER_EXPERT;
+    GemmArgs n0 = a0, n1 = a1; // narrow items: column blocks of 64 (SwiGLU) or 128 columns
+    n0.n_tiles = gated ? F / 64 : (F + 127) / 128;
+    n1.n_tiles = (H + 127) / 128;
+    if (narrow) {
         if (e == cudaSuccess)
-            e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+            e = gated ? launch_gemm_select<GEMM_SWIGLU>(m_x, m_w1, a0, n0, st)
+                      : launch_gemm_select<GEMM_ACT>(m_x, m_w1, a0, n0, st);
+        if (e == cudaSuccess) e = record(events, n_events, 3, st);
+        if (e == cudaSuccess) e = launch_gemm_select<GEMM_SCALE>(m_h, m_w2, a1, n1, st);
+        if (e == cudaSuccess) e = record(events, n_events, 4, st);
     } else {
-        if (e == cudaSuccess) e = launch_gemm_any<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+        if (gated) {
+            if (e == cudaSuccess)
+                e = launch_gemm_any<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+        } else {
+            if (e == cudaSuccess)
+                e = launch_gemm_any<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+        }
+        if (e == cudaSuccess) e = record(events, n_events, 3, st);
+        if (e == cudaSuccess)
+            e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
+        if (e == cudaSuccess) e = record(events, n_events, 4, st);
     }
-    if (e == cudaSuccess) e = record(events, n_events, 3, st);
-    if (e == cudaSuccess) e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
-    if (e == cudaSuccess) e = record(events, n_events, 4, st);
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);
     return to_status(e);
@@ -929,10 +965,11 @@ int moe_set_gemm_mode(int mode)
     return g_gemm_mode.exchange(mode);
 }
 
-int moe_set_work_order(int interleave)
+int moe_set_work_order(int order)
 {
-    if (interleave != 0 && interleave != 1) return -1;
-    return g_interleave.exchange(interleave);
+    if (order != MOE_ORDER_EXPERT && order != MOE_ORDER_MIXED && order != MOE_ORDER_NARROW)
+        return -1;
+    return g_order.exchange(order);
 }
 
 int moe_set_router_mode(int mode)

@@ -100,7 +100,9 @@ def test_forward_launch_count_follows_the_modes(lib):
     decode = moe.Problem.from_config(synth.CONFIGS["skew_decode"])
     prev_r = moe.moe_set_router_mode(moe.ROUTER_AUTO)
     prev_g = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
+    prev_o = moe.moe_set_work_order(moe.ORDER_EXPERT)
     try:
+        # router 2 (3 with the filter) + dispatch 3 + layer0, layer1, combine
         assert moe.moe_forward_launches(mixtral) == 8   # E = 8: sequential router
         assert moe.moe_forward_launches(qwen2) == 9     # T*E >= 2^16: filter router
         assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential router
@@ -109,16 +111,19 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(mixtral) == 8   # the filter needs E > 16
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
         assert moe.moe_forward_launches(qwen2) == 8
+        moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
+        assert moe.moe_forward_launches(qwen2) == 8
         moe.moe_set_gemm_mode(moe.GEMM_FUSED)
         assert moe.moe_forward_launches(qwen2) == 6
-        moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)
+        moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)        # gathers x; no narrow launches
         assert moe.moe_forward_launches(qwen2) == 9
         assert moe.moe_forward_launches(moe.Problem.make(0, 128, 128, 8, 2)) == 0
         assert moe.moe_forward_launches(moe.Problem.make(4, 100, 128, 8, 2)) == -1  # H % 64
     finally:
         moe.moe_set_router_mode(prev_r)
         moe.moe_set_gemm_mode(prev_g)
+        moe.moe_set_work_order(prev_o)
     with pytest.raises(ValueError):
         moe.moe_set_router_mode(7)
     with pytest.raises(ValueError):
-        moe.moe_set_work_order(2)
+        moe.moe_set_work_order(3)

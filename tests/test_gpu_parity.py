@@ -372,21 +372,43 @@ def test_forward_with_filter_router():
     assert_out_close(out, ref, cfg.name)
 
 
-@pytest.mark.parametrize("name", ["skew_small", "skew"])
-def test_work_order_does_not_change_the_output(name):
-    """Interleaving single-tile experts' GEMM items among the others only reorders work: the
-    layer output is bitwise the same as in expert-major order."""
+@pytest.mark.parametrize("name", ["skew_small", "skew", "skew_decode"])
+def test_work_orders_agree(name):
+    """Expert-major and mixed orders only reorder work items: bitwise the same layer output.
+    The narrow kernel for single-tile experts computes the same products with the operands
+    swapped: within the parity tolerance of the others."""
     cfg = (cfg_small("skew_small", 900, 256, 192, 64, 4, zipf_s=1.2) if name == "skew_small"
-           else synth.CONFIGS["skew"])
+           else synth.CONFIGS[name])
     inp = synth.make_inputs(cfg, seed=16, device="cuda")
-    outs = []
-    for order in (1, 0):
+    outs = {}
+    for order in (moe.ORDER_EXPERT, moe.ORDER_MIXED, moe.ORDER_NARROW):
         prev = moe.moe_set_work_order(order)
         try:
-            outs.append(run_forward(cfg, inp)[0])
+            outs[order] = run_forward(cfg, inp)[0]
         finally:
             moe.moe_set_work_order(prev)
-    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(outs[moe.ORDER_EXPERT], outs[moe.ORDER_MIXED])
+    a = outs[moe.ORDER_EXPERT].float()
+    d = (outs[moe.ORDER_NARROW].float() - a).abs()
+    assert bool(torch.all(d <= ATOL + RTOL * a.abs())), float(d.max())
+
+
+@pytest.mark.parametrize("order", [0, 1, 2], ids=["expert", "mixed", "narrow"])
+def test_forward_orders_match_oracle(order):
+    """A mix of multi-tile and single-tile experts (ragged row counts, some experts empty)
+    against the oracle in every work order."""
+    cfg = cfg_small("orders", 700, 320, 256, 32, 3, zipf_s=1.5)
+    inp = synth.make_inputs(cfg, seed=17)
+    prev = moe.moe_set_work_order(order)
+    try:
+        out, idx, w, _ = run_forward(cfg, inp)
+    finally:
+        moe.moe_set_work_order(prev)
+    b = inp["bias"].numpy()
+    ref, ref_idx, _ = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                         bits(inp["W2"]), cfg.k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert_out_close(out, ref, f"order {order}")
 
 
 def test_gemm_variants_agree():
