@@ -16,4 +16,6 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
 
-    return oracle.load()
+    # test_oracle_mutants.py runs the pins against deliberately broken builds of the oracle
+    mutant = os.environ.get("ORACLE_LIB_UNDER_TEST")
+    return oracle.load(mutant) if mutant else oracle.load()

@@ -1,0 +1,76 @@
+"""The oracle's pins must catch plausible mistakes in the oracle itself.
+
+Each mutant below plants one slip in a copy of oracle/moe_oracle.c (a dropped term, a
+transposed operand, a wrong index, order or tie-break, a wrong constant or sign, a wider
+accumulator), builds it, and runs tests/test_oracle_pins.py against that build. Every mutant
+must make at least one pin fail. Mutations that leave the result mathematically unchanged
+(for example dropping the max shift of the softmax) are not mistakes and are not listed.
+"""
+import os
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+from pathlib import Path
+
+import pytest
+
+import oracle
+
+ROOT = Path(__file__).resolve().parents[1]
+SRC = ROOT / "oracle" / "moe_oracle.c"
+
+MUTANTS = [
+    ("router_wider_accumulator", "float acc = 0.0f;", "double acc = 0.0;"),
+    ("router_h_descending",
+     "for (int h = 0; h < H; ++h) {\n                float p",
+     "for (int h = H - 1; h >= 0; --h) {\n                float p"),
+    ("router_drops_bias", "if (bias) acc = acc + bias[e];", ""),
+    ("router_transposed_gate", "bf16_to_float(Wg[(size_t)h * E + e])",
+     "bf16_to_float(Wg[(size_t)e * H + h])"),
+    ("topk_ties_to_higher_id", "l[e] > l[best]", "l[e] >= l[best]"),
+    ("gates_over_all_experts", "if (gate == ORACLE_GATE_SOFTMAX_ALL) {",
+     "if (gate != ORACLE_GATE_SOFTMAX_ALL) {"),
+    ("silu_wrong_sign", "z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
+    ("swiglu_gate_up_swapped", "silu(z[f]) * z[F + f]", "silu(z[F + f]) * z[f]"),
+    ("gelu_wrong_constant", "0.044715", "0.04715"),
+    ("w2_transposed", "y[n] += a * (double)bf16_to_float(wrow[n]);",
+     "y[n] += a * (double)bf16_to_float(W2e[(size_t)n * F + f]);"),
+    ("ffn_first_x_only", "double xh = (double)bf16_to_float(xrow[h]);",
+     "double xh = (double)bf16_to_float(xrow[0]);"),
+    ("combine_drops_gate", "s += w[(size_t)t * k + j] * y[(size_t)r * H + n];",
+     "s += y[(size_t)r * H + n];"),
+    ("token_path_drops_gate", "o[n] += w[j] * y[n];", "o[n] += y[n];"),
+    ("dispatch_pads_down", "((counts[e] + m_tile - 1) / m_tile) * m_tile",
+     "(counts[e] / m_tile) * m_tile"),
+    ("dispatch_not_stable",
+     "for (int t = 0; t < T; ++t) {\n        for (int j = 0; j < k; ++j) {\n            int e = idx[(size_t)t * k + j];\n            int r = poff[e] + cursor[e];",
+     "for (int t = T - 1; t >= 0; --t) {\n        for (int j = 0; j < k; ++j) {\n            int e = idx[(size_t)t * k + j];\n            int r = poff[e] + cursor[e];"),
+    ("bf16_ties_away_from_zero", "nearbyint(scaled)", "round(scaled)"),
+    ("bf16_seven_bits", "ldexp(m, 8)", "ldexp(m, 7)"),
+]
+
+
+def _run_mutant(tmp_path, name, old, new):
+    text = SRC.read_text()
+    if text.count(old) != 1:
+        return f"{name}: the mutation site is not unique"
+    d = tmp_path / name
+    d.mkdir()
+    src = d / "moe_oracle.c"
+    src.write_text(text.replace(old, new))
+    lib = oracle.build(force=True, src=src, out=d / "liboracle_mutant.so")
+    env = dict(os.environ, ORACLE_LIB_UNDER_TEST=str(lib), OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", str(ROOT / "tests" / "test_oracle_pins.py"),
+                        "-x", "-q", "-p", "no:cacheprovider"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    if r.returncode != 1:
+        return f"{name}: no pin failed (exit {r.returncode})\n{r.stdout[-1500:]}"
+    return None
+
+
+def test_pins_catch_every_mutant(tmp_path):
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        results = list(ex.map(lambda m: _run_mutant(tmp_path, *m), MUTANTS))
+    missed = [r for r in results if r]
+    assert not missed, "\n".join(missed)
