@@ -34,7 +34,12 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DOMINANT_KERNEL = "moe_grouped_gemm_kernel<0>"  # layer0 grouped GEMM + SwiGLU
+# layer0 grouped GEMM + SwiGLU, by GEMM mode (the single-CTA launch is the select kernel,
+# which runs the 128-row body, or the operand-swapped one when every expert is single-tile)
+DOMINANT_KERNEL = {"auto": "moe_grouped_gemm_select_kernel<0>",
+                   "single": "moe_grouped_gemm_select_kernel<0>",
+                   "pair": "moe_grouped_gemm_pair_kernel<0>",
+                   "fused": "moe_fused_layer_kernel<0>"}
 
 
 def parse_args():
@@ -309,10 +314,12 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     args_fwd = (p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out, ws)
 
+    idx_buf = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
     for _ in range(W):
-        moe.moe_forward(*args_fwd)
+        moe.moe_forward(*args_fwd, idx_buf)
     torch.cuda.synchronize(dev)
     assert moe.moe_get_device_status(ws) == 0, "device status after warm-up"
+    active_experts = int(torch.unique(idx_buf).numel())  # for the layer0 byte count below
 
     # stage events of every timed step (recorded on the launch stream by the library)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGE_EVENTS)]
@@ -380,14 +387,28 @@ def run_ours(args):
     regime = "sustained" if sustained else "burst"
     tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
     layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
-    gemm0_flops = (4 if cfg.act == 0 else 2) * cfg.T * cfg.k * cfg.H * cfg.F
+    # layer0: useful FLOPs (padding rows not counted) and algorithmic bytes (each active
+    # expert's W1 once, x once, h of the routed rows written once); the bound is whichever
+    # takes longer at the measured peaks
+    w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
+    gemm0_flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
+    gemm0_bytes = 2 * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H + cfg.T * cfg.k * cfg.F)
     g0_ms = stage_ms["layer0_gemm_swiglu"]
-    g0_tflops = gemm0_flops / (g0_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": DOMINANT_KERNEL, "achieved": g0_tflops,
-                "peak": tf_peak, "unit": "TFLOP/s", "frac": g0_tflops / tf_peak,
-                "traffic": traffic_for(DOMINANT_KERNEL, cfg.name),
-                "peak_source": f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)",
-                "algorithmic_flops_per_launch": gemm0_flops, "ms_per_launch": g0_ms}
+    g0_s = g0_ms / 1e3
+    kernel = DOMINANT_KERNEL[args.gemm_mode]
+    hbm_bound = gemm0_bytes / (peaks["hbm_gbs"] * 1e9) > gemm0_flops / (tf_peak * 1e12)
+    if hbm_bound:
+        achieved, peak, unit = gemm0_bytes / g0_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        psrc = f"{peak_src} HBM copy bandwidth"
+    else:
+        achieved, peak, unit = gemm0_flops / g0_s / 1e12, tf_peak, "TFLOP/s"
+        psrc = f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)"
+    roofline = {"bound": "hbm" if hbm_bound else "tensor", "kernel": kernel,
+                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic_for(kernel, cfg.name), "peak_source": psrc,
+                "algorithmic_flops_per_launch": gemm0_flops,
+                "algorithmic_bytes_per_launch": gemm0_bytes, "active_experts": active_experts,
+                "ms_per_launch": g0_ms}
 
     line = {
         "metric": "MoE-layer forward tokens/s", "value": n * cfg.T / (ms_per_step / 1e3),
