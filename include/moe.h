@@ -73,10 +73,15 @@ typedef enum {
  * SOFTMAX_TOPK: softmax over the k selected logits. In exact arithmetic this equals a
  *   softmax over all E logits renormalised over the selected k (Mixtral's "softmax over
  *   the top-k logits" and Qwen2's "renormalised top-k gates" are the same function).
- * SOFTMAX_ALL: the full-E softmax values of the selected experts, not renormalised. */
+ * SOFTMAX_ALL: the full-E softmax values of the selected experts, not renormalised.
+ * SELECT_BIAS: the bias steers the selection only (load balancing by a per-expert bias
+ *   instead of an auxiliary loss): experts are selected by the logit plus bias[e] (the
+ *   same fp32 sum as in the other modes), and the gates are the softmax over the k selected
+ *   experts' logits without the bias. With a NULL bias it equals SOFTMAX_TOPK. */
 typedef enum {
     MOE_GATE_SOFTMAX_TOPK = 0,
-    MOE_GATE_SOFTMAX_ALL = 1
+    MOE_GATE_SOFTMAX_ALL = 1,
+    MOE_GATE_SELECT_BIAS = 2
 } moe_gate;
 
 typedef struct {

@@ -15,6 +15,7 @@ from ._native import (  # noqa: F401
     ACT_RELU,
     ACT_SWIGLU,
     GATE_SOFTMAX_ALL,
+    GATE_SELECT_BIAS,
     GATE_SOFTMAX_TOPK,
     MOE_NUM_STAGE_EVENTS,
     MoeError,

@@ -16,7 +16,7 @@ import torch
 from .build import LIB_PATH
 
 ACT_SWIGLU, ACT_GELU_TANH, ACT_RELU, ACT_IDENTITY = 0, 1, 2, 3
-GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL = 0, 1
+GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL, GATE_SELECT_BIAS = 0, 1, 2
 MOE_NUM_STAGE_EVENTS = 6
 M_TILE = 128
 

@@ -43,7 +43,9 @@ moe_status check_problem(const moe_problem *p)
     if (p->T < 0 || p->H <= 0 || p->F <= 0 || p->E <= 0 || p->top_k <= 0) return MOE_ERR_INVALID_ARG;
     if (p->top_k > p->E) return MOE_ERR_INVALID_ARG;
     if (p->act < MOE_ACT_SWIGLU || p->act > MOE_ACT_IDENTITY) return MOE_ERR_INVALID_ARG;
-    if (p->gate != MOE_GATE_SOFTMAX_TOPK && p->gate != MOE_GATE_SOFTMAX_ALL) return MOE_ERR_INVALID_ARG;
+    if (p->gate != MOE_GATE_SOFTMAX_TOPK && p->gate != MOE_GATE_SOFTMAX_ALL &&
+        p->gate != MOE_GATE_SELECT_BIAS)
+        return MOE_ERR_INVALID_ARG;
     if (p->m_tile != M_TILE) return MOE_ERR_UNSUPPORTED;
     if (p->H % 64 != 0 || p->F % 64 != 0) return MOE_ERR_UNSUPPORTED;
     if (p->E > 1024) return MOE_ERR_UNSUPPORTED;
@@ -89,7 +91,7 @@ FilterPlan filter_plan(const moe_problem *p)
     FilterPlan f{false, 1, 0, 0, 0, 0.0f};
     const int T = p->T, H = p->H, E = p->E;
     if (T <= 0 || E <= 16 || E > RF_MAX_E || (E % 8) != 0 || (H % gemm::BK) != 0 ||
-        p->gate != MOE_GATE_SOFTMAX_TOPK || (int64_t)T * E >= (1LL << 31) / RF_SPLIT_MAX)
+        p->gate == MOE_GATE_SOFTMAX_ALL || (int64_t)T * E >= (1LL << 31) / RF_SPLIT_MAX)
         return f;
     const int kb = H / gemm::BK;
     const int tiles = ((T + gemm::BM - 1) / gemm::BM) * ((E + gemm::BN - 1) / gemm::BN);
@@ -347,6 +349,7 @@ cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
     r.bt = fp.bt;
     r.ring_bytes = fp.ring_bytes;
     r.cA = fp.cA;
+    r.gate = p->gate;
     r.status = status;
     r.timeout_ns = g_timeout_ns.load();
     const size_t smem = fp.smem;
@@ -383,20 +386,22 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     // blocks of the large-E tile (64 tokens x 64 experts); fewer than the SMs: go narrow
     const int64_t large_blocks = (int64_t)((T + 63) / 64) * ((E + 63) / 64);
     const int sms = sm_count() > 0 ? sm_count() : 148;
+    // selection bias: the logits stay without it, the top-k kernel adds it to the keys
+    const float *lbias = (p->gate == MOE_GATE_SELECT_BIAS) ? nullptr : bias;
     if (E <= 8 && T >= 64 * sms / 2) {
-        launch_route_logits<ROUTE_SMALL_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+        launch_route_logits<ROUTE_SMALL_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     } else if (E > 8 && E <= 16 && T >= 32 * sms / 2) {
-        launch_route_logits<ROUTE_MID_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+        launch_route_logits<ROUTE_MID_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     } else if (E > 16 && large_blocks >= sms / 2) {
-        launch_route_logits<ROUTE_LARGE_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+        launch_route_logits<ROUTE_LARGE_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     } else {
-        launch_route_logits<ROUTE_NARROW_CFG>(xb, wb, bias, logits, T, H, E, status, st);
+        launch_route_logits<ROUTE_NARROW_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)TOPK_WARPS * E * sizeof(float);
     route_topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(
-        logits, topk_idx, topk_w, T, E, p->top_k, p->gate);
+        logits, topk_idx, topk_w, T, E, p->top_k, p->gate, bias);
     return cudaGetLastError();
 }
 

@@ -255,9 +255,13 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
 constexpr int TOPK_WARPS = 8; // tokens per block
 
 // One warp per token. Dynamic shared memory: TOPK_WARPS * E floats.
+// gate 2 (selection bias): `logits` are without the bias; the selection keys are
+// logits[t][e] + bias[e] (the same fp32 addition the logits kernel makes in the other
+// modes) and the gates use the logits without the bias, shifted by their maximum.
 __global__ void __launch_bounds__(TOPK_WARPS * 32)
     route_topk_kernel(const float *__restrict__ logits, int32_t *__restrict__ topk_idx,
-                      float *__restrict__ topk_w, int T, int E, int k, int gate)
+                      float *__restrict__ topk_w, int T, int E, int k, int gate,
+                      const float *__restrict__ bias)
 {
     extern __shared__ float srow[];
     const int warp = threadIdx.x >> 5;
@@ -266,7 +270,8 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
     if (t >= T) return;
     float *row = srow + (size_t)warp * E;
     const float *lg = logits + (size_t)t * E;
-    for (int e = lane; e < E; e += 32) row[e] = lg[e];
+    const bool sel_bias = (gate == 2) && bias != nullptr;
+    for (int e = lane; e < E; e += 32) row[e] = sel_bias ? lg[e] + bias[e] : lg[e];
     __syncwarp();
 
     float sel_val = 0.0f; // lane j keeps the j-th selected logit (j < k <= 32 covered below)
@@ -287,14 +292,22 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
         // every lane now holds the winner (bv, bi); a non-finite row (unsupported input)
         // must still not index outside the row
         if (bi < 0 || bi >= E) bi = 0;
-        if (j == 0) top = bv;
+        const float gv = (gate == 2) ? lg[bi] : bv; // the gate's logit (no bias in mode 2)
+        if (j == 0) top = gv;
         if (lane == 0) {
             topk_idx[(size_t)t * k + j] = bi;
             row[bi] = -INFINITY; // removed from later rounds (logits are finite)
         }
-        if (j < 32 && j == lane) sel_val = bv;
-        if (j >= 32 && lane == 0) topk_w[(size_t)t * k + j] = bv; // stash; rescaled below
+        if (j < 32 && j == lane) sel_val = gv;
+        if (j >= 32 && lane == 0) topk_w[(size_t)t * k + j] = gv; // stash; rescaled below
         __syncwarp();
+    }
+    if (gate == 2) { // the largest selected logit (the first selected one need not be)
+        float m = -INFINITY;
+        for (int j = lane; j < k; j += 32) m = fmaxf(m, (j < 32) ? sel_val : topk_w[(size_t)t * k + j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        top = m;
     }
 
     // gate weights: w_j = exp(l_j - l_0) / denom

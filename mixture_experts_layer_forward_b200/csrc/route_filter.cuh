@@ -140,6 +140,7 @@ struct RfArgs {
     int T, H, E, k, S, bt;
     int ring_bytes;           // bytes of the chunk ring (region 0)
     float cA;                 // interval coefficient of ||x|| ||w||
+    int gate;                 // MOE_GATE_SOFTMAX_TOPK, or 2: the bias steers the selection only
     int *status;
     int64_t timeout_ns;
 };
@@ -431,21 +432,17 @@ __global__ void __launch_bounds__(RF_THREADS)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar(slot));
             }
-            if (ok && active) {
-                float v0 = acc0;
-                if (a.bias != nullptr) v0 = v0 + a.bias[e0];
-                exact[tl * E + e0] = v0;
-                if (e1 < E) {
-                    float v1 = acc1;
-                    if (a.bias != nullptr) v1 = v1 + a.bias[e1];
-                    exact[tl * E + e1] = v1;
-                }
+            if (ok && active) { // the sequential logits without the bias
+                exact[tl * E + e0] = acc0;
+                if (e1 < E) exact[tl * E + e1] = acc1;
             }
         }
     }
     __syncthreads(); // exact logits complete
 
     // ---- d. top k of the candidates' exact logits (ties to the lower id) and the gates ----
+    // Selection key: logit + bias (one fp32 addition, as the sequential router's logits);
+    // gate value: the key, or with the selection bias (gate 2) the logit without the bias.
     for (int tl = warp; tl < nt; tl += RF_WARPS) {
         const int t = t0 + tl;
         const float *row = exact + tl * E;
@@ -458,13 +455,14 @@ __global__ void __launch_bounds__(RF_THREADS)
             int best = (int)0x80000000, bi = 0x7fffffff;
             for (int e = lane, i = 0; e < E; e += 32, ++i) {
                 if ((removed >> i) & 1u) continue;
-                const int key = rf_key(row[e]);
+                const float v = (a.bias != nullptr) ? row[e] + a.bias[e] : row[e];
+                const int key = rf_key(v);
                 if (key > best) { best = key; bi = e; } // e ascending: keeps the lower id
             }
             const int mx = __reduce_max_sync(0xffffffffu, best);
             int w = (int)__reduce_min_sync(0xffffffffu, (unsigned)(best == mx ? bi : 0x7fffffff));
             if (w < 0 || w >= E) w = 0; // unsupported non-finite rows still index the row
-            const float bv = rf_unkey(mx);
+            const float bv = (a.gate == 2) ? row[w] : rf_unkey(mx);
             if ((w & 31) == lane) removed |= 1u << (w >> 5);
             if (j == 0) top = bv;
             if (lane == 0) a.topk_idx[(size_t)t * k + j] = w;
@@ -472,6 +470,14 @@ __global__ void __launch_bounds__(RF_THREADS)
             if (j >= 32 && lane == 0) a.topk_w[(size_t)t * k + j] = bv;
         }
         __syncwarp();
+        if (a.gate == 2) { // the largest selected logit (the first selected one need not be)
+            float m = -INFINITY;
+            for (int j = lane; j < k; j += 32)
+                m = fmaxf(m, (j < 32) ? sel_val : a.topk_w[(size_t)t * k + j]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            top = m;
+        }
         float denom = 0.0f;
         for (int j = lane; j < k; j += 32) {
             const float v = (j < 32) ? sel_val : a.topk_w[(size_t)t * k + j];

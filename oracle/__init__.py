@@ -23,7 +23,7 @@ _SRC = _HERE / "moe_oracle.c"
 _LIB = _HERE / "liboracle.so"
 
 ACT_SWIGLU, ACT_GELU_TANH, ACT_RELU, ACT_IDENTITY = 0, 1, 2, 3
-GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL = 0, 1
+GATE_SOFTMAX_TOPK, GATE_SOFTMAX_ALL, GATE_SELECT_BIAS = 0, 1, 2
 
 # Portable flags: the library may be built on one host and run on another.
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fopenmp"]
@@ -56,6 +56,8 @@ def load(path: Path | None = None) -> ctypes.CDLL:
     lib.oracle_router_logits.restype = None
     lib.oracle_topk_gates.argtypes = [i32, i32, i32, i32, vp, vp, vp]
     lib.oracle_topk_gates.restype = i32
+    lib.oracle_topk_gates_bias.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.oracle_topk_gates_bias.restype = i32
     lib.oracle_dispatch.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, i64]
     lib.oracle_dispatch.restype = i32
     lib.oracle_expert_ffn_row.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
@@ -97,13 +99,15 @@ def router_logits(x, Wg, bias=None, lib=None):
     return out
 
 
-def topk_gates(logits, k, gate=GATE_SOFTMAX_TOPK, lib=None):
+def topk_gates(logits, k, gate=GATE_SOFTMAX_TOPK, lib=None, bias=None):
+    """bias: used by GATE_SELECT_BIAS only (the logits then exclude it)."""
     lib = lib or load()
     logits = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = logits.shape
     idx = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
-    rc = lib.oracle_topk_gates(T, E, k, gate, _p(logits), _p(idx), _p(w))
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    rc = lib.oracle_topk_gates_bias(T, E, k, gate, _p(logits), _p(b), _p(idx), _p(w))
     if rc:
         raise ValueError(f"oracle_topk_gates rc={rc}")
     return idx, w

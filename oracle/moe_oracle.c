@@ -23,7 +23,9 @@
  *   - selection: the k largest logits, ties broken toward the lower expert id;
  *   - gates: softmax over the k selected logits (equal, in exact arithmetic, to a softmax
  *     over all E followed by renormalisation over the selected k); a second mode keeps
- *     the full-E softmax values without renormalisation;
+ *     the full-E softmax values without renormalisation; a third (a load-balancing bias
+ *     that steers the selection only, not on the pages) selects by logit + bias and takes
+ *     the gates from the logits without the bias;
  *   - experts: SwiGLU with W1 [E, H, 2F] (columns [0,F) gate, [F,2F) up) or a plain
  *     activation with W1 [E, H, F]; W2 is [E, F, H];
  *   - no capacity limit: every routed (token, expert) pair is computed;
@@ -53,6 +55,7 @@
 
 #define ORACLE_GATE_SOFTMAX_TOPK 0
 #define ORACLE_GATE_SOFTMAX_ALL 1
+#define ORACLE_GATE_SELECT_BIAS 2
 
 /* ---------------------------------------------------------------------------------------
  * bf16 helpers
@@ -103,27 +106,38 @@ void oracle_router_logits(int T, int H, int E, const uint16_t *x, const uint16_t
 }
 
 /* Top-k selection and gate weights for one token.
- * Selection: repeatedly take the largest remaining logit; on equal values the lower
- * expert id wins (scan ascending, replace only on strictly greater). Equal compares as
- * floats, so +0 and -0 tie.
+ * Selection: repeatedly take the largest remaining key; on equal keys the lower expert id
+ * wins (scan ascending, replace only on strictly greater). Equal compares as floats, so +0
+ * and -0 tie. The key is the logit, or for SELECT_BIAS the fp32 sum l[e] + bias[e] (the
+ * same single addition that adds the bias to the logits in the other modes).
  * Gates (fp64):
  *   SOFTMAX_TOPK: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0), i, j over the selected k;
  *   SOFTMAX_ALL : w_j = exp(l_j - l_0) / sum_e exp(l_e - l_0), e over all E
- *                 (l_0 is the largest logit in both cases). */
-static void topk_one(int E, int k, int gate, const float *l, int32_t *idx, double *w,
-                     unsigned char *taken)
+ *                 (l_0 is the largest logit in both cases);
+ *   SELECT_BIAS : as SOFTMAX_TOPK on the logits without the bias, shifted by the largest
+ *                 of them. */
+static float sel_key(int gate, const float *l, const float *bias, int e)
+{
+    return (gate == ORACLE_GATE_SELECT_BIAS && bias) ? l[e] + bias[e] : l[e];
+}
+
+static void topk_one(int E, int k, int gate, const float *l, const float *bias, int32_t *idx,
+                     double *w, unsigned char *taken)
 {
     memset(taken, 0, (size_t)E);
     for (int j = 0; j < k; ++j) {
         int best = -1;
         for (int e = 0; e < E; ++e) {
             if (taken[e]) continue;
-            if (best < 0 || l[e] > l[best]) best = e;
+            if (best < 0 || sel_key(gate, l, bias, e) > sel_key(gate, l, bias, best)) best = e;
         }
         taken[best] = 1;
         idx[j] = best;
     }
     double m = (double)l[idx[0]];
+    if (gate == ORACLE_GATE_SELECT_BIAS)
+        for (int j = 1; j < k; ++j)
+            if ((double)l[idx[j]] > m) m = (double)l[idx[j]];
     double denom = 0.0;
     if (gate == ORACLE_GATE_SOFTMAX_ALL) {
         for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
@@ -133,8 +147,10 @@ static void topk_one(int E, int k, int gate, const float *l, int32_t *idx, doubl
     for (int j = 0; j < k; ++j) w[j] = exp((double)l[idx[j]] - m) / denom;
 }
 
-/* logits: [T,E] fp32 -> idx: [T,k] int32 (in selection order), w: [T,k] fp64. */
-int oracle_topk_gates(int T, int E, int k, int gate, const float *logits, int32_t *idx, double *w)
+/* logits: [T,E] fp32 -> idx: [T,k] int32 (in selection order), w: [T,k] fp64.
+ * bias [E] (or NULL) is used by SELECT_BIAS only; the logits then exclude it. */
+int oracle_topk_gates_bias(int T, int E, int k, int gate, const float *logits, const float *bias,
+                           int32_t *idx, double *w)
 {
     if (T < 0 || E < 1 || k < 1 || k > E) return -1;
     int bad = 0;
@@ -148,11 +164,17 @@ int oracle_topk_gates(int T, int E, int k, int gate, const float *logits, int32_
                 bad = 1;
                 continue;
             }
-            topk_one(E, k, gate, logits + (size_t)t * E, idx + (size_t)t * k, w + (size_t)t * k, taken);
+            topk_one(E, k, gate, logits + (size_t)t * E, bias, idx + (size_t)t * k,
+                     w + (size_t)t * k, taken);
         }
         free(taken);
     }
     return bad ? -2 : 0;
+}
+
+int oracle_topk_gates(int T, int E, int k, int gate, const float *logits, int32_t *idx, double *w)
+{
+    return oracle_topk_gates_bias(T, E, k, gate, logits, NULL, idx, w);
 }
 
 /* ---------------------------------------------------------------------------------------
@@ -344,9 +366,9 @@ int oracle_moe_forward(int T, int H, int F, int E, int k, int act, int gate, int
         goto done;
     }
 
-    /* 1. route */
-    oracle_router_logits(T, H, E, x, Wg, bias, logits);
-    rc = oracle_topk_gates(T, E, k, gate, logits, idx, w);
+    /* 1. route (with a selection-only bias the logits exclude it) */
+    oracle_router_logits(T, H, E, x, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, logits);
+    rc = oracle_topk_gates_bias(T, E, k, gate, logits, bias, idx, w);
     if (rc) goto done;
 
     /* 2. dispatch */
@@ -451,8 +473,9 @@ int oracle_moe_tokens(int T, int H, int F, int E, int k, int act, int gate, int 
             }
             {
                 int t = tokens[i];
-                oracle_router_logits(1, H, E, x + (size_t)t * H, Wg, bias, l);
-                topk_one(E, k, gate, l, sel, w, taken);
+                oracle_router_logits(1, H, E, x + (size_t)t * H, Wg,
+                                     gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, l);
+                topk_one(E, k, gate, l, bias, sel, w, taken);
                 double *o = out + (size_t)i * H;
                 for (int n = 0; n < H; ++n) o[n] = 0.0;
                 for (int j = 0; j < k; ++j) {

@@ -86,6 +86,10 @@ ROUTE_CASES = [
     ("e8_tile", 5000, 192, 8, 2, False, 0.0, 0),
     ("e16_tile", 2500, 320, 16, 2, True, 0.0, 0),
     ("e320_tile", 2100, 128, 320, 8, False, 1.2, 0),
+    # selection-only bias (gate 2): SIMT top-k, and the filter's finalize
+    ("e8_selbias", 300, 256, 8, 2, False, 1.2, 2),
+    ("e64_selbias", 130, 384, 64, 8, False, 1.2, 2),
+    ("e256_selbias_tile", 2100, 128, 256, 8, False, 1.2, 2),
 ]
 
 
@@ -108,9 +112,11 @@ def test_route_bit_exact(case, router_mode):
     bias = inp["bias"].cuda() if inp["bias"] is not None else None
     moe.moe_route(p, inp["x"].cuda(), inp["Wg"].cuda(), bias, idx, w, ws)
     assert moe.moe_get_device_status(ws) == 0
+    b = None if bias is None else inp["bias"].numpy()
+    # with the selection-only bias the logits exclude it and the top-k adds it to the keys
     logits = oracle.router_logits(bits(inp["x"]), bits(inp["Wg"]),
-                                  None if bias is None else inp["bias"].numpy())
-    ref_idx, ref_w = oracle.topk_gates(logits, k, gate=gate)
+                                  None if gate == moe.GATE_SELECT_BIAS else b)
+    ref_idx, ref_w = oracle.topk_gates(logits, k, gate=gate, bias=b)
     assert np.array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
 
@@ -152,10 +158,11 @@ def test_route_rounding_level_ties(router_mode, unscaled):
     np.testing.assert_allclose(got_w, ref_w, rtol=1e-5, atol=1e-7)
 
 
-def test_route_filter_matches_sequential_bitwise():
+@pytest.mark.parametrize("gate", [0, 2], ids=["softmax_topk", "select_bias"])
+def test_route_filter_matches_sequential_bitwise(gate):
     """Both router variants give bit-identical indices and gates (the gates are computed from
     the same sequential fp32 logits)."""
-    cfg = cfg_small("filter_vs_seq", 1000, 512, 64, 128, 8, zipf_s=1.2)
+    cfg = cfg_small("filter_vs_seq", 1000, 512, 64, 128, 8, zipf_s=1.2, gate=gate)
     inp = synth.make_inputs(cfg, seed=22)
     p = moe.Problem.from_config(cfg)
     res = []
@@ -409,6 +416,25 @@ def test_forward_orders_match_oracle(order):
                                          bits(inp["W2"]), cfg.k)
     assert np.array_equal(idx.cpu().numpy(), ref_idx)
     assert_out_close(out, ref, f"order {order}")
+
+
+def test_forward_with_selection_bias():
+    """The whole layer with the selection-only bias (a strong Zipf prior steers the choice,
+    the gates ignore it), on the sequential and the filter router."""
+    cfg = cfg_small("selbias_fwd", 400, 256, 192, 64, 4, zipf_s=1.5, gate=moe.GATE_SELECT_BIAS)
+    inp = synth.make_inputs(cfg, seed=18)
+    b = inp["bias"].numpy()
+    ref, ref_idx, ref_w = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                             bits(inp["W2"]), cfg.k, gate=cfg.gate)
+    for mode in (moe.ROUTER_SEQUENTIAL, moe.ROUTER_FILTER):
+        prev = moe.moe_set_router_mode(mode)
+        try:
+            out, idx, w, _ = run_forward(cfg, inp)
+        finally:
+            moe.moe_set_router_mode(prev)
+        assert np.array_equal(idx.cpu().numpy(), ref_idx)
+        np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+        assert_out_close(out, ref, f"selection bias, router {mode}")
 
 
 def test_gemm_variants_agree():

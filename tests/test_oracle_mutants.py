@@ -27,7 +27,8 @@ MUTANTS = [
     ("router_drops_bias", "if (bias) acc = acc + bias[e];", ""),
     ("router_transposed_gate", "bf16_to_float(Wg[(size_t)h * E + e])",
      "bf16_to_float(Wg[(size_t)e * H + h])"),
-    ("topk_ties_to_higher_id", "l[e] > l[best]", "l[e] >= l[best]"),
+    ("topk_ties_to_higher_id", "sel_key(gate, l, bias, e) > sel_key(gate, l, bias, best)",
+     "sel_key(gate, l, bias, e) >= sel_key(gate, l, bias, best)"),
     ("gates_over_all_experts", "if (gate == ORACLE_GATE_SOFTMAX_ALL) {",
      "if (gate != ORACLE_GATE_SOFTMAX_ALL) {"),
     ("silu_wrong_sign", "z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
@@ -47,13 +48,17 @@ MUTANTS = [
      "for (int t = T - 1; t >= 0; --t) {\n        for (int j = 0; j < k; ++j) {\n            int e = idx[(size_t)t * k + j];\n            int r = poff[e] + cursor[e];"),
     ("bf16_ties_away_from_zero", "nearbyint(scaled)", "round(scaled)"),
     ("bf16_seven_bits", "ldexp(m, 8)", "ldexp(m, 7)"),
+    ("select_bias_logits_keep_bias",
+     "oracle_router_logits(T, H, E, x, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, logits);",
+     "oracle_router_logits(T, H, E, x, Wg, bias, logits);"),
+    ("select_bias_ignored_in_selection", "? l[e] + bias[e] : l[e];", "? l[e] : l[e];"),
 ]
 
 
 def _run_mutant(tmp_path, name, old, new):
     text = SRC.read_text()
     if text.count(old) != 1:
-        return f"{name}: the mutation site is not unique"
+        return f"{name}: the mutation site is missing or not unique"
     d = tmp_path / name
     d.mkdir()
     src = d / "moe_oracle.c"

@@ -175,6 +175,37 @@ def test_gates_match_full_softmax_then_renormalise(oracle_lib):
     assert np.all(w1 == 1.0)
 
 
+def test_selection_bias_closed_form(oracle_lib):
+    """SELECT_BIAS: the bias decides which experts are selected, the gates come from the
+    logits without it (hand-worked: raw logits [3, 1, 2, 0], bias [0, 5, 0, 4] give keys
+    [3, 6, 2, 4], so experts 1 then 3; gates softmax([1, 0]) shifted by its max, 1)."""
+    x = bf16([[1.0, 1.0]])
+    Wg = bf16([[2.0, 0.0, 1.0, 0.0], [1.0, 1.0, 1.0, 0.0]])      # logits [3, 1, 2, 0]
+    bias = np.array([0.0, 5.0, 0.0, 4.0], np.float32)
+    raw = oracle.router_logits(x, Wg, None, lib=oracle_lib)
+    assert raw.tolist() == [[3.0, 1.0, 2.0, 0.0]]
+    idx, w = oracle.topk_gates(raw, 2, gate=oracle.GATE_SELECT_BIAS, bias=bias, lib=oracle_lib)
+    assert idx.tolist() == [[1, 3]]
+    e1 = math.exp(-1.0)
+    np.testing.assert_allclose(w, [[1 / (1 + e1), e1 / (1 + e1)]], rtol=1e-15)
+    # SOFTMAX_TOPK on the biased logits selects the same experts but gates by [6, 4]
+    idx0, w0 = oracle.topk_gates(oracle.router_logits(x, Wg, bias, lib=oracle_lib), 2,
+                                 lib=oracle_lib)
+    e2 = math.exp(-2.0)
+    assert idx0.tolist() == [[1, 3]]
+    np.testing.assert_allclose(w0, [[1 / (1 + e2), e2 / (1 + e2)]], rtol=1e-15)
+    # ties of the keys still go to the lower id; no bias gives SOFTMAX_TOPK exactly
+    tie = np.array([[1.0, 0.0, 2.0]], np.float32)
+    idx_t, _ = oracle.topk_gates(tie, 1, gate=oracle.GATE_SELECT_BIAS,
+                                 bias=np.array([1.0, 2.0, 0.0], np.float32), lib=oracle_lib)
+    assert idx_t.tolist() == [[0]]                               # keys [2, 2, 2]
+    rng = np.random.default_rng(9)
+    l = rng.standard_normal((20, 7)).astype(np.float32)
+    a = oracle.topk_gates(l, 3, gate=oracle.GATE_SELECT_BIAS, lib=oracle_lib)
+    b = oracle.topk_gates(l, 3, lib=oracle_lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
 # ------------------------------------------------------------------------------------
 # dispatch: counting sort against a library stable sort, plus invariants
 # ------------------------------------------------------------------------------------
@@ -273,7 +304,8 @@ def test_identity_experts_reproduce_x(oracle_lib):
 @pytest.mark.parametrize("act,gate,use_bias", [(oracle.ACT_SWIGLU, oracle.GATE_SOFTMAX_TOPK, False),
                                                (oracle.ACT_SWIGLU, oracle.GATE_SOFTMAX_ALL, True),
                                                (oracle.ACT_GELU_TANH, oracle.GATE_SOFTMAX_TOPK, True),
-                                               (oracle.ACT_RELU, oracle.GATE_SOFTMAX_TOPK, False)])
+                                               (oracle.ACT_RELU, oracle.GATE_SOFTMAX_TOPK, False),
+                                               (oracle.ACT_SWIGLU, oracle.GATE_SELECT_BIAS, True)])
 def test_layer_equals_dense_masked_sum_over_all_experts(oracle_lib, act, gate, use_bias):
     """Brute force: run every expert on every token (numpy matmuls), then mask with the
     gate matrix; routing from fp64 logits with a full stable sort."""
@@ -289,10 +321,14 @@ def test_layer_equals_dense_masked_sum_over_all_experts(oracle_lib, act, gate, u
     xf = widen(x)
     # the fp32 logits are pinned by the router tests above; from here on everything is
     # recomputed independently: full stable sort, full softmax, every expert on every token
-    l = oracle.router_logits(x, Wg, bias, lib=oracle_lib).astype(np.float64)
-    l_exact = xf @ widen(Wg) + (0 if bias is None else bias.astype(np.float64))
+    sel_bias = gate == oracle.GATE_SELECT_BIAS
+    l32 = oracle.router_logits(x, Wg, None if sel_bias else bias, lib=oracle_lib)
+    l = l32.astype(np.float64)
+    l_exact = xf @ widen(Wg) + (0 if (bias is None or sel_bias) else bias.astype(np.float64))
     np.testing.assert_allclose(l, l_exact, rtol=0, atol=1e-3)
-    sel = np.argsort(-l, axis=1, kind="stable")[:, :k]
+    # selection keys: the logits, or with a selection bias their fp32 sum with it
+    keys = (l32 + bias).astype(np.float64) if sel_bias else l
+    sel = np.argsort(-keys, axis=1, kind="stable")[:, :k]
     G = np.zeros((T, E))
     p = np.exp(l - l.max(axis=1, keepdims=True))
     for t in range(T):
