@@ -357,26 +357,29 @@ def run_ours(args):
     stage_ms = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
                 for j, nm in enumerate(stage_names)}
 
-    # end to end through the public API with host buffers (x in, out back, every step)
+    # end to end through the public API with host buffers: every step copies its x in and
+    # its out back (pinned host memory); moe_forward_host_batches overlaps step i's compute
+    # with step i+1's copy in and step i-1's copy out
     e2e = None
     if not args.no_e2e:
         x_h = inp["x"].cpu().pin_memory()
-        out_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
-        for _ in range(2):
-            moe.moe_forward_host(p, x_h, inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out_h, ws)
+        out_h = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        outs = [out_h[i & 1] for i in range(K)]
+        moe.moe_forward_host_batches(p, [x_h, x_h], inp["Wg"], inp["bias"], inp["W1"], inp["W2"],
+                                     out_h, ws)
         dp.barrier(dev)
         torch.cuda.synchronize(dev)
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record(stream)
-        for _ in range(K):
-            moe.moe_forward_host(p, x_h, inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out_h, ws)
+        moe.moe_forward_host_batches(p, [x_h] * K, inp["Wg"], inp["bias"], inp["W1"], inp["W2"],
+                                     outs, ws)
         e2.record(stream)
         torch.cuda.synchronize(dev)
         dp.barrier(dev)
         e2e_ms = dp.max_over_ranks(s2.elapsed_time(e2), device=dev) / K
         e2e = {"value": n * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
-               "ms_per_step": e2e_ms}
+               "ms_per_step": e2e_ms, "api": "moe_forward_host_batches (copies overlapped across steps)"}
 
     peaks, peak_src = load_peaks()
     # Denominator in the clock regime the kernels ran in: the power-capped (sustained) GEMM

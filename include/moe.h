@@ -16,8 +16,9 @@
  *   - bf16 tensors are passed as moe_bf16 (the raw 16-bit pattern), row-major, 16-byte
  *     aligned. int32/fp32 tensors are 4-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). All work is enqueued
- *     asynchronously on it; no entry point synchronises except moe_get_device_status and
- *     moe_forward_host (which waits for its own device-to-host copy).
+ *     asynchronously on it; no entry point synchronises except moe_get_device_status,
+ *     moe_forward_host and moe_forward_host_batches (which wait for their own
+ *     device-to-host copies).
  *   - Host-detectable errors (NULL pointers, unsupported sizes, a short workspace) are
  *     returned at once and nothing is launched. Errors found on the device (an expert id
  *     out of range, a bounded wait that ran out) are written to a status word in the
@@ -178,6 +179,20 @@ MOE_API moe_status moe_forward_staged(const moe_problem *p, const moe_bf16 *x, c
 MOE_API moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const moe_bf16 *Wg,
                             const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
                             moe_bf16 *out_host, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_forward on a stream of n_batches host batches: batch i reads x_host[i] and writes
+ * out_host[i] (each [T, H] bf16, pinned host memory for overlap; arrays of n_batches
+ * pointers; the same buffer may appear several times). Batch i+1's host-to-device copy and
+ * batch i-1's device-to-host copy run on two library-owned copy streams while batch i
+ * computes on `stream`; the x and out staging buffers in the workspace are double-buffered
+ * (moe_workspace_size covers them). Every batch still copies its own input in and its own
+ * output out. Returns after the last output has landed in host memory. The copy streams
+ * and their events are created on the first call on a device and kept for the process. */
+MOE_API moe_status moe_forward_host_batches(const moe_problem *p, int n_batches,
+                                            const moe_bf16 *const *x_host, const moe_bf16 *Wg,
+                                            const float *bias, const moe_bf16 *W1,
+                                            const moe_bf16 *W2, moe_bf16 *const *out_host,
+                                            void *ws, size_t ws_bytes, void *stream);
 
 /* Combine (§2.1: gather and reduce the top-k outputs).
  *   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] ), fp32 sum, j ascending.

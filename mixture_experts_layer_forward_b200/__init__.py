@@ -26,6 +26,7 @@ from ._native import (  # noqa: F401
     moe_dispatch,
     moe_forward,
     moe_forward_host,
+    moe_forward_host_batches,
     moe_forward_launches,
     moe_forward_staged,
     moe_get_device_status,

@@ -83,6 +83,7 @@ def library() -> ctypes.CDLL:
             "moe_forward_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                     ctypes.POINTER(vp), i32], i32),
             "moe_forward_host": ([P, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_forward_host_batches": ([P, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
             "moe_get_device_status": ([vp, vp], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
@@ -227,6 +228,24 @@ def moe_forward_host(p, x_host, Wg, bias, W1, W2, out_host, ws, stream=None):
                                     _ptr(out_host, bf, "out_host", cuda=False), w, n,
                                     _stream(stream))
     _check("moe_forward_host", rc)
+
+
+def moe_forward_host_batches(p, xs_host, Wg, bias, W1, W2, outs_host, ws, stream=None):
+    """A stream of host batches (lists of pinned [T, H] bf16 tensors): each batch's copies in
+    and out overlap the neighbouring batches' compute. Returns when the last output landed."""
+    bf = torch.bfloat16
+    n = len(xs_host)
+    if len(outs_host) != n:
+        raise ValueError("xs_host and outs_host differ in length")
+    xa = (ctypes.c_void_p * max(n, 1))(*[_ptr(x, bf, "x_host", cuda=False) for x in xs_host])
+    oa = (ctypes.c_void_p * max(n, 1))(*[_ptr(o, bf, "out_host", cuda=False) for o in outs_host])
+    w, nb = _ws(ws)
+    rc = library().moe_forward_host_batches(ctypes.byref(p), n, ctypes.cast(xa, ctypes.c_void_p),
+                                            _ptr(Wg, bf, "Wg"), _ptr(bias, torch.float32, "bias"),
+                                            _ptr(W1, bf, "W1"), _ptr(W2, bf, "W2"),
+                                            ctypes.cast(oa, ctypes.c_void_p), w, nb,
+                                            _stream(stream))
+    _check("moe_forward_host_batches", rc)
 
 
 def moe_combine(p, ys, inv_pos, out, ws=None, stream=None):

@@ -69,7 +69,7 @@ struct Layout {
         counts, offsets, poff, tile_off,
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
-        x_stage, out_stage;
+        x_stage, out_stage, x_stage2, out_stage2;
     size_t end_route, end_dispatch, end_forward, end_host;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
@@ -176,6 +176,8 @@ Layout make_layout(const moe_problem *p)
     L.end_forward = o;
     L.x_stage = take(T * H * 2);
     L.out_stage = take(T * H * 2);
+    L.x_stage2 = take(T * H * 2); // second staging pair: moe_forward_host_batches
+    L.out_stage2 = take(T * H * 2);
     L.end_host = o;
     return L;
 }
@@ -883,6 +885,34 @@ moe_status moe_forward_staged(const moe_problem *p, const moe_bf16 *x, const moe
                         static_cast<cudaStream_t>(stream), events, n_events);
 }
 
+// Two copy streams and per-slot events for moe_forward_host_batches, created once per device.
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+    bool ok = false;
+};
+HostPipe *host_pipe()
+{
+    static std::mutex mu;
+    static HostPipe pipes[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    HostPipe &hp = pipes[dev];
+    if (!hp.ok) {
+        bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; i < 2 && good; ++i)
+            good = cudaEventCreateWithFlags(&hp.h2d_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&hp.d2h_done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) return nullptr;
+        hp.ok = true;
+    }
+    return &hp;
+}
+
 moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const moe_bf16 *Wg,
                             const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
                             moe_bf16 *out_host, void *ws, size_t ws_bytes, void *stream)
@@ -904,6 +934,60 @@ moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const 
     if (s != MOE_OK) return s;
     if (bytes > 0 && cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MOE_ERR_CUDA;
+    return to_status(cudaStreamSynchronize(st));
+}
+
+moe_status moe_forward_host_batches(const moe_problem *p, int n_batches,
+                                    const moe_bf16 *const *x_host, const moe_bf16 *Wg,
+                                    const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                                    moe_bf16 *const *out_host, void *ws, size_t ws_bytes,
+                                    void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (n_batches < 0 || ws == nullptr || (n_batches > 0 && (x_host == nullptr || out_host == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n_batches && p->T > 0; ++i)
+        if (x_host[i] == nullptr || out_host[i] == nullptr) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_host) return MOE_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (n_batches == 0) return MOE_OK;
+    HostPipe *hp = host_pipe();
+    if (hp == nullptr) return MOE_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)p->T * p->H * 2;
+    moe_bf16 *xs[2] = {at<moe_bf16>(ws, L.x_stage), at<moe_bf16>(ws, L.x_stage2)};
+    moe_bf16 *os[2] = {at<moe_bf16>(ws, L.out_stage), at<moe_bf16>(ws, L.out_stage2)};
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    // the copies start after the work already queued on the caller's stream
+    if (!ok(cudaEventRecord(hp->start, st)) || !ok(cudaStreamWaitEvent(hp->h2d, hp->start, 0)) ||
+        !ok(cudaStreamWaitEvent(hp->d2h, hp->start, 0)))
+        return MOE_ERR_CUDA;
+    for (int i = 0; i < n_batches; ++i) {
+        const int b = i & 1;
+        // x slot b is free once batch i-2 computed; out slot b once its copy-out landed
+        if (i >= 2 && !ok(cudaStreamWaitEvent(hp->h2d, hp->comp_done[b], 0))) return MOE_ERR_CUDA;
+        if (bytes > 0 &&
+            !ok(cudaMemcpyAsync(xs[b], x_host[i], bytes, cudaMemcpyHostToDevice, hp->h2d)))
+            return MOE_ERR_CUDA;
+        if (!ok(cudaEventRecord(hp->h2d_done[b], hp->h2d)) ||
+            !ok(cudaStreamWaitEvent(st, hp->h2d_done[b], 0)) ||
+            (i >= 2 && !ok(cudaStreamWaitEvent(st, hp->d2h_done[b], 0))))
+            return MOE_ERR_CUDA;
+        s = forward_impl(p, xs[b], Wg, bias, W1, W2, os[b], nullptr, nullptr, ws, ws_bytes, st,
+                         nullptr, 0);
+        if (s != MOE_OK) return s;
+        if (!ok(cudaEventRecord(hp->comp_done[b], st)) ||
+            !ok(cudaStreamWaitEvent(hp->d2h, hp->comp_done[b], 0)))
+            return MOE_ERR_CUDA;
+        if (bytes > 0 &&
+            !ok(cudaMemcpyAsync(out_host[i], os[b], bytes, cudaMemcpyDeviceToHost, hp->d2h)))
+            return MOE_ERR_CUDA;
+        if (!ok(cudaEventRecord(hp->d2h_done[b], hp->d2h))) return MOE_ERR_CUDA;
+    }
+    // the caller's stream continues after the last copy-out; wait for it here
+    if (!ok(cudaStreamWaitEvent(st, hp->d2h_done[(n_batches - 1) & 1], 0))) return MOE_ERR_CUDA;
     return to_status(cudaStreamSynchronize(st));
 }
 

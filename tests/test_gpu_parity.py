@@ -487,6 +487,25 @@ def test_forward_host_buffers():
     assert torch.equal(out_h, out_d.cpu())
 
 
+def test_forward_host_batches_pipeline():
+    """A stream of host batches with overlapped copies gives, batch by batch, exactly the
+    outputs of moe_forward on the same inputs (including repeated buffers)."""
+    cfg = cfg_small("host_batches", 300, 256, 256, 16, 2)
+    base = synth.make_inputs(cfg, seed=19)
+    p = moe.Problem.from_config(cfg)
+    ws = alloc_ws(p)
+    xs = [synth.make_inputs(cfg, seed=19, x_seed=100 + i)["x"].pin_memory() for i in range(5)]
+    xs.append(xs[0])                                  # the same input buffer twice
+    outs = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in xs]
+    d = {k: (v.cuda() if v is not None else None) for k, v in base.items()}
+    moe.moe_forward_host_batches(p, xs, d["Wg"], d["bias"], d["W1"], d["W2"], outs, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    for i, x in enumerate(xs):
+        want = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward(p, x.cuda(), d["Wg"], d["bias"], d["W1"], d["W2"], want, ws)
+        assert torch.equal(outs[i], want.cpu()), f"batch {i}"
+
+
 # ---------------------------------------------------------------------------------------
 # full-size workloads (the bench configurations), launched exactly as the bench does
 # ---------------------------------------------------------------------------------------
