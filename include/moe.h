@@ -276,13 +276,14 @@ MOE_API int moe_set_work_order(int order);
 
 /* Router variant (a tuning and test hook; not thread-safe). All give the same routing and
  * gates (the selection is always made on the sequential fp32 logits, see moe_route):
- * MOE_ROUTER_FILTER: for 16 < E <= 512 with E % 8 == 0, MOE_GATE_SOFTMAX_TOPK and 16-byte
+ * MOE_ROUTER_FILTER: for 8 <= E <= 512 with E % 8 == 0, a gate other than SOFTMAX_ALL and 16-byte
  *   aligned x and Wg, the logits are first computed on the tensor cores; every expert whose
  *   logit interval (a rigorous bound on the difference between the two fp32 sums) cannot
  *   reach the top k is dropped, and only the rest get the sequential fp32 logit (other
  *   problems use the sequential router);
  * MOE_ROUTER_SEQUENTIAL: every (token, expert) logit is computed sequentially;
- * MOE_ROUTER_AUTO (default): the filter where it applies and T * E >= 2^16, else sequential.
+ * MOE_ROUTER_AUTO (default): the filter where it applies, E >= 16 and T * E >= 2^16, else
+ *   sequential.
  * moe_route_noalloc always uses the sequential router.
  * Returns the previous mode, or -1 for an unknown mode. */
 #define MOE_ROUTER_AUTO 0

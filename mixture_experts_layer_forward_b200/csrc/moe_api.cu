@@ -90,7 +90,7 @@ FilterPlan filter_plan(const moe_problem *p)
 {
     FilterPlan f{false, 1, 0, 0, 0, 0.0f};
     const int T = p->T, H = p->H, E = p->E;
-    if (T <= 0 || E <= 16 || E > RF_MAX_E || (E % 8) != 0 || (H % gemm::BK) != 0 ||
+    if (T <= 0 || E < 8 || E > RF_MAX_E || (E % 8) != 0 || (H % gemm::BK) != 0 ||
         p->gate == MOE_GATE_SOFTMAX_ALL || (int64_t)T * E >= (1LL << 31) / RF_SPLIT_MAX)
         return f;
     const int kb = H / gemm::BK;
@@ -366,10 +366,11 @@ cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
 bool route_uses_filter(const moe_problem *p)
 {
     const int mode = g_router_mode.load();
-    // AUTO takes the filter from 2^16 logits on (below, its fixed costs -- the W_g transpose,
-    // the GEMM and one chain of H dependent FMAs per candidate -- outweigh the savings)
+    // AUTO takes the filter from 16 experts and 2^16 logits on (below, its fixed costs -- the
+    // W_g transpose, the GEMM and one chain of H dependent FMAs per candidate -- outweigh the
+    // savings: measured slower on the Mixtral-shaped E = 8 router and the T = 64 decode one)
     const bool want = mode == MOE_ROUTER_FILTER ||
-                      (mode == MOE_ROUTER_AUTO && (int64_t)p->T * p->E >= (1 << 16));
+                      (mode == MOE_ROUTER_AUTO && p->E >= 16 && (int64_t)p->T * p->E >= (1 << 16));
     return want && filter_plan(p).ok;
 }
 

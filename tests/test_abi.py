@@ -106,9 +106,12 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(mixtral) == 8   # E = 8: sequential router
         assert moe.moe_forward_launches(qwen2) == 9     # T*E >= 2^16: filter router
         assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential router
+        phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
+        assert moe.moe_forward_launches(phi35) == 9     # E = 16: filter router
         moe.moe_set_router_mode(moe.ROUTER_FILTER)
         assert moe.moe_forward_launches(decode) == 9
-        assert moe.moe_forward_launches(mixtral) == 8   # the filter needs E > 16
+        assert moe.moe_forward_launches(mixtral) == 9   # forced: E = 8 qualifies
+        assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 8  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
         assert moe.moe_forward_launches(qwen2) == 8
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
