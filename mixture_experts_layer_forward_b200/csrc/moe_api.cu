@@ -334,9 +334,11 @@ cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
     a.timeout_ns = g_timeout_ns.load();
     err = launch_gemm<GEMM_LOGITS>(mx, mw, a, a.dense_m_tiles * a.n_tiles * fp.split, st);
     if (err != cudaSuccess) return err;
+    CUtensorMap mxs, mws; // the exact kernel's streams: bt rows of x, 64 rows of W_g^T per box
+    if (!make_map_2d(&mxs, xb, (uint64_t)T, (uint64_t)H, (uint32_t)fp.bt) ||
+        !make_map_2d(&mws, fb.wgt, (uint64_t)E, (uint64_t)H, RF_WBOX))
+        return cudaErrorInvalidValue;
     RfArgs r{};
-    r.x = xb;
-    r.WgT = reinterpret_cast<const __nv_bfloat16 *>(fb.wgt);
     r.wpart = fb.wnorm;
     r.xsq = fb.xsq;
     r.bias = bias;
@@ -358,7 +360,7 @@ cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
     err = cudaFuncSetAttribute(route_filter_exact_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    route_filter_exact_kernel<<<(T + fp.bt - 1) / fp.bt, RF_THREADS, smem, st>>>(r);
+    route_filter_exact_kernel<<<(T + fp.bt - 1) / fp.bt, RF_THREADS, smem, st>>>(mxs, mws, r);
     return cudaGetLastError();
 }
 

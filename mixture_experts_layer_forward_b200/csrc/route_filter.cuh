@@ -21,11 +21,11 @@
 //      b. an expert whose upper end is below the k-th largest lower end L cannot be in the
 //         top k: the k experts holding the k largest lower ends have exact logits >= L, all
 //         strictly above the excluded one's. The rest are the candidates;
-//      c. every candidate (token, expert) pair gets its exact sequential logit. Two producer
-//         warps stream the x rows of the block's tokens and the W_g^T rows of the union of
-//         their candidates through a ring of 64-value chunks (cp.async, completion counted on
-//         mbarriers); in eight consumer warps a thread owns two candidates of one token, so one
-//         x load serves two chains;
+//      c. every candidate (token, expert) pair gets its exact sequential logit. A producer
+//         thread streams 64-value chunks through a ring: per chunk one 2D TMA box of the
+//         block's x rows and the W_g^T rows of the candidates' id range (64-row boxes),
+//         128-byte swizzled, completion counted on mbarriers; in eight consumer warps a
+//         thread owns two candidates of one token, so one x load serves two chains;
 //      d. top k among the candidates' exact logits, ties to the lower expert id, and the gates
 //         from those exact logits, in the same arithmetic as route_topk_kernel.
 // Hence the selection, its order and the gates equal those of the full sequential router.
@@ -38,13 +38,11 @@ namespace moe {
 
 constexpr int RF_CWARPS = 8;                 // consumer warps (pair chains)
 constexpr int RF_CTHREADS = RF_CWARPS * 32;
-constexpr int RF_PWARPS = 2;                 // producer warps (cp.async)
-constexpr int RF_PTHREADS = RF_PWARPS * 32;
-constexpr int RF_WARPS = RF_CWARPS + RF_PWARPS;
+constexpr int RF_WARPS = RF_CWARPS + 1;      // + one producer warp (TMA, one thread)
 constexpr int RF_THREADS = RF_WARPS * 32;
-constexpr int RF_HC = 64;                    // h values per streamed chunk
-constexpr int RF_ROW = 144;                  // staged row: 128 bytes + 16, so 16-byte column v
-                                             // of row r sits in bank group (r + v) mod 8
+constexpr int RF_HC = 64;                    // h values per streamed chunk: 128-byte rows,
+                                             // 16-byte column v of row r at (v ^ (r & 7))
+constexpr int RF_WBOX = 64;                  // W_g^T rows per TMA box (8 KB)
 constexpr int RF_NS_MAX = 16;                // deepest chunk ring
 constexpr int RF_MAX_BT = 32;                // tokens per block
 constexpr int RF_BLOCKS_PER_SM = 2;          // blocks the token split aims to co-schedule
@@ -128,9 +126,9 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// The exact kernel also takes two tensor maps: x [T, H] with bt-row boxes and W_g^T [E, H]
+// with RF_WBOX-row boxes, both 64 columns wide, 128-byte swizzle.
 struct RfArgs {
-    const __nv_bfloat16 *x;   // [T, H]
-    const __nv_bfloat16 *WgT; // [E, H]
     const float *wpart;       // [ceil(H / RF_SLAB), E] partial sums of squares of W_g
     const float *xsq;         // [S, T] partial sums of squares of the x rows
     const float *bias;        // [E] or nullptr
@@ -145,25 +143,34 @@ struct RfArgs {
     int64_t timeout_ns;
 };
 
-// Shared memory of route_filter_exact_kernel. Region 0 holds the filter logits [bt][E + 1],
-// then the chunk ring; the exact logits of the candidates have their own [bt][E].
+// Shared memory of route_filter_exact_kernel (from a 1024-byte aligned base). Region 0 holds
+// the filter logits [bt][E + 1], then the chunk ring; the exact logits of the candidates
+// have their own [bt][E].
 __host__ __device__ inline size_t rf_region0_bytes(int bt, int E, int ring_bytes)
 {
     const size_t mrow = (size_t)bt * (E + 1) * 4;
     const size_t r = (size_t)ring_bytes > mrow ? (size_t)ring_bytes : mrow;
-    return (r + 127) & ~(size_t)127;
+    return (r + 1023) & ~(size_t)1023;
 }
 __host__ __device__ inline size_t rf_smem_bytes(int bt, int E, int ring_bytes)
 {
     const int ew = (E + 31) / 32;
-    return rf_region0_bytes(bt, E, ring_bytes) + (size_t)bt * E * 4 /*exact*/ +
-           2 * RF_NS_MAX * 8 /*mbarriers*/ +
-           (size_t)(bt + E) * 8 /*row sources*/ + (size_t)E * 4 /*wn*/ +
-           (size_t)bt * ew * 4 /*cand*/ + (size_t)E * 4 * 2 /*union*/ + 16 * 4 * 2 /*words*/ +
-           (size_t)(RF_MAX_BT + 1) * 4 * 2 /*tok_off, unit_off*/ + 16 /*U, abort*/;
+    return 1024 /*alignment slack*/ + rf_region0_bytes(bt, E, ring_bytes) +
+           (size_t)bt * E * 4 /*exact*/ + 2 * RF_NS_MAX * 8 /*mbarriers*/ +
+           (size_t)E * 4 /*wn*/ + (size_t)bt * ew * 4 /*cand*/ +
+           (size_t)(RF_MAX_BT + 1) * 4 * 2 /*tok_off, unit_off*/ + 16 /*range, abort*/;
 }
-// Smallest ring that holds two chunks of every row a block can stage.
-__host__ __device__ inline int rf_ring_min(int bt, int E) { return 2 * (bt + E) * RF_ROW; }
+// Bytes of one ring stage: the x box (bt rows, padded to 1024 bytes for the swizzle) and
+// nbw W_g^T boxes.
+__host__ __device__ inline int rf_stage_bytes(int bt, int nbw)
+{
+    return ((bt * 128 + 1023) & ~1023) + nbw * RF_WBOX * 128;
+}
+// Smallest ring that holds two chunks when the candidates span every expert.
+__host__ __device__ inline int rf_ring_min(int bt, int E)
+{
+    return 2 * rf_stage_bytes(bt, (E + RF_WBOX - 1) / RF_WBOX);
+}
 
 // r-th set bit (r >= 0) of the candidate words of one token; E when there is none
 __device__ __forceinline__ int rf_nth_bit(const uint32_t *words, int ew, int r, int E)
@@ -181,9 +188,12 @@ __device__ __forceinline__ int rf_nth_bit(const uint32_t *words, int ew, int r, 
 }
 
 __global__ void __launch_bounds__(RF_THREADS)
-    route_filter_exact_kernel(const RfArgs a)
+    route_filter_exact_kernel(const __grid_constant__ CUtensorMap tmx,
+                              const __grid_constant__ CUtensorMap tmw, const RfArgs a)
 {
-    extern __shared__ __align__(128) uint8_t rf_smem[];
+    extern __shared__ uint8_t rf_smem_raw[];
+    uint8_t *rf_smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(rf_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int E = a.E, H = a.H, T = a.T, k = a.k, bt = a.bt;
     const int ew = (E + 31) / 32;
     const int ME = E + 1; // padded filter-logit row
@@ -191,18 +201,12 @@ __global__ void __launch_bounds__(RF_THREADS)
     float *mrow = reinterpret_cast<float *>(rf_smem);                // a/b: [bt][E + 1]
     float *exact = reinterpret_cast<float *>(rf_smem + r0);          // [bt][E] exact logits
     uint64_t *bars = reinterpret_cast<uint64_t *>(exact + (size_t)bt * E); // full, empty
-    const __nv_bfloat16 **row_src =
-        reinterpret_cast<const __nv_bfloat16 **>(bars + 2 * RF_NS_MAX); // [bt + U] row starts
-    float *wn = reinterpret_cast<float *>(row_src + bt + E);        // [E] >= ||w_e||
+    float *wn = reinterpret_cast<float *>(bars + 2 * RF_NS_MAX);     // [E] >= ||w_e||
     uint32_t *cand = reinterpret_cast<uint32_t *>(wn + E);          // [bt][ew]
-    int *uni_row = reinterpret_cast<int *>(cand + (size_t)bt * ew); // [E] expert -> W row
-    int *uni_list = uni_row + E;                                     // [U] W row -> expert
-    uint32_t *uword = reinterpret_cast<uint32_t *>(uni_list + E);   // [16] union words
-    int *ubase = reinterpret_cast<int *>(uword + 16);                // [16] their ranks
-    int *tok_off = ubase + 16;                                       // [bt + 1] candidates
+    int *tok_off = reinterpret_cast<int *>(cand + (size_t)bt * ew); // [bt + 1] candidates
     int *unit_off = tok_off + RF_MAX_BT + 1;                         // [bt + 1] pair units
-    int *n_union = unit_off + RF_MAX_BT + 1;
-    volatile int *abort_flag = n_union + 1;
+    int *e_range = unit_off + RF_MAX_BT + 1;                         // lowest, highest candidate
+    volatile int *abort_flag = e_range + 2;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (RF_NS_MAX + s); };
@@ -214,11 +218,13 @@ __global__ void __launch_bounds__(RF_THREADS)
 
     if (tid == 0) {
         for (int i = 0; i < RF_NS_MAX; ++i) {
-            mbar_init(full_bar(i), RF_PTHREADS);
+            mbar_init(full_bar(i), 1);
             mbar_init(empty_bar(i), RF_CWARPS);
         }
         *abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&tmx);
+        tma_prefetch_desc(&tmw);
     }
 
     // ---- column norms and filter logits (summed over the splits, + bias) ----
@@ -323,72 +329,67 @@ __global__ void __launch_bounds__(RF_THREADS)
             unit_off[bt] = uinc;
         }
     } else if (warp == 1) {
+        // id range of the candidate experts of the block's tokens (streamed as W_g^T rows)
         uint32_t uw = 0u; // union word `lane` (ew <= 16)
         if (lane < ew)
             for (int tl = 0; tl < bt; ++tl) uw |= cand[tl * ew + lane];
-        const int pc = __popc(uw);
-        int up = pc;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, up, off);
-            if (lane >= off) up += o;
-        }
-        if (lane < ew) {
-            uword[lane] = uw;
-            ubase[lane] = up - pc;
-        }
-        if (lane == 31) *n_union = up;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += RF_THREADS) {
-        const uint32_t uw = uword[e >> 5];
-        const int b = e & 31;
-        if ((uw >> b) & 1u) {
-            const int r = ubase[e >> 5] + __popc(uw & ((1u << b) - 1u));
-            uni_row[e] = r;
-            uni_list[r] = e;
-            row_src[bt + r] = a.WgT + (size_t)e * H;
-        } else {
-            uni_row[e] = -1;
+        const int lo = uw ? lane * 32 + __ffs(uw) - 1 : 0x7fffffff;
+        const int hi = uw ? lane * 32 + 31 - __clz(uw) : -1;
+        const int lo_all = __reduce_min_sync(0xffffffffu, lo);
+        const int hi_all = __reduce_max_sync(0xffffffffu, hi);
+        if (lane == 0) {
+            e_range[0] = hi_all >= 0 ? lo_all : 0;
+            e_range[1] = hi_all >= 0 ? hi_all : -1;
         }
     }
-    for (int r = tid; r < bt; r += RF_THREADS) row_src[r] = a.x + (size_t)(t0 + (r < nt ? r : 0)) * H;
     __syncthreads();
 
     // ---- c. exact sequential logits of the candidate pairs ----
-    // Producer warps stream chunk g of every pass into ring slot g % ns; each producer thread
-    // arrives on full[slot] once its copies have landed; the consumer warps release the slot
-    // on empty[slot].
-    const int U = *n_union;
+    // One producer thread streams chunk g of every pass into ring slot g % ns: a 2D TMA box
+    // of the block's x rows and nbw boxes of the W_g^T rows e_lo.. (the candidates' id range),
+    // counted on full[slot]; the consumer warps release the slot on empty[slot]. In a slot,
+    // row r of a box holds its 16-byte column v at (v ^ (r & 7)) (128-byte swizzle).
+    const int e_lo = e_range[0];
+    const int n_rows_w = e_range[1] - e_lo + 1; // 0 when the block has no candidate
+    const int nbw = (n_rows_w + RF_WBOX - 1) / RF_WBOX;
     const int NU = unit_off[bt];
-    const int rows = bt + U;
-    const uint32_t stage_bytes = (uint32_t)rows * RF_ROW;
+    const uint32_t xs_bytes = (uint32_t)((bt * 128 + 1023) & ~1023);
+    const uint32_t stage_bytes = (uint32_t)rf_stage_bytes(bt, nbw);
     int ns = a.ring_bytes / (int)stage_bytes;
     if (ns > RF_NS_MAX) ns = RF_NS_MAX;
-    if (ns < 2) ns = 2; // the host sizes the ring for two chunks of bt + E rows
+    if (ns < 2) ns = 2; // the host sizes the ring for two chunks of every expert's rows
     const int nchunk = H / RF_HC;
     const int npass = (NU + RF_CTHREADS - 1) / RF_CTHREADS;
     const int total = npass * nchunk;
 
     if (warp >= RF_CWARPS) {
-        // ---------------- producers ----------------
-        const int pt = tid - RF_CTHREADS;
-        const uint32_t ring0 = smem_u32(rf_smem);
-        for (int g = 0; g < total; ++g) {
-            const int slot = g % ns;
-            if (g >= ns && !mbar_wait_bounded(empty_bar(slot), (uint32_t)((g / ns - 1) & 1),
-                                              abort_flag, a.timeout_ns, a.status, 180))
-                break;
-            const int h0 = (g % nchunk) * RF_HC;
-            const uint32_t base = ring0 + (uint32_t)slot * stage_bytes;
-            for (int p = pt; p < rows * 8; p += RF_PTHREADS) {
-                const int r = p >> 3, v = p & 7;
-                cp_async_16(base + (uint32_t)(r * RF_ROW + v * 16), row_src[r] + h0 + v * 8,
-                            r >= bt || r < nt);
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            fence_proxy_async_smem(); // the filter logits written here before are dead
+            const uint32_t ring0 = smem_u32(rf_smem);
+            const uint32_t tx = (uint32_t)bt * 128 + (uint32_t)nbw * RF_WBOX * 128;
+            int issued = 0;
+            for (int g = 0; g < total; ++g) {
+                const int slot = g % ns;
+                if (g >= ns && !mbar_wait_bounded(empty_bar(slot), (uint32_t)((g / ns - 1) & 1),
+                                                  abort_flag, a.timeout_ns, a.status, 180))
+                    break;
+                const int h0 = (g % nchunk) * RF_HC;
+                const uint32_t base = ring0 + (uint32_t)slot * stage_bytes;
+                mbar_arrive_expect_tx(full_bar(slot), tx);
+                tma_load_2d(base, &tmx, full_bar(slot), h0, t0);
+                for (int b = 0; b < nbw; ++b)
+                    tma_load_2d(base + xs_bytes + (uint32_t)b * RF_WBOX * 128, &tmw, full_bar(slot),
+                                h0, e_lo + b * RF_WBOX);
+                issued = g + 1;
             }
-            cp_async_arrive_noinc(full_bar(slot));
+            // every box issued has landed before the block moves on (immediate unless aborted)
+            volatile int never = 0;
+            for (int g = issued - 1; g >= 0 && g >= issued - ns; --g)
+                mbar_wait_bounded(full_bar(g % ns), (uint32_t)((g / ns) & 1), &never, a.timeout_ns,
+                                  nullptr, 0);
         }
-        cp_async_wait_all(); // this thread's copies have landed before the block moves on
+        __syncwarp();
     } else {
         // ---------------- consumers ----------------
         bool ok = true;
@@ -402,9 +403,11 @@ __global__ void __launch_bounds__(RF_THREADS)
                 e0 = rf_nth_bit(cand + tl * ew, ew, r, E);
                 e1 = rf_nth_bit(cand + tl * ew, ew, r + 1, E); // E: this unit has one chain
             }
-            const uint32_t xo = (uint32_t)(tl * RF_ROW);
-            const uint32_t wo0 = (uint32_t)((bt + (active ? uni_row[e0] : 0)) * RF_ROW);
-            const uint32_t wo1 = (e1 < E) ? (uint32_t)((bt + uni_row[e1]) * RF_ROW) : wo0;
+            const int r0w = active ? e0 - e_lo : 0;
+            const int r1w = (e1 < E) ? e1 - e_lo : r0w;
+            const uint32_t xo = (uint32_t)tl * 128, xk = (uint32_t)(tl & 7) << 4;
+            const uint32_t wo0 = xs_bytes + (uint32_t)r0w * 128, wk0 = (uint32_t)(r0w & 7) << 4;
+            const uint32_t wo1 = xs_bytes + (uint32_t)r1w * 128, wk1 = (uint32_t)(r1w & 7) << 4;
             float acc0 = 0.0f, acc1 = 0.0f;
             for (int c = 0; c < nchunk; ++c) {
                 const int g = pass * nchunk + c;
@@ -417,12 +420,12 @@ __global__ void __launch_bounds__(RF_THREADS)
                 }
                 if (active) {
                     const uint8_t *st = rf_smem + (size_t)slot * stage_bytes;
-                    const uint4 *xa = reinterpret_cast<const uint4 *>(st + xo);
-                    const uint4 *w0 = reinterpret_cast<const uint4 *>(st + wo0);
-                    const uint4 *w1 = reinterpret_cast<const uint4 *>(st + wo1);
 #pragma unroll
                     for (int vv = 0; vv < RF_HC / 8; ++vv) { // h ascending: storage order
-                        const uint4 p = xa[vv], q0 = w0[vv], q1 = w1[vv];
+                        const uint32_t v16 = (uint32_t)vv << 4;
+                        const uint4 p = *reinterpret_cast<const uint4 *>(st + xo + (v16 ^ xk));
+                        const uint4 q0 = *reinterpret_cast<const uint4 *>(st + wo0 + (v16 ^ wk0));
+                        const uint4 q1 = *reinterpret_cast<const uint4 *>(st + wo1 + (v16 ^ wk1));
                         fma2x2_bf16(p.x, q0.x, q1.x, acc0, acc1);
                         fma2x2_bf16(p.y, q0.y, q1.y, acc0, acc1);
                         fma2x2_bf16(p.z, q0.z, q1.z, acc0, acc1);
