@@ -90,6 +90,7 @@ ROUTE_CASES = [
     ("e8_selbias", 300, 256, 8, 2, False, 1.2, 2),
     ("e64_selbias", 130, 384, 64, 8, False, 1.2, 2),
     ("e256_selbias_tile", 2100, 128, 256, 8, False, 1.2, 2),
+    ("e512_max_filter", 600, 192, 512, 16, False, 1.2, 0),
 ]
 
 
@@ -337,6 +338,8 @@ FWD_CASES = [
     cfg_small("relu", 150, 128, 320, 8, 2, act=2),
     cfg_small("identity", 90, 128, 192, 8, 2, act=3),
     cfg_small("deep_k", 64, 1024, 128, 8, 2),               # long K loop, ring wraps many times
+    cfg_small("max_experts", 1500, 128, 64, 1024, 8),       # E at its limit, every expert single-tile
+    cfg_small("wide_filter", 700, 192, 128, 512, 6, zipf_s=1.2),  # largest E of the filter router
 ]
 
 
