@@ -58,6 +58,8 @@ def load(path: Path | None = None) -> ctypes.CDLL:
     lib.oracle_topk_gates.restype = i32
     lib.oracle_topk_gates_bias.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
     lib.oracle_topk_gates_bias.restype = i32
+    lib.oracle_shared_tokens.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp, vp]
+    lib.oracle_shared_tokens.restype = i32
     lib.oracle_dispatch.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, i64]
     lib.oracle_dispatch.restype = i32
     lib.oracle_expert_ffn_row.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
@@ -210,3 +212,21 @@ def moe_tokens(x, Wg, bias, W1, W2, k, tokens, act=ACT_SWIGLU, gate=GATE_SOFTMAX
     if rc:
         raise ValueError(f"oracle_moe_tokens rc={rc}")
     return out, idx, w
+
+
+def shared_tokens(x, W1s, W2s, w_sg, tokens, lib=None):
+    """Shared-expert term g_t * FFN_s(x_t) for the listed tokens (fp64 [ntok, H]).
+    W1s [H, 2Fs], W2s [Fs, H], w_sg [H] or None (gate 1)."""
+    lib = lib or load()
+    x, W1s, W2s = _u16(x), _u16(W1s), _u16(W2s)
+    wg = None if w_sg is None else _u16(w_sg)
+    T, H = x.shape
+    Fs = W2s.shape[0]
+    assert W1s.shape == (H, 2 * Fs) and W2s.shape == (Fs, H)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    out = np.empty((tokens.size, H), np.float64)
+    rc = lib.oracle_shared_tokens(T, H, Fs, _p(x), _p(W1s), _p(W2s), _p(wg), tokens.size,
+                                  _p(tokens), _p(out))
+    if rc:
+        raise ValueError(f"oracle_shared_tokens rc={rc}")
+    return out

@@ -497,3 +497,48 @@ int oracle_moe_tokens(int T, int H, int F, int E, int k, int act, int gate, int 
     }
     return bad ? -4 : 0;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Shared expert (a model feature outside the pages: Qwen2-MoE's shared expert)
+ * ------------------------------------------------------------------------------------- */
+
+/* For each listed token: out[i] = g_t * FFN_s(x_t), with FFN_s a SwiGLU FFN
+ * (W1s [H, 2Fs]: columns [0,Fs) gate, [Fs,2Fs) up; W2s [Fs, H]) and the token's gate
+ * g_t = 1 / (1 + exp(-sum_h x_t[h] w_sg[h])) (fp64), or g_t = 1 without w_sg (NULL).
+ * The layer with a shared expert is the routed layer's output plus this term.
+ * out: [ntok, H] fp64. */
+int oracle_shared_tokens(int T, int H, int Fs, const uint16_t *x, const uint16_t *W1s,
+                         const uint16_t *W2s, const uint16_t *w_sg, int ntok, const int32_t *tokens,
+                         double *out)
+{
+    if (H < 1 || Fs < 1 || ntok < 0) return -1;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -2;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        double *scratch = (double *)malloc(sizeof(double) * 2 * (size_t)Fs);
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < ntok; ++i) {
+            if (!y || !scratch) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            const uint16_t *xr = x + (size_t)tokens[i] * H;
+            double g = 1.0;
+            if (w_sg) {
+                double z = 0.0;
+                for (int h = 0; h < H; ++h)
+                    z += (double)bf16_to_float(xr[h]) * (double)bf16_to_float(w_sg[h]);
+                g = 1.0 / (1.0 + exp(-z));
+            }
+            ffn_row(H, Fs, ORACLE_ACT_SWIGLU, 0, xr, W1s, W2s, y, scratch);
+            for (int n = 0; n < H; ++n) out[(size_t)i * H + n] = g * y[n];
+        }
+        free(y);
+        free(scratch);
+    }
+    return bad ? -4 : 0;
+}

@@ -52,6 +52,9 @@ MUTANTS = [
      "oracle_router_logits(T, H, E, x, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, logits);",
      "oracle_router_logits(T, H, E, x, Wg, bias, logits);"),
     ("select_bias_ignored_in_selection", "? l[e] + bias[e] : l[e];", "? l[e] : l[e];"),
+    ("shared_gate_wrong_sign", "g = 1.0 / (1.0 + exp(-z));", "g = 1.0 / (1.0 + exp(z));"),
+    ("shared_ffn_uses_gate_half_only", "ffn_row(H, Fs, ORACLE_ACT_SWIGLU, 0, xr, W1s, W2s, y, scratch);",
+     "ffn_row(H, Fs, ORACLE_ACT_GELU_TANH, 0, xr, W1s, W2s, y, scratch);"),
 ]
 
 

@@ -366,3 +366,31 @@ def test_round_a_bf16_flag_changes_only_by_rounding(oracle_lib):
     b, _, _ = oracle.moe_forward(x, Wg, None, W1, W2, k, round_a_bf16=True, lib=oracle_lib)
     assert not np.array_equal(a, b)
     np.testing.assert_allclose(a, b, rtol=0, atol=2**-8 * np.abs(a).max() * 2)
+
+
+# ------------------------------------------------------------------------------------
+# shared expert (a model feature outside the pages)
+# ------------------------------------------------------------------------------------
+
+def test_shared_expert_term(oracle_lib):
+    """g_t * FFN_s(x_t): without a gate vector it is the dense SwiGLU FFN (numpy), with a zero
+    gate vector exactly half of it, and the gate is the logistic function of x . w_sg
+    (hand-checked on exact small integers)."""
+    T, H, Fs = 11, 64, 48
+    x = rand_bf16((T, H), 61)
+    W1s = rand_bf16((H, 2 * Fs), 62, std=1 / math.sqrt(H))
+    W2s = rand_bf16((Fs, H), 63, std=1 / math.sqrt(Fs))
+    toks = np.arange(T, dtype=np.int32)
+    dense = _np_ffn(widen(x), widen(W1s), widen(W2s), oracle.ACT_SWIGLU, Fs)
+    full = oracle.shared_tokens(x, W1s, W2s, None, toks, lib=oracle_lib)
+    np.testing.assert_allclose(full, dense, rtol=1e-10, atol=1e-12)
+    half = oracle.shared_tokens(x, W1s, W2s, bf16(np.zeros(H)), toks, lib=oracle_lib)
+    np.testing.assert_array_equal(half, 0.5 * full)
+    # gate on exact integers: x_0 . w_sg = 1*2 + 1*(-3) = -1 for the first token below
+    xi = np.zeros((2, H)); xi[0, :2] = [1, 1]; xi[1, :3] = [2, 0, 1]
+    wsg = np.zeros(H); wsg[:3] = [2, -3, 1]                      # z = [-1, 5]
+    xb = bf16(xi)
+    g_ffn = oracle.shared_tokens(xb, W1s, W2s, None, np.array([0, 1], np.int32), lib=oracle_lib)
+    got = oracle.shared_tokens(xb, W1s, W2s, bf16(wsg), np.array([0, 1], np.int32), lib=oracle_lib)
+    for i, z in enumerate([-1.0, 5.0]):
+        np.testing.assert_allclose(got[i], g_ffn[i] / (1 + math.exp(-z)), rtol=1e-14, atol=1e-300)
