@@ -194,6 +194,33 @@ MOE_API moe_status moe_forward_host_batches(const moe_problem *p, int n_batches,
                                             const moe_bf16 *W2, moe_bf16 *const *out_host,
                                             void *ws, size_t ws_bytes, void *stream);
 
+/* Shared expert (Qwen2-MoE style; a model feature beyond the pages): a SwiGLU FFN that
+ * every token passes through, added to the routed experts' output with a per-token gate:
+ *   out[t] = sum_j w_j FFN_{e_j}(x_t) + g_t FFN_s(x_t),   g_t = sigmoid(x_t . w_sg)
+ * (g_t = 1 when w_sg is NULL). W1s [H, 2 F_s] bf16 (columns [0, F_s) gate, [F_s, 2 F_s)
+ * up), W2s [F_s, H] bf16, w_sg [H] bf16; F_s % 64 == 0; device pointers, 16-byte aligned.
+ * Precision as the routed experts: bf16 h_s and gated rows, the final sum in fp32 (the
+ * shared row after the k routed ones), one bf16 rounding. */
+typedef struct {
+    int32_t F_s;
+    const moe_bf16 *W1s;
+    const moe_bf16 *W2s;
+    const moe_bf16 *w_sg;
+} moe_shared_expert;
+
+/* Workspace bytes for moe_forward_shared on *p with a shared expert of width F_s (it also
+ * covers every other entry point); 0 if invalid. */
+MOE_API size_t moe_workspace_size_shared(const moe_problem *p, int32_t F_s);
+
+/* moe_forward plus the shared expert. Its three kernels (the gate, then the dense SwiGLU
+ * and gate-scaled GEMMs over all T tokens rounded up to 128 rows) run after the dispatch;
+ * the combine adds its rows. moe_forward_launches(p) + 3 kernels. */
+MOE_API moe_status moe_forward_shared(const moe_problem *p, const moe_bf16 *x,
+                                      const moe_bf16 *Wg, const float *bias, const moe_bf16 *W1,
+                                      const moe_bf16 *W2, const moe_shared_expert *shared,
+                                      moe_bf16 *out, int32_t *topk_idx_out, float *topk_w_out,
+                                      void *ws, size_t ws_bytes, void *stream);
+
 /* Combine (§2.1: gather and reduce the top-k outputs).
  *   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] ), fp32 sum, j ascending.
  * ys [ys_rows, H] bf16 holds expert-sorted rows that already carry their gate weight;

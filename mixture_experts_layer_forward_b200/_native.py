@@ -51,6 +51,12 @@ class Problem(ctypes.Structure):
         return cls.make(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, cfg.act, cfg.gate)
 
 
+class SharedExpert(ctypes.Structure):
+    """moe_shared_expert: width F_s and device pointers of W1s [H, 2F_s], W2s [F_s, H], w_sg [H]."""
+    _fields_ = [("F_s", ctypes.c_int32), ("W1s", ctypes.c_void_p), ("W2s", ctypes.c_void_p),
+                ("w_sg", ctypes.c_void_p)]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -84,6 +90,9 @@ def library() -> ctypes.CDLL:
                                     ctypes.POINTER(vp), i32], i32),
             "moe_forward_host": ([P, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_forward_host_batches": ([P, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_workspace_size_shared": ([P, i32], sz),
+            "moe_forward_shared": ([P, vp, vp, vp, vp, vp, ctypes.POINTER(SharedExpert), vp, vp,
+                                    vp, vp, sz, vp], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
             "moe_get_device_status": ([vp, vp], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
@@ -246,6 +255,26 @@ def moe_forward_host_batches(p, xs_host, Wg, bias, W1, W2, outs_host, ws, stream
                                             ctypes.cast(oa, ctypes.c_void_p), w, nb,
                                             _stream(stream))
     _check("moe_forward_host_batches", rc)
+
+
+def moe_workspace_size_shared(p: Problem, F_s: int) -> int:
+    return int(library().moe_workspace_size_shared(ctypes.byref(p), int(F_s)))
+
+
+def moe_forward_shared(p, x, Wg, bias, W1, W2, W1s, W2s, w_sg, out, ws, topk_idx_out=None,
+                       topk_w_out=None, stream=None):
+    """moe_forward plus a shared expert: W1s [H, 2F_s], W2s [F_s, H], w_sg [H] or None."""
+    bf = torch.bfloat16
+    sh = SharedExpert(int(W2s.shape[0]), _ptr(W1s, bf, "W1s"), _ptr(W2s, bf, "W2s"),
+                      _ptr(w_sg, bf, "w_sg"))
+    w, n = _ws(ws)
+    rc = library().moe_forward_shared(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                                      _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
+                                      _ptr(W2, bf, "W2"), ctypes.byref(sh), _ptr(out, bf, "out"),
+                                      _ptr(topk_idx_out, torch.int32, "topk_idx_out"),
+                                      _ptr(topk_w_out, torch.float32, "topk_w_out"), w, n,
+                                      _stream(stream))
+    _check("moe_forward_shared", rc)
 
 
 def moe_combine(p, ys, inv_pos, out, ws=None, stream=None):

@@ -41,6 +41,7 @@ struct FusedArgs {
     __nv_bfloat16 *out;     // [T, H]
     int T, H, k;
     int64_t ys_rows;
+    const __nv_bfloat16 *ys_shared; // [T, H] shared-expert rows added last, or nullptr
     int fault_skip;         // test hook: layer0 item whose ready signal is withheld (-1: none)
 };
 
@@ -144,6 +145,17 @@ __device__ __forceinline__ void fused_combine(const FusedArgs &fa, int stripe, i
                 a[i][2] += bf16_lo(u[i].y); a[i][3] += bf16_hi(u[i].y);
                 a[i][4] += bf16_lo(u[i].z); a[i][5] += bf16_hi(u[i].z);
                 a[i][6] += bf16_lo(u[i].w); a[i][7] += bf16_hi(u[i].w);
+            }
+        }
+        if (fa.ys_shared != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (t[i] >= fa.T) continue;
+                const uint4 u = *reinterpret_cast<const uint4 *>(fa.ys_shared + (size_t)t[i] * fa.H + col);
+                a[i][0] += bf16_lo(u.x); a[i][1] += bf16_hi(u.x);
+                a[i][2] += bf16_lo(u.y); a[i][3] += bf16_hi(u.y);
+                a[i][4] += bf16_lo(u.z); a[i][5] += bf16_hi(u.z);
+                a[i][6] += bf16_lo(u.w); a[i][7] += bf16_hi(u.w);
             }
         }
 #pragma unroll

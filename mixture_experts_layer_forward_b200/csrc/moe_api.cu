@@ -69,8 +69,8 @@ struct Layout {
         counts, offsets, poff, tile_off,
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
-        x_stage, out_stage, x_stage2, out_stage2;
-    size_t end_route, end_dispatch, end_forward, end_host;
+        x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys;
+    size_t end_route, end_dispatch, end_forward, end_host, end_shared;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
 };
@@ -127,7 +127,7 @@ FilterPlan filter_plan(const moe_problem *p)
     return f;
 }
 
-Layout make_layout(const moe_problem *p)
+Layout make_layout(const moe_problem *p, int F_s = 0)
 {
     Layout L{};
     const size_t T = (size_t)p->T, H = (size_t)p->H, F = (size_t)p->F, E = (size_t)p->E,
@@ -179,6 +179,12 @@ Layout make_layout(const moe_problem *p)
     L.x_stage2 = take(T * H * 2); // second staging pair: moe_forward_host_batches
     L.out_stage2 = take(T * H * 2);
     L.end_host = o;
+    // shared expert (moe_forward_shared): gate, h_s and ys_s over T rounded up to 128 rows
+    const size_t Tpad = (T + M_TILE - 1) / M_TILE * M_TILE;
+    L.sh_gate = take(F_s > 0 ? Tpad * 4 : 0);
+    L.sh_h = take(F_s > 0 ? Tpad * (size_t)F_s * 2 : 0);
+    L.sh_ys = take(F_s > 0 ? Tpad * H * 2 : 0);
+    L.end_shared = o;
     return L;
 }
 
@@ -458,7 +464,7 @@ cudaError_t launch_gather(const moe_problem *p, const moe_bf16 *x, const int32_t
 
 cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_rows,
                            const int32_t *inv_pos, moe_bf16 *out, int *status, int clear_status,
-                           cudaStream_t st)
+                           cudaStream_t st, const moe_bf16 *ys_shared = nullptr)
 {
     const int64_t vecs = (int64_t)p->T * (p->H / 8);
     int64_t blocks = (vecs + 255) / 256;
@@ -468,7 +474,8 @@ cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_
     combine_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows,
                                                inv_pos, p->T, p->H, p->top_k,
                                                reinterpret_cast<__nv_bfloat16 *>(out), status,
-                                               clear_status);
+                                               clear_status,
+                                               reinterpret_cast<const __nv_bfloat16 *>(ys_shared));
     return cudaGetLastError();
 }
 
@@ -592,10 +599,55 @@ cudaError_t record(void *const *events, int n, int i, cudaStream_t st)
     return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
 }
 
+// The shared expert's GEMMs (dense over all tokens, padded to whole 128-row tiles): the
+// gate, layer0 (SwiGLU) into h_s, layer1 (gate-scaled) into ys_s; the combine adds ys_s.
+cudaError_t launch_shared(const moe_problem *p, const moe_bf16 *x, const moe_shared_expert *sh,
+                          float *g, moe_bf16 *hs, moe_bf16 *ys_s, int *status, int64_t timeout,
+                          cudaStream_t st)
+{
+    const int T = p->T, H = p->H, Fs = sh->F_s;
+    const int mt = (T + gemm::BM - 1) / gemm::BM, Tpad = mt * gemm::BM;
+    shared_gate_kernel<<<(Tpad + 7) / 8, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(x),
+        reinterpret_cast<const __nv_bfloat16 *>(sh->w_sg), T, H, Tpad, g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    CUtensorMap m_x, m_w1, m_h, m_w2;
+    if (!make_map_2d(&m_x, x, (uint64_t)T, (uint64_t)H, gemm::BM) ||
+        !make_map_3d(&m_w1, sh->W1s, 1, (uint64_t)H, (uint64_t)(2 * Fs)) ||
+        !make_map_2d(&m_h, hs, (uint64_t)Tpad, (uint64_t)Fs, gemm::BM) ||
+        !make_map_3d(&m_w2, sh->W2s, 1, (uint64_t)Fs, (uint64_t)H))
+        return cudaErrorInvalidValue;
+    GemmArgs a0{};
+    a0.dense_m_tiles = mt;
+    a0.dense_rows = Tpad;
+    a0.k_split = 1;
+    a0.out = reinterpret_cast<__nv_bfloat16 *>(hs);
+    a0.ld_out = Fs;
+    a0.n_cols = Fs;
+    a0.up_col = Fs;
+    a0.n_tiles = (Fs + 127) / 128;
+    a0.k_blocks = H / gemm::BK;
+    a0.act = MOE_ACT_SWIGLU;
+    a0.status = status;
+    a0.timeout_ns = timeout;
+    GemmArgs a1 = a0;
+    a1.row_w = g;
+    a1.out = reinterpret_cast<__nv_bfloat16 *>(ys_s);
+    a1.ld_out = H;
+    a1.n_cols = H;
+    a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+    a1.k_blocks = Fs / gemm::BK;
+    e = launch_gemm<GEMM_SWIGLU>(m_x, m_w1, a0, mt * a0.n_tiles, st);
+    if (e != cudaSuccess) return e;
+    return launch_gemm<GEMM_SCALE>(m_h, m_w2, a1, mt * a1.n_tiles, st);
+}
+
 moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
-                        cudaStream_t st, void *const *events, int n_events)
+                        cudaStream_t st, void *const *events, int n_events,
+                        const moe_shared_expert *sh = nullptr)
 {
     moe_status s = check_problem(p);
     if (s != MOE_OK) return s;
@@ -700,6 +752,15 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
     a1.k_blocks = F / gemm::BK;
 
+    // shared expert (dense over all tokens): its rows are added by the combine
+    moe_bf16 *ys_s = nullptr;
+    if (sh != nullptr && e == cudaSuccess) {
+        const Layout LS = make_layout(p, sh->F_s);
+        ys_s = at<moe_bf16>(ws, LS.sh_ys);
+        e = launch_shared(p, x, sh, at<float>(ws, LS.sh_gate), at<moe_bf16>(ws, LS.sh_h), ys_s,
+                          status, timeout, st);
+    }
+
     if (g_gemm_mode.load() == MOE_GEMM_FUSED) {
         // one persistent launch: layer0 -> layer1 -> combine, tile-level ready flags
         FusedArgs fa{};
@@ -713,6 +774,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         fa.H = H;
         fa.k = p->top_k;
         fa.ys_rows = L.pmax;
+        fa.ys_shared = reinterpret_cast<const __nv_bfloat16 *>(ys_s);
         fa.fault_skip = g_fault_skip.load();
         const int max_work = L.max_tiles * (a0.n_tiles + a1.n_tiles) +
                              a1.n_tiles * ((p->T + COMBINE_TOKENS - 1) / COMBINE_TOKENS);
@@ -753,7 +815,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
             e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
         if (e == cudaSuccess) e = record(events, n_events, 4, st);
     }
-    if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st);
+    if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, ys_s);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);
     return to_status(e);
 }
@@ -938,6 +1000,31 @@ moe_status moe_forward_host(const moe_problem *p, const moe_bf16 *x_host, const 
     if (bytes > 0 && cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     return to_status(cudaStreamSynchronize(st));
+}
+
+size_t moe_workspace_size_shared(const moe_problem *p, int32_t F_s)
+{
+    if (check_problem(p) != MOE_OK || F_s <= 0 || F_s % 64 != 0) return 0;
+    return make_layout(p, F_s).end_shared;
+}
+
+moe_status moe_forward_shared(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                              const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                              const moe_shared_expert *shared, moe_bf16 *out,
+                              int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (shared == nullptr || shared->F_s <= 0 || shared->W1s == nullptr || shared->W2s == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (shared->F_s % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!aligned16(shared->W1s) || !aligned16(shared->W2s) ||
+        (shared->w_sg != nullptr && !aligned16(shared->w_sg)))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < make_layout(p, shared->F_s).end_shared) return MOE_ERR_WORKSPACE;
+    return forward_impl(p, x, Wg, bias, W1, W2, out, topk_idx_out, topk_w_out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), nullptr, 0, shared);
 }
 
 moe_status moe_forward_host_batches(const moe_problem *p, int n_batches,

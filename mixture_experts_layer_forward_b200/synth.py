@@ -57,7 +57,7 @@ CONFIGS = {
     "skew_decode": LayerConfig("skew_decode", T=64, H=7168, F=2048, E=256, k=8, zipf_s=1.2),
 }
 
-_TENSOR_IDS = {"x": 1, "Wg": 2, "W1": 3, "W2": 4}
+_TENSOR_IDS = {"x": 1, "Wg": 2, "W1": 3, "W2": 4, "W1s": 5, "W2s": 6, "w_sg": 7}
 
 
 def tensor_seed(seed: int, name: str) -> int:
@@ -110,6 +110,15 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, device="cpu", x_seed: int | Non
     W2 = _randn_bf16_chunked((E, F, H), tensor_seed(seed, "W2"), 1.0 / math.sqrt(F), device)
     bias = zipf_log_prior(E, cfg.zipf_s).to(device) if cfg.zipf_s > 0 else None
     return dict(x=x, Wg=Wg, W1=W1, W2=W2, bias=bias)
+
+
+def make_shared_weights(H: int, Fs: int, seed: int = 0, device="cpu", gate: bool = True):
+    """Shared-expert weights (W1s [H, 2Fs], W2s [Fs, H], w_sg [H] or None), drawn with the
+    same scaling as the routed experts' (std 1/sqrt(fan-in))."""
+    W1s = _randn_bf16((H, 2 * Fs), tensor_seed(seed, "W1s"), 1.0 / math.sqrt(H), device)
+    W2s = _randn_bf16((Fs, H), tensor_seed(seed, "W2s"), 1.0 / math.sqrt(Fs), device)
+    w_sg = _randn_bf16((H,), tensor_seed(seed, "w_sg"), 1.0 / math.sqrt(H), device) if gate else None
+    return W1s, W2s, w_sg
 
 
 def bf16_bits(t: torch.Tensor):

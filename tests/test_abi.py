@@ -130,3 +130,16 @@ def test_forward_launch_count_follows_the_modes(lib):
         moe.moe_set_router_mode(7)
     with pytest.raises(ValueError):
         moe.moe_set_work_order(3)
+
+
+def test_shared_expert_workspace_and_checks(lib):
+    """Host-only checks of the shared-expert entry points (no kernel launched)."""
+    p = moe.Problem.make(300, 256, 192, 16, 2)
+    base = moe.moe_workspace_size(p)
+    assert moe.moe_workspace_size_shared(p, 320) > base
+    assert moe.moe_workspace_size_shared(p, 100) == 0      # F_s % 64
+    assert moe.moe_workspace_size_shared(p, 0) == 0
+    sh = moe.SharedExpert(320, None, None, None)            # no weights: invalid argument
+    rc = lib.moe_forward_shared(ctypes.byref(p), None, None, None, None, None, ctypes.byref(sh),
+                                None, None, None, None, 0, None)
+    assert rc == -1

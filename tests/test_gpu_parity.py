@@ -509,6 +509,51 @@ def test_forward_host_batches_pipeline():
         assert torch.equal(outs[i], want.cpu()), f"batch {i}"
 
 
+@pytest.mark.parametrize("with_gate", [True, False], ids=["gated", "ungated"])
+def test_forward_shared_matches_oracle(gemm_mode, with_gate):
+    """Routed experts plus a shared expert (Fs % 128 == 64, ragged T) against the oracle."""
+    cfg = cfg_small("shared", 300, 256, 192, 16, 2, zipf_s=1.2)
+    Fs = 320
+    inp = synth.make_inputs(cfg, seed=20)
+    W1s, W2s, w_sg = synth.make_shared_weights(cfg.H, Fs, 21, gate=with_gate)
+    p = moe.Problem.from_config(cfg)
+    ws = torch.empty(moe.moe_workspace_size_shared(p, Fs), dtype=torch.uint8, device="cuda")
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward_shared(p, d["x"], d["Wg"], d["bias"], d["W1"], d["W2"], W1s.cuda(), W2s.cuda(),
+                           None if w_sg is None else w_sg.cuda(), out, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    b = inp["bias"].numpy()
+    ref, _, _ = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                   bits(inp["W2"]), cfg.k)
+    ref = ref + oracle.shared_tokens(bits(inp["x"]), bits(W1s), bits(W2s),
+                                     None if w_sg is None else bits(w_sg), np.arange(cfg.T))
+    assert_out_close(out, ref, f"shared, gate {with_gate}")
+
+
+def test_forward_shared_full_size_qwen2():
+    """The Qwen2-shaped layer with a 20480-wide shared expert (Qwen2-57B-A14B's), on a token
+    sample checked one by one against the oracle."""
+    cfg = synth.CONFIGS["qwen2"]
+    Fs = 20480
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    W1s, W2s, w_sg = synth.make_shared_weights(cfg.H, Fs, 22, device="cuda")
+    p = moe.Problem.from_config(cfg)
+    ws = torch.empty(moe.moe_workspace_size_shared(p, Fs), dtype=torch.uint8, device="cuda")
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward_shared(p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], W1s, W2s,
+                           w_sg, out, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    host = {k: (bits(v) if v is not None and v.dtype == torch.bfloat16 else v) for k, v in inp.items()}
+    toks = np.unique(np.random.default_rng(3).choice(cfg.T, size=12, replace=False)).astype(np.int32)
+    toks = np.concatenate([toks, np.array([cfg.T - 1], np.int32)])
+    b = None if inp["bias"] is None else inp["bias"].cpu().numpy()
+    ref, _, _ = oracle.moe_tokens(host["x"], host["Wg"], b, host["W1"], host["W2"], cfg.k, toks,
+                                  act=cfg.act, gate=cfg.gate)
+    ref = ref + oracle.shared_tokens(host["x"], bits(W1s), bits(W2s), bits(w_sg), toks)
+    assert_out_close(out[torch.from_numpy(toks).long().cuda()], ref, "qwen2 + shared")
+
+
 # ---------------------------------------------------------------------------------------
 # full-size workloads (the bench configurations), launched exactly as the bench does
 # ---------------------------------------------------------------------------------------
