@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
+    ap.add_argument("--router-only", action="store_true",
+                    help="time moe_route alone (router logits + top-k); no expert weights allocated")
     return ap.parse_args()
 
 
@@ -91,7 +93,7 @@ def config_dict(cfg, args, n):
         "workload": WORKLOAD_NAMES.get(args.workload, args.workload) + f" ({cfg.name})",
         "T_per_gpu": cfg.T, "H": cfg.H, "F": cfg.F, "E": cfg.E, "top_k": cfg.k,
         "act": ["swiglu", "gelu_tanh", "relu", "identity"][cfg.act],
-        "gate": ["softmax_topk", "softmax_all"][cfg.gate],
+        "gate": ["softmax_topk", "softmax_all", "select_bias"][cfg.gate],
         "global_tokens": cfg.T * n, "parallelism": f"dp{n} replicas (no collective)",
         "l2": "inputs larger than L2 (per-step working set >> 126 MB); no flush",
         "seed": args.seed,
@@ -443,10 +445,49 @@ def run_ours(args):
     return 0
 
 
+def run_router(args):
+    """Router alone on one GPU: K timed moe_route calls on the workload's x and W_g."""
+    import torch
+
+    import mixture_experts_layer_forward_b200 as moe
+    from mixture_experts_layer_forward_b200 import synth
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = workload(args)
+    K, W = args.steps, max(3, args.warmup)
+    inp = synth.make_inputs(cfg, seed=args.seed, device=dev, experts=False)
+    p = moe.Problem.from_config(cfg)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+    call = lambda: moe.moe_route(p, inp["x"], inp["Wg"], inp["bias"], idx, w, ws)
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(K):
+        call()
+    end.record()
+    torch.cuda.synchronize(dev)
+    assert moe.moe_get_device_status(ws) == 0
+    ms = start.elapsed_time(end) / K
+    cfgd = config_dict(cfg, args, 1)
+    cfgd["l2"] = "no flush between calls (x and W_g may stay in L2)"
+    emit({"metric": "MoE router tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
+          "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+          "dtype": "f32 logits from bf16 inputs", "data": "synthetic", "config": cfgd,
+          "router": "filter" if moe.moe_route_uses_filter(p) else "sequential"})
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.router_only:
+        return run_router(args)
     return run_ours(args)
 
 

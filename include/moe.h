@@ -318,6 +318,10 @@ MOE_API int moe_set_work_order(int order);
 #define MOE_ROUTER_FILTER 2
 MOE_API int moe_set_router_mode(int mode);
 
+/* 1 if moe_route / moe_forward on *p take the filter router under the current router mode,
+ * 0 if the sequential one, -1 if *p is invalid. */
+MOE_API int moe_route_uses_filter(const moe_problem *p);
+
 /* Test hook for the bounded ready-flag waits of MOE_GEMM_FUSED: the layer0 work item with
  * this index (in the kernel's static work queue) withholds its ready signal, so the layer1
  * tiles that need it wait until the timeout (moe_set_wait_timeout_ns) and the call reports

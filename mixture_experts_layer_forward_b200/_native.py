@@ -81,6 +81,7 @@ def library() -> ctypes.CDLL:
         sig = {
             "moe_workspace_size": ([P], sz),
             "moe_forward_launches": ([P], i32),
+            "moe_route_uses_filter": ([P], i32),
             "moe_padded_rows_max": ([P], i64),
             "moe_route": ([P, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_route_noalloc": ([P, vp, vp, vp, vp, vp, vp], i32),
@@ -158,6 +159,14 @@ def moe_workspace_size(p: Problem) -> int:
 def moe_forward_launches(p: Problem) -> int:
     """Kernels one moe_forward call on p launches under the current GEMM and router modes."""
     return int(library().moe_forward_launches(ctypes.byref(p)))
+
+
+def moe_route_uses_filter(p: Problem) -> bool:
+    """Whether the router on p takes the filter variant under the current router mode."""
+    rc = int(library().moe_route_uses_filter(ctypes.byref(p)))
+    if rc < 0:
+        raise ValueError("moe_route_uses_filter: invalid problem")
+    return rc == 1
 
 
 def moe_padded_rows_max(p: Problem) -> int:

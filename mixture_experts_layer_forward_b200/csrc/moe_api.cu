@@ -1158,6 +1158,12 @@ int moe_set_router_mode(int mode)
     return g_router_mode.exchange(mode);
 }
 
+int moe_route_uses_filter(const moe_problem *p)
+{
+    if (check_problem(p) != MOE_OK) return -1;
+    return route_uses_filter(p) ? 1 : 0;
+}
+
 int moe_set_fault_injection(int layer0_item)
 {
     return g_fault_skip.exchange(layer0_item < 0 ? -1 : layer0_item);

@@ -95,19 +95,23 @@ def zipf_log_prior(E: int, s: float) -> torch.Tensor:
     return p.log().to(torch.float32)
 
 
-def make_inputs(cfg: LayerConfig, seed: int = 0, device="cpu", x_seed: int | None = None):
+def make_inputs(cfg: LayerConfig, seed: int = 0, device="cpu", x_seed: int | None = None,
+                experts: bool = True):
     """Return dict(x, Wg, W1, W2, bias) on ``device`` (bias is None unless cfg.zipf_s > 0).
 
     ``x_seed`` overrides the seed of x only (data-parallel replicas draw their own batch
-    while sharing the weights)."""
+    while sharing the weights). ``experts=False`` leaves W1 and W2 out (None), for the router
+    alone; the other tensors are the same draws."""
     T, H, F, E = cfg.T, cfg.H, cfg.F, cfg.E
     w1_cols = 2 * F if cfg.act == ACT_SWIGLU else F
     xs = tensor_seed(seed if x_seed is None else x_seed, "x")
     x = _randn_bf16((T, H), xs, 1.0, device)
     Wg = _randn_bf16((H, E), tensor_seed(seed, "Wg"),
                      1.0 if cfg.gate_std_unscaled else 1.0 / math.sqrt(H), device)
-    W1 = _randn_bf16_chunked((E, H, w1_cols), tensor_seed(seed, "W1"), 1.0 / math.sqrt(H), device)
-    W2 = _randn_bf16_chunked((E, F, H), tensor_seed(seed, "W2"), 1.0 / math.sqrt(F), device)
+    W1 = W2 = None
+    if experts:
+        W1 = _randn_bf16_chunked((E, H, w1_cols), tensor_seed(seed, "W1"), 1.0 / math.sqrt(H), device)
+        W2 = _randn_bf16_chunked((E, F, H), tensor_seed(seed, "W2"), 1.0 / math.sqrt(F), device)
     bias = zipf_log_prior(E, cfg.zipf_s).to(device) if cfg.zipf_s > 0 else None
     return dict(x=x, Wg=Wg, W1=W1, W2=W2, bias=bias)
 

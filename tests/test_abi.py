@@ -143,3 +143,16 @@ def test_shared_expert_workspace_and_checks(lib):
     rc = lib.moe_forward_shared(ctypes.byref(p), None, None, None, None, None, ctypes.byref(sh),
                                 None, None, None, None, 0, None)
     assert rc == -1
+
+
+def test_route_uses_filter_follows_mode_and_shape(lib):
+    skew = moe.Problem.make(4096, 7168, 2048, 256, 8)
+    mixtral = moe.Problem.make(8192, 4096, 14336, 8, 2)
+    assert moe.moe_route_uses_filter(skew) and not moe.moe_route_uses_filter(mixtral)
+    prev = moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
+    try:
+        assert not moe.moe_route_uses_filter(skew)
+        moe.moe_set_router_mode(moe.ROUTER_FILTER)
+        assert moe.moe_route_uses_filter(mixtral)
+    finally:
+        moe.moe_set_router_mode(prev)
