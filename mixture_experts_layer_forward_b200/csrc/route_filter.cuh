@@ -187,6 +187,85 @@ __device__ __forceinline__ int rf_nth_bit(const uint32_t *words, int ew, int r, 
     return E;
 }
 
+// Key of the k-th largest lower interval end of one token (one warp), counted with
+// multiplicity: per round the warp maximum of the remaining lower ends and how many experts
+// hold it. Lane owns e = lane + 32 i (i < NS, NS * 32 >= E); its keys stay in registers and
+// a taken one becomes INT_MIN.
+template <int NS>
+__device__ __forceinline__ int rf_kth_lower(const float *mr, const float *wn, float cx, int E,
+                                            int k, int lane)
+{
+    int lk[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        lk[i] = (int)0x80000000;
+        if (e < E) {
+            const float m = mr[e];
+            lk[i] = rf_key(m - (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)));
+        }
+    }
+    int taken = 0, Lk = (int)0x80000000;
+    while (taken < k) {
+        int best = (int)0x80000000;
+#pragma unroll
+        for (int i = 0; i < NS; ++i) best = lk[i] > best ? lk[i] : best;
+        const int mx = __reduce_max_sync(0xffffffffu, best);
+        Lk = mx;
+        if (mx == (int)0x80000000) break; // nothing left (non-finite input)
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < NS; ++i)
+            if (lk[i] == mx) {
+                lk[i] = (int)0x80000000;
+                ++mine;
+            }
+        taken += (int)__reduce_add_sync(0xffffffffu, (unsigned)mine);
+    }
+    return Lk;
+}
+
+// Top k of one token's candidates (one warp), ties to the lower expert id: writes
+// idx_t[j] and returns, in lane j (j < 32), the gate value of the j-th selection (the
+// selection key, or with the selection bias the logit without it); selections j >= 32 go to
+// w_t[j] for the caller's softmax. *top receives the first selected value.
+template <int NS>
+__device__ __forceinline__ float rf_topk_token(const float *row, const uint32_t *cw,
+                                               const float *bias, int E, int k, int gate,
+                                               int32_t *idx_t, float *w_t, int lane, float *top)
+{
+    int fk[NS]; // selection keys of the lane's candidates, INT_MIN otherwise or once selected
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        fk[i] = (int)0x80000000;
+        if (e < E && ((cw[i] >> lane) & 1u))
+            fk[i] = rf_key((bias != nullptr) ? row[e] + bias[e] : row[e]);
+    }
+    float sel_val = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        int best = (int)0x80000000, bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < NS; ++i)
+            if (fk[i] > best) { // i ascending: keeps the lower id
+                best = fk[i];
+                bi = lane + 32 * i;
+            }
+        const int mx = __reduce_max_sync(0xffffffffu, best);
+        int w = (int)__reduce_min_sync(0xffffffffu, (unsigned)(best == mx ? bi : 0x7fffffff));
+        if (w < 0 || w >= E) w = 0; // unsupported non-finite rows still index the row
+        const float bv = (gate == 2) ? row[w] : rf_unkey(mx);
+#pragma unroll
+        for (int i = 0; i < NS; ++i)
+            if (lane + 32 * i == w) fk[i] = (int)0x80000000;
+        if (j == 0) *top = bv;
+        if (lane == 0) idx_t[j] = w;
+        if (j < 32 && j == lane) sel_val = bv;
+        if (j >= 32 && lane == 0) w_t[j] = bv;
+    }
+    return sel_val;
+}
+
 __global__ void __launch_bounds__(RF_THREADS)
     route_filter_exact_kernel(const __grid_constant__ CUtensorMap tmx,
                               const __grid_constant__ CUtensorMap tmw, const RfArgs a)
@@ -196,6 +275,7 @@ __global__ void __launch_bounds__(RF_THREADS)
         (reinterpret_cast<uintptr_t>(rf_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int E = a.E, H = a.H, T = a.T, k = a.k, bt = a.bt;
     const int ew = (E + 31) / 32;
+    const int nslot = ew <= 1 ? 1 : ew <= 2 ? 2 : ew <= 4 ? 4 : ew <= 8 ? 8 : RF_MAX_E / 32;
     const int ME = E + 1; // padded filter-logit row
     const size_t r0 = rf_region0_bytes(bt, E, a.ring_bytes);
     float *mrow = reinterpret_cast<float *>(rf_smem);                // a/b: [bt][E + 1]
@@ -238,7 +318,7 @@ __global__ void __launch_bounds__(RF_THREADS)
         }
         wn[e] = rf_norm_up(s, H);
     }
-#pragma unroll 2
+#pragma unroll 4
     for (int q = tid; q < E * bt; q += RF_THREADS) {
         const int e = q / bt, tl = q - e * bt; // consecutive threads: consecutive tokens
         if (tl < nt) {
@@ -263,32 +343,14 @@ __global__ void __launch_bounds__(RF_THREADS)
         float ss = 0.0f; // ||x_t||^2 from the filter GEMM's per-split partial sums
         for (int j = 0; j < a.S; ++j) ss += a.xsq[(size_t)j * T + t0 + tl];
         const float cx = a.cA * rf_norm_up(ss, H);
-        // L = k-th largest lower end, counted with multiplicity: per round the warp maximum of
-        // the remaining lower ends and how many experts hold it (lane owns e = lane + 32 i)
-        uint32_t removed = 0u;
-        int taken = 0, Lk = (int)0x80000000;
-        while (taken < k) {
-            int best = (int)0x80000000;
-            for (int e = lane, i = 0; e < E; e += 32, ++i) {
-                if ((removed >> i) & 1u) continue;
-                const float m = mr[e];
-                const int key = rf_key(m - (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)));
-                best = key > best ? key : best;
-            }
-            const int mx = __reduce_max_sync(0xffffffffu, best);
-            int mine = 0;
-            for (int e = lane, i = 0; e < E; e += 32, ++i) {
-                if ((removed >> i) & 1u) continue;
-                const float m = mr[e];
-                const int key = rf_key(m - (cx * wn[e] + 2.3841858e-7f * (fabsf(m) + 1.0f)));
-                if (key == mx) {
-                    removed |= 1u << i;
-                    ++mine;
-                }
-            }
-            taken += (int)__reduce_add_sync(0xffffffffu, (unsigned)mine);
-            Lk = mx;
-            if (mx == (int)0x80000000) break; // nothing left (non-finite input)
+        // L = k-th largest lower end, counted with multiplicity
+        int Lk;
+        switch (nslot) {
+        case 1: Lk = rf_kth_lower<1>(mr, wn, cx, E, k, lane); break;
+        case 2: Lk = rf_kth_lower<2>(mr, wn, cx, E, k, lane); break;
+        case 4: Lk = rf_kth_lower<4>(mr, wn, cx, E, k, lane); break;
+        case 8: Lk = rf_kth_lower<8>(mr, wn, cx, E, k, lane); break;
+        default: Lk = rf_kth_lower<RF_MAX_E / 32>(mr, wn, cx, E, k, lane); break;
         }
         const float L = rf_unkey(Lk);
         for (int w0 = 0; w0 < ew; ++w0) {
@@ -450,27 +512,17 @@ __global__ void __launch_bounds__(RF_THREADS)
         const int t = t0 + tl;
         const float *row = exact + tl * E;
         const uint32_t *cw = cand + tl * ew;
-        uint32_t removed = 0u; // lane owns e = lane + 32 i; non-candidates count as removed
-        for (int e = lane, i = 0; e < E; e += 32, ++i)
-            if (!((cw[e >> 5] >> (e & 31)) & 1u)) removed |= 1u << i;
-        float sel_val = 0.0f, top = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            int best = (int)0x80000000, bi = 0x7fffffff;
-            for (int e = lane, i = 0; e < E; e += 32, ++i) {
-                if ((removed >> i) & 1u) continue;
-                const float v = (a.bias != nullptr) ? row[e] + a.bias[e] : row[e];
-                const int key = rf_key(v);
-                if (key > best) { best = key; bi = e; } // e ascending: keeps the lower id
-            }
-            const int mx = __reduce_max_sync(0xffffffffu, best);
-            int w = (int)__reduce_min_sync(0xffffffffu, (unsigned)(best == mx ? bi : 0x7fffffff));
-            if (w < 0 || w >= E) w = 0; // unsupported non-finite rows still index the row
-            const float bv = (a.gate == 2) ? row[w] : rf_unkey(mx);
-            if ((w & 31) == lane) removed |= 1u << (w >> 5);
-            if (j == 0) top = bv;
-            if (lane == 0) a.topk_idx[(size_t)t * k + j] = w;
-            if (j < 32 && j == lane) sel_val = bv;
-            if (j >= 32 && lane == 0) a.topk_w[(size_t)t * k + j] = bv;
+        float top = 0.0f, sel_val;
+        int32_t *idx_t = a.topk_idx + (size_t)t * k;
+        float *w_t = a.topk_w + (size_t)t * k;
+        switch (nslot) {
+        case 1: sel_val = rf_topk_token<1>(row, cw, a.bias, E, k, a.gate, idx_t, w_t, lane, &top); break;
+        case 2: sel_val = rf_topk_token<2>(row, cw, a.bias, E, k, a.gate, idx_t, w_t, lane, &top); break;
+        case 4: sel_val = rf_topk_token<4>(row, cw, a.bias, E, k, a.gate, idx_t, w_t, lane, &top); break;
+        case 8: sel_val = rf_topk_token<8>(row, cw, a.bias, E, k, a.gate, idx_t, w_t, lane, &top); break;
+        default:
+            sel_val = rf_topk_token<RF_MAX_E / 32>(row, cw, a.bias, E, k, a.gate, idx_t, w_t, lane, &top);
+            break;
         }
         __syncwarp();
         if (a.gate == 2) { // the largest selected logit (the first selected one need not be)
