@@ -70,6 +70,20 @@ def load(path: Path | None = None) -> ctypes.CDLL:
     lib.oracle_moe_forward.restype = i32
     lib.oracle_moe_tokens.argtypes = [i32] * 8 + [vp] * 5 + [i32, vp, vp, vp, vp]
     lib.oracle_moe_tokens.restype = i32
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_encode_n.argtypes = [i64, vp, vp]
+    lib.oracle_e4m3_encode_n.restype = None
+    lib.oracle_e4m3_decode_n.argtypes = [i64, vp, vp]
+    lib.oracle_e4m3_decode_n.restype = None
+    lib.oracle_quant_rows_fp8.argtypes = [i32, i32, vp, vp, vp]
+    lib.oracle_quant_rows_fp8.restype = None
+    lib.oracle_quant_cols_fp8.argtypes = [i32, i32, i32, vp, vp, vp]
+    lib.oracle_quant_cols_fp8.restype = None
+    lib.oracle_moe_tokens_fp8.argtypes = [i32] * 7 + [vp] * 7 + [i32, vp, vp, vp, vp]
+    lib.oracle_moe_tokens_fp8.restype = i32
     _lib_cache[p] = lib
     return lib
 
@@ -230,3 +244,77 @@ def shared_tokens(x, W1s, W2s, w_sg, tokens, lib=None):
     if rc:
         raise ValueError(f"oracle_shared_tokens rc={rc}")
     return out
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 (e4m3) experts: a precision variant outside the pages (see moe_oracle.c for the
+# reading: per-row scales of x and h, per-output-column scales of W1 and W2)
+# ---------------------------------------------------------------------------------------
+
+def e4m3_encode(v, lib=None):
+    """float32 values -> e4m3 codes (uint8), nearest with ties to even, saturating."""
+    lib = lib or load()
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib.oracle_e4m3_encode_n(v.size, _p(v), _p(out))
+    return out
+
+
+def e4m3_decode(c, lib=None):
+    """e4m3 codes (uint8) -> their values (fp64; NaN for the NaN codes)."""
+    lib = lib or load()
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib.oracle_e4m3_decode_n(c.size, _p(c), _p(out))
+    return out
+
+
+def quant_rows_fp8(src, lib=None):
+    """bf16 bit patterns [rows, cols] -> (codes [rows, cols] uint8, scales [rows] fp32)."""
+    lib = lib or load()
+    src = _u16(src)
+    rows, cols = src.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty(rows, np.float32)
+    lib.oracle_quant_rows_fp8(rows, cols, _p(src), _p(q), _p(s))
+    return q, s
+
+
+def quant_cols_fp8(W, lib=None):
+    """Expert weights, bf16 bit patterns [E, K, N] -> (codes [E, N, K] uint8, scales [E, N])."""
+    lib = lib or load()
+    W = _u16(W)
+    E, K, N = W.shape
+    q = np.empty((E, N, K), np.uint8)
+    s = np.empty((E, N), np.float32)
+    lib.oracle_quant_cols_fp8(E, K, N, _p(W), _p(q), _p(s))
+    return q, s
+
+
+def moe_tokens_fp8(x, Wg, bias, W1q, s1, W2q, s2, k, tokens, act=ACT_SWIGLU,
+                   gate=GATE_SOFTMAX_TOPK, lib=None):
+    """Layer output with e4m3 experts for the listed tokens (fp64 [ntok, H]), plus the
+    routing. W1q [E, w1_cols, H], s1 [E, w1_cols], W2q [E, H, F], s2 [E, H]."""
+    lib = lib or load()
+    x, Wg = _u16(x), _u16(Wg)
+    T, H = x.shape
+    E = Wg.shape[1]
+    W1q = np.ascontiguousarray(W1q, dtype=np.uint8)
+    W2q = np.ascontiguousarray(W2q, dtype=np.uint8)
+    s1 = np.ascontiguousarray(s1, dtype=np.float32)
+    s2 = np.ascontiguousarray(s2, dtype=np.float32)
+    F = W2q.shape[2]
+    w1_cols = 2 * F if act == ACT_SWIGLU else F
+    assert W1q.shape == (E, w1_cols, H) and s1.shape == (E, w1_cols)
+    assert W2q.shape == (E, H, F) and s2.shape == (E, H)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    n = tokens.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((n, H), np.float64)
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    rc = lib.oracle_moe_tokens_fp8(T, H, F, E, k, act, gate, _p(x), _p(Wg), _p(b), _p(W1q),
+                                   _p(s1), _p(W2q), _p(s2), n, _p(tokens), _p(out), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle_moe_tokens_fp8 rc={rc}")
+    return out, idx, w

@@ -44,6 +44,7 @@
  * order of any sum.
  */
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -539,6 +540,223 @@ int oracle_shared_tokens(int T, int H, int Fs, const uint16_t *x, const uint16_t
         }
         free(y);
         free(scratch);
+    }
+    return bad ? -4 : 0;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * FP8 experts (a precision variant outside the pages; the pages fix no precision)
+ *
+ * Reading taken:
+ *   - element format: e4m3 of the OCP 8-bit floating-point formats: 1 sign bit, 4 exponent
+ *     bits (bias 7), 3 mantissa bits, no infinities, S.1111.111 is NaN, so the largest
+ *     finite magnitude is 1.75 * 2^8 = 448; exponent field 0 holds m * 2^-9, m = 1..7;
+ *   - conversion: nearest value, ties to the even code; magnitudes above 448 and infinities
+ *     saturate to 448; NaN stays NaN;
+ *   - scaling: one fp32 scale per token row of x and of h (over the K values of the row),
+ *     one per output column of W1 and W2 (over K): r = 448 / amax, s = amax / 448, both
+ *     rounded to fp32, code = e4m3(v * r) with the product rounded to fp32; a vector whose
+ *     r is not finite (amax zero or tiny) takes r = s = 1;
+ *   - GEMMs: exact products of the decoded codes, summed, times s_row * s_col;
+ *   - between the layers h is held in bf16, as in the bf16 path, and then quantised per row.
+ *     This one rounding step is parity unpinned: its effect (one bf16 rounding of h before
+ *     the row quantisation) is far below what the pins resolve; every other step is pinned.
+ * ------------------------------------------------------------------------------------- */
+
+double oracle_e4m3_decode(uint8_t c)
+{
+    const int s = c >> 7, ef = (c >> 3) & 15, m = c & 7;
+    if (ef == 15 && m == 7) return NAN;
+    const double v = ef == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, ef - 7);
+    return s ? -v : v;
+}
+
+uint8_t oracle_e4m3_encode(float v)
+{
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a > 448.0) return sign | 0x7E;
+    int code;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: the nearest multiple of 2^-9 (8 * 2^-9 is the smallest normal,
+         * whose code is 8) */
+        code = (int)nearbyint(ldexp(a, 9));
+    } else {
+        int e;
+        frexp(a, &e); /* a in [2^(e-1), 2^e) */
+        const int ex = e - 1;
+        const int m = (int)nearbyint((ldexp(a, -ex) - 1.0) * 8.0); /* 0..8; 8 carries */
+        code = ((ex + 7) << 3) + m;
+    }
+    return (uint8_t)(sign | code);
+}
+
+void oracle_e4m3_encode_n(int64_t n, const float *v, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
+}
+
+void oracle_e4m3_decode_n(int64_t n, const uint8_t *c, double *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(c[i]);
+}
+
+/* scales of one vector with largest magnitude amax: *r = 448 / amax, *s = amax / 448 */
+static void fp8_scales(float amax, float *r, float *s)
+{
+    *r = 448.0f / amax;
+    *s = amax / 448.0f;
+    if (!isfinite(*r)) {
+        *r = 1.0f;
+        *s = 1.0f;
+    }
+}
+
+/* n values v[i * stride] -> codes q[i * qstride] and the vector's dequantisation scale */
+static float quant_vec(int n, const float *v, ptrdiff_t stride, uint8_t *q, ptrdiff_t qstride)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        const float a = fabsf(v[(ptrdiff_t)i * stride]);
+        if (a > amax) amax = a;
+    }
+    float r, s;
+    fp8_scales(amax, &r, &s);
+    for (int i = 0; i < n; ++i) q[(ptrdiff_t)i * qstride] = oracle_e4m3_encode(v[(ptrdiff_t)i * stride] * r);
+    return s;
+}
+
+/* Row quantisation of a bf16 matrix src [rows, cols] -> dst [rows, cols] codes, scale [rows]. */
+void oracle_quant_rows_fp8(int rows, int cols, const uint16_t *src, uint8_t *dst, float *scale)
+{
+#pragma omp parallel
+    {
+        float *v = (float *)malloc(sizeof(float) * (size_t)cols);
+#pragma omp for schedule(static)
+        for (int r = 0; r < rows; ++r) {
+            if (!v) continue;
+            for (int c = 0; c < cols; ++c) v[c] = bf16_to_float(src[(size_t)r * cols + c]);
+            scale[r] = quant_vec(cols, v, 1, dst + (size_t)r * cols, 1);
+        }
+        free(v);
+    }
+}
+
+/* Column quantisation of expert weights W [E, K, N] (N contiguous): per column n of expert
+ * e, the K values W[e][:, n] -> Wq[e][n][:] (the transpose: K contiguous), scale [E, N]. */
+void oracle_quant_cols_fp8(int E, int K, int N, const uint16_t *W, uint8_t *Wq, float *scale)
+{
+#pragma omp parallel
+    {
+        float *v = (float *)malloc(sizeof(float) * (size_t)K);
+#pragma omp for schedule(static)
+        for (int64_t en = 0; en < (int64_t)E * N; ++en) {
+            if (!v) continue;
+            const int64_t e = en / N, n = en % N;
+            const uint16_t *col = W + (size_t)e * K * N + n;
+            for (int kk = 0; kk < K; ++kk) v[kk] = bf16_to_float(col[(size_t)kk * N]);
+            scale[en] = quant_vec(K, v, 1, Wq + (size_t)en * K, 1);
+        }
+        free(v);
+    }
+}
+
+/* One expert on one token with e4m3 operands (xq, sx: the token's quantised row):
+ *   z_c = (sum_h dec(xq_h) * dec(W1q[c][h])) * sx * s1[c]     (W1q [w1_cols, H], fp64);
+ *   a_f = silu(z_f) * z_{F+f} (SwiGLU) or act(z_f), rounded to bf16 (the stored h);
+ *   hq, sh = the row quantisation of a;
+ *   y_n = (sum_f dec(hq_f) * dec(W2q[n][f])) * sh * s2[n]      (W2q [H, F]).
+ * dec: the 256-entry decode table. z must hold 2F doubles, hf F floats, hq F bytes. */
+static void ffn_row_fp8(int H, int F, int act, const double *dec, const uint8_t *xq, float sx,
+                        const uint8_t *W1q, const float *s1, const uint8_t *W2q, const float *s2,
+                        double *y, double *z, float *hf, uint8_t *hq)
+{
+    const int gated = (act == ORACLE_ACT_SWIGLU);
+    const int w1_cols = gated ? 2 * F : F;
+    for (int c = 0; c < w1_cols; ++c) {
+        const uint8_t *wr = W1q + (size_t)c * H;
+        double acc = 0.0;
+        for (int h = 0; h < H; ++h) acc += dec[xq[h]] * dec[wr[h]];
+        z[c] = acc * (double)sx * (double)s1[c];
+    }
+    for (int f = 0; f < F; ++f) {
+        const double a = gated ? silu(z[f]) * z[f + F] : act_apply(act, z[f]);
+        hf[f] = (float)oracle_round_to_bf16(a);
+    }
+    const float sh = quant_vec(F, hf, 1, hq, 1);
+    for (int n = 0; n < H; ++n) {
+        const uint8_t *wr = W2q + (size_t)n * F;
+        double acc = 0.0;
+        for (int f = 0; f < F; ++f) acc += dec[hq[f]] * dec[wr[f]];
+        y[n] = acc * (double)sh * (double)s2[n];
+    }
+}
+
+/* The layer output for a list of tokens with e4m3 experts: the routing of oracle_moe_tokens
+ * (bf16 x and W_g, fp32 logits), then out[t] = sum_j w_j * FFN8_{e_j}(x_t) with the token's
+ * row quantised as above. W1q [E, w1_cols, H] with scales s1 [E, w1_cols]; W2q [E, H, F]
+ * with s2 [E, H] (as oracle_quant_cols_fp8 writes them). out [ntok, H] fp64. */
+int oracle_moe_tokens_fp8(int T, int H, int F, int E, int k, int act, int gate, const uint16_t *x,
+                          const uint16_t *Wg, const float *bias, const uint8_t *W1q,
+                          const float *s1, const uint8_t *W2q, const float *s2, int ntok,
+                          const int32_t *tokens, double *out, int32_t *idx_out, double *w_out)
+{
+    if (H < 1 || F < 1 || E < 1 || k < 1 || k > E || ntok < 0) return -1;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -2;
+    const int w1_cols = act == ORACLE_ACT_SWIGLU ? 2 * F : F;
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = oracle_e4m3_decode((uint8_t)c);
+    int bad = 0;
+#pragma omp parallel
+    {
+        float *l = (float *)malloc(sizeof(float) * (size_t)E);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        double *z = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+        float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+        uint8_t *xq = (uint8_t *)malloc((size_t)H);
+        float *hf = (float *)malloc(sizeof(float) * (size_t)F);
+        uint8_t *hq = (uint8_t *)malloc((size_t)F);
+        const int ok = l && taken && sel && w && y && z && xf && xq && hf && hq;
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < ntok; ++i) {
+            if (!ok) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            const int t = tokens[i];
+            const uint16_t *xr = x + (size_t)t * H;
+            oracle_router_logits(1, H, E, xr, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, l);
+            topk_one(E, k, gate, l, bias, sel, w, taken);
+            for (int h = 0; h < H; ++h) xf[h] = bf16_to_float(xr[h]);
+            const float sx = quant_vec(H, xf, 1, xq, 1);
+            double *o = out + (size_t)i * H;
+            for (int n = 0; n < H; ++n) o[n] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                const int e = sel[j];
+                ffn_row_fp8(H, F, act, dec, xq, sx, W1q + (size_t)e * w1_cols * H,
+                            s1 + (size_t)e * w1_cols, W2q + (size_t)e * H * F, s2 + (size_t)e * H,
+                            y, z, hf, hq);
+                for (int n = 0; n < H; ++n) o[n] += y[n] * w[j];
+            }
+            if (idx_out) memcpy(idx_out + (size_t)i * k, sel, sizeof(int32_t) * (size_t)k);
+            if (w_out) memcpy(w_out + (size_t)i * k, w, sizeof(double) * (size_t)k);
+        }
+        free(l);
+        free(taken);
+        free(sel);
+        free(w);
+        free(y);
+        free(z);
+        free(xf);
+        free(xq);
+        free(hf);
+        free(hq);
     }
     return bad ? -4 : 0;
 }

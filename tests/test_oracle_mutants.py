@@ -53,6 +53,18 @@ MUTANTS = [
      "oracle_router_logits(T, H, E, x, Wg, bias, logits);"),
     ("select_bias_ignored_in_selection", "? l[e] + bias[e] : l[e];", "? l[e] : l[e];"),
     ("shared_gate_wrong_sign", "g = 1.0 / (1.0 + exp(-z));", "g = 1.0 / (1.0 + exp(z));"),
+    ("e4m3_ties_away_from_zero", "code = ((ex + 7) << 3) + m;",
+     "code = ((ex + 7) << 3) + (int)round((ldexp(a, -ex) - 1.0) * 8.0);"),
+    ("e4m3_no_subnormals", "code = (int)nearbyint(ldexp(a, 9));", "code = 0;"),
+    ("e4m3_exponent_bias_8", "const int ex = e - 1;", "const int ex = e - 2;"),
+    ("fp8_scale_for_e5m2_range", "*r = 448.0f / amax;", "*r = 240.0f / amax;"),
+    ("fp8_weight_scale_per_row", "for (int kk = 0; kk < K; ++kk) v[kk] = bf16_to_float(col[(size_t)kk * N]);",
+     "for (int kk = 0; kk < K; ++kk) v[kk] = bf16_to_float(col[(size_t)kk]);"),
+    ("fp8_h_scale_dropped", "y[n] = acc * (double)sh * (double)s2[n];", "y[n] = acc * (double)s2[n];"),
+    ("fp8_x_scale_dropped", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)s1[c];"),
+    ("fp8_w1_scale_of_column_0", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)sx * (double)s1[0];"),
+    ("fp8_gate_up_swapped", "silu(z[f]) * z[f + F]", "silu(z[f + F]) * z[f]"),
+    ("fp8_token_path_drops_gate", "o[n] += y[n] * w[j];", "o[n] += y[n];"),
     ("shared_ffn_uses_gate_half_only", "ffn_row(H, Fs, ORACLE_ACT_SWIGLU, 0, xr, W1s, W2s, y, scratch);",
      "ffn_row(H, Fs, ORACLE_ACT_GELU_TANH, 0, xr, W1s, W2s, y, scratch);"),
 ]

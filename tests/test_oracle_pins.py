@@ -394,3 +394,134 @@ def test_shared_expert_term(oracle_lib):
     got = oracle.shared_tokens(xb, W1s, W2s, bf16(wsg), np.array([0, 1], np.int32), lib=oracle_lib)
     for i, z in enumerate([-1.0, 5.0]):
         np.testing.assert_allclose(got[i], g_ffn[i] / (1 + math.exp(-z)), rtol=1e-14, atol=1e-300)
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 (e4m3) experts (a precision variant outside the pages)
+# ---------------------------------------------------------------------------------------
+
+def _e4m3_table():
+    """Every e4m3 code's value written out from the format's definition (sign, 4-bit
+    exponent with bias 7, 3-bit mantissa, subnormals at exponent 0, S.1111.111 NaN), built
+    here with Python integer arithmetic, independently of the oracle's decoder."""
+    vals = []
+    for c in range(256):
+        s, ef, m = c >> 7, (c >> 3) & 15, c & 7
+        if ef == 15 and m == 7:
+            vals.append(math.nan)
+            continue
+        v = m * 2.0 ** -9 if ef == 0 else (8 + m) * 2.0 ** (ef - 10)
+        vals.append(-v if s else v)
+    return np.array(vals)
+
+
+def test_e4m3_decode_known_codes(oracle_lib):
+    table = _e4m3_table()
+    got = oracle.e4m3_decode(np.arange(256, dtype=np.uint8), lib=oracle_lib)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(table))
+    ok = ~np.isnan(table)
+    np.testing.assert_array_equal(got[ok], table[ok])
+    # a few values stated outright
+    assert got[0x38] == 1.0 and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+    assert got[0x08] == 2.0 ** -6 and got[0x40] == 2.0 and got[0x3F] == 1.875
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and got[0xB8] == -1.0
+    # the positive finite codes are strictly increasing
+    assert np.all(np.diff(got[:0x7F]) > 0)
+
+
+def test_e4m3_encode_is_nearest_ties_to_even(oracle_lib):
+    """Brute force over every finite code: the nearest value, ties to the even code,
+    magnitudes above 448 saturate, on the codes' values, their midpoints, the floats just
+    either side of each midpoint, random values and the special values."""
+    table = _e4m3_table()
+    pos = table[:0x7F]  # codes 0x00..0x7E, increasing
+    mids = (pos[:-1] + pos[1:]) / 2
+    mids32 = mids.astype(np.float32)
+    assert np.all(mids32.astype(np.float64) == mids)  # the midpoints are exact in fp32
+    rng = np.random.default_rng(7)
+    v = np.concatenate([
+        pos, mids32, np.nextafter(mids32, np.float32(np.inf)), np.nextafter(mids32, np.float32(0)),
+        rng.uniform(-500, 500, 20000), rng.uniform(-0.02, 0.02, 20000),
+        np.ldexp(rng.uniform(1, 2, 5000), rng.integers(-12, 10, 5000)),
+        [448.0, 449.0, 463.9, 464.0, 480.0, 1e6, 2.0 ** -10, 3 * 2.0 ** -11]]).astype(np.float32)
+    v = np.concatenate([v, -v])
+    got = oracle.e4m3_encode(v, lib=oracle_lib)
+    a = np.abs(v.astype(np.float64))
+    d = np.abs(a[:, None] - pos[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    # among equally near codes take the even one (at most two are equally near)
+    code = np.where(cand & (np.arange(0x7F)[None, :] % 2 == 0), np.arange(0x7F)[None, :], 999).min(axis=1)
+    code = np.where(cand.sum(axis=1) == 1, d.argmin(axis=1), code)
+    code = np.where(a > 448.0, 0x7E, code)
+    want = (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+    np.testing.assert_array_equal(got, want)
+    specials = np.array([np.inf, -np.inf, np.nan, -0.0, 0.0], np.float32)
+    sg = oracle.e4m3_encode(specials, lib=oracle_lib)
+    assert list(sg[:2]) == [0x7E, 0xFE] and (sg[2] & 0x7F) == 0x7F and list(sg[3:]) == [0x80, 0x00]
+
+
+def test_fp8_row_quantisation_worked_example(oracle_lib):
+    """Row [100, 1, -2, 0]: r = 448/100 = 4.48 -> 448 (0x7E), 4.48 -> 4.5 (0x49),
+    -8.96 -> -9 (0xD1), 0 (0x00); scale 100/448 in fp32. A zero row keeps scale 1."""
+    q, s = oracle.quant_rows_fp8(bf16([[100, 1, -2, 0], [0, 0, 0, 0]]), lib=oracle_lib)
+    assert list(q[0]) == [0x7E, 0x49, 0xD1, 0x00] and list(q[1]) == [0, 0, 0, 0]
+    assert s[0] == np.float32(100) / np.float32(448) and s[1] == 1.0
+
+
+def test_fp8_column_quantisation_worked_example(oracle_lib):
+    """W [1, K=3, N=2], columns (100, 1, -2) and (0.5, -0.25, 0.125): per-column scales and
+    the transposed (K contiguous) code layout. Column 1: r = 896 -> 448 (0x7E),
+    -224 (0xF6), 112 (0x6E)."""
+    W = bf16([[[100, 0.5], [1, -0.25], [-2, 0.125]]])
+    q, s = oracle.quant_cols_fp8(W, lib=oracle_lib)
+    assert q.shape == (1, 2, 3)
+    assert list(q[0, 0]) == [0x7E, 0x49, 0xD1] and list(q[0, 1]) == [0x7E, 0xF6, 0x6E]
+    assert s[0, 0] == np.float32(100) / np.float32(448) and s[0, 1] == np.float32(0.5) / np.float32(448)
+
+
+def _fp8_layer(seed, T, H, F, E, k, act):
+    g = torch.Generator().manual_seed(seed)
+    w1c = 2 * F if act == oracle.ACT_SWIGLU else F
+    x = rand_bf16((T, H), seed)
+    Wg = rand_bf16((H, E), seed + 1, 1 / math.sqrt(H))
+    # columns of very different size (factors 1/8 .. 2), so a scale taken from the wrong
+    # column or row is far off
+    c1 = 2.0 ** (np.arange(w1c) % 5 - 3)
+    c2 = 2.0 ** (np.arange(H) % 5 - 3)
+    W1 = (torch.randn(E, H, w1c, generator=g) / math.sqrt(H) * torch.from_numpy(c1).float())
+    W2 = (torch.randn(E, F, H, generator=g) / math.sqrt(F) * torch.from_numpy(c2).float())
+    return x, Wg, synth.bf16_bits(W1.to(torch.bfloat16)), synth.bf16_bits(W2.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_SWIGLU, oracle.ACT_RELU])
+def test_fp8_layer_is_close_to_bf16_layer(oracle_lib, act):
+    """The e4m3 layer equals the bf16 layer up to the quantisation error: each code is within
+    2^-4 relative of its value (3 mantissa bits), so the outputs agree to a few percent."""
+    T, H, F, E, k = 24, 128, 96, 4, 2
+    x, Wg, W1, W2 = _fp8_layer(3, T, H, F, E, k, act)
+    W1q, s1 = oracle.quant_cols_fp8(W1, lib=oracle_lib)
+    W2q, s2 = oracle.quant_cols_fp8(W2, lib=oracle_lib)
+    toks = np.arange(T)
+    ref, ridx, _ = oracle.moe_tokens(x, Wg, None, W1, W2, k, toks, act=act, lib=oracle_lib)
+    got, gidx, _ = oracle.moe_tokens_fp8(x, Wg, None, W1q, s1, W2q, s2, k, toks, act=act,
+                                        lib=oracle_lib)
+    np.testing.assert_array_equal(gidx, ridx)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 0.08, rel
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_IDENTITY, oracle.ACT_RELU])
+def test_fp8_layer_scales_exactly_with_the_input(oracle_lib, act):
+    """One expert (gate 1): with a positively homogeneous activation, x -> 2^j x leaves every
+    code unchanged and multiplies every scale, hence the output, by exactly 2^j."""
+    T, H, F, E, k = 8, 64, 64, 1, 1
+    x, Wg, W1, W2 = _fp8_layer(5, T, H, F, E, k, act)
+    W1q, s1 = oracle.quant_cols_fp8(W1, lib=oracle_lib)
+    W2q, s2 = oracle.quant_cols_fp8(W2, lib=oracle_lib)
+    toks = np.arange(T)
+    out, _, _ = oracle.moe_tokens_fp8(x, Wg, None, W1q, s1, W2q, s2, k, toks, act=act, lib=oracle_lib)
+    x8 = bf16(widen(x) * 8.0)
+    out8, _, _ = oracle.moe_tokens_fp8(x8, Wg, None, W1q, s1, W2q, s2, k, toks, act=act, lib=oracle_lib)
+    np.testing.assert_array_equal(out8, 8.0 * out)
+    assert np.abs(out).max() > 0
