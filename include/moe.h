@@ -221,6 +221,60 @@ MOE_API moe_status moe_forward_shared(const moe_problem *p, const moe_bf16 *x,
                                       moe_bf16 *out, int32_t *topk_idx_out, float *topk_w_out,
                                       void *ws, size_t ws_bytes, void *stream);
 
+/* FP8 experts (a precision variant beyond the pages, which fix no precision).
+ * Element format e4m3 (OCP 8-bit floating point: 1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, largest finite magnitude 448), stored as one byte per value.
+ * Scaling of one vector v (a token row of x or of h over its K values, or one output column
+ * of W1 or W2 over its K values): r = 448 / max|v|, s = max|v| / 448, both rounded to fp32
+ * (r = s = 1 when r is not finite); code = e4m3(v * r), the product rounded to fp32, then
+ * the nearest e4m3 value, ties to even, saturating at 448; v ~ decode(code) * s.
+ * Weights are stored transposed, K contiguous: W1q [E, w1_cols, H] with s1 [E, w1_cols]
+ * (w1_cols = 2F for SwiGLU, columns [0,F) gate and [F,2F) up, else F), W2q [E, H, F] with
+ * s2 [E, H]. The FP8 path needs H % 128 == 0 and F % 128 == 0 (MOE_ERR_UNSUPPORTED
+ * otherwise). All pointers are device pointers, 16-byte aligned. */
+typedef uint8_t moe_fp8;
+
+/* One-off preparation: the e4m3 codes and per-column scales of W1 [E, H, w1_cols] and
+ * W2 [E, F, H] (bf16, as moe_forward takes them). Asynchronous on `stream`. */
+MOE_API moe_status moe_quantize_experts_fp8(const moe_problem *p, const moe_bf16 *W1,
+                                            const moe_bf16 *W2, moe_fp8 *W1q, float *s1,
+                                            moe_fp8 *W2q, float *s2, void *stream);
+
+/* Per-row quantisation of src [rows, cols] bf16 (cols % 8 == 0; src 16-byte and dst 8-byte
+ * aligned) into dst [rows, cols] codes and scale [rows]: the step moe_forward_fp8 applies
+ * to x and to h. */
+MOE_API moe_status moe_quantize_rows_fp8(const moe_bf16 *src, int64_t rows, int32_t cols,
+                                         moe_fp8 *dst, float *scale, void *stream);
+
+/* Workspace bytes for moe_forward_fp8 on *p (it covers every bf16 entry point as well);
+ * 0 if *p is invalid or unsupported on the FP8 path. */
+MOE_API size_t moe_workspace_size_fp8(const moe_problem *p);
+
+/* The layer with e4m3 experts. Routing and dispatch are the bf16 path's (x and W_g in bf16,
+ * fp32 logits, bit-identical selection). Then: x rows quantised; layer0 on codes
+ * (tcgen05 kind::f8f6f4, fp32 accumulation), each accumulator times s_x[token] * s1[column],
+ * the activation, h stored bf16; h rows quantised; layer1 on codes, times
+ * s_h[row] * s2[column] * the gate weight, stored bf16; the combine as moe_forward.
+ * moe_forward_launches(p) counts the same route and dispatch kernels; this path launches
+ * 2 + 3 + 1 + 1 + 1 + 1 kernels after the router (dispatch, x quantisation, layer0,
+ * h quantisation, layer1, combine). */
+MOE_API moe_status moe_forward_fp8(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                                   const float *bias, const moe_fp8 *W1q, const float *s1,
+                                   const moe_fp8 *W2q, const float *s2, moe_bf16 *out,
+                                   int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* moe_forward_fp8 with caller events recorded at the MOE_NUM_STAGE_EVENTS stage boundaries
+ * (as moe_forward_staged; the x quantisation is in the dispatch stage, the h quantisation
+ * in the layer1 stage). */
+MOE_API moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *x,
+                                          const moe_bf16 *Wg, const float *bias,
+                                          const moe_fp8 *W1q, const float *s1,
+                                          const moe_fp8 *W2q, const float *s2, moe_bf16 *out,
+                                          int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                                          size_t ws_bytes, void *stream, void *const *events,
+                                          int32_t n_events);
+
 /* Combine (§2.1: gather and reduce the top-k outputs).
  *   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] ), fp32 sum, j ascending.
  * ys [ys_rows, H] bf16 holds expert-sorted rows that already carry their gate weight;

@@ -94,6 +94,12 @@ def library() -> ctypes.CDLL:
             "moe_workspace_size_shared": ([P, i32], sz),
             "moe_forward_shared": ([P, vp, vp, vp, vp, vp, ctypes.POINTER(SharedExpert), vp, vp,
                                     vp, vp, sz, vp], i32),
+            "moe_workspace_size_fp8": ([P], sz),
+            "moe_quantize_experts_fp8": ([P, vp, vp, vp, vp, vp, vp, vp], i32),
+            "moe_quantize_rows_fp8": ([vp, i64, i32, vp, vp, vp], i32),
+            "moe_forward_fp8": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "moe_forward_fp8_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                        ctypes.POINTER(vp), i32], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
             "moe_get_device_status": ([vp, vp], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
@@ -284,6 +290,68 @@ def moe_forward_shared(p, x, Wg, bias, W1, W2, W1s, W2s, w_sg, out, ws, topk_idx
                                       _ptr(topk_w_out, torch.float32, "topk_w_out"), w, n,
                                       _stream(stream))
     _check("moe_forward_shared", rc)
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 (e4m3) experts: codes are torch.uint8 tensors, scales torch.float32
+# ---------------------------------------------------------------------------------------
+
+def moe_workspace_size_fp8(p: Problem) -> int:
+    """Workspace bytes for moe_forward_fp8 (0: invalid or unsupported on the FP8 path)."""
+    return int(library().moe_workspace_size_fp8(ctypes.byref(p)))
+
+
+def moe_quantize_experts_fp8(p, W1, W2, W1q, s1, W2q, s2, stream=None):
+    """W1 [E, H, w1_cols], W2 [E, F, H] bf16 -> W1q [E, w1_cols, H], W2q [E, H, F] uint8 codes
+    and per-column scales s1 [E, w1_cols], s2 [E, H] float32."""
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    rc = library().moe_quantize_experts_fp8(ctypes.byref(p), _ptr(W1, bf, "W1"), _ptr(W2, bf, "W2"),
+                                            _ptr(W1q, u8, "W1q"), _ptr(s1, f32, "s1"),
+                                            _ptr(W2q, u8, "W2q"), _ptr(s2, f32, "s2"),
+                                            _stream(stream))
+    _check("moe_quantize_experts_fp8", rc)
+
+
+def moe_quantize_rows_fp8(src, dst, scale, stream=None):
+    """src [rows, cols] bf16 -> dst [rows, cols] uint8 codes, scale [rows] float32."""
+    rows, cols = src.shape
+    rc = library().moe_quantize_rows_fp8(_ptr(src, torch.bfloat16, "src"), ctypes.c_int64(rows),
+                                         cols, _ptr(dst, torch.uint8, "dst"),
+                                         _ptr(scale, torch.float32, "scale"), _stream(stream))
+    _check("moe_quantize_rows_fp8", rc)
+
+
+def _fp8_args(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out, topk_w_out):
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    return (ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"), _ptr(bias, f32, "bias"),
+            _ptr(W1q, u8, "W1q"), _ptr(s1, f32, "s1"), _ptr(W2q, u8, "W2q"), _ptr(s2, f32, "s2"),
+            _ptr(out, bf, "out"), _ptr(topk_idx_out, torch.int32, "topk_idx_out"),
+            _ptr(topk_w_out, f32, "topk_w_out"))
+
+
+def moe_forward_fp8(p, x, Wg, bias, W1q, s1, W2q, s2, out, ws, topk_idx_out=None,
+                    topk_w_out=None, stream=None):
+    """The layer with e4m3 experts (codes and scales from moe_quantize_experts_fp8)."""
+    w, n = _ws(ws)
+    rc = library().moe_forward_fp8(*_fp8_args(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out,
+                                              topk_w_out), w, n, _stream(stream))
+    _check("moe_forward_fp8", rc)
+
+
+def moe_forward_fp8_staged(p, x, Wg, bias, W1q, s1, W2q, s2, out, ws, events, topk_idx_out=None,
+                           topk_w_out=None, stream=None):
+    """moe_forward_fp8 with MOE_NUM_STAGE_EVENTS timing events at the stage boundaries."""
+    w, n = _ws(ws)
+    if len(events) != MOE_NUM_STAGE_EVENTS:
+        raise ValueError(f"need {MOE_NUM_STAGE_EVENTS} events")
+    for ev in events:
+        if ev.cuda_event == 0:
+            ev.record()
+    arr = (ctypes.c_void_p * MOE_NUM_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    rc = library().moe_forward_fp8_staged(*_fp8_args(p, x, Wg, bias, W1q, s1, W2q, s2, out,
+                                                     topk_idx_out, topk_w_out), w, n,
+                                          _stream(stream), arr, MOE_NUM_STAGE_EVENTS)
+    _check("moe_forward_fp8_staged", rc)
 
 
 def moe_combine(p, ys, inv_pos, out, ws=None, stream=None):

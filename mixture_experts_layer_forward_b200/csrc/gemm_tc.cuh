@@ -61,6 +61,10 @@ constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*b_mn_major=*/true);
+// e4m3 operands: both K-major; a K step of 128 values is the same 128-byte row as 64 bf16
+// values, so the stage layout, the swizzle and the four MMAs per stage are unchanged
+constexpr uint32_t IDESC_F8 = idesc_e4m3_f32(BM, BN);
+constexpr int B8_BOX_ROWS = 128; // e4m3 B tile: two boxes of 128 weight rows x 128 K bytes
 // descriptor strides
 constexpr uint32_t A_SBO = 1024; // 8 rows x 128 B
 constexpr uint32_t A_LBO = 16;   // unused for swizzled K-major
@@ -115,6 +119,12 @@ struct GemmArgs {
     float *out_f32;
     float *xsq_f32; // optional: sum of squares of every A row over each split's K range,
                     // [k_split, dense_rows] (the epilogue warps read the staged A tiles)
+    // e4m3 operands (moe_grouped_gemm_f8_kernel): the accumulator of row r, column c of
+    // expert e is multiplied by a_scale[token of r] (gathered rows) or a_scale[r], then by
+    // b_scale[e * b_scale_ld + c]
+    const float *a_scale;
+    const float *b_scale;
+    int b_scale_ld;
 };
 
 __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
@@ -181,11 +191,22 @@ __device__ __forceinline__ float act_f(int act, float z)
 // Epilogue of one accumulator tile for the 32 rows of this warp: thread `lane` owns row `row`
 // and reads its TMEM lane `t_row` (already offset to the accumulator buffer). Warp-collective
 // (tcgen05.ld), so the whole warp calls it.
-template <int KIND>
+template <int KIND, bool F8 = false>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt,
-                                              int ks = 0)
+                                              int ks = 0, int e = 0)
 {
     using namespace gemm;
+    // e4m3 operands: the row's scale (0 for pad rows, whose outputs are never read)
+    float sa = 1.0f;
+    if (F8) {
+        if (args.gather_idx != nullptr) {
+            const int t = row < args.gather_len ? args.gather_idx[row] : -1;
+            sa = (t >= 0 && t < args.gather_rows) ? args.a_scale[t] : 0.0f;
+        } else {
+            sa = args.a_scale[row];
+        }
+    }
+    const float *sb = F8 ? args.b_scale + (size_t)e * args.b_scale_ld : nullptr;
     if (KIND == GEMM_SWIGLU) {
         __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * 128;
 #pragma unroll 1
@@ -198,13 +219,31 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
+                    float sg[8], su[8]; // column scales of the 8 gate and 8 up columns
+                    if (F8) {
+                        const int c0 = nt * 128 + c * 32 + v * 8;
+                        const float4 *pg = reinterpret_cast<const float4 *>(sb + c0);
+                        const float4 *pu = reinterpret_cast<const float4 *>(sb + args.up_col + c0);
+                        const float4 g0 = pg[0], g1 = pg[1], u0 = pu[0], u1 = pu[1];
+                        sg[0] = g0.x; sg[1] = g0.y; sg[2] = g0.z; sg[3] = g0.w;
+                        sg[4] = g1.x; sg[5] = g1.y; sg[6] = g1.z; sg[7] = g1.w;
+                        su[0] = u0.x; su[1] = u0.y; su[2] = u0.z; su[3] = u0.w;
+                        su[4] = u1.x; su[5] = u1.y; su[6] = u1.z; su[7] = u1.w;
+                    }
                     uint32_t p[4];
 #pragma unroll
                     for (int h2 = 0; h2 < 4; ++h2) {
                         const int i = v * 8 + h2 * 2;
-                        const float a0 = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-                        const float a1 =
-                            silu_f(__uint_as_float(g[i + 1])) * __uint_as_float(u[i + 1]);
+                        float g0 = __uint_as_float(g[i]), g1 = __uint_as_float(g[i + 1]);
+                        float u0 = __uint_as_float(u[i]), u1 = __uint_as_float(u[i + 1]);
+                        if (F8) {
+                            g0 = (g0 * sa) * sg[h2 * 2];
+                            g1 = (g1 * sa) * sg[h2 * 2 + 1];
+                            u0 = (u0 * sa) * su[h2 * 2];
+                            u1 = (u1 * sa) * su[h2 * 2 + 1];
+                        }
+                        const float a0 = silu_f(g0) * u0;
+                        const float a1 = silu_f(g1) * u1;
                         p[h2] = pack_bf16x2(a0, a1);
                     }
                     dst[v] = make_uint4(p[0], p[1], p[2], p[3]);
@@ -240,12 +279,23 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
+                    float sc[8]; // column scales of these 8 columns
+                    if (F8) {
+                        const float4 *pc = reinterpret_cast<const float4 *>(sb + nt * BN + c * 32 + v * 8);
+                        const float4 c0 = pc[0], c1 = pc[1];
+                        sc[0] = c0.x; sc[1] = c0.y; sc[2] = c0.z; sc[3] = c0.w;
+                        sc[4] = c1.x; sc[5] = c1.y; sc[6] = c1.z; sc[7] = c1.w;
+                    }
                     uint32_t p[4];
 #pragma unroll
                     for (int h2 = 0; h2 < 4; ++h2) {
                         const int i = v * 8 + h2 * 2;
                         float a0 = __uint_as_float(r[i]);
                         float a1 = __uint_as_float(r[i + 1]);
+                        if (F8) {
+                            a0 = (a0 * sa) * sc[h2 * 2];
+                            a1 = (a1 * sa) * sc[h2 * 2 + 1];
+                        }
                         if (KIND == GEMM_SCALE) {
                             a0 *= wt;
                             a1 *= wt;
@@ -263,7 +313,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
-template <int KIND>
+template <int KIND, bool F8 = false>
 __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                                  const GemmArgs &args, uint8_t *smem, int w_first,
                                                  int w_step)
@@ -341,10 +391,18 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                     }
                     const uint32_t a_dst = smem_u32(smem + s * STAGE);
                     const uint32_t b_dst = a_dst + A_TILE;
-                    mbar_arrive_expect_tx(full_bar(s), (gather ? 0 : A_TILE) + nbox * B_BOX);
+                    mbar_arrive_expect_tx(full_bar(s),
+                                          (gather ? 0 : A_TILE) + (F8 ? B_TILE : nbox * B_BOX));
                     armed[s] = (int)ph;
-                    if (!gather) tma_load_2d(a_dst, &tmA, full_bar(s), kb * BK, mt * BM);
-                    for (int i = 0; i < nbox; ++i) {
+                    // the x coordinate is the K offset in elements: 128 B per k-block either way
+                    if (!gather) tma_load_2d(a_dst, &tmA, full_bar(s), kb * (F8 ? 128 : BK), mt * BM);
+                    if (F8) { // K-major e4m3 weights [E, N rows, K]: two boxes of 128 rows
+                        const int r0 = (KIND == GEMM_SWIGLU) ? nt * 128 : nt * BN;
+                        const int r1 = (KIND == GEMM_SWIGLU) ? args.up_col + nt * 128 : nt * BN + B8_BOX_ROWS;
+                        tma_load_3d(b_dst, &tmB, full_bar(s), kb * 128, r0, e);
+                        tma_load_3d(b_dst + B8_BOX_ROWS * 128, &tmB, full_bar(s), kb * 128, r1, e);
+                    }
+                    for (int i = 0; i < (F8 ? 0 : nbox); ++i) {
                         int col;
                         if (KIND == GEMM_SWIGLU)
                             col = (i < 2 ? nt * 128 + i * 64 : args.up_col + nt * 128 + (i - 2) * 64);
@@ -403,13 +461,23 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                     const uint32_t a_addr = smem_u32(smem + s * STAGE);
                     const uint32_t b_addr = a_addr + A_TILE;
                     const uint64_t a_desc = sw128_desc(a_addr, A_LBO, A_SBO);
-                    const uint64_t b_desc = sw128_desc(b_addr, B_LBO, B_SBO);
+                    if (F8) {
+                        // both K-major: +32 B (32 e4m3 values) per MMA inside the swizzle atom
+                        const uint64_t b_desc = sw128_desc(b_addr, A_LBO, A_SBO);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        // A: +32 B per K=16 step inside the swizzle atom; B: +16 rows x 128 B
-                        umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
-                                  b_desc + (uint64_t)((k * 16 * 128) >> 4), idesc,
-                                  (kb != kb_first || k != 0) ? 1u : 0u);
+                        for (int k = 0; k < 4; ++k)
+                            umma_f8(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                    b_desc + (uint64_t)((k * 32) >> 4), IDESC_F8,
+                                    (kb != kb_first || k != 0) ? 1u : 0u);
+                    } else {
+                        const uint64_t b_desc = sw128_desc(b_addr, B_LBO, B_SBO);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            // A: +32 B per K=16 step inside the swizzle atom; B: +16 rows x 128 B
+                            umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                      b_desc + (uint64_t)((k * 16 * 128) >> 4), idesc,
+                                      (kb != kb_first || k != 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit(empty_bar(s));
                     if (++s == STAGES) {
@@ -440,13 +508,17 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             for (int w = w_first; w < total; w += w_step) {
                 int e, mt, nt;
                 gemm_map_work(w, args, e, mt, nt);
-                const __nv_bfloat16 *src[8];
+                // row addresses in bytes: a k-block is the next 128 bytes of every row (64
+                // bf16 or 128 e4m3 values)
+                const uint8_t *src[8];
+                const size_t ld_bytes = (size_t)args.gather_ld * (F8 ? 1 : 2);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int64_t r = (int64_t)mt * BM + r0 + 16 * i;
                     int t = (r < args.gather_len) ? args.gather_idx[r] : -1;
                     if (t < 0 || t >= args.gather_rows) t = 0; // pad rows read token 0; never used
-                    src[i] = args.gather_src + (size_t)t * args.gather_ld + chunk * 8;
+                    src[i] = reinterpret_cast<const uint8_t *>(args.gather_src) + (size_t)t * ld_bytes +
+                             chunk * 16;
                 }
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) { // layer0 only: never split
@@ -461,7 +533,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                     for (int i = 0; i < 8; ++i) {
                         const int r = r0 + 16 * i;
                         const uint32_t dst = a_dst + r * 128 + ((chunk ^ (r & 7)) << 4);
-                        cp_async_16_cg(dst, src[i] + kb * BK);
+                        cp_async_16_cg(dst, src[i] + (size_t)kb * 128);
                     }
                     cp_async_arrive_noinc(full_bar(s));
                     if (++s == STAGES) {
@@ -526,7 +598,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             tc_fence_after();
             const int row = mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            epilogue_rows<KIND>(args, t_row, row, nt, ks);
+            epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
@@ -551,6 +623,20 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     grouped_gemm_cta<KIND>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
+}
+
+// The same persistent grouped GEMM on e4m3 operands (tcgen05 kind::f8f6f4): A rows of 128-
+// value k-blocks (gathered x codes for layer0, h codes by TMA for layer1), B the expert's
+// K-major code matrix [N rows, K]; the epilogue applies the row and column scales first.
+template <int KIND>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_grouped_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
+                               const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    grouped_gemm_cta<KIND, true>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
 }
 
 

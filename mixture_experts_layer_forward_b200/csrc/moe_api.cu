@@ -11,6 +11,7 @@
 
 #include "combine.cuh"
 #include "dispatch.cuh"
+#include "fp8.cuh"
 #include "fused.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -69,8 +70,8 @@ struct Layout {
         counts, offsets, poff, tile_off,
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
-        x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys;
-    size_t end_route, end_dispatch, end_forward, end_host, end_shared;
+        x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys, xq, sx, hq, sh;
+    size_t end_route, end_dispatch, end_forward, end_host, end_shared, end_fp8;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
 };
@@ -127,7 +128,7 @@ FilterPlan filter_plan(const moe_problem *p)
     return f;
 }
 
-Layout make_layout(const moe_problem *p, int F_s = 0)
+Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false)
 {
     Layout L{};
     const size_t T = (size_t)p->T, H = (size_t)p->H, F = (size_t)p->F, E = (size_t)p->E,
@@ -185,6 +186,12 @@ Layout make_layout(const moe_problem *p, int F_s = 0)
     L.sh_h = take(F_s > 0 ? Tpad * (size_t)F_s * 2 : 0);
     L.sh_ys = take(F_s > 0 ? Tpad * H * 2 : 0);
     L.end_shared = o;
+    // FP8 experts (moe_forward_fp8): e4m3 codes of x and h with their row scales
+    L.xq = take(fp8 ? T * H : 0);
+    L.sx = take(fp8 ? T * 4 : 0);
+    L.hq = take(fp8 ? P * F : 0);
+    L.sh = take(fp8 ? P * 4 : 0);
+    L.end_fp8 = o;
     return L;
 }
 
@@ -261,6 +268,35 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows
     cuuint32_t box[3] = {64, 64, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D uint8 [rows, cols] (e4m3 codes); box = 128 bytes x box_rows rows, 128-byte swizzle.
+bool make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D uint8 [depth, rows, cols] (per-expert e4m3 code matrices, K contiguous);
+// box = 128 bytes x 128 rows x 1, 128-byte swizzle.
+bool make_map_3d_u8(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {cols, rows, depth};
+    cuuint64_t strides[2] = {cols, rows * cols};
+    cuuint32_t box[3] = {128, (cuuint32_t)gemm::B8_BOX_ROWS, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -495,6 +531,51 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
 }
 
 template <int KIND>
+cudaError_t launch_gemm_f8(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                           int max_work, cudaStream_t st)
+{
+    auto kern = moe_grouped_gemm_f8_kernel<KIND>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    int grid = sm_count();
+    if (grid <= 0) grid = 148;
+    if (grid > max_work) grid = max_work;
+    if (grid < 1) grid = 1;
+    const int threads = args.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    kern<<<grid, threads, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const moe_bf16 *src, int64_t rows, int cols, const DispatchMeta *meta,
+                              uint8_t *dst, float *scale, cudaStream_t st)
+{
+    if (rows <= 0) return cudaSuccess;
+    int grid = sm_count() * 8;
+    if (grid <= 0) grid = 1184;
+    if ((int64_t)grid > rows) grid = (int)rows;
+    quant_rows_fp8_kernel<<<grid, Q_THREADS, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(src),
+                                                      rows, cols, meta, M_TILE, dst, scale);
+    return cudaGetLastError();
+}
+
+// W [E, K, N] -> Wq [E, N, K] codes and per-column scales [E, N]
+cudaError_t launch_quant_cols(const moe_bf16 *W, int E, int K, int N, uint8_t *Wq, float *scale,
+                              cudaStream_t st)
+{
+    const __nv_bfloat16 *w = reinterpret_cast<const __nv_bfloat16 *>(W);
+    quant_cols_amax_kernel<<<dim3((N + 127) / 128, E), 256, 0, st>>>(w, K, N, scale);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    quant_cols_codes_kernel<<<dim3(N / 64, K / 64, E), 256, 0, st>>>(w, K, N, scale, Wq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n = (int64_t)E * N;
+    quant_cols_scale_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(scale, n);
+    return cudaGetLastError();
+}
+
+template <int KIND>
 cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
                              int max_work, cudaStream_t st)
 {
@@ -643,6 +724,30 @@ cudaError_t launch_shared(const moe_problem *p, const moe_bf16 *x, const moe_sha
     return launch_gemm<GEMM_SCALE>(m_h, m_w2, a1, mt * a1.n_tiles, st);
 }
 
+// The dispatch outputs inside the caller's workspace.
+DispatchOut dispatch_bufs(void *ws, const Layout &L)
+{
+    DispatchOut d;
+    d.counts = at<int32_t>(ws, L.counts);
+    d.offsets = at<int32_t>(ws, L.offsets);
+    d.poff = at<int32_t>(ws, L.poff);
+    d.gather_idx = at<int32_t>(ws, L.gather_idx);
+    d.inv_pos = at<int32_t>(ws, L.inv_pos);
+    d.tile_off = at<int32_t>(ws, L.tile_off);
+    d.tile_expert = at<int32_t>(ws, L.tile_expert);
+    d.chunk = at<int32_t>(ws, L.chunk);
+    d.ptile_off = at<int32_t>(ws, L.ptile_off);
+    d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
+    d.hot_off = at<int32_t>(ws, L.hot_off);
+    d.hot_tile_expert = at<int32_t>(ws, L.hot_tile_expert);
+    d.cold_tile = at<int32_t>(ws, L.cold_tile);
+    d.ready = at<int>(ws, L.ready);
+    d.n_ready = L.n_ready;
+    d.row_w = at<float>(ws, L.row_w);
+    d.meta = at<DispatchMeta>(ws, L.meta);
+    return d;
+}
+
 moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
@@ -671,24 +776,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     }
     int32_t *topk_idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
     float *topk_w = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
-    DispatchOut d;
-    d.counts = at<int32_t>(ws, L.counts);
-    d.offsets = at<int32_t>(ws, L.offsets);
-    d.poff = at<int32_t>(ws, L.poff);
-    d.gather_idx = at<int32_t>(ws, L.gather_idx);
-    d.inv_pos = at<int32_t>(ws, L.inv_pos);
-    d.tile_off = at<int32_t>(ws, L.tile_off);
-    d.tile_expert = at<int32_t>(ws, L.tile_expert);
-    d.chunk = at<int32_t>(ws, L.chunk);
-    d.ptile_off = at<int32_t>(ws, L.ptile_off);
-    d.ptile_expert = at<int32_t>(ws, L.ptile_expert);
-    d.hot_off = at<int32_t>(ws, L.hot_off);
-    d.hot_tile_expert = at<int32_t>(ws, L.hot_tile_expert);
-    d.cold_tile = at<int32_t>(ws, L.cold_tile);
-    d.ready = at<int>(ws, L.ready);
-    d.n_ready = L.n_ready;
-    d.row_w = at<float>(ws, L.row_w);
-    d.meta = at<DispatchMeta>(ws, L.meta);
+    const DispatchOut d = dispatch_bufs(ws, L);
     moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
     moe_bf16 *h = at<moe_bf16>(ws, L.h);
     moe_bf16 *ys = at<moe_bf16>(ws, L.ys);
@@ -816,6 +904,119 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         if (e == cudaSuccess) e = record(events, n_events, 4, st);
     }
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, ys_s);
+    if (e == cudaSuccess) e = record(events, n_events, 5, st);
+    return to_status(e);
+}
+
+// Shapes the FP8 expert path supports: both GEMMs' K (H and F) in whole 128-value k-blocks.
+moe_status check_problem_fp8(const moe_problem *p)
+{
+    const moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (p->H % 128 != 0 || p->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// The layer with e4m3 experts: route and dispatch as in forward_impl (bf16 x and W_g), then
+// x rows quantised, layer0 on codes (single-CTA persistent kernel, kind::f8f6f4, gathered
+// rows), h rows quantised, layer1 on codes, the combine. Stage events as moe_forward_staged
+// (the x quantisation falls in the dispatch stage, the h quantisation in the layer1 stage).
+moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                            const float *bias, const moe_fp8 *W1q, const float *s1,
+                            const moe_fp8 *W2q, const float *s2, moe_bf16 *out,
+                            int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                            cudaStream_t st, void *const *events, int n_events)
+{
+    moe_status s = check_problem_fp8(p);
+    if (s != MOE_OK) return s;
+    if (n_events != 0 && (n_events != MOE_NUM_STAGE_EVENTS || events == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (ws == nullptr || (p->T > 0 && (x == nullptr || out == nullptr)) || Wg == nullptr ||
+        W1q == nullptr || W2q == nullptr || s1 == nullptr || s2 == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, 0, true);
+    if (ws_bytes < L.end_fp8) return MOE_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(W1q) || !aligned16(W2q) || !aligned16(Wg) ||
+        !aligned16(s1) || !aligned16(s2) || !aligned16(ws) || !aligned4(bias) ||
+        !aligned4(topk_idx_out) || !aligned4(topk_w_out))
+        return MOE_ERR_INVALID_ARG;
+    int *status = at<int>(ws, L.status);
+    if (p->T == 0) {
+        cudaError_t e = cudaMemsetAsync(status, 0, 8, st);
+        for (int i = 0; i < n_events && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+        return to_status(e);
+    }
+    int32_t *topk_idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+    float *topk_w = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
+    const DispatchOut d = dispatch_bufs(ws, L);
+    moe_bf16 *h = at<moe_bf16>(ws, L.h);
+    moe_bf16 *ys = at<moe_bf16>(ws, L.ys);
+    uint8_t *xq = at<uint8_t>(ws, L.xq), *hq = at<uint8_t>(ws, L.hq);
+    float *sx = at<float>(ws, L.sx), *sh = at<float>(ws, L.sh);
+
+    const int F = p->F, H = p->H, E = p->E;
+    const bool gated = (p->act == MOE_ACT_SWIGLU);
+    const int w1_cols = gated ? 2 * F : F;
+    CUtensorMap m_x, m_w1, m_h, m_w2;
+    if (!make_map_2d_u8(&m_x, xq, (uint64_t)p->T, (uint64_t)H, 1) || // unused: rows are gathered
+        !make_map_3d_u8(&m_w1, W1q, (uint64_t)E, (uint64_t)w1_cols, (uint64_t)H) ||
+        !make_map_2d_u8(&m_h, hq, (uint64_t)L.pmax, (uint64_t)F, gemm::BM) ||
+        !make_map_3d_u8(&m_w2, W2q, (uint64_t)E, (uint64_t)H, (uint64_t)F))
+        return MOE_ERR_CUDA;
+
+    const int64_t timeout = g_timeout_ns.load();
+    const FilterBufs fb = filter_bufs(ws, L);
+    cudaError_t e = record(events, n_events, 0, st);
+    if (e == cudaSuccess)
+        e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st,
+                         &fb);
+    if (e == cudaSuccess) e = record(events, n_events, 1, st);
+    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
+    if (e == cudaSuccess) e = launch_quant_rows(x, p->T, H, nullptr, xq, sx, st);
+    if (e == cudaSuccess) e = record(events, n_events, 2, st);
+
+    GemmArgs a0{};
+    a0.tile_off = d.tile_off;
+    a0.tile_expert = d.tile_expert;
+    a0.meta = d.meta;
+    a0.order = ORDER_EXPERT;
+    a0.gather_idx = d.gather_idx;
+    a0.gather_len = L.pmax;
+    a0.gather_src = reinterpret_cast<const __nv_bfloat16 *>(xq); // bytes: the codes of x
+    a0.gather_rows = p->T;
+    a0.gather_ld = H;
+    a0.out = reinterpret_cast<__nv_bfloat16 *>(h);
+    a0.ld_out = F;
+    a0.n_cols = F;
+    a0.k_blocks = H / 128;
+    a0.up_col = F;
+    a0.act = p->act;
+    a0.status = status;
+    a0.timeout_ns = timeout;
+    a0.n_tiles = gated ? F / 128 : (F + gemm::BN - 1) / gemm::BN;
+    a0.a_scale = sx;
+    a0.b_scale = s1;
+    a0.b_scale_ld = w1_cols;
+    GemmArgs a1 = a0;
+    a1.gather_idx = nullptr; // layer1 reads the h codes in place (TMA)
+    a1.row_w = d.row_w;
+    a1.out = reinterpret_cast<__nv_bfloat16 *>(ys);
+    a1.ld_out = H;
+    a1.n_cols = H;
+    a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+    a1.k_blocks = F / 128;
+    a1.a_scale = sh;
+    a1.b_scale = s2;
+    a1.b_scale_ld = H;
+
+    if (e == cudaSuccess)
+        e = gated ? launch_gemm_f8<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st)
+                  : launch_gemm_f8<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+    if (e == cudaSuccess) e = record(events, n_events, 3, st);
+    if (e == cudaSuccess) e = launch_quant_rows(h, L.pmax, F, d.meta, hq, sh, st);
+    if (e == cudaSuccess) e = launch_gemm_f8<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
+    if (e == cudaSuccess) e = record(events, n_events, 4, st);
+    if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, nullptr);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);
     return to_status(e);
 }
@@ -1162,6 +1363,63 @@ int moe_route_uses_filter(const moe_problem *p)
 {
     if (check_problem(p) != MOE_OK) return -1;
     return route_uses_filter(p) ? 1 : 0;
+}
+
+size_t moe_workspace_size_fp8(const moe_problem *p)
+{
+    if (check_problem_fp8(p) != MOE_OK) return 0;
+    return make_layout(p, 0, true).end_fp8;
+}
+
+moe_status moe_quantize_rows_fp8(const moe_bf16 *src, int64_t rows, int32_t cols, moe_fp8 *dst,
+                                 float *scale, void *stream)
+{
+    if (rows < 0 || cols <= 0 || cols % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (src == nullptr || dst == nullptr || scale == nullptr || !aligned16(src) ||
+        (reinterpret_cast<uintptr_t>(dst) & 7u) != 0 || !aligned4(scale))
+        return MOE_ERR_INVALID_ARG;
+    return to_status(launch_quant_rows(src, rows, cols, nullptr, dst, scale,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_quantize_experts_fp8(const moe_problem *p, const moe_bf16 *W1, const moe_bf16 *W2,
+                                    moe_fp8 *W1q, float *s1, moe_fp8 *W2q, float *s2, void *stream)
+{
+    moe_status s = check_problem_fp8(p);
+    if (s != MOE_OK) return s;
+    if (W1 == nullptr || W2 == nullptr || W1q == nullptr || W2q == nullptr || s1 == nullptr ||
+        s2 == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(W1) || !aligned16(W2) || !aligned16(W1q) || !aligned16(W2q) || !aligned16(s1) ||
+        !aligned16(s2))
+        return MOE_ERR_INVALID_ARG;
+    const int w1_cols = p->act == MOE_ACT_SWIGLU ? 2 * p->F : p->F;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_quant_cols(W1, p->E, p->H, w1_cols, W1q, s1, st);
+    if (e == cudaSuccess) e = launch_quant_cols(W2, p->E, p->F, p->H, W2q, s2, st);
+    return to_status(e);
+}
+
+moe_status moe_forward_fp8(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                           const float *bias, const moe_fp8 *W1q, const float *s1,
+                           const moe_fp8 *W2q, const float *s2, moe_bf16 *out,
+                           int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                           void *stream)
+{
+    return forward_impl_fp8(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out, topk_w_out, ws,
+                            ws_bytes, static_cast<cudaStream_t>(stream), nullptr, 0);
+}
+
+moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                                  const float *bias, const moe_fp8 *W1q, const float *s1,
+                                  const moe_fp8 *W2q, const float *s2, moe_bf16 *out,
+                                  int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                                  size_t ws_bytes, void *stream, void *const *events,
+                                  int32_t n_events)
+{
+    return forward_impl_fp8(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out, topk_w_out, ws,
+                            ws_bytes, static_cast<cudaStream_t>(stream), events, n_events);
 }
 
 int moe_set_fault_injection(int layer0_item)

@@ -212,6 +212,19 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// tcgen05.mma kind::f8f6f4 (cta_group::1): D[tmem] (+)= A * B with 8-bit operands (K = 32
+// per instruction, i.e. 32 bytes of every row, the same bytes as one kind::f16 step).
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on the mbarrier when every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
@@ -265,6 +278,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | (1u << 10)                                // B format: bf16
            | (0u << 15)                                // A major: K
            | ((b_mn_major ? 1u : 0u) << 16)            // B major
+           | ((uint32_t)(N >> 3) << 17)                // N / 8
+           | ((uint32_t)(M >> 4) << 24);               // M / 16
+}
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: fp32 accumulator, e4m3 A and B (format
+// code 0 in both fields), both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                                   // D format: f32
+           | (0u << 7)                                 // A format: e4m3
+           | (0u << 10)                                // B format: e4m3
            | ((uint32_t)(N >> 3) << 17)                // N / 8
            | ((uint32_t)(M >> 4) << 24);               // M / 16
 }

@@ -156,3 +156,16 @@ def test_route_uses_filter_follows_mode_and_shape(lib):
         assert moe.moe_route_uses_filter(mixtral)
     finally:
         moe.moe_set_router_mode(prev)
+
+
+def test_fp8_workspace_and_argument_checks(lib):
+    p = moe.Problem.make(300, 256, 256, 16, 2)
+    assert moe.moe_workspace_size_fp8(p) > moe.moe_workspace_size(p)
+    assert moe.moe_workspace_size_fp8(moe.Problem.make(300, 192, 256, 16, 2)) == 0  # H % 128
+    assert moe.moe_workspace_size_fp8(moe.Problem.make(300, 256, 192, 16, 2)) == 0  # F % 128
+    # host-detected errors: nothing is launched
+    assert lib.moe_quantize_rows_fp8(None, 4, 12, None, None, None) == -1             # cols % 8
+    assert lib.moe_quantize_experts_fp8(ctypes.byref(p), None, None, None, None, None, None,
+                                        None) == -1
+    assert lib.moe_forward_fp8(ctypes.byref(p), None, None, None, None, None, None, None, None,
+                               None, None, None, 0, None) == -1
