@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
+    ap.add_argument("--fp8", action="store_true",
+                    help="e4m3 experts (moe_forward_fp8; weights quantised once before timing)")
     ap.add_argument("--router-only", action="store_true",
                     help="time moe_route alone (router logits + top-k); no expert weights allocated")
     return ap.parse_args()
@@ -98,6 +100,7 @@ def config_dict(cfg, args, n):
         "l2": "inputs larger than L2 (per-step working set >> 126 MB); no flush",
         "seed": args.seed,
         "gemm_mode": getattr(args, "gemm_mode", "auto"),
+        "experts": "e4m3 codes, fp32 row/column scales" if getattr(args, "fp8", False) else "bf16",
     }
 
 
@@ -311,14 +314,31 @@ def run_ours(args):
     inp = synth.make_inputs(cfg, seed=args.seed, device=dev,
                             x_seed=dp.replica_x_seed(args.seed, rank) if world > 1 else None)
     p = moe.Problem.from_config(cfg)
-    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    args_fwd = (p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out, ws)
+    if args.fp8:
+        # one-off weight preparation, outside the timed region
+        w1c = 2 * cfg.F if cfg.act == 0 else cfg.F
+        q = (torch.empty(cfg.E, w1c, cfg.H, dtype=torch.uint8, device=dev),
+             torch.empty(cfg.E, w1c, dtype=torch.float32, device=dev),
+             torch.empty(cfg.E, cfg.H, cfg.F, dtype=torch.uint8, device=dev),
+             torch.empty(cfg.E, cfg.H, dtype=torch.float32, device=dev))
+        moe.moe_quantize_experts_fp8(p, inp["W1"], inp["W2"], *q)
+        del inp["W1"], inp["W2"]
+        torch.cuda.empty_cache()
+        ws = torch.empty(moe.moe_workspace_size_fp8(p), dtype=torch.uint8, device=dev)
+        args_fwd = (p, inp["x"], inp["Wg"], inp["bias"], *q, out, ws)
+        fwd = lambda idx=None: moe.moe_forward_fp8(*args_fwd, topk_idx_out=idx)
+        fwd_staged = lambda ev: moe.moe_forward_fp8_staged(*args_fwd, ev)
+    else:
+        ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
+        args_fwd = (p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out, ws)
+        fwd = lambda idx=None: moe.moe_forward(*args_fwd, idx)
+        fwd_staged = lambda ev: moe.moe_forward_staged(*args_fwd, ev)
 
     idx_buf = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
     for _ in range(W):
-        moe.moe_forward(*args_fwd, idx_buf)
+        fwd(idx_buf)
     torch.cuda.synchronize(dev)
     assert moe.moe_get_device_status(ws) == 0, "device status after warm-up"
     active_experts = int(torch.unique(idx_buf).numel())  # for the layer0 byte count below
@@ -342,7 +362,7 @@ def run_ours(args):
     t_begin = time.time()
     start.record(stream)
     for i in range(K):
-        moe.moe_forward_staged(*args_fwd, evs[i])
+        fwd_staged(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     t_end = time.time()
@@ -363,7 +383,7 @@ def run_ours(args):
     # its out back (pinned host memory); moe_forward_host_batches overlaps step i's compute
     # with step i+1's copy in and step i-1's copy out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.fp8:
         x_h = inp["x"].cpu().pin_memory()
         out_h = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         outs = [out_h[i & 1] for i in range(K)]
@@ -391,23 +411,29 @@ def run_ours(args):
                                  clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]))
     regime = "sustained" if sustained else "burst"
     tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
+    # the e4m3 contraction's peak: the measured bf16 peak times the nominal ratio (4.5 / 2.25)
+    gemm_peak = 2.0 * tf_peak if args.fp8 else tf_peak
     layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
     # layer0: useful FLOPs (padding rows not counted) and algorithmic bytes (each active
     # expert's W1 once, x once, h of the routed rows written once); the bound is whichever
     # takes longer at the measured peaks
     w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
     gemm0_flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
-    gemm0_bytes = 2 * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H + cfg.T * cfg.k * cfg.F)
+    # (e4m3 experts: 1-byte weights and x codes; h is still written in bf16)
+    wb = 1 if args.fp8 else 2
+    gemm0_bytes = (wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) +
+                   2 * cfg.T * cfg.k * cfg.F)
     g0_ms = stage_ms["layer0_gemm_swiglu"]
     g0_s = g0_ms / 1e3
-    kernel = DOMINANT_KERNEL[args.gemm_mode]
-    hbm_bound = gemm0_bytes / (peaks["hbm_gbs"] * 1e9) > gemm0_flops / (tf_peak * 1e12)
+    kernel = "moe_grouped_gemm_f8_kernel<0>" if args.fp8 else DOMINANT_KERNEL[args.gemm_mode]
+    hbm_bound = gemm0_bytes / (peaks["hbm_gbs"] * 1e9) > gemm0_flops / (gemm_peak * 1e12)
     if hbm_bound:
         achieved, peak, unit = gemm0_bytes / g0_s / 1e9, peaks["hbm_gbs"], "GB/s"
         psrc = f"{peak_src} HBM copy bandwidth"
     else:
-        achieved, peak, unit = gemm0_flops / g0_s / 1e12, tf_peak, "TFLOP/s"
-        psrc = f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)"
+        achieved, peak, unit = gemm0_flops / g0_s / 1e12, gemm_peak, "TFLOP/s"
+        psrc = (f"{peak_src} bf16 {regime} x 2 (nominal e4m3/bf16 ratio)" if args.fp8 else
+                f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)")
     roofline = {"bound": "hbm" if hbm_bound else "tensor", "kernel": kernel,
                 "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic_for(kernel, cfg.name), "peak_source": psrc,
@@ -418,21 +444,24 @@ def run_ours(args):
     line = {
         "metric": "MoE-layer forward tokens/s", "value": n * cfg.T / (ms_per_step / 1e3),
         "unit": "tokens/s", "n_gpus": n, "steps": K, "warmup": W, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 experts (bf16 router, fp32 accumulation)" if args.fp8 else "bf16",
         "data": "synthetic (seeded random inputs and random-init weights of the layer's shape)",
         "config": config_dict(cfg, args, n),
         "tflops": layer_tflops * n,
-        "layer_roofline": {"bound": "tensor", "achieved": layer_tflops, "peak": tf_peak,
-                           "unit": "TFLOP/s per GPU", "frac": layer_tflops / tf_peak,
-                           "peak_source": f"{peak_src} bf16 {regime}"},
+        "layer_roofline": {"bound": "tensor", "achieved": layer_tflops, "peak": gemm_peak,
+                           "unit": "TFLOP/s per GPU", "frac": layer_tflops / gemm_peak,
+                           "peak_source": f"{peak_src} bf16 {regime}" + (" x 2" if args.fp8 else "")},
         "roofline": roofline,
         "stage_ms": stage_ms,
-        "gpu_launches": moe.moe_forward_launches(p) * K,
+        # FP8: router, 3 dispatch kernels, x quantisation, layer0, h quantisation, layer1, combine
+        "gpu_launches": ((3 if moe.moe_route_uses_filter(p) else 2) + 8 if args.fp8 else
+                         moe.moe_forward_launches(p)) * K,
         "clocks": clocks,
         "e2e": e2e,
     }
 
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and not args.fp8:
         hin = host_inputs(inp)
         v, n_tok, t, threads = cpu_oracle_sample(cfg, hin, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
