@@ -425,7 +425,7 @@ def run_ours(args):
                    2 * cfg.T * cfg.k * cfg.F)
     g0_ms = stage_ms["layer0_gemm_swiglu"]
     g0_s = g0_ms / 1e3
-    kernel = "moe_grouped_gemm_f8_kernel<0>" if args.fp8 else DOMINANT_KERNEL[args.gemm_mode]
+    kernel = "moe_grouped_gemm_select_f8_kernel<0>" if args.fp8 else DOMINANT_KERNEL[args.gemm_mode]
     hbm_bound = gemm0_bytes / (peaks["hbm_gbs"] * 1e9) > gemm0_flops / (gemm_peak * 1e12)
     if hbm_bound:
         achieved, peak, unit = gemm0_bytes / g0_s / 1e9, peaks["hbm_gbs"], "GB/s"

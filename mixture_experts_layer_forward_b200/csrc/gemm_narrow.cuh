@@ -23,6 +23,10 @@
 // Roles, barriers, bounded waits and TMEM handling follow gemm_tc.cuh: warp 0 TMA producer,
 // warp 1 MMA issuer (two accumulators of up to 128 columns), warps 2-5 epilogue, warps 6-9
 // layer0 row gather.
+// e4m3 operands (F8): the weight codes are K-major ([E, N rows, K]), so A is two boxes of 64
+// weight rows x 128 K bytes (the same 8 KB per box), both operands K-major, the MMA
+// kind::f8f6f4; the epilogue multiplies each accumulator by its row's and column's scales
+// first (as gemm_tc.cuh's).
 #pragma once
 
 #include "gemm_tc.cuh"
@@ -94,7 +98,7 @@ __device__ __forceinline__ NarrowItem narrow_item(int w, const GemmArgs &a)
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
-template <int KIND>
+template <int KIND, bool F8 = false>
 __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                                                         const CUtensorMap &tmX,
                                                         const GemmArgs &args, uint8_t *smem,
@@ -169,9 +173,13 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                         const int col = (KIND == GEMM_SWIGLU)
                                             ? (i == 0 ? it.cb * 64 : args.up_col + it.cb * 64)
                                             : it.cb * BM + i * 64;
-                        tma_load_3d(a_dst + i * A_BOX, &tmW, full_bar(s), col, kb * BK, it.e);
+                        if (F8) // K-major codes: x = the k-block's byte offset, y = weight row
+                            tma_load_3d(a_dst + i * A_BOX, &tmW, full_bar(s), kb * 128, col, it.e);
+                        else
+                            tma_load_3d(a_dst + i * A_BOX, &tmW, full_bar(s), col, kb * BK, it.e);
                     }
-                    if (!gather) tma_load_2d(b_dst, &tmX, full_bar(s), kb * BK, it.mt * 128);
+                    if (!gather)
+                        tma_load_2d(b_dst, &tmX, full_bar(s), kb * (F8 ? 128 : BK), it.mt * 128);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -194,7 +202,8 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
             bool ok = true;
             for (int w = w_first; ok && w < total; w += w_step, ++it_n) {
                 const NarrowItem it = narrow_item(w, args);
-                const uint32_t idesc = idesc_bf16_f32_swapped(BM, it.n_pad);
+                const uint32_t idesc =
+                    F8 ? idesc_e4m3_f32(BM, it.n_pad) : idesc_bf16_f32_swapped(BM, it.n_pad);
                 const int acc = it_n & 1;
                 const uint32_t aph = (uint32_t)(it_n >> 1) & 1u;
                 if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, args.timeout_ns,
@@ -214,14 +223,24 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * STAGE);
                     const uint32_t b_addr = a_addr + A_TILE;
-                    const uint64_t a_desc = sw128_desc(a_addr, A_LBO, A_SBO);
                     const uint64_t b_desc = sw128_desc(b_addr, B_LBO, B_SBO);
+                    if (F8) {
+                        // both K-major: +32 B (32 e4m3 values) per MMA
+                        const uint64_t a_desc = sw128_desc(a_addr, B_LBO, B_SBO);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        // A (MN-major): +16 K rows x 128 B per K=16 step; B (K-major): +32 B
-                        umma_bf16(d_tmem, a_desc + (uint64_t)((k * 16 * 128) >> 4),
-                                  b_desc + (uint64_t)((k * 32) >> 4), idesc,
-                                  (kb | k) != 0 ? 1u : 0u);
+                        for (int k = 0; k < 4; ++k)
+                            umma_f8(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                    b_desc + (uint64_t)((k * 32) >> 4), idesc,
+                                    (kb | k) != 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t a_desc = sw128_desc(a_addr, A_LBO, A_SBO);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            // A (MN-major): +16 K rows x 128 B per K=16 step; B (K-major): +32 B
+                            umma_bf16(d_tmem, a_desc + (uint64_t)((k * 16 * 128) >> 4),
+                                      b_desc + (uint64_t)((k * 32) >> 4), idesc,
+                                      (kb | k) != 0 ? 1u : 0u);
+                        }
                     }
                     umma_commit(empty_bar(s));
                     if (++s == STAGES) {
@@ -248,13 +267,15 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
             uint32_t ph = 0;
             for (int w = w_first; w < total; w += w_step) {
                 const NarrowItem it = narrow_item(w, args);
-                const __nv_bfloat16 *src[8];
+                const uint8_t *src[8]; // byte addresses: a k-block is 128 bytes of a row
+                const size_t ld_bytes = (size_t)args.gather_ld * (F8 ? 1 : 2);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int64_t r = (int64_t)it.mt * 128 + r0 + 16 * i;
                     int t = (r < args.gather_len) ? args.gather_idx[r] : -1;
                     if (t < 0 || t >= args.gather_rows) t = 0; // pad rows read token 0
-                    src[i] = args.gather_src + (size_t)t * args.gather_ld + chunk * 8;
+                    src[i] = reinterpret_cast<const uint8_t *>(args.gather_src) + (size_t)t * ld_bytes +
+                             chunk * 16;
                 }
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
@@ -270,7 +291,7 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                         const int r = r0 + 16 * i;
                         if (r < it.n_pad) {
                             const uint32_t dst = b_dst + r * 128 + ((chunk ^ (r & 7)) << 4);
-                            cp_async_16_cg(dst, src[i] + kb * BK);
+                            cp_async_16_cg(dst, src[i] + (size_t)kb * 128);
                         }
                     }
                     cp_async_arrive_noinc(full_bar(s));
@@ -300,12 +321,37 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 128);
             const int64_t row0 = (int64_t)it.mt * 128;
+            // e4m3: this lane's weight-column scale (SwiGLU: q < 2 gate, q >= 2 up columns)
+            float sb = 1.0f;
+            if (F8) {
+                const int wcol = (KIND == GEMM_SWIGLU)
+                                     ? (q < 2 ? it.cb * 64 + q * 32 + lane
+                                              : args.up_col + it.cb * 64 + (q - 2) * 32 + lane)
+                                     : it.cb * BM + q * 32 + lane;
+                sb = wcol < args.b_scale_ld ? args.b_scale[(size_t)it.e * args.b_scale_ld + wcol] : 0.0f;
+            }
 #pragma unroll 1
             for (int c0 = 0; c0 < it.n_pad; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c0, r);
                 tmem_ld_wait();
                 const int nc = (it.n_pad - c0) < 32 ? (it.n_pad - c0) : 32;
+                if (F8) { // row scale (0 for pad rows), then this lane's column scale
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i < nc) {
+                            const int64_t row = row0 + c0 + i;
+                            float sa;
+                            if (args.gather_idx != nullptr) {
+                                const int t = row < args.gather_len ? args.gather_idx[row] : -1;
+                                sa = (t >= 0 && t < args.gather_rows) ? args.a_scale[t] : 0.0f;
+                            } else {
+                                sa = args.a_scale[row];
+                            }
+                            r[i] = __float_as_uint((__uint_as_float(r[i]) * sa) * sb);
+                        }
+                    }
+                }
                 if (KIND == GEMM_SWIGLU) {
                     if (q >= 2) { // up columns: hand them to the gate lanes
                         float *dst = xch + (size_t)((q - 2) * 32 + lane) * XCH_LD + c0;
@@ -387,6 +433,25 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         grouped_gemm_narrow_cta<KIND>(tmB, tmA, narrow, smem, blockIdx.x, gridDim.x);
     else
         grouped_gemm_cta<KIND>(tmA, tmB, wide, smem, blockIdx.x, gridDim.x);
+}
+
+// The e4m3 form of moe_grouped_gemm_select_kernel: the narrow body reads the weight codes
+// through tmWn (64-row boxes), the 128-row body through tmB (128-row boxes).
+template <int KIND>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_grouped_gemm_select_f8_kernel(const __grid_constant__ CUtensorMap tmA,
+                                      const __grid_constant__ CUtensorMap tmB,
+                                      const __grid_constant__ CUtensorMap tmWn,
+                                      const GemmArgs wide, const GemmArgs narrow)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int num_cold = wide.meta->num_cold;
+    if (num_cold > 0 && num_cold == wide.meta->num_tiles)
+        grouped_gemm_narrow_cta<KIND, true>(tmWn, tmA, narrow, smem, blockIdx.x, gridDim.x);
+    else
+        grouped_gemm_cta<KIND, true>(tmA, tmB, wide, smem, blockIdx.x, gridDim.x);
 }
 
 } // namespace moe

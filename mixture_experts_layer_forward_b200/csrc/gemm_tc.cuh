@@ -119,7 +119,7 @@ struct GemmArgs {
     float *out_f32;
     float *xsq_f32; // optional: sum of squares of every A row over each split's K range,
                     // [k_split, dense_rows] (the epilogue warps read the staged A tiles)
-    // e4m3 operands (moe_grouped_gemm_f8_kernel): the accumulator of row r, column c of
+    // e4m3 operands (moe_grouped_gemm_select_f8_kernel): the accumulator of row r, column c of
     // expert e is multiplied by a_scale[token of r] (gathered rows) or a_scale[r], then by
     // b_scale[e * b_scale_ld + c]
     const float *a_scale;
@@ -625,19 +625,6 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     grouped_gemm_cta<KIND>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
 }
 
-// The same persistent grouped GEMM on e4m3 operands (tcgen05 kind::f8f6f4): A rows of 128-
-// value k-blocks (gathered x codes for layer0, h codes by TMA for layer1), B the expert's
-// K-major code matrix [N rows, K]; the epilogue applies the row and column scales first.
-template <int KIND>
-__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
-    moe_grouped_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
-                               const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    grouped_gemm_cta<KIND, true>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
-}
 
 
 // ---------------------------------------------------------------------------------------

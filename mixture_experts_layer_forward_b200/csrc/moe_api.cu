@@ -287,14 +287,15 @@ bool make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t co
 }
 
 // 3D uint8 [depth, rows, cols] (per-expert e4m3 code matrices, K contiguous);
-// box = 128 bytes x 128 rows x 1, 128-byte swizzle.
-bool make_map_3d_u8(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols)
+// box = 128 bytes x box_rows rows x 1, 128-byte swizzle.
+bool make_map_3d_u8(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows = gemm::B8_BOX_ROWS)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[3] = {cols, rows, depth};
     cuuint64_t strides[2] = {cols, rows * cols};
-    cuuint32_t box[3] = {128, (cuuint32_t)gemm::B8_BOX_ROWS, 1};
+    cuuint32_t box[3] = {128, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -530,20 +531,21 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
     return cudaGetLastError();
 }
 
+// e4m3 layer GEMM: one launch whose CTAs run the narrow (operand-swapped) body when every
+// expert owns a single m-tile, the 128-row body otherwise (decided on the device).
 template <int KIND>
-cudaError_t launch_gemm_f8(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
-                           int max_work, cudaStream_t st)
+cudaError_t launch_gemm_select_f8(const CUtensorMap &ta, const CUtensorMap &tb,
+                                  const CUtensorMap &twn, const GemmArgs &wide,
+                                  const GemmArgs &narrow, cudaStream_t st)
 {
-    auto kern = moe_grouped_gemm_f8_kernel<KIND>;
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    constexpr int smem = gemm::SMEM_BYTES > gemmn::SMEM_BYTES ? gemm::SMEM_BYTES : gemmn::SMEM_BYTES;
+    auto kern = moe_grouped_gemm_select_f8_kernel<KIND>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     int grid = sm_count();
     if (grid <= 0) grid = 148;
-    if (grid > max_work) grid = max_work;
-    if (grid < 1) grid = 1;
-    const int threads = args.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
-    kern<<<grid, threads, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+    const int threads = wide.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    kern<<<grid, threads, smem, st>>>(ta, tb, twn, wide, narrow);
     return cudaGetLastError();
 }
 
@@ -957,11 +959,14 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     const int F = p->F, H = p->H, E = p->E;
     const bool gated = (p->act == MOE_ACT_SWIGLU);
     const int w1_cols = gated ? 2 * F : F;
-    CUtensorMap m_x, m_w1, m_h, m_w2;
+    CUtensorMap m_x, m_w1, m_h, m_w2, n_w1, n_w2;
     if (!make_map_2d_u8(&m_x, xq, (uint64_t)p->T, (uint64_t)H, 1) || // unused: rows are gathered
         !make_map_3d_u8(&m_w1, W1q, (uint64_t)E, (uint64_t)w1_cols, (uint64_t)H) ||
         !make_map_2d_u8(&m_h, hq, (uint64_t)L.pmax, (uint64_t)F, gemm::BM) ||
-        !make_map_3d_u8(&m_w2, W2q, (uint64_t)E, (uint64_t)H, (uint64_t)F))
+        !make_map_3d_u8(&m_w2, W2q, (uint64_t)E, (uint64_t)H, (uint64_t)F) ||
+        // the narrow body's weight boxes: 64 rows
+        !make_map_3d_u8(&n_w1, W1q, (uint64_t)E, (uint64_t)w1_cols, (uint64_t)H, 64) ||
+        !make_map_3d_u8(&n_w2, W2q, (uint64_t)E, (uint64_t)H, (uint64_t)F, 64))
         return MOE_ERR_CUDA;
 
     const int64_t timeout = g_timeout_ns.load();
@@ -1008,13 +1013,19 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     a1.a_scale = sh;
     a1.b_scale = s2;
     a1.b_scale_ld = H;
+    // narrow items (every expert single-tile): column blocks of 64 (SwiGLU) or 128 columns
+    GemmArgs n0 = a0, n1 = a1;
+    n0.expert_rows = n1.expert_rows = d.counts;
+    n0.cold_tile = n1.cold_tile = d.cold_tile;
+    n0.n_tiles = gated ? F / 64 : (F + 127) / 128;
+    n1.n_tiles = (H + 127) / 128;
 
     if (e == cudaSuccess)
-        e = gated ? launch_gemm_f8<GEMM_SWIGLU>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st)
-                  : launch_gemm_f8<GEMM_ACT>(m_x, m_w1, a0, L.max_tiles * a0.n_tiles, st);
+        e = gated ? launch_gemm_select_f8<GEMM_SWIGLU>(m_x, m_w1, n_w1, a0, n0, st)
+                  : launch_gemm_select_f8<GEMM_ACT>(m_x, m_w1, n_w1, a0, n0, st);
     if (e == cudaSuccess) e = record(events, n_events, 3, st);
     if (e == cudaSuccess) e = launch_quant_rows(h, L.pmax, F, d.meta, hq, sh, st);
-    if (e == cudaSuccess) e = launch_gemm_f8<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
+    if (e == cudaSuccess) e = launch_gemm_select_f8<GEMM_SCALE>(m_h, m_w2, n_w2, a1, n1, st);
     if (e == cudaSuccess) e = record(events, n_events, 4, st);
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, nullptr);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);

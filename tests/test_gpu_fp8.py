@@ -93,6 +93,9 @@ FP8_CASES = [
     ("many_experts", 77, 128, 128, 64, 8, 0, 0.0),
     ("relu", 260, 256, 384, 4, 2, 2, 0.0),
     ("gelu_odd_n_tiles", 150, 384, 128, 4, 1, 1, 0.0),
+    # every expert single-tile: the operand-swapped narrow body
+    ("narrow_swiglu", 16, 256, 384, 32, 4, 0, 1.2),
+    ("narrow_relu", 40, 384, 256, 16, 2, 2, 0.0),
 ]
 
 
