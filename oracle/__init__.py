@@ -84,6 +84,10 @@ def load(path: Path | None = None) -> ctypes.CDLL:
     lib.oracle_quant_cols_fp8.restype = None
     lib.oracle_moe_tokens_fp8.argtypes = [i32] * 7 + [vp] * 7 + [i32, vp, vp, vp, vp]
     lib.oracle_moe_tokens_fp8.restype = i32
+    lib.oracle_moe_backward.argtypes = [i32] * 7 + [vp] * 11
+    lib.oracle_moe_backward.restype = i32
+    lib.oracle_moe_backward_dx_tokens.argtypes = [i32] * 7 + [vp] * 6 + [i32, vp, vp]
+    lib.oracle_moe_backward_dx_tokens.restype = i32
     _lib_cache[p] = lib
     return lib
 
@@ -318,3 +322,42 @@ def moe_tokens_fp8(x, Wg, bias, W1q, s1, W2q, s2, k, tokens, act=ACT_SWIGLU,
     if rc:
         raise ValueError(f"oracle_moe_tokens_fp8 rc={rc}")
     return out, idx, w
+
+
+# ---------------------------------------------------------------------------------------
+# Backward pass (training; beyond the pages): gradients of the layer for a given dL/dout
+# ---------------------------------------------------------------------------------------
+
+def moe_backward(x, Wg, bias, W1, W2, dy, k, act=ACT_SWIGLU, gate=GATE_SOFTMAX_TOPK, lib=None):
+    """All gradients (fp64): dict(dx [T,H], dWg [H,E], dbias [E], dW1 [E,H,w1c], dW2 [E,F,H])."""
+    lib = lib or load()
+    x, Wg, W1, W2, dy = _u16(x), _u16(Wg), _u16(W1), _u16(W2), _u16(dy)
+    T, H = x.shape
+    E, H1, F = _ffn_dims(W1, W2, act)
+    assert H1 == H and Wg.shape == (H, E) and dy.shape == (T, H)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    g = dict(dx=np.empty((T, H)), dWg=np.empty((H, E)), dbias=np.empty(E),
+             dW1=np.empty(W1.shape), dW2=np.empty(W2.shape))
+    rc = lib.oracle_moe_backward(T, H, F, E, k, act, gate, _p(x), _p(Wg), _p(b), _p(W1), _p(W2),
+                                 _p(dy), _p(g["dx"]), _p(g["dWg"]), _p(g["dbias"]), _p(g["dW1"]),
+                                 _p(g["dW2"]))
+    if rc:
+        raise ValueError(f"oracle_moe_backward rc={rc}")
+    return g
+
+
+def moe_backward_dx_tokens(x, Wg, bias, W1, W2, dy, k, tokens, act=ACT_SWIGLU,
+                           gate=GATE_SOFTMAX_TOPK, lib=None):
+    """Input gradient dx (fp64 [ntok, H]) of the listed tokens only."""
+    lib = lib or load()
+    x, Wg, W1, W2, dy = _u16(x), _u16(Wg), _u16(W1), _u16(W2), _u16(dy)
+    T, H = x.shape
+    E, _, F = _ffn_dims(W1, W2, act)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((tokens.size, H))
+    rc = lib.oracle_moe_backward_dx_tokens(T, H, F, E, k, act, gate, _p(x), _p(Wg), _p(b), _p(W1),
+                                           _p(W2), _p(dy), tokens.size, _p(tokens), _p(out))
+    if rc:
+        raise ValueError(f"oracle_moe_backward_dx_tokens rc={rc}")
+    return out

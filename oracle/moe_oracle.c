@@ -760,3 +760,218 @@ int oracle_moe_tokens_fp8(int T, int H, int F, int E, int k, int act, int gate, 
     }
     return bad ? -4 : 0;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Backward pass (training; a next-work item beyond the pages, which describe the forward)
+ *
+ * The forward is out[t] = sum_j w_j(t) y_{e_j}(x_t), y_e(x) = FFN_e(x) as in ffn_row, the
+ * selection fixed (piecewise constant in the inputs, so it carries no gradient), the gates
+ * w = softmax over the selected logits. Given dy = dL/dout (bf16 [T, H]), for each token t
+ * and selection j (e = e_j), in fp64 (the logits that feed the gates are the forward's fp32
+ * ones):
+ *   dw_j   = dy[t] . y_e(x_t)
+ *   dl_j   = w_j (dw_j - sum_i w_i dw_i)             (softmax over the selected logits)
+ *   gy     = w_j dy[t]                                (gradient at the expert output)
+ *   dW2[e] += a^T gy,  da = gy W2[e]^T                (a: the expert's hidden activation)
+ *   SwiGLU: dg_f = da_f u_f silu'(g_f), du_f = da_f silu(g_f); others: dz_f = da_f act'(z_f)
+ *   dW1[e] += x_t^T dz,  dx[t] += dz W1[e]^T
+ *   router: dx[t] += dl_j W_g[:, e],  dW_g[:, e] += x_t dl_j,  dbias[e] += dl_j
+ *           (SELECT_BIAS: the gates do not see the bias, so dbias stays 0)
+ * silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + e^-g). Gate mode SOFTMAX_ALL is not covered.
+ * ------------------------------------------------------------------------------------- */
+
+static double act_grad(int act, double z)
+{
+    switch (act) {
+    case ORACLE_ACT_GELU_TANH: {
+        const double c = sqrt(2.0 / acos(-1.0));
+        const double k3 = 4.4715e-2; /* the cubic coefficient of the tanh form */
+        const double th = tanh(c * (z + k3 * z * z * z));
+        return 0.5 * (1.0 + th) + 0.5 * z * (1.0 - th * th) * c * (1.0 + 3.0 * k3 * z * z);
+    }
+    case ORACLE_ACT_RELU:
+        return z > 0.0 ? 1.0 : 0.0;
+    case ORACLE_ACT_IDENTITY:
+    default:
+        return 1.0;
+    }
+}
+
+/* One (token, expert) pair: adds its contributions to dx_t [H], dW1e, dW2e (when not NULL)
+ * and returns dw = dy . y. gscale is the gate w_j. z, a, da: scratch of 2F, F, F doubles. */
+static double pair_backward(int H, int F, int act, const uint16_t *xr, const uint16_t *dyr,
+                            double gscale, const uint16_t *W1e, const uint16_t *W2e, double *dx_t,
+                            double *dW1e, double *dW2e, double *z, double *a, double *da)
+{
+    const int gated = (act == ORACLE_ACT_SWIGLU);
+    const int w1_cols = gated ? 2 * F : F;
+    for (int c = 0; c < w1_cols; ++c) z[c] = 0.0;
+    for (int h = 0; h < H; ++h) {
+        const double xh = (double)bf16_to_float(xr[h]);
+        const uint16_t *wrow = W1e + (size_t)h * w1_cols;
+        for (int c = 0; c < w1_cols; ++c) z[c] += xh * (double)bf16_to_float(wrow[c]);
+    }
+    for (int f = 0; f < F; ++f) a[f] = gated ? z[F + f] * silu(z[f]) : act_apply(act, z[f]);
+    /* dw = dy . (a W2); da = w dy W2^T; dW2 += a^T (w dy) */
+    double dw = 0.0;
+    for (int f = 0; f < F; ++f) {
+        const uint16_t *wrow = W2e + (size_t)f * H;
+        double s = 0.0;
+        for (int n = 0; n < H; ++n) s += (double)bf16_to_float(dyr[n]) * (double)bf16_to_float(wrow[n]);
+        dw += a[f] * s;
+        da[f] = gscale * s;
+        if (dW2e) {
+            double *drow = dW2e + (size_t)f * H;
+            for (int n = 0; n < H; ++n) drow[n] += a[f] * gscale * (double)bf16_to_float(dyr[n]);
+        }
+    }
+    /* dz (in place of z's gradient: reuse a as the gate part, z[F..] for up when gated) */
+    double *dz = z; /* the pre-activations are read before being overwritten below */
+    if (gated) {
+        for (int f = 0; f < F; ++f) {
+            const double g = z[f], u = z[F + f];
+            const double s = 1.0 / (1.0 + exp(-g));
+            const double dg = da[f] * u * s * (1.0 + g * (1.0 - s));
+            const double du = da[f] * g * s;
+            dz[f] = dg;
+            dz[F + f] = du;
+        }
+    } else {
+        for (int f = 0; f < F; ++f) dz[f] = da[f] * act_grad(act, z[f]);
+    }
+    for (int h = 0; h < H; ++h) {
+        const double xh = (double)bf16_to_float(xr[h]);
+        const uint16_t *wrow = W1e + (size_t)h * w1_cols;
+        double s = 0.0;
+        for (int c = 0; c < w1_cols; ++c) s += dz[c] * (double)bf16_to_float(wrow[c]);
+        dx_t[h] += s;
+        if (dW1e) {
+            double *drow = dW1e + (size_t)h * w1_cols;
+            for (int c = 0; c < w1_cols; ++c) drow[c] += xh * dz[c];
+        }
+    }
+    return dw;
+}
+
+/* Gradients of the whole layer (all T tokens): dx [T,H], dWg [H,E], dbias [E],
+ * dW1 [E,H,w1_cols], dW2 [E,F,H], all fp64; dy [T,H] bf16. Tokens are taken in order, so
+ * the weight-gradient sums run over tokens ascending. Returns -3 for SOFTMAX_ALL. */
+int oracle_moe_backward(int T, int H, int F, int E, int k, int act, int gate, const uint16_t *x,
+                        const uint16_t *Wg, const float *bias, const uint16_t *W1,
+                        const uint16_t *W2, const uint16_t *dy, double *dx, double *dWg,
+                        double *dbias, double *dW1, double *dW2)
+{
+    if (T < 0 || H < 1 || F < 1 || E < 1 || k < 1 || k > E) return -1;
+    if (gate == ORACLE_GATE_SOFTMAX_ALL) return -3;
+    const size_t w1e = w1_expert_elems(H, F, act);
+    const size_t w2e = (size_t)F * H;
+    memset(dx, 0, sizeof(double) * (size_t)T * H);
+    memset(dWg, 0, sizeof(double) * (size_t)H * E);
+    memset(dbias, 0, sizeof(double) * (size_t)E);
+    memset(dW1, 0, sizeof(double) * w1e * E);
+    memset(dW2, 0, sizeof(double) * w2e * E);
+    float *l = (float *)malloc(sizeof(float) * (size_t)E);
+    unsigned char *taken = (unsigned char *)malloc((size_t)E);
+    int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+    double *w = (double *)malloc(sizeof(double) * (size_t)k);
+    double *dw = (double *)malloc(sizeof(double) * (size_t)k);
+    double *z = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+    double *a = (double *)malloc(sizeof(double) * (size_t)F);
+    double *da = (double *)malloc(sizeof(double) * (size_t)F);
+    int rc = (l && taken && sel && w && dw && z && a && da) ? 0 : -4;
+    for (int t = 0; t < T && rc == 0; ++t) {
+        const uint16_t *xr = x + (size_t)t * H, *dyr = dy + (size_t)t * H;
+        oracle_router_logits(1, H, E, xr, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, l);
+        topk_one(E, k, gate, l, bias, sel, w, taken);
+        double *dxt = dx + (size_t)t * H;
+        for (int j = 0; j < k; ++j) {
+            const int e = sel[j];
+            dw[j] = pair_backward(H, F, act, xr, dyr, w[j], W1 + (size_t)e * w1e, W2 + (size_t)e * w2e,
+                                  dxt, dW1 + (size_t)e * w1e, dW2 + (size_t)e * w2e, z, a, da);
+        }
+        double wdw = 0.0;
+        for (int j = 0; j < k; ++j) wdw += w[j] * dw[j];
+        for (int j = 0; j < k; ++j) {
+            const int e = sel[j];
+            const double dl = (dw[j] - wdw) * w[j];
+            for (int h = 0; h < H; ++h) {
+                const size_t he = (size_t)h * E + e;
+                dxt[h] += dl * (double)bf16_to_float(Wg[he]);
+                dWg[he] += (double)bf16_to_float(xr[h]) * dl;
+            }
+            if (gate != ORACLE_GATE_SELECT_BIAS) dbias[e] += dl;
+        }
+    }
+    free(l);
+    free(taken);
+    free(sel);
+    free(w);
+    free(dw);
+    free(z);
+    free(a);
+    free(da);
+    return rc;
+}
+
+/* dx for a list of tokens only (each token's input gradient needs nothing of the others):
+ * dx_out [ntok, H] fp64. */
+int oracle_moe_backward_dx_tokens(int T, int H, int F, int E, int k, int act, int gate,
+                                  const uint16_t *x, const uint16_t *Wg, const float *bias,
+                                  const uint16_t *W1, const uint16_t *W2, const uint16_t *dy,
+                                  int ntok, const int32_t *tokens, double *dx_out)
+{
+    if (T < 0 || H < 1 || F < 1 || E < 1 || k < 1 || k > E || ntok < 0) return -1;
+    if (gate == ORACLE_GATE_SOFTMAX_ALL) return -3;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -2;
+    const size_t w1e = w1_expert_elems(H, F, act);
+    const size_t w2e = (size_t)F * H;
+    int bad = 0;
+#pragma omp parallel
+    {
+        float *l = (float *)malloc(sizeof(float) * (size_t)E);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        double *dw = (double *)malloc(sizeof(double) * (size_t)k);
+        double *z = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        double *da = (double *)malloc(sizeof(double) * (size_t)F);
+        const int ok = l && taken && sel && w && dw && z && a && da;
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < ntok; ++i) {
+            if (!ok) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            const int t = tokens[i];
+            const uint16_t *xr = x + (size_t)t * H, *dyr = dy + (size_t)t * H;
+            oracle_router_logits(1, H, E, xr, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, l);
+            topk_one(E, k, gate, l, bias, sel, w, taken);
+            double *dxt = dx_out + (size_t)i * H;
+            for (int h = 0; h < H; ++h) dxt[h] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                const int e = sel[j];
+                dw[j] = pair_backward(H, F, act, xr, dyr, w[j], W1 + (size_t)e * w1e,
+                                      W2 + (size_t)e * w2e, dxt, NULL, NULL, z, a, da);
+            }
+            double wdw = 0.0;
+            for (int j = 0; j < k; ++j) wdw += w[j] * dw[j];
+            for (int j = 0; j < k; ++j) {
+                const double dl = w[j] * (dw[j] - wdw);
+                for (int h = 0; h < H; ++h)
+                    dxt[h] += dl * (double)bf16_to_float(Wg[(size_t)h * E + sel[j]]);
+            }
+        }
+        free(l);
+        free(taken);
+        free(sel);
+        free(w);
+        free(dw);
+        free(z);
+        free(a);
+        free(da);
+    }
+    return bad ? -4 : 0;
+}

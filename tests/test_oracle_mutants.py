@@ -65,6 +65,15 @@ MUTANTS = [
     ("fp8_w1_scale_of_column_0", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)sx * (double)s1[0];"),
     ("fp8_gate_up_swapped", "silu(z[f]) * z[f + F]", "silu(z[f + F]) * z[f]"),
     ("fp8_token_path_drops_gate", "o[n] += y[n] * w[j];", "o[n] += y[n];"),
+    ("bwd_silu_derivative_drops_term", "const double dg = da[f] * u * s * (1.0 + g * (1.0 - s));",
+     "const double dg = da[f] * u * s;"),
+    ("bwd_up_gradient_uses_up", "const double du = da[f] * g * s;", "const double du = da[f] * u * s;"),
+    ("bwd_softmax_not_centred", "const double dl = (dw[j] - wdw) * w[j];", "const double dl = dw[j] * w[j];"),
+    ("bwd_dbias_with_selection_bias", "if (gate != ORACLE_GATE_SELECT_BIAS) dbias[e] += dl;",
+     "dbias[e] += dl;"),
+    ("bwd_dW2_without_gate", "drow[n] += a[f] * gscale * (double)bf16_to_float(dyr[n]);",
+     "drow[n] += a[f] * (double)bf16_to_float(dyr[n]);"),
+    ("bwd_dx_tokens_not_centred", "const double dl = w[j] * (dw[j] - wdw);", "const double dl = w[j] * dw[j];"),
     ("shared_ffn_uses_gate_half_only", "ffn_row(H, Fs, ORACLE_ACT_SWIGLU, 0, xr, W1s, W2s, y, scratch);",
      "ffn_row(H, Fs, ORACLE_ACT_GELU_TANH, 0, xr, W1s, W2s, y, scratch);"),
 ]

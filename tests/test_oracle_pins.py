@@ -525,3 +525,83 @@ def test_fp8_layer_scales_exactly_with_the_input(oracle_lib, act):
     out8, _, _ = oracle.moe_tokens_fp8(x8, Wg, None, W1q, s1, W2q, s2, k, toks, act=act, lib=oracle_lib)
     np.testing.assert_array_equal(out8, 8.0 * out)
     assert np.abs(out).max() > 0
+
+
+# ---------------------------------------------------------------------------------------
+# Backward pass (training; beyond the pages)
+# ---------------------------------------------------------------------------------------
+
+def _autograd_grads(x, Wg, bias, W1, W2, dy, k, act, gate, idx):
+    """Gradients of sum(dy * out) by torch autograd (float64) of the layer written with the
+    selection fixed to idx: a derivative the oracle's hand-written backward does not share."""
+    t = lambda a: torch.from_numpy(widen(a)).requires_grad_(True)
+    X, G, A, B = t(x), t(Wg), t(W1), t(W2)
+    b = torch.from_numpy(np.asarray(bias, np.float64)).requires_grad_(True) if bias is not None else None
+    logits = X @ G
+    if b is not None and gate != oracle.GATE_SELECT_BIAS:
+        logits = logits + b
+    sel = torch.from_numpy(idx.astype(np.int64))
+    w = torch.softmax(torch.gather(logits, 1, sel), dim=1)
+    F = W2.shape[1]
+    out = torch.zeros_like(X)
+    for j in range(k):
+        for e in range(W1.shape[0]):
+            rows = (sel[:, j] == e).nonzero().flatten()
+            if rows.numel() == 0:
+                continue
+            z = X[rows] @ A[e]
+            if act == oracle.ACT_SWIGLU:
+                a = torch.nn.functional.silu(z[:, :F]) * z[:, F:]
+            elif act == oracle.ACT_RELU:
+                a = torch.relu(z)
+            elif act == oracle.ACT_GELU_TANH:
+                a = torch.nn.functional.gelu(z, approximate="tanh")
+            else:
+                a = z
+            out = out.index_add(0, rows, w[rows, j:j + 1] * (a @ B[e]))
+    loss = (out * torch.from_numpy(widen(dy))).sum()
+    params = [X, G, A, B] + ([b] if b is not None else [])
+    grads = torch.autograd.grad(loss, params, allow_unused=True)
+    names = ["dx", "dWg", "dW1", "dW2"] + (["dbias"] if b is not None else [])
+    return {n: (g.numpy() if g is not None else np.zeros(p.shape)) for n, g, p in zip(names, grads, params)}
+
+
+@pytest.mark.parametrize("act,gate,use_bias", [
+    (oracle.ACT_SWIGLU, oracle.GATE_SOFTMAX_TOPK, True),
+    (oracle.ACT_SWIGLU, oracle.GATE_SELECT_BIAS, True),
+    (oracle.ACT_GELU_TANH, oracle.GATE_SOFTMAX_TOPK, False),
+    (oracle.ACT_RELU, oracle.GATE_SOFTMAX_TOPK, True),
+], ids=["swiglu_bias", "swiglu_select_bias", "gelu", "relu_bias"])
+def test_backward_matches_autograd(oracle_lib, act, gate, use_bias):
+    T, H, F, E, k = 20, 32, 24, 6, 2
+    w1c = 2 * F if act == oracle.ACT_SWIGLU else F
+    x = rand_bf16((T, H), 31)
+    Wg = rand_bf16((H, E), 32, 0.5)
+    W1 = rand_bf16((E, H, w1c), 33, 1 / math.sqrt(H))
+    W2 = rand_bf16((E, F, H), 34, 1 / math.sqrt(F))
+    dy = rand_bf16((T, H), 35)
+    bias = np.random.default_rng(36).normal(0, 0.5, E).astype(np.float32) if use_bias else None
+    g = oracle.moe_backward(x, Wg, bias, W1, W2, dy, k, act=act, gate=gate, lib=oracle_lib)
+    logits = oracle.router_logits(x, Wg, None if gate == oracle.GATE_SELECT_BIAS else bias,
+                                  lib=oracle_lib)
+    idx, _ = oracle.topk_gates(logits, k, gate=gate, bias=bias, lib=oracle_lib)
+    ref = _autograd_grads(x, Wg, bias, W1, W2, dy, k, act, gate, idx)
+    # the oracle's gates come from fp32 logits, autograd's from fp64 ones: ~1e-7 relative
+    for name in ref:
+        np.testing.assert_allclose(g[name], ref[name], rtol=1e-5, atol=1e-6, err_msg=name)
+    if use_bias and gate == oracle.GATE_SELECT_BIAS:
+        assert np.all(g["dbias"] == 0)
+    assert np.abs(g["dW1"]).max() > 0 and np.abs(g["dWg"]).max() > 0
+
+
+def test_backward_dx_tokens_equals_full_backward(oracle_lib):
+    T, H, F, E, k = 16, 32, 16, 4, 2
+    x = rand_bf16((T, H), 41)
+    Wg = rand_bf16((H, E), 42)
+    W1 = rand_bf16((E, H, 2 * F), 43, 1 / math.sqrt(H))
+    W2 = rand_bf16((E, F, H), 44, 1 / math.sqrt(F))
+    dy = rand_bf16((T, H), 45)
+    full = oracle.moe_backward(x, Wg, None, W1, W2, dy, k, lib=oracle_lib)
+    toks = np.array([3, 0, 15, 7])
+    part = oracle.moe_backward_dx_tokens(x, Wg, None, W1, W2, dy, k, toks, lib=oracle_lib)
+    np.testing.assert_array_equal(part, full["dx"][toks])
