@@ -275,6 +275,28 @@ MOE_API moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *
                                           size_t ws_bytes, void *stream, void *const *events,
                                           int32_t n_events);
 
+/* Backward pass (training; beyond the pages, which describe the forward).
+ * Given dout = dL/dout [T, H] bf16, the gradients of the layer moe_forward computes, with the
+ * selection held fixed (it is piecewise constant) and the gates the softmax over the
+ * selected logits:
+ *   dx [T, H] bf16, dWg [H, E] fp32, dbias [E] fp32 (zero with MOE_GATE_SELECT_BIAS, or
+ *   without a bias), dW1 [E, H, w1_cols] bf16, dW2 [E, F, H] bf16.
+ * Per routed row (token t, selection j, expert e): dw_j = dout_t . y_e(x_t),
+ * dl_j = w_j (dw_j - sum_i w_i dw_i), gy = w_j dout_t, dW2[e] += a^T gy, da = gy W2[e]^T,
+ * dz = da * act'(z) (SwiGLU: [da up silu'(g), da silu(g)]), dW1[e] += x_t^T dz,
+ * dx_t += dz W1[e]^T + dl_j W_g[:, e], dW_g[:, e] += x_t dl_j, dbias[e] += dl_j.
+ * The call recomputes the routing, the dispatch and z = x W1 (it needs no state from a
+ * forward call). bf16 intermediates with fp32 accumulation; sums over tokens in the
+ * experts' row order. Needs H % 128 == 0, F % 128 == 0 and a gate mode other than
+ * MOE_GATE_SOFTMAX_ALL (MOE_ERR_UNSUPPORTED otherwise). Device pointers, 16-byte aligned
+ * (4-byte for the fp32 ones). */
+MOE_API size_t moe_backward_workspace_size(const moe_problem *p);
+MOE_API moe_status moe_backward(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                                const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                                const moe_bf16 *dout, moe_bf16 *dx, float *dWg, float *dbias,
+                                moe_bf16 *dW1, moe_bf16 *dW2, void *ws, size_t ws_bytes,
+                                void *stream);
+
 /* Combine (§2.1: gather and reduce the top-k outputs).
  *   out[t][n] = bf16_rne( sum_{j=0..k-1} ys[inv_pos[t][j]][n] ), fp32 sum, j ascending.
  * ys [ys_rows, H] bf16 holds expert-sorted rows that already carry their gate weight;

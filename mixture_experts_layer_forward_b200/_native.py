@@ -100,6 +100,8 @@ def library() -> ctypes.CDLL:
             "moe_forward_fp8": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_forward_fp8_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                         ctypes.POINTER(vp), i32], i32),
+            "moe_backward_workspace_size": ([P], sz),
+            "moe_backward": ([P] + [vp] * 12 + [sz, vp], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
             "moe_get_device_status": ([vp, vp], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
@@ -352,6 +354,23 @@ def moe_forward_fp8_staged(p, x, Wg, bias, W1q, s1, W2q, s2, out, ws, events, to
                                                      topk_idx_out, topk_w_out), w, n,
                                           _stream(stream), arr, MOE_NUM_STAGE_EVENTS)
     _check("moe_forward_fp8_staged", rc)
+
+
+def moe_backward_workspace_size(p: Problem) -> int:
+    """Workspace bytes for moe_backward (0: invalid or unsupported shape / gate mode)."""
+    return int(library().moe_backward_workspace_size(ctypes.byref(p)))
+
+
+def moe_backward(p, x, Wg, bias, W1, W2, dout, dx, dWg, dbias, dW1, dW2, ws, stream=None):
+    """Gradients of the layer: dx, dW1, dW2 bf16; dWg [H, E], dbias [E] float32."""
+    bf, f32 = torch.bfloat16, torch.float32
+    w, n = _ws(ws)
+    rc = library().moe_backward(ctypes.byref(p), _ptr(x, bf, "x"), _ptr(Wg, bf, "Wg"),
+                                _ptr(bias, f32, "bias"), _ptr(W1, bf, "W1"), _ptr(W2, bf, "W2"),
+                                _ptr(dout, bf, "dout"), _ptr(dx, bf, "dx"), _ptr(dWg, f32, "dWg"),
+                                _ptr(dbias, f32, "dbias"), _ptr(dW1, bf, "dW1"),
+                                _ptr(dW2, bf, "dW2"), w, n, _stream(stream))
+    _check("moe_backward", rc)
 
 
 def moe_combine(p, ys, inv_pos, out, ws=None, stream=None):

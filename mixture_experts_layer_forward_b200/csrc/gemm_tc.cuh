@@ -73,6 +73,14 @@ constexpr uint32_t B_LBO = B_BOX; // next 64-column block
 } // namespace gemm
 
 enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2, GEMM_LOGITS = 3 };
+// Operand layouts of grouped_gemm_cta:
+//   BMODE_FWD     B = the expert's weight matrix as stored [K, N] (MN-major; e4m3 codes are
+//                 stored K-major instead, see F8);
+//   BMODE_KMAJOR  B = the expert's matrix [N rows, K] read K-major (backward: dy . W2^T and
+//                 dz . W1^T, where the forward's weight is the transposed operand);
+//   BMODE_WGRAD   weight gradients: D[e] = A_e^T B_e over the expert's padded rows r (K),
+//                 A [rows, M] and B [rows, N] both read MN-major.
+enum GemmBMode { BMODE_FWD = 0, BMODE_KMAJOR = 1, BMODE_WGRAD = 2 };
 enum GemmOrder { ORDER_EXPERT = 0, ORDER_MIXED = 1 };
 
 struct GemmArgs {
@@ -125,6 +133,11 @@ struct GemmArgs {
     const float *a_scale;
     const float *b_scale;
     int b_scale_ld;
+    // BMODE_WGRAD: wg_experts experts, each an output of wg_mtiles 128-row tiles (M =
+    // 128 * wg_mtiles) by n_tiles 256-column tiles; expert e's K is its padded rows
+    // [128 tile_off[e], 128 tile_off[e + 1]); out[(e * M + m) * ld_out + n]
+    int wg_experts;
+    int wg_mtiles;
 };
 
 __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
@@ -313,7 +326,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
-template <int KIND, bool F8 = false>
+// BMODE_WGRAD work item w: expert-major, then N tile, then M tile; its k-blocks of 64 rows
+__device__ __forceinline__ void wgrad_item(int w, const GemmArgs &a, int &e, int &mt, int &nt,
+                                           int &kb0, int &kb1)
+{
+    const int per = a.wg_mtiles * a.n_tiles;
+    e = w / per;
+    const int r = w - e * per;
+    mt = r % a.wg_mtiles;
+    nt = r / a.wg_mtiles;
+    kb0 = a.tile_off[e] * (gemm::BM / gemm::BK);
+    kb1 = a.tile_off[e + 1] * (gemm::BM / gemm::BK);
+}
+
+template <int KIND, bool F8 = false, int BMODE = BMODE_FWD>
 __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                                  const GemmArgs &args, uint8_t *smem, int w_first,
                                                  int w_step)
@@ -361,15 +387,31 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_tiles = args.dense_m_tiles > 0 ? args.dense_m_tiles : args.meta->num_tiles;
+    const bool wgrad = (BMODE == BMODE_WGRAD);
+    const int num_tiles = wgrad ? 0 : (args.dense_m_tiles > 0 ? args.dense_m_tiles : args.meta->num_tiles);
     const int n_split = (args.dense_m_tiles > 0 && args.k_split > 1) ? args.k_split : 1;
-    const int total = num_tiles * args.n_tiles * n_split;
+    const int total = wgrad ? args.wg_experts * args.wg_mtiles * args.n_tiles
+                            : num_tiles * args.n_tiles * n_split;
     const int KB = args.k_blocks;
     // k-blocks [kb_lo(ks), kb_lo(ks + 1)) belong to split ks (n_split <= KB: none is empty)
     auto kb_lo = [&](int ks) { return (int)(((int64_t)ks * KB) / n_split); };
+    // k-block range of work item w (per expert for BMODE_WGRAD, possibly empty)
+    auto kb_range = [&](int w, int &e, int &mt, int &nt, int &kb0, int &kb1) {
+        if (wgrad) {
+            wgrad_item(w, args, e, mt, nt, kb0, kb1);
+        } else {
+            int ks;
+            gemm_map_work(w, args, e, mt, nt, ks);
+            kb0 = kb_lo(ks);
+            kb1 = kb_lo(ks + 1);
+        }
+    };
     // B boxes of 64 columns per k-block; the router filter narrows N to what E needs
     const int nbox = (KIND == GEMM_LOGITS && args.n_boxes >= 1 && args.n_boxes < 4) ? args.n_boxes : 4;
-    const uint32_t idesc = (nbox == 4) ? IDESC : idesc_bf16_f32(BM, nbox * 64, /*b_mn_major=*/true);
+    const uint32_t idesc = BMODE == BMODE_KMAJOR ? idesc_bf16_f32(BM, BN, /*b_mn_major=*/false)
+                           : BMODE == BMODE_WGRAD ? (IDESC | (1u << 15)) // A MN-major too
+                           : (nbox == 4) ? IDESC
+                                         : idesc_bf16_f32(BM, nbox * 64, /*b_mn_major=*/true);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -381,9 +423,9 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             for (int i = 0; i < STAGES; ++i) armed[i] = -1;
             bool ok = true;
             for (int w = w_first; ok && w < total; w += w_step) {
-                int e, mt, nt, ks;
-                gemm_map_work(w, args, e, mt, nt, ks);
-                for (int kb = kb_lo(ks); kb < kb_lo(ks + 1); ++kb) {
+                int e, mt, nt, kb0, kb1;
+                kb_range(w, e, mt, nt, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, args.timeout_ns,
                                            args.status, 100 + KIND)) {
                         ok = false;
@@ -391,24 +433,37 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                     }
                     const uint32_t a_dst = smem_u32(smem + s * STAGE);
                     const uint32_t b_dst = a_dst + A_TILE;
-                    mbar_arrive_expect_tx(full_bar(s),
-                                          (gather ? 0 : A_TILE) + (F8 ? B_TILE : nbox * B_BOX));
+                    mbar_arrive_expect_tx(full_bar(s), (gather ? 0 : A_TILE) +
+                                                           ((F8 || BMODE != BMODE_FWD) ? B_TILE : nbox * B_BOX));
                     armed[s] = (int)ph;
+                    if (BMODE == BMODE_WGRAD) {
+                        // A [rows, M] MN-major: two boxes of 64 M columns x 64 rows; B [rows, N]
+                        // (a depth-1 3D map) MN-major: four boxes of 64 N columns x 64 rows
+                        tma_load_2d(a_dst, &tmA, full_bar(s), mt * BM, kb * BK);
+                        tma_load_2d(a_dst + B_BOX, &tmA, full_bar(s), mt * BM + 64, kb * BK);
+                        for (int i = 0; i < 4; ++i)
+                            tma_load_3d(b_dst + i * B_BOX, &tmB, full_bar(s), nt * BN + i * 64, kb * BK, 0);
+                    } else {
                     // the x coordinate is the K offset in elements: 128 B per k-block either way
                     if (!gather) tma_load_2d(a_dst, &tmA, full_bar(s), kb * (F8 ? 128 : BK), mt * BM);
+                    if (BMODE == BMODE_KMAJOR) { // bf16 [E, N rows, K]: two boxes of 128 rows
+                        tma_load_3d(b_dst, &tmB, full_bar(s), kb * BK, nt * BN, e);
+                        tma_load_3d(b_dst + 128 * 128, &tmB, full_bar(s), kb * BK, nt * BN + 128, e);
+                    }
                     if (F8) { // K-major e4m3 weights [E, N rows, K]: two boxes of 128 rows
                         const int r0 = (KIND == GEMM_SWIGLU) ? nt * 128 : nt * BN;
                         const int r1 = (KIND == GEMM_SWIGLU) ? args.up_col + nt * 128 : nt * BN + B8_BOX_ROWS;
                         tma_load_3d(b_dst, &tmB, full_bar(s), kb * 128, r0, e);
                         tma_load_3d(b_dst + B8_BOX_ROWS * 128, &tmB, full_bar(s), kb * 128, r1, e);
                     }
-                    for (int i = 0; i < (F8 ? 0 : nbox); ++i) {
+                    for (int i = 0; i < ((F8 || BMODE != BMODE_FWD) ? 0 : nbox); ++i) {
                         int col;
                         if (KIND == GEMM_SWIGLU)
                             col = (i < 2 ? nt * 128 + i * 64 : args.up_col + nt * 128 + (i - 2) * 64);
                         else
                             col = nt * BN + i * 64;
                         tma_load_3d(b_dst + i * B_BOX, &tmB, full_bar(s), col, kb * BK, e);
+                    }
                     }
                     if (++s == STAGES) {
                         s = 0;
@@ -442,13 +497,12 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                int ks = 0;
-                if (n_split > 1) {
+                int kb_first = 0, kb_end = KB;
+                if (n_split > 1 || wgrad) {
                     int e_, mt_, nt_;
-                    gemm_map_work(w, args, e_, mt_, nt_, ks);
+                    kb_range(w, e_, mt_, nt_, kb_first, kb_end);
                 }
-                const int kb_first = kb_lo(ks);
-                for (int kb = kb_first; kb < kb_lo(ks + 1); ++kb) {
+                for (int kb = kb_first; kb < kb_end; ++kb) {
                     if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, args.timeout_ns, args.status,
                                            120 + KIND)) {
                         ok = false;
@@ -469,12 +523,25 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                             umma_f8(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
                                     b_desc + (uint64_t)((k * 32) >> 4), IDESC_F8,
                                     (kb != kb_first || k != 0) ? 1u : 0u);
+                    } else if (BMODE == BMODE_KMAJOR) {
+                        // both K-major: +32 B per K=16 step
+                        const uint64_t b_desc = sw128_desc(b_addr, A_LBO, A_SBO);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                      b_desc + (uint64_t)((k * 32) >> 4), idesc,
+                                      (kb != kb_first || k != 0) ? 1u : 0u);
                     } else {
+                        // MN-major A (BMODE_WGRAD: next 64-column block one box further) and
+                        // B: +16 K rows x 128 B per K=16 step
+                        const uint64_t a_mn = sw128_desc(a_addr, B_LBO, B_SBO);
                         const uint64_t b_desc = sw128_desc(b_addr, B_LBO, B_SBO);
 #pragma unroll
                         for (int k = 0; k < BK / 16; ++k) {
                             // A: +32 B per K=16 step inside the swizzle atom; B: +16 rows x 128 B
-                            umma_bf16(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                            umma_bf16(d_tmem,
+                                      wgrad ? a_mn + (uint64_t)((k * 16 * 128) >> 4)
+                                            : a_desc + (uint64_t)((k * 32) >> 4),
                                       b_desc + (uint64_t)((k * 16 * 128) >> 4), idesc,
                                       (kb != kb_first || k != 0) ? 1u : 0u);
                         }
@@ -552,8 +619,11 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
         int rs = 0;             // stage ring position (row_sq only)
         uint32_t rph = 0;
         for (int w = w_first; w < total; w += w_step, ++it) {
-            int e, mt, nt, ks;
-            gemm_map_work(w, args, e, mt, nt, ks);
+            int e, mt, nt, ks = 0, kb0 = 0, kb1 = 1;
+            if (wgrad)
+                wgrad_item(w, args, e, mt, nt, kb0, kb1);
+            else
+                gemm_map_work(w, args, e, mt, nt, ks);
             if (row_sq) {
                 // sum of squares of this thread's A row over the item's k-blocks (the order of
                 // the 16-byte pieces does not matter; lane-rotated reads avoid bank conflicts)
@@ -596,9 +666,16 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             // the TMEM loads below are warp-collective: the whole warp continues or stops
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int row = mt * BM + q * 32 + lane;
+            const int row = wgrad ? (e * args.wg_mtiles + mt) * BM + q * 32 + lane
+                                  : mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e);
+            if (wgrad && kb1 == kb0) { // an expert without rows: a zero gradient
+                uint4 *orow = reinterpret_cast<uint4 *>(args.out + (size_t)row * args.ld_out + nt * BN);
+                for (int c = 0; c < BN / 8; ++c)
+                    if (nt * BN + c * 8 < args.n_cols) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
@@ -626,6 +703,18 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
 }
 
 
+// The backward GEMMs (identity epilogue, bf16 out): BMODE_KMAJOR for the data gradients
+// through the transposed weights, BMODE_WGRAD for the weight gradients.
+template <int BMODE>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA,
+                                const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    grouped_gemm_cta<GEMM_ACT, false, BMODE>(tmA, tmB, args, smem, blockIdx.x, gridDim.x);
+}
 
 // ---------------------------------------------------------------------------------------
 // CTA-pair variant: tcgen05.mma.cta_group::2, M = 256 (128 rows per CTA), N = 256.

@@ -9,6 +9,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "backward.cuh"
 #include "combine.cuh"
 #include "dispatch.cuh"
 #include "fp8.cuh"
@@ -70,8 +71,9 @@ struct Layout {
         counts, offsets, poff, tile_off,
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
-        x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys, xq, sx, hq, sh;
-    size_t end_route, end_dispatch, end_forward, end_host, end_shared, end_fp8;
+        x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys, xq, sx, hq, sh,
+        bgu, ba, bdxp, bdw, bdl;
+    size_t end_route, end_dispatch, end_forward, end_host, end_shared, end_fp8, end_bwd;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
 };
@@ -128,7 +130,7 @@ FilterPlan filter_plan(const moe_problem *p)
     return f;
 }
 
-Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false)
+Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd = false)
 {
     Layout L{};
     const size_t T = (size_t)p->T, H = (size_t)p->H, F = (size_t)p->F, E = (size_t)p->E,
@@ -192,6 +194,15 @@ Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false)
     L.hq = take(fp8 ? P * F : 0);
     L.sh = take(fp8 ? P * 4 : 0);
     L.end_fp8 = o;
+    // backward (moe_backward): recomputed pre-activations, overwritten by their gradient;
+    // hidden activations; the expert rows' input gradients; per-row gate and logit gradients
+    const size_t w1c = p->act == MOE_ACT_SWIGLU ? 2 * F : F;
+    L.bgu = take(bwd ? P * w1c * 2 : 0);
+    L.ba = take(bwd ? P * F * 2 : 0);
+    L.bdxp = take(bwd ? P * H * 2 : 0);
+    L.bdw = take(bwd ? P * 4 : 0);
+    L.bdl = take(bwd ? P * 4 : 0);
+    L.end_bwd = o;
     return L;
 }
 
@@ -258,14 +269,15 @@ bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D bf16 [depth, rows, cols]; box = 64 columns x 64 rows x 1, 128-byte swizzle.
-bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols)
+// 3D bf16 [depth, rows, cols]; box = 64 columns x box_rows rows x 1, 128-byte swizzle.
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows = 64)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[3] = {cols, rows, depth};
     cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -335,7 +347,8 @@ template <int KIND>
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
                         int max_work, cudaStream_t st);
 bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
-bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols);
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows);
 
 FilterBufs filter_bufs(void *ws, const Layout &L)
 {
@@ -910,6 +923,184 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     return to_status(e);
 }
 
+template <int BMODE>
+cudaError_t launch_gemm_bwd(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                            int max_work, cudaStream_t st)
+{
+    auto kern = moe_grouped_gemm_bwd_kernel<BMODE>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    int grid = sm_count();
+    if (grid <= 0) grid = 148;
+    if (grid > max_work) grid = max_work;
+    if (grid < 1) grid = 1;
+    const int threads = args.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    kern<<<grid, threads, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+    return cudaGetLastError();
+}
+
+// Shapes the backward supports: the weight-gradient GEMMs' M (F and H) in whole 128-row
+// tiles; the gates a softmax over the selected logits.
+moe_status check_problem_bwd(const moe_problem *p)
+{
+    const moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (p->H % 128 != 0 || p->F % 128 != 0 || p->gate == MOE_GATE_SOFTMAX_ALL)
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// The layer's gradients (see backward.cuh): route and dispatch as the forward; x rows
+// gathered (x_perm); z = x W1 recomputed (identity epilogue); u = dy W2^T (dy rows gathered,
+// W2 read K-major); the row pass (a, dz in place of z, gy, dw); logit gradients; dW2 = a^T gy
+// and dW1 = x_perm^T dz per expert; dx_perm = dz W1^T (W1 read K-major); dx; dW_g and dbias.
+moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                         const moe_bf16 *dy, moe_bf16 *dx, float *dWg, float *dbias, moe_bf16 *dW1,
+                         moe_bf16 *dW2, void *ws, size_t ws_bytes, cudaStream_t st)
+{
+    moe_status s = check_problem_bwd(p);
+    if (s != MOE_OK) return s;
+    if (ws == nullptr || Wg == nullptr || W1 == nullptr || W2 == nullptr || dWg == nullptr ||
+        dbias == nullptr || dW1 == nullptr || dW2 == nullptr ||
+        (p->T > 0 && (x == nullptr || dy == nullptr || dx == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, 0, false, true);
+    if (ws_bytes < L.end_bwd) return MOE_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(Wg) || !aligned16(W1) || !aligned16(W2) || !aligned16(dy) ||
+        !aligned16(dx) || !aligned16(dW1) || !aligned16(dW2) || !aligned4(dWg) || !aligned4(dbias) ||
+        !aligned4(bias) || !aligned16(ws))
+        return MOE_ERR_INVALID_ARG;
+    const int T = p->T, H = p->H, F = p->F, E = p->E, k = p->top_k;
+    const bool gated = (p->act == MOE_ACT_SWIGLU);
+    const int w1c = gated ? 2 * F : F;
+    int *status = at<int>(ws, L.status);
+    if (T == 0) { // no rows: every gradient is zero
+        cudaError_t e = cudaMemsetAsync(status, 0, 8, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dWg, 0, (size_t)H * E * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dbias, 0, (size_t)E * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dW1, 0, (size_t)E * H * w1c * 2, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dW2, 0, (size_t)E * F * H * 2, st);
+        return to_status(e);
+    }
+    int32_t *topk_idx = at<int32_t>(ws, L.topk_idx);
+    float *topk_w = at<float>(ws, L.topk_w);
+    const DispatchOut d = dispatch_bufs(ws, L);
+    moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
+    moe_bf16 *u = at<moe_bf16>(ws, L.h);   // [P, F]
+    moe_bf16 *gy = at<moe_bf16>(ws, L.ys); // [P, H]
+    moe_bf16 *gu = at<moe_bf16>(ws, L.bgu), *a = at<moe_bf16>(ws, L.ba);
+    moe_bf16 *dxp = at<moe_bf16>(ws, L.bdxp);
+    float *dw_row = at<float>(ws, L.bdw), *dl_row = at<float>(ws, L.bdl);
+
+    CUtensorMap m_x, m_w1, m_w2k, m_gu, m_a, m_gy, m_xp, m_dz, m_w1k;
+    if (!make_map_2d(&m_x, x, (uint64_t)T, (uint64_t)H, 1) || // unused: rows are gathered
+        !make_map_3d(&m_w1, W1, (uint64_t)E, (uint64_t)H, (uint64_t)w1c) ||
+        !make_map_3d(&m_w2k, W2, (uint64_t)E, (uint64_t)F, (uint64_t)H, 128) ||
+        !make_map_2d(&m_a, a, (uint64_t)L.pmax, (uint64_t)F, 64) ||
+        !make_map_3d(&m_gy, gy, 1, (uint64_t)L.pmax, (uint64_t)H) ||
+        !make_map_2d(&m_xp, x_perm, (uint64_t)L.pmax, (uint64_t)H, 64) ||
+        !make_map_3d(&m_dz, gu, 1, (uint64_t)L.pmax, (uint64_t)w1c) ||
+        !make_map_2d(&m_gu, gu, (uint64_t)L.pmax, (uint64_t)w1c, gemm::BM) ||
+        !make_map_3d(&m_w1k, W1, (uint64_t)E, (uint64_t)H, (uint64_t)w1c, 128))
+        return MOE_ERR_CUDA;
+    const int64_t timeout = g_timeout_ns.load();
+    const FilterBufs fb = filter_bufs(ws, L);
+    cudaError_t e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status,
+                                 st, &fb);
+    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
+    if (e == cudaSuccess) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
+
+    GemmArgs g{};
+    g.tile_off = d.tile_off;
+    g.tile_expert = d.tile_expert;
+    g.meta = d.meta;
+    g.order = ORDER_EXPERT;
+    g.act = MOE_ACT_IDENTITY;
+    g.status = status;
+    g.timeout_ns = timeout;
+    g.gather_len = L.pmax;
+    g.gather_rows = T;
+    g.gather_ld = H;
+    // z = x W1 (recomputed pre-activations), x rows gathered
+    GemmArgs gz = g;
+    gz.gather_idx = d.gather_idx;
+    gz.gather_src = reinterpret_cast<const __nv_bfloat16 *>(x);
+    gz.out = reinterpret_cast<__nv_bfloat16 *>(gu);
+    gz.ld_out = gz.n_cols = w1c;
+    gz.n_tiles = (w1c + gemm::BN - 1) / gemm::BN;
+    gz.k_blocks = H / gemm::BK;
+    if (e == cudaSuccess) e = launch_gemm<GEMM_ACT>(m_x, m_w1, gz, L.max_tiles * gz.n_tiles, st);
+    // u = dy W2^T, dy rows gathered
+    GemmArgs gu_ = g;
+    gu_.gather_idx = d.gather_idx;
+    gu_.gather_src = reinterpret_cast<const __nv_bfloat16 *>(dy);
+    gu_.out = reinterpret_cast<__nv_bfloat16 *>(u);
+    gu_.ld_out = gu_.n_cols = F;
+    gu_.n_tiles = (F + gemm::BN - 1) / gemm::BN;
+    gu_.k_blocks = H / gemm::BK;
+    if (e == cudaSuccess)
+        e = launch_gemm_bwd<BMODE_KMAJOR>(m_x, m_w2k, gu_, L.max_tiles * gu_.n_tiles, st);
+    // row pass: a, dz (in place of z), gy, dw
+    if (e == cudaSuccess) {
+        int grid = sm_count() * 8;
+        if (grid <= 0) grid = 1184;
+        bwd_rows_kernel<<<grid, BWD_THREADS, 0, st>>>(
+            reinterpret_cast<__nv_bfloat16 *>(gu), reinterpret_cast<const __nv_bfloat16 *>(u),
+            reinterpret_cast<const __nv_bfloat16 *>(dy), d.gather_idx, d.row_w, d.meta, M_TILE, F, H,
+            T, p->act, reinterpret_cast<__nv_bfloat16 *>(a), reinterpret_cast<__nv_bfloat16 *>(gy),
+            dw_row);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        bwd_router_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(topk_w, d.inv_pos, dw_row, T, k, dl_row);
+        e = cudaGetLastError();
+    }
+    // weight gradients: dW2[e] = a_e^T gy_e, dW1[e] = x_perm_e^T dz_e
+    GemmArgs w2 = g;
+    w2.wg_experts = E;
+    w2.wg_mtiles = F / gemm::BM;
+    w2.out = reinterpret_cast<__nv_bfloat16 *>(dW2);
+    w2.ld_out = w2.n_cols = H;
+    w2.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+    if (e == cudaSuccess)
+        e = launch_gemm_bwd<BMODE_WGRAD>(m_a, m_gy, w2, E * w2.wg_mtiles * w2.n_tiles, st);
+    GemmArgs w1 = g;
+    w1.wg_experts = E;
+    w1.wg_mtiles = H / gemm::BM;
+    w1.out = reinterpret_cast<__nv_bfloat16 *>(dW1);
+    w1.ld_out = w1.n_cols = w1c;
+    w1.n_tiles = (w1c + gemm::BN - 1) / gemm::BN;
+    if (e == cudaSuccess)
+        e = launch_gemm_bwd<BMODE_WGRAD>(m_xp, m_dz, w1, E * w1.wg_mtiles * w1.n_tiles, st);
+    // dx_perm = dz W1^T (dz rows by TMA, W1 read K-major)
+    GemmArgs gx = g;
+    gx.out = reinterpret_cast<__nv_bfloat16 *>(dxp);
+    gx.ld_out = gx.n_cols = H;
+    gx.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+    gx.k_blocks = w1c / gemm::BK;
+    if (e == cudaSuccess)
+        e = launch_gemm_bwd<BMODE_KMAJOR>(m_gu, m_w1k, gx, L.max_tiles * gx.n_tiles, st);
+    if (e == cudaSuccess) {
+        int grid = sm_count() * 8;
+        if (grid <= 0) grid = 1184;
+        if (grid > T) grid = T;
+        bwd_dx_kernel<<<grid, BWD_THREADS, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(dxp),
+                                                     d.inv_pos, topk_idx, dl_row,
+                                                     reinterpret_cast<const __nv_bfloat16 *>(Wg), T,
+                                                     H, E, k, reinterpret_cast<__nv_bfloat16 *>(dx));
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        bwd_router_weights_kernel<<<dim3(E, (H + BWD_THREADS - 1) / BWD_THREADS), BWD_THREADS, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(x), d.gather_idx, d.poff, d.counts, dl_row, H, E,
+            (bias != nullptr && p->gate != MOE_GATE_SELECT_BIAS) ? 1 : 0, dWg, dbias);
+        e = cudaGetLastError();
+    }
+    return to_status(e);
+}
+
 // Shapes the FP8 expert path supports: both GEMMs' K (H and F) in whole 128-value k-blocks.
 moe_status check_problem_fp8(const moe_problem *p)
 {
@@ -1431,6 +1622,21 @@ moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *x, const
 {
     return forward_impl_fp8(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out, topk_w_out, ws,
                             ws_bytes, static_cast<cudaStream_t>(stream), events, n_events);
+}
+
+size_t moe_backward_workspace_size(const moe_problem *p)
+{
+    if (check_problem_bwd(p) != MOE_OK) return 0;
+    return make_layout(p, 0, false, true).end_bwd;
+}
+
+moe_status moe_backward(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
+                        const float *bias, const moe_bf16 *W1, const moe_bf16 *W2,
+                        const moe_bf16 *dout, moe_bf16 *dx, float *dWg, float *dbias,
+                        moe_bf16 *dW1, moe_bf16 *dW2, void *ws, size_t ws_bytes, void *stream)
+{
+    return backward_impl(p, x, Wg, bias, W1, W2, dout, dx, dWg, dbias, dW1, dW2, ws, ws_bytes,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int moe_set_fault_injection(int layer0_item)

@@ -169,3 +169,10 @@ def test_fp8_workspace_and_argument_checks(lib):
                                         None) == -1
     assert lib.moe_forward_fp8(ctypes.byref(p), None, None, None, None, None, None, None, None,
                                None, None, None, 0, None) == -1
+
+
+def test_backward_workspace_and_argument_checks(lib):
+    p = moe.Problem.make(300, 256, 256, 16, 2)
+    assert moe.moe_backward_workspace_size(p) > moe.moe_workspace_size(p)
+    assert moe.moe_backward_workspace_size(moe.Problem.make(300, 256, 192, 16, 2)) == 0   # F % 128
+    assert lib.moe_backward(ctypes.byref(p), *([None] * 12), 0, None) == -1
