@@ -64,6 +64,8 @@ def parse_args():
                     help="target CPU seconds of the oracle sample")
     ap.add_argument("--fp8", action="store_true",
                     help="e4m3 experts (moe_forward_fp8; weights quantised once before timing)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time moe_backward (the layer's gradients) instead of the forward")
     ap.add_argument("--router-only", action="store_true",
                     help="time moe_route alone (router logits + top-k); no expert weights allocated")
     return ap.parse_args()
@@ -511,12 +513,79 @@ def run_router(args):
     return 0
 
 
+def run_backward(args):
+    """The layer's backward on one GPU: K timed moe_backward calls (each recomputes the
+    routing, the dispatch and z = x W1) on a seeded dL/dout."""
+    import torch
+
+    import mixture_experts_layer_forward_b200 as moe
+    from mixture_experts_layer_forward_b200 import synth
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = workload(args)
+    K, W = args.steps, max(3, args.warmup)
+    inp = synth.make_inputs(cfg, seed=args.seed, device=dev)
+    p = moe.Problem.from_config(cfg)
+    g = torch.Generator(device=dev).manual_seed(args.seed + 1)
+    dy = torch.randn(cfg.T, cfg.H, generator=g, device=dev).to(torch.bfloat16)
+    w1c = 2 * cfg.F if cfg.act == 0 else cfg.F
+    dx = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    dWg = torch.empty(cfg.H, cfg.E, dtype=torch.float32, device=dev)
+    dbias = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    dW1 = torch.empty(cfg.E, cfg.H, w1c, dtype=torch.bfloat16, device=dev)
+    dW2 = torch.empty(cfg.E, cfg.F, cfg.H, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(moe.moe_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+    call = lambda: moe.moe_backward(p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], dy,
+                                    dx, dWg, dbias, dW1, dW2, ws)
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize(dev)
+    assert moe.moe_get_device_status(ws) == 0
+    sampler = None
+    if not args.no_clocks:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        sampler.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    start.record()
+    for _ in range(K):
+        call()
+    end.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop(t_begin, time.time()) if sampler is not None else None
+    assert moe.moe_get_device_status(ws) == 0
+    ms = start.elapsed_time(end) / K
+    # GEMM FLOPs: z = x W1 recomputed (2 T k H w1c), u = dy W2^T (2 T k H F), dW2 (2 T k F H),
+    # dW1 (2 T k H w1c), dx rows (2 T k w1c H); "useful" leaves out the recomputation
+    tk = cfg.T * cfg.k
+    flops = 2 * tk * cfg.H * (3 * w1c + 2 * cfg.F)
+    useful = flops - 2 * tk * cfg.H * w1c
+    peaks, peak_src = load_peaks()
+    sustained = bool(clocks and ("sw_power_cap" in clocks["reasons"] or
+                                 clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]))
+    tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
+    tf = flops / (ms / 1e3) / 1e12
+    emit({"metric": "MoE-layer backward tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
+          "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+          "dtype": "bf16 (fp32 accumulation)", "data": "synthetic", "config": config_dict(cfg, args, 1),
+          "gemm_tflops": tf, "useful_tflops": useful / (ms / 1e3) / 1e12,
+          "roofline": {"bound": "tensor", "achieved": tf, "peak": tf_peak, "unit": "TFLOP/s",
+                       "frac": tf / tf_peak,
+                       "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}"},
+          "clocks": clocks})
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.router_only:
         return run_router(args)
+    if args.backward:
+        return run_backward(args)
     return run_ours(args)
 
 
