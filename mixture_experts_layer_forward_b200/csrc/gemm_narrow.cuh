@@ -62,24 +62,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_swapped(int M, int N)
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// and-vote over the threads of a named barrier (all of them must reach it)
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred)
-{
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\t"
-                 "setp.ne.u32 p, %1, 0;\n\t"
-                 "bar.red.and.pred q, %2, %3, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r)
-                 : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
-                 : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Work item w -> cold expert slot j, column block cb, its m-tile, expert and padded row count.
 struct NarrowItem {
     int cb, mt, e, rows, n_pad;

@@ -58,7 +58,11 @@ constexpr int NUM_THREADS = 192;      // TMA warp, MMA warp, 4 epilogue warps
 constexpr int GATHER_THREADS = 128;   // 4 more warps that gather layer0 A rows (cp.async)
 constexpr int NUM_THREADS_GATHER = NUM_THREADS + GATHER_THREADS;
 constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE + NUM_BARS * 8 + 16;
+constexpr int SCALE_STAGE = 2 * BN * 4; // e4m3: the items' column scales, one buffer per accumulator
+// the scale buffers start on a 128-byte boundary after the barriers, the TMEM slot and the
+// abort flag (16-byte reads)
+constexpr int SCALE_OFF = STAGES * STAGE + ((NUM_BARS * 8 + 16 + 127) & ~127);
+constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + SCALE_OFF + SCALE_STAGE;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*b_mn_major=*/true);
 // e4m3 operands: both K-major; a K step of 128 values is the same 128-byte row as 64 bf16
@@ -133,6 +137,8 @@ struct GemmArgs {
     const float *a_scale;
     const float *b_scale;
     int b_scale_ld;
+    const int32_t *scale_idx; // a_scale index of each padded row when the rows arrive
+                              // already gathered (CTA-pair layer0); else gather_idx, or none
     // BMODE_WGRAD: wg_experts experts, each an output of wg_mtiles 128-row tiles (M =
     // 128 * wg_mtiles) by n_tiles 256-column tiles; expert e's K is its padded rows
     // [128 tile_off[e], 128 tile_off[e + 1]); out[(e * M + m) * ld_out + n]
@@ -189,7 +195,9 @@ __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, 
     gemm_map_work(w, a, e, mt, nt, ks);
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+// silu(z) = z * sigmoid(z), with the fast exponential and an IEEE reciprocal (1 + e^-z = inf
+// gives 0; NaN propagates)
+__device__ __forceinline__ float silu_f(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
 
 __device__ __forceinline__ float act_f(int act, float z)
 {
@@ -204,16 +212,19 @@ __device__ __forceinline__ float act_f(int act, float z)
 // Epilogue of one accumulator tile for the 32 rows of this warp: thread `lane` owns row `row`
 // and reads its TMEM lane `t_row` (already offset to the accumulator buffer). Warp-collective
 // (tcgen05.ld), so the whole warp calls it.
+// sbs: the item's column scales staged in shared memory (e4m3; SwiGLU: 128 gate then 128 up
+// columns, else the tile's 256 columns), or nullptr to read them from global memory
 template <int KIND, bool F8 = false>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt,
-                                              int ks = 0, int e = 0)
+                                              int ks = 0, int e = 0, const float *sbs = nullptr)
 {
     using namespace gemm;
     // e4m3 operands: the row's scale (0 for pad rows, whose outputs are never read)
     float sa = 1.0f;
     if (F8) {
-        if (args.gather_idx != nullptr) {
-            const int t = row < args.gather_len ? args.gather_idx[row] : -1;
+        const int32_t *si = args.scale_idx != nullptr ? args.scale_idx : args.gather_idx;
+        if (si != nullptr) {
+            const int t = row < args.gather_len ? si[row] : -1;
             sa = (t >= 0 && t < args.gather_rows) ? args.a_scale[t] : 0.0f;
         } else {
             sa = args.a_scale[row];
@@ -235,8 +246,10 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
                     float sg[8], su[8]; // column scales of the 8 gate and 8 up columns
                     if (F8) {
                         const int c0 = nt * 128 + c * 32 + v * 8;
-                        const float4 *pg = reinterpret_cast<const float4 *>(sb + c0);
-                        const float4 *pu = reinterpret_cast<const float4 *>(sb + args.up_col + c0);
+                        const float4 *pg = reinterpret_cast<const float4 *>(
+                            sbs ? sbs + c * 32 + v * 8 : sb + c0);
+                        const float4 *pu = reinterpret_cast<const float4 *>(
+                            sbs ? sbs + 128 + c * 32 + v * 8 : sb + args.up_col + c0);
                         const float4 g0 = pg[0], g1 = pg[1], u0 = pu[0], u1 = pu[1];
                         sg[0] = g0.x; sg[1] = g0.y; sg[2] = g0.z; sg[3] = g0.w;
                         sg[4] = g1.x; sg[5] = g1.y; sg[6] = g1.z; sg[7] = g1.w;
@@ -294,7 +307,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
                 for (int v = 0; v < 4; ++v) {
                     float sc[8]; // column scales of these 8 columns
                     if (F8) {
-                        const float4 *pc = reinterpret_cast<const float4 *>(sb + nt * BN + c * 32 + v * 8);
+                        const float4 *pc = reinterpret_cast<const float4 *>(
+                            sbs ? sbs + c * 32 + v * 8 : sb + nt * BN + c * 32 + v * 8);
                         const float4 c0 = pc[0], c1 = pc[1];
                         sc[0] = c0.x; sc[1] = c0.y; sc[2] = c0.z; sc[3] = c0.w;
                         sc[4] = c1.x; sc[5] = c1.y; sc[6] = c1.z; sc[7] = c1.w;
@@ -326,6 +340,24 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
+// and-vote over the threads of a named barrier (all of them must reach it)
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+                 : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // BMODE_WGRAD work item w: expert-major, then N tile, then M tile; its k-blocks of 64 rows
 __device__ __forceinline__ void wgrad_item(int w, const GemmArgs &a, int &e, int &mt, int &nt,
                                            int &kb0, int &kb1)
@@ -354,6 +386,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
     const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *scale_stage = reinterpret_cast<float *>(smem + SCALE_OFF);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -663,8 +696,10 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             bool ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, args.timeout_ns,
                                         args.status, 140 + KIND);
-            // the TMEM loads below are warp-collective: the whole warp continues or stops
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // the TMEM loads below are warp-collective: the whole warp continues or stops;
+            // with e4m3 the four epilogue warps also meet at a named barrier per item, so
+            // they continue or stop together
+            if (F8 ? !named_bar_and(1, 128, ok) : !__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int row = wgrad ? (e * args.wg_mtiles + mt) * BM + q * 32 + lane
                                   : mt * BM + q * 32 + lane;
@@ -673,6 +708,20 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                 uint4 *orow = reinterpret_cast<uint4 *>(args.out + (size_t)row * args.ld_out + nt * BN);
                 for (int c = 0; c < BN / 8; ++c)
                     if (nt * BN + c * 8 < args.n_cols) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+            } else if (F8) {
+                // the item's 256 column scales into shared memory once (the four epilogue
+                // warps, 2 each), then broadcast reads; one buffer per accumulator, so a
+                // warp rewrites a buffer only after every warp passed the next item's barrier
+                float *sbs = scale_stage + acc * BN;
+                const float *sbg = args.b_scale + (size_t)e * args.b_scale_ld;
+                for (int i = q * 32 + lane; i < BN; i += 128) {
+                    const int col = (KIND == GEMM_SWIGLU)
+                                        ? (i < 128 ? nt * 128 + i : args.up_col + nt * 128 + i - 128)
+                                        : nt * BN + i;
+                    sbs[i] = col < args.b_scale_ld ? sbg[col] : 0.0f;
+                }
+                named_bar_sync(1, 128);
+                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e, sbs);
             } else {
                 epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e);
             }
@@ -739,6 +788,7 @@ constexpr int STAGE = A_TILE + B_TILE;       // 32 KB per CTA
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16;
 constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, /*b_mn_major=*/true);
+constexpr uint32_t IDESC_F8 = idesc_e4m3_f32(256, 256);
 constexpr uint16_t PAIR_MASK = 0x3;
 } // namespace gemm2
 
@@ -753,7 +803,10 @@ __device__ __forceinline__ void gemm_map_pair(int w, const GemmArgs &a, int &e, 
     nt = local / cnt;
 }
 
-template <int KIND>
+// F8: e4m3 operands, both K-major: each CTA loads 128 rows x 128 bytes of A (its m-tile of
+// gathered x codes or h codes) and one 128-row box of the expert's K-major weight codes (its
+// half of N: the gate or up rows for SwiGLU); kind::f8f6f4, the scales in the epilogue.
+template <int KIND, bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm::NUM_THREADS, 1)
     moe_grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args)
@@ -844,9 +897,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm::NUM_THREADS, 1
                     tma_gather4_pair(a_dst + lane * 512, &tmA, leader_full, kb * BK, rows[0],
                                      rows[1], rows[2], rows[3]);
                 } else if (lane == 0) {
-                    tma_load_2d_pair(a_dst, &tmA, leader_full, kb * BK, my_mt * 128);
+                    tma_load_2d_pair(a_dst, &tmA, leader_full, kb * (F8 ? 128 : BK), my_mt * 128);
                 }
-                if (lane == 0) {
+                if (F8 && lane == 0) { // K-major codes: this CTA's 128 weight rows
+                    const int row = (KIND == GEMM_SWIGLU) ? (rank == 0 ? 0 : args.up_col) + nt * 128
+                                                          : nt * gemm::BN + (int)rank * 128;
+                    tma_load_3d_pair(b_dst, &tmB, leader_full, kb * 128, row, e);
+                }
+                if (!F8 && lane == 0) {
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         int col;
@@ -897,12 +955,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm::NUM_THREADS, 1
                         const uint32_t a_addr = smem_u32(smem + s * STAGE);
                         const uint32_t b_addr = a_addr + A_TILE;
                         const uint64_t a_desc = sw128_desc(a_addr, gemm::A_LBO, gemm::A_SBO);
-                        const uint64_t b_desc = sw128_desc(b_addr, gemm::B_LBO, gemm::B_SBO);
+                        if (F8) { // both K-major: +32 B per MMA
+                            const uint64_t b_desc = sw128_desc(b_addr, gemm::A_LBO, gemm::A_SBO);
 #pragma unroll
-                        for (int k = 0; k < BK / 16; ++k) {
-                            umma_bf16_pair(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
-                                           b_desc + (uint64_t)((k * 16 * 128) >> 4), gemm2::IDESC,
-                                           (kb | k) != 0 ? 1u : 0u);
+                            for (int k = 0; k < 4; ++k)
+                                umma_f8_pair(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                             b_desc + (uint64_t)((k * 32) >> 4), gemm2::IDESC_F8,
+                                             (kb | k) != 0 ? 1u : 0u);
+                        } else {
+                            const uint64_t b_desc = sw128_desc(b_addr, gemm::B_LBO, gemm::B_SBO);
+#pragma unroll
+                            for (int k = 0; k < BK / 16; ++k) {
+                                umma_bf16_pair(d_tmem, a_desc + (uint64_t)((k * 32) >> 4),
+                                               b_desc + (uint64_t)((k * 16 * 128) >> 4),
+                                               gemm2::IDESC, (kb | k) != 0 ? 1u : 0u);
+                            }
                         }
                         umma_commit_pair(empty_bar(s), gemm2::PAIR_MASK);
                         if (++s == STAGES) {
@@ -938,7 +1005,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm::NUM_THREADS, 1
                 const int row = my_mt * 128 + q * 32 + lane;
                 const uint32_t t_row =
                     tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * gemm::BN);
-                epilogue_rows<KIND>(args, t_row, row, nt);
+                epilogue_rows<KIND, F8>(args, t_row, row, nt, 0, e);
             }
             tc_fence_before();
             __syncwarp();

@@ -590,16 +590,16 @@ cudaError_t launch_quant_cols(const moe_bf16 *W, int E, int K, int N, uint8_t *W
     return cudaGetLastError();
 }
 
-template <int KIND>
+template <int KIND, bool F8 = false>
 cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
                              int max_work, cudaStream_t st)
 {
-    auto kern = moe_grouped_gemm_pair_kernel<KIND>;
+    auto kern = moe_grouped_gemm_pair_kernel<KIND, F8>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     // persistent grid: as many CTA pairs as can be resident at once (one CTA per SM)
-    static int cache[64][3] = {{0}};
+    static int cache[64][3] = {{0}}; // the e4m3 form has the same block size and shared memory
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     int &pairs = cache[dev][KIND];
@@ -1211,12 +1211,38 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     n0.n_tiles = gated ? F / 64 : (F + 127) / 128;
     n1.n_tiles = (H + 127) / 128;
 
+    if (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR) {
+        // CTA pairs: the x code rows gathered first (one byte per value: a row of H codes is
+        // moved as H / 2 two-byte elements), read by TMA; the scales looked up per row
+        uint8_t *xq_perm = at<uint8_t>(ws, L.x_perm);
+        CUtensorMap m_xp;
+        if (!make_map_2d_u8(&m_xp, xq_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM))
+            return MOE_ERR_CUDA;
+        moe_problem ph = *p;
+        ph.H = H / 2;
+        if (e == cudaSuccess)
+            e = launch_gather(&ph, reinterpret_cast<const moe_bf16 *>(xq), d.gather_idx, d.meta,
+                              reinterpret_cast<moe_bf16 *>(xq_perm), st);
+        GemmArgs p0 = a0, p1 = a1;
+        p0.ptile_off = p1.ptile_off = d.ptile_off;
+        p0.ptile_expert = p1.ptile_expert = d.ptile_expert;
+        p0.scale_idx = d.gather_idx;
+        p0.gather_idx = nullptr;
+        if (e == cudaSuccess)
+            e = gated ? launch_gemm_pair<GEMM_SWIGLU, true>(m_xp, m_w1, p0, L.max_tiles * p0.n_tiles, st)
+                      : launch_gemm_pair<GEMM_ACT, true>(m_xp, m_w1, p0, L.max_tiles * p0.n_tiles, st);
+        if (e == cudaSuccess) e = record(events, n_events, 3, st);
+        if (e == cudaSuccess) e = launch_quant_rows(h, L.pmax, F, d.meta, hq, sh, st);
+        if (e == cudaSuccess)
+            e = launch_gemm_pair<GEMM_SCALE, true>(m_h, m_w2, p1, L.max_tiles * p1.n_tiles, st);
+    } else {
     if (e == cudaSuccess)
         e = gated ? launch_gemm_select_f8<GEMM_SWIGLU>(m_x, m_w1, n_w1, a0, n0, st)
                   : launch_gemm_select_f8<GEMM_ACT>(m_x, m_w1, n_w1, a0, n0, st);
     if (e == cudaSuccess) e = record(events, n_events, 3, st);
     if (e == cudaSuccess) e = launch_quant_rows(h, L.pmax, F, d.meta, hq, sh, st);
     if (e == cudaSuccess) e = launch_gemm_select_f8<GEMM_SCALE>(m_h, m_w2, n_w2, a1, n1, st);
+    }
     if (e == cudaSuccess) e = record(events, n_events, 4, st);
     if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, nullptr);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);

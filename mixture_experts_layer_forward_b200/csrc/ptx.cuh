@@ -391,6 +391,18 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
         : "memory");
 }
 
+// The CTA-pair form of umma_f8 (cta_group::2, issued by the pair's leader).
+__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // When the pair MMAs issued so far complete, arrive once on the mbarrier at this shared-
 // memory offset in every CTA of `cta_mask`.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask)

@@ -99,8 +99,15 @@ FP8_CASES = [
 ]
 
 
+@pytest.fixture(params=[moe.GEMM_SINGLE_CTA, moe.GEMM_CTA_PAIR], ids=["single_cta", "cta_pair"])
+def fp8_gemm_mode(request):
+    prev = moe.moe_set_gemm_mode(request.param)
+    yield request.param
+    moe.moe_set_gemm_mode(prev)
+
+
 @pytest.mark.parametrize("case", FP8_CASES, ids=[c[0] for c in FP8_CASES])
-def test_forward_fp8_matches_oracle(case):
+def test_forward_fp8_matches_oracle(case, fp8_gemm_mode):
     name, T, H, F, E, k, act, zipf = case
     cfg = synth.LayerConfig(name, T=T, H=H, F=F, E=E, k=k, act=act, zipf_s=zipf)
     inp = synth.make_inputs(cfg, seed=13)
