@@ -369,12 +369,17 @@ MOE_API int moe_set_gemm_mode(int mode);
  * MOE_ORDER_NARROW (default): as MOE_ORDER_EXPERT, except that when every routed expert is
  *   cold (decode-sized batches) the device runs the layer with the operands swapped (the
  *   weight tile is the MMA's M = 128, the expert's rows rounded up to 16 its N): the same
- *   weight bytes with far less tensor-core work (measured 5-7% faster per GEMM there).
+ *   weight bytes with far less tensor-core work (measured 5-7% faster per GEMM there);
+ * MOE_ORDER_PHASED: in each launch every CTA first runs its share of the cold experts'
+ *   items in that operand-swapped form (all SMs streaming cold weights at once), then its
+ *   share of the other experts' 128-row items (as MOE_ORDER_NARROW when all are cold or
+ *   none is). Also used by moe_forward_fp8.
  * The layer outputs agree within the parity tolerance in every order; MOE_ORDER_EXPERT and
  * MOE_ORDER_MIXED are bitwise identical. Returns the previous order, or -1. */
 #define MOE_ORDER_EXPERT 0
 #define MOE_ORDER_MIXED 1
 #define MOE_ORDER_NARROW 2
+#define MOE_ORDER_PHASED 3
 MOE_API int moe_set_work_order(int order);
 
 /* Router variant (a tuning and test hook; not thread-safe). All give the same routing and

@@ -396,7 +396,7 @@ def moe_set_wait_timeout_ns(ns: int) -> int:
 
 GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED = 0, 1, 2, 3
 ROUTER_AUTO, ROUTER_SEQUENTIAL, ROUTER_FILTER = 0, 1, 2
-ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW = 0, 1, 2
+ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW, ORDER_PHASED = 0, 1, 2, 3
 
 
 def moe_set_fault_injection(layer0_item: int) -> int:
@@ -405,8 +405,8 @@ def moe_set_fault_injection(layer0_item: int) -> int:
 
 
 def moe_set_work_order(order: int) -> int:
-    """ORDER_EXPERT, ORDER_MIXED or ORDER_NARROW (default): how the single-CTA grouped GEMMs
-    treat experts with a single m-tile. Returns the previous order."""
+    """ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW or ORDER_PHASED: how the single-CTA grouped
+    GEMMs treat experts with a single m-tile. Returns the previous order."""
     rc = int(library().moe_set_work_order(int(order)))
     if rc < 0:
         raise ValueError(f"unknown work order {order}")

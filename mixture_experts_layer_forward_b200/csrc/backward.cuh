@@ -228,4 +228,17 @@ __global__ void __launch_bounds__(BWD_THREADS)
     }
 }
 
+// Zero the per-expert slabs (slab_vec 16-byte vectors each) of the experts without routed
+// rows; the weight-gradient GEMMs write the others. Grid (chunks, E).
+__global__ void zero_inactive_slabs_kernel(uint4 *__restrict__ dst, int64_t slab_vec,
+                                           const int32_t *__restrict__ counts)
+{
+    const int e = blockIdx.y;
+    if (counts[e] > 0) return;
+    uint4 *slab = dst + (size_t)e * slab_vec;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < slab_vec;
+         i += (int64_t)gridDim.x * blockDim.x)
+        slab[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 } // namespace moe

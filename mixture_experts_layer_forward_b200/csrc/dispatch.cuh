@@ -29,6 +29,7 @@ struct DispatchMeta {
     int padded_rows; // P_pad = num_tiles * M_TILE
     int num_ptiles;  // sum_e ceil(ceil(c_e / M_TILE) / 2): pairs of m-tiles of one expert
     int num_cold;    // experts with exactly one m-tile (their weights are read for one tile)
+    int num_active;  // experts with at least one routed row
 };
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(1024)
                          int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
                          int64_t padded_rows_max, int *__restrict__ ready, int n_ready,
                          int32_t *__restrict__ hot_off, int32_t *__restrict__ hot_tile_expert,
-                         int32_t *__restrict__ cold_tile)
+                         int32_t *__restrict__ cold_tile, int32_t *__restrict__ active_list)
 {
     // the fused layer kernel's tile-level ready counters start from zero on every call
     for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(1024)
     const int hot_t = ntile >= 2 ? ntile : 0;
     const int inc_h = block_inclusive_scan_1024(hot_t, warp_sums);
     const int inc_1 = block_inclusive_scan_1024(ntile == 1 ? 1 : 0, warp_sums);
+    const int inc_a = block_inclusive_scan_1024(c > 0 ? 1 : 0, warp_sums);
     if (e < E) {
         if (offsets != nullptr) {
             offsets[e + 1] = inc_c;
@@ -155,11 +157,13 @@ __global__ void __launch_bounds__(1024)
             for (int i = 0; i < hot_t; ++i) hot_tile_expert[inc_h - hot_t + i] = e;
             if (ntile == 1) cold_tile[inc_1 - 1] = tile_first;
         }
+        if (active_list != nullptr && c > 0) active_list[inc_a - 1] = e; // ascending ids
         if (e == E - 1) {
             meta->num_tiles = inc_t;
             meta->padded_rows = poff_next;
             meta->num_ptiles = inc_p;
             meta->num_cold = inc_1;
+            meta->num_active = inc_a;
             s_poff[E] = poff_next;
         }
     }

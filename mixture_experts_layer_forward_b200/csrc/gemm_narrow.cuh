@@ -80,11 +80,13 @@ __device__ __forceinline__ NarrowItem narrow_item(int w, const GemmArgs &a)
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
+// relinquish = false keeps the CTA's TMEM allocation permit for a second body afterwards.
 template <int KIND, bool F8 = false>
 __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                                                         const CUtensorMap &tmX,
                                                         const GemmArgs &args, uint8_t *smem,
-                                                        int w_first, int w_step)
+                                                        int w_first, int w_step,
+                                                        bool relinquish = true)
 {
     using namespace gemmn;
     float *xch = reinterpret_cast<float *>(smem + STAGES * STAGE); // [64][XCH_LD]
@@ -119,7 +121,7 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        if (relinquish) tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -391,6 +393,29 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
 
 namespace moe {
 
+// Phased order (wide.order == ORDER_HOT): every CTA first runs its share of the cold
+// experts' items in the narrow body (their weights streamed by all SMs at once, the MMA N
+// cut to the rows), then its share of the hot experts' 128-row items. Between the bodies the
+// narrow body's mbarriers are invalidated and the generic writes to shared memory ordered
+// before the wide body's TMA writes; the narrow body keeps the TMEM allocation permit.
+template <int KIND, bool F8>
+__device__ __forceinline__ void phased_bodies(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                              const CUtensorMap &tmWn, const GemmArgs &wide,
+                                              const GemmArgs &narrow, uint8_t *smem)
+{
+    if (wide.meta->num_cold > 0) {
+        grouped_gemm_narrow_cta<KIND, F8>(tmWn, tmA, narrow, smem, blockIdx.x, gridDim.x, false);
+        fence_proxy_async_smem();
+        if (threadIdx.x == 0) {
+            const uint32_t bar0 = smem_u32(smem + gemmn::STAGES * gemmn::STAGE + gemmn::XCH_BYTES);
+            for (int i = 0; i < gemmn::NUM_BARS; ++i) mbar_inval(bar0 + 8u * i);
+        }
+        __syncthreads();
+    }
+    if (wide.meta->num_cold < wide.meta->num_tiles)
+        grouped_gemm_cta<KIND, F8>(tmA, tmB, wide, smem, blockIdx.x, gridDim.x);
+}
+
 // One launch per layer that picks its kernel body on the device from the dispatch counts:
 // when every routed expert owns a single m-tile (decode-sized batches), all CTAs run the
 // narrow items; otherwise all CTAs run the 128-row items of every expert (args.order).
@@ -411,7 +436,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int num_cold = wide.meta->num_cold;
-    if (num_cold > 0 && num_cold == wide.meta->num_tiles)
+    if (wide.order == ORDER_HOT)
+        phased_bodies<KIND, false>(tmA, tmB, tmB, wide, narrow, smem);
+    else if (num_cold > 0 && num_cold == wide.meta->num_tiles)
         grouped_gemm_narrow_cta<KIND>(tmB, tmA, narrow, smem, blockIdx.x, gridDim.x);
     else
         grouped_gemm_cta<KIND>(tmA, tmB, wide, smem, blockIdx.x, gridDim.x);
@@ -430,7 +457,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int num_cold = wide.meta->num_cold;
-    if (num_cold > 0 && num_cold == wide.meta->num_tiles)
+    if (wide.order == ORDER_HOT)
+        phased_bodies<KIND, true>(tmA, tmB, tmWn, wide, narrow, smem);
+    else if (num_cold > 0 && num_cold == wide.meta->num_tiles)
         grouped_gemm_narrow_cta<KIND, true>(tmWn, tmA, narrow, smem, blockIdx.x, gridDim.x);
     else
         grouped_gemm_cta<KIND, true>(tmA, tmB, wide, smem, blockIdx.x, gridDim.x);

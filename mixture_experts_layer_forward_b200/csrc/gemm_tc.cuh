@@ -85,7 +85,7 @@ enum GemmKind { GEMM_SWIGLU = 0, GEMM_ACT = 1, GEMM_SCALE = 2, GEMM_LOGITS = 3 }
 //   BMODE_WGRAD   weight gradients: D[e] = A_e^T B_e over the expert's padded rows r (K),
 //                 A [rows, M] and B [rows, N] both read MN-major.
 enum GemmBMode { BMODE_FWD = 0, BMODE_KMAJOR = 1, BMODE_WGRAD = 2 };
-enum GemmOrder { ORDER_EXPERT = 0, ORDER_MIXED = 1 };
+enum GemmOrder { ORDER_EXPERT = 0, ORDER_MIXED = 1, ORDER_HOT = 2 };
 
 struct GemmArgs {
     const int32_t *tile_off;    // [E+1] first m-tile of each expert
@@ -96,7 +96,9 @@ struct GemmArgs {
     // Work order over the experts' m-tiles ("cold" experts have one m-tile, so their weight
     // tiles are streamed for a single tile; the others are "hot"):
     //   ORDER_EXPERT  expert-major over all m-tiles;
-    //   ORDER_MIXED   the cold experts' items spread evenly among the hot ones.
+    //   ORDER_MIXED   the cold experts' items spread evenly among the hot ones;
+    //   ORDER_HOT     the hot experts' m-tiles only, expert-major (the cold experts' items
+    //                 run in the narrow body first: moe_grouped_gemm_select_kernel).
     // hot_off [E+1] prefixes the hot experts' m-tiles, hot_tile_expert lists the expert of
     // each hot m-tile, cold_tile the m-tile of each cold expert (written by the dispatch scan).
     int order;
@@ -144,6 +146,7 @@ struct GemmArgs {
     // [128 tile_off[e], 128 tile_off[e + 1]); out[(e * M + m) * ld_out + n]
     int wg_experts;
     int wg_mtiles;
+    const int32_t *active_list; // BMODE_WGRAD: only these experts (meta->num_active of them)
 };
 
 __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
@@ -158,17 +161,20 @@ __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, 
         ks = r / a.n_tiles;
         return;
     }
-    if (a.order == ORDER_MIXED) {
-        const int64_t total = (int64_t)a.meta->num_tiles * a.n_tiles;
-        const int64_t cold = (int64_t)a.meta->num_cold * a.n_tiles;
-        const int64_t cb = (int64_t)w * cold / total;        // cold items before slot w
-        const int64_t cb1 = ((int64_t)w + 1) * cold / total;
-        if (cb1 > cb) { // slot w holds cold item cb: the expert's single m-tile, n-tile cb % n
-            const int j = (int)(cb / a.n_tiles);
-            nt = (int)(cb - (int64_t)j * a.n_tiles);
-            mt = a.cold_tile[j];
-            e = a.tile_expert[mt];
-            return;
+    if (a.order == ORDER_MIXED || a.order == ORDER_HOT) {
+        int64_t cb = 0;
+        if (a.order == ORDER_MIXED) {
+            const int64_t total = (int64_t)a.meta->num_tiles * a.n_tiles;
+            const int64_t cold = (int64_t)a.meta->num_cold * a.n_tiles;
+            cb = (int64_t)w * cold / total;                   // cold items before slot w
+            const int64_t cb1 = ((int64_t)w + 1) * cold / total;
+            if (cb1 > cb) { // slot w holds cold item cb: the expert's single m-tile, n-tile cb % n
+                const int j = (int)(cb / a.n_tiles);
+                nt = (int)(cb - (int64_t)j * a.n_tiles);
+                mt = a.cold_tile[j];
+                e = a.tile_expert[mt];
+                return;
+            }
         }
         const int h = (int)(w - cb); // hot item h, in the hot experts' expert-major order
         e = a.hot_tile_expert[h / a.n_tiles];
@@ -363,8 +369,9 @@ __device__ __forceinline__ void wgrad_item(int w, const GemmArgs &a, int &e, int
                                            int &kb0, int &kb1)
 {
     const int per = a.wg_mtiles * a.n_tiles;
-    e = w / per;
-    const int r = w - e * per;
+    const int j = w / per;
+    e = a.active_list != nullptr ? a.active_list[j] : j;
+    const int r = w - j * per;
     mt = r % a.wg_mtiles;
     nt = r / a.wg_mtiles;
     kb0 = a.tile_off[e] * (gemm::BM / gemm::BK);
@@ -421,9 +428,13 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
     const uint32_t tmem_base = *tmem_slot;
 
     const bool wgrad = (BMODE == BMODE_WGRAD);
-    const int num_tiles = wgrad ? 0 : (args.dense_m_tiles > 0 ? args.dense_m_tiles : args.meta->num_tiles);
+    const int num_tiles = wgrad ? 0
+                          : args.dense_m_tiles > 0 ? args.dense_m_tiles
+                          : args.order == ORDER_HOT ? args.meta->num_tiles - args.meta->num_cold
+                                                    : args.meta->num_tiles;
     const int n_split = (args.dense_m_tiles > 0 && args.k_split > 1) ? args.k_split : 1;
-    const int total = wgrad ? args.wg_experts * args.wg_mtiles * args.n_tiles
+    const int total = wgrad ? (args.active_list != nullptr ? args.meta->num_active : args.wg_experts) *
+                                  args.wg_mtiles * args.n_tiles
                             : num_tiles * args.n_tiles * n_split;
     const int KB = args.k_blocks;
     // k-blocks [kb_lo(ks), kb_lo(ks + 1)) belong to split ks (n_split <= KB: none is empty)

@@ -72,7 +72,7 @@ struct Layout {
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
         x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys, xq, sx, hq, sh,
-        bgu, ba, bdxp, bdw, bdl;
+        bgu, ba, bdxp, bdw, bdl, bact;
     size_t end_route, end_dispatch, end_forward, end_host, end_shared, end_fp8, end_bwd;
     int64_t pmax;
     int nchunk, max_tiles, n_ready;
@@ -202,6 +202,7 @@ Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd
     L.bdxp = take(bwd ? P * H * 2 : 0);
     L.bdw = take(bwd ? P * 4 : 0);
     L.bdl = take(bwd ? P * 4 : 0);
+    L.bact = take(bwd ? E * 4 : 0);
     L.end_bwd = o;
     return L;
 }
@@ -470,6 +471,7 @@ struct DispatchOut {
     int32_t *counts, *offsets, *poff, *gather_idx, *inv_pos, *tile_off, *tile_expert, *chunk;
     int32_t *ptile_off, *ptile_expert;
     int32_t *hot_off, *hot_tile_expert, *cold_tile;
+    int32_t *active_list = nullptr; // experts with rows, ascending (moe_backward)
     int *ready;
     int n_ready;
     float *row_w;
@@ -492,7 +494,8 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
                                              o.tile_off, o.tile_expert, o.ptile_off,
                                              o.ptile_expert, o.meta, o.gather_idx, o.row_w,
                                              L.pmax, o.ready, o.ready ? o.n_ready : 0,
-                                             o.hot_off, o.hot_tile_expert, o.cold_tile);
+                                             o.hot_off, o.hot_tile_expert, o.cold_tile,
+                                             o.active_list);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
@@ -893,8 +896,10 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     // work order of the single-CTA launches; MOE_ORDER_NARROW lets the device run the
     // operand-swapped body (N = the experts' row counts) when every expert is single-tile
     const int order = g_order.load();
-    const bool narrow = (order == MOE_ORDER_NARROW) && !pair;
-    a0.order = a1.order = (order == MOE_ORDER_MIXED) ? ORDER_MIXED : ORDER_EXPERT;
+    const bool narrow = (order == MOE_ORDER_NARROW || order == MOE_ORDER_PHASED) && !pair;
+    a0.order = a1.order = order == MOE_ORDER_MIXED    ? ORDER_MIXED
+                          : order == MOE_ORDER_PHASED ? ORDER_HOT
+                                                      : ORDER_EXPERT;
     GemmArgs n0 = a0, n1 = a1; // narrow items: column blocks of 64 (SwiGLU) or 128 columns
     n0.n_tiles = gated ? F / 64 : (F + 127) / 128;
     n1.n_tiles = (H + 127) / 128;
@@ -986,7 +991,8 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     }
     int32_t *topk_idx = at<int32_t>(ws, L.topk_idx);
     float *topk_w = at<float>(ws, L.topk_w);
-    const DispatchOut d = dispatch_bufs(ws, L);
+    DispatchOut d = dispatch_bufs(ws, L);
+    d.active_list = at<int32_t>(ws, L.bact);
     moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
     moe_bf16 *u = at<moe_bf16>(ws, L.h);   // [P, F]
     moe_bf16 *gy = at<moe_bf16>(ws, L.ys); // [P, H]
@@ -1057,8 +1063,18 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
         bwd_router_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(topk_w, d.inv_pos, dw_row, T, k, dl_row);
         e = cudaGetLastError();
     }
-    // weight gradients: dW2[e] = a_e^T gy_e, dW1[e] = x_perm_e^T dz_e
+    // weight gradients: zero for the experts without rows; dW2[e] = a_e^T gy_e and
+    // dW1[e] = x_perm_e^T dz_e for the others (the active list from the dispatch)
+    if (e == cudaSuccess) {
+        const int64_t v1 = (int64_t)H * w1c / 8, v2 = (int64_t)F * H / 8;
+        zero_inactive_slabs_kernel<<<dim3((unsigned)((v1 + 255) / 256 < 64 ? (v1 + 255) / 256 : 64), E), 256, 0, st>>>(
+            reinterpret_cast<uint4 *>(dW1), v1, d.counts);
+        zero_inactive_slabs_kernel<<<dim3((unsigned)((v2 + 255) / 256 < 64 ? (v2 + 255) / 256 : 64), E), 256, 0, st>>>(
+            reinterpret_cast<uint4 *>(dW2), v2, d.counts);
+        e = cudaGetLastError();
+    }
     GemmArgs w2 = g;
+    w2.active_list = d.active_list;
     w2.wg_experts = E;
     w2.wg_mtiles = F / gemm::BM;
     w2.out = reinterpret_cast<__nv_bfloat16 *>(dW2);
@@ -1067,6 +1083,7 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     if (e == cudaSuccess)
         e = launch_gemm_bwd<BMODE_WGRAD>(m_a, m_gy, w2, E * w2.wg_mtiles * w2.n_tiles, st);
     GemmArgs w1 = g;
+    w1.active_list = d.active_list;
     w1.wg_experts = E;
     w1.wg_mtiles = H / gemm::BM;
     w1.out = reinterpret_cast<__nv_bfloat16 *>(dW1);
@@ -1175,7 +1192,11 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     a0.tile_off = d.tile_off;
     a0.tile_expert = d.tile_expert;
     a0.meta = d.meta;
-    a0.order = ORDER_EXPERT;
+    a0.hot_off = d.hot_off;
+    a0.hot_tile_expert = d.hot_tile_expert;
+    a0.cold_tile = d.cold_tile;
+    // the select kernels below: MOE_ORDER_PHASED runs the cold experts' items narrow first
+    a0.order = g_order.load() == MOE_ORDER_PHASED ? ORDER_HOT : ORDER_EXPERT;
     a0.gather_idx = d.gather_idx;
     a0.gather_len = L.pmax;
     a0.gather_src = reinterpret_cast<const __nv_bfloat16 *>(xq); // bytes: the codes of x
@@ -1575,7 +1596,8 @@ int moe_set_gemm_mode(int mode)
 
 int moe_set_work_order(int order)
 {
-    if (order != MOE_ORDER_EXPERT && order != MOE_ORDER_MIXED && order != MOE_ORDER_NARROW)
+    if (order != MOE_ORDER_EXPERT && order != MOE_ORDER_MIXED && order != MOE_ORDER_NARROW &&
+        order != MOE_ORDER_PHASED)
         return -1;
     return g_order.exchange(order);
 }

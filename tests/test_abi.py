@@ -129,7 +129,7 @@ def test_forward_launch_count_follows_the_modes(lib):
     with pytest.raises(ValueError):
         moe.moe_set_router_mode(7)
     with pytest.raises(ValueError):
-        moe.moe_set_work_order(3)
+        moe.moe_set_work_order(4)
 
 
 def test_shared_expert_workspace_and_checks(lib):

@@ -122,6 +122,27 @@ def test_forward_fp8_matches_oracle(case, fp8_gemm_mode):
     assert_close(out, ref, name)
 
 
+@pytest.mark.parametrize("case", FP8_CASES[:2], ids=[c[0] for c in FP8_CASES[:2]])
+def test_forward_fp8_phased_order_matches_oracle(case):
+    """The phased order (single-tile experts in the narrow body first) on the FP8 path."""
+    name, T, H, F, E, k, act, zipf = case
+    cfg = synth.LayerConfig(name, T=T, H=H, F=F, E=E, k=k, act=act, zipf_s=zipf)
+    inp = synth.make_inputs(cfg, seed=13)
+    p = moe.Problem.from_config(cfg)
+    prev = moe.moe_set_work_order(moe.ORDER_PHASED)
+    try:
+        out, idx = forward_fp8(p, inp, quantize_on_gpu(p, inp))
+    finally:
+        moe.moe_set_work_order(prev)
+    r1q, r1s = oracle.quant_cols_fp8(bits(inp["W1"]))
+    r2q, r2s = oracle.quant_cols_fp8(bits(inp["W2"]))
+    b = None if inp["bias"] is None else inp["bias"].numpy()
+    ref, ridx, _ = oracle.moe_tokens_fp8(bits(inp["x"]), bits(inp["Wg"]), b, r1q, r1s, r2q, r2s,
+                                         k, np.arange(T), act=act)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    assert_close(out, ref, name)
+
+
 def test_forward_fp8_close_to_bf16_path():
     """The FP8 layer stays within its quantisation error of the bf16 layer on the GPU."""
     cfg = synth.LayerConfig("cmp", T=512, H=512, F=256, E=8, k=2)

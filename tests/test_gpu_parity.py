@@ -391,7 +391,7 @@ def test_work_orders_agree(name):
            else synth.CONFIGS[name])
     inp = synth.make_inputs(cfg, seed=16, device="cuda")
     outs = {}
-    for order in (moe.ORDER_EXPERT, moe.ORDER_MIXED, moe.ORDER_NARROW):
+    for order in (moe.ORDER_EXPERT, moe.ORDER_MIXED, moe.ORDER_NARROW, moe.ORDER_PHASED):
         prev = moe.moe_set_work_order(order)
         try:
             outs[order] = run_forward(cfg, inp)[0]
@@ -399,11 +399,12 @@ def test_work_orders_agree(name):
             moe.moe_set_work_order(prev)
     assert torch.equal(outs[moe.ORDER_EXPERT], outs[moe.ORDER_MIXED])
     a = outs[moe.ORDER_EXPERT].float()
-    d = (outs[moe.ORDER_NARROW].float() - a).abs()
-    assert bool(torch.all(d <= ATOL + RTOL * a.abs())), float(d.max())
+    for order in (moe.ORDER_NARROW, moe.ORDER_PHASED):
+        d = (outs[order].float() - a).abs()
+        assert bool(torch.all(d <= ATOL + RTOL * a.abs())), (order, float(d.max()))
 
 
-@pytest.mark.parametrize("order", [0, 1, 2], ids=["expert", "mixed", "narrow"])
+@pytest.mark.parametrize("order", [0, 1, 2, 3], ids=["expert", "mixed", "narrow", "phased"])
 def test_forward_orders_match_oracle(order):
     """A mix of multi-tile and single-tile experts (ragged row counts, some experts empty)
     against the oracle in every work order."""
