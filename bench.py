@@ -344,6 +344,14 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     assert moe.moe_get_device_status(ws) == 0, "device status after warm-up"
     active_experts = int(torch.unique(idx_buf).numel())  # for the layer0 byte count below
+    counts = torch.bincount(idx_buf.flatten().long(), minlength=cfg.E).cpu()
+    nz = counts[counts > 0]
+    routing = {"active_experts": active_experts,
+               "rows_max": int(counts.max()), "rows_min_active": int(nz.min()) if nz.numel() else 0,
+               "single_tile_experts": int(((counts > 0) & (counts <= 128)).sum()),
+               "padded_rows": int(((counts + 127) // 128 * 128).sum()), "routed_rows": cfg.T * cfg.k}
+    if cfg.E <= 64:
+        routing["expert_histogram"] = [int(c) for c in counts]
 
     # stage events of every timed step (recorded on the launch stream by the library)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGE_EVENTS)]
@@ -376,6 +384,21 @@ def run_ours(args):
     assert status == 0, f"device status {status}"
     ms = dp.max_over_ranks(ms_local, device=dev)
     ms_per_step = ms / K
+
+    # the same layer with a cold L2: a 256 MiB buffer written before each step (outside each
+    # step's events); a reported figure beside the warm, back-to-back value above
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n_cold = min(K, 20)
+    cold_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_cold)]
+    for a, b in cold_ev:
+        flush.zero_()
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    cold_ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in cold_ev) / n_cold, device=dev)
+    del flush
 
     stage_names = ["route", "dispatch", "layer0_gemm_swiglu", "layer1_gemm_scale", "combine"]
     stage_ms = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
@@ -461,6 +484,9 @@ def run_ours(args):
                          moe.moe_forward_launches(p)) * K,
         "clocks": clocks,
         "e2e": e2e,
+        "cold_l2": {"ms_per_step": cold_ms, "steps": n_cold,
+                    "how": "256 MiB buffer written before each step, outside its events"},
+        "routing": routing,
     }
 
     if rank == 0 and not args.no_cpu_baseline and not args.fp8:
