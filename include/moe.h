@@ -275,6 +275,20 @@ MOE_API moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *
                                           size_t ws_bytes, void *stream, void *const *events,
                                           int32_t n_events);
 
+/* The experts alone, for rows whose expert and gate are already known: the step each rank
+ * runs on the rows it received under expert parallelism (the pages' multi-GPU layout, §2.1
+ * and §3.1: experts sharded across GPUs, tokens exchanged all-to-all), or a caller's own
+ * router. With p->top_k == 1 and p->E the experts held here, for each row r < p->T:
+ *   out[r] = bf16(gate[r] * FFN_{expert[r]}(x[r]))
+ * computed exactly as moe_forward computes a routed row (dispatch into 128-row expert tiles,
+ * the same GEMMs and epilogues, one bf16 rounding of the gated row). expert [T] int32 in
+ * [0, E) (an id outside it is reported as MOE_ERR_DEVICE_BAD_INDEX through
+ * moe_get_device_status), gate [T] fp32. Workspace: moe_workspace_size(p). */
+MOE_API moe_status moe_experts_forward(const moe_problem *p, const moe_bf16 *x,
+                                       const int32_t *expert, const float *gate,
+                                       const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
+                                       void *ws, size_t ws_bytes, void *stream);
+
 /* Backward pass (training; beyond the pages, which describe the forward).
  * Given dout = dL/dout [T, H] bf16, the gradients of the layer moe_forward computes, with the
  * selection held fixed (it is piecewise constant) and the gates the softmax over the

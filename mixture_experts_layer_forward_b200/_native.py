@@ -100,6 +100,7 @@ def library() -> ctypes.CDLL:
             "moe_forward_fp8": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "moe_forward_fp8_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                         ctypes.POINTER(vp), i32], i32),
+            "moe_experts_forward": ([P] + [vp] * 7 + [sz, vp], i32),
             "moe_backward_workspace_size": ([P], sz),
             "moe_backward": ([P] + [vp] * 12 + [sz, vp], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -354,6 +355,18 @@ def moe_forward_fp8_staged(p, x, Wg, bias, W1q, s1, W2q, s2, out, ws, events, to
                                                      topk_idx_out, topk_w_out), w, n,
                                           _stream(stream), arr, MOE_NUM_STAGE_EVENTS)
     _check("moe_forward_fp8_staged", rc)
+
+
+def moe_experts_forward(p, x, expert, gate, W1, W2, out, ws, stream=None):
+    """out[r] = gate[r] * FFN_{expert[r]}(x[r]) for rows with known routing (p.top_k == 1)."""
+    bf = torch.bfloat16
+    w, n = _ws(ws)
+    rc = library().moe_experts_forward(ctypes.byref(p), _ptr(x, bf, "x"),
+                                       _ptr(expert, torch.int32, "expert"),
+                                       _ptr(gate, torch.float32, "gate"), _ptr(W1, bf, "W1"),
+                                       _ptr(W2, bf, "W2"), _ptr(out, bf, "out"), w, n,
+                                       _stream(stream))
+    _check("moe_experts_forward", rc)
 
 
 def moe_backward_workspace_size(p: Problem) -> int:

@@ -770,14 +770,17 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                         cudaStream_t st, void *const *events, int n_events,
-                        const moe_shared_expert *sh = nullptr)
+                        const moe_shared_expert *sh = nullptr,
+                        const int32_t *given_idx = nullptr, const float *given_w = nullptr)
 {
     moe_status s = check_problem(p);
     if (s != MOE_OK) return s;
     if (n_events != 0 && (n_events != MOE_NUM_STAGE_EVENTS || events == nullptr))
         return MOE_ERR_INVALID_ARG;
-    if (ws == nullptr || (p->T > 0 && (x == nullptr || out == nullptr)) || Wg == nullptr ||
-        W1 == nullptr || W2 == nullptr)
+    const bool given = (given_idx != nullptr); // routing supplied: no router launch, no W_g
+    if (ws == nullptr || (p->T > 0 && (x == nullptr || out == nullptr)) ||
+        (Wg == nullptr && !given) || W1 == nullptr || W2 == nullptr ||
+        (given && p->T > 0 && given_w == nullptr))
         return MOE_ERR_INVALID_ARG;
     const Layout L = make_layout(p);
     if (ws_bytes < L.end_forward) return MOE_ERR_WORKSPACE;
@@ -792,8 +795,10 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         for (int i = 0; i < n_events && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
         return to_status(e);
     }
-    int32_t *topk_idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
-    float *topk_w = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
+    int32_t *topk_idx = given ? const_cast<int32_t *>(given_idx)
+                              : (topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx));
+    float *topk_w = given ? const_cast<float *>(given_w)
+                          : (topk_w_out ? topk_w_out : at<float>(ws, L.topk_w));
     const DispatchOut d = dispatch_bufs(ws, L);
     moe_bf16 *x_perm = at<moe_bf16>(ws, L.x_perm);
     moe_bf16 *h = at<moe_bf16>(ws, L.h);
@@ -816,11 +821,12 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     const int64_t timeout = g_timeout_ns.load();
     const FilterBufs fb = filter_bufs(ws, L);
     cudaError_t e = record(events, n_events, 0, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !given)
         e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st,
                          &fb);
     if (e == cudaSuccess) e = record(events, n_events, 1, st);
-    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
+    // with the routing supplied the dispatch clears the status word (and checks the ids)
+    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, given ? 1 : 0, st);
     if (e == cudaSuccess && pair) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
     if (e == cudaSuccess) e = record(events, n_events, 2, st);
 
@@ -1670,6 +1676,19 @@ moe_status moe_forward_fp8_staged(const moe_problem *p, const moe_bf16 *x, const
 {
     return forward_impl_fp8(p, x, Wg, bias, W1q, s1, W2q, s2, out, topk_idx_out, topk_w_out, ws,
                             ws_bytes, static_cast<cudaStream_t>(stream), events, n_events);
+}
+
+moe_status moe_experts_forward(const moe_problem *p, const moe_bf16 *x, const int32_t *expert,
+                               const float *gate, const moe_bf16 *W1, const moe_bf16 *W2,
+                               moe_bf16 *out, void *ws, size_t ws_bytes, void *stream)
+{
+    if (p != nullptr && p->top_k != 1) return MOE_ERR_INVALID_ARG;
+    if (p != nullptr && p->T > 0 && (expert == nullptr || gate == nullptr || !aligned4(expert) ||
+                                     !aligned4(gate)))
+        return MOE_ERR_INVALID_ARG;
+    return forward_impl(p, x, nullptr, nullptr, W1, W2, out, nullptr, nullptr, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), nullptr, 0, nullptr,
+                        p != nullptr && p->T > 0 ? expert : nullptr, gate);
 }
 
 size_t moe_backward_workspace_size(const moe_problem *p)

@@ -1,0 +1,127 @@
+"""Expert parallelism: the layer with its experts sharded across GPUs.
+
+This is the pages' multi-GPU layout (Comet: Fine-grained Computation-communication
+Overlapping for Mixture-of-Experts, §2.1 "MoE Structure" and §3.1: experts are placed on
+different GPUs, the routed tokens travel to their experts' GPU before layer0 and the expert
+outputs travel back after layer1, by all-to-all). Each rank holds E / world experts
+(experts r * E_local .. (r + 1) * E_local - 1 on rank r), a replicated router, and its own
+tokens:
+
+1. route its tokens (moe_route on the full W_g);
+2. order its T * k routed pairs by destination rank, stable in (token, selection) order;
+3. all-to-all the row counts, then the x rows, the local expert ids and the gates;
+4. run its experts on the rows it received (moe_experts_forward: the same per-row
+   arithmetic as moe_forward, so every gated row is bitwise the row moe_forward computes);
+5. all-to-all the gated rows back, in the order they were sent;
+6. combine: out[t] = bf16(sum over j ascending of row (t, j)), fp32 sum (moe_combine).
+
+bf16 rows cross the collectives as int32 words (the same bytes, two values per word, a
+dtype every backend carries). The exchange runs on NCCL between GPUs; the expert and combine
+steps are pluggable, so the plan is also exercised on CPU (gloo) by the tests.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def experts_per_rank(E: int, world: int) -> int:
+    if E % world != 0:
+        raise ValueError(f"E = {E} experts do not shard evenly over {world} ranks")
+    return E // world
+
+
+def dispatch_plan(topk_idx: torch.Tensor, E: int, world: int):
+    """For the [T, k] routing of this rank: the stable order of its T * k pairs by
+    destination rank, the number of pairs sent to each rank, and each sent pair's expert id
+    local to its destination."""
+    e_loc = experts_per_rank(E, world)
+    flat = topk_idx.reshape(-1).long()
+    dest = torch.div(flat, e_loc, rounding_mode="floor")
+    order = torch.argsort(dest, stable=True)
+    send_counts = torch.bincount(dest, minlength=world)
+    local_ids = (flat - dest * e_loc)[order]
+    return order, send_counts, local_ids
+
+
+def _exchange(send: torch.Tensor, send_counts, recv_counts, group):
+    """all-to-all of the rows of `send` (already in destination order). bf16 rows travel as
+    int32 words (two values each, H even)."""
+    bf = send.dtype == torch.bfloat16
+    bits = send.contiguous().view(torch.int32) if bf else send.contiguous()
+    shape = (int(sum(recv_counts)),) + tuple(bits.shape[1:])
+    recv = torch.empty(shape, dtype=bits.dtype, device=send.device)
+    dist.all_to_all_single(recv, bits, output_split_sizes=list(recv_counts),
+                           input_split_sizes=list(send_counts), group=group)
+    return recv.view(torch.bfloat16) if bf else recv
+
+
+def ep_forward(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int,
+               expert_fn, combine_fn, group=None) -> torch.Tensor:
+    """Steps 2-6 above for this rank's tokens x [T, H] (bf16) routed to topk_idx / topk_w
+    [T, k]. expert_fn(rows [R, H], local ids [R] int32, gates [R] fp32) -> gated rows [R, H]
+    bf16 for this rank's experts; combine_fn(rows [T * k, H], inv_pos [T, k] int32) -> out."""
+    world = dist.get_world_size(group)
+    T, k = topk_idx.shape
+    order, send_counts, local_ids = dispatch_plan(topk_idx, E, world)
+    send_counts = send_counts.to(device=x.device, dtype=torch.int64)
+    recv_counts = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv_counts, send_counts, group=group)
+    sc, rc = send_counts.tolist(), recv_counts.tolist() # split sizes on the host
+    tok = torch.div(order, k, rounding_mode="floor").to(x.device)
+    rows = _exchange(x.index_select(0, tok), sc, rc, group)
+    ids = _exchange(local_ids.to(device=x.device, dtype=torch.int32), sc, rc, group)
+    gates = _exchange(topk_w.reshape(-1)[order.to(topk_w.device)].float(), sc, rc, group)
+    y = expert_fn(rows, ids, gates)
+    back = _exchange(y, rc, sc, group)                # row i of `back` is pair order[i]
+    inv = torch.empty_like(order)
+    inv[order] = torch.arange(order.numel(), device=order.device)
+    return combine_fn(back, inv.view(T, k).to(device=x.device, dtype=torch.int32))
+
+
+def gpu_expert_fn(H: int, F: int, E_local: int, W1_local, W2_local, act: int = 0):
+    """expert_fn running moe_experts_forward on this GPU's expert weights."""
+    from . import _native as moe
+
+    def fn(rows, ids, gates):
+        R = rows.shape[0]
+        p = moe.Problem.make(R, H, F, E_local, 1, act)
+        out = torch.empty(R, H, dtype=torch.bfloat16, device=rows.device)
+        ws = torch.empty(max(moe.moe_workspace_size(p), 1), dtype=torch.uint8, device=rows.device)
+        moe.moe_experts_forward(p, rows, ids, gates, W1_local, W2_local, out, ws)
+        if moe.moe_get_device_status(ws) != 0:
+            raise RuntimeError("moe_experts_forward reported a device error")
+        return out
+
+    return fn
+
+
+def gpu_combine_fn(H: int, F: int, E: int, k: int):
+    """combine_fn running moe_combine (fp32 sum over j ascending, one bf16 rounding)."""
+    from . import _native as moe
+
+    def fn(back, inv_pos):
+        T = inv_pos.shape[0]
+        p = moe.Problem.make(T, H, F, E, k)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=back.device)
+        moe.moe_combine(p, back, inv_pos, out)
+        return out
+
+    return fn
+
+
+def ep_moe_forward(p, x, Wg, bias, W1_local, W2_local, group=None):
+    """The whole layer under expert parallelism on this rank's GPU: route (replicated W_g,
+    all E experts), exchange, local experts, exchange back, combine. p is the full layer's
+    problem (all E experts, this rank's T tokens); W1_local / W2_local hold this rank's
+    E / world experts."""
+    from . import _native as moe
+
+    world = dist.get_world_size(group)
+    e_loc = experts_per_rank(p.E, world)
+    idx = torch.empty(p.T, p.top_k, dtype=torch.int32, device=x.device)
+    w = torch.empty(p.T, p.top_k, dtype=torch.float32, device=x.device)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=x.device)
+    moe.moe_route(p, x, Wg, bias, idx, w, ws)
+    return ep_forward(x, idx, w, p.E, gpu_expert_fn(p.H, p.F, e_loc, W1_local, W2_local, p.act),
+                      gpu_combine_fn(p.H, p.F, p.E, p.top_k), group)
