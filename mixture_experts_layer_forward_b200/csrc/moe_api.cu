@@ -456,8 +456,10 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
         launch_route_logits<ROUTE_MID_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     } else if (E > 16 && large_blocks >= sms / 2) {
         launch_route_logits<ROUTE_LARGE_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
-    } else {
+    } else if ((int64_t)((T + 7) / 8) * ((E + 15) / 16) <= sms) {
         launch_route_logits<ROUTE_NARROW_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
+    } else {
+        launch_route_logits<ROUTE_NARROW2_CFG>(xb, wb, lbias, logits, T, H, E, status, st);
     }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

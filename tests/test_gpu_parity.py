@@ -91,6 +91,9 @@ ROUTE_CASES = [
     ("e64_selbias", 130, 384, 64, 8, False, 1.2, 2),
     ("e256_selbias_tile", 2100, 128, 256, 8, False, 1.2, 2),
     ("e512_max_filter", 600, 192, 512, 16, False, 1.2, 0),
+    # small batches with many experts: both decode tile shapes of the sequential router
+    ("e256_t64_decode", 64, 512, 256, 8, False, 1.2, 0),
+    ("e256_t150_decode", 150, 512, 256, 8, False, 0.0, 0),
 ]
 
 
