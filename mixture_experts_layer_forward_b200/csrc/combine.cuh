@@ -13,6 +13,8 @@
 
 namespace moe {
 
+constexpr int COMBINE_BATCH = 2; // top-k rows whose loads one thread issues together
+
 __global__ void __launch_bounds__(256)
     combine_kernel(const __nv_bfloat16 *__restrict__ ys, int64_t ys_rows,
                    const int32_t *__restrict__ inv_pos, int T, int H, int k,
@@ -32,17 +34,34 @@ __global__ void __launch_bounds__(256)
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int r = inv_pos[(size_t)t * k + j];
-            if (r < 0 || (int64_t)r >= ys_rows) {
-                record_status(status, DEV_BAD_INDEX, 3);
-                continue;
+        // up to COMBINE_BATCH rows per round: all their indices, then all their loads, are
+        // issued before the first add, so a thread keeps several loads in flight; the adds
+        // still run with j ascending
+        for (int j0 = 0; j0 < k; j0 += COMBINE_BATCH) {
+            int rr[COMBINE_BATCH];
+#pragma unroll
+            for (int q = 0; q < COMBINE_BATCH; ++q)
+                rr[q] = (j0 + q < k) ? inv_pos[(size_t)t * k + j0 + q] : 0;
+            uint4 uu[COMBINE_BATCH];
+#pragma unroll
+            for (int q = 0; q < COMBINE_BATCH; ++q) {
+                const bool ok = (j0 + q < k) && rr[q] >= 0 && (int64_t)rr[q] < ys_rows;
+                uu[q] = ok ? *reinterpret_cast<const uint4 *>(ys + (size_t)rr[q] * H + (size_t)v * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
             }
-            const uint4 u = *reinterpret_cast<const uint4 *>(ys + (size_t)r * H + (size_t)v * 8);
-            acc[0] += bf16_lo(u.x); acc[1] += bf16_hi(u.x);
-            acc[2] += bf16_lo(u.y); acc[3] += bf16_hi(u.y);
-            acc[4] += bf16_lo(u.z); acc[5] += bf16_hi(u.z);
-            acc[6] += bf16_lo(u.w); acc[7] += bf16_hi(u.w);
+#pragma unroll
+            for (int q = 0; q < COMBINE_BATCH; ++q) {
+                if (j0 + q >= k) break;
+                if (rr[q] < 0 || (int64_t)rr[q] >= ys_rows) {
+                    record_status(status, DEV_BAD_INDEX, 3);
+                    continue;
+                }
+                const uint4 u = uu[q];
+                acc[0] += bf16_lo(u.x); acc[1] += bf16_hi(u.x);
+                acc[2] += bf16_lo(u.y); acc[3] += bf16_hi(u.y);
+                acc[4] += bf16_lo(u.z); acc[5] += bf16_hi(u.z);
+                acc[6] += bf16_lo(u.w); acc[7] += bf16_hi(u.w);
+            }
         }
         if (ys_shared != nullptr) {
             const uint4 u = *reinterpret_cast<const uint4 *>(ys_shared + (size_t)t * H + (size_t)v * 8);
