@@ -109,8 +109,9 @@ MOE_API size_t moe_workspace_size(const moe_problem *p);
 /* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
  * current GEMM and router modes, assuming 16-byte aligned operands: the
  * router (2, or 3 with the tensor-core filter), the dispatch (3) and the layers (layer0,
- * layer1 and the combine: 3; 4 with the CTA-pair GEMM, which first gathers x; 1 with
- * MOE_GEMM_FUSED).
+ * layer1 and the combine: 3; 4 when x is first gathered into expert-sorted rows, which the
+ * CTA-pair GEMM always does and the single-CTA GEMM does when T * top_k >= E * 128;
+ * 1 with MOE_GEMM_FUSED).
  * 0 for T == 0; -1 if *p is invalid. */
 MOE_API int moe_forward_launches(const moe_problem *p);
 

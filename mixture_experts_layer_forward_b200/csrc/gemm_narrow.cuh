@@ -326,8 +326,10 @@ __device__ __forceinline__ void grouped_gemm_narrow_cta(const CUtensorMap &tmW,
                         if (i < nc) {
                             const int64_t row = row0 + c0 + i;
                             float sa;
-                            if (args.gather_idx != nullptr) {
-                                const int t = row < args.gather_len ? args.gather_idx[row] : -1;
+                            const int32_t *si =
+                                args.scale_idx != nullptr ? args.scale_idx : args.gather_idx;
+                            if (si != nullptr) {
+                                const int t = row < args.gather_len ? si[row] : -1;
                                 sa = (t >= 0 && t < args.gather_rows) ? args.a_scale[t] : 0.0f;
                             } else {
                                 sa = args.a_scale[row];

@@ -102,24 +102,26 @@ def test_forward_launch_count_follows_the_modes(lib):
     prev_g = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
     prev_o = moe.moe_set_work_order(moe.ORDER_EXPERT)
     try:
-        # router 2 (3 with the filter) + dispatch 3 + layer0, layer1, combine
-        assert moe.moe_forward_launches(mixtral) == 8   # E = 8: sequential router
-        assert moe.moe_forward_launches(qwen2) == 9     # T*E >= 2^16: filter router
-        assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential router
+        # router 2 (3 with the filter) + dispatch 3 + [x gather] + layer0, layer1, combine;
+        # the bench layers gather x into sorted rows (T * k >= 128 E), decode does not
+        assert moe.moe_forward_launches(mixtral) == 9   # E = 8: sequential router
+        assert moe.moe_forward_launches(qwen2) == 10    # T*E >= 2^16: filter router
+        assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential, no gather
         phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
-        assert moe.moe_forward_launches(phi35) == 9     # E = 16: filter router
+        assert moe.moe_forward_launches(phi35) == 10    # E = 16: filter router
         moe.moe_set_router_mode(moe.ROUTER_FILTER)
         assert moe.moe_forward_launches(decode) == 9
-        assert moe.moe_forward_launches(mixtral) == 9   # forced: E = 8 qualifies
+        assert moe.moe_forward_launches(mixtral) == 10  # forced: E = 8 qualifies
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 8  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
-        assert moe.moe_forward_launches(qwen2) == 8
+        assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
-        assert moe.moe_forward_launches(qwen2) == 8
-        moe.moe_set_gemm_mode(moe.GEMM_FUSED)
+        assert moe.moe_forward_launches(qwen2) == 9
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED)           # gathers in the kernel
         assert moe.moe_forward_launches(qwen2) == 6
         moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)        # gathers x; no narrow launches
         assert moe.moe_forward_launches(qwen2) == 9
+        assert moe.moe_forward_launches(decode) == 9
         assert moe.moe_forward_launches(moe.Problem.make(0, 128, 128, 8, 2)) == 0
         assert moe.moe_forward_launches(moe.Problem.make(4, 100, 128, 8, 2)) == -1  # H % 64
     finally:
