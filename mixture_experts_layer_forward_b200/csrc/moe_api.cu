@@ -1020,7 +1020,8 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     float *dw_row = at<float>(ws, L.bdw), *dl_row = at<float>(ws, L.bdl);
 
     CUtensorMap m_x, m_w1, m_w2k, m_gu, m_a, m_gy, m_xp, m_dz, m_w1k;
-    if (!make_map_2d(&m_x, x, (uint64_t)T, (uint64_t)H, 1) || // unused: rows are gathered
+    // z = x W1 reads the expert-sorted x_perm rows (gathered for dW1 anyway) with TMA
+    if (!make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM) ||
         !make_map_3d(&m_w1, W1, (uint64_t)E, (uint64_t)H, (uint64_t)w1c) ||
         !make_map_3d(&m_w2k, W2, (uint64_t)E, (uint64_t)F, (uint64_t)H, 128) ||
         !make_map_2d(&m_a, a, (uint64_t)L.pmax, (uint64_t)F, 64) ||
@@ -1048,10 +1049,8 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     g.gather_len = L.pmax;
     g.gather_rows = T;
     g.gather_ld = H;
-    // z = x W1 (recomputed pre-activations), x rows gathered
+    // z = x W1 (recomputed pre-activations) from the sorted rows
     GemmArgs gz = g;
-    gz.gather_idx = d.gather_idx;
-    gz.gather_src = reinterpret_cast<const __nv_bfloat16 *>(x);
     gz.out = reinterpret_cast<__nv_bfloat16 *>(gu);
     gz.ld_out = gz.n_cols = w1c;
     gz.n_tiles = (w1c + gemm::BN - 1) / gemm::BN;
@@ -1065,8 +1064,10 @@ moe_status backward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     gu_.ld_out = gu_.n_cols = F;
     gu_.n_tiles = (F + gemm::BN - 1) / gemm::BN;
     gu_.k_blocks = H / gemm::BK;
+    CUtensorMap m_dy; // unused: the dy rows are gathered in the kernel
+    if (!make_map_2d(&m_dy, dy, (uint64_t)T, (uint64_t)H, 1)) return MOE_ERR_CUDA;
     if (e == cudaSuccess)
-        e = launch_gemm_bwd<BMODE_KMAJOR>(m_x, m_w2k, gu_, L.max_tiles * gu_.n_tiles, st);
+        e = launch_gemm_bwd<BMODE_KMAJOR>(m_dy, m_w2k, gu_, L.max_tiles * gu_.n_tiles, st);
     // row pass: a, dz (in place of z), gy, dw
     if (e == cudaSuccess) {
         int grid = sm_count() * 8;
