@@ -257,8 +257,9 @@ MOE_API size_t moe_workspace_size_fp8(const moe_problem *p);
  * the activation, h stored bf16; h rows quantised; layer1 on codes, times
  * s_h[row] * s2[column] * the gate weight, stored bf16; the combine as moe_forward.
  * moe_forward_launches(p) counts the same route and dispatch kernels; this path launches
- * 2 + 3 + 1 + 1 + 1 + 1 kernels after the router (dispatch, x quantisation, layer0,
- * h quantisation, layer1, combine). */
+ * 3 + 1 + 1 + 1 + 1 + 1 kernels after the router (dispatch, x quantisation, layer0,
+ * h quantisation, layer1, combine), plus one that gathers the x codes into expert-sorted
+ * rows when T * top_k >= 128 * E (layer0 then reads them with TMA). */
 MOE_API moe_status moe_forward_fp8(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                                    const float *bias, const moe_fp8 *W1q, const float *s1,
                                    const moe_fp8 *W2q, const float *s2, moe_bf16 *out,

@@ -147,6 +147,8 @@ struct GemmArgs {
     int wg_experts;
     int wg_mtiles;
     const int32_t *active_list; // BMODE_WGRAD: only these experts (meta->num_active of them)
+    int epi8; // A by TMA (no gather): warps 6..9 join the epilogue, each pair of warps on one
+              // TMEM lane quarter splits the item's column chunks (launch with 320 threads)
 };
 
 __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
@@ -220,9 +222,12 @@ __device__ __forceinline__ float act_f(int act, float z)
 // (tcgen05.ld), so the whole warp calls it.
 // sbs: the item's column scales staged in shared memory (e4m3; SwiGLU: 128 gate then 128 up
 // columns, else the tile's 256 columns), or nullptr to read them from global memory
+// Column chunks [c_lo, c_hi) of the item (32 columns each: SwiGLU 4 gate/up pairs, else 8);
+// c_hi < 0: all of them.
 template <int KIND, bool F8 = false>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_row, int row, int nt,
-                                              int ks = 0, int e = 0, const float *sbs = nullptr)
+                                              int ks = 0, int e = 0, const float *sbs = nullptr,
+                                              int c_lo = 0, int c_hi = -1)
 {
     using namespace gemm;
     // e4m3 operands: the row's scale (0 for pad rows, whose outputs are never read)
@@ -240,7 +245,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
     if (KIND == GEMM_SWIGLU) {
         __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * 128;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = c_lo; c < (c_hi < 0 ? 4 : c_hi); ++c) {
             uint32_t g[32], u[32];
             tmem_ld_32x32b_x32(t_row + c * 32, g);
             tmem_ld_32x32b_x32(t_row + 128 + c * 32, u);
@@ -303,7 +308,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
         __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * BN;
         const float wt = (KIND == GEMM_SCALE) ? args.row_w[row] : 1.0f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = c_lo; c < (c_hi < 0 ? BN / 32 : c_hi); ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_row + c * 32, r);
             tmem_ld_wait();
@@ -403,6 +408,9 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
     const bool gather = (args.gather_idx != nullptr);
     // router filter: the four epilogue warps also read every staged A tile (row norms)
     const bool row_sq = (KIND == GEMM_LOGITS) && args.xsq_f32 != nullptr;
+    // eight epilogue warps (A by TMA, 320 threads); not with the row norms or weight gradients
+    const bool epi8 = args.epi8 && !gather && !row_sq && BMODE != BMODE_WGRAD &&
+                      blockDim.x >= NUM_THREADS_GATHER;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), gather ? 1 + GATHER_THREADS : 1);
@@ -410,7 +418,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 4);
+            mbar_init(tempty_bar(a), epi8 ? 8 : 4);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -604,7 +612,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             volatile int never = 0;
             mbar_wait_bounded(done_bar, 0, &never, args.timeout_ns, args.status, 130 + KIND);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 6 && !epi8) {
         // ---------------- A-row gather: warps 6..9 (layer0 only) ----------------
         // Thread g copies 16-byte chunk (g & 7) of rows (g >> 3) + 16 i, i = 0..7, of every K
         // step. The 8 token ids of its rows are read once per tile and kept in registers
@@ -657,8 +665,15 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             cp_async_wait_all(); // this thread's copies land before the CTA exits
         }
     } else {
-        // ---------------- epilogue: warps 2..5 ----------------
+        // ---------------- epilogue: warps 2..5 (and 6..9 with epi8) ----------------
         const int q = warp & 3; // TMEM lanes 32q .. 32q+31
+        // with epi8, warps 2..5 take the first half of the item's column chunks and warps
+        // 6..9 the second; nep threads meet at the named barriers below
+        const int half = warp >= 6 ? 1 : 0;
+        const int nep = epi8 ? 256 : 128;
+        const int nchunks = (KIND == GEMM_SWIGLU) ? 4 : BN / 32;
+        const int c_lo = epi8 ? half * (nchunks / 2) : 0;
+        const int c_hi = epi8 ? c_lo + nchunks / 2 : -1;
         int it = 0;
         int rs = 0;             // stage ring position (row_sq only)
         uint32_t rph = 0;
@@ -710,7 +725,7 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
             // the TMEM loads below are warp-collective: the whole warp continues or stops;
             // with e4m3 the four epilogue warps also meet at a named barrier per item, so
             // they continue or stop together
-            if (F8 ? !named_bar_and(1, 128, ok) : !__all_sync(0xffffffffu, ok)) break;
+            if (F8 ? !named_bar_and(1, nep, ok) : !__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int row = wgrad ? (e * args.wg_mtiles + mt) * BM + q * 32 + lane
                                   : mt * BM + q * 32 + lane;
@@ -725,16 +740,16 @@ __device__ __forceinline__ void grouped_gemm_cta(const CUtensorMap &tmA, const C
                 // warp rewrites a buffer only after every warp passed the next item's barrier
                 float *sbs = scale_stage + acc * BN;
                 const float *sbg = args.b_scale + (size_t)e * args.b_scale_ld;
-                for (int i = q * 32 + lane; i < BN; i += 128) {
+                for (int i = half * 128 + q * 32 + lane; i < BN; i += nep) {
                     const int col = (KIND == GEMM_SWIGLU)
                                         ? (i < 128 ? nt * 128 + i : args.up_col + nt * 128 + i - 128)
                                         : nt * BN + i;
                     sbs[i] = col < args.b_scale_ld ? sbg[col] : 0.0f;
                 }
-                named_bar_sync(1, 128);
-                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e, sbs);
+                named_bar_sync(1, nep);
+                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e, sbs, c_lo, c_hi);
             } else {
-                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e);
+                epilogue_rows<KIND, F8>(args, t_row, row, nt, ks, e, nullptr, c_lo, c_hi);
             }
             tc_fence_before();
             __syncwarp();

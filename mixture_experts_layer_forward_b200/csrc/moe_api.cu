@@ -562,7 +562,8 @@ cudaError_t launch_gemm_select_f8(const CUtensorMap &ta, const CUtensorMap &tb,
     if (err != cudaSuccess) return err;
     int grid = sm_count();
     if (grid <= 0) grid = 148;
-    const int threads = wide.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    const int threads = (wide.gather_idx != nullptr || wide.epi8) ? gemm::NUM_THREADS_GATHER
+                                                                   : gemm::NUM_THREADS;
     kern<<<grid, threads, smem, st>>>(ta, tb, twn, wide, narrow);
     return cudaGetLastError();
 }
@@ -638,7 +639,8 @@ cudaError_t launch_gemm_select(const CUtensorMap &ta, const CUtensorMap &tb, con
     if (err != cudaSuccess) return err;
     int grid = sm_count();
     if (grid <= 0) grid = 148;
-    const int threads = wide.gather_idx != nullptr ? gemm::NUM_THREADS_GATHER : gemm::NUM_THREADS;
+    const int threads = (wide.gather_idx != nullptr || wide.epi8) ? gemm::NUM_THREADS_GATHER
+                                                                   : gemm::NUM_THREADS;
     kern<<<grid, threads, SELECT_SMEM, st>>>(ta, tb, wide, narrow);
     return cudaGetLastError();
 }
@@ -855,6 +857,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a0.meta = d.meta;
     a0.row_w = nullptr;
     a0.gather_idx = xperm ? nullptr : d.gather_idx;
+    a0.epi8 = xperm && !pair ? 1 : 0; // the idle gather warps join the epilogue
     a0.gather_len = L.pmax;
     a0.gather_src = reinterpret_cast<const __nv_bfloat16 *>(x);
     a0.gather_rows = p->T;
@@ -870,6 +873,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     a0.n_tiles = gated ? (F + 127) / 128 : (F + gemm::BN - 1) / gemm::BN;
     GemmArgs a1 = a0;
     a1.gather_idx = nullptr; // layer1 reads h rows in place
+    a1.epi8 = 0;             // four epilogue warps (eight measured slower on layer1)
     a1.row_w = d.row_w;
     a1.out = reinterpret_cast<__nv_bfloat16 *>(ys);
     a1.ld_out = H;
@@ -1188,11 +1192,12 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     const bool gated = (p->act == MOE_ACT_SWIGLU);
     const int w1_cols = gated ? 2 * F : F;
     CUtensorMap m_x, m_w1, m_h, m_w2, n_w1, n_w2;
-    // the single-CTA kernels gather the x codes inside the kernel: unlike bf16, sorting them
-    // into rows first measured no faster here (the e4m3 epilogue, not the operand feed, sets
-    // the pace) and costs a pass over the rows
-    uint8_t *xq_perm = at<uint8_t>(ws, L.x_perm); // [P_max, H] codes (CTA pairs)
-    if (!make_map_2d_u8(&m_x, xq, (uint64_t)p->T, (uint64_t)H, 1) || // unused: rows are gathered
+    // large batches (single-CTA): the x codes gathered into expert-sorted rows first and read
+    // with TMA, so the four gather warps can join the epilogue (which sets the pace with e4m3)
+    uint8_t *xq_perm = at<uint8_t>(ws, L.x_perm); // [P_max, H] codes in the x_perm region
+    const bool xperm = g_gemm_mode.load() != MOE_GEMM_CTA_PAIR && use_x_perm(p);
+    if (!(xperm ? make_map_2d_u8(&m_x, xq_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM)
+                : make_map_2d_u8(&m_x, xq, (uint64_t)p->T, (uint64_t)H, 1)) ||
         !make_map_3d_u8(&m_w1, W1q, (uint64_t)E, (uint64_t)w1_cols, (uint64_t)H) ||
         !make_map_2d_u8(&m_h, hq, (uint64_t)L.pmax, (uint64_t)F, gemm::BM) ||
         !make_map_3d_u8(&m_w2, W2q, (uint64_t)E, (uint64_t)H, (uint64_t)F) ||
@@ -1210,6 +1215,12 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     if (e == cudaSuccess) e = record(events, n_events, 1, st);
     if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, 0, st);
     if (e == cudaSuccess) e = launch_quant_rows(x, p->T, H, nullptr, xq, sx, st);
+    if (e == cudaSuccess && xperm) { // a row of H codes moves as H / 2 two-byte elements
+        moe_problem ph = *p;
+        ph.H = H / 2;
+        e = launch_gather(&ph, reinterpret_cast<const moe_bf16 *>(xq), d.gather_idx, d.meta,
+                          reinterpret_cast<moe_bf16 *>(xq_perm), st);
+    }
     if (e == cudaSuccess) e = record(events, n_events, 2, st);
 
     GemmArgs a0{};
@@ -1221,7 +1232,9 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     a0.cold_tile = d.cold_tile;
     // the select kernels below: MOE_ORDER_PHASED runs the cold experts' items narrow first
     a0.order = g_order.load() == MOE_ORDER_PHASED ? ORDER_HOT : ORDER_EXPERT;
-    a0.gather_idx = d.gather_idx;
+    a0.gather_idx = xperm ? nullptr : d.gather_idx;
+    a0.scale_idx = xperm ? d.gather_idx : nullptr; // the token of each sorted row's scale
+    a0.epi8 = xperm ? 1 : 0;
     a0.gather_len = L.pmax;
     a0.gather_src = reinterpret_cast<const __nv_bfloat16 *>(xq); // bytes: the codes of x
     a0.gather_rows = p->T;
@@ -1248,6 +1261,7 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
     a1.k_blocks = F / 128;
     a1.a_scale = sh;
     a1.scale_idx = nullptr; // h rows carry their own scales
+    a1.epi8 = 0;            // four epilogue warps (eight measured slower on layer1)
     a1.b_scale = s2;
     a1.b_scale_ld = H;
     // narrow items (every expert single-tile): column blocks of 64 (SwiGLU) or 128 columns
