@@ -107,8 +107,8 @@ typedef struct {
 MOE_API size_t moe_workspace_size(const moe_problem *p);
 
 /* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
- * current GEMM and router modes, assuming 16-byte aligned operands: the
- * router (2, or 3 with the tensor-core filter), the dispatch (3) and the layers (layer0,
+ * current GEMM and router modes, assuming 16-byte aligned operands: the router (2, or 3
+ * with the tensor-core filter), the dispatch (3; 1 for T <= 256) and the layers (layer0,
  * layer1 and the combine: 3; 4 when x is first gathered into expert-sorted rows, which the
  * CTA-pair GEMM always does and the single-CTA GEMM does when T * top_k >= E * 128;
  * 1 with MOE_GEMM_FUSED).

@@ -13,8 +13,10 @@
 
 namespace moe {
 
-constexpr int COMBINE_BATCH = 2; // top-k rows whose loads one thread issues together
-
+// BATCH = top-k rows whose loads one thread issues together: 2 for large grids (more rows
+// in flight per thread costs occupancy there), 8 when the grid is smaller than the GPU and
+// latency, not occupancy, sets the time.
+template <int BATCH>
 __global__ void __launch_bounds__(256)
     combine_kernel(const __nv_bfloat16 *__restrict__ ys, int64_t ys_rows,
                    const int32_t *__restrict__ inv_pos, int T, int H, int k,
@@ -34,23 +36,23 @@ __global__ void __launch_bounds__(256)
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-        // up to COMBINE_BATCH rows per round: all their indices, then all their loads, are
+        // up to BATCH rows per round: all their indices, then all their loads, are
         // issued before the first add, so a thread keeps several loads in flight; the adds
         // still run with j ascending
-        for (int j0 = 0; j0 < k; j0 += COMBINE_BATCH) {
-            int rr[COMBINE_BATCH];
+        for (int j0 = 0; j0 < k; j0 += BATCH) {
+            int rr[BATCH];
 #pragma unroll
-            for (int q = 0; q < COMBINE_BATCH; ++q)
+            for (int q = 0; q < BATCH; ++q)
                 rr[q] = (j0 + q < k) ? inv_pos[(size_t)t * k + j0 + q] : 0;
-            uint4 uu[COMBINE_BATCH];
+            uint4 uu[BATCH];
 #pragma unroll
-            for (int q = 0; q < COMBINE_BATCH; ++q) {
+            for (int q = 0; q < BATCH; ++q) {
                 const bool ok = (j0 + q < k) && rr[q] >= 0 && (int64_t)rr[q] < ys_rows;
                 uu[q] = ok ? *reinterpret_cast<const uint4 *>(ys + (size_t)rr[q] * H + (size_t)v * 8)
                            : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int q = 0; q < COMBINE_BATCH; ++q) {
+            for (int q = 0; q < BATCH; ++q) {
                 if (j0 + q >= k) break;
                 if (rr[q] < 0 || (int64_t)rr[q] >= ys_rows) {
                     record_status(status, DEV_BAD_INDEX, 3);

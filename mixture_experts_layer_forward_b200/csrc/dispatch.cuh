@@ -11,6 +11,8 @@
 //                           token among the chunk's tokens routed to e (a popcount over a
 //                           per-expert token bitmap, so no ordering depends on atomics)
 //   gather_rows_kernel      optional materialised x_perm[r] = x[gather_idx[r]]
+// Batches of at most one chunk (T <= 256: decode-sized) take dispatch_small_kernel instead,
+// the three steps in one block, with the same outputs.
 // Counts and bitmaps are built with shared-memory atomics whose result does not depend on
 // their order, so every output is bit-reproducible.
 #pragma once
@@ -91,35 +93,37 @@ __device__ __forceinline__ int block_inclusive_scan_1024(int v, int *warp_sums)
     return v;
 }
 
-// One block of 1024 threads; thread e owns expert e (E <= 1024).
-//   chunk_counts [nchunk][E] is rewritten in place into each chunk's base row within e.
-__global__ void __launch_bounds__(1024)
-    dispatch_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk, int E,
-                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                         int32_t *__restrict__ padded_offsets, int32_t *__restrict__ tile_off,
-                         int32_t *__restrict__ tile_expert, int32_t *__restrict__ ptile_off,
-                         int32_t *__restrict__ ptile_expert, DispatchMeta *meta,
-                         int32_t *__restrict__ gather_idx, float *__restrict__ row_w,
-                         int64_t padded_rows_max, int *__restrict__ ready, int n_ready,
-                         int32_t *__restrict__ hot_off, int32_t *__restrict__ hot_tile_expert,
-                         int32_t *__restrict__ cold_tile, int32_t *__restrict__ active_list)
+// Outputs of the scan step (all device pointers; the optional ones may be null).
+struct ScanOut {
+    int32_t *counts, *offsets, *padded_offsets, *tile_off, *tile_expert;
+    int32_t *ptile_off, *ptile_expert;
+    DispatchMeta *meta;
+    int32_t *gather_idx;
+    float *row_w;
+    int64_t padded_rows_max;
+    int *ready;
+    int n_ready;
+    int32_t *hot_off, *hot_tile_expert, *cold_tile, *active_list;
+};
+
+// Everything derived from the per-expert row counts, by one block of 1024 threads in which
+// thread e owns expert e (c = its routed rows; E <= 1024). s_poff[0..E] receives the padded
+// row offsets, s_cnt[0..E-1] the counts. Ends with a block barrier.
+__device__ __forceinline__ void dispatch_scan_body(int c, int E, const ScanOut &o, int *warp_sums,
+                                                   int *s_poff, int *s_cnt)
 {
     // the fused layer kernel's tile-level ready counters start from zero on every call
-    for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
-    __shared__ int warp_sums[32];
-    __shared__ int s_poff[1025];
+    for (int i = threadIdx.x; i < o.n_ready; i += blockDim.x) o.ready[i] = 0;
     const int e = threadIdx.x;
-    int c = 0;
-    if (e < E) {
-        int run = 0;
-        for (int ch = 0; ch < nchunk; ++ch) {
-            const int v = chunk_counts[(size_t)ch * E + e];
-            chunk_counts[(size_t)ch * E + e] = run;
-            run += v;
-        }
-        c = run;
-        if (counts != nullptr) counts[e] = c;
-    }
+    int32_t *const counts = o.counts, *const offsets = o.offsets;
+    int32_t *const padded_offsets = o.padded_offsets, *const tile_off = o.tile_off;
+    int32_t *const tile_expert = o.tile_expert, *const ptile_off = o.ptile_off;
+    int32_t *const ptile_expert = o.ptile_expert, *const hot_off = o.hot_off;
+    int32_t *const hot_tile_expert = o.hot_tile_expert, *const cold_tile = o.cold_tile;
+    int32_t *const active_list = o.active_list, *const gather_idx = o.gather_idx;
+    float *const row_w = o.row_w;
+    DispatchMeta *const meta = o.meta;
+    if (e < E && counts != nullptr) counts[e] = c;
     const int ntile = (c + M_TILE - 1) / M_TILE;
     const int inc_c = block_inclusive_scan_1024(c, warp_sums);
     const int inc_t = block_inclusive_scan_1024(ntile, warp_sums);
@@ -167,19 +171,76 @@ __global__ void __launch_bounds__(1024)
             s_poff[E] = poff_next;
         }
     }
+    if (e < E) s_cnt[e] = c;
     __syncthreads();
-    // pad rows of each expert, then everything past P_pad: gather_idx = -1, weight 0
-    if (e < E) {
-        const int first_pad = s_poff[e] + c;
-        const int end = s_poff[e] + ntile * M_TILE;
-        for (int r = first_pad; r < end; ++r) {
+    // pad rows of each expert (one warp per expert, lanes on consecutive rows), then
+    // everything past P_pad: gather_idx = -1, weight 0
+    for (int ex = threadIdx.x >> 5; ex < E; ex += blockDim.x >> 5) {
+        const int end = s_poff[ex + 1];
+        for (int r = s_poff[ex] + s_cnt[ex] + (threadIdx.x & 31); r < end; r += 32) {
             gather_idx[r] = -1;
             if (row_w != nullptr) row_w[r] = 0.0f;
         }
     }
-    for (int64_t r = (int64_t)s_poff[E] + threadIdx.x; r < padded_rows_max; r += blockDim.x) {
+    for (int64_t r = (int64_t)s_poff[E] + threadIdx.x; r < o.padded_rows_max; r += blockDim.x) {
         gather_idx[r] = -1;
         if (row_w != nullptr) row_w[r] = 0.0f;
+    }
+    __syncthreads();
+}
+
+// One block of 1024 threads; thread e owns expert e (E <= 1024).
+//   chunk_counts [nchunk][E] is rewritten in place into each chunk's base row within e.
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk, int E, ScanOut o)
+{
+    __shared__ int warp_sums[32];
+    __shared__ int s_poff[1025];
+    __shared__ int s_cnt[1024];
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < E) {
+        int run = 0;
+        // eight chunks' counts loaded before any is rewritten: eight loads in flight
+        for (int ch0 = 0; ch0 < nchunk; ch0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                v[q] = (ch0 + q < nchunk) ? chunk_counts[(size_t)(ch0 + q) * E + e] : 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (ch0 + q < nchunk) chunk_counts[(size_t)(ch0 + q) * E + e] = run;
+                run += v[q];
+            }
+        }
+        c = run;
+    }
+    dispatch_scan_body(c, E, o, warp_sums, s_poff, s_cnt);
+}
+
+// Rows of token t's k pairs: padded_offsets[e] + chunk_base[e] (null: 0) + the rank of t
+// among its chunk's tokens routed to e (tl = t's position in the chunk; bits = the chunk's
+// token bitmap per expert).
+__device__ __forceinline__ void dispatch_place_token(
+    const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w, int t, int tl, int E,
+    int k, const uint32_t *bits, const int32_t *padded_offsets, const int32_t *chunk_base,
+    int32_t *__restrict__ gather_idx, int32_t *__restrict__ inv_pos, float *__restrict__ row_w)
+{
+    const int word = tl >> 5;
+    const uint32_t bit = 1u << (tl & 31);
+    for (int j = 0; j < k; ++j) {
+        const int e = topk_idx[(size_t)t * k + j];
+        if (e < 0 || e >= E) {
+            inv_pos[(size_t)t * k + j] = -1;
+            continue;
+        }
+        const uint32_t *b = bits + e * DISPATCH_WORDS;
+        int rank = __popc(b[word] & (bit - 1u));
+        for (int w = 0; w < word; ++w) rank += __popc(b[w]);
+        const int r = padded_offsets[e] + (chunk_base != nullptr ? chunk_base[e] : 0) + rank;
+        gather_idx[r] = t;
+        inv_pos[(size_t)t * k + j] = r;
+        if (row_w != nullptr) row_w[r] = topk_w[(size_t)t * k + j];
     }
 }
 
@@ -206,20 +267,52 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     }
     __syncthreads();
     if (t >= T) return;
-    for (int j = 0; j < k; ++j) {
-        const int e = topk_idx[(size_t)t * k + j];
-        if (e < 0 || e >= E) {
-            inv_pos[(size_t)t * k + j] = -1;
-            continue;
-        }
-        const uint32_t *b = bits + e * DISPATCH_WORDS;
-        int rank = __popc(b[word] & (bit - 1u));
-        for (int w = 0; w < word; ++w) rank += __popc(b[w]);
-        const int r = padded_offsets[e] + chunk_base[(size_t)blockIdx.x * E + e] + rank;
-        gather_idx[r] = t;
-        inv_pos[(size_t)t * k + j] = r;
-        if (row_w != nullptr) row_w[r] = topk_w[(size_t)t * k + j];
+    dispatch_place_token(topk_idx, topk_w, t, tl, E, k, bits, padded_offsets,
+                         chunk_base + (size_t)blockIdx.x * E, gather_idx, inv_pos, row_w);
+}
+
+// T <= DISPATCH_CHUNK: count, scan and place in one block of 1024 threads (thread t < T owns
+// token t in the count and place steps, thread e expert e in the scan), with the outputs of
+// the three-kernel path. Dynamic shared memory: E * (DISPATCH_WORDS + 1) uint32.
+__global__ void __launch_bounds__(1024)
+    dispatch_small_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
+                          int T, int E, int k, ScanOut o, int32_t *__restrict__ inv_pos,
+                          int *status, int clear_status)
+{
+    extern __shared__ uint32_t sm_words[];
+    uint32_t *bits = sm_words;                                        // [E][DISPATCH_WORDS]
+    int *cnt = reinterpret_cast<int *>(sm_words + E * DISPATCH_WORDS); // [E]
+    __shared__ int warp_sums[32];
+    __shared__ int s_poff[1025];
+    __shared__ int s_cnt[1024];
+    if (clear_status && status != nullptr && threadIdx.x == 0) {
+        status[0] = DEV_OK;
+        status[1] = 0;
     }
+    for (int i = threadIdx.x; i < E * DISPATCH_WORDS; i += blockDim.x) bits[i] = 0u;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    const int t = threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(size_t)t * k + j];
+            if (e >= 0 && e < E) {
+                atomicAdd(&cnt[e], 1);
+                atomicOr(&bits[e * DISPATCH_WORDS + (t >> 5)], 1u << (t & 31));
+            } else {
+                record_status(status, DEV_BAD_INDEX, 1);
+            }
+            if (k <= 16) {
+                for (int j2 = 0; j2 < j; ++j2)
+                    if (topk_idx[(size_t)t * k + j2] == e) record_status(status, DEV_BAD_INDEX, 2);
+            }
+        }
+    }
+    __syncthreads();
+    dispatch_scan_body(threadIdx.x < E ? cnt[threadIdx.x] : 0, E, o, warp_sums, s_poff, s_cnt);
+    if (t < T)
+        dispatch_place_token(topk_idx, topk_w, t, t, E, k, bits, s_poff, nullptr, o.gather_idx,
+                             inv_pos, o.row_w);
 }
 
 // x_perm[r][:] = x[gather_idx[r]][:] (zeros on pad rows), for r < P_pad. One warp per row.

@@ -486,18 +486,43 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
 {
     const int T = p->T, E = p->E, k = p->top_k;
     const int nchunk = L.nchunk;
+    ScanOut so{};
+    so.counts = o.counts;
+    so.offsets = o.offsets;
+    so.padded_offsets = o.poff;
+    so.tile_off = o.tile_off;
+    so.tile_expert = o.tile_expert;
+    so.ptile_off = o.ptile_off;
+    so.ptile_expert = o.ptile_expert;
+    so.meta = o.meta;
+    so.gather_idx = o.gather_idx;
+    so.row_w = o.row_w;
+    so.padded_rows_max = L.pmax;
+    so.ready = o.ready;
+    so.n_ready = o.ready ? o.n_ready : 0;
+    so.hot_off = o.hot_off;
+    so.hot_tile_expert = o.hot_tile_expert;
+    so.cold_tile = o.cold_tile;
+    so.active_list = o.active_list;
+    if (nchunk == 1) { // one chunk of tokens: the three steps in one block
+        dispatch_small_kernel<<<1, 1024, (size_t)E * (DISPATCH_WORDS + 1) * 4, st>>>(
+            topk_idx, topk_w, T, E, k, so, o.inv_pos, status, clear_status);
+        return cudaGetLastError();
+    }
+    cudaError_t err = cudaSuccess;
+    if (clear_status && status != nullptr && nchunk > 1) {
+        // cleared before any block can record a bad id (blocks of one launch are unordered)
+        err = cudaMemsetAsync(status, 0, 8, st);
+        if (err != cudaSuccess) return err;
+        clear_status = 0;
+    }
     if (nchunk > 0) {
         dispatch_count_kernel<<<nchunk, DISPATCH_CHUNK, E * sizeof(int), st>>>(
             topk_idx, T, E, k, o.chunk, status, clear_status);
     }
-    cudaError_t err = cudaGetLastError();
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, o.counts, o.offsets, o.poff,
-                                             o.tile_off, o.tile_expert, o.ptile_off,
-                                             o.ptile_expert, o.meta, o.gather_idx, o.row_w,
-                                             L.pmax, o.ready, o.ready ? o.n_ready : 0,
-                                             o.hot_off, o.hot_tile_expert, o.cold_tile,
-                                             o.active_list);
+    dispatch_scan_kernel<<<1, 1024, 0, st>>>(o.chunk, nchunk, E, so);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
@@ -526,11 +551,12 @@ cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_
     const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    combine_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows,
-                                               inv_pos, p->T, p->H, p->top_k,
-                                               reinterpret_cast<__nv_bfloat16 *>(out), status,
-                                               clear_status,
-                                               reinterpret_cast<const __nv_bfloat16 *>(ys_shared));
+    // a grid that does not fill the GPU twice over: every thread issues all k row loads at once
+    auto kern = (blocks < 2 * cap / 16 && p->top_k > 2) ? combine_kernel<8> : combine_kernel<2>;
+    kern<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows, inv_pos,
+                                      p->T, p->H, p->top_k, reinterpret_cast<__nv_bfloat16 *>(out),
+                                      status, clear_status,
+                                      reinterpret_cast<const __nv_bfloat16 *>(ys_shared));
     return cudaGetLastError();
 }
 
@@ -1317,7 +1343,8 @@ int moe_forward_launches(const moe_problem *p)
     if (check_problem(p) != MOE_OK) return -1;
     if (p->T == 0) return 0;
     const int route = route_uses_filter(p) ? 3 : 2; // filter: prep, GEMM, exact; else logits, top-k
-    const int dispatch = 3;                          // count, scan, place
+    // count, scan, place; one block for a single chunk of tokens
+    const int dispatch = p->T <= DISPATCH_CHUNK ? 1 : 3;
     const int mode = g_gemm_mode.load();
     // layer0, layer1, combine; + the x_perm gather for CTA pairs and large batches
     const int layers = mode == MOE_GEMM_FUSED                              ? 1

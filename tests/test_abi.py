@@ -102,17 +102,17 @@ def test_forward_launch_count_follows_the_modes(lib):
     prev_g = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
     prev_o = moe.moe_set_work_order(moe.ORDER_EXPERT)
     try:
-        # router 2 (3 with the filter) + dispatch 3 + [x gather] + layer0, layer1, combine;
-        # the bench layers gather x into sorted rows (T * k >= 128 E), decode does not
+        # router 2 (3 with the filter) + dispatch 3 (1 for T <= 256) + [x gather] + layer0,
+        # layer1, combine; the bench layers gather x into sorted rows (T * k >= 128 E)
         assert moe.moe_forward_launches(mixtral) == 9   # E = 8: sequential router
         assert moe.moe_forward_launches(qwen2) == 10    # T*E >= 2^16: filter router
-        assert moe.moe_forward_launches(decode) == 8    # T*E < 2^16: sequential, no gather
+        assert moe.moe_forward_launches(decode) == 6    # T*E < 2^16: sequential, no gather
         phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
         assert moe.moe_forward_launches(phi35) == 10    # E = 16: filter router
         moe.moe_set_router_mode(moe.ROUTER_FILTER)
-        assert moe.moe_forward_launches(decode) == 9
+        assert moe.moe_forward_launches(decode) == 7
         assert moe.moe_forward_launches(mixtral) == 10  # forced: E = 8 qualifies
-        assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 8  # E % 8
+        assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
         assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
@@ -121,8 +121,11 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(qwen2) == 6
         moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)        # gathers x; no narrow launches
         assert moe.moe_forward_launches(qwen2) == 9
-        assert moe.moe_forward_launches(decode) == 9
+        assert moe.moe_forward_launches(decode) == 7
         assert moe.moe_forward_launches(moe.Problem.make(0, 128, 128, 8, 2)) == 0
+        moe.moe_set_gemm_mode(moe.GEMM_AUTO)
+        assert moe.moe_forward_launches(moe.Problem.make(256, 128, 128, 8, 2)) == 6  # one chunk
+        assert moe.moe_forward_launches(moe.Problem.make(257, 128, 128, 8, 2)) == 8  # two
         assert moe.moe_forward_launches(moe.Problem.make(4, 100, 128, 8, 2)) == -1  # H % 64
     finally:
         moe.moe_set_router_mode(prev_r)

@@ -242,8 +242,10 @@ def distinct_idx(T, E, k, seed, skew=False):
     return np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
 
 
+# T <= 256 takes the one-block dispatch kernel, larger T the three-kernel path
 DISPATCH_CASES = [(300, 8, 2, False), (1000, 64, 8, False), (513, 256, 8, True), (1, 4, 1, False),
-                  (128, 1, 1, False), (40, 8, 8, False), (2048, 1024, 4, True), (77, 3, 3, False)]
+                  (128, 1, 1, False), (40, 8, 8, False), (2048, 1024, 4, True), (77, 3, 3, False),
+                  (256, 1024, 8, True), (256, 8, 2, False), (257, 8, 2, False), (64, 256, 8, True)]
 
 
 @pytest.mark.parametrize("T,E,k,skew", DISPATCH_CASES)
@@ -278,12 +280,13 @@ def test_dispatch_bit_exact(T, E, k, skew):
     assert torch.equal(xp, want)
 
 
-def test_dispatch_reports_bad_expert_id():
-    T, E, k = 50, 8, 2
+@pytest.mark.parametrize("T", [50, 700])
+def test_dispatch_reports_bad_expert_id(T):
+    E, k = 8, 2
     p = moe.Problem.make(T, 64, 64, E, k)
     ws = alloc_ws(p)
     idx = torch.from_numpy(distinct_idx(T, E, k, 1)).cuda()
-    idx[7, 1] = E + 3
+    idx[T - 7, 1] = E + 3
     pmax = moe.moe_padded_rows_max(p)
     bufs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, E + 1, pmax)]
     inv = torch.empty(T, k, dtype=torch.int32, device="cuda")
