@@ -479,12 +479,9 @@ def run_ours(args):
                            "peak_source": f"{peak_src} bf16 {regime}" + (" x 2" if args.fp8 else "")},
         "roofline": roofline,
         "stage_ms": stage_ms,
-        # FP8: router, 3 dispatch kernels (1 for T <= 256), x quantisation, [the gather of the
-        # x codes into sorted rows when T * k >= 128 E], layer0, h quantisation, layer1, combine
-        "gpu_launches": ((3 if moe.moe_route_uses_filter(p) else 2) +
-                         (6 if cfg.T <= 256 else 8) +
-                         (1 if cfg.T * cfg.k >= 128 * cfg.E else 0) if args.fp8 else
-                         moe.moe_forward_launches(p)) * K,
+        # FP8: the bf16 path's launches (router, dispatch, [the gather into sorted rows],
+        # layer0, layer1, combine) plus the x and h quantisers
+        "gpu_launches": (moe.moe_forward_launches(p) + (2 if args.fp8 else 0)) * K,
         "clocks": clocks,
         "e2e": e2e,
         "cold_l2": {"ms_per_step": cold_ms, "steps": n_cold,

@@ -1375,7 +1375,8 @@ moe_status moe_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg
         return MOE_ERR_INVALID_ARG;
     const Layout L = make_layout(p);
     if (ws_bytes < L.end_route) return MOE_ERR_WORKSPACE;
-    if (!aligned16(x) || !aligned16(ws) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(topk_w))
+    if (!aligned16(x) || !aligned16(Wg) || !aligned16(ws) || !aligned4(bias) || !aligned4(topk_idx) ||
+        !aligned4(topk_w))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = at<int>(ws, L.status);
@@ -1394,7 +1395,7 @@ moe_status moe_route_noalloc(const moe_problem *p, const moe_bf16 *x, const moe_
     if (p->T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr))
         return MOE_ERR_INVALID_ARG;
     if ((int64_t)p->T * p->E > (int64_t)MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_UNSUPPORTED;
-    if (!aligned16(x) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(topk_w))
+    if (!aligned16(x) || !aligned16(Wg) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(topk_w))
         return MOE_ERR_INVALID_ARG;
     if (p->T == 0) return MOE_OK;
     float *logits = route_noalloc_scratch();

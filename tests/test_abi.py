@@ -78,6 +78,11 @@ def test_host_side_argument_checks(lib):
     args = [fake] * 6 + [None, None]
     assert lib.moe_forward(ctypes.byref(good), *args, fake, 16, None) == -3
     assert lib.moe_route(ctypes.byref(good), fake, fake, None, fake, fake, fake, 16, None) == -3
+    # a gate matrix off the 16-byte boundary is rejected before any launch
+    off = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.moe_route(ctypes.byref(good), fake, off, None, fake, fake, fake,
+                         moe.moe_workspace_size(good), None) == -1
+    assert lib.moe_route_noalloc(ctypes.byref(good), fake, off, None, fake, fake, None) == -1
     assert lib.moe_get_device_status(None, None) == -1
     assert lib.moe_status_string(-5) == b"MOE_ERR_DEVICE_TIMEOUT"
 
