@@ -224,16 +224,16 @@ bool aligned4(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) 
 
 int sm_count()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64]; // per device; 0 = not yet queried (static: zeroed)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     if (dev < 0 || dev >= 64) return 0;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -631,10 +631,12 @@ cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     // persistent grid: as many CTA pairs as can be resident at once (one CTA per SM)
-    static int cache[64][3] = {{0}}; // the e4m3 form has the same block size and shared memory
+    // per device and kind (the e4m3 form has the same block size and shared memory); 0 = not
+    // yet queried
+    static std::atomic<int> cache[64][3];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int &pairs = cache[dev][KIND];
+    int pairs = cache[dev][KIND].load(std::memory_order_relaxed);
     if (pairs == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
@@ -644,6 +646,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const
         err = cudaOccupancyMaxActiveClusters(&n, (const void *)kern, &cfg);
         if (err != cudaSuccess) return err;
         pairs = n > 0 ? n : 1;
+        cache[dev][KIND].store(pairs, std::memory_order_relaxed);
     }
     int npairs = pairs;
     if (npairs > max_work) npairs = max_work;
