@@ -186,3 +186,65 @@ def test_backward_workspace_and_argument_checks(lib):
     assert moe.moe_backward_workspace_size(p) > moe.moe_workspace_size(p)
     assert moe.moe_backward_workspace_size(moe.Problem.make(300, 256, 192, 16, 2)) == 0   # F % 128
     assert lib.moe_backward(ctypes.byref(p), *([None] * 12), 0, None) == -1
+
+
+def _header_prototypes():
+    text = "\n".join(h.read_text() for h in sorted((ROOT / "include").glob("*.h")))
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"MOE_API\s+([^;(]*?)\b(moe_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S):
+        params = " ".join(m.group(3).split())
+        plist = [] if params in ("", "void") else [q.strip() for q in params.split(",")]
+        protos[m.group(2)] = (" ".join(m.group(1).split()), plist)
+    return protos
+
+
+def _ctype_kind(c_decl):
+    """Category of a C parameter or return type: pointer, size, i64 or i32."""
+    if "*" in c_decl:
+        return "pointer"
+    words = c_decl.replace("const ", "").split()
+    base = words[0]
+    if base == "size_t":
+        return "size"
+    if base == "int64_t":
+        return "i64"
+    if base in ("int", "int32_t", "moe_status"):
+        return "i32"
+    raise AssertionError(f"unexpected C type {c_decl!r}")
+
+
+def _ctypes_kind(t):
+    if t is ctypes.c_void_p or t is ctypes.c_char_p or (
+            isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    if t is ctypes.c_size_t:
+        return "size"
+    if t is ctypes.c_int64:
+        return "i64"
+    if t is ctypes.c_int:
+        return "i32"
+    raise AssertionError(f"unexpected ctypes type {t!r}")
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every prototype in include/ has a ctypes signature in the binding with the same number
+    of arguments and the same kind (pointer, size_t, int64, int) of each argument and of the
+    result: a parameter added on one side only would otherwise shift every later argument."""
+    protos = _header_prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, params) in protos.items():
+        f = getattr(lib, name)
+        assert f.argtypes is not None, f"{name}: no argtypes in the binding"
+        assert len(f.argtypes) == len(params), (name, len(f.argtypes), len(params))
+        for i, (c_decl, t) in enumerate(zip(params, f.argtypes)):
+            assert _ctype_kind(c_decl) == _ctypes_kind(t), (name, i, c_decl, t)
+        assert _ctype_kind(ret) == _ctypes_kind(f.restype), (name, ret, f.restype)
+
+
+def test_every_entry_point_has_a_python_function():
+    """The package exposes each C entry point under its own name (moe_status_string is used
+    inside the binding's error messages)."""
+    for name in declared_functions():
+        if name != "moe_status_string":
+            assert callable(getattr(moe, name, None)), name
