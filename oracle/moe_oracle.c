@@ -559,8 +559,8 @@ int oracle_shared_tokens(int T, int H, int Fs, const uint16_t *x, const uint16_t
  *     r is not finite (amax zero or tiny) takes r = s = 1;
  *   - GEMMs: exact products of the decoded codes, summed, times s_row * s_col;
  *   - between the layers h is held in bf16, as in the bf16 path, and then quantised per row.
- *     This one rounding step is parity unpinned: its effect (one bf16 rounding of h before
- *     the row quantisation) is far below what the pins resolve; every other step is pinned.
+ *     A bf16 rounding can only move a value onto an e4m3 rounding midpoint, never across
+ *     one, so it shows in the codes only through ties; the pins include such a tie.
  * ------------------------------------------------------------------------------------- */
 
 double oracle_e4m3_decode(uint8_t c)

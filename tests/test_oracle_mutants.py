@@ -65,6 +65,7 @@ MUTANTS = [
     ("fp8_w1_scale_of_column_0", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)sx * (double)s1[0];"),
     ("fp8_gate_up_swapped", "silu(z[f]) * z[f + F]", "silu(z[f + F]) * z[f]"),
     ("fp8_token_path_drops_gate", "o[n] += y[n] * w[j];", "o[n] += y[n];"),
+    ("fp8_h_not_rounded_to_bf16", "hf[f] = (float)oracle_round_to_bf16(a);", "hf[f] = (float)a;"),
     ("bwd_silu_derivative_drops_term", "const double dg = da[f] * u * s * (1.0 + g * (1.0 - s));",
      "const double dg = da[f] * u * s;"),
     ("bwd_up_gradient_uses_up", "const double du = da[f] * g * s;", "const double du = da[f] * u * s;"),

@@ -494,6 +494,31 @@ def _fp8_layer(seed, T, H, F, E, k, act):
     return x, Wg, synth.bf16_bits(W1.to(torch.bfloat16)), synth.bf16_bits(W2.to(torch.bfloat16))
 
 
+def test_fp8_h_is_held_in_bf16_before_its_row_quantisation(oracle_lib):
+    """Hand-worked: one token x = (1, 1, 1), one expert, identity activation, H = 3, F = 2.
+    x codes 448 each, s_x = fl32(1/448). W1 column 0 = (448, 0, 0): codes (448, 0, 0),
+    s = 1, so z0 = 448^2 * s_x = 448 (1 + 4.5e-8). W1 column 1 = (1, 1/16, 146 * 2^-22):
+    r = 448, codes (448, 28, 2^-6) (146 * 2^-22 * 448 = 0.01559 rounds to the smallest
+    normal), s = fl32(1/448), so z1 = 476.015625 / 448 (1 + 9e-8) = 1.0625349.
+    h in bf16: (448, 1.0625), so amax = 448, r_h = s_h = 1 and 1.0625 is a tie between the
+    e4m3 values 1 and 1.125 that goes to the even code, 1. W2 column 0 = (0, 1) picks h1:
+    out[0] = 1 * 448 * fl32(1/448) = 1 (1 + 4.5e-8). Held in fp32 instead, amax would be
+    fl32(z0) > 448, r_h < 1 and h1 * r_h = 1.0625349 would take the code 1.125. W2 column 1 =
+    (1, 0) picks h0: out[1] = 448 (1 + 4.5e-8); column 2 is zero (scale 1, codes 0)."""
+    x = bf16([[1, 1, 1]])
+    Wg = bf16([[1], [0], [0]])
+    W1 = bf16([[[448, 1], [0, 1 / 16], [0, 146 * 2.0 ** -22]]])      # [E, H, F]
+    W2 = bf16([[[0, 1, 0], [1, 0, 0]]])                              # [E, F, H]
+    W1q, s1 = oracle.quant_cols_fp8(W1, lib=oracle_lib)
+    W2q, s2 = oracle.quant_cols_fp8(W2, lib=oracle_lib)
+    assert list(W1q[0, 1]) == [0x7E, 0x5E, 0x08]                     # 448, 28, 2^-6
+    out, idx, w = oracle.moe_tokens_fp8(x, Wg, None, W1q, s1, W2q, s2, 1, np.arange(1),
+                                        act=oracle.ACT_IDENTITY, lib=oracle_lib)
+    assert idx[0, 0] == 0 and w[0, 0] == 1.0
+    assert abs(out[0, 0] - 1.0) < 1e-6, out[0, 0]                    # not 1.125
+    assert abs(out[0, 1] - 448.0) < 1e-3 and out[0, 2] == 0.0
+
+
 @pytest.mark.parametrize("act", [oracle.ACT_SWIGLU, oracle.ACT_RELU])
 def test_fp8_layer_is_close_to_bf16_layer(oracle_lib, act):
     """The e4m3 layer equals the bf16 layer up to the quantisation error: each code is within
