@@ -263,16 +263,22 @@ def test_permute_then_unpermute_is_identity(oracle_lib):
 # ------------------------------------------------------------------------------------
 
 def _np_act(act, z):
+    """The activations from torch's library implementations (fp64), not retyped here."""
+    zt = torch.from_numpy(np.ascontiguousarray(z, dtype=np.float64))
     if act == oracle.ACT_GELU_TANH:
-        return 0.5 * z * (1 + np.tanh(math.sqrt(2 / math.pi) * (z + 0.044715 * z**3)))
+        return torch.nn.functional.gelu(zt, approximate="tanh").numpy()
     if act == oracle.ACT_RELU:
-        return np.maximum(z, 0)
+        return torch.relu(zt).numpy()
     return z
 
 
 def _np_ffn(x64, W1e, W2e, act, F):
     z = x64 @ W1e
-    a = z[:, :F] / (1 + np.exp(-z[:, :F])) * z[:, F:] if act == oracle.ACT_SWIGLU else _np_act(act, z)
+    if act == oracle.ACT_SWIGLU:
+        g = torch.from_numpy(np.ascontiguousarray(z[:, :F]))
+        a = torch.nn.functional.silu(g).numpy() * z[:, F:]
+    else:
+        a = _np_act(act, z)
     return a @ W2e
 
 
