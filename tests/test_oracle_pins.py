@@ -433,6 +433,9 @@ def test_e4m3_decode_known_codes(oracle_lib):
     assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and got[0xB8] == -1.0
     # the positive finite codes are strictly increasing
     assert np.all(np.diff(got[:0x7F]) > 0)
+    # and torch's float8_e4m3fn type reads every finite code the same way
+    lib_vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    np.testing.assert_array_equal(got[ok], lib_vals.numpy()[ok])
 
 
 def test_e4m3_encode_is_nearest_ties_to_even(oracle_lib):
@@ -462,6 +465,10 @@ def test_e4m3_encode_is_nearest_ties_to_even(oracle_lib):
     code = np.where(a > 448.0, 0x7E, code)
     want = (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
     np.testing.assert_array_equal(got, want)
+    # torch's float32 -> float8_e4m3fn conversion (nearest, ties to even) agrees in range
+    inr = np.abs(v) <= 448.0
+    lib_codes = torch.from_numpy(v[inr]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(got[inr], lib_codes)
     specials = np.array([np.inf, -np.inf, np.nan, -0.0, 0.0], np.float32)
     sg = oracle.e4m3_encode(specials, lib=oracle_lib)
     assert list(sg[:2]) == [0x7E, 0xFE] and (sg[2] & 0x7F) == 0x7F and list(sg[3:]) == [0x80, 0x00]
