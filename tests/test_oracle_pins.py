@@ -78,6 +78,16 @@ def test_round_to_bf16_hand_cases(oracle_lib):
     }
     for v, want in cases.items():
         assert oracle.round_to_bf16(v, lib=oracle_lib) == want, v
+    # fp32 inputs: torch's float32 -> bfloat16 conversion (one nearest-even rounding) agrees,
+    # on random values and on the fp32 neighbours of bf16 midpoints
+    rng = np.random.default_rng(4)
+    r = np.ldexp(rng.uniform(1, 2, 3000), rng.integers(-60, 60, 3000)) * rng.choice([-1, 1], 3000)
+    mids = np.ldexp(2.0 * np.arange(128, 256) + 1, -8).astype(np.float32)  # (2m+1)/256 in [1, 2)
+    v32 = np.concatenate([r.astype(np.float32), mids, np.nextafter(mids, np.float32(2)),
+                          np.nextafter(mids, np.float32(0))])
+    lib_vals = torch.from_numpy(v32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.round_to_bf16(float(v), lib=oracle_lib) for v in v32])
+    np.testing.assert_array_equal(got, lib_vals)
 
 
 # ------------------------------------------------------------------------------------
