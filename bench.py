@@ -489,7 +489,8 @@ def run_ours(args):
         "routing": routing,
     }
 
-    if rank == 0 and not args.no_cpu_baseline and not args.fp8:
+    # the CPU oracle baseline: rank 0 of a one-GPU run only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         hin = host_inputs(inp)
         v, n_tok, t, threads = cpu_oracle_sample(cfg, hin, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
