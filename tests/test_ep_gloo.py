@@ -1,6 +1,6 @@
-"""Expert parallelism on CPU (gloo, world size 2): the exchange plan of ep.ep_forward.
+"""Expert parallelism on CPU (gloo, world sizes 2 and 4): the exchange plan of ep.ep_forward.
 
-Each rank routes its own tokens with the oracle's router, keeps half of the experts, and
+Each rank routes its own tokens with the oracle's router, keeps E / world of the experts, and
 runs the same row function on the rows it receives; the result must equal, bit for bit,
 the same row function applied to its own routed pairs with all experts at hand and combined
 in the same order: the exchange only moves rows. The GPU form of the two steps
@@ -75,11 +75,12 @@ def _worker(rank, world, port, tmpdir, skewed):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("skewed", [False, True], ids=["balanced", "one_rank_idle"])
-def test_ep_exchange_matches_local_compute(tmp_path, skewed):
-    port = 29600 + (11 if skewed else 0) + os.getpid() % 97
-    mp.spawn(_worker, args=(2, port, str(tmp_path), skewed), nprocs=2, join=True)
-    assert all(os.path.exists(tmp_path / f"ok{r}") for r in range(2))
+@pytest.mark.parametrize("world,skewed", [(2, False), (2, True), (4, False)],
+                         ids=["balanced", "one_rank_idle", "four_ranks"])
+def test_ep_exchange_matches_local_compute(tmp_path, world, skewed):
+    port = 29600 + (11 if skewed else 0) + (23 if world == 4 else 0) + os.getpid() % 97
+    mp.spawn(_worker, args=(world, port, str(tmp_path), skewed), nprocs=world, join=True)
+    assert all(os.path.exists(tmp_path / f"ok{r}") for r in range(world))
 
 
 def test_dispatch_plan_is_stable_and_local():
