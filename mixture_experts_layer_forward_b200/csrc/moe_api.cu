@@ -719,7 +719,12 @@ float *route_noalloc_scratch()
     std::lock_guard<std::mutex> lock(mu);
     if (cache[dev] == nullptr) {
         void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_route_noalloc_logits) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_route_noalloc_logits) != cudaSuccess) {
+            // consume the failure so that it is not reported again by the next launch check
+            // of this host thread (the caller returns MOE_ERR_CUDA for it)
+            (void)cudaGetLastError();
+            return nullptr;
+        }
         cache[dev] = static_cast<float *>(ptr);
     }
     return cache[dev];

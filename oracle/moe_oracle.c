@@ -18,7 +18,7 @@
  *     experts.                                         -> oracle_dispatch
  *   - §2.2.2: routing is decided at run time, so the per-expert row counts vary.
  *
- * Readings taken where the pages are silent (each one is listed in the design notes):
+ * Readings taken where the pages are silent:
  *   - router: logits = x . W_g (+ an optional per-expert bias), W_g stored [H, E];
  *   - selection: the k largest logits, ties broken toward the lower expert id;
  *   - gates: softmax over the k selected logits (equal, in exact arithmetic, to a softmax

@@ -6,9 +6,13 @@ device heap), or a serving loop that must not call cudaMalloc/cudaFree after sta
 because those calls can synchronise the device and stall other streams. Its logits scratch
 is a fixed array inside the library instead of a caller-provided workspace.
 
-This file is named so that pytest collects it last: if it fails, a run that stops at the
-first failure has already run every other test. It passes alone in a fresh process and
-after the rest of the suite.
+The file name sorts last, so pytest collects these tests after every other file. That is
+only about reporting: if a test here fails, a run that stops at its first failure (-x) has
+already run and reported the rest of the suite. Nothing here depends on what ran before:
+the tests pass alone in a fresh process and after the whole suite.
+
+The routing is checked against the CPU oracle (indices bit-exact, gates within 1e-6
+relative) and against moe_route with a caller workspace.
 """
 import ctypes
 
@@ -17,6 +21,7 @@ import pytest
 import torch
 
 import mixture_experts_layer_forward_b200 as moe
+import oracle
 from mixture_experts_layer_forward_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -59,16 +64,29 @@ def _route_noalloc_c_abi(cfg, inp):
     return idx, w
 
 
-def test_noalloc_route_matches_workspace_route_on_two_calls_in_a_row():
-    # two different layers back to back: the second call must not see the first one's logits
+def _oracle_route(cfg, inp):
+    b = None if inp["bias"] is None else inp["bias"].numpy()
+    # with the selection-only bias the logits exclude it and the top-k adds it to the keys
+    logits = oracle.router_logits(synth.bf16_bits(inp["x"]), synth.bf16_bits(inp["Wg"]),
+                                  None if cfg.gate == moe.GATE_SELECT_BIAS else b)
+    return oracle.topk_gates(logits, cfg.k, gate=cfg.gate, bias=b)
+
+
+def test_noalloc_route_matches_oracle_on_two_calls_in_a_row():
+    # different layers back to back: a later call must not see an earlier call's logits
     cases = [synth.LayerConfig("a", T=4096, H=512, F=64, E=256, k=8, zipf_s=1.2),
-             synth.LayerConfig("b", T=3000, H=1024, F=64, E=8, k=2)]
+             synth.LayerConfig("b", T=3000, H=1024, F=64, E=8, k=2),
+             synth.LayerConfig("c", T=1000, H=256, F=64, E=64, k=4, zipf_s=1.2,
+                               gate=moe.GATE_SELECT_BIAS)]
     for i, cfg in enumerate(cases):
         inp = synth.make_inputs(cfg, seed=20 + i)
-        idx_ref, w_ref = _route_with_workspace(cfg, inp)
+        ref_idx, ref_w = _oracle_route(cfg, inp)
+        idx_ws, w_ws = _route_with_workspace(cfg, inp)
         idx, w = _route_noalloc_c_abi(cfg, inp)
-        assert torch.equal(idx, idx_ref), cfg.name
-        np.testing.assert_allclose(w.cpu().numpy(), w_ref.cpu().numpy(), rtol=1e-5, atol=1e-7)
+        assert np.array_equal(idx.cpu().numpy(), ref_idx), cfg.name
+        np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-6, atol=1e-7)
+        assert torch.equal(idx, idx_ws), cfg.name
+        np.testing.assert_allclose(w.cpu().numpy(), w_ws.cpu().numpy(), rtol=1e-6, atol=1e-7)
 
 
 def test_noalloc_route_rejects_sizes_beyond_its_scratch():
