@@ -59,6 +59,9 @@ def parse_args():
                     help="grouped-GEMM variant (moe_set_gemm_mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="measure only the named workload (default: the Mixtral-shaped run also "
+                         "reports the other four bench workloads under 'workloads')")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
@@ -112,6 +115,143 @@ def load_peaks():
         d = json.loads(p.read_text())
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_peak(peaks, clocks, fp8=False):
+    """Tensor-core peak for the clock regime of a timed region, read from the median sampled
+    SM clock: the measured burst figure when the median is within 10% of the maximum clock,
+    the measured sustained (power-capped) figure otherwise. e4m3: the bf16 figure times the
+    nominal e4m3/bf16 ratio of 2. Returns (peak, burst_peak, regime, clock_frac)."""
+    mult = 2.0 if fp8 else 1.0
+    burst = peaks["bf16_tflops"] * mult
+    sust = (peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]) * mult
+    cf = None
+    if clocks and clocks.get("sm_max_mhz"):
+        cf = clocks["sm_mhz"] / clocks["sm_max_mhz"]
+    regime = "sustained" if (cf is not None and cf < 0.9) else "burst"
+    return (sust if regime == "sustained" else burst), burst, regime, cf
+
+
+def tensor_fracs(achieved, peaks, clocks, fp8=False):
+    """frac against the regime's peak, against the burst peak, and against the burst peak
+    scaled by the sampled clock (median SM MHz / max MHz), with the figures used."""
+    peak, burst, regime, cf = tensor_peak(peaks, clocks, fp8)
+    d = {"peak": peak, "frac": achieved / peak, "regime": regime, "peak_burst": burst,
+         "frac_burst": achieved / burst}
+    if cf is not None:
+        d["clock_frac"] = cf
+        d["frac_clock_scaled"] = achieved / (burst * cf)
+    return d
+
+
+def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, kernel):
+    """Roofline of the layer0 grouped GEMM (the dominant kernel): useful FLOPs (padding rows
+    not counted) and algorithmic bytes (each active expert's W1 once, x once, h of the routed
+    rows written once); the bound is whichever takes longer at the measured peaks."""
+    w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
+    flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
+    wb = 1 if fp8 else 2   # e4m3 experts: 1-byte weights and x codes; h is still bf16
+    nbytes = wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) + 2 * cfg.T * cfg.k * cfg.F
+    g0_s = g0_ms / 1e3
+    tpk, _, _, _ = tensor_peak(peaks, clocks, fp8)
+    hbm_bound = nbytes / (peaks["hbm_gbs"] * 1e9) > flops / (tpk * 1e12)
+    r = {"bound": "hbm" if hbm_bound else "tensor", "kernel": kernel}
+    if hbm_bound:
+        achieved = nbytes / g0_s / 1e9
+        r.update({"achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                  "frac": achieved / peaks["hbm_gbs"],
+                  "peak_source": f"{peak_src} HBM copy bandwidth"})
+    else:
+        achieved = flops / g0_s / 1e12
+        r.update({"achieved": achieved, "unit": "TFLOP/s"})
+        r.update(tensor_fracs(achieved, peaks, clocks, fp8))
+        r["peak_source"] = (f"{peak_src} bf16 {r['regime']}" + (" x 2 (nominal e4m3/bf16 ratio)" if fp8 else "") +
+                            "; regime from the median sampled SM clock (>= 0.9 of max: burst)")
+    r.update({"traffic": traffic_for(kernel, cfg.name), "algorithmic_flops_per_launch": flops,
+              "algorithmic_bytes_per_launch": nbytes, "active_experts": active_experts,
+              "ms_per_launch": g0_ms})
+    return r
+
+
+STAGE_NAMES = ["route", "dispatch", "layer0_gemm_swiglu", "layer1_gemm_scale", "combine"]
+
+
+def new_sampler(torch, dev, enabled):
+    if not enabled:
+        return None
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    smp = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    smp.start()
+    return smp
+
+
+def timed_staged(torch, fwd_staged, K, stream, dev, sampler, barrier=None):
+    """K back-to-back staged forwards between two events on the launch stream; returns
+    (total ms, per-stage mean ms, clock summary of the timed region)."""
+    import mixture_experts_layer_forward_b200 as moe
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGE_EVENTS)]
+           for _ in range(K)]
+    for row in evs:          # create the CUDA events now, outside the timed region
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    start.record(stream)
+    for i in range(K):
+        fwd_staged(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_end = time.time()
+    if barrier is not None:
+        barrier()
+    clocks = sampler.stop(t_begin, t_end) if sampler is not None else None
+    stage_ms = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+                for j, nm in enumerate(STAGE_NAMES)}
+    return start.elapsed_time(end), stage_ms, clocks
+
+
+def measure_workload(torch, name, dev, K, W, seed, clocks_on, peaks, peak_src):
+    """One workload (its own inputs and weights) on this GPU: K staged layer forwards after W
+    warm-up ones; step time, stage times, clocks and the layer0 roofline."""
+    import mixture_experts_layer_forward_b200 as moe
+    from mixture_experts_layer_forward_b200 import synth
+
+    cfg = synth.CONFIGS[name]
+    stream = torch.cuda.current_stream(dev)
+    inp = synth.make_inputs(cfg, seed=seed, device=dev)
+    p = moe.Problem.from_config(cfg)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    a = (p, inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W2"], out, ws)
+    for _ in range(W):
+        moe.moe_forward(*a, idx)
+    torch.cuda.synchronize(dev)
+    assert moe.moe_get_device_status(ws) == 0, f"{name}: device status after warm-up"
+    active = int(torch.unique(idx).numel())
+    sampler = new_sampler(torch, dev, clocks_on)
+    ms, stage_ms, clocks = timed_staged(torch, lambda ev: moe.moe_forward_staged(*a, ev), K,
+                                        stream, dev, sampler)
+    assert moe.moe_get_device_status(ws) == 0, f"{name}: device status"
+    ms_step = ms / K
+    tflops = cfg.useful_flops / (ms_step / 1e3) / 1e12
+    layer = {"bound": "tensor", "achieved": tflops, "unit": "TFLOP/s"}
+    layer.update(tensor_fracs(tflops, peaks, clocks))
+    res = {"workload": WORKLOAD_NAMES.get(name, name), "T": cfg.T, "H": cfg.H, "F": cfg.F,
+           "E": cfg.E, "top_k": cfg.k, "steps": K, "warmup": W, "ms_per_step": ms_step,
+           "tokens_per_s": cfg.T / (ms_step / 1e3), "tflops": tflops, "layer_roofline": layer,
+           "stage_ms": stage_ms,
+           "roofline": layer0_roofline(cfg, stage_ms["layer0_gemm_swiglu"], active, peaks, peak_src,
+                                       clocks, False, DOMINANT_KERNEL["auto"]),
+           "clocks": clocks, "active_experts": active}
+    del inp, out, ws, idx, a
+    torch.cuda.empty_cache()
+    return res
 
 
 def source_hash(files):
@@ -353,33 +493,10 @@ def run_ours(args):
     if cfg.E <= 64:
         routing["expert_histogram"] = [int(c) for c in counts]
 
-    # stage events of every timed step (recorded on the launch stream by the library)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGE_EVENTS)]
-           for _ in range(K)]
-    for row in evs:          # create the CUDA events now, outside the timed region
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize(dev)
-    clocks = None
-    sampler = None
-    if not args.no_clocks:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
-        sampler.start()
-    dp.barrier(dev)
-    torch.cuda.synchronize(dev)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_begin = time.time()
-    start.record(stream)
-    for i in range(K):
-        fwd_staged(evs[i])
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    t_end = time.time()
-    dp.barrier(dev)
-    if sampler is not None:
-        clocks = sampler.stop(t_begin, t_end)
-    ms_local = start.elapsed_time(end)
+    # K staged steps: stage events recorded on the launch stream by the library
+    sampler = new_sampler(torch, dev, not args.no_clocks)
+    ms_local, stage_ms, clocks = timed_staged(torch, fwd_staged, K, stream, dev, sampler,
+                                              barrier=lambda: dp.barrier(dev))
     status = moe.moe_get_device_status(ws)
     assert status == 0, f"device status {status}"
     ms = dp.max_over_ranks(ms_local, device=dev)
@@ -400,9 +517,6 @@ def run_ours(args):
     cold_ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in cold_ev) / n_cold, device=dev)
     del flush
 
-    stage_names = ["route", "dispatch", "layer0_gemm_swiglu", "layer1_gemm_scale", "combine"]
-    stage_ms = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
-                for j, nm in enumerate(stage_names)}
 
     # end to end through the public API with host buffers: every step copies its x in and
     # its out back (pinned host memory); moe_forward_host_batches overlaps step i's compute
@@ -429,42 +543,13 @@ def run_ours(args):
                "ms_per_step": e2e_ms, "api": "moe_forward_host_batches (copies overlapped across steps)"}
 
     peaks, peak_src = load_peaks()
-    # Denominator in the clock regime the kernels ran in: the power-capped (sustained) GEMM
-    # peak when the power cap throttled the SM clock during the timed region or the clock sat
-    # well below its maximum, the burst peak otherwise.
-    sustained = bool(clocks and ("sw_power_cap" in clocks["reasons"] or
-                                 clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]))
-    regime = "sustained" if sustained else "burst"
-    tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
-    # the e4m3 contraction's peak: the measured bf16 peak times the nominal ratio (4.5 / 2.25)
-    gemm_peak = 2.0 * tf_peak if args.fp8 else tf_peak
     layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
-    # layer0: useful FLOPs (padding rows not counted) and algorithmic bytes (each active
-    # expert's W1 once, x once, h of the routed rows written once); the bound is whichever
-    # takes longer at the measured peaks
-    w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
-    gemm0_flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
-    # (e4m3 experts: 1-byte weights and x codes; h is still written in bf16)
-    wb = 1 if args.fp8 else 2
-    gemm0_bytes = (wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) +
-                   2 * cfg.T * cfg.k * cfg.F)
-    g0_ms = stage_ms["layer0_gemm_swiglu"]
-    g0_s = g0_ms / 1e3
     kernel = "moe_grouped_gemm_select_f8_kernel<0>" if args.fp8 else DOMINANT_KERNEL[args.gemm_mode]
-    hbm_bound = gemm0_bytes / (peaks["hbm_gbs"] * 1e9) > gemm0_flops / (gemm_peak * 1e12)
-    if hbm_bound:
-        achieved, peak, unit = gemm0_bytes / g0_s / 1e9, peaks["hbm_gbs"], "GB/s"
-        psrc = f"{peak_src} HBM copy bandwidth"
-    else:
-        achieved, peak, unit = gemm0_flops / g0_s / 1e12, gemm_peak, "TFLOP/s"
-        psrc = (f"{peak_src} bf16 {regime} x 2 (nominal e4m3/bf16 ratio)" if args.fp8 else
-                f"{peak_src} bf16 {regime} (sampled clock-event reasons decide the regime)")
-    roofline = {"bound": "hbm" if hbm_bound else "tensor", "kernel": kernel,
-                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": traffic_for(kernel, cfg.name), "peak_source": psrc,
-                "algorithmic_flops_per_launch": gemm0_flops,
-                "algorithmic_bytes_per_launch": gemm0_bytes, "active_experts": active_experts,
-                "ms_per_launch": g0_ms}
+    roofline = layer0_roofline(cfg, stage_ms["layer0_gemm_swiglu"], active_experts, peaks, peak_src,
+                               clocks, args.fp8, kernel)
+    layer_roof = {"bound": "tensor", "achieved": layer_tflops, "unit": "TFLOP/s per GPU"}
+    layer_roof.update(tensor_fracs(layer_tflops, peaks, clocks, args.fp8))
+    layer_roof["peak_source"] = f"{peak_src} bf16 {layer_roof['regime']}" + (" x 2" if args.fp8 else "")
 
     line = {
         "metric": "MoE-layer forward tokens/s", "value": n * cfg.T / (ms_per_step / 1e3),
@@ -474,9 +559,7 @@ def run_ours(args):
         "data": "synthetic (seeded random inputs and random-init weights of the layer's shape)",
         "config": config_dict(cfg, args, n),
         "tflops": layer_tflops * n,
-        "layer_roofline": {"bound": "tensor", "achieved": layer_tflops, "peak": gemm_peak,
-                           "unit": "TFLOP/s per GPU", "frac": layer_tflops / gemm_peak,
-                           "peak_source": f"{peak_src} bf16 {regime}" + (" x 2" if args.fp8 else "")},
+        "layer_roofline": layer_roof,
         "roofline": roofline,
         "stage_ms": stage_ms,
         # FP8: the bf16 path's launches (router, dispatch, [the gather into sorted rows],
@@ -489,9 +572,24 @@ def run_ours(args):
         "routing": routing,
     }
 
+    # the other bench workloads, measured in the same run (one GPU only): step time, stage
+    # times, layer0 roofline and clocks of each, beside the headline Mixtral-shaped layer
+    if world == 1 and not args.fp8 and not args.no_workloads and args.workload == "mixtral" and \
+            not any(getattr(args, k) is not None for k in ("T", "E", "k", "H", "F")):
+        hin = host_inputs(inp) if (rank == 0 and not args.no_cpu_baseline) else None
+        del inp, out, ws, args_fwd, fwd, fwd_staged
+        torch.cuda.empty_cache()
+        Kw = max(1, min(K, 20))
+        line["workloads"] = {
+            nm: measure_workload(torch, nm, dev, Kw, W, args.seed, not args.no_clocks, peaks, peak_src)
+            for nm in ("phi35", "qwen2", "skew", "skew_decode")}
+    else:
+        hin = None
+
     # the CPU oracle baseline: rank 0 of a one-GPU run only
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
-        hin = host_inputs(inp)
+        if hin is None:
+            hin = host_inputs(inp)
         v, n_tok, t, threads = cpu_oracle_sample(cfg, hin, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{n_tok} random tokens of the {cfg.T}-token batch, "
@@ -590,17 +688,15 @@ def run_backward(args):
     flops = 2 * tk * cfg.H * (3 * w1c + 2 * cfg.F)
     useful = flops - 2 * tk * cfg.H * w1c
     peaks, peak_src = load_peaks()
-    sustained = bool(clocks and ("sw_power_cap" in clocks["reasons"] or
-                                 clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]))
-    tf_peak = (peaks.get("bf16_tflops_sustained") if sustained else None) or peaks["bf16_tflops"]
     tf = flops / (ms / 1e3) / 1e12
+    rf = {"bound": "tensor", "achieved": tf, "unit": "TFLOP/s"}
+    rf.update(tensor_fracs(tf, peaks, clocks))
+    rf["peak_source"] = f"{peak_src} bf16 {rf['regime']}; regime from the median sampled SM clock"
     emit({"metric": "MoE-layer backward tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
           "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
           "dtype": "bf16 (fp32 accumulation)", "data": "synthetic", "config": config_dict(cfg, args, 1),
           "gemm_tflops": tf, "useful_tflops": useful / (ms / 1e3) / 1e12,
-          "roofline": {"bound": "tensor", "achieved": tf, "peak": tf_peak, "unit": "TFLOP/s",
-                       "frac": tf / tf_peak,
-                       "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}"},
+          "roofline": rf,
           "clocks": clocks})
     return 0
 
