@@ -69,6 +69,8 @@ def parse_args():
                     help="e4m3 experts (moe_forward_fp8; weights quantised once before timing)")
     ap.add_argument("--backward", action="store_true",
                     help="time moe_backward (the layer's gradients) instead of the forward")
+    ap.add_argument("--router-mode", choices=["auto", "sequential", "filter"], default="auto",
+                    help="router variant (moe_set_router_mode)")
     ap.add_argument("--router-only", action="store_true",
                     help="time moe_route alone (router logits + top-k); no expert weights allocated")
     return ap.parse_args()
@@ -381,6 +383,11 @@ def host_inputs(inp):
             synth.bf16_bits(inp["W2"]), b)
 
 
+def set_router_mode(moe, args):
+    moe.moe_set_router_mode({"auto": moe.ROUTER_AUTO, "sequential": moe.ROUTER_SEQUENTIAL,
+                             "filter": moe.ROUTER_FILTER}[args.router_mode])
+
+
 def emit(obj):
     print(json.dumps(obj), flush=True)
 
@@ -452,6 +459,7 @@ def run_ours(args):
     K, W = args.steps, max(3, args.warmup)
     moe.moe_set_gemm_mode({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE_CTA,
                            "pair": moe.GEMM_CTA_PAIR, "fused": moe.GEMM_FUSED}[args.gemm_mode])
+    set_router_mode(moe, args)
 
     inp = synth.make_inputs(cfg, seed=args.seed, device=dev,
                             x_seed=dp.replica_x_seed(args.seed, rank) if world > 1 else None)
@@ -612,6 +620,7 @@ def run_router(args):
     dev = torch.device("cuda", 0)
     cfg = workload(args)
     K, W = args.steps, max(3, args.warmup)
+    set_router_mode(moe, args)
     inp = synth.make_inputs(cfg, seed=args.seed, device=dev, experts=False)
     p = moe.Problem.from_config(cfg)
     ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)

@@ -351,24 +351,6 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
 }
 
 // The whole CTA: work items w_first, w_first + w_step, ... (smem 1024-byte aligned).
-// and-vote over the threads of a named barrier (all of them must reach it)
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred)
-{
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\t"
-                 "setp.ne.u32 p, %1, 0;\n\t"
-                 "bar.red.and.pred q, %2, %3, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r)
-                 : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
-                 : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // BMODE_WGRAD work item w: expert-major, then N tile, then M tile; its k-blocks of 64 rows
 __device__ __forceinline__ void wgrad_item(int w, const GemmArgs &a, int &e, int &mt, int &nt,
                                            int &kb0, int &kb1)

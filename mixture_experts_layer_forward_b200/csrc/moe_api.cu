@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -14,6 +15,7 @@
 #include "dispatch.cuh"
 #include "fp8.cuh"
 #include "fused.cuh"
+#include "route_chain.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
@@ -270,6 +272,22 @@ bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D bf16 row-major [rows, cols] without swizzle; box = box_cols x box_rows (box_cols * 2 a
+// multiple of 16 bytes).
+bool make_map_2d_plain(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                       uint32_t box_cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D bf16 [depth, rows, cols]; box = 64 columns x box_rows rows x 1, 128-byte swizzle.
 bool make_map_3d(CUtensorMap *m, const void *base, uint64_t depth, uint64_t rows, uint64_t cols,
                  uint32_t box_rows = 64)
@@ -421,6 +439,65 @@ cudaError_t launch_route_filter(const moe_problem *p, const FilterPlan &fp,
     return cudaGetLastError();
 }
 
+// The one-launch router for up to 32 experts (route_chain.cuh): E a multiple of 8 (whole
+// 16-byte W_g rows for its TMA boxes).
+bool route_uses_chain(const moe_problem *p)
+{
+    return p->E % 8 == 0 && p->E <= 32 && p->H % 64 == 0;
+}
+
+template <int EPT, int G>
+cudaError_t launch_route_chain_t(const moe_problem *p, const __nv_bfloat16 *x,
+                                 const __nv_bfloat16 *Wg, const float *bias, int32_t *topk_idx,
+                                 float *topk_w, int *status, cudaStream_t st)
+{
+    const int T = p->T, H = p->H, E = p->E;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    // about one CTA per SM: tt tokens each (at most 256 box rows, RC_MAX_CONSUMERS threads)
+    int tt = (T + sms - 1) / sms;
+    tt = std::max(1, std::min(tt, std::min(256, RC_MAX_CONSUMERS / G)));
+    const int ncw = (tt * G + 31) / 32;
+    int stages = RC_MAX_STAGES;
+    RcLayout L = rc_layout(tt, E, EPT * G, stages);
+    while (stages > 3 && L.total + 1024 > RC_SMEM_BUDGET) {
+        --stages;
+        L = rc_layout(tt, E, EPT * G, stages);
+    }
+    const int smem = L.total + 1024;
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    CUtensorMap mx, mw;
+    if (!make_map_2d(&mx, x, (uint64_t)T, (uint64_t)H, (uint32_t)tt) ||
+        !make_map_2d_plain(&mw, Wg, (uint64_t)H, (uint64_t)E, (uint32_t)E, RC_HC))
+        return cudaErrorInvalidValue;
+    RcArgs a{};
+    a.bias = bias;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.T = T;
+    a.H = H;
+    a.E = E;
+    a.k = p->top_k;
+    a.gate = p->gate;
+    a.tt = tt;
+    a.stages = stages;
+    a.status = status;
+    a.timeout_ns = g_timeout_ns.load();
+    auto kern = route_chain_kernel<EPT, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(T + tt - 1) / tt, 32 + ncw * 32, smem, st>>>(mx, mw, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_chain(const moe_problem *p, const __nv_bfloat16 *x, const __nv_bfloat16 *Wg,
+                               const float *bias, int32_t *topk_idx, float *topk_w, int *status,
+                               cudaStream_t st)
+{
+    if (p->E <= 8) return launch_route_chain_t<4, 2>(p, x, Wg, bias, topk_idx, topk_w, status, st);
+    if (p->E <= 16) return launch_route_chain_t<4, 4>(p, x, Wg, bias, topk_idx, topk_w, status, st);
+    return launch_route_chain_t<4, 8>(p, x, Wg, bias, topk_idx, topk_w, status, st);
+}
+
 // Router choice for AUTO / FILTER / SEQUENTIAL (operands assumed 16-byte aligned).
 bool route_uses_filter(const moe_problem *p)
 {
@@ -445,6 +522,9 @@ cudaError_t launch_route(const moe_problem *p, const moe_bf16 *x, const moe_bf16
     if (filter != nullptr && aligned16(x) && aligned16(Wg) && route_uses_filter(p))
         return launch_route_filter(p, filter_plan(p), xb, wb, bias, topk_idx, topk_w, logits,
                                    *filter, status, st);
+    // up to 32 experts: logits and top-k in one launch, no logits buffer
+    if (aligned16(x) && aligned16(Wg) && route_uses_chain(p))
+        return launch_route_chain(p, xb, wb, bias, topk_idx, topk_w, status, st);
     // blocks of the large-E tile (64 tokens x 64 experts); fewer than the SMs: go narrow
     const int64_t large_blocks = (int64_t)((T + 63) / 64) * ((E + 63) / 64);
     const int sms = sm_count() > 0 ? sm_count() : 148;
@@ -1350,7 +1430,8 @@ int moe_forward_launches(const moe_problem *p)
 {
     if (check_problem(p) != MOE_OK) return -1;
     if (p->T == 0) return 0;
-    const int route = route_uses_filter(p) ? 3 : 2; // filter: prep, GEMM, exact; else logits, top-k
+    // filter: prep, GEMM, exact; up to 32 experts: one launch; else logits, top-k
+    const int route = route_uses_filter(p) ? 3 : route_uses_chain(p) ? 1 : 2;
     // count, scan, place; one block for a single chunk of tokens
     const int dispatch = p->T <= DISPATCH_CHUNK ? 1 : 3;
     const int mode = g_gemm_mode.load();

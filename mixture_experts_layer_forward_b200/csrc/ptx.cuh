@@ -107,6 +107,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// and-vote over the threads of a named barrier (all of them must reach it)
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+                 : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------
 // TMA: tiled bulk tensor loads global -> shared, completion counted on an mbarrier.
 // ---------------------------------------------------------------------------------------

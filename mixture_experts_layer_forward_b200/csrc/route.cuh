@@ -259,22 +259,17 @@ __global__ void __launch_bounds__((BT / RT) * (BE / RE))
 
 constexpr int TOPK_WARPS = 8; // tokens per block
 
-// One warp per token. Dynamic shared memory: TOPK_WARPS * E floats.
-// gate 2 (selection bias): `logits` are without the bias; the selection keys are
-// logits[t][e] + bias[e] (the same fp32 addition the logits kernel makes in the other
-// modes) and the gates use the logits without the bias, shifted by their maximum.
-__global__ void __launch_bounds__(TOPK_WARPS * 32)
-    route_topk_kernel(const float *__restrict__ logits, int32_t *__restrict__ topk_idx,
-                      float *__restrict__ topk_w, int T, int E, int k, int gate,
-                      const float *__restrict__ bias)
+// One warp selects the k largest keys of one token's E logits and writes the token's expert
+// ids and gate weights. `lg` holds the logits (without the bias in gate mode 2), `row` is a
+// scratch row of E floats in shared memory owned by this warp.
+// Keys: the logits, or in gate mode 2 (selection bias) logits[e] + bias[e] (the same fp32
+// addition the logits kernels make in the other modes); the gates use the logits without the
+// bias, shifted by their maximum. k rounds of a warp argmax, ties to the lower expert id.
+__device__ __forceinline__ void topk_row_warp(const float *lg, float *row, int E, int k, int gate,
+                                              const float *__restrict__ bias,
+                                              int32_t *__restrict__ idx_out,
+                                              float *__restrict__ w_out, int lane)
 {
-    extern __shared__ float srow[];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * TOPK_WARPS + warp;
-    if (t >= T) return;
-    float *row = srow + (size_t)warp * E;
-    const float *lg = logits + (size_t)t * E;
     const bool sel_bias = (gate == 2) && bias != nullptr;
     for (int e = lane; e < E; e += 32) row[e] = sel_bias ? lg[e] + bias[e] : lg[e];
     __syncwarp();
@@ -300,16 +295,16 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
         const float gv = (gate == 2) ? lg[bi] : bv; // the gate's logit (no bias in mode 2)
         if (j == 0) top = gv;
         if (lane == 0) {
-            topk_idx[(size_t)t * k + j] = bi;
+            idx_out[j] = bi;
             row[bi] = -INFINITY; // removed from later rounds (logits are finite)
         }
         if (j < 32 && j == lane) sel_val = gv;
-        if (j >= 32 && lane == 0) topk_w[(size_t)t * k + j] = gv; // stash; rescaled below
+        if (j >= 32 && lane == 0) w_out[j] = gv; // stash; rescaled below
         __syncwarp();
     }
     if (gate == 2) { // the largest selected logit (the first selected one need not be)
         float m = -INFINITY;
-        for (int j = lane; j < k; j += 32) m = fmaxf(m, (j < 32) ? sel_val : topk_w[(size_t)t * k + j]);
+        for (int j = lane; j < k; j += 32) m = fmaxf(m, (j < 32) ? sel_val : w_out[j]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         top = m;
@@ -321,7 +316,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
         for (int e = lane; e < E; e += 32) denom += expf(lg[e] - top);
     } else {
         for (int j = lane; j < k; j += 32) {
-            const float v = (j < 32) ? sel_val : topk_w[(size_t)t * k + j];
+            const float v = (j < 32) ? sel_val : w_out[j];
             denom += expf(v - top);
         }
     }
@@ -329,9 +324,24 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
     for (int off = 16; off > 0; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
     __syncwarp();
     for (int j = lane; j < k; j += 32) {
-        const float v = (j < 32) ? sel_val : topk_w[(size_t)t * k + j];
-        topk_w[(size_t)t * k + j] = expf(v - top) / denom;
+        const float v = (j < 32) ? sel_val : w_out[j];
+        w_out[j] = expf(v - top) / denom;
     }
+}
+
+// One warp per token. Dynamic shared memory: TOPK_WARPS * E floats.
+__global__ void __launch_bounds__(TOPK_WARPS * 32)
+    route_topk_kernel(const float *__restrict__ logits, int32_t *__restrict__ topk_idx,
+                      float *__restrict__ topk_w, int T, int E, int k, int gate,
+                      const float *__restrict__ bias)
+{
+    extern __shared__ float srow[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * TOPK_WARPS + warp;
+    if (t >= T) return;
+    topk_row_warp(logits + (size_t)t * E, srow + (size_t)warp * E, E, k, gate, bias,
+                  topk_idx + (size_t)t * k, topk_w + (size_t)t * k, lane);
 }
 
 } // namespace moe

@@ -107,9 +107,10 @@ def test_forward_launch_count_follows_the_modes(lib):
     prev_g = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
     prev_o = moe.moe_set_work_order(moe.ORDER_EXPERT)
     try:
-        # router 2 (3 with the filter) + dispatch 3 (1 for T <= 256) + [x gather] + layer0,
-        # layer1, combine; the bench layers gather x into sorted rows (T * k >= 128 E)
-        assert moe.moe_forward_launches(mixtral) == 9   # E = 8: sequential router
+        # router 1 (up to 32 experts, E % 8 == 0), 2 (more experts, sequential) or 3 (the
+        # filter) + dispatch 3 (1 for T <= 256) + [x gather] + layer0, layer1, combine; the
+        # bench layers gather x into sorted rows (T * k >= 128 E)
+        assert moe.moe_forward_launches(mixtral) == 8   # E = 8: one-launch router
         assert moe.moe_forward_launches(qwen2) == 10    # T*E >= 2^16: filter router
         assert moe.moe_forward_launches(decode) == 6    # T*E < 2^16: sequential, no gather
         phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
@@ -119,6 +120,8 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(mixtral) == 10  # forced: E = 8 qualifies
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
+        assert moe.moe_forward_launches(phi35) == 8     # E = 16: one-launch router
+        assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
         assert moe.moe_forward_launches(qwen2) == 9
@@ -129,8 +132,8 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(decode) == 7
         assert moe.moe_forward_launches(moe.Problem.make(0, 128, 128, 8, 2)) == 0
         moe.moe_set_gemm_mode(moe.GEMM_AUTO)
-        assert moe.moe_forward_launches(moe.Problem.make(256, 128, 128, 8, 2)) == 6  # one chunk
-        assert moe.moe_forward_launches(moe.Problem.make(257, 128, 128, 8, 2)) == 8  # two
+        assert moe.moe_forward_launches(moe.Problem.make(256, 128, 128, 8, 2)) == 5  # one chunk
+        assert moe.moe_forward_launches(moe.Problem.make(257, 128, 128, 8, 2)) == 7  # two
         assert moe.moe_forward_launches(moe.Problem.make(4, 100, 128, 8, 2)) == -1  # H % 64
     finally:
         moe.moe_set_router_mode(prev_r)

@@ -97,6 +97,11 @@ ROUTE_CASES = [
     # small batches with many experts: both decode tile shapes of the sequential router
     ("e256_t64_decode", 64, 512, 256, 8, False, 1.2, 0),
     ("e256_t150_decode", 150, 512, 256, 8, False, 0.0, 0),
+    # the one-launch router's thread shapes (2, 4 and 8 threads per token)
+    ("e32_k4", 500, 384, 32, 4, False, 1.2, 0),
+    ("e24_selbias", 300, 192, 24, 3, False, 1.2, 2),
+    ("e32_all", 200, 128, 32, 5, False, 0.0, 1),
+    ("e16_t1", 1, 640, 16, 2, False, 0.0, 0),
 ]
 
 
@@ -137,12 +142,13 @@ def _route(p, x, Wg, bias, T, k):
     return idx.cpu().numpy(), w.cpu().numpy()
 
 
+@pytest.mark.parametrize("E,k", [(64, 8), (32, 4), (16, 2), (8, 2)])
 @pytest.mark.parametrize("unscaled", [False, True], ids=["scaled", "unscaled"])
-def test_route_rounding_level_ties(router_mode, unscaled):
+def test_route_rounding_level_ties(router_mode, unscaled, E, k):
     """Every expert has the same exact real logit; they differ only in the fp32 rounding of
     the sequential sum (gate columns are one column with pairs of entries swapped where the
     token has equal values), so the choice is made at the last bit of the fp32 logits."""
-    T, H, E, k = 300, 256, 64, 8
+    T, H = 300, 256
     g = torch.Generator().manual_seed(21)
     x = torch.randn(T, H, generator=g)
     for j in range(6):
@@ -183,7 +189,7 @@ def test_route_filter_matches_sequential_bitwise(gate):
     assert np.array_equal(res[0][1].view(np.uint32), res[1][1].view(np.uint32))
 
 
-@pytest.mark.parametrize("name", ["qwen2", "skew", "skew_decode"])
+@pytest.mark.parametrize("name", ["mixtral", "phi35", "qwen2", "skew", "skew_decode"])
 def test_route_filter_matches_sequential_full_size(name):
     """The bench workloads with many experts: filter and sequential routers agree bitwise."""
     cfg = synth.CONFIGS[name]
