@@ -69,6 +69,10 @@ def parse_args():
                     help="e4m3 experts (moe_forward_fp8; weights quantised once before timing)")
     ap.add_argument("--backward", action="store_true",
                     help="time moe_backward (the layer's gradients) instead of the forward")
+    ap.add_argument("--trace", default=None, metavar="FILE",
+                    help="after timing, run one forward with the persistent launch's schedule "
+                         "trace on; write the raw records to FILE (.npy) and a summary into the "
+                         "JSON line")
     ap.add_argument("--router-mode", choices=["auto", "sequential", "filter"], default="auto",
                     help="router variant (moe_set_router_mode)")
     ap.add_argument("--router-only", action="store_true",
@@ -146,14 +150,30 @@ def tensor_fracs(achieved, peaks, clocks, fp8=False):
     return d
 
 
-def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, kernel):
-    """Roofline of the layer0 grouped GEMM (the dominant kernel): useful FLOPs (padding rows
-    not counted) and algorithmic bytes (each active expert's W1 once, x once, h of the routed
-    rows written once); the bound is whichever takes longer at the measured peaks."""
+def launches_in_mode(moe, p, mode):
+    prev = moe.moe_set_gemm_mode(mode)
+    try:
+        return moe.moe_forward_launches(p)
+    finally:
+        moe.moe_set_gemm_mode(prev)
+
+
+def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, kernel, fused=False):
+    """Roofline of the dominant kernel. Separate launches: the layer0 grouped GEMM, with its
+    useful FLOPs (padding rows not counted) and algorithmic bytes (each active expert's W1
+    once, x once, h of the routed rows written once). One persistent launch (`fused`):
+    layer0 + layer1 + combine, with both GEMMs' useful FLOPs and the bytes that must cross
+    HBM (the active experts' W1 and W2, the sorted x rows, the output). The bound is
+    whichever takes longer at the measured peaks."""
     w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
-    flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
     wb = 1 if fp8 else 2   # e4m3 experts: 1-byte weights and x codes; h is still bf16
-    nbytes = wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) + 2 * cfg.T * cfg.k * cfg.F
+    if fused:
+        flops = 2 * cfg.T * cfg.k * cfg.H * (w1_cols + cfg.F)
+        nbytes = (wb * (active_experts * cfg.H * (w1_cols + cfg.F) + cfg.T * cfg.k * cfg.H) +
+                  2 * cfg.T * cfg.H)
+    else:
+        flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
+        nbytes = wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) + 2 * cfg.T * cfg.k * cfg.F
     g0_s = g0_ms / 1e3
     tpk, _, _, _ = tensor_peak(peaks, clocks, fp8)
     hbm_bound = nbytes / (peaks["hbm_gbs"] * 1e9) > flops / (tpk * 1e12)
@@ -176,6 +196,50 @@ def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, ke
 
 
 STAGE_NAMES = ["route", "dispatch", "layer0_gemm_swiglu", "layer1_gemm_scale", "combine"]
+
+
+def schedule_trace(torch, moe, fwd, dev, out_file, cap=1 << 18):
+    """One forward with the persistent launch's schedule trace on. Summary: the span of each
+    kind of work item (layer0 and layer1 tile epilogues, combine items), the gap between
+    the last layer0 and the first layer1 tile, and how much of the combine work ended
+    inside the layer1 window (the in-device analogue of hidden communication)."""
+    import numpy as np
+
+    rec = torch.zeros(4 + 4 * cap, dtype=torch.int64, device=dev)
+    moe.moe_set_schedule_trace(rec, cap)
+    try:
+        fwd()
+        torch.cuda.synchronize(dev)
+    finally:
+        moe.moe_set_schedule_trace(None, 0)
+    n = min(int(rec[0].item()), cap)
+    r = rec[4:4 + 4 * n].view(n, 4).cpu().numpy().astype(np.int64)
+    if out_file:
+        np.save(out_file, r)
+    if n == 0:
+        return {"records": 0}
+    kind = r[:, 0] >> 32
+    t0 = r[:, 2] - r[:, 2].min()
+    t1 = r[:, 3] - r[:, 2].min()
+    summ = {"records": n, "span_us": float(t1.max()) / 1e3}
+    names = {0: "layer0", 1: "layer1", 2: "combine"}
+    for k, nm in names.items():
+        m = kind == k
+        if m.any():
+            summ[nm] = {"items": int(m.sum()), "first_begin_us": float(t0[m].min()) / 1e3,
+                        "last_end_us": float(t1[m].max()) / 1e3,
+                        "busy_us_sum": float((t1[m] - t0[m]).sum()) / 1e3,
+                        "sms": int(len(np.unique(r[m, 1])))}
+    if (kind == 0).any() and (kind == 1).any():
+        summ["layer0_to_layer1_gap_us"] = float(t0[kind == 1].min() - t1[kind == 0].max()) / 1e3
+    if (kind == 2).any() and (kind == 1).any():
+        end1 = t1[kind == 1].max()
+        c = kind == 2
+        dur = (t1[c] - t0[c]).astype(np.float64)
+        inside = np.clip(np.minimum(t1[c], end1) - t0[c], 0, None).astype(np.float64)
+        summ["combine_hidden_frac"] = float(inside.sum() / max(dur.sum(), 1.0))
+        summ["combine_after_layer1_us"] = float(max(0, t1[c].max() - end1)) / 1e3
+    return summ
 
 
 def new_sampler(torch, dev, enabled):
@@ -244,13 +308,30 @@ def measure_workload(torch, name, dev, K, W, seed, clocks_on, peaks, peak_src):
     tflops = cfg.useful_flops / (ms_step / 1e3) / 1e12
     layer = {"bound": "tensor", "achieved": tflops, "unit": "TFLOP/s"}
     layer.update(tensor_fracs(tflops, peaks, clocks))
+    fused = moe.moe_forward_launches(p) < launches_in_mode(moe, p, moe.GEMM_SINGLE_CTA)
+    lay = ("layer0_gemm_swiglu", "layer1_gemm_scale", "combine")
+    g_ms = sum(stage_ms[k] for k in lay) if fused else stage_ms["layer0_gemm_swiglu"]
+    kernel = "moe_fused_layer_kernel<0>" if fused else DOMINANT_KERNEL["auto"]
     res = {"workload": WORKLOAD_NAMES.get(name, name), "T": cfg.T, "H": cfg.H, "F": cfg.F,
            "E": cfg.E, "top_k": cfg.k, "steps": K, "warmup": W, "ms_per_step": ms_step,
            "tokens_per_s": cfg.T / (ms_step / 1e3), "tflops": tflops, "layer_roofline": layer,
-           "stage_ms": stage_ms,
-           "roofline": layer0_roofline(cfg, stage_ms["layer0_gemm_swiglu"], active, peaks, peak_src,
-                                       clocks, False, DOMINANT_KERNEL["auto"]),
+           "stage_ms": stage_ms, "launch": "persistent" if fused else "separate",
+           "roofline": layer0_roofline(cfg, g_ms, active, peaks, peak_src, clocks, False, kernel,
+                                       fused),
            "clocks": clocks, "active_experts": active}
+    if fused:
+        prev = moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)
+        try:
+            for _ in range(W):
+                moe.moe_forward(*a, idx)
+            ms_s, stage_s, _ = timed_staged(torch, lambda ev: moe.moe_forward_staged(*a, ev), K,
+                                            stream, dev, None)
+        finally:
+            moe.moe_set_gemm_mode(prev)
+        sep = sum(stage_s[k] for k in lay)
+        res["overlap"] = {"separate_ms_per_step": ms_s / K, "separate_stage_ms": stage_s,
+                          "separate_layers_ms": sep, "fused_layers_ms": g_ms,
+                          "hidden_frac": 1.0 - g_ms / sep}
     del inp, out, ws, idx, a
     torch.cuda.empty_cache()
     return res
@@ -552,9 +633,19 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     layer_tflops = cfg.useful_flops / (ms_per_step / 1e3) / 1e12
-    kernel = "moe_grouped_gemm_select_f8_kernel<0>" if args.fp8 else DOMINANT_KERNEL[args.gemm_mode]
-    roofline = layer0_roofline(cfg, stage_ms["layer0_gemm_swiglu"], active_experts, peaks, peak_src,
-                               clocks, args.fp8, kernel)
+    # the persistent launch replaces layer0, layer1 and the combine (stage events 3..5 all
+    # mark its end)
+    fused = (not args.fp8 and
+             moe.moe_forward_launches(p) < launches_in_mode(moe, p, moe.GEMM_SINGLE_CTA))
+    if fused:
+        kernel = "moe_fused_layer_kernel<0>" if cfg.act == 0 else "moe_fused_layer_kernel<1>"
+        g_ms = sum(stage_ms[k] for k in ("layer0_gemm_swiglu", "layer1_gemm_scale", "combine"))
+    else:
+        kernel = ("moe_grouped_gemm_select_f8_kernel<0>" if args.fp8
+                  else DOMINANT_KERNEL[args.gemm_mode])
+        g_ms = stage_ms["layer0_gemm_swiglu"]
+    roofline = layer0_roofline(cfg, g_ms, active_experts, peaks, peak_src, clocks, args.fp8, kernel,
+                               fused)
     layer_roof = {"bound": "tensor", "achieved": layer_tflops, "unit": "TFLOP/s per GPU"}
     layer_roof.update(tensor_fracs(layer_tflops, peaks, clocks, args.fp8))
     layer_roof["peak_source"] = f"{peak_src} bf16 {layer_roof['regime']}" + (" x 2" if args.fp8 else "")
@@ -579,6 +670,31 @@ def run_ours(args):
                     "how": "256 MiB buffer written before each step, outside its events"},
         "routing": routing,
     }
+
+    # the three-launch form of the same layer, staged: the sum of its stage times against
+    # the default launch (hidden-overlap ratio: the share of the separate stages' time that
+    # the default form does not spend, the in-device analogue of hidden communication)
+    if not args.fp8 and fused:
+        prev = moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)
+        try:
+            for _ in range(W):
+                fwd()
+            Ks = max(1, min(K, 20))
+            ms_s, stage_s, _ = timed_staged(torch, fwd_staged, Ks, stream, dev, None)
+        finally:
+            moe.moe_set_gemm_mode(prev)
+        sep = {k: v for k, v in stage_s.items()}
+        sum_layers = sep["layer0_gemm_swiglu"] + sep["layer1_gemm_scale"] + sep["combine"]
+        fused_ms = stage_ms["layer0_gemm_swiglu"] + stage_ms["layer1_gemm_scale"] + stage_ms["combine"]
+        line["overlap"] = {
+            "separate_stage_ms": sep, "separate_ms_per_step": ms_s / Ks,
+            "fused_layers_ms": fused_ms, "separate_layers_ms": sum_layers,
+            "hidden_frac": 1.0 - fused_ms / sum_layers,
+            "combine_ms": sep["combine"],
+            "how": "layer0 + layer1 + combine as three launches (staged, same run) against the "
+                   "one persistent launch"}
+    if args.trace is not None and not args.fp8:
+        line["schedule_trace"] = schedule_trace(torch, moe, fwd, dev, args.trace or None)
 
     # the other bench workloads, measured in the same run (one GPU only): step time, stage
     # times, layer0 roofline and clocks of each, beside the headline Mixtral-shaped layer

@@ -107,11 +107,12 @@ typedef struct {
 MOE_API size_t moe_workspace_size(const moe_problem *p);
 
 /* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
- * current GEMM and router modes, assuming 16-byte aligned operands: the router (2, or 3
- * with the tensor-core filter), the dispatch (3; 1 for T <= 256) and the layers (layer0,
- * layer1 and the combine: 3; 4 when x is first gathered into expert-sorted rows, which the
- * CTA-pair GEMM always does and the single-CTA GEMM does when T * top_k >= E * 128;
- * 1 with MOE_GEMM_FUSED).
+ * current GEMM and router modes, assuming 16-byte aligned operands: the router (1 for up to
+ * 32 experts when E is a multiple of 8, 3 with the tensor-core filter, else 2), the dispatch
+ * (3; 1 for T <= 256), the gather of x into expert-sorted rows (1 when T * top_k >= E * 128,
+ * and always for the CTA-pair GEMM) and the layers (layer0, layer1 and the combine: 3; or
+ * 1 for the persistent launch that MOE_GEMM_FUSED forces and MOE_GEMM_AUTO picks for
+ * T * top_k >= E * 128 with E <= 8).
  * 0 for T == 0; -1 if *p is invalid. */
 MOE_API int moe_forward_launches(const moe_problem *p);
 
@@ -371,8 +372,14 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
 #define MOE_GEMM_CTA_PAIR 2
 /* MOE_GEMM_FUSED: layer0, layer1 and the combine in one persistent launch, scheduled by
  * tile-level ready flags (a layer1 tile starts when layer0 has finished its 128 h rows; a
- * combine stripe starts when layer1 has finished that 256-column stripe of every tile).
- * Stage events 3..5 of moe_forward_staged then all mark the end of that one launch. */
+ * combine item -- a 256-column stripe of a block of tokens -- reads each of its rows as
+ * soon as layer1 has stored that stripe of the row's tile). In every CTA four warps move
+ * data: during layer0 they gather token rows or take half of each tile's epilogue, during
+ * layer1 they run the combine beside the GEMM pipeline. MOE_GEMM_AUTO takes this launch
+ * when T * top_k >= E * 128 (every expert averages a full 128-row tile) and E <= 8: layer1
+ * runs expert-major, so the combine's window beside it is about 1/E of layer1, and with
+ * more experts the separate launches measured faster. Otherwise the separate launches. Stage events 3..5 of moe_forward_staged then all mark the end of that one
+ * launch. */
 #define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
 
@@ -426,6 +433,16 @@ MOE_API int moe_route_uses_filter(const moe_problem *p);
  * leaves within a few timeouts and the context stays usable. -1 switches it off (default).
  * Returns the previous value. Not thread-safe; meant for tests. */
 MOE_API int moe_set_fault_injection(int layer0_item);
+
+/* Schedule trace of the persistent (fused) launch, for profiling; off by default.
+ * `records` is a device buffer of 4 + 4 * capacity uint64 values owned by the caller; pass
+ * nullptr to switch the trace off. The caller zeroes records[0] (the record counter) before
+ * a traced call. Each finished work item appends {kind << 32 | item, SM id, begin ns, end ns}
+ * at records[4 + 4 i] (globaltimer nanoseconds; kind 0 = a layer0 tile's epilogue, 1 = a
+ * layer1 tile's epilogue, 2 = a combine item); items past `capacity` are counted but not
+ * stored. Not thread-safe; meant for profiling runs (it adds one atomic per work item).
+ * Returns MOE_OK, or MOE_ERR_INVALID_ARG for a negative capacity. */
+MOE_API moe_status moe_set_schedule_trace(void *records, int64_t capacity);
 
 #ifdef __cplusplus
 }

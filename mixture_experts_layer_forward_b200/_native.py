@@ -109,6 +109,7 @@ def library() -> ctypes.CDLL:
             "moe_set_wait_timeout_ns": ([i64], i64),
             "moe_set_gemm_mode": ([i32], i32),
             "moe_set_fault_injection": ([i32], i32),
+            "moe_set_schedule_trace": ([vp, i64], i32),
             "moe_set_router_mode": ([i32], i32),
             "moe_set_work_order": ([i32], i32),
         }
@@ -415,6 +416,21 @@ ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW, ORDER_PHASED = 0, 1, 2, 3
 def moe_set_fault_injection(layer0_item: int) -> int:
     """Test hook: withhold the ready signal of one layer0 work item of the fused kernel."""
     return int(library().moe_set_fault_injection(int(layer0_item)))
+
+
+def moe_set_schedule_trace(records, capacity: int) -> None:
+    """Record the persistent launch's schedule into ``records`` (a CUDA uint64/int64 tensor of
+    at least 4 + 4 * capacity elements; element 0 counts the records), or switch the trace off
+    with ``records=None``."""
+    if records is None:
+        rc = int(library().moe_set_schedule_trace(None, 0))
+    else:
+        if records.numel() < 4 + 4 * int(capacity) or records.element_size() != 8:
+            raise ValueError("records: need 4 + 4 * capacity 64-bit elements")
+        rc = int(library().moe_set_schedule_trace(ctypes.c_void_p(records.data_ptr()),
+                                                 int(capacity)))
+    if rc != 0:
+        raise MoeError("moe_set_schedule_trace", rc)
 
 
 def moe_set_work_order(order: int) -> int:

@@ -7,43 +7,65 @@
 //   - shared-tensor dependency resolving (Comet §3.1.1): the tensor shared by layer0 and
 //     layer1 is h; layer0 produces it in 128-row M tiles, and a layer1 tile only needs the
 //     h rows of its own M tile, so layer1 work starts tile by tile as layer0 finishes rows;
-//   - layer1 is decomposed along N (§3.1.1, column-wise §3.1.2): a combine item reduces one
-//     256-column stripe of the output, and needs only that stripe of every layer1 tile;
+//   - layer1 is decomposed along N (§3.1.1): a combine item reduces one 256-column stripe of
+//     the output for a block of tokens, and needs only that stripe of the layer1 tiles that
+//     hold its tokens' rows;
+//   - thread-block specialisation (§3.2.1) at warp granularity: in every CTA one warp moves
+//     the GEMM operands (TMA), one issues the MMAs, four drain the accumulators, and four
+//     more are the data-movement warps: during layer0 they gather token rows (small batches)
+//     or take half of each tile's epilogue (rows arrive by TMA from the expert-sorted copy),
+//     and during layer1 they run the combine, concurrently with the GEMM pipeline of their
+//     own SM; the per-shape choice of this arrangement is fused_plan() in the host code
+//     (§3.2.2 adaptive workload assignment);
 //   - the tile-signalling design's producer (one persistent kernel over all local experts)
 //     and its consumer driven by ready flags as tiles finish: here both live in one launch,
-//     the ready flags are gpu-scope counters in global memory, and every wait is bounded.
+//     the flags are in global memory, and every wait is bounded.
 //
-// Work items form one static queue in dependency order:
-//   [ layer0 tiles (expert, m, n) | layer1 tiles (expert, m, n) | combine (stripe, tokens) ]
-// CTA b takes items b, b + grid, b + 2 grid, ... All CTAs are resident at once (one per SM),
-// every item waits only on items earlier in the queue, and a CTA finishes all its earlier
-// items before waiting, so the waits always end.
-//   ready0[m] counts finished layer0 column tiles of M tile m; a layer1 tile of m waits for
-//             ready0[m] == layer0 N tiles before its TMA loads of h;
-//   ready1[n] counts finished layer1 M tiles of column stripe n; a combine item of stripe n
-//             waits for ready1[n] == number of M tiles.
-// Writers publish with a gpu-scope release after their stores and a generic-to-async proxy
-// fence (layer1 reads h with TMA); readers acquire, then fence again before their TMA.
+// Work:
+//   GEMM queue [ layer0 tiles (expert, m, n) | layer1 tiles (expert, m, n) ], both expert-
+//   major (an expert's weight stripe and its rows stay in L2 across its tiles); CTA b takes
+//   items b, b + grid, ... All CTAs are resident at once (one per SM), every item waits only
+//   on items earlier in the queue, and a CTA finishes its earlier items before waiting.
+//   Combine queue: (stripe, token block) items, stripe-major; CTA b's data-movement warps
+//   take items b, b + grid, ... after their layer0 duties; they wait only on layer1 tiles,
+//   and layer1 never waits on them.
+//   ready0[m]             counts finished layer0 column tiles of M tile m; a layer1 tile of m
+//                         waits for ready0[m] == layer0 N tiles before its TMA loads of h;
+//   ready1[n * tiles + m] is set to 1 once layer1 tile (m, stripe n) is stored; a combine
+//                         item waits, row by row, for the flag of the tile holding the row.
+// Writers publish with a gpu-scope release after their stores (plus a generic-to-async proxy
+// fence before ready0, since layer1 reads h with TMA); readers acquire.
 #pragma once
 
 #include "gemm_tc.cuh"
 
 namespace moe {
 
-constexpr int COMBINE_TOKENS = 128; // tokens per combine item
+constexpr int COMBINE_TOKENS = 128; // tokens per combine item unless fused_plan() says otherwise
 
 struct FusedArgs {
-    GemmArgs l0;            // layer0: rows gathered from x, W1, writes h
+    GemmArgs l0;            // layer0: A = x_perm by TMA (a_tma) or rows gathered from x
     GemmArgs l1;            // layer1: h rows by TMA, W2, writes ys (gate-scaled)
     int *ready0;            // [max_tiles]
-    int *ready1;            // [layer1 N tiles]
+    int *done0;             // finished layer0 items (all of them: every M tile is ready)
+    int *comb_next;         // next unclaimed combine item
+    int *ready1;            // [l1.n_tiles, max_tiles]
+    int max_tiles;
     const int32_t *inv_pos; // [T, k]
     __nv_bfloat16 *out;     // [T, H]
     int T, H, k;
     int64_t ys_rows;
     const __nv_bfloat16 *ys_shared; // [T, H] shared-expert rows added last, or nullptr
+    int a_tma;              // 1: layer0 A rows by TMA (expert-sorted copy of x)
+    int comb_tokens;        // tokens per combine item, a multiple of 32
     int fault_skip;         // test hook: layer0 item whose ready signal is withheld (-1: none)
+    // optional schedule trace: records of 4 x uint64 {kind << 32 | item, smid, t_begin_ns,
+    // t_end_ns}; trace[0] is the record counter, records start at trace[4]; nullptr: off
+    unsigned long long *trace;
+    int64_t trace_cap;      // records that fit after the counter
 };
+
+enum : int { TRACE_L0 = 0, TRACE_L1 = 1, TRACE_COMBINE = 2 };
 
 __device__ __forceinline__ int ld_acquire_gpu(const int *p)
 {
@@ -57,9 +79,40 @@ __device__ __forceinline__ void red_release_gpu_add(int *p, int v)
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_release_gpu(int *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_global()
 {
     asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// arrive on an mbarrier with an arrival count (the phase expects that many more arrivals)
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t cnt)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(cnt) : "memory");
+}
+
+__device__ __forceinline__ uint32_t smid_u32()
+{
+    uint32_t v;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(v));
+    return v;
+}
+
+__device__ __forceinline__ void trace_record(const FusedArgs &fa, int kind, int item, uint64_t t0,
+                                             uint64_t t1)
+{
+    if (fa.trace == nullptr) return;
+    const unsigned long long i = atomicAdd(fa.trace, 1ull);
+    if ((int64_t)i >= fa.trace_cap) return;
+    unsigned long long *r = fa.trace + 4 + 4 * i;
+    r[0] = ((unsigned long long)kind << 32) | (unsigned)item;
+    r[1] = smid_u32();
+    r[2] = t0;
+    r[3] = t1;
 }
 
 // Bounded wait for *p >= target with acquire semantics. False after an abort elsewhere in
@@ -69,9 +122,11 @@ __device__ __forceinline__ bool flag_wait_bounded(const int *p, int target, vola
 {
     if (ld_acquire_gpu(p) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint32_t nap = 64; // exponential backoff up to 2 us: pollers stay off the L2 meanwhile
 #pragma unroll 1
     while (true) {
-        __nanosleep(128);
+        __nanosleep(nap);
+        if (nap < 2048) nap <<= 1;
         if (ld_acquire_gpu(p) >= target) return true;
         if (*abort_flag) return false;
         if ((int64_t)(globaltimer_ns() - t0) > timeout_ns) {
@@ -83,70 +138,113 @@ __device__ __forceinline__ bool flag_wait_bounded(const int *p, int target, vola
 }
 
 struct FusedItem {
-    int phase; // 0 layer0, 1 layer1, 2 combine
+    int phase; // 0 layer0, 1 layer1
     int e, mt, nt;
 };
 
-__device__ __forceinline__ FusedItem fused_item(int w, const FusedArgs &fa, int total0, int total1)
+__device__ __forceinline__ FusedItem fused_item(int w, const FusedArgs &fa, int total0)
 {
     FusedItem it{};
     if (w < total0) {
         it.phase = 0;
         gemm_map_work(w, fa.l0, it.e, it.mt, it.nt);
-    } else if (w < total0 + total1) {
+    } else {
         it.phase = 1;
         gemm_map_work(w - total0, fa.l1, it.e, it.mt, it.nt);
-    } else {
-        const int v = w - total0 - total1;
-        const int chunks = (fa.T + COMBINE_TOKENS - 1) / COMBINE_TOKENS;
-        it.phase = 2;
-        it.nt = v / chunks; // output column stripe
-        it.mt = v % chunks; // token chunk
-        it.e = 0;
     }
     return it;
 }
 
-// Combine of one item (256-column stripe x 128 tokens) by eight warps: warp wq (0..7) takes
-// tokens wq, wq + 8, ... of the chunk, eight of them at a time so that eight 16-byte rows per
-// lane are in flight; lane l owns columns stripe*256 + 8l .. +7. Sum over j ascending in fp32,
-// one bf16 rounding.
-__device__ __forceinline__ void fused_combine(const FusedArgs &fa, int stripe, int chunk, int wq,
-                                              int lane, int *status)
+// Bounded wait until the layer1 tiles (stripe `stripe`) that hold the k rows of eight tokens
+// t[0..7] are all stored: lane q checks row (token q & 7, selection q >> 3) and the warp votes,
+// so one round of loads covers all 8 k flags. The rows are the same for every lane; the warp
+// barrier after the vote orders every lane's later loads after the lanes' acquires.
+__device__ __forceinline__ bool combine_rows_ready(const FusedArgs &fa, const int *flags, const int (&t)[8],
+                                                   int lane, volatile int *abort_flag, int *status)
+{
+    const uint64_t t_start = globaltimer_ns();
+    uint32_t nap = 64;
+#pragma unroll 1
+    while (true) {
+        bool ready = true;
+        for (int q = lane; q < 8 * fa.k; q += 32) {
+            const int tok = t[0] + (q & 7) * 4; // t[i] = t[0] + 4 i
+            if (tok >= fa.T) continue;
+            const int rr = fa.inv_pos[(size_t)tok * fa.k + (q >> 3)];
+            if (rr < 0 || (int64_t)rr >= fa.ys_rows || (rr >> 7) >= fa.max_tiles) continue;
+            if (ld_acquire_gpu(flags + (rr >> 7)) == 0) ready = false;
+        }
+        if (__all_sync(0xffffffffu, ready)) break;
+        if (*abort_flag) return false;
+        if ((int64_t)(globaltimer_ns() - t_start) > fa.l0.timeout_ns) {
+            *abort_flag = 1;
+            record_status(status, DEV_TIMEOUT, 332);
+            return false;
+        }
+        __nanosleep(nap);
+        if (nap < 1024) nap <<= 1;
+    }
+    __syncwarp();
+    return true;
+}
+
+// Combine of one item (256-column stripe x comb_tokens tokens) by a group of four warps:
+// warp wq (0..3) takes tokens wq, wq + 4, ... of the block, eight at a time; lane l owns
+// columns stripe*256 + 8l .. +7. For each group of eight tokens it waits until the layer1
+// tiles holding their rows are stored, then loads the rows two selections at a time (16
+// loads in flight per lane) and sums over j ascending in fp32 with one bf16 rounding.
+// Returns false when a wait gave up (timeout or abort).
+__device__ __forceinline__ bool fused_combine(const FusedArgs &fa, int stripe, int chunk, int wq,
+                                              int lane, volatile int *abort_flag, int *status)
 {
     const int col = stripe * gemm::BN + lane * 8;
-    if (col >= fa.H) return;
+    const bool have_col = col < fa.H;
     const __nv_bfloat16 *ys = fa.l1.out;
-    for (int g = 0; g < COMBINE_TOKENS / 64; ++g) {
+    const int *flags = fa.ready1 + (size_t)stripe * fa.max_tiles;
+    for (int g = 0; g < fa.comb_tokens / 32; ++g) {
         int t[8];
         float a[8][8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            t[i] = chunk * COMBINE_TOKENS + g * 64 + i * 8 + wq;
+            t[i] = chunk * fa.comb_tokens + g * 32 + i * 4 + wq;
 #pragma unroll
             for (int c = 0; c < 8; ++c) a[i][c] = 0.0f;
         }
-        for (int j = 0; j < fa.k; ++j) {
-            uint4 u[8];
+        if (t[0] >= fa.T) break; // the block's remaining groups are past the batch
+        if (!combine_rows_ready(fa, flags, t, lane, abort_flag, status)) return false;
+        for (int j0 = 0; j0 < fa.k; j0 += 2) {
+            uint4 u[2][8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                u[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (t[i] < fa.T) {
-                    const int r = fa.inv_pos[(size_t)t[i] * fa.k + j];
-                    if (r >= 0 && (int64_t)r < fa.ys_rows)
-                        u[i] = *reinterpret_cast<const uint4 *>(ys + (size_t)r * fa.H + col);
-                    else
-                        record_status(status, DEV_BAD_INDEX, 331);
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = j0 + jj;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    u[jj][i] = make_uint4(0u, 0u, 0u, 0u);
+                    if (j < fa.k && t[i] < fa.T) {
+                        const int r = fa.inv_pos[(size_t)t[i] * fa.k + j];
+                        if (r >= 0 && (int64_t)r < fa.ys_rows && (r >> 7) < fa.max_tiles) {
+                            if (have_col)
+                                u[jj][i] = *reinterpret_cast<const uint4 *>(ys + (size_t)r * fa.H + col);
+                        } else if (lane == 0) {
+                            record_status(status, DEV_BAD_INDEX, 331);
+                        }
+                    }
                 }
             }
+            // j ascending: the first selection of the pair, then the second
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                a[i][0] += bf16_lo(u[i].x); a[i][1] += bf16_hi(u[i].x);
-                a[i][2] += bf16_lo(u[i].y); a[i][3] += bf16_hi(u[i].y);
-                a[i][4] += bf16_lo(u[i].z); a[i][5] += bf16_hi(u[i].z);
-                a[i][6] += bf16_lo(u[i].w); a[i][7] += bf16_hi(u[i].w);
+            for (int jj = 0; jj < 2; ++jj) {
+                if (j0 + jj >= fa.k) break;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    a[i][0] += bf16_lo(u[jj][i].x); a[i][1] += bf16_hi(u[jj][i].x);
+                    a[i][2] += bf16_lo(u[jj][i].y); a[i][3] += bf16_hi(u[jj][i].y);
+                    a[i][4] += bf16_lo(u[jj][i].z); a[i][5] += bf16_hi(u[jj][i].z);
+                    a[i][6] += bf16_lo(u[jj][i].w); a[i][7] += bf16_hi(u[jj][i].w);
+                }
             }
         }
+        if (!have_col) continue;
         if (fa.ys_shared != nullptr) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -169,11 +267,39 @@ __device__ __forceinline__ void fused_combine(const FusedArgs &fa, int stripe, i
             *reinterpret_cast<uint4 *>(fa.out + (size_t)t[i] * fa.H + col) = o;
         }
     }
+    return true;
+}
+
+// Combine items from the launch-wide queue (stripe-major), taken one at a time by a group of
+// four warps (128 threads meeting at named barrier `bar`): the group's first thread claims
+// the next item with an atomic and shares it through shared memory. Returns false on abort.
+__device__ __forceinline__ bool combine_queue(const FusedArgs &fa, int group_warp, int lane, int bar,
+                                              volatile int *slot, volatile int *abort_flag,
+                                              int *status)
+{
+    const int nchunk = (fa.T + fa.comb_tokens - 1) / fa.comb_tokens;
+    const int total2 = fa.l1.n_tiles * nchunk;
+    bool ok = true;
+    while (true) {
+        if (group_warp == 0 && lane == 0) *slot = atomicAdd(fa.comb_next, 1);
+        named_bar_sync(bar, 128);
+        const int j = *slot;
+        named_bar_sync(bar, 128); // everyone has read the slot before it is overwritten
+        if (j >= total2 || !ok) break;
+        const uint64_t t_begin = globaltimer_ns();
+        ok = fused_combine(fa, j / nchunk, j % nchunk, group_warp, lane, abort_flag, status);
+        // a group stops only together: vote at the next claim
+        ok = named_bar_and(bar, 128, ok);
+        if (ok && group_warp == 0 && lane == 0) trace_record(fa, TRACE_COMBINE, j, t_begin, globaltimer_ns());
+        if (!ok) break;
+    }
+    return ok;
 }
 
 template <int KIND0>
 __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
-    moe_fused_layer_kernel(const __grid_constant__ CUtensorMap tmW1,
+    moe_fused_layer_kernel(const __grid_constant__ CUtensorMap tmA0,
+                           const __grid_constant__ CUtensorMap tmW1,
                            const __grid_constant__ CUtensorMap tmH,
                            const __grid_constant__ CUtensorMap tmW2, const FusedArgs fa)
 {
@@ -190,7 +316,9 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *warps_done = reinterpret_cast<int *>(tmem_slot + 2); // [2], per accumulator buffer
+    // [4] ring of part counters, then the two combine groups' claimed-item slots (inside the
+    // shared-memory allocation: the GEMM's column-scale buffers, unused here, follow)
+    int *warps_done = reinterpret_cast<int *>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -198,21 +326,27 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     const GemmArgs &l1 = fa.l1;
     int *status = l0.status;
     const int64_t tmo = l0.timeout_ns;
+    const bool a_tma = fa.a_tma != 0;
+    // layer0 epilogue parts: warps 2..5, and with A by TMA also warps 6..9 (half the chunks each)
+    const int parts0 = a_tma ? 8 : 4;
+    const int nch0 = (KIND0 == GEMM_SWIGLU) ? 4 : BN / 32;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1 + GATHER_THREADS); // TMA arrive + one per gather thread
+            // TMA arrive (+ one per gather thread when layer0 rows are gathered in the kernel;
+            // the producer adds those arrivals itself for layer1 stages)
+            mbar_init(full_bar(s), a_tma ? 1 : 1 + GATHER_THREADS);
             mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 4);
+            mbar_init(tempty_bar(a), parts0);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
-        warps_done[0] = 0;
-        warps_done[1] = 0;
+        for (int i = 0; i < 4; ++i) warps_done[i] = 0;
         fence_mbar_init();
+        if (a_tma) tma_prefetch_desc(&tmA0);
         tma_prefetch_desc(&tmW1);
         tma_prefetch_desc(&tmH);
         tma_prefetch_desc(&tmW2);
@@ -228,9 +362,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
 
     const int num_tiles = l0.meta->num_tiles;
     const int total0 = num_tiles * l0.n_tiles;
-    const int total1 = num_tiles * l1.n_tiles;
-    const int total2 = l1.n_tiles * ((fa.T + COMBINE_TOKENS - 1) / COMBINE_TOKENS);
-    const int total = total0 + total1 + total2;
+    const int total = total0 + num_tiles * l1.n_tiles;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -241,13 +373,14 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
 #pragma unroll
             for (int i = 0; i < STAGES; ++i) armed[i] = -1;
             bool ok = true;
+            bool all0 = false; // every layer0 item finished: no more per-tile waits
             for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-                const FusedItem it = fused_item(w, fa, total0, total1);
-                if (it.phase == 2) continue;
+                const FusedItem it = fused_item(w, fa, total0);
                 if (it.phase == 1) {
                     // layer1 needs every layer0 column tile of its M tile
-                    if (!flag_wait_bounded(fa.ready0 + it.mt, l0.n_tiles, abort_flag, tmo, status,
-                                           300)) {
+                    if (!all0) all0 = ld_acquire_gpu(fa.done0) >= total0;
+                    if (!all0 && !flag_wait_bounded(fa.ready0 + it.mt, l0.n_tiles, abort_flag, tmo,
+                                                    status, 300)) {
                         ok = false;
                         break;
                     }
@@ -261,9 +394,13 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                     }
                     const uint32_t a_dst = smem_u32(smem + s * STAGE);
                     const uint32_t b_dst = a_dst + A_TILE;
-                    mbar_arrive_expect_tx(full_bar(s), it.phase == 0 ? B_TILE : STAGE);
+                    const bool a_here = it.phase == 1 || a_tma;
+                    mbar_arrive_expect_tx(full_bar(s), a_here ? STAGE : B_TILE);
+                    // layer1 stages when layer0 gathers: the gather warps do not arrive
+                    if (it.phase == 1 && !a_tma) mbar_arrive_cnt(full_bar(s), GATHER_THREADS);
                     armed[s] = (int)ph;
                     if (it.phase == 0) {
+                        if (a_tma) tma_load_2d(a_dst, &tmA0, full_bar(s), kb * BK, it.mt * BM);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             int col;
@@ -301,8 +438,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             int n = 0; // accumulator tiles issued
             bool ok = true;
             for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-                const FusedItem it = fused_item(w, fa, total0, total1);
-                if (it.phase == 2) continue;
+                const FusedItem it = fused_item(w, fa, total0);
                 const int acc = n & 1;
                 const uint32_t aph = (uint32_t)(n >> 1) & 1u;
                 if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, tmo, status, 310)) {
@@ -317,7 +453,8 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                         ok = false;
                         break;
                     }
-                    fence_proxy_async_smem(); // gathered rows arrive through the generic proxy
+                    // gathered rows arrive through the generic proxy
+                    if (it.phase == 0 && !a_tma) fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * STAGE);
                     const uint32_t b_addr = a_addr + A_TILE;
@@ -342,28 +479,26 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             volatile int never = 0;
             mbar_wait_bounded(done_bar, 0, &never, tmo, status, 312);
         }
-    } else if (warp >= 6) {
-        // ---------------- layer0 A-row gather (cp.async), warps 6..9 ----------------
-        const int g = threadIdx.x - NUM_THREADS;
-        const int chunk = g & 7;
-        const int r0 = g >> 3;
-        int s = 0;
-        uint32_t ph = 0;
+    } else {
+        // ---------------- epilogue warps 2..5 and data-movement warps 6..9 ----------------
+        const bool dm = warp >= 6;
+        const int q = warp & 3; // TMEM lanes 32q .. 32q+31
+        int n = 0;
         bool ok = true;
+        // gather mode: ring position of the data-movement warps (layer0 stages only)
+        int gs = 0;
+        uint32_t gph = 0;
+        const int g = threadIdx.x - NUM_THREADS;
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-            const FusedItem it = fused_item(w, fa, total0, total1);
-            if (it.phase == 2) {
-                // the gather warps help with the combine (warps 4..7 of its eight)
-                ok = flag_wait_bounded(fa.ready1 + it.nt, num_tiles, abort_flag, tmo, status, 332);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    ok = false;
-                    break;
-                }
-                fused_combine(fa, it.nt, it.mt, 4 + (warp - 6), lane, status);
-                continue;
-            }
-            const __nv_bfloat16 *src[8];
-            if (it.phase == 0) {
+            const FusedItem it = fused_item(w, fa, total0);
+            if (dm && it.phase == 1) break; // the data-movement warps serve layer0 items only
+            if (dm && !a_tma) {
+                // ---- A-row gather for a layer0 item (cp.async): thread g copies 16-byte chunk
+                // (g & 7) of rows (g >> 3) + 16 i; its 8 token ids are read once per tile and
+                // kept in registers (Comet §4: row indices cached in registers)
+                const int chunk = g & 7;
+                const int r0 = g >> 3;
+                const __nv_bfloat16 *src[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int64_t r = (int64_t)it.mt * BM + r0 + 16 * i;
@@ -371,80 +506,89 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
                     if (t < 0 || t >= l0.gather_rows) t = 0;
                     src[i] = l0.gather_src + (size_t)t * l0.gather_ld + chunk * 8;
                 }
-            }
-            const int KB = it.phase == 0 ? l0.k_blocks : l1.k_blocks;
-            for (int kb = 0; kb < KB; ++kb) {
-                ok = mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, tmo, status, 320);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    ok = false;
-                    break;
-                }
-                if (it.phase == 0) {
-                    const uint32_t a_dst = smem_u32(smem + s * STAGE);
+                for (int kb = 0; kb < l0.k_blocks; ++kb) {
+                    ok = mbar_wait_bounded(empty_bar(gs), gph ^ 1u, abort_flag, tmo, status, 320);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_u32(smem + gs * STAGE);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int r = r0 + 16 * i;
                         cp_async_16_cg(a_dst + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * BK);
                     }
+                    cp_async_arrive_noinc(full_bar(gs));
+                    if (++gs == STAGES) {
+                        gs = 0;
+                        gph ^= 1u;
+                    }
                 }
-                // layer1 stages carry no gathered rows: the arrival is immediate
-                cp_async_arrive_noinc(full_bar(s));
-                if (++s == STAGES) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-        }
-        cp_async_wait_all();
-    } else {
-        // ---------------- epilogue + combine: warps 2..5 ----------------
-        const int q = warp & 3;
-        int n = 0;
-        for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const FusedItem it = fused_item(w, fa, total0, total1);
-            if (it.phase == 2) {
-                // combine stripe it.nt for tokens it.mt*128 .. +127: out = sum_j ys[inv_pos]
-                bool ok = flag_wait_bounded(fa.ready1 + it.nt, num_tiles, abort_flag, tmo, status,
-                                            330);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                fused_combine(fa, it.nt, it.mt, q, lane, status);
                 continue;
             }
+            // ---- epilogue of a GEMM item (warps 2..5; warps 6..9 for the second half of a
+            // layer0 tile when its A rows came by TMA)
             const int acc = n & 1;
             const uint32_t aph = (uint32_t)(n >> 1) & 1u;
-            bool ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, tmo, status, 340);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            ok = mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, tmo, status, 340);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            const uint64_t t_begin = globaltimer_ns();
             tc_fence_after();
             const int row = it.mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            if (it.phase == 0)
-                epilogue_rows<KIND0>(l0, t_row, row, it.nt);
-            else
+            if (it.phase == 0) {
+                const int c_lo = (a_tma && dm) ? nch0 / 2 : 0;
+                const int c_hi = a_tma ? c_lo + nch0 / 2 : -1;
+                epilogue_rows<KIND0>(l0, t_row, row, it.nt, 0, 0, nullptr, c_lo, c_hi);
+            } else {
                 epilogue_rows<GEMM_SCALE>(l1, t_row, row, it.nt);
-            // Ready signal: the last of the four epilogue warps to finish this tile publishes
-            // it (before releasing the accumulator, so a buffer's counter is never reused
-            // while a slower warp still holds the previous tile).
+            }
+            // The accumulator is free as soon as its TMEM reads are done (layer1 items with
+            // eight epilogue parts configured: warps 2..5 stand for 6..9).
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cnt(tempty_bar(acc), (it.phase == 1 && a_tma) ? 2u : 1u);
+            // Ready signal: every part makes its stores visible, then the last of the item's
+            // parts publishes it. The part counters form a ring of 4 indexed by the CTA's item
+            // count: slot n & 3 is reused by item n + 4, whose parts can only arrive after
+            // every warp (this one included) has finished item n + 2.
             __threadfence();
             __syncwarp();
             if (lane == 0) {
-                const int prev = atomicAdd(&warps_done[acc], 1);
-                if (prev == 3) {
-                    warps_done[acc] = 0;
+                const int parts = it.phase == 0 ? parts0 : 4;
+                const int prev = atomicAdd(&warps_done[n & 3], 1);
+                if (prev == parts - 1) {
+                    warps_done[n & 3] = 0;
                     __threadfence();
-                    const bool withhold = (it.phase == 0 && w == fa.fault_skip);
-                    if (!withhold) {
-                        fence_proxy_async_global();
-                        red_release_gpu_add(it.phase == 0 ? fa.ready0 + it.mt : fa.ready1 + it.nt, 1);
+                    if (it.phase == 0) {
+                        if (w != fa.fault_skip) {
+                            fence_proxy_async_global();
+                            red_release_gpu_add(fa.ready0 + it.mt, 1);
+                            red_release_gpu_add(fa.done0, 1);
+                        }
+                    } else {
+                        st_release_gpu(fa.ready1 + (size_t)it.nt * fa.max_tiles + it.mt, 1);
                     }
+                    trace_record(fa, it.phase == 0 ? TRACE_L0 : TRACE_L1, w, t_begin, globaltimer_ns());
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
             ++n;
         }
+        if (dm && !a_tma) cp_async_wait_all(); // this thread's copies land first
+        // combine: the data-movement warps from the end of their layer0 duties (beside the
+        // layer1 GEMM pipeline), the epilogue warps once this CTA's GEMM items are done
+        // (each group of four warps decides together whether to go on: named barrier 2 for
+        // the data-movement warps, 3 for the epilogue warps)
+        volatile int *slots = reinterpret_cast<volatile int *>(warps_done + 4);
+        const int bar = dm ? 2 : 3;
+        if (named_bar_and(bar, 128, ok))
+            combine_queue(fa, dm ? warp - 6 : warp - 2, lane, bar, slots + (dm ? 0 : 1), abort_flag,
+                          status);
     }
-
     __syncwarp();
     tc_fence_before();
     __syncthreads();

@@ -34,6 +34,9 @@ std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fault_skip{-1};
 // router variant for many experts: MOE_ROUTER_AUTO (tensor-core filter) or sequential only
 std::atomic<int> g_router_mode{MOE_ROUTER_AUTO};
+// optional schedule trace of the fused launch (device buffer and its record capacity)
+std::atomic<unsigned long long *> g_trace{nullptr};
+std::atomic<int64_t> g_trace_cap{0};
 // grouped-GEMM work order (MOE_ORDER_*; test and tuning hook)
 std::atomic<int> g_order{MOE_ORDER_NARROW};
 
@@ -169,7 +172,9 @@ Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd
     L.hot_off = take((E + 1) * 4);
     L.hot_tile_expert = take((size_t)L.max_tiles * 4);
     L.cold_tile = take(E * 4);
-    L.n_ready = L.max_tiles + (int)((H + 255) / 256); // fused kernel: per M tile, per stripe
+    // fused kernel: a counter per M tile (layer0), a flag per (stripe, M tile) (layer1), the
+    // count of finished layer0 items and the combine queue's next item
+    L.n_ready = L.max_tiles * (1 + (int)((H + 255) / 256)) + 2;
     L.ready = take((size_t)L.n_ready * 4);
     L.gather_idx = take(P * 4);
     L.inv_pos = take(T * K * 4);
@@ -765,8 +770,8 @@ cudaError_t launch_gemm_any(const CUtensorMap &ta, const CUtensorMap &tb, const 
 }
 
 template <int KIND0>
-cudaError_t launch_fused(const CUtensorMap &w1, const CUtensorMap &hm, const CUtensorMap &w2,
-                         const FusedArgs &fa, int max_work, cudaStream_t st)
+cudaError_t launch_fused(const CUtensorMap &a0, const CUtensorMap &w1, const CUtensorMap &hm,
+                         const CUtensorMap &w2, const FusedArgs &fa, int max_work, cudaStream_t st)
 {
     auto kern = moe_fused_layer_kernel<KIND0>;
     cudaError_t err =
@@ -777,7 +782,7 @@ cudaError_t launch_fused(const CUtensorMap &w1, const CUtensorMap &hm, const CUt
     if (grid <= 0) grid = 148;
     if (grid > max_work) grid = max_work;
     if (grid < 1) grid = 1;
-    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(w1, hm, w2, fa);
+    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(a0, w1, hm, w2, fa);
     return cudaGetLastError();
 }
 
@@ -893,6 +898,42 @@ bool use_x_perm(const moe_problem *p)
     return (int64_t)p->T * p->top_k >= (int64_t)p->E * M_TILE;
 }
 
+// Per-shape plan of the layer's GEMM and combine work (Comet §3.2.2: the split between
+// data-movement and compute work is chosen per shape). `fused`: one persistent launch in
+// which each SM's four data-movement warps first serve layer0 (row gather or half of each
+// epilogue) and then run the combine beside the layer1 GEMM pipeline; otherwise three
+// launches (layer0, layer1, combine). `comb_tokens`: tokens per combine item.
+// Why the rule: layer1 runs expert-major (each expert's h rows stay in L2 across its 256-
+// column stripes), so a combine item can start only when the last expert its tokens touch
+// has stored that stripe; the window in which the combine overlaps layer1 is about 1/E of
+// layer1. Timed on one B200 (alternating launches, 20 layers each, under the power cap):
+//   E = 8  (Mixtral-shaped): 5.19 ms persistent against 5.26 ms separate, and in one staged
+//          run 4.61 against 4.73 ms for the three stages (combine 99.8% hidden);
+//   E = 16 (Phi-3.5-shaped): 5.08 against 4.67 ms; E = 64 (Qwen2-shaped): 4.36 against
+//          3.57 ms; E = 256 (skewed): 4.89 against 4.63 ms -- the combine waits for the last
+//          experts and runs exposed on eight warps per SM, and the longer full-power launch
+//          settles at a lower clock.
+// So the persistent launch is taken for large batches with at most 8 experts; decode-sized
+// batches (single-tile experts) keep the separate launches and their operand-swapped body.
+struct FusedPlan {
+    bool fused;
+    int comb_tokens;
+};
+
+FusedPlan fused_plan(const moe_problem *p)
+{
+    FusedPlan f;
+    f.fused = use_x_perm(p) && p->E <= 8;
+    f.comb_tokens = p->T >= 2048 ? COMBINE_TOKENS : 64;
+    return f;
+}
+
+bool run_fused(const moe_problem *p)
+{
+    const int mode = g_gemm_mode.load();
+    return mode == MOE_GEMM_FUSED || (mode == MOE_GEMM_AUTO && fused_plan(p).fused);
+}
+
 moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
@@ -938,7 +979,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     // the single-CTA kernel), or gathered from x inside the kernel by cp.async warps (decode-
     // sized batches, whose padded rows would be mostly zeros, and the fused launch)
     const bool pair = (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR);
-    const bool xperm = pair || (g_gemm_mode.load() != MOE_GEMM_FUSED && use_x_perm(p));
+    const bool fused = !pair && run_fused(p);
+    const bool xperm = pair || use_x_perm(p);
     const bool a_ok = xperm ? make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM)
                             : make_map_2d(&m_x, x, (uint64_t)p->T, (uint64_t)H, 1);
     if (!a_ok ||
@@ -1004,13 +1046,17 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
                           status, timeout, st);
     }
 
-    if (g_gemm_mode.load() == MOE_GEMM_FUSED) {
+    if (fused) {
         // one persistent launch: layer0 -> layer1 -> combine, tile-level ready flags
+        const FusedPlan plan = fused_plan(p);
         FusedArgs fa{};
         fa.l0 = a0;
         fa.l1 = a1;
         fa.ready0 = d.ready;
         fa.ready1 = d.ready + L.max_tiles;
+        fa.done0 = d.ready + L.n_ready - 2;
+        fa.comb_next = d.ready + L.n_ready - 1;
+        fa.max_tiles = L.max_tiles;
         fa.inv_pos = d.inv_pos;
         fa.out = reinterpret_cast<__nv_bfloat16 *>(out);
         fa.T = p->T;
@@ -1018,12 +1064,17 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         fa.k = p->top_k;
         fa.ys_rows = L.pmax;
         fa.ys_shared = reinterpret_cast<const __nv_bfloat16 *>(ys_s);
+        fa.a_tma = xperm ? 1 : 0;
+        fa.comb_tokens = plan.comb_tokens;
         fa.fault_skip = g_fault_skip.load();
-        const int max_work = L.max_tiles * (a0.n_tiles + a1.n_tiles) +
-                             a1.n_tiles * ((p->T + COMBINE_TOKENS - 1) / COMBINE_TOKENS);
+        fa.trace = g_trace.load();
+        fa.trace_cap = g_trace_cap.load();
+        const int max_work = L.max_tiles * (a0.n_tiles + a1.n_tiles);
         if (e == cudaSuccess) {
-            e = gated ? launch_fused<GEMM_SWIGLU>(m_w1, m_h, m_w2, fa, max_work, st)
-                      : launch_fused<GEMM_ACT>(m_w1, m_h, m_w2, fa, max_work, st);
+            // (a0.epi8 is for the separate launches; the fused kernel splits layer0's epilogue
+            // itself when its rows come by TMA)
+            e = gated ? launch_fused<GEMM_SWIGLU>(m_x, m_w1, m_h, m_w2, fa, max_work, st)
+                      : launch_fused<GEMM_ACT>(m_x, m_w1, m_h, m_w2, fa, max_work, st);
         }
         // the three stages share one launch: their boundaries coincide at its end
         for (int i = 3; i < 6 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
@@ -1435,11 +1486,12 @@ int moe_forward_launches(const moe_problem *p)
     // count, scan, place; one block for a single chunk of tokens
     const int dispatch = p->T <= DISPATCH_CHUNK ? 1 : 3;
     const int mode = g_gemm_mode.load();
-    // layer0, layer1, combine; + the x_perm gather for CTA pairs and large batches
-    const int layers = mode == MOE_GEMM_FUSED                              ? 1
-                       : (mode == MOE_GEMM_CTA_PAIR || use_x_perm(p)) ? 4
-                                                                       : 3;
-    return route + dispatch + layers;
+    const bool pair = mode == MOE_GEMM_CTA_PAIR;
+    // + the x_perm gather (CTA pairs, large batches); then layer0, layer1, combine, or the one
+    // persistent launch
+    const int gather = (pair || use_x_perm(p)) ? 1 : 0;
+    const int layers = (!pair && run_fused(p)) ? 1 : 3;
+    return route + dispatch + gather + layers;
 }
 
 size_t moe_workspace_size(const moe_problem *p)
@@ -1856,6 +1908,14 @@ moe_status moe_backward(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
 {
     return backward_impl(p, x, Wg, bias, W1, W2, dout, dx, dWg, dbias, dW1, dW2, ws, ws_bytes,
                          static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_set_schedule_trace(void *records, int64_t capacity)
+{
+    if (capacity < 0) return MOE_ERR_INVALID_ARG;
+    g_trace_cap.store(records == nullptr ? 0 : capacity);
+    g_trace.store(static_cast<unsigned long long *>(records));
+    return MOE_OK;
 }
 
 int moe_set_fault_injection(int layer0_item)

@@ -84,6 +84,8 @@ def test_host_side_argument_checks(lib):
                          moe.moe_workspace_size(good), None) == -1
     assert lib.moe_route_noalloc(ctypes.byref(good), fake, off, None, fake, fake, None) == -1
     assert lib.moe_get_device_status(None, None) == -1
+    assert lib.moe_set_schedule_trace(None, -1) == -1
+    assert lib.moe_set_schedule_trace(None, 0) == 0
     assert lib.moe_status_string(-5) == b"MOE_ERR_DEVICE_TIMEOUT"
 
 
@@ -110,23 +112,30 @@ def test_forward_launch_count_follows_the_modes(lib):
         # router 1 (up to 32 experts, E % 8 == 0), 2 (more experts, sequential) or 3 (the
         # filter) + dispatch 3 (1 for T <= 256) + [x gather] + layer0, layer1, combine; the
         # bench layers gather x into sorted rows (T * k >= 128 E)
-        assert moe.moe_forward_launches(mixtral) == 8   # E = 8: one-launch router
+        # large batches (T*k >= 128 E) gather x into sorted rows and take the persistent
+        # launch: router + dispatch 3 + gather + 1
+        # (E <= 8: the persistent launch)
+        assert moe.moe_forward_launches(mixtral) == 6   # E = 8: one-launch router
         assert moe.moe_forward_launches(qwen2) == 10    # T*E >= 2^16: filter router
-        assert moe.moe_forward_launches(decode) == 6    # T*E < 2^16: sequential, no gather
+        assert moe.moe_forward_launches(decode) == 6    # T*E < 2^16: sequential, three layers
         phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
         assert moe.moe_forward_launches(phi35) == 10    # E = 16: filter router
         moe.moe_set_router_mode(moe.ROUTER_FILTER)
         assert moe.moe_forward_launches(decode) == 7
-        assert moe.moe_forward_launches(mixtral) == 10  # forced: E = 8 qualifies
+        assert moe.moe_forward_launches(mixtral) == 8   # forced: E = 8 qualifies
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
         assert moe.moe_forward_launches(phi35) == 8     # E = 16: one-launch router
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         assert moe.moe_forward_launches(qwen2) == 9
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED)           # forced: the persistent launch
+        assert moe.moe_forward_launches(qwen2) == 7
+        moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)      # three layer launches
+        assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside
         assert moe.moe_forward_launches(qwen2) == 9
-        moe.moe_set_gemm_mode(moe.GEMM_FUSED)           # gathers in the kernel
-        assert moe.moe_forward_launches(qwen2) == 6
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED)           # forced on a decode batch: no gather
+        assert moe.moe_forward_launches(decode) == 4
         moe.moe_set_gemm_mode(moe.GEMM_CTA_PAIR)        # gathers x; no narrow launches
         assert moe.moe_forward_launches(qwen2) == 9
         assert moe.moe_forward_launches(decode) == 7

@@ -27,8 +27,11 @@ def _forward(cfg, d, ws):
     return out, moe.moe_get_device_status(ws)
 
 
-def test_withheld_ready_signal_times_out_and_context_recovers():
-    cfg = synth.LayerConfig("fault", T=300, H=256, F=256, E=8, k=2)
+# T*k < 128 E: layer0 rows gathered in the kernel; T*k >= 128 E: sorted rows by TMA, and the
+# data-movement warps take half of each layer0 epilogue before the combine
+@pytest.mark.parametrize("T,E", [(300, 8), (700, 4)], ids=["gathered_rows", "sorted_rows"])
+def test_withheld_ready_signal_times_out_and_context_recovers(T, E):
+    cfg = synth.LayerConfig("fault", T=T, H=256, F=256, E=E, k=2)
     inp = synth.make_inputs(cfg, seed=21)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     ws = torch.empty(moe.moe_workspace_size(moe.Problem.from_config(cfg)), dtype=torch.uint8,
