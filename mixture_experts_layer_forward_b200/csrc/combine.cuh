@@ -21,12 +21,13 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const __nv_bfloat16 *__restrict__ ys, int64_t ys_rows,
                    const int32_t *__restrict__ inv_pos, int T, int H, int k,
                    __nv_bfloat16 *__restrict__ out, int *status, int clear_status,
-                   const __nv_bfloat16 *__restrict__ ys_shared)
+                   const __nv_bfloat16 *__restrict__ ys_shared, const int *__restrict__ n_rows)
 {
     if (clear_status && status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
         status[0] = DEV_OK;
         status[1] = 0;
     }
+    if (n_rows != nullptr) T = min(T, *n_rows); // output rows past *n_rows are left untouched
     const int vec_per_row = H / 8;
     const int64_t total = (int64_t)T * vec_per_row;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;

@@ -36,7 +36,8 @@ struct DispatchMeta {
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
     dispatch_count_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
-                          int32_t *__restrict__ chunk_counts, int *status, int clear_status)
+                          int32_t *__restrict__ chunk_counts, int *status, int clear_status,
+                          const int *__restrict__ n_rows)
 {
     extern __shared__ int cnt[];
     if (clear_status && status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -46,7 +47,9 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     const int t = blockIdx.x * DISPATCH_CHUNK + threadIdx.x;
-    if (t < T) {
+    // n_rows (optional, device): only tokens t < *n_rows are routed
+    const int Tn = n_rows != nullptr ? min(T, *n_rows) : T;
+    if (t < Tn) {
         for (int j = 0; j < k; ++j) {
             const int e = topk_idx[(size_t)t * k + j];
             if (e >= 0 && e < E) {
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
                           int T, int E, int k, const int32_t *__restrict__ chunk_base,
                           const int32_t *__restrict__ padded_offsets,
                           int32_t *__restrict__ gather_idx, int32_t *__restrict__ inv_pos,
-                          float *__restrict__ row_w)
+                          float *__restrict__ row_w, const int *__restrict__ n_rows)
 {
     extern __shared__ uint32_t bits[];
     for (int i = threadIdx.x; i < E * DISPATCH_WORDS; i += blockDim.x) bits[i] = 0u;
@@ -259,6 +262,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     const int t = blockIdx.x * DISPATCH_CHUNK + tl;
     const int word = tl >> 5;
     const uint32_t bit = 1u << (tl & 31);
+    T = n_rows != nullptr ? min(T, *n_rows) : T; // tokens past *n_rows are not routed
     if (t < T) {
         for (int j = 0; j < k; ++j) {
             const int e = topk_idx[(size_t)t * k + j];
@@ -271,13 +275,13 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
                          chunk_base + (size_t)blockIdx.x * E, gather_idx, inv_pos, row_w);
 }
 
-// T <= DISPATCH_CHUNK: count, scan and place in one block of 1024 threads (thread t < T owns
-// token t in the count and place steps, thread e expert e in the scan), with the outputs of
-// the three-kernel path. Dynamic shared memory: E * (DISPATCH_WORDS + 1) uint32.
+// T <= DISPATCH_CHUNK: count, scan and place in one block of 1024 threads (the threads stride
+// over the T * k (token, selection) pairs in the count and place steps; thread e owns expert
+// e in the scan), with the outputs of the three-kernel path. Dynamic shared memory: E * (DISPATCH_WORDS + 1) uint32.
 __global__ void __launch_bounds__(1024)
     dispatch_small_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
                           int T, int E, int k, ScanOut o, int32_t *__restrict__ inv_pos,
-                          int *status, int clear_status)
+                          int *status, int clear_status, const int *__restrict__ n_rows)
 {
     extern __shared__ uint32_t sm_words[];
     uint32_t *bits = sm_words;                                        // [E][DISPATCH_WORDS]
@@ -292,27 +296,42 @@ __global__ void __launch_bounds__(1024)
     for (int i = threadIdx.x; i < E * DISPATCH_WORDS; i += blockDim.x) bits[i] = 0u;
     for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
-    const int t = threadIdx.x;
-    if (t < T) {
-        for (int j = 0; j < k; ++j) {
-            const int e = topk_idx[(size_t)t * k + j];
-            if (e >= 0 && e < E) {
-                atomicAdd(&cnt[e], 1);
-                atomicOr(&bits[e * DISPATCH_WORDS + (t >> 5)], 1u << (t & 31));
-            } else {
-                record_status(status, DEV_BAD_INDEX, 1);
-            }
-            if (k <= 16) {
-                for (int j2 = 0; j2 < j; ++j2)
-                    if (topk_idx[(size_t)t * k + j2] == e) record_status(status, DEV_BAD_INDEX, 2);
-            }
+    // One (token, selection) pair per thread and step, so that the pairs' loads are
+    // independent. A token's experts must be distinct: a pair that finds its (expert, token)
+    // bit already set is a repeat.
+    const int P = (n_rows != nullptr ? min(T, *n_rows) : T) * k; // tokens past *n_rows: not routed
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+        const int t = q / k;
+        const int e = topk_idx[q];
+        if (e >= 0 && e < E) {
+            atomicAdd(&cnt[e], 1);
+            const uint32_t bit = 1u << (t & 31);
+            if (atomicOr(&bits[e * DISPATCH_WORDS + (t >> 5)], bit) & bit)
+                record_status(status, DEV_BAD_INDEX, 2);
+        } else {
+            record_status(status, DEV_BAD_INDEX, 1);
         }
     }
     __syncthreads();
     dispatch_scan_body(threadIdx.x < E ? cnt[threadIdx.x] : 0, E, o, warp_sums, s_poff, s_cnt);
-    if (t < T)
-        dispatch_place_token(topk_idx, topk_w, t, t, E, k, bits, s_poff, nullptr, o.gather_idx,
-                             inv_pos, o.row_w);
+    // placement of each pair: its row is the expert's padded offset plus the number of
+    // earlier tokens of the expert (ascending token order within the expert)
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+        const int t = q / k;
+        const int e = topk_idx[q];
+        if (e < 0 || e >= E) {
+            inv_pos[q] = -1;
+            continue;
+        }
+        const uint32_t *b = bits + e * DISPATCH_WORDS;
+        const int word = t >> 5;
+        int rank = __popc(b[word] & ((1u << (t & 31)) - 1u));
+        for (int w = 0; w < word; ++w) rank += __popc(b[w]);
+        const int r = s_poff[e] + rank;
+        o.gather_idx[r] = t;
+        inv_pos[q] = r;
+        if (o.row_w != nullptr) o.row_w[r] = topk_w[q];
+    }
 }
 
 // x_perm[r][:] = x[gather_idx[r]][:] (zeros on pad rows), for r < P_pad. One warp per row.
