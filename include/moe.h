@@ -292,6 +292,64 @@ MOE_API moe_status moe_experts_forward(const moe_problem *p, const moe_bf16 *x,
                                        const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                                        void *ws, size_t ws_bytes, void *stream);
 
+/* moe_experts_forward on the first *n_rows of its T rows, where n_rows is a device int32
+ * read by the kernels (the host never reads it): the count of rows a rank received in the
+ * device-driven expert-parallel exchange. Rows t >= *n_rows are not routed and their output
+ * rows are left untouched; p->T is the capacity (sizes the workspace and the launches).
+ * Always the separate launches (layer0, layer1, a k = 1 combine). Otherwise as
+ * moe_experts_forward. */
+MOE_API moe_status moe_experts_forward_n(const moe_problem *p, const moe_bf16 *x,
+                                         const int32_t *expert, const float *gate,
+                                         const int32_t *n_rows, const moe_bf16 *W1,
+                                         const moe_bf16 *W2, moe_bf16 *out, void *ws,
+                                         size_t ws_bytes, void *stream);
+
+/* Expert parallelism with the exchange driven by the device (Comet: Fine-grained
+ * Computation-communication Overlapping for Mixture-of-Experts, §2.1, §3.1: the routed
+ * tokens travel to their experts' GPU and the outputs back; §4: the GPU issues the
+ * transfers). Rank r of `world` holds experts [r * E / world, (r + 1) * E / world). Every
+ * rank owns buffers that every rank can address (symmetric allocations): a counts table
+ * [world, world] int32, receive buffers rows [recv_cap, H] bf16, ids [recv_cap] int32,
+ * gates [recv_cap] fp32, origins [recv_cap] int64, and a return buffer [T * k, H] bf16. The
+ * pointer arguments `tables`, `rows`, `ids`, `gates`, `origin`, `back` are DEVICE arrays of
+ * `world` pointers (entry r: rank r's buffer as this GPU addresses it). The host never reads
+ * the routing. The caller synchronises the ranks between the steps (a barrier of all ranks
+ * on the stream, e.g. the symmetric-memory barrier):
+ *   1. moe_route and moe_dispatch on this rank's tokens (all E experts);
+ *   2. moe_ep_publish_counts: this rank's rows per destination (from `offsets`, the
+ *      dispatch's [E+1] unpadded offsets) into row `rank` of every rank's table;  -- barrier
+ *   3. moe_ep_scatter: every routed pair (t, j) goes, by stores into the destination's
+ *      buffers, to slot (rows lower ranks send there) + (its position among this rank's rows
+ *      for that destination, in the dispatch's expert-then-token order), with its local
+ *      expert id, gate and origin (rank << 32 | t * k + j); writes n_recv[0] = the rows this
+ *      rank receives (a device int);                                               -- barrier
+ *   4. moe_experts_forward_n on the receive buffers (E / world experts, k = 1, T = recv_cap,
+ *      n_rows = n_recv);
+ *   5. moe_ep_return: received row i goes to row (origin & 0xffffffff) of rank
+ *      (origin >> 32)'s return buffer;                                             -- barrier
+ *   6. moe_combine of the return buffer with inv_pos[t][j] = t * k + j.
+ * Every gated row is bitwise the row moe_forward computes on one GPU. Errors (an expert id
+ * outside [0, E), a slot past recv_cap, a bad origin) go to the status word of `ws`
+ * (moe_workspace_size of the scatter's problem; for moe_ep_return the workspace of the
+ * step-4 call) as MOE_ERR_DEVICE_BAD_INDEX. recv_cap >= world * T * min(k, E / world) holds
+ * every routing. The stores to other GPUs are plain stores; nothing loads another GPU's
+ * memory. */
+MOE_API moe_status moe_ep_publish_counts(const moe_problem *p, int32_t world, int32_t rank,
+                                         const int32_t *offsets, int32_t *const *tables,
+                                         void *stream);
+MOE_API moe_status moe_ep_scatter(const moe_problem *p, int32_t world, int32_t rank,
+                                  const moe_bf16 *x, const int32_t *topk_idx,
+                                  const float *topk_w, const int32_t *offsets,
+                                  const int32_t *padded_offsets, const int32_t *inv_pos,
+                                  const int32_t *table, moe_bf16 *const *rows,
+                                  int32_t *const *ids, float *const *gates,
+                                  int64_t *const *origin, int64_t recv_cap, int32_t *n_recv,
+                                  void *ws, size_t ws_bytes, void *stream);
+MOE_API moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y,
+                                 const int64_t *origin, const int32_t *n_recv, int64_t recv_cap,
+                                 moe_bf16 *const *back, int64_t back_rows, void *ws,
+                                 void *stream);
+
 /* Backward pass (training; beyond the pages, which describe the forward).
  * Given dout = dL/dout [T, H] bf16, the gradients of the layer moe_forward computes, with the
  * selection held fixed (it is piecewise constant) and the gates the softmax over the

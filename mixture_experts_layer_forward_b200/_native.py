@@ -101,6 +101,10 @@ def library() -> ctypes.CDLL:
             "moe_forward_fp8_staged": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                         ctypes.POINTER(vp), i32], i32),
             "moe_experts_forward": ([P] + [vp] * 7 + [sz, vp], i32),
+            "moe_experts_forward_n": ([P] + [vp] * 8 + [sz, vp], i32),
+            "moe_ep_publish_counts": ([P, i32, i32, vp, vp, vp], i32),
+            "moe_ep_scatter": ([P, i32, i32] + [vp] * 11 + [i64, vp, vp, sz, vp], i32),
+            "moe_ep_return": ([i32, i32, vp, vp, vp, i64, vp, i64, vp, vp], i32),
             "moe_backward_workspace_size": ([P], sz),
             "moe_backward": ([P] + [vp] * 12 + [sz, vp], i32),
             "moe_combine": ([P, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -368,6 +372,58 @@ def moe_experts_forward(p, x, expert, gate, W1, W2, out, ws, stream=None):
                                        _ptr(W2, bf, "W2"), _ptr(out, bf, "out"), w, n,
                                        _stream(stream))
     _check("moe_experts_forward", rc)
+
+
+def moe_experts_forward_n(p, x, expert, gate, n_rows, W1, W2, out, ws, stream=None):
+    """moe_experts_forward on the first n_rows[0] rows (n_rows: a CUDA int32 tensor read on
+    the device); rows past it are not computed and their output rows are left untouched."""
+    bf = torch.bfloat16
+    w, n = _ws(ws)
+    rc = library().moe_experts_forward_n(ctypes.byref(p), _ptr(x, bf, "x"),
+                                         _ptr(expert, torch.int32, "expert"),
+                                         _ptr(gate, torch.float32, "gate"),
+                                         _ptr(n_rows, torch.int32, "n_rows"), _ptr(W1, bf, "W1"),
+                                         _ptr(W2, bf, "W2"), _ptr(out, bf, "out"), w, n,
+                                         _stream(stream))
+    _check("moe_experts_forward_n", rc)
+
+
+def moe_ep_publish_counts(p, world, rank, offsets, tables, stream=None):
+    """Row `rank` of every rank's counts table (tables: CUDA int64 tensor of world device
+    addresses) = this rank's rows per destination, from the dispatch's [E+1] offsets."""
+    rc = library().moe_ep_publish_counts(ctypes.byref(p), int(world), int(rank),
+                                         _ptr(offsets, torch.int32, "offsets"),
+                                         _ptr(tables, torch.int64, "tables"), _stream(stream))
+    _check("moe_ep_publish_counts", rc)
+
+
+def moe_ep_scatter(p, world, rank, x, topk_idx, topk_w, offsets, padded_offsets, inv_pos, table,
+                   rows, ids, gates, origin, recv_cap, n_recv, ws, stream=None):
+    """Stores every routed pair of this rank into its destination's receive buffers (the
+    address arguments rows / ids / gates / origin: CUDA int64 tensors of world device
+    addresses); n_recv[0] = rows this rank receives."""
+    i64 = torch.int64
+    w, n = _ws(ws)
+    rc = library().moe_ep_scatter(
+        ctypes.byref(p), int(world), int(rank), _ptr(x, torch.bfloat16, "x"),
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(padded_offsets, torch.int32, "padded_offsets"),
+        _ptr(inv_pos, torch.int32, "inv_pos"), _ptr(table, torch.int32, "table"),
+        _ptr(rows, i64, "rows"), _ptr(ids, i64, "ids"), _ptr(gates, i64, "gates"),
+        _ptr(origin, i64, "origin"), int(recv_cap), _ptr(n_recv, torch.int32, "n_recv"), w, n,
+        _stream(stream))
+    _check("moe_ep_scatter", rc)
+
+
+def moe_ep_return(H, world, y, origin, n_recv, recv_cap, back, back_rows, ws, stream=None):
+    """Stores each received row's expert output into its origin rank's return buffer (back:
+    CUDA int64 tensor of world device addresses)."""
+    rc = library().moe_ep_return(int(H), int(world), _ptr(y, torch.bfloat16, "y"),
+                                 _ptr(origin, torch.int64, "origin"),
+                                 _ptr(n_recv, torch.int32, "n_recv"), int(recv_cap),
+                                 _ptr(back, torch.int64, "back"), int(back_rows),
+                                 _ptr(ws, torch.uint8, "ws"), _stream(stream))
+    _check("moe_ep_return", rc)
 
 
 def moe_backward_workspace_size(p: Problem) -> int:

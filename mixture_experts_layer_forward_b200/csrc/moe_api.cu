@@ -13,6 +13,7 @@
 #include "backward.cuh"
 #include "combine.cuh"
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "fp8.cuh"
 #include "fused.cuh"
 #include "route_chain.cuh"
@@ -567,7 +568,7 @@ struct DispatchOut {
 
 cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t *topk_idx,
                             const float *topk_w, const DispatchOut &o, int *status, int clear_status,
-                            cudaStream_t st)
+                            cudaStream_t st, const int32_t *n_rows = nullptr)
 {
     const int T = p->T, E = p->E, k = p->top_k;
     const int nchunk = L.nchunk;
@@ -591,7 +592,7 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     so.active_list = o.active_list;
     if (nchunk == 1) { // one chunk of tokens: the three steps in one block
         dispatch_small_kernel<<<1, 1024, (size_t)E * (DISPATCH_WORDS + 1) * 4, st>>>(
-            topk_idx, topk_w, T, E, k, so, o.inv_pos, status, clear_status);
+            topk_idx, topk_w, T, E, k, so, o.inv_pos, status, clear_status, n_rows);
         return cudaGetLastError();
     }
     cudaError_t err = cudaSuccess;
@@ -603,7 +604,7 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     }
     if (nchunk > 0) {
         dispatch_count_kernel<<<nchunk, DISPATCH_CHUNK, E * sizeof(int), st>>>(
-            topk_idx, T, E, k, o.chunk, status, clear_status);
+            topk_idx, T, E, k, o.chunk, status, clear_status, n_rows);
     }
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -612,7 +613,7 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     if (err != cudaSuccess) return err;
     if (nchunk > 0) {
         dispatch_place_kernel<<<nchunk, DISPATCH_CHUNK, (size_t)E * DISPATCH_WORDS * 4, st>>>(
-            topk_idx, topk_w, T, E, k, o.chunk, o.poff, o.gather_idx, o.inv_pos, o.row_w);
+            topk_idx, topk_w, T, E, k, o.chunk, o.poff, o.gather_idx, o.inv_pos, o.row_w, n_rows);
     }
     return cudaGetLastError();
 }
@@ -629,7 +630,8 @@ cudaError_t launch_gather(const moe_problem *p, const moe_bf16 *x, const int32_t
 
 cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_rows,
                            const int32_t *inv_pos, moe_bf16 *out, int *status, int clear_status,
-                           cudaStream_t st, const moe_bf16 *ys_shared = nullptr)
+                           cudaStream_t st, const moe_bf16 *ys_shared = nullptr,
+                           const int32_t *n_rows = nullptr)
 {
     const int64_t vecs = (int64_t)p->T * (p->H / 8);
     int64_t blocks = (vecs + 255) / 256;
@@ -641,7 +643,7 @@ cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_
     kern<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows, inv_pos,
                                       p->T, p->H, p->top_k, reinterpret_cast<__nv_bfloat16 *>(out),
                                       status, clear_status,
-                                      reinterpret_cast<const __nv_bfloat16 *>(ys_shared));
+                                      reinterpret_cast<const __nv_bfloat16 *>(ys_shared), n_rows);
     return cudaGetLastError();
 }
 
@@ -939,7 +941,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                         cudaStream_t st, void *const *events, int n_events,
                         const moe_shared_expert *sh = nullptr,
-                        const int32_t *given_idx = nullptr, const float *given_w = nullptr)
+                        const int32_t *given_idx = nullptr, const float *given_w = nullptr,
+                        const int32_t *n_rows = nullptr)
 {
     moe_status s = check_problem(p);
     if (s != MOE_OK) return s;
@@ -979,7 +982,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     // the single-CTA kernel), or gathered from x inside the kernel by cp.async warps (decode-
     // sized batches, whose padded rows would be mostly zeros, and the fused launch)
     const bool pair = (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR);
-    const bool fused = !pair && run_fused(p);
+    const bool fused = !pair && n_rows == nullptr && run_fused(p);
     const bool xperm = pair || use_x_perm(p);
     const bool a_ok = xperm ? make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM)
                             : make_map_2d(&m_x, x, (uint64_t)p->T, (uint64_t)H, 1);
@@ -997,7 +1000,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
                          &fb);
     if (e == cudaSuccess) e = record(events, n_events, 1, st);
     // with the routing supplied the dispatch clears the status word (and checks the ids)
-    if (e == cudaSuccess) e = launch_dispatch(p, L, topk_idx, topk_w, d, status, given ? 1 : 0, st);
+    if (e == cudaSuccess)
+        e = launch_dispatch(p, L, topk_idx, topk_w, d, status, given ? 1 : 0, st, n_rows);
     if (e == cudaSuccess && xperm) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
     if (e == cudaSuccess) e = record(events, n_events, 2, st);
 
@@ -1111,7 +1115,8 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
             e = launch_gemm_any<GEMM_SCALE>(m_h, m_w2, a1, L.max_tiles * a1.n_tiles, st);
         if (e == cudaSuccess) e = record(events, n_events, 4, st);
     }
-    if (e == cudaSuccess) e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, ys_s);
+    if (e == cudaSuccess)
+        e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, ys_s, n_rows);
     if (e == cudaSuccess) e = record(events, n_events, 5, st);
     return to_status(e);
 }
@@ -1893,6 +1898,105 @@ moe_status moe_experts_forward(const moe_problem *p, const moe_bf16 *x, const in
     return forward_impl(p, x, nullptr, nullptr, W1, W2, out, nullptr, nullptr, ws, ws_bytes,
                         static_cast<cudaStream_t>(stream), nullptr, 0, nullptr,
                         p != nullptr && p->T > 0 ? expert : nullptr, gate);
+}
+
+moe_status moe_experts_forward_n(const moe_problem *p, const moe_bf16 *x, const int32_t *expert,
+                                 const float *gate, const int32_t *n_rows, const moe_bf16 *W1,
+                                 const moe_bf16 *W2, moe_bf16 *out, void *ws, size_t ws_bytes,
+                                 void *stream)
+{
+    if (p != nullptr && p->top_k != 1) return MOE_ERR_INVALID_ARG;
+    if (p != nullptr && p->T > 0 &&
+        (expert == nullptr || gate == nullptr || n_rows == nullptr || !aligned4(expert) ||
+         !aligned4(gate) || !aligned4(n_rows)))
+        return MOE_ERR_INVALID_ARG;
+    return forward_impl(p, x, nullptr, nullptr, W1, W2, out, nullptr, nullptr, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), nullptr, 0, nullptr,
+                        p != nullptr && p->T > 0 ? expert : nullptr, gate,
+                        p != nullptr && p->T > 0 ? n_rows : nullptr);
+}
+
+moe_status moe_ep_publish_counts(const moe_problem *p, int32_t world, int32_t rank,
+                                 const int32_t *offsets, int32_t *const *tables, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (world < 1 || rank < 0 || rank >= world || p->E % world != 0 || offsets == nullptr ||
+        tables == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    ep_publish_counts_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        offsets, p->E / world, world, rank, tables);
+    return to_status(cudaGetLastError());
+}
+
+moe_status moe_ep_scatter(const moe_problem *p, int32_t world, int32_t rank, const moe_bf16 *x,
+                          const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
+                          const int32_t *padded_offsets, const int32_t *inv_pos,
+                          const int32_t *table, moe_bf16 *const *rows, int32_t *const *ids,
+                          float *const *gates, int64_t *const *origin, int64_t recv_cap,
+                          int32_t *n_recv, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status s = check_problem(p);
+    if (s != MOE_OK) return s;
+    if (world < 1 || rank < 0 || rank >= world || p->E % world != 0 || recv_cap < 0 ||
+        (int64_t)p->T * p->top_k >= ((int64_t)1 << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (ws == nullptr || n_recv == nullptr || table == nullptr || rows == nullptr ||
+        ids == nullptr || gates == nullptr || origin == nullptr ||
+        (p->T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr ||
+                      offsets == nullptr || padded_offsets == nullptr || inv_pos == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(p);
+    if (ws_bytes < L.end_route) return MOE_ERR_WORKSPACE;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    EpScatterArgs a{};
+    a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.offsets = offsets;
+    a.poff = padded_offsets;
+    a.inv_pos = inv_pos;
+    a.table = table;
+    a.rows = reinterpret_cast<__nv_bfloat16 *const *>(rows);
+    a.ids = ids;
+    a.gates = gates;
+    a.origin = reinterpret_cast<long long *const *>(origin);
+    a.recv_cap = recv_cap;
+    a.n_recv = n_recv;
+    a.T = p->T;
+    a.H = p->H;
+    a.E = p->E;
+    a.k = p->top_k;
+    a.E_loc = p->E / world;
+    a.world = world;
+    a.rank = rank;
+    a.status = at<int>(ws, L.status);
+    const int64_t pairs = (int64_t)p->T * p->top_k;
+    int64_t blocks = (pairs * 32 + 255) / 256;
+    const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    ep_scatter_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return to_status(cudaGetLastError());
+}
+
+moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y, const int64_t *origin,
+                         const int32_t *n_recv, int64_t recv_cap, moe_bf16 *const *back,
+                         int64_t back_rows, void *ws, void *stream)
+{
+    if (H <= 0 || H % 64 != 0 || world < 1 || y == nullptr || origin == nullptr ||
+        n_recv == nullptr || back == nullptr || ws == nullptr || recv_cap < 0 || back_rows < 0 ||
+        !aligned16(y) || !aligned16(ws))
+        return MOE_ERR_INVALID_ARG;
+    int64_t blocks = (recv_cap * 32 + 255) / 256;
+    const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    ep_return_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(y), reinterpret_cast<const long long *>(origin),
+        n_recv, H, world, back_rows, reinterpret_cast<__nv_bfloat16 *const *>(back),
+        static_cast<int *>(ws));
+    return to_status(cudaGetLastError());
 }
 
 size_t moe_backward_workspace_size(const moe_problem *p)

@@ -17,7 +17,16 @@ tokens:
 
 bf16 rows cross the collectives as int32 words (the same bytes, two values per word, a
 dtype every backend carries). The exchange runs on NCCL between GPUs; the expert and combine
-steps are pluggable, so the plan is also exercised on CPU (gloo) by the tests.
+steps are pluggable, so the plan is also exercised on CPU (gloo) by the tests. NCCL's
+all-to-all needs the split sizes on the host, so step 3 reads the counts back (one device
+synchronisation per layer).
+
+ep_moe_forward_device is the same layer with the exchange driven by the device instead
+(csrc/ep.cuh): the counts, the row positions and the transfers stay on the GPU, the rows are
+stored straight into the destination's receive buffers (symmetric memory every rank can
+address), and the host never reads the routing; the ranks meet at device barriers between
+the steps. Not measured on several GPUs here (one GPU per run); its one-rank form is tested
+against moe_forward.
 """
 from __future__ import annotations
 
@@ -125,3 +134,91 @@ def ep_moe_forward(p, x, Wg, bias, W1_local, W2_local, group=None):
     moe.moe_route(p, x, Wg, bias, idx, w, ws)
     return ep_forward(x, idx, w, p.E, gpu_expert_fn(p.H, p.F, e_loc, W1_local, W2_local, p.act),
                       gpu_combine_fn(p.H, p.F, p.E, p.top_k), group)
+
+
+class DeviceExchange:
+    """Buffers of ep_moe_forward_device in symmetric memory (every rank can address every
+    rank's copy) and the device arrays of their per-rank addresses. One instance per layer
+    shape and process group; the ranks must create it in the same order (a collective)."""
+
+    def __init__(self, p, group=None, device=None):
+        import torch.distributed._symmetric_memory as symm_mem
+
+        from . import _native as moe
+
+        self.group = group if group is not None else dist.group.WORLD
+        self.world = dist.get_world_size(self.group)
+        self.rank = dist.get_rank(self.group)
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        e_loc = experts_per_rank(p.E, self.world)
+        self.p = p
+        self.e_loc = e_loc
+        # every rank sends each destination at most min(k, E_loc) rows per token
+        self.recv_cap = self.world * p.T * min(p.top_k, e_loc)
+        self.bufs = {}
+        self.handles = {}
+        self.addr = {}
+        for name, shape, dtype in (("table", (self.world * self.world,), torch.int32),
+                                   ("rows", (self.recv_cap, p.H), torch.bfloat16),
+                                   ("ids", (self.recv_cap,), torch.int32),
+                                   ("gates", (self.recv_cap,), torch.float32),
+                                   ("origin", (self.recv_cap,), torch.int64),
+                                   ("back", (p.T * p.top_k, p.H), torch.bfloat16)):
+            t = symm_mem.empty(*shape, dtype=dtype, device=dev)
+            h = symm_mem.rendezvous(t, self.group)
+            base = h.buffer_ptrs[self.rank]
+            off = t.data_ptr() - base
+            self.bufs[name] = t
+            self.handles[name] = h
+            self.addr[name] = torch.tensor([b + off for b in h.buffer_ptrs], dtype=torch.int64,
+                                           device=dev)
+        self.n_recv = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.recv_problem = moe.Problem.make(self.recv_cap, p.H, p.F, e_loc, 1, p.act)
+        self.ws_route = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device=dev)
+        self.ws_recv = torch.empty(moe.moe_workspace_size(self.recv_problem), dtype=torch.uint8,
+                                   device=dev)
+        self.y = torch.empty(self.recv_cap, p.H, dtype=torch.bfloat16, device=dev)
+        k = p.top_k
+        self.identity = torch.arange(p.T * k, dtype=torch.int32, device=dev).view(p.T, k)
+
+    def barrier(self, channel):
+        self.handles["table"].barrier(channel=channel)
+
+
+def ep_moe_forward_device(xch: DeviceExchange, x, Wg, bias, W1_local, W2_local):
+    """The whole layer under expert parallelism, exchange driven by the device (csrc/ep.cuh):
+    route and dispatch this rank's tokens, publish the counts, barrier, store the rows into
+    their destinations' buffers, barrier, run this rank's experts on the rows it received
+    (row count on the device), store the outputs back into their origins' return buffers,
+    barrier, combine. Returns out [T, H] bf16; no host read of the routing."""
+    from . import _native as moe
+
+    p = xch.p
+    dev = x.device
+    T, k, E = p.T, p.top_k, p.E
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    moe.moe_route(p, x, Wg, bias, idx, w, xch.ws_route)
+    pmax = moe.moe_padded_rows_max(p)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    poff = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    gather_idx = torch.empty(pmax, dtype=torch.int32, device=dev)
+    inv_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    moe.moe_dispatch(p, idx, counts, offsets, poff, gather_idx, inv_pos, xch.ws_route)
+    moe.moe_ep_publish_counts(p, xch.world, xch.rank, offsets, xch.addr["table"])
+    xch.barrier(0)
+    a = xch.addr
+    moe.moe_ep_scatter(p, xch.world, xch.rank, x, idx, w, offsets, poff, inv_pos,
+                       xch.bufs["table"], a["rows"], a["ids"], a["gates"], a["origin"],
+                       xch.recv_cap, xch.n_recv, xch.ws_route)
+    xch.barrier(1)
+    moe.moe_experts_forward_n(xch.recv_problem, xch.bufs["rows"], xch.bufs["ids"],
+                              xch.bufs["gates"], xch.n_recv, W1_local, W2_local, xch.y,
+                              xch.ws_recv)
+    moe.moe_ep_return(p.H, xch.world, xch.y, xch.bufs["origin"], xch.n_recv, xch.recv_cap,
+                      a["back"], T * k, xch.ws_recv)
+    xch.barrier(2)
+    out = torch.empty(T, p.H, dtype=torch.bfloat16, device=dev)
+    moe.moe_combine(p, xch.bufs["back"], xch.identity, out)
+    return out

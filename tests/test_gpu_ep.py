@@ -1,6 +1,9 @@
 """The expert-parallel building blocks on one GPU: moe_experts_forward reproduces the routed
-rows of moe_forward bit for bit, and ep.ep_moe_forward over a one-rank NCCL group equals
-moe_forward. The multi-rank exchange itself is tested on CPU (tests/test_ep_gloo.py)."""
+rows of moe_forward bit for bit, ep.ep_moe_forward over a one-rank NCCL group equals
+moe_forward, and so does the device-driven exchange (ep.ep_moe_forward_device: counts,
+positions and row transfers on the GPU, symmetric-memory buffers, device barriers) run by
+one rank, twice in a row on the same buffers. The multi-rank NCCL exchange plan is tested on
+CPU (tests/test_ep_gloo.py); several GPUs are not available to these tests."""
 import os
 
 import numpy as np
@@ -78,3 +81,50 @@ def test_ep_single_rank_equals_forward():
     finally:
         dist.destroy_process_group()
     assert torch.equal(got.view(torch.int16), out.view(torch.int16))
+
+
+def test_experts_forward_n_computes_only_the_counted_rows():
+    """moe_experts_forward_n with a device row count: the first n rows equal
+    moe_experts_forward on those rows, the rows past n are left untouched."""
+    T, n = 300, 173
+    cfg = synth.LayerConfig("rows_n", T=T, H=256, F=256, E=4, k=1)
+    inp = synth.make_inputs(cfg, seed=31, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(5)
+    ids = torch.randint(0, 4, (T,), generator=g, device="cuda", dtype=torch.int32)
+    gates = torch.rand(T, generator=g, device="cuda")
+    p = moe.Problem.make(T, 256, 256, 4, 1)
+    ws = torch.empty(moe.moe_workspace_size(p), dtype=torch.uint8, device="cuda")
+    y = torch.full((T, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    n_rows = torch.tensor([n], dtype=torch.int32, device="cuda")
+    moe.moe_experts_forward_n(p, inp["x"], ids, gates, n_rows, inp["W1"], inp["W2"], y, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    pn = moe.Problem.make(n, 256, 256, 4, 1)
+    wsn = torch.empty(moe.moe_workspace_size(pn), dtype=torch.uint8, device="cuda")
+    yn = torch.empty(n, 256, dtype=torch.bfloat16, device="cuda")
+    moe.moe_experts_forward(pn, inp["x"][:n].contiguous(), ids[:n].contiguous(),
+                            gates[:n].contiguous(), inp["W1"], inp["W2"], yn, wsn)
+    assert moe.moe_get_device_status(wsn) == 0
+    assert torch.equal(y[:n].view(torch.int16), yn.view(torch.int16))
+    assert bool(torch.all(y[n:] == 7.0))
+
+
+@pytest.mark.parametrize("T,E,k,zipf", [(500, 8, 2, 1.2), (96, 16, 4, 0.0)])
+def test_device_exchange_single_rank_equals_forward(T, E, k, zipf):
+    cfg = synth.LayerConfig("epd", T=T, H=256, F=256, E=E, k=k, zipf_s=zipf)
+    inp = synth.make_inputs(cfg, seed=6, device="cuda")
+    p, out, _, _ = _forward(cfg, inp)
+    port = 29800 + os.getpid() % 97
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        xch = ep.DeviceExchange(p)
+        got = [ep.ep_moe_forward_device(xch, inp["x"], inp["Wg"], inp["bias"], inp["W1"],
+                                        inp["W2"]) for _ in range(2)]
+        torch.cuda.synchronize()
+        st = (moe.moe_get_device_status(xch.ws_route), moe.moe_get_device_status(xch.ws_recv))
+        del xch
+    finally:
+        dist.destroy_process_group()
+    assert st == (0, 0)
+    for g in got:
+        assert torch.equal(g.view(torch.int16), out.view(torch.int16))
