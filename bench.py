@@ -692,7 +692,12 @@ def run_ours(args):
             "hidden_frac": 1.0 - fused_ms / sum_layers,
             "combine_ms": sep["combine"],
             "how": "layer0 + layer1 + combine as three launches (staged, same run) against the "
-                   "one persistent launch"}
+                   "one persistent launch",
+            # the layer0 grouped GEMM of the separate launches, for comparison with runs
+            # whose dominant kernel is that launch
+            "separate_layer0_roofline": layer0_roofline(
+                cfg, sep["layer0_gemm_swiglu"], active_experts, peaks, peak_src, clocks, False,
+                DOMINANT_KERNEL["single"])}
     if args.trace is not None and not args.fp8:
         line["schedule_trace"] = schedule_trace(torch, moe, fwd, dev, args.trace or None)
 

@@ -45,3 +45,52 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_do_no_work():
     assert run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_roofline_fractions_follow_the_sampled_clock():
+    """The tensor peak regime is read from the median sampled SM clock (burst at >= 0.9 of
+    the maximum, sustained below), and the line carries the burst and clock-scaled fractions
+    too, so each can be recomputed from the JSON line and the measured peaks."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+
+    peaks = {"hbm_gbs": 6520.2, "bf16_tflops": 1656.8, "bf16_tflops_sustained": 1388.7}
+    # a short run at the maximum clock, a few power-cap samples: burst
+    hot = {"sm_mhz": 1942.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    d = bench.tensor_fracs(1333.0, peaks, hot)
+    assert d["regime"] == "burst" and d["peak"] == 1656.8
+    assert abs(d["frac"] - 1333.0 / 1656.8) < 1e-12 and d["frac"] == d["frac_burst"]
+    assert abs(d["frac_clock_scaled"] - 1333.0 / (1656.8 * 1942.0 / 1965.0)) < 1e-12
+    # a long run settled under the cap: sustained
+    capped = {"sm_mhz": 1340.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    d = bench.tensor_fracs(1100.0, peaks, capped)
+    assert d["regime"] == "sustained" and d["peak"] == 1388.7
+    assert abs(d["frac_burst"] - 1100.0 / 1656.8) < 1e-12
+    # no clock record: burst, no clock-scaled figure
+    d = bench.tensor_fracs(1000.0, peaks, None)
+    assert d["regime"] == "burst" and "frac_clock_scaled" not in d
+    # e4m3: twice the bf16 figures
+    d = bench.tensor_fracs(2000.0, peaks, hot, fp8=True)
+    assert d["peak"] == 2 * 1656.8
+
+
+def test_layer0_roofline_bound_and_bytes():
+    """Separate launches: layer0's useful FLOPs 4TkHF (SwiGLU) and its algorithmic bytes; the
+    persistent launch: both GEMMs' FLOPs 6TkHF and the compulsory bytes."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from mixture_experts_layer_forward_b200 import synth
+
+    cfg = synth.CONFIGS["mixtral"]
+    peaks = {"hbm_gbs": 6520.2, "bf16_tflops": 1656.8, "bf16_tflops_sustained": 1388.7}
+    r = bench.layer0_roofline(cfg, 2.9, 8, peaks, "measured", None, False, "k")
+    T, k, H, F = cfg.T, cfg.k, cfg.H, cfg.F
+    assert r["algorithmic_flops_per_launch"] == 4 * T * k * H * F
+    assert r["algorithmic_bytes_per_launch"] == 2 * (8 * H * 2 * F + T * H) + 2 * T * k * F
+    assert r["bound"] == "tensor"
+    r = bench.layer0_roofline(cfg, 4.6, 8, peaks, "measured", None, False, "k", fused=True)
+    assert r["algorithmic_flops_per_launch"] == 6 * T * k * H * F
+    assert r["algorithmic_bytes_per_launch"] == 2 * (8 * H * 3 * F + T * k * H) + 2 * T * H
+    decode = synth.CONFIGS["skew_decode"]
+    r = bench.layer0_roofline(decode, 0.46, 49, peaks, "measured", None, False, "k")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
