@@ -106,14 +106,15 @@ typedef struct {
  * calls on one stream. 0 if *p is invalid. */
 MOE_API size_t moe_workspace_size(const moe_problem *p);
 
-/* Number of kernels one moe_forward (or moe_forward_staged) call on *p launches under the
- * current GEMM and router modes, assuming 16-byte aligned operands: the router (1 for up to
- * 32 experts when E is a multiple of 8, 3 with the tensor-core filter, else 2), the dispatch
- * (3; 1 for T <= 256), the gather of x into expert-sorted rows (1 when T * top_k >= E * 128,
- * and always for the CTA-pair GEMM) and the layers (layer0, layer1 and the combine: 3; or
- * 1 for the persistent launch that MOE_GEMM_FUSED forces and MOE_GEMM_AUTO picks for
- * T * top_k >= E * 128 with E <= 8).
- * 0 for T == 0; -1 if *p is invalid. */
+/* Number of kernels one moe_forward call on *p launches under the current GEMM and router
+ * modes, assuming 16-byte aligned operands: 1 for the whole-layer launch
+ * (moe_set_whole_layer_launch); otherwise the router (1 for up to 32 experts when E is a
+ * multiple of 8, 3 with the tensor-core filter, else 2), the dispatch (3; 1 for T <= 256),
+ * the gather of x into expert-sorted rows (1 when T * top_k >= E * 128, and always for the
+ * CTA-pair GEMM) and the layers (layer0, layer1 and the combine: 3; or 1 for the persistent
+ * launch that MOE_GEMM_FUSED forces and MOE_GEMM_AUTO picks for T * top_k >= E * 128 with
+ * E <= 8). moe_forward_staged never takes the whole-layer launch (its stage events need the
+ * stages' own launches). 0 for T == 0; -1 if *p is invalid. */
 MOE_API int moe_forward_launches(const moe_problem *p);
 
 /* Upper bound on the padded row count P_pad = sum_e ceil(c_e / m_tile) * m_tile, namely
@@ -440,6 +441,23 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
  * launch. */
 #define MOE_GEMM_FUSED 3
 MOE_API int moe_set_gemm_mode(int mode);
+
+/* Whole-layer launch (Comet §5.3: the small-batch gains come from taking the host-driven
+ * steps out of the layer; here the route and dispatch steps join the persistent launch).
+ * On by default. It applies when the persistent launch runs (MOE_GEMM_FUSED, or
+ * MOE_GEMM_AUTO's choice), E == 8, the layer's routing is computed (not supplied), the
+ * router is the one-launch exact router (not the tensor-core filter), no stage events are
+ * requested and x, W_g are 16-byte aligned. Every CTA of the persistent launch (one per SM)
+ * then first routes about T / SMs tokens and counts its selections per expert; the CTAs
+ * meet at a grid-wide barrier (a counter in the workspace's status block); each derives the
+ * experts' offsets, CTA 0 writes the dispatch outputs, and each places its own pairs
+ * (expert-major, ascending token order within an expert -- the rows of the separate
+ * dispatch) and copies their x rows into the expert-sorted buffer; after a second barrier
+ * the GEMM phases begin. moe_forward is then one kernel launch after one 32-byte memset of
+ * the status block. The outputs equal those of the separate launches bit for bit, except
+ * that pad rows of the expert-sorted copy of x are not written. on = 0 turns it off
+ * (routing and dispatch as their own launches). Returns the previous setting. */
+MOE_API int moe_set_whole_layer_launch(int on);
 
 /* Work order of the single-CTA grouped-GEMM launches (a tuning and test hook; not
  * thread-safe). An expert with a single m-tile ("cold": at most m_tile routed rows) has its

@@ -116,6 +116,7 @@ def library() -> ctypes.CDLL:
             "moe_set_schedule_trace": ([vp, i64], i32),
             "moe_set_router_mode": ([i32], i32),
             "moe_set_work_order": ([i32], i32),
+            "moe_set_whole_layer_launch": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -513,3 +514,9 @@ def moe_set_gemm_mode(mode: int) -> int:
     if rc < 0:
         raise ValueError(f"unknown GEMM mode {mode}")
     return rc
+
+
+def moe_set_whole_layer_launch(on: bool) -> bool:
+    """Routing and dispatch inside the persistent launch where it applies (on by default);
+    returns the previous setting."""
+    return bool(library().moe_set_whole_layer_launch(1 if on else 0))

@@ -109,6 +109,73 @@ struct ScanOut {
     int32_t *hot_off, *hot_tile_expert, *cold_tile, *active_list;
 };
 
+// Outputs of expert e (< E) from its routed rows c and the inclusive scans over experts of:
+// c, its m-tiles, its m-tile pairs, its m-tiles if it has two or more ("hot"), 1 if it has
+// exactly one ("cold"), 1 if it has rows. s_poff[e] receives the expert's padded row offset
+// and, from the last expert, s_poff[E] = P_pad.
+__device__ __forceinline__ void scan_write_expert(int e, int E, int c, int inc_c, int inc_t,
+                                                  int inc_p, int inc_h, int inc_1, int inc_a,
+                                                  const ScanOut &o, int *s_poff)
+{
+    const int ntile = (c + M_TILE - 1) / M_TILE;
+    const int nptile = (ntile + 1) / 2;
+    const int hot_t = ntile >= 2 ? ntile : 0;
+    if (o.counts != nullptr) o.counts[e] = c;
+    if (o.offsets != nullptr) {
+        o.offsets[e + 1] = inc_c;
+        if (e == 0) o.offsets[0] = 0;
+    }
+    const int poff_next = inc_t * M_TILE;
+    const int tile_first = inc_t - ntile;
+    o.padded_offsets[e + 1] = poff_next;
+    o.tile_off[e + 1] = inc_t;
+    if (e == 0) {
+        o.padded_offsets[0] = 0;
+        o.tile_off[0] = 0;
+    }
+    s_poff[e] = tile_first * M_TILE;
+    for (int i = 0; i < ntile; ++i) o.tile_expert[tile_first + i] = e;
+    if (o.ptile_off != nullptr) {
+        o.ptile_off[e + 1] = inc_p;
+        if (e == 0) o.ptile_off[0] = 0;
+        for (int i = 0; i < nptile; ++i) o.ptile_expert[inc_p - nptile + i] = e;
+    }
+    if (o.hot_off != nullptr) {
+        o.hot_off[e + 1] = inc_h;
+        if (e == 0) o.hot_off[0] = 0;
+        for (int i = 0; i < hot_t; ++i) o.hot_tile_expert[inc_h - hot_t + i] = e;
+        if (ntile == 1) o.cold_tile[inc_1 - 1] = tile_first;
+    }
+    if (o.active_list != nullptr && c > 0) o.active_list[inc_a - 1] = e; // ascending ids
+    if (e == E - 1) {
+        o.meta->num_tiles = inc_t;
+        o.meta->padded_rows = poff_next;
+        o.meta->num_ptiles = inc_p;
+        o.meta->num_cold = inc_1;
+        o.meta->num_active = inc_a;
+        s_poff[E] = poff_next;
+    }
+}
+
+// Pad rows of each expert (rows s_poff[e] + s_cnt[e] .. s_poff[e + 1]) and every row past
+// P_pad = s_poff[E]: gather_idx = -1, weight 0. Thread `tid` of `nt` (a multiple of 32): one
+// warp per expert, lanes on consecutive rows.
+__device__ __forceinline__ void scan_write_pads(int E, const ScanOut &o, const int *s_poff,
+                                                const int *s_cnt, int tid, int nt)
+{
+    for (int ex = tid >> 5; ex < E; ex += nt >> 5) {
+        const int end = s_poff[ex + 1];
+        for (int r = s_poff[ex] + s_cnt[ex] + (tid & 31); r < end; r += 32) {
+            o.gather_idx[r] = -1;
+            if (o.row_w != nullptr) o.row_w[r] = 0.0f;
+        }
+    }
+    for (int64_t r = (int64_t)s_poff[E] + tid; r < o.padded_rows_max; r += nt) {
+        o.gather_idx[r] = -1;
+        if (o.row_w != nullptr) o.row_w[r] = 0.0f;
+    }
+}
+
 // Everything derived from the per-expert row counts, by one block of 1024 threads in which
 // thread e owns expert e (c = its routed rows; E <= 1024). s_poff[0..E] receives the padded
 // row offsets, s_cnt[0..E-1] the counts. Ends with a block barrier.
@@ -118,78 +185,49 @@ __device__ __forceinline__ void dispatch_scan_body(int c, int E, const ScanOut &
     // the fused layer kernel's tile-level ready counters start from zero on every call
     for (int i = threadIdx.x; i < o.n_ready; i += blockDim.x) o.ready[i] = 0;
     const int e = threadIdx.x;
-    int32_t *const counts = o.counts, *const offsets = o.offsets;
-    int32_t *const padded_offsets = o.padded_offsets, *const tile_off = o.tile_off;
-    int32_t *const tile_expert = o.tile_expert, *const ptile_off = o.ptile_off;
-    int32_t *const ptile_expert = o.ptile_expert, *const hot_off = o.hot_off;
-    int32_t *const hot_tile_expert = o.hot_tile_expert, *const cold_tile = o.cold_tile;
-    int32_t *const active_list = o.active_list, *const gather_idx = o.gather_idx;
-    float *const row_w = o.row_w;
-    DispatchMeta *const meta = o.meta;
-    if (e < E && counts != nullptr) counts[e] = c;
     const int ntile = (c + M_TILE - 1) / M_TILE;
     const int inc_c = block_inclusive_scan_1024(c, warp_sums);
     const int inc_t = block_inclusive_scan_1024(ntile, warp_sums);
-    const int nptile = (ntile + 1) / 2;
-    const int inc_p = block_inclusive_scan_1024(nptile, warp_sums);
+    const int inc_p = block_inclusive_scan_1024((ntile + 1) / 2, warp_sums);
     // work classes of the grouped GEMMs: "cold" experts (one m-tile) stream their weights for
     // a single tile; the rest ("hot") reuse each weight tile across their m-tiles
-    const int hot_t = ntile >= 2 ? ntile : 0;
-    const int inc_h = block_inclusive_scan_1024(hot_t, warp_sums);
+    const int inc_h = block_inclusive_scan_1024(ntile >= 2 ? ntile : 0, warp_sums);
     const int inc_1 = block_inclusive_scan_1024(ntile == 1 ? 1 : 0, warp_sums);
     const int inc_a = block_inclusive_scan_1024(c > 0 ? 1 : 0, warp_sums);
     if (e < E) {
-        if (offsets != nullptr) {
-            offsets[e + 1] = inc_c;
-            if (e == 0) offsets[0] = 0;
-        }
-        const int poff_next = inc_t * M_TILE;
-        const int tile_first = inc_t - ntile;
-        padded_offsets[e + 1] = poff_next;
-        tile_off[e + 1] = inc_t;
-        if (e == 0) {
-            padded_offsets[0] = 0;
-            tile_off[0] = 0;
-        }
-        s_poff[e] = tile_first * M_TILE;
-        for (int i = 0; i < ntile; ++i) tile_expert[tile_first + i] = e;
-        if (ptile_off != nullptr) {
-            ptile_off[e + 1] = inc_p;
-            if (e == 0) ptile_off[0] = 0;
-            for (int i = 0; i < nptile; ++i) ptile_expert[inc_p - nptile + i] = e;
-        }
-        if (hot_off != nullptr) {
-            hot_off[e + 1] = inc_h;
-            if (e == 0) hot_off[0] = 0;
-            for (int i = 0; i < hot_t; ++i) hot_tile_expert[inc_h - hot_t + i] = e;
-            if (ntile == 1) cold_tile[inc_1 - 1] = tile_first;
-        }
-        if (active_list != nullptr && c > 0) active_list[inc_a - 1] = e; // ascending ids
-        if (e == E - 1) {
-            meta->num_tiles = inc_t;
-            meta->padded_rows = poff_next;
-            meta->num_ptiles = inc_p;
-            meta->num_cold = inc_1;
-            meta->num_active = inc_a;
-            s_poff[E] = poff_next;
-        }
-    }
-    if (e < E) s_cnt[e] = c;
-    __syncthreads();
-    // pad rows of each expert (one warp per expert, lanes on consecutive rows), then
-    // everything past P_pad: gather_idx = -1, weight 0
-    for (int ex = threadIdx.x >> 5; ex < E; ex += blockDim.x >> 5) {
-        const int end = s_poff[ex + 1];
-        for (int r = s_poff[ex] + s_cnt[ex] + (threadIdx.x & 31); r < end; r += 32) {
-            gather_idx[r] = -1;
-            if (row_w != nullptr) row_w[r] = 0.0f;
-        }
-    }
-    for (int64_t r = (int64_t)s_poff[E] + threadIdx.x; r < o.padded_rows_max; r += blockDim.x) {
-        gather_idx[r] = -1;
-        if (row_w != nullptr) row_w[r] = 0.0f;
+        scan_write_expert(e, E, c, inc_c, inc_t, inc_p, inc_h, inc_1, inc_a, o, s_poff);
+        s_cnt[e] = c;
     }
     __syncthreads();
+    scan_write_pads(E, o, s_poff, s_cnt, threadIdx.x, blockDim.x);
+    __syncthreads();
+}
+
+// Inclusive scan over the lanes of one warp.
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane)
+{
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    return v;
+}
+
+// The scan outputs for E <= 32 experts by one warp (lane e owns expert e, c = its rows):
+// the same values as dispatch_scan_body. s_poff[0..E] receives the padded row offsets.
+__device__ __forceinline__ void dispatch_scan_warp(int c, int E, const ScanOut &o, int *s_poff,
+                                                   int lane)
+{
+    if (lane >= E) c = 0;
+    const int ntile = (c + M_TILE - 1) / M_TILE;
+    const int inc_c = warp_inclusive_scan(c, lane);
+    const int inc_t = warp_inclusive_scan(ntile, lane);
+    const int inc_p = warp_inclusive_scan((ntile + 1) / 2, lane);
+    const int inc_h = warp_inclusive_scan(ntile >= 2 ? ntile : 0, lane);
+    const int inc_1 = warp_inclusive_scan(ntile == 1 ? 1 : 0, lane);
+    const int inc_a = warp_inclusive_scan(c > 0 ? 1 : 0, lane);
+    if (lane < E) scan_write_expert(lane, E, c, inc_c, inc_t, inc_p, inc_h, inc_1, inc_a, o, s_poff);
 }
 
 // One block of 1024 threads; thread e owns expert e (E <= 1024).
@@ -332,6 +370,113 @@ __global__ void __launch_bounds__(1024)
         inv_pos[q] = r;
         if (o.row_w != nullptr) o.row_w[r] = topk_w[q];
     }
+}
+
+// In-launch dispatch of the whole-layer launch (routing, dispatch, the expert GEMMs and the
+// combine in one persistent launch). The routing left, per group g of tt tokens (tokens
+// g * tt .. g * tt + tt - 1), its selections per expert in group_counts[g][e]; after a
+// grid-wide barrier every CTA runs dispatch_front for the groups it routed. The outputs are
+// those of the three dispatch kernels and the gather, except that x_perm's pad rows are not
+// written (their layer0 and layer1 rows are never combined).
+struct FrontDispatch {
+    const int32_t *group_counts; // [n_groups][E]
+    int n_groups, tt;
+    const int32_t *topk_idx;     // [T, k]
+    const float *topk_w;         // [T, k]
+    int T, E, k, H;
+    ScanOut so;                  // CTA 0 writes the scan outputs and clears so.ready
+    int32_t *inv_pos;            // [T, k]
+    const __nv_bfloat16 *x;      // [T, H]
+    __nv_bfloat16 *x_perm;       // [P_pad, H]
+};
+
+// Shared-memory scratch of dispatch_front, in ints (E <= 32, tt <= 128).
+__host__ __device__ inline int front_scratch_ints(int n_groups, int E)
+{
+    return (n_groups + 1) * E + (E + 1) + 4 * E;
+}
+
+// All threads of the CTA; groups g_first, g_first + g_step, ... are this CTA's. Ends with a
+// CTA barrier; every thread has fenced its x_perm stores for the async proxy (TMA readers).
+__device__ __forceinline__ void dispatch_front(const FrontDispatch &d, int g_first, int g_step,
+                                               int *scratch)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int E = d.E, G = d.n_groups, k = d.k;
+    int *pref = scratch;                                              // [G + 1][E]
+    int *s_poff = pref + (size_t)(G + 1) * E;                          // [E + 1]
+    uint32_t *bits = reinterpret_cast<uint32_t *>(s_poff + E + 1);     // [E][4]
+    // 1. per expert, the exclusive prefix of the selections over the groups (the rows of
+    //    lower token ids come first within an expert), one warp per expert; row G: totals
+    for (int e = warp; e < E; e += nw) {
+        int run = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            const int v = g < G ? d.group_counts[(size_t)g * E + e] : 0;
+            const int inc = warp_inclusive_scan(v, lane);
+            if (g < G) pref[(size_t)g * E + e] = run + inc - v;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) pref[(size_t)G * E + e] = run;
+    }
+    __syncthreads();
+    const int *total = pref + (size_t)G * E;
+    // 2. padded offsets (every CTA); CTA 0 also writes the scan outputs, the pad markers and
+    //    clears the ready counters of the GEMM phases
+    if (warp == 0) {
+        const int c = lane < E ? total[lane] : 0;
+        if (blockIdx.x == 0) {
+            dispatch_scan_warp(c, E, d.so, s_poff, lane);
+        } else {
+            const int ntile = (c + M_TILE - 1) / M_TILE;
+            const int inc_t = warp_inclusive_scan(ntile, lane);
+            if (lane < E) s_poff[lane] = (inc_t - ntile) * M_TILE;
+            if (lane == E - 1) s_poff[E] = inc_t * M_TILE;
+        }
+    }
+    if (blockIdx.x == 0)
+        for (int i = tid; i < d.so.n_ready; i += nt) d.so.ready[i] = 0;
+    __syncthreads();
+    if (blockIdx.x == 0) scan_write_pads(E, d.so, s_poff, total, tid, nt);
+    // 3. rows of this CTA's pairs (expert, then token order), and their x rows
+    const int chunks = d.H / 8;
+    for (int g = g_first; g < G; g += g_step) {
+        const int t0 = g * d.tt;
+        const int ntg = min(d.tt, d.T - t0);
+        for (int i = tid; i < 4 * E; i += nt) bits[i] = 0u;
+        __syncthreads();
+        const int P = ntg * k;
+        const size_t q0 = (size_t)t0 * k;
+        for (int q = tid; q < P; q += nt) {
+            const int tl = q / k;
+            const int e = d.topk_idx[q0 + q];
+            if (e >= 0 && e < E) atomicOr(&bits[e * 4 + (tl >> 5)], 1u << (tl & 31));
+        }
+        __syncthreads();
+        // one warp per pair: lane 0 writes the indices, the warp copies the row
+        for (int q = warp; q < P; q += nw) {
+            const int tl = q / k;
+            const int t = t0 + tl;
+            const int e = d.topk_idx[q0 + q];
+            if (e < 0 || e >= E) continue;
+            const uint32_t *b = bits + e * 4;
+            const int wd = tl >> 5;
+            int rank = __popc(b[wd] & ((1u << (tl & 31)) - 1u));
+            for (int w = 0; w < wd; ++w) rank += __popc(b[w]);
+            const int r = s_poff[e] + pref[(size_t)g * E + e] + rank;
+            if (lane == 0) {
+                d.so.gather_idx[r] = t;
+                d.inv_pos[q0 + q] = r;
+                if (d.so.row_w != nullptr) d.so.row_w[r] = d.topk_w[q0 + q];
+            }
+            const uint4 *src = reinterpret_cast<const uint4 *>(d.x + (size_t)t * d.H);
+            uint4 *dst = reinterpret_cast<uint4 *>(d.x_perm + (size_t)r * d.H);
+#pragma unroll 4
+            for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+        }
+        __syncthreads(); // the bitmaps are reused by the next group
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // x_perm[r][:] = x[gather_idx[r]][:] (zeros on pad rows), for r < P_pad. One warp per row.

@@ -38,8 +38,21 @@
 #pragma once
 
 #include "gemm_tc.cuh"
+#include "route_chain.cuh"
 
 namespace moe {
+
+// The front of the whole-layer launch: routing (route_chain.cuh, with warp 0 issuing its TMA
+// copies and warps 2 .. 2 + ncw - 1 walking the chains) of the token groups b, b + grid, ...,
+// a grid-wide barrier, the in-launch dispatch (dispatch.cuh), and a second barrier after
+// which every CTA sees the dispatch outputs and every x_perm row.
+struct FrontArgs {
+    RcArgs ra;        // router; ra.group_counts receives the per-group selections
+    int ncw;          // consumer warps of the router (1..8)
+    int n_groups;     // ceil(T / ra.tt)
+    FrontDispatch fd; // in-launch dispatch
+    int *gbar;        // grid-barrier counter, zero when the launch starts
+};
 
 constexpr int COMBINE_TOKENS = 128; // tokens per combine item unless fused_plan() says otherwise
 
@@ -63,6 +76,7 @@ struct FusedArgs {
     // t_end_ns}; trace[0] is the record counter, records start at trace[4]; nullptr: off
     unsigned long long *trace;
     int64_t trace_cap;      // records that fit after the counter
+    FrontArgs front;        // whole-layer launch only (FRONT = true)
 };
 
 enum : int { TRACE_L0 = 0, TRACE_L1 = 1, TRACE_COMBINE = 2 };
@@ -135,6 +149,53 @@ __device__ __forceinline__ bool flag_wait_bounded(const int *p, int target, vola
             return false;
         }
     }
+}
+
+// Grid-wide barrier of a persistent launch (every CTA resident): the CTA's threads meet, thread
+// 0 publishes the CTA's writes and waits, bounded, until `target` CTA arrivals have been
+// counted on `ctr` (a launch-wide counter: the n-th barrier of the launch waits for n * grid).
+__device__ __forceinline__ bool grid_barrier(int *ctr, int target, volatile int *abort_flag,
+                                             int64_t timeout_ns, int *status, int where)
+{
+    __syncthreads();
+    int ok = 1;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        red_release_gpu_add(ctr, 1);
+        ok = flag_wait_bounded(ctr, target, abort_flag, timeout_ns, status, where) ? 1 : 0;
+    }
+    return __syncthreads_and(ok) != 0;
+}
+
+// Routing, dispatch and the row copy of the whole-layer launch, in the GEMM stages' shared
+// memory (free until the GEMM phases start). False when a wait gave up.
+template <int G>
+__device__ __forceinline__ bool fused_front(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
+                                            const FusedArgs &fa, uint8_t *smem,
+                                            volatile int *abort_flag, int *status, int64_t tmo)
+{
+    const FrontArgs &f = fa.front;
+    const RcLayout L = rc_layout(f.ra.tt, f.ra.E, 4 * G, f.ra.stages);
+    if (threadIdx.x == 0) {
+        rc_init(smem, L, f.ra.stages, f.ncw);
+        tma_prefetch_desc(tmRX);
+        tma_prefetch_desc(tmRW);
+    }
+    __syncthreads();
+    bool ok = rc_run<4, G>(tmRX, tmRW, f.ra, smem, 0, 2, f.ncw, blockIdx.x, gridDim.x, f.n_groups, 1);
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    if (threadIdx.x == 0) rc_fini(smem, L, f.ra.stages);
+    if (!ok) {
+        *abort_flag = 1;
+        return false;
+    }
+    // every CTA's routing (top-k and per-group counts) is complete
+    if (!grid_barrier(f.gbar, (int)gridDim.x, abort_flag, tmo, status, 350)) return false;
+    dispatch_front(f.fd, blockIdx.x, gridDim.x, reinterpret_cast<int *>(smem));
+    // every CTA's rows, indices and (CTA 0) the dispatch outputs are in place
+    if (!grid_barrier(f.gbar, 2 * (int)gridDim.x, abort_flag, tmo, status, 351)) return false;
+    fence_proxy_async_global(); // x_perm was written by generic stores; layer0 reads it by TMA
+    return true;
 }
 
 struct FusedItem {
@@ -296,12 +357,16 @@ __device__ __forceinline__ bool combine_queue(const FusedArgs &fa, int group_war
     return ok;
 }
 
-template <int KIND0>
+// FRONT: the launch also routes and dispatches the tokens first (the whole layer in one
+// launch; its router tensor maps tmRX, tmRW are used only then).
+template <int KIND0, bool FRONT>
 __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     moe_fused_layer_kernel(const __grid_constant__ CUtensorMap tmA0,
                            const __grid_constant__ CUtensorMap tmW1,
                            const __grid_constant__ CUtensorMap tmH,
-                           const __grid_constant__ CUtensorMap tmW2, const FusedArgs fa)
+                           const __grid_constant__ CUtensorMap tmW2,
+                           const __grid_constant__ CUtensorMap tmRX,
+                           const __grid_constant__ CUtensorMap tmRW, const FusedArgs fa)
 {
     using namespace gemm;
     extern __shared__ uint8_t smem_raw[];
@@ -360,7 +425,10 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_tiles = l0.meta->num_tiles;
+    bool front_ok = true;
+    if constexpr (FRONT) front_ok = fused_front<2>(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo);
+
+    const int num_tiles = front_ok ? l0.meta->num_tiles : 0;
     const int total0 = num_tiles * l0.n_tiles;
     const int total = total0 + num_tiles * l1.n_tiles;
 
@@ -585,7 +653,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         // the data-movement warps, 3 for the epilogue warps)
         volatile int *slots = reinterpret_cast<volatile int *>(warps_done + 4);
         const int bar = dm ? 2 : 3;
-        if (named_bar_and(bar, 128, ok))
+        if (named_bar_and(bar, 128, ok && front_ok))
             combine_queue(fa, dm ? warp - 6 : warp - 2, lane, bar, slots + (dm ? 0 : 1), abort_flag,
                           status);
     }

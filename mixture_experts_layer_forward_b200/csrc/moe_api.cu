@@ -40,6 +40,8 @@ std::atomic<unsigned long long *> g_trace{nullptr};
 std::atomic<int64_t> g_trace_cap{0};
 // grouped-GEMM work order (MOE_ORDER_*; test and tuning hook)
 std::atomic<int> g_order{MOE_ORDER_NARROW};
+// whole-layer launch (routing and dispatch inside the persistent launch) where it applies
+std::atomic<int> g_front{1};
 
 // ---------------------------------------------------------------------------------------
 // problem checks and workspace layout
@@ -74,7 +76,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
     size_t status, meta, logits, wgt, wnorm, xsq, topk_idx, topk_w, chunk,
-        counts, offsets, poff, tile_off,
+        counts, offsets, poff, tile_off, gcount,
         tile_expert, ptile_off, ptile_expert, hot_off, hot_tile_expert, cold_tile, ready,
         gather_idx, inv_pos, row_w, x_perm, h, ys,
         x_stage, out_stage, x_stage2, out_stage2, sh_gate, sh_h, sh_ys, xq, sx, hq, sh,
@@ -163,6 +165,8 @@ Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd
     L.topk_idx = take(T * K * 4);
     L.topk_w = take(T * K * 4);
     L.chunk = take((size_t)L.nchunk * E * 4);
+    // whole-layer launch: selections per group of at least 8 tokens and expert
+    L.gcount = take((T + 7) / 8 * E * 4);
     L.counts = take(E * 4);
     L.offsets = take((E + 1) * 4);
     L.poff = take((E + 1) * 4);
@@ -566,12 +570,9 @@ struct DispatchOut {
     DispatchMeta *meta;
 };
 
-cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t *topk_idx,
-                            const float *topk_w, const DispatchOut &o, int *status, int clear_status,
-                            cudaStream_t st, const int32_t *n_rows = nullptr)
+// The scan step's outputs in the workspace.
+ScanOut scan_out(const Layout &L, const DispatchOut &o)
 {
-    const int T = p->T, E = p->E, k = p->top_k;
-    const int nchunk = L.nchunk;
     ScanOut so{};
     so.counts = o.counts;
     so.offsets = o.offsets;
@@ -590,6 +591,16 @@ cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t
     so.hot_tile_expert = o.hot_tile_expert;
     so.cold_tile = o.cold_tile;
     so.active_list = o.active_list;
+    return so;
+}
+
+cudaError_t launch_dispatch(const moe_problem *p, const Layout &L, const int32_t *topk_idx,
+                            const float *topk_w, const DispatchOut &o, int *status, int clear_status,
+                            cudaStream_t st, const int32_t *n_rows = nullptr)
+{
+    const int T = p->T, E = p->E, k = p->top_k;
+    const int nchunk = L.nchunk;
+    const ScanOut so = scan_out(L, o);
     if (nchunk == 1) { // one chunk of tokens: the three steps in one block
         dispatch_small_kernel<<<1, 1024, (size_t)E * (DISPATCH_WORDS + 1) * 4, st>>>(
             topk_idx, topk_w, T, E, k, so, o.inv_pos, status, clear_status, n_rows);
@@ -771,21 +782,47 @@ cudaError_t launch_gemm_any(const CUtensorMap &ta, const CUtensorMap &tb, const 
     return launch_gemm<KIND>(ta, tb, args, max_work, st);
 }
 
-template <int KIND0>
+template <int KIND0, bool FRONT>
 cudaError_t launch_fused(const CUtensorMap &a0, const CUtensorMap &w1, const CUtensorMap &hm,
-                         const CUtensorMap &w2, const FusedArgs &fa, int max_work, cudaStream_t st)
+                         const CUtensorMap &w2, const CUtensorMap &rx, const CUtensorMap &rw,
+                         const FusedArgs &fa, int max_work, cudaStream_t st)
 {
-    auto kern = moe_fused_layer_kernel<KIND0>;
+    auto kern = moe_fused_layer_kernel<KIND0, FRONT>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     // every CTA must be resident at once (the ready-flag waits rely on it): one per SM
     int grid = sm_count();
     if (grid <= 0) grid = 148;
-    if (grid > max_work) grid = max_work;
+    if (!FRONT && grid > max_work) grid = max_work; // (the whole-layer launch: one CTA per SM)
     if (grid < 1) grid = 1;
-    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(a0, w1, hm, w2, fa);
+    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(a0, w1, hm, w2, rx, rw, fa);
     return cudaGetLastError();
+}
+
+// Whole-layer launch (routing and dispatch inside the persistent launch): the routing's token
+// groups and ring for one CTA per SM. `ok` is false where the shape does not fit it.
+struct FrontPlan {
+    bool ok;
+    int grid, tt, n_groups, ncw, stages;
+};
+
+FrontPlan front_plan(const moe_problem *p)
+{
+    FrontPlan f{};
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    f.grid = sms;
+    // tokens per group: about one group per SM, at most 128 (two consumer threads per token
+    // on the eight non-GEMM-issuing warps), at least 8 (the per-group count buffer)
+    f.tt = std::max(8, std::min(128, (p->T + sms - 1) / sms));
+    f.n_groups = (p->T + f.tt - 1) / f.tt;
+    f.ncw = (f.tt * 2 + 31) / 32;
+    const int budget = gemm::STAGES * gemm::STAGE; // the GEMM stages' shared memory
+    f.stages = RC_MAX_STAGES;
+    while (f.stages > 3 && rc_layout(f.tt, p->E, 8, f.stages).total > budget) --f.stages;
+    f.ok = p->E == 8 && rc_layout(f.tt, p->E, 8, f.stages).total <= budget &&
+           (int64_t)front_scratch_ints(f.n_groups, p->E) * 4 <= budget;
+    return f;
 }
 
 moe_status to_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -936,6 +973,14 @@ bool run_fused(const moe_problem *p)
     return mode == MOE_GEMM_FUSED || (mode == MOE_GEMM_AUTO && fused_plan(p).fused);
 }
 
+// The persistent launch also routes and dispatches (a computed routing, no stage events and
+// 16-byte aligned operands besides): one-launch exact router, rows read by TMA from x_perm.
+bool whole_layer(const moe_problem *p)
+{
+    return g_front.load() != 0 && g_gemm_mode.load() != MOE_GEMM_CTA_PAIR && run_fused(p) &&
+           use_x_perm(p) && route_uses_chain(p) && !route_uses_filter(p) && front_plan(p).ok;
+}
+
 moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
                         const float *bias, const moe_bf16 *W1, const moe_bf16 *W2, moe_bf16 *out,
                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
@@ -984,6 +1029,10 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     const bool pair = (g_gemm_mode.load() == MOE_GEMM_CTA_PAIR);
     const bool fused = !pair && n_rows == nullptr && run_fused(p);
     const bool xperm = pair || use_x_perm(p);
+    // the whole layer in one launch: the persistent launch routes and dispatches first (its
+    // router is the one-launch exact router; stage events need the stages' own launches)
+    const FrontPlan fpl = front_plan(p);
+    const bool one = fused && !given && n_events == 0 && whole_layer(p);
     const bool a_ok = xperm ? make_map_2d(&m_x, x_perm, (uint64_t)L.pmax, (uint64_t)H, gemm::BM)
                             : make_map_2d(&m_x, x, (uint64_t)p->T, (uint64_t)H, 1);
     if (!a_ok ||
@@ -995,15 +1044,24 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
     const int64_t timeout = g_timeout_ns.load();
     const FilterBufs fb = filter_bufs(ws, L);
     cudaError_t e = record(events, n_events, 0, st);
-    if (e == cudaSuccess && !given)
-        e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st,
-                         &fb);
-    if (e == cudaSuccess) e = record(events, n_events, 1, st);
-    // with the routing supplied the dispatch clears the status word (and checks the ids)
-    if (e == cudaSuccess)
-        e = launch_dispatch(p, L, topk_idx, topk_w, d, status, given ? 1 : 0, st, n_rows);
-    if (e == cudaSuccess && xperm) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
-    if (e == cudaSuccess) e = record(events, n_events, 2, st);
+    CUtensorMap m_rx = m_x, m_rw = m_x; // the router's maps (whole-layer launch only)
+    if (one) {
+        // status word and grid-barrier counter (same 256-byte block) start from zero
+        if (!make_map_2d(&m_rx, x, (uint64_t)p->T, (uint64_t)H, (uint32_t)fpl.tt) ||
+            !make_map_2d_plain(&m_rw, Wg, (uint64_t)H, (uint64_t)E, (uint32_t)E, RC_HC))
+            return MOE_ERR_CUDA;
+        if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 32, st);
+    } else {
+        if (e == cudaSuccess && !given)
+            e = launch_route(p, x, Wg, bias, topk_idx, topk_w, at<float>(ws, L.logits), status, st,
+                             &fb);
+        if (e == cudaSuccess) e = record(events, n_events, 1, st);
+        // with the routing supplied the dispatch clears the status word (and checks the ids)
+        if (e == cudaSuccess)
+            e = launch_dispatch(p, L, topk_idx, topk_w, d, status, given ? 1 : 0, st, n_rows);
+        if (e == cudaSuccess && xperm) e = launch_gather(p, x, d.gather_idx, d.meta, x_perm, st);
+        if (e == cudaSuccess) e = record(events, n_events, 2, st);
+    }
 
     GemmArgs a0{};
     a0.tile_off = d.tile_off;
@@ -1074,11 +1132,48 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         fa.trace = g_trace.load();
         fa.trace_cap = g_trace_cap.load();
         const int max_work = L.max_tiles * (a0.n_tiles + a1.n_tiles);
+        if (one) {
+            FrontArgs &f = fa.front;
+            f.ra.bias = bias;
+            f.ra.topk_idx = topk_idx;
+            f.ra.topk_w = topk_w;
+            f.ra.T = p->T;
+            f.ra.H = H;
+            f.ra.E = E;
+            f.ra.k = p->top_k;
+            f.ra.gate = p->gate;
+            f.ra.tt = fpl.tt;
+            f.ra.stages = fpl.stages;
+            f.ra.status = status;
+            f.ra.timeout_ns = timeout;
+            f.ra.group_counts = at<int32_t>(ws, L.gcount);
+            f.ncw = fpl.ncw;
+            f.n_groups = fpl.n_groups;
+            FrontDispatch &fd = f.fd;
+            fd.group_counts = f.ra.group_counts;
+            fd.n_groups = fpl.n_groups;
+            fd.tt = fpl.tt;
+            fd.topk_idx = topk_idx;
+            fd.topk_w = topk_w;
+            fd.T = p->T;
+            fd.E = E;
+            fd.k = p->top_k;
+            fd.H = H;
+            fd.so = scan_out(L, d);
+            fd.inv_pos = d.inv_pos;
+            fd.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+            fd.x_perm = reinterpret_cast<__nv_bfloat16 *>(x_perm);
+            f.gbar = status + 4;
+        }
         if (e == cudaSuccess) {
             // (a0.epi8 is for the separate launches; the fused kernel splits layer0's epilogue
             // itself when its rows come by TMA)
-            e = gated ? launch_fused<GEMM_SWIGLU>(m_x, m_w1, m_h, m_w2, fa, max_work, st)
-                      : launch_fused<GEMM_ACT>(m_x, m_w1, m_h, m_w2, fa, max_work, st);
+            if (one)
+                e = gated ? launch_fused<GEMM_SWIGLU, true>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st)
+                          : launch_fused<GEMM_ACT, true>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st);
+            else
+                e = gated ? launch_fused<GEMM_SWIGLU, false>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st)
+                          : launch_fused<GEMM_ACT, false>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st);
         }
         // the three stages share one launch: their boundaries coincide at its end
         for (int i = 3; i < 6 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
@@ -1496,7 +1591,12 @@ int moe_forward_launches(const moe_problem *p)
     // persistent launch
     const int gather = (pair || use_x_perm(p)) ? 1 : 0;
     const int layers = (!pair && run_fused(p)) ? 1 : 3;
-    return route + dispatch + gather + layers;
+    return whole_layer(p) ? 1 : route + dispatch + gather + layers;
+}
+
+int moe_set_whole_layer_launch(int on)
+{
+    return g_front.exchange(on != 0 ? 1 : 0);
 }
 
 size_t moe_workspace_size(const moe_problem *p)

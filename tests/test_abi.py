@@ -115,7 +115,14 @@ def test_forward_launch_count_follows_the_modes(lib):
         # large batches (T*k >= 128 E) gather x into sorted rows and take the persistent
         # launch: router + dispatch 3 + gather + 1
         # (E <= 8: the persistent launch)
-        assert moe.moe_forward_launches(mixtral) == 6   # E = 8: one-launch router
+        # E = 8 with the one-launch router: the whole layer in the persistent launch
+        assert moe.moe_forward_launches(mixtral) == 1
+        assert moe.moe_set_whole_layer_launch(False) is True
+        try:
+            assert moe.moe_forward_launches(mixtral) == 6   # router, dispatch 3, gather, layers
+        finally:
+            moe.moe_set_whole_layer_launch(True)
+        assert moe.moe_forward_launches(moe.Problem.make(1000, 256, 256, 8, 2)) == 1
         assert moe.moe_forward_launches(qwen2) == 10    # T*E >= 2^16: filter router
         assert moe.moe_forward_launches(decode) == 6    # T*E < 2^16: sequential, three layers
         phi35 = moe.Problem.from_config(synth.CONFIGS["phi35"])
@@ -125,6 +132,7 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(mixtral) == 8   # forced: E = 8 qualifies
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         moe.moe_set_router_mode(moe.ROUTER_SEQUENTIAL)
+        assert moe.moe_forward_launches(mixtral) == 1   # the one-launch router again
         assert moe.moe_forward_launches(phi35) == 8     # E = 16: one-launch router
         assert moe.moe_forward_launches(moe.Problem.make(64, 128, 128, 4, 2)) == 6  # E % 8
         assert moe.moe_forward_launches(qwen2) == 9

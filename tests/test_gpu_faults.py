@@ -28,8 +28,10 @@ def _forward(cfg, d, ws):
 
 
 # T*k < 128 E: layer0 rows gathered in the kernel; T*k >= 128 E: sorted rows by TMA, and the
-# data-movement warps take half of each layer0 epilogue before the combine
-@pytest.mark.parametrize("T,E", [(300, 8), (700, 4)], ids=["gathered_rows", "sorted_rows"])
+# data-movement warps take half of each layer0 epilogue before the combine; E = 8 with sorted
+# rows: the whole layer in one launch (routing and dispatch first, then the same GEMM phases)
+@pytest.mark.parametrize("T,E", [(300, 8), (700, 4), (1100, 8)],
+                         ids=["gathered_rows", "sorted_rows", "whole_layer"])
 def test_withheld_ready_signal_times_out_and_context_recovers(T, E):
     cfg = synth.LayerConfig("fault", T=T, H=256, F=256, E=E, k=2)
     inp = synth.make_inputs(cfg, seed=21)

@@ -477,6 +477,48 @@ def test_gemm_variants_agree():
         moe.moe_set_gemm_mode(prev)
 
 
+# The persistent launch that also routes and dispatches (E == 8, T * k >= 128 E, the one-launch
+# router): short last h chunk, 8-token groups with idle CTAs, softmax over all experts with
+# GELU, the selection-only bias with k = 3, and 128-token groups with two groups on some CTAs.
+WHOLE_CASES = [
+    cfg_small("wl_e8", 1100, 192, 384, 8, 2, zipf_s=0.5),
+    cfg_small("wl_groups8", 1000, 512, 256, 8, 2),
+    cfg_small("wl_gelu_all", 1500, 256, 320, 8, 2, act=1, gate=1),
+    cfg_small("wl_selbias", 1200, 256, 256, 8, 3, zipf_s=1.5, gate=moe.GATE_SELECT_BIAS),
+    cfg_small("wl_two_groups", 20000, 256, 128, 8, 2),
+]
+
+
+@pytest.mark.parametrize("cfg", WHOLE_CASES, ids=[c.name for c in WHOLE_CASES])
+def test_whole_layer_launch_matches_oracle_and_separate_launches(cfg):
+    """One launch for the whole layer: the routing, gates and output are bitwise those of
+    the separate route and dispatch launches, and match the oracle."""
+    inp = synth.make_inputs(cfg, seed=19)
+    p = moe.Problem.from_config(cfg)
+    prev = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
+    try:
+        assert moe.moe_forward_launches(p) == 1
+        one = run_forward(cfg, inp)
+        prev_w = moe.moe_set_whole_layer_launch(False)
+        try:
+            assert moe.moe_forward_launches(p) > 1
+            sep = run_forward(cfg, inp)
+        finally:
+            moe.moe_set_whole_layer_launch(prev_w)
+        again = run_forward(cfg, inp, one[3])  # the same workspace again: counters restart
+    finally:
+        moe.moe_set_gemm_mode(prev)
+    for a, b, what in zip(one[:3], sep[:3], ("out", "topk_idx", "topk_w")):
+        assert torch.equal(a, b), what
+    assert torch.equal(one[0], again[0])
+    b = None if inp["bias"] is None else inp["bias"].numpy()
+    ref, ref_idx, ref_w = oracle.moe_forward(bits(inp["x"]), bits(inp["Wg"]), b, bits(inp["W1"]),
+                                             bits(inp["W2"]), cfg.k, act=cfg.act, gate=cfg.gate)
+    assert np.array_equal(one[1].cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(one[2].cpu().numpy(), ref_w, rtol=GATE_RTOL, atol=GATE_ATOL)
+    assert_out_close(one[0], ref, cfg.name)
+
+
 def test_forward_all_tokens_on_one_expert():
     cfg = cfg_small("one_hot", 300, 128, 128, 8, 1)
     inp = synth.make_inputs(cfg, seed=12)
