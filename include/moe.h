@@ -351,6 +351,75 @@ MOE_API moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y,
                                  moe_bf16 *const *back, int64_t back_rows, void *ws,
                                  void *stream);
 
+/* Expert-parallel layer with the exchange overlapped with the expert GEMMs, one persistent
+ * launch per GPU (Comet §3.1.2: layer0 tiles start as their rows arrive, layer1 rows return
+ * as their tiles finish; §4: the GPU issues fine-grained transfers; the tile-signalling
+ * abstract: transfers fired and awaited per tile through ready flags). Rank r of `world`
+ * (1 <= world <= MOE_EP_MAX_WORLD, world dividing E) holds experts [r * E / world,
+ * (r + 1) * E / world) and its own T tokens; the router (E a multiple of 8, E <= 32, H a
+ * multiple of 64) is replicated. In the launch, every CTA of rank r:
+ *   1. routes a group of r's tokens (the exact router), and writes the group's selections per
+ *      expert into every rank's counts buffer; a barrier of r's CTAs; r raises its flag in
+ *      every rank's flags buffer (value `epoch`) and waits for every rank's flag in its own;
+ *   2. derives, from every rank's counts, where each of r's pairs goes -- row = destination
+ *      d's padded offset of the expert + the rows of lower source ranks + r's earlier tokens
+ *      (d's receive buffer is expert-sorted, 128-row padded, source rank then token within an
+ *      expert); CTA 0 writes r's receive-side tile list; a barrier of r's CTAs;
+ *   3. four data-movement warps per CTA store each of r's pairs' x row, gate and origin into
+ *      the destination's receive buffers and then add 1 to the destination's arrival count
+ *      of that 128-row tile; meanwhile the GEMM pipeline runs r's experts: a layer0 tile
+ *      waits only until its rows have arrived; a layer1 tile waits for its layer0 rows (the
+ *      tile-level counters of the persistent launch) and its epilogue stores each gated row
+ *      straight into row t * k + j of the origin's return buffer and adds 1 to the origin's
+ *      count of that token;
+ *   4. the combine sums the k returned rows of each of r's tokens (j ascending, fp32, one
+ *      bf16 rounding) as soon as all of the token's row stripes are back.
+ * Stores to other GPUs are plain 16-byte stores followed by a system-scope fence before the
+ * count; nothing loads another GPU's memory, no TMA reads another GPU's memory, and every
+ * wait is bounded (MOE_ERR_DEVICE_TIMEOUT in the status word of the rank's workspace). Every
+ * gated row is bitwise the row moe_forward computes on one GPU, so `out` is bitwise
+ * moe_forward's output for r's tokens with all E experts.
+ * Buffers: each rank owns the eight exchange buffers of moe_ep_buffer_sizes, addressable by
+ * every rank (symmetric allocations; zero-filled once before the first call); entry d of
+ * each pointer table of moe_ep_rank is rank d's buffer as this GPU addresses it. Calls on
+ * the same buffers pass epoch 1, 2, 3, ... (the same on every rank for one layer call).
+ * n_local: ranks this launch carries -- 1 on a GPU per rank; up to MOE_EP_MAX_LOCAL to run
+ * several ranks on one GPU (all their buffers on this GPU; each rank gets 1/n_local of the
+ * SMs), which is how the ranks' interplay is tested with one GPU. All ranks of a layer call
+ * must launch (their waits on one another are bounded, not avoided). */
+#define MOE_EP_MAX_WORLD 8
+#define MOE_EP_MAX_LOCAL 4
+#define MOE_EP_NUM_BUFFERS 8
+typedef struct {
+    moe_problem p;           /* this rank's tokens T; all E experts; top_k, act, gate */
+    int32_t world, rank;
+    int32_t epoch;           /* > 0, increasing call to call on the same buffers */
+    const moe_bf16 *x;       /* [T, H] this rank's tokens */
+    const moe_bf16 *Wg;      /* [H, E] router (the same on every rank) */
+    const float *bias;       /* [E] or NULL */
+    const moe_bf16 *W1;      /* [E / world, H, 2F] (SwiGLU) or [E / world, H, F]: r's experts */
+    const moe_bf16 *W2;      /* [E / world, F, H] */
+    moe_bf16 *out;           /* [T, H] */
+    int32_t *topk_idx;       /* [T, top_k] or NULL (kept in the workspace) */
+    float *topk_w;           /* [T, top_k] or NULL */
+    void *ws;                /* moe_ep_workspace_size bytes, 256-byte aligned */
+    size_t ws_bytes;
+    /* every rank's exchange buffers (index d: rank d's), in the order of moe_ep_buffer_sizes:
+     * counts, flags, recv_rows, recv_gate, recv_origin, arrive, back, back_cnt */
+    void *buf[MOE_EP_NUM_BUFFERS][MOE_EP_MAX_WORLD];
+} moe_ep_rank;
+
+/* Bytes of each exchange buffer of one rank for ranks of T tokens (*p) in a world of
+ * `world`: sizes[0..7] = counts, flags, recv_rows, recv_gate, recv_origin, arrive, back,
+ * back_cnt (each to be 256-byte aligned, zero-filled once). MOE_OK or an error code. */
+MOE_API moe_status moe_ep_buffer_sizes(const moe_problem *p, int32_t world, int64_t *sizes);
+/* Workspace bytes of one rank (0 if *p or world is invalid). */
+MOE_API size_t moe_ep_workspace_size(const moe_problem *p, int32_t world);
+/* The layer for the n_local ranks ranks[0 .. n_local - 1] on this GPU, one launch on
+ * `stream` (after a 32-byte memset per rank). MOE_OK, MOE_ERR_INVALID_ARG (shapes, world,
+ * alignment, router not applicable), MOE_ERR_WORKSPACE or MOE_ERR_CUDA. */
+MOE_API moe_status moe_ep_layer_forward(const moe_ep_rank *ranks, int32_t n_local, void *stream);
+
 /* Backward pass (training; beyond the pages, which describe the forward).
  * Given dout = dL/dout [T, H] bf16, the gradients of the layer moe_forward computes, with the
  * selection held fixed (it is piecewise constant) and the gates the softmax over the

@@ -57,6 +57,24 @@ class SharedExpert(ctypes.Structure):
                 ("w_sg", ctypes.c_void_p)]
 
 
+EP_MAX_WORLD = 8
+EP_MAX_LOCAL = 4
+EP_BUFFERS = ("counts", "flags", "recv_rows", "recv_gate", "recv_origin", "arrive", "back",
+              "back_cnt")
+
+
+class EpRank(ctypes.Structure):
+    """moe_ep_rank: one rank of moe_ep_layer_forward (device pointers; buf[b][d] is rank d's
+    exchange buffer b as this GPU addresses it, b in the order of EP_BUFFERS)."""
+    _fields_ = [("p", Problem), ("world", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("epoch", ctypes.c_int32), ("x", ctypes.c_void_p), ("Wg", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("W1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p),
+                ("topk_w", ctypes.c_void_p), ("ws", ctypes.c_void_p),
+                ("ws_bytes", ctypes.c_size_t),
+                ("buf", (ctypes.c_void_p * EP_MAX_WORLD) * len(EP_BUFFERS))]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -117,6 +135,9 @@ def library() -> ctypes.CDLL:
             "moe_set_router_mode": ([i32], i32),
             "moe_set_work_order": ([i32], i32),
             "moe_set_whole_layer_launch": ([i32], i32),
+            "moe_ep_buffer_sizes": ([P, i32, ctypes.POINTER(ctypes.c_int64)], i32),
+            "moe_ep_workspace_size": ([P, i32], sz),
+            "moe_ep_layer_forward": ([ctypes.POINTER(EpRank), i32, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -520,3 +541,50 @@ def moe_set_whole_layer_launch(on: bool) -> bool:
     """Routing and dispatch inside the persistent launch where it applies (on by default);
     returns the previous setting."""
     return bool(library().moe_set_whole_layer_launch(1 if on else 0))
+
+
+def moe_ep_buffer_sizes(p: Problem, world: int) -> list[int]:
+    """Bytes of each of a rank's exchange buffers (EP_BUFFERS order)."""
+    sizes = (ctypes.c_int64 * len(EP_BUFFERS))()
+    rc = library().moe_ep_buffer_sizes(ctypes.byref(p), int(world), sizes)
+    _check("moe_ep_buffer_sizes", rc)
+    return [int(v) for v in sizes]
+
+
+def moe_ep_workspace_size(p: Problem, world: int) -> int:
+    n = int(library().moe_ep_workspace_size(ctypes.byref(p), int(world)))
+    if n == 0:
+        raise MoeError("moe_ep_workspace_size", -1)
+    return n
+
+
+def ep_rank(p: Problem, world: int, rank: int, epoch: int, x, Wg, bias, W1, W2, out, ws,
+            buffers, topk_idx=None, topk_w=None) -> EpRank:
+    """The moe_ep_rank of one rank. buffers[b][d]: rank d's buffer b as an int (its address on
+    this GPU) or a tensor on this GPU."""
+    r = EpRank()
+    r.p = p
+    r.world, r.rank, r.epoch = int(world), int(rank), int(epoch)
+    r.x = _ptr(x, torch.bfloat16, "x")
+    r.Wg = _ptr(Wg, torch.bfloat16, "Wg")
+    r.bias = _ptr(bias, torch.float32, "bias")
+    r.W1 = _ptr(W1, torch.bfloat16, "W1")
+    r.W2 = _ptr(W2, torch.bfloat16, "W2")
+    r.out = _ptr(out, torch.bfloat16, "out")
+    r.topk_idx = _ptr(topk_idx, torch.int32, "topk_idx")
+    r.topk_w = _ptr(topk_w, torch.float32, "topk_w")
+    r.ws = _ptr(ws, torch.uint8, "ws")
+    r.ws_bytes = ws.numel()
+    for b in range(len(EP_BUFFERS)):
+        for d in range(world):
+            v = buffers[b][d]
+            r.buf[b][d] = v if isinstance(v, int) else v.data_ptr()
+    return r
+
+
+def moe_ep_layer_forward(ranks, stream=None):
+    """One launch for the ranks in `ranks` (EpRank structures; all on this GPU)."""
+    n = len(ranks)
+    arr = (EpRank * n)(*ranks)
+    rc = library().moe_ep_layer_forward(arr, n, _stream(stream))
+    _check("moe_ep_layer_forward", rc)

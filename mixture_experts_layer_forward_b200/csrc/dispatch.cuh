@@ -396,10 +396,11 @@ __host__ __device__ inline int front_scratch_ints(int n_groups, int E)
     return (n_groups + 1) * E + (E + 1) + 4 * E;
 }
 
-// All threads of the CTA; groups g_first, g_first + g_step, ... are this CTA's. Ends with a
-// CTA barrier; every thread has fenced its x_perm stores for the async proxy (TMA readers).
+// All threads of the CTA; groups g_first, g_first + g_step, ... are this CTA's; the lead CTA
+// writes the scan outputs. Every thread has fenced its x_perm stores for the async proxy
+// (TMA readers) at the end.
 __device__ __forceinline__ void dispatch_front(const FrontDispatch &d, int g_first, int g_step,
-                                               int *scratch)
+                                               bool lead, int *scratch)
 {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
     const int E = d.E, G = d.n_groups, k = d.k;
@@ -425,7 +426,7 @@ __device__ __forceinline__ void dispatch_front(const FrontDispatch &d, int g_fir
     //    clears the ready counters of the GEMM phases
     if (warp == 0) {
         const int c = lane < E ? total[lane] : 0;
-        if (blockIdx.x == 0) {
+        if (lead) {
             dispatch_scan_warp(c, E, d.so, s_poff, lane);
         } else {
             const int ntile = (c + M_TILE - 1) / M_TILE;
@@ -434,10 +435,10 @@ __device__ __forceinline__ void dispatch_front(const FrontDispatch &d, int g_fir
             if (lane == E - 1) s_poff[E] = inc_t * M_TILE;
         }
     }
-    if (blockIdx.x == 0)
+    if (lead)
         for (int i = tid; i < d.so.n_ready; i += nt) d.so.ready[i] = 0;
     __syncthreads();
-    if (blockIdx.x == 0) scan_write_pads(E, d.so, s_poff, total, tid, nt);
+    if (lead) scan_write_pads(E, d.so, s_poff, total, tid, nt);
     // 3. rows of this CTA's pairs (expert, then token order), and their x rows
     const int chunks = d.H / 8;
     for (int g = g_first; g < G; g += g_step) {

@@ -54,6 +54,31 @@ struct FrontArgs {
     int *gbar;        // grid-barrier counter, zero when the launch starts
 };
 
+// Expert parallelism inside the persistent launch (Comet §3.1.2 and §4; the tile-signalling
+// abstract): rank r holds experts [r * e_loc, (r + 1) * e_loc). Every rank owns the buffers
+// below (every rank can address every rank's copy: [world] arrays of pointers, plain
+// loads and stores over NVLink); a rank's copy of the receive buffers holds the rows routed
+// to its experts in its own expert-sorted, 128-row padded order (expert, then source rank,
+// then source token), so that its layer0 reads them with TMA from its own memory.
+struct EpArgs {
+    int world, rank, e_loc;
+    int epoch;                                // this call's number (> 0): barrier flags reach it
+    int32_t *all_counts[EP_MAX_WORLD];        // [world][n_groups][E] every source's group counts
+    int *flags[EP_MAX_WORLD];                 // [world] barrier flags, one per source rank
+    __nv_bfloat16 *recv_rows[EP_MAX_WORLD];   // [recv_cap][H] rows routed to the rank's experts
+    float *recv_gate[EP_MAX_WORLD];           // [recv_cap] their gate weights (0 on pad rows)
+    long long *recv_origin[EP_MAX_WORLD];     // [recv_cap] (source rank << 32) | (t * k + j); -1 pads
+    int *arrive[EP_MAX_WORLD];                // [max_tiles] rows arrived per local M tile
+    __nv_bfloat16 *back[EP_MAX_WORLD];        // [T * k][H] gated rows returned to their origin
+    int *back_cnt[EP_MAX_WORLD];              // [T] row stripes returned per token
+    int64_t recv_cap;
+    int max_tiles;
+    int32_t *slot;                            // [T * k] this rank's pairs: destination row
+    int32_t *dest;                            // [T * k] this rank's pairs: destination rank
+};
+
+enum : int { FUSED_LAYERS = 0, FUSED_WHOLE = 1, FUSED_EP = 2 };
+
 constexpr int COMBINE_TOKENS = 128; // tokens per combine item unless fused_plan() says otherwise
 
 struct FusedArgs {
@@ -76,7 +101,8 @@ struct FusedArgs {
     // t_end_ns}; trace[0] is the record counter, records start at trace[4]; nullptr: off
     unsigned long long *trace;
     int64_t trace_cap;      // records that fit after the counter
-    FrontArgs front;        // whole-layer launch only (FRONT = true)
+    FrontArgs front;        // whole-layer and expert-parallel launches
+    EpArgs ep;              // expert-parallel launch (world > 0)
 };
 
 enum : int { TRACE_L0 = 0, TRACE_L1 = 1, TRACE_COMBINE = 2 };
@@ -96,6 +122,24 @@ __device__ __forceinline__ void red_release_gpu_add(int *p, int v)
 __device__ __forceinline__ void st_release_gpu(int *p, int v)
 {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// system scope (flags and counters that other GPUs write or read over NVLink)
+__device__ __forceinline__ int ld_acquire_sys(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.sys.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_sys_add(int *p, int v)
+{
+    asm volatile("red.release.sys.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_release_sys(int *p, int v)
+{
+    asm volatile("st.release.sys.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_global()
@@ -129,19 +173,22 @@ __device__ __forceinline__ void trace_record(const FusedArgs &fa, int kind, int 
     r[3] = t1;
 }
 
-// Bounded wait for *p >= target with acquire semantics. False after an abort elsewhere in
-// the CTA or after timeout_ns (then the abort flag is raised and DEV_TIMEOUT recorded).
+// Bounded wait for *p >= target with acquire semantics (gpu scope, or system scope for
+// values that other GPUs write). False after an abort elsewhere in the CTA or after
+// timeout_ns (then the abort flag is raised and DEV_TIMEOUT recorded).
+template <bool SYS = false>
 __device__ __forceinline__ bool flag_wait_bounded(const int *p, int target, volatile int *abort_flag,
                                                   int64_t timeout_ns, int *status, int where)
 {
-    if (ld_acquire_gpu(p) >= target) return true;
+    auto ld = [](const int *q) { return SYS ? ld_acquire_sys(q) : ld_acquire_gpu(q); };
+    if (ld(p) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t nap = 64; // exponential backoff up to 2 us: pollers stay off the L2 meanwhile
 #pragma unroll 1
     while (true) {
         __nanosleep(nap);
         if (nap < 2048) nap <<= 1;
-        if (ld_acquire_gpu(p) >= target) return true;
+        if (ld(p) >= target) return true;
         if (*abort_flag) return false;
         if ((int64_t)(globaltimer_ns() - t0) > timeout_ns) {
             *abort_flag = 1;
@@ -154,13 +201,17 @@ __device__ __forceinline__ bool flag_wait_bounded(const int *p, int target, vola
 // Grid-wide barrier of a persistent launch (every CTA resident): the CTA's threads meet, thread
 // 0 publishes the CTA's writes and waits, bounded, until `target` CTA arrivals have been
 // counted on `ctr` (a launch-wide counter: the n-th barrier of the launch waits for n * grid).
+// sys: the CTAs' earlier stores also went to other GPUs, and are made visible at system
+// scope before the arrival.
 __device__ __forceinline__ bool grid_barrier(int *ctr, int target, volatile int *abort_flag,
-                                             int64_t timeout_ns, int *status, int where)
+                                             int64_t timeout_ns, int *status, int where,
+                                             bool sys = false)
 {
     __syncthreads();
     int ok = 1;
     if (threadIdx.x == 0) {
-        __threadfence();
+        if (sys) __threadfence_system();
+        else __threadfence();
         red_release_gpu_add(ctr, 1);
         ok = flag_wait_bounded(ctr, target, abort_flag, timeout_ns, status, where) ? 1 : 0;
     }
@@ -169,12 +220,12 @@ __device__ __forceinline__ bool grid_barrier(int *ctr, int target, volatile int 
 
 // Routing, dispatch and the row copy of the whole-layer launch, in the GEMM stages' shared
 // memory (free until the GEMM phases start). False when a wait gave up.
+// Routing of the CTA's token groups (cta, cta + ncta, ...) in the GEMM stages' shared memory.
 template <int G>
-__device__ __forceinline__ bool fused_front(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
-                                            const FusedArgs &fa, uint8_t *smem,
-                                            volatile int *abort_flag, int *status, int64_t tmo)
+__device__ __forceinline__ bool front_route(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
+                                            const FrontArgs &f, uint8_t *smem,
+                                            volatile int *abort_flag, int cta, int ncta)
 {
-    const FrontArgs &f = fa.front;
     const RcLayout L = rc_layout(f.ra.tt, f.ra.E, 4 * G, f.ra.stages);
     if (threadIdx.x == 0) {
         rc_init(smem, L, f.ra.stages, f.ncw);
@@ -182,20 +233,220 @@ __device__ __forceinline__ bool fused_front(const CUtensorMap *tmRX, const CUten
         tma_prefetch_desc(tmRW);
     }
     __syncthreads();
-    bool ok = rc_run<4, G>(tmRX, tmRW, f.ra, smem, 0, 2, f.ncw, blockIdx.x, gridDim.x, f.n_groups, 1);
+    bool ok = rc_run<4, G>(tmRX, tmRW, f.ra, smem, 0, 2, f.ncw, cta, ncta, f.n_groups, 1);
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
     if (threadIdx.x == 0) rc_fini(smem, L, f.ra.stages);
-    if (!ok) {
-        *abort_flag = 1;
-        return false;
-    }
+    if (!ok) *abort_flag = 1;
+    return ok;
+}
+
+__device__ __forceinline__ bool front_route_any(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
+                                                const FrontArgs &f, uint8_t *smem,
+                                                volatile int *abort_flag, int cta, int ncta)
+{
+    // consumer threads per token: 4 experts each
+    if (f.ra.E <= 8) return front_route<2>(tmRX, tmRW, f, smem, abort_flag, cta, ncta);
+    if (f.ra.E <= 16) return front_route<4>(tmRX, tmRW, f, smem, abort_flag, cta, ncta);
+    return front_route<8>(tmRX, tmRW, f, smem, abort_flag, cta, ncta);
+}
+
+// Routing, dispatch and the row copy of the whole-layer launch (E == 8). False when a wait
+// gave up.
+__device__ __forceinline__ bool fused_front(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
+                                            const FusedArgs &fa, uint8_t *smem,
+                                            volatile int *abort_flag, int *status, int64_t tmo,
+                                            int cta, int ncta)
+{
+    const FrontArgs &f = fa.front;
+    if (!front_route<2>(tmRX, tmRW, f, smem, abort_flag, cta, ncta)) return false;
     // every CTA's routing (top-k and per-group counts) is complete
-    if (!grid_barrier(f.gbar, (int)gridDim.x, abort_flag, tmo, status, 350)) return false;
-    dispatch_front(f.fd, blockIdx.x, gridDim.x, reinterpret_cast<int *>(smem));
+    if (!grid_barrier(f.gbar, ncta, abort_flag, tmo, status, 350)) return false;
+    dispatch_front(f.fd, cta, ncta, cta == 0, reinterpret_cast<int *>(smem));
     // every CTA's rows, indices and (CTA 0) the dispatch outputs are in place
-    if (!grid_barrier(f.gbar, 2 * (int)gridDim.x, abort_flag, tmo, status, 351)) return false;
+    if (!grid_barrier(f.gbar, 2 * ncta, abort_flag, tmo, status, 351)) return false;
     fence_proxy_async_global(); // x_perm was written by generic stores; layer0 reads it by TMA
     return true;
+}
+
+// Offsets of the expert-parallel launch, after every rank's group counts have arrived
+// (all CTAs; scratch in shared memory): where each of this rank's pairs goes (destination
+// rank and row, into ep.dest / ep.slot), and on CTA 0 this rank's receive-side dispatch
+// outputs for its e_loc experts (the tile list of its GEMMs, pad markers) and the cleared
+// ready counters of its GEMM phases.
+__device__ __forceinline__ void ep_offsets(const FusedArgs &fa, int cta, int ncta, int *scratch)
+{
+    const EpArgs &ep = fa.ep;
+    const FrontArgs &f = fa.front;
+    const ScanOut &so = f.fd.so;
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int W = ep.world, E = f.ra.E, EL = ep.e_loc, G = f.n_groups, k = f.ra.k;
+    int *tot = scratch;                         // [W][E] rows per source rank and expert
+    int *pref = tot + W * E;                    // [G][E] this rank's prefix over its groups
+    int *poffD = pref + (size_t)G * E;          // [W][EL + 1] padded offsets of every rank
+    int *cntL = poffD + W * (EL + 1);           // [EL] rows of this rank's experts
+    int *base = cntL + EL;                      // [E] rows of lower source ranks per expert
+    uint32_t *bits = reinterpret_cast<uint32_t *>(base + E); // [E][4] group token bitmap
+    const int32_t *ac = ep.all_counts[ep.rank];  // this rank's copy: [W][G][E]
+    // 1. totals per source and expert; this rank's exclusive prefix over its groups
+    for (int i = warp; i < W * E; i += nw) {
+        const int sr = i / E, e = i - sr * E;
+        const int32_t *c = ac + (size_t)sr * G * E + e;
+        int run = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            const int v = g < G ? c[(size_t)g * E] : 0;
+            const int inc = warp_inclusive_scan(v, lane);
+            if (sr == ep.rank && g < G) pref[(size_t)g * E + e] = run + inc - v;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) tot[sr * E + e] = run;
+    }
+    __syncthreads();
+    // 2. every rank's padded offsets (warp d: rank d's experts), the bases, and (CTA 0) the
+    //    scan outputs of this rank's experts
+    for (int d = warp; d < W; d += nw) {
+        int c = 0;
+        if (lane < EL)
+            for (int sr = 0; sr < W; ++sr) c += tot[sr * E + d * EL + lane];
+        if (d == ep.rank && cta == 0) {
+            dispatch_scan_warp(c, EL, so, poffD + d * (EL + 1), lane);
+        } else {
+            const int ntile = (c + M_TILE - 1) / M_TILE;
+            const int inc_t = warp_inclusive_scan(ntile, lane);
+            if (lane < EL) poffD[d * (EL + 1) + lane] = (inc_t - ntile) * M_TILE;
+            if (lane == EL - 1) poffD[d * (EL + 1) + EL] = inc_t * M_TILE;
+        }
+        if (d == ep.rank && lane < EL) cntL[lane] = c;
+    }
+    for (int e = tid; e < E; e += nt) {
+        int b = 0;
+        for (int sr = 0; sr < ep.rank; ++sr) b += tot[sr * E + e];
+        base[e] = b;
+    }
+    if (cta == 0)
+        for (int i = tid; i < so.n_ready; i += nt) so.ready[i] = 0;
+    __syncthreads();
+    if (cta == 0) {
+        // pad rows: no token (-1), gate 0, no origin (their layer1 rows are not returned)
+        const int *pl = poffD + ep.rank * (EL + 1);
+        scan_write_pads(EL, so, pl, cntL, tid, nt);
+        long long *org = ep.recv_origin[ep.rank];
+        for (int ex = warp; ex < EL; ex += nw)
+            for (int r = pl[ex] + cntL[ex] + lane; r < pl[ex + 1]; r += 32) org[r] = -1;
+    }
+    // 3. destinations of this rank's pairs: rank d = e / e_loc, row = d's padded offset of
+    //    the expert + rows of lower source ranks + this rank's earlier groups + the token's
+    //    rank in its group
+    for (int g = cta; g < G; g += ncta) {
+        const int t0 = g * f.ra.tt;
+        const int ntg = min(f.ra.tt, f.ra.T - t0);
+        for (int i = tid; i < 4 * E; i += nt) bits[i] = 0u;
+        __syncthreads();
+        const int P = ntg * k;
+        const size_t q0 = (size_t)t0 * k;
+        for (int q = tid; q < P; q += nt) {
+            const int tl = q / k;
+            const int e = f.ra.topk_idx[q0 + q];
+            if (e >= 0 && e < E) atomicOr(&bits[e * 4 + (tl >> 5)], 1u << (tl & 31));
+        }
+        __syncthreads();
+        for (int q = tid; q < P; q += nt) {
+            const int tl = q / k;
+            const int e = f.ra.topk_idx[q0 + q];
+            if (e < 0 || e >= E) {
+                ep.dest[q0 + q] = -1;
+                continue;
+            }
+            const uint32_t *b = bits + e * 4;
+            const int wd = tl >> 5;
+            int rk = __popc(b[wd] & ((1u << (tl & 31)) - 1u));
+            for (int w = 0; w < wd; ++w) rk += __popc(b[w]);
+            const int d = e / EL;
+            ep.dest[q0 + q] = d;
+            ep.slot[q0 + q] = poffD[d * (EL + 1) + (e - d * EL)] + base[e] + pref[(size_t)g * E + e] + rk;
+        }
+        __syncthreads();
+    }
+}
+
+// Shared-memory scratch of ep_offsets, in ints.
+__host__ __device__ inline int ep_scratch_ints(int world, int E, int e_loc, int n_groups)
+{
+    return world * E + n_groups * E + world * (e_loc + 1) + e_loc + E + 4 * E;
+}
+
+// The front of the expert-parallel launch: routing of this rank's tokens, their group
+// counts published to every rank, a barrier of all ranks (each rank's flag in every rank's
+// memory), the offsets, and a barrier of this rank's CTAs.
+__device__ __forceinline__ bool ep_front(const CUtensorMap *tmRX, const CUtensorMap *tmRW,
+                                         const FusedArgs &fa, uint8_t *smem,
+                                         volatile int *abort_flag, int *status, int64_t tmo,
+                                         int cta, int ncta)
+{
+    const FrontArgs &f = fa.front;
+    const EpArgs &ep = fa.ep;
+    const int E = f.ra.E, G = f.n_groups;
+    if (!front_route_any(tmRX, tmRW, f, smem, abort_flag, cta, ncta)) return false;
+    // this CTA's groups' counts into every rank's copy; CTA 0 clears this rank's receive
+    // counters (no rank writes them before this rank's flag is up)
+    for (int g = cta; g < G; g += ncta)
+        for (int i = threadIdx.x; i < ep.world * E; i += blockDim.x) {
+            const int d = i / E, e = i - d * E;
+            ep.all_counts[d][((size_t)ep.rank * G + g) * E + e] = f.ra.group_counts[(size_t)g * E + e];
+        }
+    if (cta == 0) {
+        for (int i = threadIdx.x; i < ep.max_tiles; i += blockDim.x) ep.arrive[ep.rank][i] = 0;
+        for (int i = threadIdx.x; i < fa.T; i += blockDim.x) ep.back_cnt[ep.rank][i] = 0;
+    }
+    if (!grid_barrier(f.gbar, ncta, abort_flag, tmo, status, 360, true)) return false;
+    // every rank: its counts are everywhere and its receive counters are clear
+    if (cta == 0 && threadIdx.x == 0) {
+        __threadfence_system();
+        for (int d = 0; d < ep.world; ++d) st_release_sys(ep.flags[d] + ep.rank, ep.epoch);
+    }
+    int ok = 1;
+    if (threadIdx.x == 0)
+        for (int sr = 0; sr < ep.world && ok; ++sr)
+            ok = flag_wait_bounded<true>(ep.flags[ep.rank] + sr, ep.epoch, abort_flag, tmo, status, 361) ? 1 : 0;
+    if (!__syncthreads_and(ok)) return false;
+    ep_offsets(fa, cta, ncta, reinterpret_cast<int *>(smem));
+    return grid_barrier(f.gbar, 2 * ncta, abort_flag, tmo, status, 362);
+}
+
+// The data-movement warps' scatter of the expert-parallel launch (after ep_front; four
+// warps, `dw` 0..3): each of this CTA's pairs sends its token's x row, gate and origin to
+// its destination row, then counts the row on the destination's M tile (after a
+// system-scope fence, so the destination's layer0 may read the row once the count is up).
+__device__ __forceinline__ void ep_scatter(const FusedArgs &fa, int cta, int ncta, int dw, int lane)
+{
+    const EpArgs &ep = fa.ep;
+    const FrontArgs &f = fa.front;
+    const int k = f.ra.k, H = f.fd.H, G = f.n_groups;
+    const int chunks = H / 8;
+    for (int g = cta; g < G; g += ncta) {
+        const int t0 = g * f.ra.tt;
+        const int P = min(f.ra.tt, f.ra.T - t0) * k;
+        const size_t q0 = (size_t)t0 * k;
+        for (int qq = dw; qq < P; qq += 4) {
+            const size_t q = q0 + qq;
+            const int d = ep.dest[q];
+            if (d < 0 || d >= ep.world) continue;
+            const int slot = ep.slot[q];
+            if (slot < 0 || (int64_t)slot >= ep.recv_cap) continue;
+            const int t = (int)(q / k);
+            const uint4 *src = reinterpret_cast<const uint4 *>(f.fd.x + (size_t)t * H);
+            uint4 *dst = reinterpret_cast<uint4 *>(ep.recv_rows[d] + (size_t)slot * H);
+#pragma unroll 4
+            for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+            if (lane == 0) {
+                ep.recv_gate[d][slot] = f.ra.topk_w[q];
+                ep.recv_origin[d][slot] = ((long long)ep.rank << 32) | (long long)q;
+            }
+            __threadfence_system();
+            __syncwarp();
+            if (lane == 0) red_release_sys_add(ep.arrive[d] + (slot >> 7), 1);
+        }
+    }
 }
 
 struct FusedItem {
@@ -225,15 +476,26 @@ __device__ __forceinline__ bool combine_rows_ready(const FusedArgs &fa, const in
 {
     const uint64_t t_start = globaltimer_ns();
     uint32_t nap = 64;
+    const bool ep = fa.ep.world > 0;
+    // expert parallelism: every stripe of the token's k rows has come back
+    const int ep_need = fa.k * fa.l1.n_tiles;
 #pragma unroll 1
     while (true) {
         bool ready = true;
-        for (int q = lane; q < 8 * fa.k; q += 32) {
-            const int tok = t[0] + (q & 7) * 4; // t[i] = t[0] + 4 i
-            if (tok >= fa.T) continue;
-            const int rr = fa.inv_pos[(size_t)tok * fa.k + (q >> 3)];
-            if (rr < 0 || (int64_t)rr >= fa.ys_rows || (rr >> 7) >= fa.max_tiles) continue;
-            if (ld_acquire_gpu(flags + (rr >> 7)) == 0) ready = false;
+        if (ep) {
+            if (lane < 8) {
+                const int tok = t[0] + lane * 4;
+                if (tok < fa.T && ld_acquire_sys(fa.ep.back_cnt[fa.ep.rank] + tok) < ep_need)
+                    ready = false;
+            }
+        } else {
+            for (int q = lane; q < 8 * fa.k; q += 32) {
+                const int tok = t[0] + (q & 7) * 4; // t[i] = t[0] + 4 i
+                if (tok >= fa.T) continue;
+                const int rr = fa.inv_pos[(size_t)tok * fa.k + (q >> 3)];
+                if (rr < 0 || (int64_t)rr >= fa.ys_rows || (rr >> 7) >= fa.max_tiles) continue;
+                if (ld_acquire_gpu(flags + (rr >> 7)) == 0) ready = false;
+            }
         }
         if (__all_sync(0xffffffffu, ready)) break;
         if (*abort_flag) return false;
@@ -260,7 +522,9 @@ __device__ __forceinline__ bool fused_combine(const FusedArgs &fa, int stripe, i
 {
     const int col = stripe * gemm::BN + lane * 8;
     const bool have_col = col < fa.H;
-    const __nv_bfloat16 *ys = fa.l1.out;
+    const bool ep = fa.ep.world > 0;
+    // expert parallelism: the returned rows, row t * k + j of the rank's own buffer
+    const __nv_bfloat16 *ys = ep ? fa.ep.back[fa.ep.rank] : fa.l1.out;
     const int *flags = fa.ready1 + (size_t)stripe * fa.max_tiles;
     for (int g = 0; g < fa.comb_tokens / 32; ++g) {
         int t[8];
@@ -282,8 +546,8 @@ __device__ __forceinline__ bool fused_combine(const FusedArgs &fa, int stripe, i
                 for (int i = 0; i < 8; ++i) {
                     u[jj][i] = make_uint4(0u, 0u, 0u, 0u);
                     if (j < fa.k && t[i] < fa.T) {
-                        const int r = fa.inv_pos[(size_t)t[i] * fa.k + j];
-                        if (r >= 0 && (int64_t)r < fa.ys_rows && (r >> 7) < fa.max_tiles) {
+                        const int r = ep ? t[i] * fa.k + j : fa.inv_pos[(size_t)t[i] * fa.k + j];
+                        if (ep || (r >= 0 && (int64_t)r < fa.ys_rows && (r >> 7) < fa.max_tiles)) {
                             if (have_col)
                                 u[jj][i] = *reinterpret_cast<const uint4 *>(ys + (size_t)r * fa.H + col);
                         } else if (lane == 0) {
@@ -357,16 +621,17 @@ __device__ __forceinline__ bool combine_queue(const FusedArgs &fa, int group_war
     return ok;
 }
 
-// FRONT: the launch also routes and dispatches the tokens first (the whole layer in one
-// launch; its router tensor maps tmRX, tmRW are used only then).
-template <int KIND0, bool FRONT>
-__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
-    moe_fused_layer_kernel(const __grid_constant__ CUtensorMap tmA0,
-                           const __grid_constant__ CUtensorMap tmW1,
-                           const __grid_constant__ CUtensorMap tmH,
-                           const __grid_constant__ CUtensorMap tmW2,
-                           const __grid_constant__ CUtensorMap tmRX,
-                           const __grid_constant__ CUtensorMap tmRW, const FusedArgs fa)
+// The persistent layer launch on CTAs cta = 0 .. ncta - 1 (one per SM, all resident).
+// MODE: FUSED_LAYERS layer0 -> layer1 -> combine; FUSED_WHOLE routes and dispatches the
+// tokens first (router maps tmRX, tmRW); FUSED_EP is the expert-parallel layer of one rank
+// (ep_front, then the data-movement warps scatter the rank's rows to their experts' ranks
+// while the GEMM pipeline runs the rank's experts on the rows that have arrived, layer1
+// returns each gated row to its origin, and the combine sums the rows that came back).
+template <int KIND0, int MODE>
+__device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const CUtensorMap &tmW1,
+                                                 const CUtensorMap &tmH, const CUtensorMap &tmW2,
+                                                 const CUtensorMap &tmRX, const CUtensorMap &tmRW,
+                                                 const FusedArgs &fa, int cta, int ncta)
 {
     using namespace gemm;
     extern __shared__ uint8_t smem_raw[];
@@ -392,8 +657,10 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     int *status = l0.status;
     const int64_t tmo = l0.timeout_ns;
     const bool a_tma = fa.a_tma != 0;
-    // layer0 epilogue parts: warps 2..5, and with A by TMA also warps 6..9 (half the chunks each)
-    const int parts0 = a_tma ? 8 : 4;
+    // layer0 epilogue parts: warps 2..5, and with A by TMA also warps 6..9 (half the chunks
+    // each; not in the expert-parallel launch, whose data-movement warps scatter rows then)
+    const bool split0 = a_tma && MODE != FUSED_EP;
+    const int parts0 = split0 ? 8 : 4;
     const int nch0 = (KIND0 == GEMM_SWIGLU) ? 4 : BN / 32;
 
     if (threadIdx.x == 0) {
@@ -426,7 +693,10 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     bool front_ok = true;
-    if constexpr (FRONT) front_ok = fused_front<2>(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo);
+    if constexpr (MODE == FUSED_WHOLE)
+        front_ok = fused_front(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo, cta, ncta);
+    if constexpr (MODE == FUSED_EP)
+        front_ok = ep_front(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo, cta, ncta);
 
     const int num_tiles = front_ok ? l0.meta->num_tiles : 0;
     const int total0 = num_tiles * l0.n_tiles;
@@ -442,8 +712,19 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             for (int i = 0; i < STAGES; ++i) armed[i] = -1;
             bool ok = true;
             bool all0 = false; // every layer0 item finished: no more per-tile waits
-            for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            for (int w = cta; ok && w < total; w += ncta) {
                 const FusedItem it = fused_item(w, fa, total0);
+                if (MODE == FUSED_EP && it.phase == 0) {
+                    // the tile's rows have arrived from their source ranks (count per M tile)
+                    const int first = l0.tile_off[it.e];
+                    const int need = min(BM, l0.expert_rows[it.e] - (it.mt - first) * BM);
+                    if (!flag_wait_bounded<true>(fa.ep.arrive[fa.ep.rank] + it.mt, need, abort_flag, tmo,
+                                                 status, 363)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global(); // rows written by generic stores, read by TMA
+                }
                 if (it.phase == 1) {
                     // layer1 needs every layer0 column tile of its M tile
                     if (!all0) all0 = ld_acquire_gpu(fa.done0) >= total0;
@@ -505,7 +786,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             uint32_t ph = 0;
             int n = 0; // accumulator tiles issued
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+            for (int w = cta; ok && w < total; w += ncta) {
                 const FusedItem it = fused_item(w, fa, total0);
                 const int acc = n & 1;
                 const uint32_t aph = (uint32_t)(n >> 1) & 1u;
@@ -557,9 +838,10 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         int gs = 0;
         uint32_t gph = 0;
         const int g = threadIdx.x - NUM_THREADS;
-        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        for (int w = cta; ok && w < total; w += ncta) {
             const FusedItem it = fused_item(w, fa, total0);
-            if (dm && it.phase == 1) break; // the data-movement warps serve layer0 items only
+            // the data-movement warps serve layer0 items only (none in the expert-parallel launch)
+            if (dm && (it.phase == 1 || MODE == FUSED_EP)) break;
             if (dm && !a_tma) {
                 // ---- A-row gather for a layer0 item (cp.async): thread g copies 16-byte chunk
                 // (g & 7) of rows (g >> 3) + 16 i; its 8 token ids are read once per tile and
@@ -608,18 +890,27 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             const int row = it.mt * BM + q * 32 + lane;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             if (it.phase == 0) {
-                const int c_lo = (a_tma && dm) ? nch0 / 2 : 0;
-                const int c_hi = a_tma ? c_lo + nch0 / 2 : -1;
+                const int c_lo = (split0 && dm) ? nch0 / 2 : 0;
+                const int c_hi = split0 ? c_lo + nch0 / 2 : -1;
                 epilogue_rows<KIND0>(l0, t_row, row, it.nt, 0, 0, nullptr, c_lo, c_hi);
             } else {
                 epilogue_rows<GEMM_SCALE>(l1, t_row, row, it.nt);
+                if (MODE == FUSED_EP) {
+                    // the row's stripe went to its origin: count it there once it is visible
+                    const long long o = l1.row_dst[row];
+                    if (o >= 0) {
+                        __threadfence_system();
+                        const int q = (int)(o & 0xffffffffll);
+                        red_release_sys_add(fa.ep.back_cnt[(int)(o >> 32)] + q / fa.k, 1);
+                    }
+                }
             }
             // The accumulator is free as soon as its TMEM reads are done (layer1 items with
             // eight epilogue parts configured: warps 2..5 stand for 6..9).
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive_cnt(tempty_bar(acc), (it.phase == 1 && a_tma) ? 2u : 1u);
+                mbar_arrive_cnt(tempty_bar(acc), (it.phase == 1 && split0) ? 2u : 1u);
             // Ready signal: every part makes its stores visible, then the last of the item's
             // parts publishes it. The part counters form a ring of 4 indexed by the CTA's item
             // count: slot n & 3 is reused by item n + 4, whose parts can only arrive after
@@ -647,6 +938,8 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
             ++n;
         }
         if (dm && !a_tma) cp_async_wait_all(); // this thread's copies land first
+        // expert parallelism: the data-movement warps send this rank's rows out first
+        if (MODE == FUSED_EP && dm && front_ok) ep_scatter(fa, cta, ncta, warp - 6, lane);
         // combine: the data-movement warps from the end of their layer0 duties (beside the
         // layer1 GEMM pipeline), the epilogue warps once this CTA's GEMM items are done
         // (each group of four warps decides together whether to go on: named barrier 2 for
@@ -664,6 +957,46 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+}
+
+// FRONT: the launch also routes and dispatches the tokens first (the whole layer in one
+// launch; its router tensor maps tmRX, tmRW are used only then).
+template <int KIND0, bool FRONT>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_fused_layer_kernel(const __grid_constant__ CUtensorMap tmA0,
+                           const __grid_constant__ CUtensorMap tmW1,
+                           const __grid_constant__ CUtensorMap tmH,
+                           const __grid_constant__ CUtensorMap tmW2,
+                           const __grid_constant__ CUtensorMap tmRX,
+                           const __grid_constant__ CUtensorMap tmRW, const FusedArgs fa)
+{
+    fused_layer_body<KIND0, FRONT ? FUSED_WHOLE : FUSED_LAYERS>(tmA0, tmW1, tmH, tmW2, tmRX, tmRW, fa,
+                                                               blockIdx.x, gridDim.x);
+}
+
+// The expert-parallel layer: one launch per GPU, each GPU a rank; or, to exercise several
+// ranks on one GPU, one launch holding n_local ranks (CTA b plays rank b % n_local; the
+// ranks' buffers all live on this GPU, and their waits on one another stay inside the
+// launch, whose CTAs are all resident).
+constexpr int EP_MAX_LOCAL = 4;
+struct EpRankMaps {
+    CUtensorMap a0, w1, h, w2, rx, rw;
+};
+struct EpLaunch {
+    EpRankMaps maps[EP_MAX_LOCAL];
+    FusedArgs fa[EP_MAX_LOCAL];
+    int n_local;
+};
+
+template <int KIND0>
+__global__ void __launch_bounds__(gemm::NUM_THREADS_GATHER, 1)
+    moe_ep_layer_kernel(const __grid_constant__ EpLaunch L)
+{
+    const int nl = L.n_local;
+    const int r = (int)(blockIdx.x % (unsigned)nl);
+    const EpRankMaps &m = L.maps[r];
+    fused_layer_body<KIND0, FUSED_EP>(m.a0, m.w1, m.h, m.w2, m.rx, m.rw, L.fa[r],
+                                      (int)(blockIdx.x / (unsigned)nl), (int)(gridDim.x / (unsigned)nl));
 }
 
 } // namespace moe

@@ -45,6 +45,9 @@
 
 namespace moe {
 
+// ranks of the expert-parallel layer at most (pointer tables travel in kernel parameters)
+constexpr int EP_MAX_WORLD = 8;
+
 namespace gemm {
 constexpr int BM = 128;
 constexpr int BN = 256;
@@ -149,6 +152,12 @@ struct GemmArgs {
     const int32_t *active_list; // BMODE_WGRAD: only these experts (meta->num_active of them)
     int epi8; // A by TMA (no gather): warps 6..9 join the epilogue, each pair of warps on one
               // TMEM lane quarter splits the item's column chunks (launch with 320 threads)
+    // Expert parallelism (GEMM_SCALE rows returned to their origin): row r's output goes to
+    // row (row_dst[r] & 0xffffffff) of peer_out[row_dst[r] >> 32] (another GPU's buffer:
+    // plain 16-byte stores), and is not stored at all where row_dst[r] < 0 (pad rows);
+    // row_dst == nullptr: rows go to `out`.
+    const long long *row_dst;
+    __nv_bfloat16 *peer_out[EP_MAX_WORLD];
 };
 
 __device__ __forceinline__ void gemm_map_work(int w, const GemmArgs &a, int &e, int &mt, int &nt,
@@ -306,13 +315,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs &args, uint32_t t_r
         }
     } else {
         __nv_bfloat16 *orow = args.out + (size_t)row * args.ld_out + nt * BN;
+        bool keep = true;
+        if (KIND == GEMM_SCALE && args.row_dst != nullptr) {
+            const long long o = args.row_dst[row];
+            keep = o >= 0;
+            if (keep)
+                orow = args.peer_out[(int)(o >> 32)] + (size_t)(o & 0xffffffffll) * args.ld_out + nt * BN;
+        }
         const float wt = (KIND == GEMM_SCALE) ? args.row_w[row] : 1.0f;
 #pragma unroll 1
         for (int c = c_lo; c < (c_hi < 0 ? BN / 32 : c_hi); ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_row + c * 32, r);
             tmem_ld_wait();
-            if (nt * BN + c * 32 < args.n_cols) {
+            if (keep && nt * BN + c * 32 < args.n_cols) {
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {

@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <memory>
 #include <mutex>
 
 #include "backward.cuh"
@@ -138,7 +139,8 @@ FilterPlan filter_plan(const moe_problem *p)
     return f;
 }
 
-Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd = false)
+Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd = false,
+                   bool no_rows = false)
 {
     Layout L{};
     const size_t T = (size_t)p->T, H = (size_t)p->H, F = (size_t)p->F, E = (size_t)p->E,
@@ -185,9 +187,11 @@ Layout make_layout(const moe_problem *p, int F_s = 0, bool fp8 = false, bool bwd
     L.inv_pos = take(T * K * 4);
     L.row_w = take(P * 4);
     L.end_dispatch = o;
-    L.x_perm = take(P * H * 2); // materialised gather, used by the CTA-pair GEMM variant
+    // materialised gather (large batches, the CTA-pair GEMM variant); no_rows: the rows live
+    // elsewhere (the expert-parallel layer's receive buffer) and layer1 writes no ys
+    L.x_perm = take(no_rows ? 0 : P * H * 2);
     L.h = take(P * F * 2);
-    L.ys = take(P * H * 2);
+    L.ys = take(no_rows ? 0 : P * H * 2);
     L.end_forward = o;
     L.x_stage = take(T * H * 2);
     L.out_stage = take(T * H * 2);
@@ -1575,6 +1579,244 @@ moe_status forward_impl_fp8(const moe_problem *p, const moe_bf16 *x, const moe_b
 
 } // namespace
 
+// ---------------------------------------------------------------------------------------
+// expert-parallel layer, one persistent launch per GPU (fused.cuh, FUSED_EP)
+// ---------------------------------------------------------------------------------------
+
+// Workspace of one rank: the receive side is a layer of E / world experts over
+// recv_cap = pmax of world * T * min(k, E / world) one-selection rows (its h, tile lists,
+// ready counters; the rows themselves are in the exchange buffers), then this rank's
+// routing, its group counts and its pairs' destinations.
+struct EpLayout {
+    moe_problem pr; // the receive side as a problem: T = rows, E = E / world, top_k = 1
+    Layout L;
+    int64_t recv_cap;
+    size_t topk_idx, topk_w, gcount, slot, dest, end;
+};
+
+bool ep_shape_ok(const moe_problem *p, int world)
+{
+    return check_problem(p) == MOE_OK && world >= 1 && world <= MOE_EP_MAX_WORLD &&
+           p->E % world == 0 && p->T > 0 && p->E % 8 == 0 && p->E <= 32 && p->H % 64 == 0;
+}
+
+EpLayout make_layout_ep(const moe_problem *p, int world)
+{
+    EpLayout X{};
+    const int el = p->E / world;
+    X.pr = *p;
+    X.pr.T = world * p->T * std::min(p->top_k, el);
+    X.pr.E = el;
+    X.pr.top_k = 1;
+    X.L = make_layout(&X.pr, 0, false, false, true);
+    X.recv_cap = X.L.pmax;
+    size_t o = X.L.end_forward;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align256(o + (bytes ? bytes : 1));
+        return at;
+    };
+    const size_t TK = (size_t)p->T * p->top_k;
+    X.topk_idx = take(TK * 4);
+    X.topk_w = take(TK * 4);
+    X.gcount = take(((size_t)p->T + 7) / 8 * p->E * 4);
+    X.slot = take(TK * 4);
+    X.dest = take(TK * 4);
+    X.end = o;
+    return X;
+}
+
+// Token groups and router ring of one rank's CTAs (ncta = SMs / n_local).
+struct EpPlan {
+    bool ok;
+    int ncta, G, tt, n_groups, ncw, stages;
+};
+
+EpPlan ep_plan(const moe_problem *p, int world, int n_local)
+{
+    EpPlan f{};
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    f.ncta = sms / n_local;
+    f.G = p->E <= 8 ? 2 : p->E <= 16 ? 4 : 8; // consumer threads per token (4 experts each)
+    f.tt = std::max(8, std::min(256 / f.G, (p->T + f.ncta - 1) / f.ncta));
+    f.n_groups = (p->T + f.tt - 1) / f.tt;
+    f.ncw = (f.tt * f.G + 31) / 32;
+    const int budget = gemm::STAGES * gemm::STAGE;
+    f.stages = RC_MAX_STAGES;
+    while (f.stages > 3 && rc_layout(f.tt, p->E, 4 * f.G, f.stages).total > budget) --f.stages;
+    const int el = p->E / world;
+    f.ok = f.ncta >= 1 && rc_layout(f.tt, p->E, 4 * f.G, f.stages).total <= budget &&
+           (int64_t)ep_scratch_ints(world, p->E, el, f.n_groups) * 4 <= budget;
+    return f;
+}
+
+template <int KIND0>
+cudaError_t launch_ep_layer(const EpLaunch &L, int grid, cudaStream_t st)
+{
+    auto kern = moe_ep_layer_kernel<KIND0>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, gemm::NUM_THREADS_GATHER, gemm::SMEM_BYTES, st>>>(L);
+    return cudaGetLastError();
+}
+
+moe_status ep_layer_impl(const moe_ep_rank *ranks, int n_local, cudaStream_t st)
+{
+    if (ranks == nullptr || n_local < 1 || n_local > MOE_EP_MAX_LOCAL) return MOE_ERR_INVALID_ARG;
+    const moe_problem *p = &ranks[0].p;
+    const int world = ranks[0].world;
+    if (!ep_shape_ok(p, world)) return MOE_ERR_INVALID_ARG;
+    const EpPlan plan = ep_plan(p, world, n_local);
+    if (!plan.ok) return MOE_ERR_INVALID_ARG;
+    const EpLayout X = make_layout_ep(p, world);
+    const int el = p->E / world;
+    const int F = p->F, H = p->H;
+    const bool gated = (p->act == MOE_ACT_SWIGLU);
+    static_assert(MOE_EP_MAX_LOCAL == EP_MAX_LOCAL && MOE_EP_MAX_WORLD == EP_MAX_WORLD, "limits");
+    auto *Lp = new EpLaunch(); // large: kept off the stack
+    std::unique_ptr<EpLaunch> hold(Lp);
+    EpLaunch &L = *Lp;
+    L.n_local = n_local;
+    for (int i = 0; i < n_local; ++i) {
+        const moe_ep_rank &R = ranks[i];
+        const moe_problem &q = R.p;
+        if (q.T != p->T || q.H != p->H || q.F != p->F || q.E != p->E || q.top_k != p->top_k ||
+            q.act != p->act || q.gate != p->gate || R.world != world || R.rank < 0 ||
+            R.rank >= world || R.epoch <= 0)
+            return MOE_ERR_INVALID_ARG;
+        for (int j = 0; j < i; ++j)
+            if (ranks[j].rank == R.rank) return MOE_ERR_INVALID_ARG;
+        if (R.ws == nullptr || R.ws_bytes < X.end) return MOE_ERR_WORKSPACE;
+        if (R.x == nullptr || R.Wg == nullptr || R.W1 == nullptr || R.W2 == nullptr ||
+            R.out == nullptr || !aligned16(R.x) || !aligned16(R.Wg) || !aligned16(R.W1) ||
+            !aligned16(R.W2) || !aligned16(R.out) || !aligned16(R.ws) || !aligned4(R.bias) ||
+            !aligned4(R.topk_idx) || !aligned4(R.topk_w))
+            return MOE_ERR_INVALID_ARG;
+        for (int b = 0; b < MOE_EP_NUM_BUFFERS; ++b)
+            for (int d = 0; d < world; ++d)
+                if (R.buf[b][d] == nullptr || !aligned16(R.buf[b][d])) return MOE_ERR_INVALID_ARG;
+
+        void *ws = R.ws;
+        const Layout &LL = X.L;
+        const DispatchOut d = dispatch_bufs(ws, LL);
+        int *status = at<int>(ws, LL.status);
+        moe_bf16 *h = at<moe_bf16>(ws, LL.h);
+        int32_t *topk_idx = R.topk_idx ? R.topk_idx : at<int32_t>(ws, X.topk_idx);
+        float *topk_w = R.topk_w ? R.topk_w : at<float>(ws, X.topk_w);
+        auto *recv_rows = reinterpret_cast<const moe_bf16 *>(R.buf[2][R.rank]);
+        EpRankMaps &m = L.maps[i];
+        if (!make_map_2d(&m.a0, recv_rows, (uint64_t)X.recv_cap, (uint64_t)H, gemm::BM) ||
+            !make_map_3d(&m.w1, R.W1, (uint64_t)el, (uint64_t)H, (uint64_t)(gated ? 2 * F : F)) ||
+            !make_map_2d(&m.h, h, (uint64_t)X.recv_cap, (uint64_t)F, gemm::BM) ||
+            !make_map_3d(&m.w2, R.W2, (uint64_t)el, (uint64_t)F, (uint64_t)H) ||
+            !make_map_2d(&m.rx, R.x, (uint64_t)p->T, (uint64_t)H, (uint32_t)plan.tt) ||
+            !make_map_2d_plain(&m.rw, R.Wg, (uint64_t)H, (uint64_t)p->E, (uint32_t)p->E, RC_HC))
+            return MOE_ERR_CUDA;
+
+        GemmArgs a0{};
+        a0.tile_off = d.tile_off;
+        a0.tile_expert = d.tile_expert;
+        a0.ptile_off = d.ptile_off;
+        a0.ptile_expert = d.ptile_expert;
+        a0.expert_rows = d.counts;
+        a0.hot_off = d.hot_off;
+        a0.hot_tile_expert = d.hot_tile_expert;
+        a0.cold_tile = d.cold_tile;
+        a0.meta = d.meta;
+        a0.gather_len = X.recv_cap;
+        a0.out = reinterpret_cast<__nv_bfloat16 *>(h);
+        a0.ld_out = F;
+        a0.n_cols = F;
+        a0.k_blocks = H / gemm::BK;
+        a0.up_col = F;
+        a0.act = p->act;
+        a0.status = status;
+        a0.timeout_ns = g_timeout_ns.load();
+        a0.n_tiles = gated ? (F + 127) / 128 : (F + gemm::BN - 1) / gemm::BN;
+        GemmArgs a1 = a0;
+        a1.row_w = reinterpret_cast<const float *>(R.buf[3][R.rank]);
+        a1.out = reinterpret_cast<__nv_bfloat16 *>(h); // unused: every row is returned or skipped
+        a1.row_dst = reinterpret_cast<const long long *>(R.buf[4][R.rank]);
+        for (int dd = 0; dd < world; ++dd) a1.peer_out[dd] = reinterpret_cast<__nv_bfloat16 *>(R.buf[6][dd]);
+        a1.ld_out = H;
+        a1.n_cols = H;
+        a1.n_tiles = (H + gemm::BN - 1) / gemm::BN;
+        a1.k_blocks = F / gemm::BK;
+
+        FusedArgs &fa = L.fa[i];
+        fa = FusedArgs{};
+        fa.l0 = a0;
+        fa.l1 = a1;
+        fa.ready0 = d.ready;
+        fa.ready1 = d.ready + LL.max_tiles;
+        fa.done0 = d.ready + LL.n_ready - 2;
+        fa.comb_next = d.ready + LL.n_ready - 1;
+        fa.max_tiles = LL.max_tiles;
+        fa.inv_pos = d.inv_pos;
+        fa.out = reinterpret_cast<__nv_bfloat16 *>(R.out);
+        fa.T = p->T;
+        fa.H = H;
+        fa.k = p->top_k;
+        fa.ys_rows = (int64_t)p->T * p->top_k;
+        fa.a_tma = 1;
+        fa.comb_tokens = fused_plan(p).comb_tokens;
+        fa.fault_skip = -1;
+        fa.trace = i == 0 ? g_trace.load() : nullptr;
+        fa.trace_cap = g_trace_cap.load();
+        FrontArgs &f = fa.front;
+        f.ra.bias = R.bias;
+        f.ra.topk_idx = topk_idx;
+        f.ra.topk_w = topk_w;
+        f.ra.T = p->T;
+        f.ra.H = H;
+        f.ra.E = p->E;
+        f.ra.k = p->top_k;
+        f.ra.gate = p->gate;
+        f.ra.tt = plan.tt;
+        f.ra.stages = plan.stages;
+        f.ra.status = status;
+        f.ra.timeout_ns = a0.timeout_ns;
+        f.ra.group_counts = at<int32_t>(ws, X.gcount);
+        f.ncw = plan.ncw;
+        f.n_groups = plan.n_groups;
+        f.fd.T = p->T;
+        f.fd.E = el;
+        f.fd.k = p->top_k;
+        f.fd.H = H;
+        f.fd.x = reinterpret_cast<const __nv_bfloat16 *>(R.x);
+        f.fd.so = scan_out(LL, d);
+        f.fd.so.row_w = reinterpret_cast<float *>(R.buf[3][R.rank]); // pad rows: gate 0
+        f.gbar = status + 4;
+        EpArgs &ep = fa.ep;
+        ep.world = world;
+        ep.rank = R.rank;
+        ep.e_loc = el;
+        ep.epoch = R.epoch;
+        for (int dd = 0; dd < world; ++dd) {
+            ep.all_counts[dd] = reinterpret_cast<int32_t *>(R.buf[0][dd]);
+            ep.flags[dd] = reinterpret_cast<int *>(R.buf[1][dd]);
+            ep.recv_rows[dd] = reinterpret_cast<__nv_bfloat16 *>(R.buf[2][dd]);
+            ep.recv_gate[dd] = reinterpret_cast<float *>(R.buf[3][dd]);
+            ep.recv_origin[dd] = reinterpret_cast<long long *>(R.buf[4][dd]);
+            ep.arrive[dd] = reinterpret_cast<int *>(R.buf[5][dd]);
+            ep.back[dd] = reinterpret_cast<__nv_bfloat16 *>(R.buf[6][dd]);
+            ep.back_cnt[dd] = reinterpret_cast<int *>(R.buf[7][dd]);
+        }
+        ep.recv_cap = X.recv_cap;
+        ep.max_tiles = LL.max_tiles;
+        ep.slot = at<int32_t>(ws, X.slot);
+        ep.dest = at<int32_t>(ws, X.dest);
+        // status word and grid-barrier counter start from zero
+        cudaError_t e = cudaMemsetAsync(status, 0, 32, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    const int grid = n_local * plan.ncta;
+    const cudaError_t e = gated ? launch_ep_layer<GEMM_SWIGLU>(L, grid, st)
+                                : launch_ep_layer<GEMM_ACT>(L, grid, st);
+    return to_status(e);
+}
+
 extern "C" {
 
 int moe_forward_launches(const moe_problem *p)
@@ -2097,6 +2339,33 @@ moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y, const int6
         n_recv, H, world, back_rows, reinterpret_cast<__nv_bfloat16 *const *>(back),
         static_cast<int *>(ws));
     return to_status(cudaGetLastError());
+}
+
+moe_status moe_ep_buffer_sizes(const moe_problem *p, int32_t world, int64_t *sizes)
+{
+    if (sizes == nullptr || !ep_shape_ok(p, world)) return MOE_ERR_INVALID_ARG;
+    const EpLayout X = make_layout_ep(p, world);
+    const int64_t T = p->T, H = p->H, E = p->E, k = p->top_k;
+    sizes[0] = (int64_t)world * ((T + 7) / 8) * E * 4; // counts [world][groups][E]
+    sizes[1] = (int64_t)world * 4;                     // flags
+    sizes[2] = X.recv_cap * H * 2;                     // recv_rows
+    sizes[3] = X.recv_cap * 4;                         // recv_gate
+    sizes[4] = X.recv_cap * 8;                         // recv_origin
+    sizes[5] = (int64_t)X.L.max_tiles * 4;             // arrive
+    sizes[6] = T * k * H * 2;                          // back
+    sizes[7] = T * 4;                                  // back_cnt
+    return MOE_OK;
+}
+
+size_t moe_ep_workspace_size(const moe_problem *p, int32_t world)
+{
+    if (!ep_shape_ok(p, world)) return 0;
+    return make_layout_ep(p, world).end;
+}
+
+moe_status moe_ep_layer_forward(const moe_ep_rank *ranks, int32_t n_local, void *stream)
+{
+    return ep_layer_impl(ranks, n_local, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t moe_backward_workspace_size(const moe_problem *p)

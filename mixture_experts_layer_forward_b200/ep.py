@@ -27,6 +27,16 @@ stored straight into the destination's receive buffers (symmetric memory every r
 address), and the host never reads the routing; the ranks meet at device barriers between
 the steps. Not measured on several GPUs here (one GPU per run); its one-rank form is tested
 against moe_forward.
+
+EpLayer is the layer with the exchange overlapped with the expert GEMMs, one persistent launch
+per GPU (moe_ep_layer_forward, csrc/fused.cuh): the rows are stored into the experts' ranks'
+expert-sorted receive buffers by four warps per SM while the same SMs run the rank's experts,
+a layer0 tile starting as soon as its rows have arrived (an arrival count per tile, Comet
+§3.1.2 and §4; the tile-signalling abstract); layer1 stores every gated row straight into its
+origin's return buffer and counts it there, and the origin's combine sums a token's rows as
+soon as they are all back. ep_layer_forward_local runs several ranks in one launch on one
+GPU (each rank a share of the SMs, all buffers on this GPU): the same kernels and waits as
+one GPU per rank, which is how the ranks' interplay is tested here.
 """
 from __future__ import annotations
 
@@ -222,3 +232,74 @@ def ep_moe_forward_device(xch: DeviceExchange, x, Wg, bias, W1_local, W2_local):
     out = torch.empty(T, p.H, dtype=torch.bfloat16, device=dev)
     moe.moe_combine(p, xch.bufs["back"], xch.identity, out)
     return out
+
+
+def ep_layer_buffers(p, world: int, device=None):
+    """One rank's exchange buffers for moe_ep_layer_forward, zero-filled (plain device
+    tensors: for several ranks on one GPU)."""
+    from . import _native as moe
+
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    return [torch.zeros(max(n, 16), dtype=torch.uint8, device=dev)
+            for n in moe.moe_ep_buffer_sizes(p, world)]
+
+
+def ep_layer_forward_local(p, xs, Wg, bias, W1s, W2s, outs, bufs, wss, epoch: int,
+                           stream=None):
+    """The expert-parallel layer for world = len(xs) ranks in one launch on this GPU: rank r's
+    tokens xs[r] [T, H], its experts W1s[r] [E/world, H, 2F], W2s[r] [E/world, F, H], its
+    output outs[r] [T, H], its buffers bufs[r] (ep_layer_buffers) and workspace wss[r]
+    (moe_ep_workspace_size bytes). epoch: 1, 2, ... on successive calls with these buffers."""
+    from . import _native as moe
+
+    world = len(xs)
+    if world > moe.EP_MAX_LOCAL:
+        raise ValueError(f"at most {moe.EP_MAX_LOCAL} ranks in one launch")
+    table = [[bufs[d][b] for d in range(world)] for b in range(len(moe.EP_BUFFERS))]
+    ranks = [moe.ep_rank(p, world, r, epoch, xs[r], Wg, bias, W1s[r], W2s[r], outs[r], wss[r],
+                         table) for r in range(world)]
+    moe.moe_ep_layer_forward(ranks, stream)
+
+
+class EpLayer:
+    """The expert-parallel layer, one GPU per rank (moe_ep_layer_forward with one rank per
+    launch). The exchange buffers are symmetric allocations (every rank addresses every
+    rank's copy); the ranks must create it together (a collective) and then call forward
+    together, once per layer call."""
+
+    def __init__(self, p, group=None, device=None):
+        import torch.distributed._symmetric_memory as symm_mem
+
+        from . import _native as moe
+
+        self.group = group if group is not None else dist.group.WORLD
+        self.world = dist.get_world_size(self.group)
+        self.rank = dist.get_rank(self.group)
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        experts_per_rank(p.E, self.world)
+        self.p = p
+        self.epoch = 0
+        self.bufs, self.handles, self.table = [], [], []
+        for n in moe.moe_ep_buffer_sizes(p, self.world):
+            t = symm_mem.empty(max(n, 16), dtype=torch.uint8, device=dev)
+            t.zero_()
+            h = symm_mem.rendezvous(t, self.group)
+            off = t.data_ptr() - h.buffer_ptrs[self.rank]
+            self.bufs.append(t)
+            self.handles.append(h)
+            self.table.append([int(b) + off for b in h.buffer_ptrs])
+        self.ws = torch.empty(moe.moe_ep_workspace_size(p, self.world), dtype=torch.uint8,
+                              device=dev)
+        torch.cuda.synchronize(dev)
+        self.handles[0].barrier(channel=0) # every rank's buffers are zero
+
+    def forward(self, x, Wg, bias, W1_local, W2_local, out=None):
+        from . import _native as moe
+
+        self.epoch += 1
+        if out is None:
+            out = torch.empty(self.p.T, self.p.H, dtype=torch.bfloat16, device=x.device)
+        r = moe.ep_rank(self.p, self.world, self.rank, self.epoch, x, Wg, bias, W1_local,
+                        W2_local, out, self.ws, self.table)
+        moe.moe_ep_layer_forward([r])
+        return out

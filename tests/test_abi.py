@@ -268,3 +268,25 @@ def test_every_entry_point_has_a_python_function():
     for name in declared_functions():
         if name != "moe_status_string":
             assert callable(getattr(moe, name, None)), name
+
+
+def test_ep_layer_sizes_and_checks(lib):
+    """Host-only: the exchange buffer sizes of the expert-parallel layer, and the shapes it
+    refuses (no kernel launched)."""
+    p = moe.Problem.make(8192, 4096, 14336, 8, 2)
+    world = 2
+    sizes = moe.moe_ep_buffer_sizes(p, world)
+    recv_cap = world * 8192 * 2 + 4 * 127   # rows routed to E / world experts, each padded
+    assert sizes == [world * 1024 * 8 * 4, world * 4, recv_cap * 4096 * 2, recv_cap * 4,
+                     recv_cap * 8, (recv_cap // 128 + 1) * 4, 8192 * 2 * 4096 * 2, 8192 * 4]
+    assert moe.moe_ep_workspace_size(p, world) > 0
+    for bad_world in (0, 3, 9):            # must divide E = 8 and be at most 8
+        assert lib.moe_ep_workspace_size(ctypes.byref(p), bad_world) == 0
+    wide = moe.Problem.make(512, 256, 256, 64, 2)   # the one-launch router takes E <= 32
+    assert lib.moe_ep_workspace_size(ctypes.byref(wide), 2) == 0
+    assert lib.moe_ep_layer_forward(None, 1, None) == -1
+    r = moe.EpRank()
+    r.p = p
+    r.world, r.rank, r.epoch = world, 0, 0          # epoch must be positive
+    assert lib.moe_ep_layer_forward(ctypes.byref(r), 1, None) == -1
+    assert lib.moe_ep_layer_forward(ctypes.byref(r), 5, None) == -1  # more ranks than one launch takes

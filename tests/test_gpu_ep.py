@@ -128,3 +128,104 @@ def test_device_exchange_single_rank_equals_forward(T, E, k, zipf):
     assert st == (0, 0)
     for g in got:
         assert torch.equal(g.view(torch.int16), out.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------------------
+# the expert-parallel layer with the exchange overlapped with the GEMMs (one persistent launch
+# per rank; here every rank of the world in one launch on this GPU)
+# ---------------------------------------------------------------------------------------
+
+EP_LAYER_CASES = [
+    # name, world, T per rank, H, F, E, k, zipf, gate
+    ("w1_e8", 1, 600, 256, 256, 8, 2, 0.0, 0),
+    ("w2_e8", 2, 700, 256, 320, 8, 2, 0.8, 0),
+    ("w4_e8", 4, 500, 192, 256, 8, 2, 0.0, 0),
+    ("w2_e16_k4", 2, 300, 256, 256, 16, 4, 1.2, 0),
+    ("w4_e32_k4", 4, 257, 128, 192, 32, 4, 1.2, 0),
+    ("w2_e8_selbias", 2, 400, 256, 256, 8, 3, 1.5, 2),
+]
+
+
+def _ep_layer_inputs(world, T, H, F, E, k, zipf, gate, seed):
+    cfg = synth.LayerConfig("ep_layer", T=T * world, H=H, F=F, E=E, k=k, zipf_s=zipf, gate=gate)
+    inp = synth.make_inputs(cfg, seed=seed, device="cuda")
+    xs = [inp["x"][r * T:(r + 1) * T].contiguous() for r in range(world)]
+    el = E // world
+    W1s = [inp["W1"][r * el:(r + 1) * el].contiguous() for r in range(world)]
+    W2s = [inp["W2"][r * el:(r + 1) * el].contiguous() for r in range(world)]
+    return inp, xs, W1s, W2s
+
+
+@pytest.mark.parametrize("name,world,T,H,F,E,k,zipf,gate", EP_LAYER_CASES,
+                         ids=[c[0] for c in EP_LAYER_CASES])
+def test_ep_layer_ranks_equal_forward(name, world, T, H, F, E, k, zipf, gate):
+    """Every rank's output of the overlapped expert-parallel layer is bitwise moe_forward's
+    on the rank's tokens with all E experts; a second call on the same buffers (next epoch)
+    gives the same."""
+    inp, xs, W1s, W2s = _ep_layer_inputs(world, T, H, F, E, k, zipf, gate, seed=31)
+    p = moe.Problem.make(T, H, F, E, k, gate=gate)
+    bufs = [ep.ep_layer_buffers(p, world) for _ in range(world)]
+    wss = [torch.empty(moe.moe_ep_workspace_size(p, world), dtype=torch.uint8, device="cuda")
+           for _ in range(world)]
+    outs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+    ep.ep_layer_forward_local(p, xs, inp["Wg"], inp["bias"], W1s, W2s, outs, bufs, wss, epoch=1)
+    torch.cuda.synchronize()
+    for r in range(world):
+        assert moe.moe_get_device_status(wss[r]) == 0, r
+    cfg_r = synth.LayerConfig("rank", T=T, H=H, F=F, E=E, k=k, gate=gate)
+    for r in range(world):
+        ref = {"x": xs[r], "Wg": inp["Wg"], "bias": inp["bias"], "W1": inp["W1"], "W2": inp["W2"]}
+        _, out_ref, _, _ = _forward(cfg_r, ref)
+        assert torch.equal(outs[r], out_ref), (name, r)
+    first = [o.clone() for o in outs]
+    ep.ep_layer_forward_local(p, xs, inp["Wg"], inp["bias"], W1s, W2s, outs, bufs, wss, epoch=2)
+    torch.cuda.synchronize()
+    for r in range(world):
+        assert moe.moe_get_device_status(wss[r]) == 0
+        assert torch.equal(outs[r], first[r])
+
+
+def test_ep_layer_matches_oracle():
+    """Two ranks in one launch against the oracle on all their tokens."""
+    import oracle
+
+    world, T, H, F, E, k = 2, 300, 256, 192, 8, 2
+    inp, xs, W1s, W2s = _ep_layer_inputs(world, T, H, F, E, k, 0.0, 0, seed=32)
+    p = moe.Problem.make(T, H, F, E, k)
+    bufs = [ep.ep_layer_buffers(p, world) for _ in range(world)]
+    wss = [torch.empty(moe.moe_ep_workspace_size(p, world), dtype=torch.uint8, device="cuda")
+           for _ in range(world)]
+    outs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+    ep.ep_layer_forward_local(p, xs, inp["Wg"], None, W1s, W2s, outs, bufs, wss, epoch=1)
+    torch.cuda.synchronize()
+    got = torch.cat(outs).float().cpu().numpy().astype(np.float64)
+    ref, _, _ = oracle.moe_forward(synth.bf16_bits(inp["x"].cpu()), synth.bf16_bits(inp["Wg"].cpu()),
+                                   None, synth.bf16_bits(inp["W1"].cpu()),
+                                   synth.bf16_bits(inp["W2"].cpu()), k)
+    assert np.all(np.abs(got - ref) <= 2e-2 + 2e-2 * np.abs(ref))
+
+
+def test_ep_layer_timeout_when_a_rank_never_comes():
+    """The ranks' waits on one another are bounded: two ranks' buffers, but only rank 0 is
+    launched; its flag wait gives up, the status word says MOE_ERR_DEVICE_TIMEOUT, and the
+    context stays usable."""
+    world, T, H, F, E, k = 2, 256, 128, 128, 8, 2
+    inp, xs, W1s, W2s = _ep_layer_inputs(world, T, H, F, E, k, 0.0, 0, seed=33)
+    p = moe.Problem.make(T, H, F, E, k)
+    bufs = [ep.ep_layer_buffers(p, world) for _ in range(world)]
+    wss = [torch.empty(moe.moe_ep_workspace_size(p, world), dtype=torch.uint8, device="cuda")
+           for _ in range(world)]
+    outs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+    table = [[bufs[d][b] for d in range(world)] for b in range(len(moe.EP_BUFFERS))]
+    r0 = moe.ep_rank(p, world, 0, 1, xs[0], inp["Wg"], None, W1s[0], W2s[0], outs[0], wss[0], table)
+    prev = moe.moe_set_wait_timeout_ns(50_000_000)
+    try:
+        moe.moe_ep_layer_forward([r0])
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status(wss[0]) == -5
+    finally:
+        moe.moe_set_wait_timeout_ns(prev)
+    # the same context: a complete call (both ranks, next epoch) succeeds
+    ep.ep_layer_forward_local(p, xs, inp["Wg"], None, W1s, W2s, outs, bufs, wss, epoch=2)
+    torch.cuda.synchronize()
+    assert all(moe.moe_get_device_status(w) == 0 for w in wss)
