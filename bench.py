@@ -75,6 +75,11 @@ def parse_args():
                          "JSON line")
     ap.add_argument("--router-mode", choices=["auto", "sequential", "filter"], default="auto",
                     help="router variant (moe_set_router_mode)")
+    ap.add_argument("--ep-local", type=int, default=0, metavar="N",
+                    help="the expert-parallel layer (moe_ep_layer_forward) with the workload's "
+                         "tokens split over N ranks carried by one launch on this GPU (each rank "
+                         "1/N of the SMs, every exchange buffer local): the EP machinery's cost "
+                         "against the single-GPU layer, not NVLink")
     ap.add_argument("--router-only", action="store_true",
                     help="time moe_route alone (router logits + top-k); no expert weights allocated")
     return ap.parse_args()
@@ -158,12 +163,14 @@ def launches_in_mode(moe, p, mode):
         moe.moe_set_gemm_mode(prev)
 
 
-def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, kernel, fused=False):
+def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, kernel, fused=False,
+                    whole=False):
     """Roofline of the dominant kernel. Separate launches: the layer0 grouped GEMM, with its
     useful FLOPs (padding rows not counted) and algorithmic bytes (each active expert's W1
     once, x once, h of the routed rows written once). One persistent launch (`fused`):
     layer0 + layer1 + combine, with both GEMMs' useful FLOPs and the bytes that must cross
-    HBM (the active experts' W1 and W2, the sorted x rows, the output). The bound is
+    HBM (the active experts' W1 and W2, the sorted x rows, the output); the whole layer in
+    that launch (`whole`) adds the router's FLOPs and its reads of x and W_g. The bound is
     whichever takes longer at the measured peaks."""
     w1_cols = 2 * cfg.F if cfg.act == 0 else cfg.F
     wb = 1 if fp8 else 2   # e4m3 experts: 1-byte weights and x codes; h is still bf16
@@ -171,6 +178,9 @@ def layer0_roofline(cfg, g0_ms, active_experts, peaks, peak_src, clocks, fp8, ke
         flops = 2 * cfg.T * cfg.k * cfg.H * (w1_cols + cfg.F)
         nbytes = (wb * (active_experts * cfg.H * (w1_cols + cfg.F) + cfg.T * cfg.k * cfg.H) +
                   2 * cfg.T * cfg.H)
+        if whole:
+            flops += 2 * cfg.T * cfg.H * cfg.E
+            nbytes += 2 * cfg.T * cfg.H + 2 * cfg.H * cfg.E
     else:
         flops = 2 * cfg.T * cfg.k * cfg.H * w1_cols
         nbytes = wb * (active_experts * cfg.H * w1_cols + cfg.T * cfg.H) + 2 * cfg.T * cfg.k * cfg.F
@@ -637,7 +647,13 @@ def run_ours(args):
     # mark its end)
     fused = (not args.fp8 and
              moe.moe_forward_launches(p) < launches_in_mode(moe, p, moe.GEMM_SINGLE_CTA))
-    if fused:
+    # the whole layer in one launch: that kernel is the step (the timed region holds it and one
+    # 32-byte memset per step), so its duration is the step's
+    whole = not args.fp8 and moe.moe_forward_launches(p) == 1
+    if whole:
+        kernel = f"moe_fused_layer_kernel<{cfg.act if cfg.act == 0 else 1}, true>"
+        g_ms = ms_per_step
+    elif fused:
         kernel = "moe_fused_layer_kernel<0>" if cfg.act == 0 else "moe_fused_layer_kernel<1>"
         g_ms = sum(stage_ms[k] for k in ("layer0_gemm_swiglu", "layer1_gemm_scale", "combine"))
     else:
@@ -645,7 +661,7 @@ def run_ours(args):
                   else DOMINANT_KERNEL[args.gemm_mode])
         g_ms = stage_ms["layer0_gemm_swiglu"]
     roofline = layer0_roofline(cfg, g_ms, active_experts, peaks, peak_src, clocks, args.fp8, kernel,
-                               fused)
+                               fused or whole, whole)
     layer_roof = {"bound": "tensor", "achieved": layer_tflops, "unit": "TFLOP/s per GPU"}
     layer_roof.update(tensor_fracs(layer_tflops, peaks, clocks, args.fp8))
     layer_roof["peak_source"] = f"{peak_src} bf16 {layer_roof['regime']}" + (" x 2" if args.fp8 else "")
@@ -768,6 +784,64 @@ def run_router(args):
     return 0
 
 
+def run_ep_local(args):
+    """The expert-parallel layer for N ranks in one launch on one GPU: rank r routes tokens
+    [r T/N, (r+1) T/N) of the workload and holds experts [r E/N, (r+1) E/N); K timed calls
+    (the same total work as the single-GPU layer; its exchange stores stay on this GPU)."""
+    import torch
+
+    import mixture_experts_layer_forward_b200 as moe
+    from mixture_experts_layer_forward_b200 import ep, synth
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = workload(args)
+    N = args.ep_local
+    K, W = args.steps, max(3, args.warmup)
+    if cfg.T % N or cfg.E % N:
+        raise SystemExit(f"--ep-local {N} must divide T = {cfg.T} and E = {cfg.E}")
+    inp = synth.make_inputs(cfg, seed=args.seed, device=dev)
+    T, el = cfg.T // N, cfg.E // N
+    xs = [inp["x"][r * T:(r + 1) * T].contiguous() for r in range(N)]
+    W1s = [inp["W1"][r * el:(r + 1) * el].contiguous() for r in range(N)]
+    W2s = [inp["W2"][r * el:(r + 1) * el].contiguous() for r in range(N)]
+    p = moe.Problem.make(T, cfg.H, cfg.F, cfg.E, cfg.k, cfg.act, cfg.gate)
+    bufs = [ep.ep_layer_buffers(p, N, dev) for _ in range(N)]
+    wss = [torch.empty(moe.moe_ep_workspace_size(p, N), dtype=torch.uint8, device=dev)
+           for _ in range(N)]
+    outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(N)]
+    epoch = [0]
+
+    def call():
+        epoch[0] += 1
+        ep.ep_layer_forward_local(p, xs, inp["Wg"], inp["bias"], W1s, W2s, outs, bufs, wss,
+                                  epoch[0])
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize(dev)
+    sampler = new_sampler(torch, dev, not args.no_clocks)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    start.record()
+    for _ in range(K):
+        call()
+    end.record()
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1) if sampler else None
+    for w in wss:
+        assert moe.moe_get_device_status(w) == 0
+    ms = start.elapsed_time(end) / K
+    cfgd = config_dict(cfg, args, 1)
+    cfgd["parallelism"] = f"ep{N} emulated: {N} ranks in one launch on one GPU"
+    emit({"metric": "MoE-layer forward tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
+          "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+          "dtype": "bf16", "data": "synthetic", "config": cfgd, "impl": "ep_local",
+          "gpu_launches": K, "clocks": clocks})
+    return 0
+
+
 def run_backward(args):
     """The layer's backward on one GPU: K timed moe_backward calls (each recomputes the
     routing, the dispatch and z = x W1) on a seeded dL/dout."""
@@ -837,6 +911,8 @@ def main():
         return run_reference(args)
     if args.router_only:
         return run_router(args)
+    if args.ep_local:
+        return run_ep_local(args)
     if args.backward:
         return run_backward(args)
     return run_ours(args)

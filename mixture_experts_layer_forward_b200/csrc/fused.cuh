@@ -105,7 +105,9 @@ struct FusedArgs {
     EpArgs ep;              // expert-parallel launch (world > 0)
 };
 
-enum : int { TRACE_L0 = 0, TRACE_L1 = 1, TRACE_COMBINE = 2 };
+// TRACE_FRONT: a CTA's routing and dispatch (launch start to the GEMM phases); TRACE_SCATTER:
+// a CTA's row sends of the expert-parallel launch (item = the CTA)
+enum : int { TRACE_L0 = 0, TRACE_L1 = 1, TRACE_COMBINE = 2, TRACE_FRONT = 3, TRACE_SCATTER = 4 };
 
 __device__ __forceinline__ int ld_acquire_gpu(const int *p)
 {
@@ -140,6 +142,13 @@ __device__ __forceinline__ void red_release_sys_add(int *p, int v)
 __device__ __forceinline__ void st_release_sys(int *p, int v)
 {
     asm volatile("st.release.sys.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// relaxed add at system scope: the release comes from a system-scope fence issued before
+// it by the same thread (fence + strong write is a release pattern)
+__device__ __forceinline__ void red_relaxed_sys_add(int *p, int v)
+{
+    asm volatile("red.relaxed.sys.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_global()
@@ -413,38 +422,63 @@ __device__ __forceinline__ bool ep_front(const CUtensorMap *tmRX, const CUtensor
     return grid_barrier(f.gbar, 2 * ncta, abort_flag, tmo, status, 362);
 }
 
-// The data-movement warps' scatter of the expert-parallel launch (after ep_front; four
-// warps, `dw` 0..3): each of this CTA's pairs sends its token's x row, gate and origin to
-// its destination row, then counts the row on the destination's M tile (after a
-// system-scope fence, so the destination's layer0 may read the row once the count is up).
-__device__ __forceinline__ void ep_scatter(const FusedArgs &fa, int cta, int ncta, int dw, int lane)
+// The scatter of the expert-parallel launch (after ep_front), by the CTA's eight epilogue and
+// data-movement warps (`dw` 0..7, meeting at named barrier `bar`; no layer0 tile can start
+// before the rows arrive, so the epilogue warps are free): every pair of this CTA's groups
+// sends its token's x row, gate and origin to its destination row; after all of them (the
+// barrier), warp 0 of the eight fences at system scope once -- the barrier puts every lane's
+// stores before that fence -- and adds each pair to its destination tile's arrival count, so
+// the destination's layer0 may read a tile once its count is complete.
+__device__ __forceinline__ void ep_scatter(const FusedArgs &fa, int cta, int ncta, int dw, int lane,
+                                           int bar)
 {
+    constexpr int NW = 8;
     const EpArgs &ep = fa.ep;
     const FrontArgs &f = fa.front;
     const int k = f.ra.k, H = f.fd.H, G = f.n_groups;
     const int chunks = H / 8;
+    auto valid = [&](size_t q, int &d, int &slot) {
+        d = ep.dest[q];
+        slot = ep.slot[q];
+        return d >= 0 && d < ep.world && slot >= 0 && (int64_t)slot < ep.recv_cap;
+    };
     for (int g = cta; g < G; g += ncta) {
         const int t0 = g * f.ra.tt;
         const int P = min(f.ra.tt, f.ra.T - t0) * k;
         const size_t q0 = (size_t)t0 * k;
-        for (int qq = dw; qq < P; qq += 4) {
+        for (int qq = dw; qq < P; qq += NW) {
             const size_t q = q0 + qq;
-            const int d = ep.dest[q];
-            if (d < 0 || d >= ep.world) continue;
-            const int slot = ep.slot[q];
-            if (slot < 0 || (int64_t)slot >= ep.recv_cap) continue;
+            int d, slot;
+            if (!valid(q, d, slot)) continue;
             const int t = (int)(q / k);
             const uint4 *src = reinterpret_cast<const uint4 *>(f.fd.x + (size_t)t * H);
             uint4 *dst = reinterpret_cast<uint4 *>(ep.recv_rows[d] + (size_t)slot * H);
-#pragma unroll 4
-            for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+            // a lane's 16-byte pieces of the row, 16 loads in flight before the stores
+            int c = lane;
+            for (; c + 15 * 32 < chunks; c += 16 * 32) {
+                uint4 v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = src[c + i * 32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[c + i * 32] = v[i];
+            }
+            for (; c < chunks; c += 32) dst[c] = src[c];
             if (lane == 0) {
                 ep.recv_gate[d][slot] = f.ra.topk_w[q];
                 ep.recv_origin[d][slot] = ((long long)ep.rank << 32) | (long long)q;
             }
-            __threadfence_system();
-            __syncwarp();
-            if (lane == 0) red_release_sys_add(ep.arrive[d] + (slot >> 7), 1);
+        }
+    }
+    named_bar_sync(bar, NW * 32);
+    if (dw != 0) return;
+    __threadfence_system();
+    for (int g = cta; g < G; g += ncta) {
+        const int t0 = g * f.ra.tt;
+        const int P = min(f.ra.tt, f.ra.T - t0) * k;
+        const size_t q0 = (size_t)t0 * k;
+        for (int qq = lane; qq < P; qq += 32) {
+            int d, slot;
+            if (valid(q0 + qq, d, slot)) red_relaxed_sys_add(ep.arrive[d] + (slot >> 7), 1);
         }
     }
 }
@@ -693,10 +727,13 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
     const uint32_t tmem_base = *tmem_slot;
 
     bool front_ok = true;
+    const uint64_t t_launch = globaltimer_ns();
     if constexpr (MODE == FUSED_WHOLE)
         front_ok = fused_front(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo, cta, ncta);
     if constexpr (MODE == FUSED_EP)
         front_ok = ep_front(&tmRX, &tmRW, fa, smem, abort_flag, status, tmo, cta, ncta);
+    if (MODE != FUSED_LAYERS && front_ok && threadIdx.x == 0)
+        trace_record(fa, TRACE_FRONT, cta, t_launch, globaltimer_ns());
 
     const int num_tiles = front_ok ? l0.meta->num_tiles : 0;
     const int total0 = num_tiles * l0.n_tiles;
@@ -831,6 +868,12 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
     } else {
         // ---------------- epilogue warps 2..5 and data-movement warps 6..9 ----------------
         const bool dm = warp >= 6;
+        if (MODE == FUSED_EP && front_ok) {
+            // expert parallelism: all eight send this rank's rows out first (named barrier 4)
+            const uint64_t t_sc = globaltimer_ns();
+            ep_scatter(fa, cta, ncta, warp - 2, lane, 4);
+            if (warp == 2 && lane == 0) trace_record(fa, TRACE_SCATTER, cta, t_sc, globaltimer_ns());
+        }
         const int q = warp & 3; // TMEM lanes 32q .. 32q+31
         int n = 0;
         bool ok = true;
@@ -895,15 +938,6 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
                 epilogue_rows<KIND0>(l0, t_row, row, it.nt, 0, 0, nullptr, c_lo, c_hi);
             } else {
                 epilogue_rows<GEMM_SCALE>(l1, t_row, row, it.nt);
-                if (MODE == FUSED_EP) {
-                    // the row's stripe went to its origin: count it there once it is visible
-                    const long long o = l1.row_dst[row];
-                    if (o >= 0) {
-                        __threadfence_system();
-                        const int q = (int)(o & 0xffffffffll);
-                        red_release_sys_add(fa.ep.back_cnt[(int)(o >> 32)] + q / fa.k, 1);
-                    }
-                }
             }
             // The accumulator is free as soon as its TMEM reads are done (layer1 items with
             // eight epilogue parts configured: warps 2..5 stand for 6..9).
@@ -911,6 +945,16 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
             __syncwarp();
             if (lane == 0)
                 mbar_arrive_cnt(tempty_bar(acc), (it.phase == 1 && split0) ? 2u : 1u);
+            if (MODE == FUSED_EP && it.phase == 1) {
+                // the row's stripe went to its origin: count it there once it is visible
+                // (after the accumulator is released, so the MMA warp does not wait for it)
+                const long long o = l1.row_dst[row];
+                if (o >= 0) {
+                    __threadfence_system();
+                    const int q = (int)(o & 0xffffffffll);
+                    red_relaxed_sys_add(fa.ep.back_cnt[(int)(o >> 32)] + q / fa.k, 1);
+                }
+            }
             // Ready signal: every part makes its stores visible, then the last of the item's
             // parts publishes it. The part counters form a ring of 4 indexed by the CTA's item
             // count: slot n & 3 is reused by item n + 4, whose parts can only arrive after
@@ -939,7 +983,7 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
         }
         if (dm && !a_tma) cp_async_wait_all(); // this thread's copies land first
         // expert parallelism: the data-movement warps send this rank's rows out first
-        if (MODE == FUSED_EP && dm && front_ok) ep_scatter(fa, cta, ncta, warp - 6, lane);
+
         // combine: the data-movement warps from the end of their layer0 duties (beside the
         // layer1 GEMM pipeline), the epilogue warps once this CTA's GEMM items are done
         // (each group of four warps decides together whether to go on: named barrier 2 for

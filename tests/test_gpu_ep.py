@@ -229,3 +229,29 @@ def test_ep_layer_timeout_when_a_rank_never_comes():
     ep.ep_layer_forward_local(p, xs, inp["Wg"], None, W1s, W2s, outs, bufs, wss, epoch=2)
     torch.cuda.synchronize()
     assert all(moe.moe_get_device_status(w) == 0 for w in wss)
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ep_layer_full_size_mixtral(world):
+    """The Mixtral-shaped layer (8192 tokens, H 4096, F 14336, 8 experts, top-2) split over
+    `world` ranks in one launch: every rank's output is bitwise moe_forward's on its tokens."""
+    cfg = synth.CONFIGS["mixtral"]
+    inp = synth.make_inputs(cfg, seed=34, device="cuda")
+    T, el = cfg.T // world, cfg.E // world
+    xs = [inp["x"][r * T:(r + 1) * T].contiguous() for r in range(world)]
+    W1s = [inp["W1"][r * el:(r + 1) * el].contiguous() for r in range(world)]
+    W2s = [inp["W2"][r * el:(r + 1) * el].contiguous() for r in range(world)]
+    p = moe.Problem.make(T, cfg.H, cfg.F, cfg.E, cfg.k)
+    bufs = [ep.ep_layer_buffers(p, world) for _ in range(world)]
+    wss = [torch.empty(moe.moe_ep_workspace_size(p, world), dtype=torch.uint8, device="cuda")
+           for _ in range(world)]
+    outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+    ep.ep_layer_forward_local(p, xs, inp["Wg"], inp["bias"], W1s, W2s, outs, bufs, wss, epoch=1)
+    torch.cuda.synchronize()
+    del bufs, W1s, W2s
+    cfg_r = synth.LayerConfig("rank", T=T, H=cfg.H, F=cfg.F, E=cfg.E, k=cfg.k)
+    for r in range(world):
+        assert moe.moe_get_device_status(wss[r]) == 0
+        ref = {"x": xs[r], "Wg": inp["Wg"], "bias": inp["bias"], "W1": inp["W1"], "W2": inp["W2"]}
+        _, out_ref, _, _ = _forward(cfg_r, ref)
+        assert torch.equal(outs[r], out_ref), r
