@@ -232,7 +232,7 @@ def schedule_trace(torch, moe, fwd, dev, out_file, cap=1 << 18):
     t0 = r[:, 2] - r[:, 2].min()
     t1 = r[:, 3] - r[:, 2].min()
     summ = {"records": n, "span_us": float(t1.max()) / 1e3}
-    names = {0: "layer0", 1: "layer1", 2: "combine"}
+    names = {0: "layer0", 1: "layer1", 2: "combine", 3: "front", 4: "scatter"}
     for k, nm in names.items():
         m = kind == k
         if m.any():

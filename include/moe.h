@@ -371,9 +371,9 @@ MOE_API moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y,
  *      waits only until its rows have arrived; a layer1 tile waits for its layer0 rows (the
  *      tile-level counters of the persistent launch) and its epilogue stores each gated row
  *      straight into row t * k + j of the origin's return buffer and adds 1 to the origin's
- *      count of that token;
+ *      count of that token and 256-column stripe;
  *   4. the combine sums the k returned rows of each of r's tokens (j ascending, fp32, one
- *      bf16 rounding) as soon as all of the token's row stripes are back.
+ *      bf16 rounding), a 256-column stripe as soon as that stripe of the k rows is back.
  * Stores to other GPUs are plain 16-byte stores followed by a system-scope fence before the
  * count; nothing loads another GPU's memory, no TMA reads another GPU's memory, and every
  * wait is bounded (MOE_ERR_DEVICE_TIMEOUT in the status word of the rank's workspace). Every

@@ -472,8 +472,17 @@ __device__ __forceinline__ void dispatch_front(const FrontDispatch &d, int g_fir
             }
             const uint4 *src = reinterpret_cast<const uint4 *>(d.x + (size_t)t * d.H);
             uint4 *dst = reinterpret_cast<uint4 *>(d.x_perm + (size_t)r * d.H);
-#pragma unroll 4
-            for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+            // a lane's 16-byte pieces of the row, 16 loads in flight before the stores (ten
+            // warps per SM copy: memory parallelism has to come from each lane)
+            int c = lane;
+            for (; c + 15 * 32 < chunks; c += 16 * 32) {
+                uint4 v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = src[c + i * 32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[c + i * 32] = v[i];
+            }
+            for (; c < chunks; c += 32) dst[c] = src[c];
         }
         __syncthreads(); // the bitmaps are reused by the next group
     }

@@ -70,7 +70,7 @@ struct EpArgs {
     long long *recv_origin[EP_MAX_WORLD];     // [recv_cap] (source rank << 32) | (t * k + j); -1 pads
     int *arrive[EP_MAX_WORLD];                // [max_tiles] rows arrived per local M tile
     __nv_bfloat16 *back[EP_MAX_WORLD];        // [T * k][H] gated rows returned to their origin
-    int *back_cnt[EP_MAX_WORLD];              // [T] row stripes returned per token
+    int *back_cnt[EP_MAX_WORLD];              // [T][H / 256] rows returned per token and stripe
     int64_t recv_cap;
     int max_tiles;
     int32_t *slot;                            // [T * k] this rank's pairs: destination row
@@ -403,9 +403,12 @@ __device__ __forceinline__ bool ep_front(const CUtensorMap *tmRX, const CUtensor
             const int d = i / E, e = i - d * E;
             ep.all_counts[d][((size_t)ep.rank * G + g) * E + e] = f.ra.group_counts[(size_t)g * E + e];
         }
-    if (cta == 0) {
+    if (cta == 0)
         for (int i = threadIdx.x; i < ep.max_tiles; i += blockDim.x) ep.arrive[ep.rank][i] = 0;
-        for (int i = threadIdx.x; i < fa.T; i += blockDim.x) ep.back_cnt[ep.rank][i] = 0;
+    {
+        const int64_t n = (int64_t)fa.T * fa.l1.n_tiles;
+        for (int64_t i = (int64_t)cta * blockDim.x + threadIdx.x; i < n; i += (int64_t)ncta * blockDim.x)
+            ep.back_cnt[ep.rank][i] = 0;
     }
     if (!grid_barrier(f.gbar, ncta, abort_flag, tmo, status, 360, true)) return false;
     // every rank: its counts are everywhere and its receive counters are clear
@@ -506,20 +509,21 @@ __device__ __forceinline__ FusedItem fused_item(int w, const FusedArgs &fa, int 
 // so one round of loads covers all 8 k flags. The rows are the same for every lane; the warp
 // barrier after the vote orders every lane's later loads after the lanes' acquires.
 __device__ __forceinline__ bool combine_rows_ready(const FusedArgs &fa, const int *flags, const int (&t)[8],
-                                                   int lane, volatile int *abort_flag, int *status)
+                                                   int stripe, int lane, volatile int *abort_flag,
+                                                   int *status)
 {
     const uint64_t t_start = globaltimer_ns();
     uint32_t nap = 64;
     const bool ep = fa.ep.world > 0;
-    // expert parallelism: every stripe of the token's k rows has come back
-    const int ep_need = fa.k * fa.l1.n_tiles;
 #pragma unroll 1
     while (true) {
         bool ready = true;
         if (ep) {
+            // expert parallelism: this stripe of the token's k rows has come back
             if (lane < 8) {
                 const int tok = t[0] + lane * 4;
-                if (tok < fa.T && ld_acquire_sys(fa.ep.back_cnt[fa.ep.rank] + tok) < ep_need)
+                if (tok < fa.T &&
+                    ld_acquire_sys(fa.ep.back_cnt[fa.ep.rank] + (size_t)tok * fa.l1.n_tiles + stripe) < fa.k)
                     ready = false;
             }
         } else {
@@ -570,7 +574,7 @@ __device__ __forceinline__ bool fused_combine(const FusedArgs &fa, int stripe, i
             for (int c = 0; c < 8; ++c) a[i][c] = 0.0f;
         }
         if (t[0] >= fa.T) break; // the block's remaining groups are past the batch
-        if (!combine_rows_ready(fa, flags, t, lane, abort_flag, status)) return false;
+        if (!combine_rows_ready(fa, flags, t, stripe, lane, abort_flag, status)) return false;
         for (int j0 = 0; j0 < fa.k; j0 += 2) {
             uint4 u[2][8];
 #pragma unroll
@@ -952,7 +956,7 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
                 if (o >= 0) {
                     __threadfence_system();
                     const int q = (int)(o & 0xffffffffll);
-                    red_relaxed_sys_add(fa.ep.back_cnt[(int)(o >> 32)] + q / fa.k, 1);
+                    red_relaxed_sys_add(fa.ep.back_cnt[(int)(o >> 32)] + (size_t)(q / fa.k) * l1.n_tiles + it.nt, 1);
                 }
             }
             // Ready signal: every part makes its stores visible, then the last of the item's

@@ -2353,7 +2353,7 @@ moe_status moe_ep_buffer_sizes(const moe_problem *p, int32_t world, int64_t *siz
     sizes[4] = X.recv_cap * 8;                         // recv_origin
     sizes[5] = (int64_t)X.L.max_tiles * 4;             // arrive
     sizes[6] = T * k * H * 2;                          // back
-    sizes[7] = T * 4;                                  // back_cnt
+    sizes[7] = T * ((H + gemm::BN - 1) / gemm::BN) * 4; // back_cnt [T][stripes]
     return MOE_OK;
 }
 

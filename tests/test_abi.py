@@ -278,7 +278,7 @@ def test_ep_layer_sizes_and_checks(lib):
     sizes = moe.moe_ep_buffer_sizes(p, world)
     recv_cap = world * 8192 * 2 + 4 * 127   # rows routed to E / world experts, each padded
     assert sizes == [world * 1024 * 8 * 4, world * 4, recv_cap * 4096 * 2, recv_cap * 4,
-                     recv_cap * 8, (recv_cap // 128 + 1) * 4, 8192 * 2 * 4096 * 2, 8192 * 4]
+                     recv_cap * 8, (recv_cap // 128 + 1) * 4, 8192 * 2 * 4096 * 2, 8192 * 16 * 4]
     assert moe.moe_ep_workspace_size(p, world) > 0
     for bad_world in (0, 3, 9):            # must divide E = 8 and be at most 8
         assert lib.moe_ep_workspace_size(ctypes.byref(p), bad_world) == 0
