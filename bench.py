@@ -835,10 +835,14 @@ def run_ep_local(args):
     ms = start.elapsed_time(end) / K
     cfgd = config_dict(cfg, args, 1)
     cfgd["parallelism"] = f"ep{N} emulated: {N} ranks in one launch on one GPU"
-    emit({"metric": "MoE-layer forward tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
-          "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
-          "dtype": "bf16", "data": "synthetic", "config": cfgd, "impl": "ep_local",
-          "gpu_launches": K, "clocks": clocks})
+    line = {"metric": "MoE-layer forward tokens/s", "value": cfg.T / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic", "config": cfgd, "impl": "ep_local",
+            "gpu_launches": K, "clocks": clocks}
+    if args.trace is not None:
+        # rank 0's CTAs record their work items (front, scatter, GEMM tiles, combine items)
+        line["schedule_trace"] = schedule_trace(torch, moe, call, dev, args.trace or None)
+    emit(line)
     return 0
 
 
