@@ -1,5 +1,15 @@
 // fused.cuh -- one persistent launch for layer0, layer1 and the combine, scheduled by
-// tile-level ready flags.
+// tile-level ready flags; optionally with the routing and dispatch in front of them (the
+// whole layer in one launch), or as one rank of the expert-parallel layer (rows exchanged
+// with the other ranks inside the launch). The body is fused_layer_body<KIND0, MODE>:
+//   FUSED_LAYERS  layer0 -> layer1 -> combine (route and dispatch ran before the launch);
+//   FUSED_WHOLE   fused_front (routing of the CTA's token groups, grid barrier, in-launch
+//                 dispatch and row copy, grid barrier), then the same GEMM phases;
+//   FUSED_EP      ep_front (routing, counts to every rank, a flag barrier of all ranks,
+//                 destinations), ep_scatter by the eight non-GEMM-issuing warps while layer0
+//                 tiles wait for their rows' arrival counts, layer1 rows stored back into
+//                 their origins' buffers with per-(token, stripe) counts, and the combine of
+//                 the rows that came back.
 //
 // Where it comes from (Comet: Fine-grained Computation-communication Overlapping for
 // Mixture-of-Experts; and "Fine-grained Computation-Communication Overlap via Tile-level
