@@ -509,6 +509,10 @@ MOE_API int64_t moe_set_wait_timeout_ns(int64_t ns);
  * more experts the separate launches measured faster. Otherwise the separate launches. Stage events 3..5 of moe_forward_staged then all mark the end of that one
  * launch. */
 #define MOE_GEMM_FUSED 3
+/* MOE_GEMM_FUSED_LAYERS: layer0 and layer1 in the persistent launch (layer1 tiles start as
+ * their M tile's h rows are done, no launch boundary between the layers), the combine as
+ * its own launch after it (full occupancy); stage event 5 then marks the combine's end. */
+#define MOE_GEMM_FUSED_LAYERS 4
 MOE_API int moe_set_gemm_mode(int mode);
 
 /* Whole-layer launch (Comet §5.3: the small-batch gains come from taking the host-driven

@@ -486,7 +486,7 @@ def moe_set_wait_timeout_ns(ns: int) -> int:
     return int(library().moe_set_wait_timeout_ns(int(ns)))
 
 
-GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED = 0, 1, 2, 3
+GEMM_AUTO, GEMM_SINGLE_CTA, GEMM_CTA_PAIR, GEMM_FUSED, GEMM_FUSED_LAYERS = 0, 1, 2, 3, 4
 ROUTER_AUTO, ROUTER_SEQUENTIAL, ROUTER_FILTER = 0, 1, 2
 ORDER_EXPERT, ORDER_MIXED, ORDER_NARROW, ORDER_PHASED = 0, 1, 2, 3
 

@@ -106,6 +106,7 @@ struct FusedArgs {
     const __nv_bfloat16 *ys_shared; // [T, H] shared-expert rows added last, or nullptr
     int a_tma;              // 1: layer0 A rows by TMA (expert-sorted copy of x)
     int comb_tokens;        // tokens per combine item, a multiple of 32
+    int comb_in_launch;     // 0: no combine in this launch (it runs as its own launch after)
     int fault_skip;         // test hook: layer0 item whose ready signal is withheld (-1: none)
     // optional schedule trace: records of 4 x uint64 {kind << 32 | item, smid, t_begin_ns,
     // t_end_ns}; trace[0] is the record counter, records start at trace[4]; nullptr: off
@@ -1004,7 +1005,7 @@ __device__ __forceinline__ void fused_layer_body(const CUtensorMap &tmA0, const 
         // the data-movement warps, 3 for the epilogue warps)
         volatile int *slots = reinterpret_cast<volatile int *>(warps_done + 4);
         const int bar = dm ? 2 : 3;
-        if (named_bar_and(bar, 128, ok && front_ok))
+        if (named_bar_and(bar, 128, ok && front_ok) && fa.comb_in_launch)
             combine_queue(fa, dm ? warp - 6 : warp - 2, lane, bar, slots + (dm ? 0 : 1), abort_flag,
                           status);
     }

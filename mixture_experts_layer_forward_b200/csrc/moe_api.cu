@@ -974,7 +974,14 @@ FusedPlan fused_plan(const moe_problem *p)
 bool run_fused(const moe_problem *p)
 {
     const int mode = g_gemm_mode.load();
-    return mode == MOE_GEMM_FUSED || (mode == MOE_GEMM_AUTO && fused_plan(p).fused);
+    return mode == MOE_GEMM_FUSED || mode == MOE_GEMM_FUSED_LAYERS ||
+           (mode == MOE_GEMM_AUTO && fused_plan(p).fused);
+}
+
+// The persistent launch runs the combine too (else the combine is its own launch after it).
+bool fused_combine_in_launch()
+{
+    return g_gemm_mode.load() != MOE_GEMM_FUSED_LAYERS;
 }
 
 // The persistent launch also routes and dispatches (a computed routing, no stage events and
@@ -982,7 +989,8 @@ bool run_fused(const moe_problem *p)
 bool whole_layer(const moe_problem *p)
 {
     return g_front.load() != 0 && g_gemm_mode.load() != MOE_GEMM_CTA_PAIR && run_fused(p) &&
-           use_x_perm(p) && route_uses_chain(p) && !route_uses_filter(p) && front_plan(p).ok;
+           fused_combine_in_launch() && use_x_perm(p) && route_uses_chain(p) &&
+           !route_uses_filter(p) && front_plan(p).ok;
 }
 
 moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 *Wg,
@@ -1132,6 +1140,7 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
         fa.ys_shared = reinterpret_cast<const __nv_bfloat16 *>(ys_s);
         fa.a_tma = xperm ? 1 : 0;
         fa.comb_tokens = plan.comb_tokens;
+        fa.comb_in_launch = fused_combine_in_launch() ? 1 : 0;
         fa.fault_skip = g_fault_skip.load();
         fa.trace = g_trace.load();
         fa.trace_cap = g_trace_cap.load();
@@ -1179,8 +1188,16 @@ moe_status forward_impl(const moe_problem *p, const moe_bf16 *x, const moe_bf16 
                 e = gated ? launch_fused<GEMM_SWIGLU, false>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st)
                           : launch_fused<GEMM_ACT, false>(m_x, m_w1, m_h, m_w2, m_rx, m_rw, fa, max_work, st);
         }
-        // the three stages share one launch: their boundaries coincide at its end
-        for (int i = 3; i < 6 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+        if (fa.comb_in_launch) {
+            // the three stages share one launch: their boundaries coincide at its end
+            for (int i = 3; i < 6 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+            return to_status(e);
+        }
+        // layer0 and layer1 share the launch; the combine follows as its own launch
+        for (int i = 3; i < 5 && e == cudaSuccess; ++i) e = record(events, n_events, i, st);
+        if (e == cudaSuccess)
+            e = launch_combine(p, ys, L.pmax, d.inv_pos, out, status, 0, st, ys_s, n_rows);
+        if (e == cudaSuccess) e = record(events, n_events, 5, st);
         return to_status(e);
     }
 
@@ -1761,6 +1778,7 @@ moe_status ep_layer_impl(const moe_ep_rank *ranks, int n_local, cudaStream_t st)
         fa.ys_rows = (int64_t)p->T * p->top_k;
         fa.a_tma = 1;
         fa.comb_tokens = fused_plan(p).comb_tokens;
+        fa.comb_in_launch = 1; // the combine of the returned rows is part of the EP launch
         fa.fault_skip = -1;
         fa.trace = i == 0 ? g_trace.load() : nullptr;
         fa.trace_cap = g_trace_cap.load();
@@ -1832,7 +1850,7 @@ int moe_forward_launches(const moe_problem *p)
     // + the x_perm gather (CTA pairs, large batches); then layer0, layer1, combine, or the one
     // persistent launch
     const int gather = (pair || use_x_perm(p)) ? 1 : 0;
-    const int layers = (!pair && run_fused(p)) ? 1 : 3;
+    const int layers = (!pair && run_fused(p)) ? (fused_combine_in_launch() ? 1 : 2) : 3;
     return whole_layer(p) ? 1 : route + dispatch + gather + layers;
 }
 
@@ -2146,7 +2164,7 @@ int64_t moe_set_wait_timeout_ns(int64_t ns)
 int moe_set_gemm_mode(int mode)
 {
     if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_SINGLE_CTA && mode != MOE_GEMM_CTA_PAIR &&
-        mode != MOE_GEMM_FUSED)
+        mode != MOE_GEMM_FUSED && mode != MOE_GEMM_FUSED_LAYERS)
         return -1;
     return g_gemm_mode.exchange(mode);
 }

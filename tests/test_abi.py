@@ -138,6 +138,10 @@ def test_forward_launch_count_follows_the_modes(lib):
         assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_gemm_mode(moe.GEMM_FUSED)           # forced: the persistent launch
         assert moe.moe_forward_launches(qwen2) == 7
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED_LAYERS)    # layers in it, the combine after
+        assert moe.moe_forward_launches(qwen2) == 8
+        assert moe.moe_forward_launches(mixtral) == 7   # no whole-layer launch then
+        moe.moe_set_gemm_mode(moe.GEMM_FUSED)
         moe.moe_set_gemm_mode(moe.GEMM_SINGLE_CTA)      # three layer launches
         assert moe.moe_forward_launches(qwen2) == 9
         moe.moe_set_work_order(moe.ORDER_NARROW)        # the same launches, SMs split inside

@@ -363,8 +363,9 @@ FWD_CASES = [
 ]
 
 
-@pytest.fixture(params=[moe.GEMM_CTA_PAIR, moe.GEMM_SINGLE_CTA, moe.GEMM_FUSED],
-                ids=["cta_pair", "single_cta", "fused"])
+@pytest.fixture(params=[moe.GEMM_CTA_PAIR, moe.GEMM_SINGLE_CTA, moe.GEMM_FUSED,
+                        moe.GEMM_FUSED_LAYERS],
+                ids=["cta_pair", "single_cta", "fused", "fused_layers"])
 def gemm_mode(request):
     prev = moe.moe_set_gemm_mode(request.param)
     yield request.param
