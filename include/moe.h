@@ -386,7 +386,11 @@ MOE_API moe_status moe_ep_return(int32_t H, int32_t world, const moe_bf16 *y,
  * n_local: ranks this launch carries -- 1 on a GPU per rank; up to MOE_EP_MAX_LOCAL to run
  * several ranks on one GPU (all their buffers on this GPU; each rank gets 1/n_local of the
  * SMs), which is how the ranks' interplay is tested with one GPU. All ranks of a layer call
- * must launch (their waits on one another are bounded, not avoided). */
+ * must launch (their waits on one another are bounded, not avoided), with the same problem
+ * (T, H, F, E, top_k, act, gate), the same n_local and the same number of SMs: the layout
+ * of the counts buffers follows the token groups, which these fix. A call that reported an
+ * error may leave other ranks' stores in flight into these buffers: zero-fill every rank's
+ * buffers again (and synchronise the ranks) before the next call. */
 #define MOE_EP_MAX_WORLD 8
 #define MOE_EP_MAX_LOCAL 4
 #define MOE_EP_NUM_BUFFERS 8
