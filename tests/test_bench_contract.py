@@ -94,3 +94,25 @@ def test_layer0_roofline_bound_and_bytes():
     decode = synth.CONFIGS["skew_decode"]
     r = bench.layer0_roofline(decode, 0.46, 49, peaks, "measured", None, False, "k")
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    # the whole layer in one launch: + the router's FLOPs and its reads of x and W_g
+    E = cfg.E
+    r = bench.layer0_roofline(cfg, 4.75, 8, peaks, "measured", None, False,
+                              "moe_fused_layer_kernel<0, true>", fused=True, whole=True)
+    assert r["algorithmic_flops_per_launch"] == 6 * T * k * H * F + 2 * T * H * E
+    assert r["algorithmic_bytes_per_launch"] == (2 * (8 * H * 3 * F + T * k * H) + 2 * T * H +
+                                                 2 * T * H + 2 * H * E)
+    assert abs(r["achieved"] - r["algorithmic_flops_per_launch"] / 4.75e-3 / 1e12) < 1e-6
+
+
+def test_traffic_is_read_only_for_unchanged_sources():
+    """roofline.traffic comes from profiles/traffic.json only while the kernel's sources hash
+    to the value recorded with the counters; the committed entries match the tree."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+
+    d = json.loads((ROOT / "profiles" / "traffic.json").read_text())
+    for kernel, per in d.items():
+        for name, ent in per.items():
+            assert bench.traffic_for(kernel, name) == ent["bytes_per_launch"], (kernel, name)
+    assert bench.traffic_for("moe_fused_layer_kernel<0, true>", "mixtral") > 0
+    assert bench.traffic_for("no_such_kernel", "mixtral") is None
