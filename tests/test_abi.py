@@ -294,3 +294,23 @@ def test_ep_layer_sizes_and_checks(lib):
     r.world, r.rank, r.epoch = world, 0, 0          # epoch must be positive
     assert lib.moe_ep_layer_forward(ctypes.byref(r), 1, None) == -1
     assert lib.moe_ep_layer_forward(ctypes.byref(r), 5, None) == -1  # more ranks than one launch takes
+
+
+@pytest.mark.parametrize("T,H,E,k,launches", [
+    (512, 256, 8, 2, 1),     # T*k = 1024 = 128 E: sorted rows, the whole layer in one launch
+    (511, 256, 8, 2, 7),     # T*k < 128 E: router, dispatch 3, layers 3 (rows gathered in-kernel)
+    (256, 128, 8, 4, 1),     # k = 4: 1024 routed rows
+    (1024, 128, 16, 2, 8),   # E = 16, T*E < 2^16: one-launch router, dispatch 3, gather, layers 3
+    (20000, 256, 8, 2, 1),   # 128-token groups, more groups than SMs
+    (600, 96, 8, 2, -1),     # H % 64 != 0: invalid
+])
+def test_whole_layer_plan_boundaries(lib, T, H, E, k, launches):
+    """Host logic only: where the whole-layer launch applies (E = 8, T*k >= 128 E, the
+    one-launch router) and what runs elsewhere."""
+    prev = moe.moe_set_gemm_mode(moe.GEMM_AUTO)
+    prev_r = moe.moe_set_router_mode(moe.ROUTER_AUTO)
+    try:
+        assert moe.moe_forward_launches(moe.Problem.make(T, H, 256, E, k)) == launches
+    finally:
+        moe.moe_set_gemm_mode(prev)
+        moe.moe_set_router_mode(prev_r)
