@@ -13,9 +13,10 @@
 
 namespace moe {
 
-// BATCH = top-k rows whose loads one thread issues together: 2 for large grids (more rows
-// in flight per thread costs occupancy there), 8 when the grid is smaller than the GPU and
-// latency, not occupancy, sets the time.
+// BATCH = top-k rows whose loads one thread issues together: on large grids 2 for k <= 3 and
+// 4 for k >= 4 (more rows in flight per thread costs occupancy there: 8 was slower at both
+// k = 2 and k = 8), 8 when the grid is smaller than the GPU and latency, not occupancy,
+// sets the time.
 template <int BATCH>
 __global__ void __launch_bounds__(256)
     combine_kernel(const __nv_bfloat16 *__restrict__ ys, int64_t ys_rows,

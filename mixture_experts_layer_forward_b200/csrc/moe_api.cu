@@ -653,8 +653,13 @@ cudaError_t launch_combine(const moe_problem *p, const moe_bf16 *ys, int64_t ys_
     const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    // a grid that does not fill the GPU twice over: every thread issues all k row loads at once
-    auto kern = (blocks < 2 * cap / 16 && p->top_k > 2) ? combine_kernel<8> : combine_kernel<2>;
+    // a grid that does not fill the GPU twice over: every thread issues all k row loads at
+    // once; large grids: four row loads in flight per thread for k >= 4 (Qwen2-shaped and
+    // skewed layers, k = 8: 113 -> 101 us, 0.80 of the measured HBM copy bandwidth; eight
+    // rows: 110 us), two for smaller k
+    auto kern = (blocks < 2 * cap / 16 && p->top_k > 2) ? combine_kernel<8>
+                : p->top_k >= 4                         ? combine_kernel<4>
+                                                        : combine_kernel<2>;
     kern<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(ys), ys_rows, inv_pos,
                                       p->T, p->H, p->top_k, reinterpret_cast<__nv_bfloat16 *>(out),
                                       status, clear_status,
