@@ -314,3 +314,18 @@ def test_whole_layer_plan_boundaries(lib, T, H, E, k, launches):
     finally:
         moe.moe_set_gemm_mode(prev)
         moe.moe_set_router_mode(prev_r)
+
+
+def test_ep_local_launch_refuses_too_many_ranks(lib):
+    """Host-only: one launch carries at most EP_MAX_LOCAL ranks (checked before any launch),
+    and the experts must split evenly over the ranks."""
+    from mixture_experts_layer_forward_b200 import ep
+
+    p = moe.Problem.make(64, 128, 128, 8, 2)
+    n = moe.EP_MAX_LOCAL + 1
+    with pytest.raises(ValueError):
+        ep.ep_layer_forward_local(p, [None] * n, None, None, [None] * n, [None] * n, [None] * n,
+                                  [None] * n, [None] * n, epoch=1)
+    with pytest.raises(ValueError):
+        ep.experts_per_rank(8, 3)
+    assert ep.experts_per_rank(8, 4) == 2
