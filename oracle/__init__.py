@@ -84,6 +84,16 @@ def load(path: Path | None = None) -> ctypes.CDLL:
     lib.oracle_quant_cols_fp8.restype = None
     lib.oracle_moe_tokens_fp8.argtypes = [i32] * 7 + [vp] * 7 + [i32, vp, vp, vp, vp]
     lib.oracle_moe_tokens_fp8.restype = i32
+    lib.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e8m0_decode.restype = ctypes.c_double
+    lib.oracle_mx_quant_rows_f32.argtypes = [i32, i32, vp, vp, vp]
+    lib.oracle_mx_quant_rows_f32.restype = i32
+    lib.oracle_mx_quant_rows.argtypes = [i32, i32, vp, vp, vp]
+    lib.oracle_mx_quant_rows.restype = i32
+    lib.oracle_mx_quant_cols.argtypes = [i32, i32, i32, vp, vp, vp]
+    lib.oracle_mx_quant_cols.restype = i32
+    lib.oracle_moe_tokens_mx.argtypes = [i32] * 7 + [vp] * 7 + [i32, vp, vp, vp, vp]
+    lib.oracle_moe_tokens_mx.restype = i32
     lib.oracle_moe_backward.argtypes = [i32] * 7 + [vp] * 11
     lib.oracle_moe_backward.restype = i32
     lib.oracle_moe_backward_dx_tokens.argtypes = [i32] * 7 + [vp] * 6 + [i32, vp, vp]
@@ -321,6 +331,84 @@ def moe_tokens_fp8(x, Wg, bias, W1q, s1, W2q, s2, k, tokens, act=ACT_SWIGLU,
                                    _p(s1), _p(W2q), _p(s2), n, _p(tokens), _p(out), _p(idx), _p(w))
     if rc:
         raise ValueError(f"oracle_moe_tokens_fp8 rc={rc}")
+    return out, idx, w
+
+
+# ---------------------------------------------------------------------------------------
+# Block-scaled FP8 (MX form: e4m3 codes, one e8m0 power-of-two scale per 32 values along K;
+# see moe_oracle.c for the reading). Oracle only: no CUDA path for this form yet.
+# ---------------------------------------------------------------------------------------
+
+def e8m0_decode(b, lib=None):
+    """e8m0 scale byte -> 2^(b - 127) (NaN for 255)."""
+    lib = lib or load()
+    return float(lib.oracle_e8m0_decode(int(b)))
+
+
+def mx_quant_rows_f32(v, lib=None):
+    """float32 values [rows, cols] (cols % 32 == 0) -> (codes [rows, cols] uint8, scale
+    bytes [rows, cols / 32] uint8)."""
+    lib = lib or load()
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, cols = v.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows, cols // 32), np.uint8)
+    if lib.oracle_mx_quant_rows_f32(rows, cols, _p(v), _p(q), _p(s)):
+        raise ValueError("cols must be a multiple of 32")
+    return q, s
+
+
+def mx_quant_rows(src, lib=None):
+    """bf16 bit patterns [rows, cols] -> (codes [rows, cols], scale bytes [rows, cols / 32])."""
+    lib = lib or load()
+    src = _u16(src)
+    rows, cols = src.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows, cols // 32), np.uint8)
+    if lib.oracle_mx_quant_rows(rows, cols, _p(src), _p(q), _p(s)):
+        raise ValueError("cols must be a multiple of 32")
+    return q, s
+
+
+def mx_quant_cols(W, lib=None):
+    """Expert weights, bf16 bit patterns [E, K, N] -> (codes [E, N, K], scale bytes
+    [E, N, K / 32]): per output column, blocks of 32 along K."""
+    lib = lib or load()
+    W = _u16(W)
+    E, K, N = W.shape
+    q = np.empty((E, N, K), np.uint8)
+    s = np.empty((E, N, K // 32), np.uint8)
+    if lib.oracle_mx_quant_cols(E, K, N, _p(W), _p(q), _p(s)):
+        raise ValueError("K must be a multiple of 32")
+    return q, s
+
+
+def moe_tokens_mx(x, Wg, bias, W1q, W1s, W2q, W2s, k, tokens, act=ACT_SWIGLU,
+                  gate=GATE_SOFTMAX_TOPK, lib=None):
+    """Layer output with MX experts for the listed tokens (fp64 [ntok, H]), plus the routing.
+    W1q [E, w1_cols, H], W1s [E, w1_cols, H / 32], W2q [E, H, F], W2s [E, H, F / 32]."""
+    lib = lib or load()
+    x, Wg = _u16(x), _u16(Wg)
+    T, H = x.shape
+    E = Wg.shape[1]
+    W1q = np.ascontiguousarray(W1q, dtype=np.uint8)
+    W2q = np.ascontiguousarray(W2q, dtype=np.uint8)
+    W1s = np.ascontiguousarray(W1s, dtype=np.uint8)
+    W2s = np.ascontiguousarray(W2s, dtype=np.uint8)
+    F = W2q.shape[2]
+    w1_cols = 2 * F if act == ACT_SWIGLU else F
+    assert W1q.shape == (E, w1_cols, H) and W1s.shape == (E, w1_cols, H // 32)
+    assert W2q.shape == (E, H, F) and W2s.shape == (E, H, F // 32)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    n = tokens.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((n, H), np.float64)
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    rc = lib.oracle_moe_tokens_mx(T, H, F, E, k, act, gate, _p(x), _p(Wg), _p(b), _p(W1q),
+                                  _p(W1s), _p(W2q), _p(W2s), n, _p(tokens), _p(out), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle_moe_tokens_mx rc={rc}")
     return out, idx, w
 
 

@@ -762,6 +762,206 @@ int oracle_moe_tokens_fp8(int T, int H, int F, int E, int k, int act, int gate, 
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Block-scaled FP8 experts (MX form; a precision variant outside the pages). Oracle only:
+ * the CUDA path for this form is not built.
+ *
+ * Reading taken (the block format of the Open Compute Project's microscaling formats: e4m3
+ * elements sharing one e8m0 scale per 32 values; the conversion is this reading's):
+ *   - a block is 32 consecutive values along the GEMM's K dimension (a row of x or h; a
+ *     column of W1 or W2 along its input dimension);
+ *   - the block's scale is the smallest power of two 2^X with amax / 2^X <= 448 (amax: the
+ *     block's largest magnitude; 448 = 1.75 * 2^8, e4m3's largest finite value), so no
+ *     element saturates: X = floor(log2(amax)) - 8, plus 1 when amax / 2^that exceeds 448;
+ *     X is clamped to [-127, 127] and stored as the e8m0 byte X + 127 (255 is NaN). (The
+ *     specification's own conversion takes X = floor(log2(amax)) - 8 and saturates the
+ *     elements that land in (448, 512); on a test layer that gave a larger error than
+ *     per-row scales, which this rule avoids);
+ *   - each element is e4m3(v / 2^X) (oracle_e4m3_encode: nearest, ties to even);
+ *   - a block of zeros takes X = -127;
+ *   - GEMMs: for each output, the sum over blocks of 2^(Xa + Xw) times the exact sum of the
+ *     block's decoded code products (fp64);
+ *   - between the layers h is held in bf16, then quantised per 32-value block of its row.
+ * ------------------------------------------------------------------------------------- */
+
+double oracle_e8m0_decode(uint8_t b)
+{
+    if (b == 255) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* one block of n <= 32 values v[i * stride] -> codes q[i], returns the e8m0 scale byte */
+static uint8_t mx_quant_block(int n, const float *v, ptrdiff_t stride, uint8_t *q)
+{
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        const double a = fabs((double)v[(ptrdiff_t)i * stride]);
+        if (a > amax) amax = a;
+    }
+    int X = -127;
+    if (amax > 0.0) {
+        int e;
+        frexp(amax, &e); /* amax in [2^(e-1), 2^e): floor(log2 amax) = e - 1 */
+        X = (e - 1) - 8;
+        if (ldexp(amax, -X) > 448.0) X += 1; /* exact: scaling by a power of two */
+        if (X < -127) X = -127;
+        if (X > 127) X = 127;
+    }
+    for (int i = 0; i < n; ++i) {
+        const double scaled = ldexp((double)v[(ptrdiff_t)i * stride], -X); /* exact: a power of two */
+        q[i] = oracle_e4m3_encode((float)scaled);
+    }
+    return (uint8_t)(X + 127);
+}
+
+/* values [rows, cols] fp32 -> codes [rows, cols], scales [rows, cols / 32] (cols % 32 == 0) */
+int oracle_mx_quant_rows_f32(int rows, int cols, const float *v, uint8_t *q, uint8_t *scale)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+    for (int r = 0; r < rows; ++r)
+        for (int b = 0; b < cols / 32; ++b)
+            scale[(size_t)r * (cols / 32) + b] =
+                mx_quant_block(32, v + (size_t)r * cols + b * 32, 1, q + (size_t)r * cols + b * 32);
+    return 0;
+}
+
+/* bf16 matrix src [rows, cols] -> codes [rows, cols], scales [rows, cols / 32] */
+int oracle_mx_quant_rows(int rows, int cols, const uint16_t *src, uint8_t *q, uint8_t *scale)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+    float v[32];
+    for (int r = 0; r < rows; ++r)
+        for (int b = 0; b < cols / 32; ++b) {
+            for (int i = 0; i < 32; ++i) v[i] = bf16_to_float(src[(size_t)r * cols + b * 32 + i]);
+            scale[(size_t)r * (cols / 32) + b] = mx_quant_block(32, v, 1, q + (size_t)r * cols + b * 32);
+        }
+    return 0;
+}
+
+/* expert weights W [E, K, N] bf16 (N contiguous) -> per column n of expert e, its K values in
+ * blocks of 32: codes Wq [E, N, K] (K contiguous), scales [E, N, K / 32] */
+int oracle_mx_quant_cols(int E, int K, int N, const uint16_t *W, uint8_t *Wq, uint8_t *scale)
+{
+    if (E < 0 || K < 0 || N < 0 || K % 32 != 0) return -1;
+    float v[32];
+    for (int64_t en = 0; en < (int64_t)E * N; ++en) {
+        const int64_t e = en / N, n = en % N;
+        const uint16_t *col = W + (size_t)e * K * N + n;
+        for (int b = 0; b < K / 32; ++b) {
+            for (int i = 0; i < 32; ++i) v[i] = bf16_to_float(col[(size_t)(b * 32 + i) * N]);
+            scale[(size_t)en * (K / 32) + b] = mx_quant_block(32, v, 1, Wq + (size_t)en * K + b * 32);
+        }
+    }
+    return 0;
+}
+
+/* sum over the K / 32 blocks of 2^(Xa + Xb) * sum of the block's decoded code products */
+static double mx_dot(int K, const double *dec, const uint8_t *qa, const uint8_t *sa,
+                     const uint8_t *qb, const uint8_t *sb)
+{
+    double acc = 0.0;
+    for (int b = 0; b < K / 32; ++b) {
+        double part = 0.0;
+        for (int i = 0; i < 32; ++i) part += dec[qa[b * 32 + i]] * dec[qb[b * 32 + i]];
+        acc += part * oracle_e8m0_decode(sa[b]) * oracle_e8m0_decode(sb[b]);
+    }
+    return acc;
+}
+
+/* One expert on one token with MX operands (xq, xs: the token's row codes and scales;
+ * W1q [w1_cols, H] with W1s [w1_cols, H / 32]; W2q [H, F] with W2s [H, F / 32]):
+ *   z_c = mx_dot over H; a = SwiGLU or act(z), rounded to bf16 (the stored h);
+ *   hq, hs = the MX quantisation of a; y_n = mx_dot over F. */
+static void ffn_row_mx(int H, int F, int act, const double *dec, const uint8_t *xq,
+                       const uint8_t *xs, const uint8_t *W1q, const uint8_t *W1s,
+                       const uint8_t *W2q, const uint8_t *W2s, double *y, double *z, float *hf,
+                       uint8_t *hq, uint8_t *hs)
+{
+    const int gated = (act == ORACLE_ACT_SWIGLU);
+    const int w1_cols = gated ? 2 * F : F;
+    for (int c = 0; c < w1_cols; ++c)
+        z[c] = mx_dot(H, dec, xq, xs, W1q + (size_t)c * H, W1s + (size_t)c * (H / 32));
+    for (int f = 0; f < F; ++f) {
+        const double a = gated ? silu(z[f]) * z[f + F] : act_apply(act, z[f]);
+        hf[f] = (float)oracle_round_to_bf16(a);
+    }
+    for (int b = 0; b < F / 32; ++b) hs[b] = mx_quant_block(32, hf + b * 32, 1, hq + b * 32);
+    for (int n = 0; n < H; ++n)
+        y[n] = mx_dot(F, dec, hq, hs, W2q + (size_t)n * F, W2s + (size_t)n * (F / 32));
+}
+
+/* The layer output for a list of tokens with MX experts: the routing of oracle_moe_tokens
+ * (bf16 x and W_g, fp32 logits), then out[t] = sum_j w_j * FFN_MX_{e_j}(x_t) with the token's
+ * row quantised per block of 32. W1q [E, w1_cols, H], W1s [E, w1_cols, H / 32]; W2q [E, H, F],
+ * W2s [E, H, F / 32] (as oracle_mx_quant_cols writes them). out [ntok, H] fp64. */
+int oracle_moe_tokens_mx(int T, int H, int F, int E, int k, int act, int gate, const uint16_t *x,
+                         const uint16_t *Wg, const float *bias, const uint8_t *W1q,
+                         const uint8_t *W1s, const uint8_t *W2q, const uint8_t *W2s, int ntok,
+                         const int32_t *tokens, double *out, int32_t *idx_out, double *w_out)
+{
+    if (H < 1 || F < 1 || E < 1 || k < 1 || k > E || ntok < 0 || H % 32 || F % 32) return -1;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -2;
+    const int w1_cols = act == ORACLE_ACT_SWIGLU ? 2 * F : F;
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = oracle_e4m3_decode((uint8_t)c);
+    int bad = 0;
+#pragma omp parallel
+    {
+        float *l = (float *)malloc(sizeof(float) * (size_t)E);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        double *z = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+        float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+        uint8_t *xq = (uint8_t *)malloc((size_t)H);
+        uint8_t *xs = (uint8_t *)malloc((size_t)H / 32);
+        float *hf = (float *)malloc(sizeof(float) * (size_t)F);
+        uint8_t *hq = (uint8_t *)malloc((size_t)F);
+        uint8_t *hs = (uint8_t *)malloc((size_t)F / 32);
+        const int ok = l && taken && sel && w && y && z && xf && xq && xs && hf && hq && hs;
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < ntok; ++i) {
+            if (!ok) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            const int t = tokens[i];
+            const uint16_t *xr = x + (size_t)t * H;
+            oracle_router_logits(1, H, E, xr, Wg, gate == ORACLE_GATE_SELECT_BIAS ? NULL : bias, l);
+            topk_one(E, k, gate, l, bias, sel, w, taken);
+            for (int h = 0; h < H; ++h) xf[h] = bf16_to_float(xr[h]);
+            for (int b = 0; b < H / 32; ++b) xs[b] = mx_quant_block(32, xf + b * 32, 1, xq + b * 32);
+            double *o = out + (size_t)i * H;
+            for (int n = 0; n < H; ++n) o[n] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                const int e = sel[j];
+                ffn_row_mx(H, F, act, dec, xq, xs, W1q + (size_t)e * w1_cols * H,
+                           W1s + (size_t)e * w1_cols * (H / 32), W2q + (size_t)e * H * F,
+                           W2s + (size_t)e * H * (F / 32), y, z, hf, hq, hs);
+                for (int n = 0; n < H; ++n) o[n] += y[n] * w[j];
+            }
+            if (idx_out) memcpy(idx_out + (size_t)i * k, sel, sizeof(int32_t) * (size_t)k);
+            if (w_out) memcpy(w_out + (size_t)i * k, w, sizeof(double) * (size_t)k);
+        }
+        free(l);
+        free(taken);
+        free(sel);
+        free(w);
+        free(y);
+        free(z);
+        free(xf);
+        free(xq);
+        free(xs);
+        free(hf);
+        free(hq);
+        free(hs);
+    }
+    return bad ? -4 : 0;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Backward pass (training; a next-work item beyond the pages, which describe the forward)
  *
  * The forward is out[t] = sum_j w_j(t) y_{e_j}(x_t), y_e(x) = FFN_e(x) as in ffn_row, the

@@ -2,8 +2,8 @@
 
 Each mutant below plants one slip in a copy of oracle/moe_oracle.c (a dropped term, a
 transposed operand, a wrong index, order or tie-break, a wrong constant or sign, a wider
-accumulator), builds it, and runs tests/test_oracle_pins.py against that build. Every mutant
-must make at least one pin fail. Mutations that leave the result mathematically unchanged
+accumulator), builds it, and runs tests/test_oracle_pins.py and tests/test_oracle_mx.py
+against that build. Every mutant must make at least one pin fail. Mutations that leave the result mathematically unchanged
 (for example dropping the max shift of the softmax) are not mistakes and are not listed.
 """
 import os
@@ -18,6 +18,8 @@ import oracle
 
 ROOT = Path(__file__).resolve().parents[1]
 SRC = ROOT / "oracle" / "moe_oracle.c"
+
+PIN_FILES = ("test_oracle_pins.py", "test_oracle_mx.py")
 
 MUTANTS = [
     ("router_wider_accumulator", "float acc = 0.0f;", "double acc = 0.0;"),
@@ -63,9 +65,15 @@ MUTANTS = [
     ("fp8_h_scale_dropped", "y[n] = acc * (double)sh * (double)s2[n];", "y[n] = acc * (double)s2[n];"),
     ("fp8_x_scale_dropped", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)s1[c];"),
     ("fp8_w1_scale_of_column_0", "z[c] = acc * (double)sx * (double)s1[c];", "z[c] = acc * (double)sx * (double)s1[0];"),
-    ("fp8_gate_up_swapped", "silu(z[f]) * z[f + F]", "silu(z[f + F]) * z[f]"),
-    ("fp8_token_path_drops_gate", "o[n] += y[n] * w[j];", "o[n] += y[n];"),
-    ("fp8_h_not_rounded_to_bf16", "hf[f] = (float)oracle_round_to_bf16(a);", "hf[f] = (float)a;"),
+    ("fp8_gate_up_swapped",
+     "silu(z[f]) * z[f + F] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    const float sh",
+     "silu(z[f + F]) * z[f] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    const float sh"),
+    ("fp8_token_path_drops_gate", "y, z, hf, hq);\n                for (int n = 0; n < H; ++n) o[n] += y[n] * w[j];",
+     "y, z, hf, hq);\n                for (int n = 0; n < H; ++n) o[n] += y[n];"),
+    ("mx_token_path_drops_gate", "y, z, hf, hq, hs);\n                for (int n = 0; n < H; ++n) o[n] += y[n] * w[j];",
+     "y, z, hf, hq, hs);\n                for (int n = 0; n < H; ++n) o[n] += y[n];"),
+    ("fp8_h_not_rounded_to_bf16", "hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    const float sh",
+     "hf[f] = (float)a;\n    }\n    const float sh"),
     ("bwd_silu_derivative_drops_term", "const double dg = da[f] * u * s * (1.0 + g * (1.0 - s));",
      "const double dg = da[f] * u * s;"),
     ("bwd_up_gradient_uses_up", "const double du = da[f] * g * s;", "const double du = da[f] * u * s;"),
@@ -75,6 +83,23 @@ MUTANTS = [
     ("bwd_dW2_without_gate", "drow[n] += a[f] * gscale * (double)bf16_to_float(dyr[n]);",
      "drow[n] += a[f] * (double)bf16_to_float(dyr[n]);"),
     ("bwd_dx_tokens_not_centred", "const double dl = w[j] * (dw[j] - wdw);", "const double dl = w[j] * dw[j];"),
+    ("mx_scale_saturating_rule", "if (ldexp(amax, -X) > 448.0) X += 1;", ""),
+    ("mx_scale_exponent_of_e5m2", "X = (e - 1) - 8;", "X = (e - 1) - 15;"),
+    ("mx_e8m0_bias_128", "return ldexp(1.0, (int)b - 127);", "return ldexp(1.0, (int)b - 128);"),
+    ("mx_dot_scale_of_block_0",
+     "acc += part * oracle_e8m0_decode(sa[b]) * oracle_e8m0_decode(sb[b]);",
+     "acc += part * oracle_e8m0_decode(sa[0]) * oracle_e8m0_decode(sb[b]);"),
+    ("mx_dot_weight_scale_dropped",
+     "acc += part * oracle_e8m0_decode(sa[b]) * oracle_e8m0_decode(sb[b]);",
+     "acc += part * oracle_e8m0_decode(sa[b]);"),
+    ("mx_weight_blocks_along_n", "v[i] = bf16_to_float(col[(size_t)(b * 32 + i) * N]);",
+     "v[i] = bf16_to_float(col[(size_t)(b * 32 + i)]);"),
+    ("mx_gate_up_swapped",
+     "silu(z[f]) * z[f + F] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    for (int b",
+     "silu(z[f + F]) * z[f] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    for (int b"),
+    ("mx_h_not_rounded_to_bf16",
+     "        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    for (int b = 0; b < F / 32; ++b)",
+     "        hf[f] = (float)a;\n    }\n    for (int b = 0; b < F / 32; ++b)"),
     ("shared_ffn_uses_gate_half_only", "ffn_row(H, Fs, ORACLE_ACT_SWIGLU, 0, xr, W1s, W2s, y, scratch);",
      "ffn_row(H, Fs, ORACLE_ACT_GELU_TANH, 0, xr, W1s, W2s, y, scratch);"),
 ]
@@ -90,7 +115,7 @@ def _run_mutant(tmp_path, name, old, new):
     src.write_text(text.replace(old, new))
     lib = oracle.build(force=True, src=src, out=d / "liboracle_mutant.so")
     env = dict(os.environ, ORACLE_LIB_UNDER_TEST=str(lib), OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", str(ROOT / "tests" / "test_oracle_pins.py"),
+    r = subprocess.run([sys.executable, "-m", "pytest", *[str(ROOT / "tests" / f) for f in PIN_FILES],
                         "-x", "-q", "-p", "no:cacheprovider"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     if r.returncode != 1:
