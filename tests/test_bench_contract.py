@@ -116,3 +116,44 @@ def test_traffic_is_read_only_for_unchanged_sources():
             assert bench.traffic_for(kernel, name) == ent["bytes_per_launch"], (kernel, name)
     assert bench.traffic_for("moe_fused_layer_kernel<0, true>", "mixtral") > 0
     assert bench.traffic_for("no_such_kernel", "mixtral") is None
+
+
+def test_profile_commands_parse_with_the_current_bench():
+    """Every bench.py command quoted in profiles/ must still run: its flags parse with
+    bench.py's own parser, its workload exists, and any other script it names is committed."""
+    import re
+
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from mixture_experts_layer_forward_b200 import synth
+
+    def expand(cmd):
+        """Each `for W in a b c; do ... done` loop, unrolled over its values."""
+        loop = re.search(r"for (\w+) in ([^;]+); do(.*?)done", cmd, re.S)
+        if not loop:
+            return [cmd]
+        var, values, body = loop.group(1), loop.group(2).split(), loop.group(3)
+        return [c for v in values
+                for c in expand(cmd[:loop.start()] + body.replace("$" + var, v) + cmd[loop.end():])]
+
+    def bench_commands():
+        for md in sorted((ROOT / "profiles").glob("*.md")):
+            for block in re.findall(r"```\n(.*?)```", md.read_text(), re.S):
+                for cmd in expand(block.replace("\\\n", " ")):
+                    for m in re.finditer(r"python (\S+\.py)([^\n&|>]*)", cmd):
+                        yield md.name, m.group(1), m.group(2).split()
+
+    checked = 0
+    for name, script, args in bench_commands():
+        assert (ROOT / script).is_file(), f"{name}: {script} is not in the tree"
+        if script != "bench.py":
+            continue
+        old = sys.argv
+        sys.argv = ["bench.py", *args]
+        try:
+            parsed = bench.parse_args()
+        finally:
+            sys.argv = old
+        assert parsed.workload in synth.CONFIGS, f"{name}: {parsed.workload}"
+        checked += 1
+    assert checked >= 10
