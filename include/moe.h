@@ -26,6 +26,11 @@
  *   - No C++ exception crosses this boundary.
  *   - The caller's buffers may not overlap each other or the workspace.
  *   - Concurrent calls that share one workspace race; give each stream its own.
+ *   - The whole-layer launch and the expert-parallel launch are persistent, one CTA per SM,
+ *     and their CTAs meet at grid-wide barriers: they expect the whole GPU. Kernels that
+ *     run at the same time on other streams can keep some CTAs from starting; the waiting
+ *     CTAs then give up after the wait timeout (moe_set_wait_timeout_ns) and the call
+ *     reports MOE_ERR_DEVICE_TIMEOUT through the status word instead of hanging.
  *
  * Supported problem sizes: T >= 0, H % 64 == 0, F % 64 == 0, 1 <= top_k <= E <= 1024,
  * m_tile == 128; anything else returns MOE_ERR_UNSUPPORTED.
