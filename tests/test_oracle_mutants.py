@@ -94,6 +94,10 @@ MUTANTS = [
      "acc += part * oracle_e8m0_decode(sa[b]);"),
     ("mx_weight_blocks_along_n", "v[i] = bf16_to_float(col[(size_t)(b * 32 + i) * N]);",
      "v[i] = bf16_to_float(col[(size_t)(b * 32 + i)]);"),
+    ("mx_w1_scales_of_expert_0", "W1s + (size_t)e * w1_cols * (H / 32), W2q",
+     "W1s, W2q"),
+    ("mx_w2_scale_stride_of_codes", "W2s + (size_t)e * H * (F / 32), y, z",
+     "W2s + (size_t)e * H * F / 64, y, z"),
     ("mx_gate_up_swapped",
      "silu(z[f]) * z[f + F] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    for (int b",
      "silu(z[f + F]) * z[f] : act_apply(act, z[f]);\n        hf[f] = (float)oracle_round_to_bf16(a);\n    }\n    for (int b"),

@@ -169,6 +169,28 @@ def test_h_is_rounded_to_bf16_before_its_block_quantisation(oracle_lib):
     assert np.all(out[0, 1:] == 0.0) and np.all(out[1] == 0.0)
 
 
+@pytest.mark.parametrize("act", [oracle.ACT_IDENTITY, oracle.ACT_RELU])
+def test_layer_scales_exactly_with_the_input(oracle_lib, act):
+    """W_g = 0: every logit is 0, so each token takes experts 0 and 1 (ties to the lower id)
+    with gates 1/2 whatever x is. With a positively homogeneous activation, x -> 2^3 x leaves
+    every code of x and of h unchanged and raises every scale byte by 3, so the output is
+    exactly 8 times the original (the bf16 rounding of h commutes with a power of two)."""
+    O = _Bound(oracle_lib)
+    cfg = synth.LayerConfig("mx_h", T=16, H=64, F=96, E=4, k=2, act=act)
+    inp = synth.make_inputs(cfg, seed=9)
+    Wg = np.zeros((cfg.H, cfg.E), np.uint16)
+    W1q, W1s = O.mx_quant_cols(_bits(inp["W1"]))
+    W2q, W2s = O.mx_quant_cols(_bits(inp["W2"]))
+    toks = np.arange(cfg.T)
+    out, idx, w = O.moe_tokens_mx(_bits(inp["x"]), Wg, None, W1q, W1s, W2q, W2s, cfg.k, toks,
+                                  act=act)
+    assert np.all(idx == [0, 1]) and np.all(w == 0.5)
+    x8 = _bits((inp["x"].float() * 8.0).to(inp["x"].dtype))
+    out8, _, _ = O.moe_tokens_mx(x8, Wg, None, W1q, W1s, W2q, W2s, cfg.k, toks, act=act)
+    np.testing.assert_array_equal(out8, 8.0 * out)
+    assert np.abs(out).max() > 0
+
+
 def test_layer_close_to_the_exact_layer(oracle_lib):
     """The MX layer against the exact (bf16 operands, fp64) layer on random data. Four
     operands are rounded to e4m3 (x, W1, h, W2), each with a relative error of at most 2^-4
